@@ -1,0 +1,389 @@
+#!/usr/bin/env python
+"""Benchmark of the looped INT4 model on B200.
+
+Workload (one step): the ~400M-unique-parameter looped LM (d_model 2048, 16 Q /
+4 KV heads of 128, SwiGLU 5632, vocab 32000, 2 pre blocks + 1 shared loop
+block, INT4 g128 body, fp16 embed/head/norms, seeded random weights) with
+L = 8: prefill of a 128-token prompt with no logits, then 128 greedy decode
+steps at batch 1 (the first decode step feeds prompt token 128; each later one
+feeds the previous argmax, on the device).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  `value` is decode tokens/s summed over ranks (each
+rank runs its own replica: weak scaling, no collective on the data path);
+prefill ms, roofline of the dominant decode kernel, the CPU oracle baseline,
+end-to-end numbers and SM clocks are extra keys.  `--impl reference` times the
+CPU oracle on this host on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "decode tok/s & prefill ms (T=128, L=8) looped INT4 model; % of roofline"
+UNIT = "tokens/s"
+PROMPT, STEPS_DECODE, LOOPS = 128, 128, 8
+WORKLOAD = "looped INT4 LM d2048 16q/4kv hd128 F5632 V32000 n_pre2 L8; prefill 128 (no logits) + 128 greedy decode, batch 1"
+
+# Algorithmic bytes per decode launch at batch 1 (weights + scales/zeros + the
+# activations each launch must read and write), d = 2048, F = 5632, V = 32000.
+D, F, V, HQ, HKV, HD = 2048, 5632, 32000, 16, 4, 128
+
+
+def _int4_bytes(K, N):
+    return K * N // 2 + (K // 128) * N * 5 // 2   # nibbles + fp16 scale + 4-bit zero
+
+
+BYTES_PER_LAUNCH = {
+    "qkv": _int4_bytes(D, (HQ + 2 * HKV) * HD) + 4 * D + 2 * D + 2 * (HQ + 2 * HKV) * HD,
+    "o_proj": _int4_bytes(HQ * HD, D) + 2 * HQ * HD + 8 * D,
+    "gate_up": _int4_bytes(D, 2 * F) + 4 * D + 2 * D + 2 * F,
+    "down": _int4_bytes(F, D) + 2 * F + 8 * D,
+    "head": V * D * 2 + 4 * D + 2 * D + 4,
+}
+
+
+def _attn_bytes_per_launch(mean_keys):
+    return 2 * HKV * HD * 2 * mean_keys + 2 * HQ * HD * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks ---
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.device_index = device_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.device_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if not getattr(self, "out", ""):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["no samples"]}
+        loaded = [s for s in sm if mx and s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------- CPU oracle --
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(weights, prompt, n_decode, om=None):
+    """Time the oracle: prefill of the prompt, then n_decode cached greedy steps.
+    Returns (prefill_s, decode_s, om)."""
+    from oracle import ref
+    if om is None:
+        om = ref.LoopedModel(weights)
+    t0 = time.perf_counter()
+    cache, logits = om.prefill(prompt[:PROMPT], LOOPS)
+    t1 = time.perf_counter()
+    tok = int(prompt[PROMPT])
+    for _ in range(n_decode):
+        logits = om.decode(cache, tok, LOOPS)
+        tok = ref.greedy(logits)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1, om
+
+
+# ------------------------------------------------------------------- arms ---
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import tl_synth
+    w = tl_synth.make_model_weights(tl_synth.LOOPED_LM, tl_synth.SEED_LM)
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, tl_synth.LOOPED_LM.vocab, PROMPT + 1)
+    n_dec = 2
+    om = None
+    pre, dec = [], []
+    for i in range(args.warmup + args.steps):
+        p, d, om = oracle_sample(w, prompt, n_dec, om)
+        if i >= args.warmup:
+            pre.append(p)
+            dec.append(d)
+    cores = blas_threads()
+    value = n_dec * len(dec) / sum(dec)
+    sample = (f"per step: oracle prefill of the 128-token prompt + {n_dec} cached greedy decode "
+              f"steps at L=8 (float64 NumPy)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * (sum(pre) + sum(dec)) / len(dec),
+        "prefill_ms": 1e3 * statistics.mean(pre),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded random weights and token ids)",
+        "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": PROMPT + STEPS_DECODE,
+                   "parallelism": "cpu oracle, rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+
+    world, rank, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+        pg = dist
+
+    shape = tl_synth.LOOPED_LM
+    w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM)
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, shape.vocab, PROMPT + 1)
+    cfg = tl.make_config(shape, max_loops=LOOPS, max_ctx=PROMPT + STEPS_DECODE, max_lanes=1)
+    tw, keep = tl.make_weights(w)
+    m = tl.tl_model_create(cfg, tw, local)
+    del keep
+
+    st = torch.cuda.Stream(device=dev)
+    d_prompt = torch.as_tensor(prompt, device=dev)
+    hist = torch.zeros(STEPS_DECODE + 1, dtype=torch.int32, device=dev)
+    hp = hist.data_ptr()
+
+    def step(ev=None):
+        with torch.cuda.stream(st):
+            if ev:
+                ev[0].record(st)
+            tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS, None, None, st)
+            if ev:
+                ev[1].record(st)
+            hist[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
+            for i in range(STEPS_DECODE):
+                tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1), st)
+            if ev:
+                ev[2].record(st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    launches0 = tl.tl_kernel_launch_count()
+    with ClockSampler(local) as clocks:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(st)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(st)
+        torch.cuda.synchronize()
+    launches = tl.tl_kernel_launch_count() - launches0
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+
+    total_ms = t_start.elapsed_time(t_end)
+    prefill_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    stats = torch.tensor([total_ms, sum(prefill_ms), sum(decode_ms)], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(stats, op=pg.ReduceOp.MAX)
+    total_ms, prefill_sum, decode_sum = (float(v) for v in stats.cpu())
+    tokens = world * STEPS_DECODE * args.steps
+    value = tokens / (decode_sum / 1e3)
+    generated = hist[1:].cpu().numpy().copy()
+
+    # ---- end to end: pinned host prompt in, generated tokens out, per step --
+    h_prompt = torch.from_numpy(prompt.copy()).pin_memory()
+    h_out = torch.empty(STEPS_DECODE, dtype=torch.int32).pin_memory()
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(st):
+            a.record(st)
+            d_prompt.copy_(h_prompt, non_blocking=True)
+            step()
+            h_out.copy_(hist[1:], non_blocking=True)
+            b.record(st)
+        b.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(e2e, op=pg.ReduceOp.MAX)
+    e2e_value = world * STEPS_DECODE * args.steps / (float(e2e.item()) / 1e3)
+    assert np.array_equal(h_out.numpy(), generated), "end-to-end run diverged from the timed run"
+
+    # ---- per-kernel profile of one decode phase (separate from the timing) -
+    with torch.cuda.stream(st):
+        tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS, None, None, st)
+        hist[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
+        st.synchronize()
+        tl.tl_model_profile_start(m)
+        for i in range(STEPS_DECODE):
+            tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1), st)
+        prof = tl.tl_model_profile_stop(m)
+    peaks = load_peaks()
+    mean_keys = PROMPT + (STEPS_DECODE + 1) / 2
+    per_class = {}
+    for name, (n, ms) in prof.items():
+        avg_us = 1e3 * ms / n
+        b = BYTES_PER_LAUNCH.get(name)
+        if name == "attn_decode":
+            b = _attn_bytes_per_launch(mean_keys)
+        per_class[name] = {"launches": n, "total_ms": round(ms, 4), "avg_us": round(avg_us, 3),
+                           "gbs": round(b / (avg_us * 1e3), 1) if b else None}
+    dom = max(per_class, key=lambda k: per_class[k]["total_ms"])
+    dom_b = BYTES_PER_LAUNCH.get(dom) or (_attn_bytes_per_launch(mean_keys) if dom == "attn_decode" else None)
+    achieved = dom_b / (per_class[dom]["avg_us"] * 1e3) if dom_b else None
+    roofline = {
+        "kernel": dom, "bound": "hbm", "achieved": round(achieved, 1) if achieved else None,
+        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
+        "traffic": None, "peak_source": peaks["source"],
+        "bytes_per_launch": dom_b,
+    }
+
+    # ---- CPU oracle baseline (rank 0, bounded sample) -----------------------
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        n_dec = 4
+        p_s, d_s, _ = oracle_sample(w, prompt, n_dec)
+        cpu = {"value": n_dec / d_s, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"oracle prefill of the 128-token prompt ({p_s:.2f} s) + {n_dec} cached "
+                         f"greedy decode steps at L=8 ({d_s:.2f} s), float64 NumPy"}
+
+    tl.tl_model_destroy(m)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total_ms / args.steps, 4),
+            "prefill_ms": round(prefill_sum / args.steps, 4),
+            "decode_ms_per_token": round(decode_sum / (args.steps * STEPS_DECODE), 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (INT4 weights)",
+            "data": "synthetic (seeded random weights and token ids)",
+            "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": PROMPT + STEPS_DECODE,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": "inputs larger than L2: each step streams ~333 MB of weights"},
+            "roofline": roofline,
+            "kernels_decode": per_class,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": int(h_prompt.numel() * 4),
+                    "d2h_bytes_per_step": int(h_out.numel() * 4)},
+            "gpu_launches": int(launches),
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,299 @@
+/*
+ * tl.h -- C ABI of the B200 (sm_100a) looped INT4 transformer library.
+ *
+ * The library computes the forward pass of a weight-shared looped transformer:
+ *   tokens -> embed -> pre blocks -> one shared loop block run L times
+ *          -> output norm -> head
+ * (TinyLoop README, "Why TinyLoop Exists"), with every block linear stored as
+ * group-wise INT4 weights with zero points, w = (q - z) * s, group 128 along K
+ * (TinyLoop README, "Status", INT4 loop / pre linears with zero points).  The
+ * loop count L is an argument of every call (TinyLoop docs, "Async API",
+ * "Scoring" and "Generation": loops= on score / generate).
+ *
+ * General conventions
+ * -------------------
+ * - Every pointer named d_* is DEVICE memory on the model's / call's device;
+ *   every pointer named h_* is HOST memory.  The caller owns all buffers it
+ *   passes; the library never frees them and keeps no pointer to them after
+ *   the call returns, except where a function says otherwise.
+ * - fp16 values travel as uint16_t bit patterns (IEEE binary16).
+ * - Arguments are validated synchronously before anything is enqueued; a call
+ *   that returns an error has enqueued nothing (apart from TL_ERR_CUDA, which
+ *   reports a failed launch).  tl_last_error() returns a one-line reason for
+ *   the last error of the calling thread.
+ * - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *   legacy default stream).  Results are ready when the stream reaches them.
+ * - One model handle must not be used by two host threads at the same time
+ *   (TinyLoop docs, "Async API", "Concurrency model": the model is not
+ *   thread-safe and callers serialise).  Calls on one handle must be ordered
+ *   on one stream.
+ * - Data-dependent device-side faults (a token id outside [0, vocab)) do not
+ *   trap: the kernel substitutes token 0, records the fault in a device flag,
+ *   and tl_check_device_error() reports it.
+ */
+#ifndef TL_H_
+#define TL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TL_OK = 0,
+  TL_ERR_INVALID_ARG = 1,    /* a NULL pointer, size or shape out of range */
+  TL_ERR_OOM = 2,            /* device allocation failed */
+  TL_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+  TL_ERR_CONTEXT_FULL = 4,   /* the lane has no room for more tokens */
+  TL_ERR_LOOPS_MISMATCH = 5, /* decode loops differ from the lane's prefill */
+  TL_ERR_NOT_PREFILLED = 6,  /* decode on a lane that holds no prompt */
+  TL_ERR_DEVICE_FLAG = 7,    /* a kernel recorded a data fault (see above) */
+  TL_ERR_UNSUPPORTED = 8     /* a shape the kernels are not built for */
+} tl_status;
+
+/* Static description of a model (TinyLoop docs, "Async API", "Constructor":
+ * max_seq_len; the dimensions are those of the Llama-family block that the
+ * README's "Status" list names: RoPE with configurable theta, GQA). */
+typedef struct {
+  int d_model;      /* hidden size; multiple of 128 */
+  int n_q_heads;    /* query heads */
+  int n_kv_heads;   /* key/value heads; divides n_q_heads (GQA) */
+  int head_dim;     /* 64 or 128; n_q_heads * head_dim is a multiple of 128 */
+  int ffn_dim;      /* SwiGLU inner size F; multiple of 128 */
+  int vocab;        /* vocabulary size; multiple of 16 */
+  int n_pre;        /* number of distinct pre blocks (>= 0) */
+  int max_loops;    /* largest L any call may use (>= 1) */
+  int max_ctx;      /* tokens per lane (prompt + generated), <= 8192 */
+  int max_lanes;    /* decode lanes, 1..16 */
+  float rms_eps;    /* RMSNorm epsilon */
+  float rope_theta; /* RoPE base */
+} tl_config;
+
+/* One INT4 linear with K inputs and N outputs, HOST memory, storage format:
+ *   qweight uint32 [N][K/8]        element k of row n is bits 4*(k%8)..+3 of
+ *                                  word k/8 (low nibble first)
+ *   scales  fp16   [N][K/128]      scale of (row, group)
+ *   qzeros  uint32 [N][ceil(K/1024)] the K/128 zero points of the row, eight
+ *                                  per word, same nibble order, unused = 0
+ * The dequantized weight is W[n][k] = (q - z) * s with no offset on z. */
+typedef struct {
+  const uint32_t *qweight;
+  const uint16_t *scales;
+  const uint32_t *qzeros;
+} tl_int4_linear;
+
+/* One transformer block (pre-norm, Llama family).
+ *   qkv:     N = (n_q_heads + 2 n_kv_heads) * head_dim, K = d_model; rows are
+ *            the q heads, then the k heads, then the v heads, head-major
+ *   o:       N = d_model, K = n_q_heads * head_dim
+ *   gate_up: N = 2 ffn_dim, K = d_model; rows [0, F) gate, [F, 2F) up
+ *   down:    N = d_model, K = ffn_dim
+ *   attn_norm, ffn_norm: fp16 [d_model] RMSNorm gains */
+typedef struct {
+  const uint16_t *attn_norm;
+  const uint16_t *ffn_norm;
+  tl_int4_linear qkv, o, gate_up, down;
+} tl_block;
+
+/* All weights, HOST memory.  embed and head are fp16 [vocab][d_model] (the
+ * head is its own matrix), out_norm fp16 [d_model], pre[n_pre] the distinct
+ * pre blocks, loop the one block shared by every loop iteration. */
+typedef struct {
+  const uint16_t *embed;
+  const uint16_t *out_norm;
+  const uint16_t *head;
+  const tl_block *pre;
+  const tl_block *loop;
+} tl_weights;
+
+typedef struct tl_model tl_model;
+typedef struct tl_linear tl_linear;
+
+/* ------------------------------------------------------------------------
+ * Model API
+ * ------------------------------------------------------------------------ */
+
+/* Copy the host weights to `device`, re-lay them out for the kernels and
+ * allocate the KV cache (max_lanes lanes x (n_pre + max_loops) layers x K/V x
+ * n_kv_heads x max_ctx x head_dim fp16, one slice per effective layer, so that
+ * every loop iteration keeps its own keys and values; TinyLoop README,
+ * "Status", GQA item) and all workspaces.  The host arrays may be freed when
+ * this returns.  On success *out owns all device memory of the model. */
+tl_status tl_model_create(const tl_config *cfg, const tl_weights *w, int device,
+                          tl_model **out);
+
+/* Free all device memory of the model.  NULL is a no-op.  The caller must make
+ * sure no work of the model is still pending on any stream. */
+void tl_model_destroy(tl_model *m);
+
+/* Run a prompt on `lane` (0 <= lane < max_lanes): n_tokens ids at positions
+ * 0..n_tokens-1 through n_pre + loops effective layers, writing each layer's
+ * keys and values to the lane's cache slices.  Any earlier content of the lane
+ * is discarded; the lane's loop count becomes `loops`.
+ *   d_tokens        int32 [n_tokens], 1 <= n_tokens <= max_ctx
+ *   loops           1 <= loops <= max_loops
+ *   d_last_logits   fp32 [vocab] logits of the last position, or NULL to skip
+ *                   the output norm and head ("no logits", TinyLoop README,
+ *                   "Current Runtime Snapshot")
+ *   d_last_argmax   int32 [1] greedy token of the last position (lowest index
+ *                   on ties), or NULL; needs the head, like the logits. */
+tl_status tl_prefill(tl_model *m, int lane, const int32_t *d_tokens, int n_tokens,
+                     int loops, float *d_last_logits, int32_t *d_last_argmax,
+                     void *stream);
+
+/* One cached decode step for n_lanes lanes at once (TinyLoop docs, "Async
+ * API", "Batch generation": per-lane loops).  Lane i feeds token d_tokens[i]
+ * at position length(lane) and attends over its own cache; each lane runs
+ * exactly its own n_pre + loops layers, and its result does not depend on
+ * which other lanes share the step.
+ *   h_lane_ids  int32 [n_lanes], distinct, each prefilled
+ *   d_tokens    int32 [n_lanes]
+ *   h_loops     int32 [n_lanes], must equal each lane's prefill loops
+ *               (else TL_ERR_LOOPS_MISMATCH)
+ *   d_logits    fp32 [n_lanes][vocab] or NULL
+ *   d_argmax    int32 [n_lanes] greedy tokens, or NULL.  May alias d_tokens:
+ *               the tokens are read before the argmax is written.
+ * Returns TL_ERR_CONTEXT_FULL if a lane already holds max_ctx tokens. */
+tl_status tl_decode_step(tl_model *m, int n_lanes, const int32_t *h_lane_ids,
+                         const int32_t *d_tokens, const int32_t *h_loops,
+                         float *d_logits, int32_t *d_argmax, void *stream);
+
+/* Stateless uncached forward (TinyLoop docs, "Async API", "Scoring",
+ * score_last): logits [vocab] of the last of n_tokens tokens.  Touches no
+ * lane (it uses a private scratch slice).  d_logits must not be NULL;
+ * d_argmax may be NULL. */
+tl_status tl_score_last(tl_model *m, const int32_t *d_tokens, int n_tokens, int loops,
+                        float *d_logits, int32_t *d_argmax, void *stream);
+
+/* Tokens currently held by a lane (0 if never prefilled). */
+tl_status tl_lane_length(const tl_model *m, int lane, int *h_length);
+
+/* Device bytes held by the model: weights (as laid out for the kernels), KV
+ * cache, and all other workspaces.  Any pointer may be NULL. */
+tl_status tl_model_info(const tl_model *m, size_t *weight_bytes, size_t *kv_bytes,
+                        size_t *workspace_bytes);
+
+/* Synchronise `stream`, read and clear the model's device fault flag.
+ * Returns TL_OK, TL_ERR_DEVICE_FLAG (a kernel saw a token id outside
+ * [0, vocab) and used token 0 instead), or TL_ERR_CUDA. */
+tl_status tl_check_device_error(tl_model *m, void *stream);
+
+/* Kernel families, for the per-kernel profiler. */
+typedef enum {
+  TL_KERNEL_EMBED = 0,        /* embedding gather */
+  TL_KERNEL_QKV = 1,          /* RMSNorm + QKV INT4 linear + RoPE + KV write */
+  TL_KERNEL_ATTN_DECODE = 2,  /* single-query cached-decode attention */
+  TL_KERNEL_O_PROJ = 3,       /* O INT4 linear + residual */
+  TL_KERNEL_GATE_UP = 4,      /* RMSNorm + gate_up INT4 linear + SwiGLU */
+  TL_KERNEL_DOWN = 5,         /* down INT4 linear + residual */
+  TL_KERNEL_HEAD = 6,         /* output norm + head + greedy argmax */
+  TL_KERNEL_ATTN_PREFILL = 7, /* tiled causal prefill attention */
+  TL_KERNEL_GEMM_TC = 8,      /* tensor-core INT4 GEMM (prefill linears) */
+  TL_KERNEL_NORM = 9,         /* stand-alone RMSNorm */
+  TL_KERNEL_SETUP = 10,       /* per-call row bookkeeping */
+  TL_KERNEL_CLASSES = 11
+} tl_kernel_class;
+
+/* Per-kernel timing (the counterpart of the pages' phase timings, TinyLoop
+ * README, "Quick CLI Tour", Benchmark with TINYLOOP_CUDA_PROFILE=1): from
+ * this call on, every launch of the model whose class bit is set in
+ * class_mask (bit c = class c) is bracketed by two CUDA events on its stream,
+ * up to 16384 launches.  Events between launches serialise them, so profiled
+ * runs are slower than unprofiled ones. */
+tl_status tl_model_profile_start(tl_model *m, unsigned class_mask);
+
+/* Stop profiling; waits for the recorded events and writes, per class,
+ * the number of timed launches and their summed duration in ms.
+ *   h_launches int [TL_KERNEL_CLASSES] or NULL, h_total_ms float [..] or NULL */
+tl_status tl_model_profile_stop(tl_model *m, int *h_launches, float *h_total_ms);
+
+/* Number of kernels this library has launched in the process so far. */
+unsigned long long tl_kernel_launch_count(void);
+
+/* ------------------------------------------------------------------------
+ * Op API: the hot-path kernels on caller-provided tensors
+ * ------------------------------------------------------------------------ */
+
+/* An INT4 linear (storage format above, HOST memory) copied to `device` and
+ * re-laid out for the kernels.  K is a multiple of 128 and 128 <= K <= 16384;
+ * 1 <= N <= 65536.  The host arrays may be freed when this returns. */
+tl_status tl_linear_create(const tl_int4_linear *w, int K, int N, int device,
+                           tl_linear **out);
+void tl_linear_destroy(tl_linear *l);
+
+/* Kernel family used by tl_linear_forward. */
+typedef enum {
+  TL_PATH_AUTO = 0,   /* GEMV for M <= 16, tensor-core GEMM otherwise */
+  TL_PATH_GEMV = 1,   /* INT4 GEMV on mma.sync, any M (16 rows per launch) */
+  TL_PATH_TC = 2      /* INT4 GEMM on tcgen05 tensor cores, any M */
+} tl_path;
+
+/* y = x W^T with fp32 accumulation (dequantisation w = (q - z) * s).
+ *   d_x  fp16 [M][K] row-major, d_y fp16 [M][N] row-major, M >= 1.
+ * Returns TL_ERR_UNSUPPORTED if `path` is not built for this shape. */
+tl_status tl_linear_forward(tl_linear *l, const uint16_t *d_x, int M, uint16_t *d_y,
+                            int path, void *stream);
+
+/* RMSNorm (tiny-llm feature list, "Root Mean Square Normalizations"):
+ * y[r][i] = fp16(x[r][i] / sqrt(mean_i(x[r][i]^2) + eps) * g[i]).
+ *   d_x fp32 [rows][d], d_g fp16 [d], d_y fp16 [rows][d]; d a multiple of 8. */
+tl_status tl_op_rmsnorm(const float *d_x, const uint16_t *d_g, int rows, int d, float eps,
+                        uint16_t *d_y, void *stream);
+
+/* In-place rotary embedding of Q or K (TinyLoop README, "Status", RoPE, fused
+ * in-place Q/K rotation with configurable theta).  Token t, head h starts at
+ * d_x + t*token_stride + h*head_stride (fp16 elements); element j and
+ * j + head_dim/2 rotate by angle pos[t] * theta^(-2j/head_dim).
+ *   d_positions int32 [n_tokens], each >= 0; head_dim even, <= 256. */
+tl_status tl_op_rope(uint16_t *d_x, int n_tokens, int n_heads, int head_dim,
+                     long long token_stride, long long head_stride,
+                     const int32_t *d_positions, float theta, void *stream);
+
+/* Single-query cached-decode GQA attention (TinyLoop README, "Current Runtime
+ * Snapshot", direct single-query decode kernel; "Status", GQA).  For batch
+ * entry b the keys and values are the planes
+ *   K_b = d_k + b*batch_stride, V_b = d_v + b*batch_stride,
+ * each laid out [n_kv_heads][ctx_stride][head_dim] fp16 and already rotated;
+ * query b (fp16 [n_q_heads][head_dim] at d_q + b*n_q_heads*head_dim, already
+ * rotated) attends to keys 0..n_keys[b]-1.  q head h reads kv head
+ * h / (n_q_heads/n_kv_heads); scale 1/sqrt(head_dim).
+ *   h_n_keys  int32 [B] HOST, 1 <= n_keys[b] <= ctx_stride
+ *   d_out     fp16 [B][n_q_heads][head_dim]
+ * Uses a library-owned device workspace (allocated on first use, grown as
+ * needed) for the split-KV partial results. */
+tl_status tl_op_gqa_decode(const uint16_t *d_q, const uint16_t *d_k, const uint16_t *d_v,
+                           long long batch_stride, int ctx_stride, const int32_t *h_n_keys,
+                           int B, int n_q_heads, int n_kv_heads, int head_dim,
+                           uint16_t *d_out, void *stream);
+
+/* Causal tiled prefill GQA attention (TinyLoop README, "Current Runtime
+ * Snapshot", tiled prefill path; tiny-llm feature list, "Tiled Online
+ * Softmax", "Causal Masking").  Queries d_q fp16 [B][T][n_q_heads][head_dim]
+ * (rotated) at positions pos0..pos0+T-1 attend to keys 0..pos0+t of the planes
+ * described as in tl_op_gqa_decode.  d_out fp16 [B][T][n_q_heads][head_dim].
+ * pos0 + T <= ctx_stride. */
+tl_status tl_op_gqa_prefill(const uint16_t *d_q, const uint16_t *d_k, const uint16_t *d_v,
+                            long long batch_stride, int ctx_stride, int T, int pos0, int B,
+                            int n_q_heads, int n_kv_heads, int head_dim, uint16_t *d_out,
+                            void *stream);
+
+/* ------------------------------------------------------------------------
+ * Misc
+ * ------------------------------------------------------------------------ */
+
+/* Static string naming a status. */
+const char *tl_status_string(tl_status s);
+
+/* One-line reason for the last non-OK status returned on the calling thread
+ * (empty string if none).  Valid until the next call on that thread. */
+const char *tl_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char *tl_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TL_H_ */

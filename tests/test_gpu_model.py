@@ -1,0 +1,210 @@
+"""The looped model end to end on the GPU against the fp64 oracle.
+
+Workloads:
+* tiny looped LM (d 256, 4/2 heads of 64, F 1024, V 512, 1 pre block, L = 4):
+  32-token prompt, then 8 greedy decode steps, batch 1;
+* the ~400M-unique looped LM (d 2048, 16/4 heads of 128, F 5632, V 32000,
+  2 pre blocks, L = 8): 128-token prompt prefilled with no logits, then greedy
+  decode steps at batch 1;
+* the same model with per-lane loops drawn from {4, 8, 16}.
+
+Decoding is teacher-forced with the oracle's tokens, so an allowed near-tie
+argmax flip cannot change later steps.  Bounds: logits max-abs <= 2e-2, argmax
+exact unless the oracle's top-2 margin is < 1e-3.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import tl_synth
+import weight_shared_looped_int4_b200 as tl
+from gpu_helpers import DEV, LOGIT_MAX_ABS, GpuModel, check_argmax, need_gpu
+from oracle import ref
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    need_gpu()
+    w = tl_synth.make_model_weights(tl_synth.TINY_LM, tl_synth.SEED_TINY)
+    om = ref.LoopedModel(w)
+    gm = GpuModel(w, max_loops=16, max_ctx=256, max_lanes=16)
+    yield w, om, gm
+    gm.close()
+
+
+def _max_abs(a, b):
+    return float(np.max(np.abs(np.asarray(a) - np.asarray(b))))
+
+
+def test_tiny_prefill_decode(tiny):
+    w, om, gm = tiny
+    L, P, steps = 4, 32, 8
+    prompt = tl_synth.make_tokens(tl_synth.SEED_TINY, w.shape.vocab, P + 1)
+    # oracle: logits at positions P .. P+steps-1 (prefill of P+1 ids = first decode step)
+    o_tokens, o_logits = om.generate_greedy(prompt, L, steps)
+    # GPU: prefill P ids with logits of position P-1, then decode prompt[P], ...
+    lg, am = gm.prefill_lane(0, prompt[:P], L)
+    _, o_prefill_logits = om.prefill(prompt[:P], L)
+    assert _max_abs(lg, o_prefill_logits) <= LOGIT_MAX_ABS
+    check_argmax(am, o_prefill_logits, "prefill")
+    fed = int(prompt[P])
+    for i in range(steps):
+        glg, gam = gm.decode([0], [fed], [L])
+        err = _max_abs(glg[0], o_logits[i])
+        assert err <= LOGIT_MAX_ABS, (i, err)
+        check_argmax(int(gam[0]), o_logits[i], f"step {i}")
+        fed = o_tokens[i]
+    assert tl.tl_lane_length(gm.handle, 0) == P + steps
+
+
+def test_tiny_score_last(tiny):
+    w, om, gm = tiny
+    for n, L in ((1, 1), (17, 3), (100, 16)):
+        toks = tl_synth.make_tokens(n + L, w.shape.vocab, n)
+        lg, am = gm.score_last(toks, L)
+        expect = om.score_last(toks, L)
+        assert _max_abs(lg, expect) <= LOGIT_MAX_ABS
+        check_argmax(am, expect, "score_last")
+
+
+def test_tiny_cached_equals_uncached_on_gpu(tiny):
+    # Decode step i must agree with a fresh uncached forward of the prefix.
+    w, om, gm = tiny
+    prompt = tl_synth.make_tokens(55, w.shape.vocab, 20)
+    gm.prefill_lane(1, prompt[:12], 4, logits=False)
+    seq = list(prompt[:12])
+    for i in range(12, 20):
+        glg, _ = gm.decode([1], [int(prompt[i])], [4])
+        seq.append(int(prompt[i]))
+        ulg, _ = gm.score_last(seq, 4)
+        assert _max_abs(glg[0], ulg) <= 2e-3
+
+
+def test_tiny_looped_equals_flattened_on_gpu(tiny):
+    # A model whose pre blocks are [pre..., loop x (L-1)] and whose loop block
+    # runs once is the same computation with distinct weight copies.
+    w, om, gm = tiny
+    L = 4
+    flat = tl_synth.ModelWeights(
+        shape=tl_synth.ModelShape(**{**w.shape.__dict__, "n_pre": w.shape.n_pre + L - 1}),
+        embed=w.embed, out_norm=w.out_norm, head=w.head,
+        pre=list(w.pre) + [w.loop] * (L - 1), loop=w.loop)
+    fm = GpuModel(flat, max_loops=1, max_ctx=64, max_lanes=1)
+    try:
+        toks = tl_synth.make_tokens(99, w.shape.vocab, 40)
+        a, _ = gm.score_last(toks, L)
+        b, _ = fm.score_last(toks, 1)
+        assert np.array_equal(a, b)
+    finally:
+        fm.close()
+
+
+def test_tiny_per_lane_loops_independent(tiny):
+    # Lanes with loops 4, 8, 16 decoded together give bitwise the results of
+    # decoding each lane alone.
+    w, om, gm = tiny
+    loops = [4, 16, 8]
+    prompts = tl_synth.make_lane_prompts(7, w.shape.vocab, 3, 10)
+    nxt = [5, 6, 7]
+    for lane, L in enumerate(loops):
+        gm.prefill_lane(2 + lane, prompts[lane], L, logits=False)
+    together, _ = gm.decode([2, 3, 4], nxt, loops)
+    for lane, L in enumerate(loops):
+        gm.prefill_lane(2 + lane, prompts[lane], L, logits=False)
+    for lane, L in enumerate(loops):
+        alone, _ = gm.decode([2 + lane], [nxt[lane]], [L])
+        assert np.array_equal(alone[0], together[lane])
+        # and against the oracle
+        cache, _ = om.prefill(prompts[lane], L)
+        expect = om.decode(cache, nxt[lane], L)
+        assert _max_abs(alone[0], expect) <= LOGIT_MAX_ABS
+
+
+def test_tiny_errors(tiny):
+    w, om, gm = tiny
+    gm.prefill_lane(5, [1, 2, 3], 4, logits=False)
+    with pytest.raises(tl.TLError) as e:
+        gm.decode([5], [1], [8])
+    assert e.value.status == tl.TL_ERR_LOOPS_MISMATCH
+    with pytest.raises(tl.TLError) as e:
+        gm.decode([15], [1], [4])
+    assert e.value.status == tl.TL_ERR_NOT_PREFILLED
+    with pytest.raises(tl.TLError) as e:
+        gm.decode([5, 5], [1, 1], [4, 4])
+    assert e.value.status == tl.TL_ERR_INVALID_ARG
+    with pytest.raises(tl.TLError) as e:
+        gm.prefill_lane(0, [1] * 300, 4)
+    assert e.value.status == tl.TL_ERR_CONTEXT_FULL
+    # a token id out of range is replaced by 0 and flagged, not trapped
+    tl.tl_check_device_error(gm.handle)
+    gm.score_last([1, w.shape.vocab + 5], 2)
+    with pytest.raises(tl.TLError) as e:
+        tl.tl_check_device_error(gm.handle)
+    assert e.value.status == tl.TL_ERR_DEVICE_FLAG
+    tl.tl_check_device_error(gm.handle)   # cleared
+
+
+def test_tiny_context_full(tiny):
+    w, om, gm = tiny
+    gm.prefill_lane(6, list(range(255)), 1, logits=False)
+    gm.decode([6], [1], [1])
+    with pytest.raises(tl.TLError) as e:
+        gm.decode([6], [1], [1])
+    assert e.value.status == tl.TL_ERR_CONTEXT_FULL
+
+
+# --------------------------------------------------------- the ~400M model ---
+
+@pytest.fixture(scope="module")
+def lm():
+    need_gpu()
+    w = tl_synth.make_model_weights(tl_synth.LOOPED_LM, tl_synth.SEED_LM)
+    om = ref.LoopedModel(w)
+    gm = GpuModel(w, max_loops=16, max_ctx=2048, max_lanes=16)
+    yield w, om, gm
+    gm.close()
+
+
+def test_lm_prefill_then_decode(lm):
+    w, om, gm = lm
+    L, P, steps = 8, 128, 6
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, w.shape.vocab, P + 1)
+    o_tokens, o_logits = om.generate_greedy(prompt, L, steps)
+    gm.prefill_lane(0, prompt[:P], L, logits=False)
+    fed = int(prompt[P])
+    for i in range(steps):
+        glg, gam = gm.decode([0], [fed], [L])
+        err = _max_abs(glg[0], o_logits[i])
+        assert err <= LOGIT_MAX_ABS, (i, err)
+        check_argmax(int(gam[0]), o_logits[i], f"step {i}")
+        fed = o_tokens[i]
+
+
+def test_lm_score_last(lm):
+    w, om, gm = lm
+    toks = tl_synth.make_tokens(17, w.shape.vocab, 77)
+    for L in (1, 8):
+        lg, am = gm.score_last(toks, L)
+        expect = om.score_last(toks, L)
+        assert _max_abs(lg, expect) <= LOGIT_MAX_ABS
+        check_argmax(am, expect, f"L={L}")
+
+
+def test_lm_lanes_per_lane_loops(lm):
+    # Lanes with loops drawn from {4, 8, 16}, prompts of 512 ids; two lanes
+    # are checked against the oracle, all against their solo runs.
+    w, om, gm = lm
+    n_lanes, P = 4, 512
+    loops = [int(v) for v in tl_synth.make_lane_loops(tl_synth.SEED_LSWEEP, n_lanes)]
+    prompts = tl_synth.make_lane_prompts(tl_synth.SEED_LSWEEP, w.shape.vocab, n_lanes, P + 1)
+    lanes = list(range(n_lanes))
+    for i in lanes:
+        gm.prefill_lane(i, prompts[i, :P], loops[i], logits=False)
+    together, am = gm.decode(lanes, [int(p[P]) for p in prompts], loops)
+    for i in (0, n_lanes - 1):
+        expect = om.score_last(prompts[i, :P + 1], loops[i])   # = decode step at position P
+        assert _max_abs(together[i], expect) <= LOGIT_MAX_ABS
+        check_argmax(int(am[i]), expect, f"lane {i}")

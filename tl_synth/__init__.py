@@ -197,10 +197,12 @@ def make_activations(seed: int, M: int, K: int) -> np.ndarray:
 
 
 def make_qkv(seed: int, batch: int, T: int, n_q_heads: int, n_kv_heads: int,
-             head_dim: int):
-    """float16 Q [B][T][Hq][hd], K and V [B][T][Hkv][hd], all ~ N(0, 1)."""
+             head_dim: int, T_q: int = None):
+    """float16 K and V [B][T][Hkv][hd], then Q [B][T_q][Hq][hd] (T_q defaults
+    to T), all ~ N(0, 1), drawn in that order from one stream."""
     rng = np.random.default_rng(seed)
-    q = rng.normal(0.0, 1.0, size=(batch, T, n_q_heads, head_dim)).astype(np.float16)
     k = rng.normal(0.0, 1.0, size=(batch, T, n_kv_heads, head_dim)).astype(np.float16)
     v = rng.normal(0.0, 1.0, size=(batch, T, n_kv_heads, head_dim)).astype(np.float16)
+    tq = T if T_q is None else T_q
+    q = rng.normal(0.0, 1.0, size=(batch, tq, n_q_heads, head_dim)).astype(np.float16)
     return q, k, v

@@ -1,0 +1,114 @@
+// Device helpers shared by the sm_100a kernels: PTX wrappers for programmatic
+// dependent launch, streaming loads, the m16n8k16 fp16 MMA and INT4 unpacking.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tl {
+
+constexpr int kGroup = 128;      // INT4 group size along K
+constexpr int kMaxLanes = 16;    // rows of activations a GEMV launch handles
+
+// ---- programmatic dependent launch -------------------------------------
+// Every kernel of the forward pass calls pdl_trigger() early (so the next
+// kernel may start its weight prefetch) and pdl_wait() before it reads any
+// activation the previous kernel wrote.  Every kernel waits, so completion is
+// transitive along the stream.
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- loads ---------------------------------------------------------------
+// Weights are read once per pass: do not keep them in L1.
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ uint2 ldg_stream2(const uint2* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+
+// ---- tensor-core MMA (m16n8k16, fp16 in, fp32 accumulate) ----------------
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ---- INT4 unpacking -------------------------------------------------------
+// (w & mask) | 0x64006400 turns the two nibbles at bits 0..3 and 16..19 into
+// the fp16 pair (1024 + n_lo, 1024 + n_hi): 0x6400 is 1024 and one unit in the
+// last place of that binade is 1, so the nibble lands in the integer part.
+__device__ __forceinline__ uint32_t nib_pair_to_h2_biased(uint32_t w) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x000F000Fu), "r"(0x64006400u));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t h2_sub(uint32_t a, uint32_t b) {
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t h2_mul(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+// Broadcast the low / high half of a pair into both halves.
+__device__ __forceinline__ uint32_t h2_lo_lo(uint32_t a) { return __byte_perm(a, 0, 0x1010); }
+__device__ __forceinline__ uint32_t h2_hi_hi(uint32_t a) { return __byte_perm(a, 0, 0x3232); }
+
+__device__ __forceinline__ float2 h2_to_f2(uint32_t a) {
+  return __half22float2(*reinterpret_cast<__half2*>(&a));
+}
+
+// Unpack one packed word of the tiled INT4 layout into the A fragment of an
+// m16n8k16 MMA, with the zero point already removed: every element is the
+// exact small integer q - z in fp16.
+//   zz = (1024 + z_row_g, 1024 + z_row_g+8) as an fp16 pair.
+__device__ __forceinline__ void unpack_a_frag(uint32_t w, uint32_t zz, uint32_t (&a)[4]) {
+  const uint32_t zlo = h2_lo_lo(zz), zhi = h2_hi_hi(zz);
+  a[0] = h2_sub(nib_pair_to_h2_biased(w), zlo);        // row g,   k 2t..2t+1
+  a[1] = h2_sub(nib_pair_to_h2_biased(w >> 4), zhi);   // row g+8, k 2t..2t+1
+  a[2] = h2_sub(nib_pair_to_h2_biased(w >> 8), zlo);   // row g,   k 2t+8..2t+9
+  a[3] = h2_sub(nib_pair_to_h2_biased(w >> 12), zhi);  // row g+8, k 2t+8..2t+9
+}
+
+// ---- reductions -----------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float silu(float u) { return u / (1.0f + expf(-u)); }
+
+// RoPE angle of pair j at position p: p * theta^(-2j/hd), evaluated in double
+// precision and returned as (cos, sin) in float.
+__device__ __forceinline__ float2 rope_cos_sin(int pos, int j, int hd, float theta) {
+  const double inv_freq = exp(-(2.0 * (double)j / (double)hd) * log((double)theta));
+  double s, c;
+  sincos((double)pos * inv_freq, &s, &c);
+  return make_float2((float)c, (float)s);
+}
+
+}  // namespace tl

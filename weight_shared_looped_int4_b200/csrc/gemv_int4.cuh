@@ -1,0 +1,332 @@
+// INT4 group-wise dequant GEMV for the decode path (and short prefill chunks):
+// y[m][n] = sum_k x[m][k] * (q[n][k] - z[n][k/128]) * s[n][k/128], m < 16.
+//
+// Definition: TinyLoop README, "Status" (INT4 loop / pre linears with zero
+// points); the group size, fp16 scale and 4-bit zero are the workload's
+// w = (q - z) * s.  The kernel design is ours, for sm_100a:
+//
+// * Weights are re-laid out at load time so that one 16-byte load of a lane
+//   holds the A fragments of four m16n8k16 MMAs (64 consecutive k of rows g
+//   and g+8 of a 16-row tile).  A warp load is 512 contiguous bytes.
+// * Unpacking is a LOP3 per nibble pair (the 1024-bias trick) and one fp16
+//   subtract of the biased zero point; q - z is an exact small integer in fp16,
+//   so the tensor-core product with the fp16 activation is exact and the MMA
+//   accumulates in fp32.  The fp16 scale is applied in fp32 once per 64-wide
+//   K chunk, so no weight is ever rounded.
+// * Each CTA owns a pair of 16-row tiles (the pair an epilogue needs: RoPE
+//   halves of one head, gate/up rows of SwiGLU, or two neighbours) and all of
+//   K; its 8 warps split (tile, K quarter) and reduce through shared memory in
+//   a fixed order, so results are deterministic and each activation row's
+//   result does not depend on how many rows share the launch.
+// * Weight prefetch is issued before griddepcontrol.wait, so it overlaps the
+//   tail of the previous kernel under programmatic dependent launch.
+// * The prologue can fuse the block's RMSNorm (fp32 residual in, fp16 out into
+//   shared memory); the epilogue fuses RoPE + KV-cache write, SwiGLU, or the
+//   residual add.
+#pragma once
+
+#include "common.cuh"
+
+namespace tl {
+
+enum GemvIn { IN_NORM = 0, IN_F16 = 1 };
+enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_ROPE_KV = 3 };
+enum PairMode { PAIR_NEIGHBOUR = 0, PAIR_OFFSET = 1, PAIR_ROPE = 2 };
+
+// Per activation row: which KV-cache lane it writes and at what position.
+struct RowCtx {
+  int lane;
+  int pos;
+};
+
+struct GemvArgs {
+  const uint4* w;      // tiled weights  [n_tiles][K/64][32] (see repack)
+  const uint2* sz;     // scales / zeros [n_tiles][K/128][8]
+  int K;               // multiple of 128
+  int n_rows;          // valid output rows N
+  int M;               // activation rows, 1..16
+  // input
+  const float* x;      // IN_NORM: fp32 [M][ldx]
+  const __half* xh;    // IN_F16:  fp16 [M][ldx]
+  int ldx;
+  const __half* gain;  // IN_NORM: RMSNorm gains [K]
+  float eps;
+  // tile pairing
+  int pair_mode;
+  int pair_off;        // PAIR_OFFSET: tiles between the two; PAIR_ROPE: hd/32
+  // outputs
+  __half* y;           // EPI_STORE / EPI_SWIGLU: fp16 [M][ldy]
+  int ldy;
+  float* resid;        // EPI_RESID: fp32 [M][ldr] += y
+  int ldr;
+  // EPI_ROPE_KV
+  __half* q_out;       // fp16 [M][ldq], rows < n_q_rows
+  int ldq;
+  int n_q_rows;        // Hq * hd
+  int n_kv_rows;       // Hkv * hd
+  int hd;
+  __half* k_plane;     // K plane of this layer for lane 0: [Hkv][ctx][hd]
+  __half* v_plane;     // V plane of this layer for lane 0
+  long long lane_stride;
+  int ctx;
+  const RowCtx* rows;  // per activation row
+  float theta;
+};
+
+constexpr int kGemvThreads = 256;
+constexpr int kGemvPrefetch = 8;
+
+__host__ __device__ inline size_t gemv_smem_bytes(int K, int nt) {
+  return (size_t)nt * 8 * (K + 8) * 2 + (size_t)4 * 2 * 16 * nt * 8 * 4;
+}
+
+template <int NT, int IN, int EPI>
+__global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int K = a.K;
+  const int ldxs = K + 8;
+  __half* xs = reinterpret_cast<__half*>(smem);
+  float* red = reinterpret_cast<float*>(smem + (size_t)NT * 8 * ldxs * 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int tsel = warp & 1, kq = warp >> 1;
+
+  int t0, t1;
+  if (a.pair_mode == PAIR_NEIGHBOUR) {
+    t0 = 2 * blockIdx.x;
+    t1 = t0 + 1;
+  } else if (a.pair_mode == PAIR_OFFSET) {
+    t0 = blockIdx.x;
+    t1 = t0 + a.pair_off;
+  } else {
+    const int head = blockIdx.x / a.pair_off, j16 = blockIdx.x % a.pair_off;
+    t0 = head * 2 * a.pair_off + j16;
+    t1 = t0 + a.pair_off;
+  }
+  const int tile = tsel ? t1 : t0;
+
+  const int n_chunks = K >> 6;
+  const int c_begin = (n_chunks * kq) >> 2;
+  const int nc = ((n_chunks * (kq + 1)) >> 2) - c_begin;
+  const uint4* wp = a.w + ((size_t)tile * n_chunks + c_begin) * 32 + lane;
+  const uint2* szp = a.sz + (size_t)tile * (K >> 7) * 8 + g;
+
+  pdl_trigger();
+
+  uint4 buf[kGemvPrefetch];
+  uint2 szb[kGemvPrefetch];
+#pragma unroll
+  for (int i = 0; i < kGemvPrefetch; ++i) {
+    if (i < nc) {
+      buf[i] = ldg_stream(wp + (size_t)i * 32);
+      szb[i] = __ldg(szp + ((c_begin + i) >> 1) * 8);
+    }
+  }
+
+  pdl_wait();
+
+  // ---- stage the activations (fp16, RMSNorm fused for IN_NORM) -----------
+  if (IN == IN_NORM) {
+    for (int m = warp; m < NT * 8; m += 8) {
+      __half* dst = xs + m * ldxs;
+      if (m < a.M) {
+        const float* src = a.x + (size_t)m * a.ldx;
+        float ss = 0.f;
+        for (int k = lane * 4; k < K; k += 128) {
+          const float4 v = *reinterpret_cast<const float4*>(src + k);
+          ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+        }
+        ss = warp_sum(ss);
+        const float rs = 1.0f / sqrtf(ss / (float)K + a.eps);
+        for (int k = lane * 4; k < K; k += 128) {
+          const float4 v = *reinterpret_cast<const float4*>(src + k);
+          const __half2 g01 = *reinterpret_cast<const __half2*>(a.gain + k);
+          const __half2 g23 = *reinterpret_cast<const __half2*>(a.gain + k + 2);
+          const float2 fg01 = __half22float2(g01), fg23 = __half22float2(g23);
+          __half2 o01 = __floats2half2_rn((v.x * rs) * fg01.x, (v.y * rs) * fg01.y);
+          __half2 o23 = __floats2half2_rn((v.z * rs) * fg23.x, (v.w * rs) * fg23.y);
+          uint2 pk;
+          pk.x = *reinterpret_cast<uint32_t*>(&o01);
+          pk.y = *reinterpret_cast<uint32_t*>(&o23);
+          *reinterpret_cast<uint2*>(dst + k) = pk;
+        }
+      } else {
+        for (int k = lane * 4; k < K; k += 128) *reinterpret_cast<uint2*>(dst + k) = make_uint2(0, 0);
+      }
+    }
+  } else {
+    for (int m = warp; m < NT * 8; m += 8) {
+      __half* dst = xs + m * ldxs;
+      if (m < a.M) {
+        const __half* src = a.xh + (size_t)m * a.ldx;
+        for (int k = lane * 8; k < K; k += 256)
+          *reinterpret_cast<uint4*>(dst + k) = *reinterpret_cast<const uint4*>(src + k);
+      } else {
+        for (int k = lane * 8; k < K; k += 256) *reinterpret_cast<uint4*>(dst + k) = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- main loop: 64-wide K chunks, 4 MMAs each ---------------------------
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+
+  for (int base = 0; base < nc; base += kGemvPrefetch) {
+#pragma unroll
+    for (int i = 0; i < kGemvPrefetch; ++i) {
+      const int ci = base + i;
+      if (ci < nc) {
+        const uint4 wv = buf[i];
+        const uint2 sv = szb[i];
+        if (ci + kGemvPrefetch < nc) {
+          buf[i] = ldg_stream(wp + (size_t)(ci + kGemvPrefetch) * 32);
+          szb[i] = __ldg(szp + ((c_begin + ci + kGemvPrefetch) >> 1) * 8);
+        }
+        const int kc = (c_begin + ci) * 64 + 2 * t;
+        float tmp[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) tmp[nt][q] = 0.f;
+        const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t af[4];
+          unpack_a_frag(words[j], sv.y, af);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const __half* xr = xs + (nt * 8 + g) * ldxs + kc + j * 16;
+            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xr);
+            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xr + 8);
+            mma_f16_16816(tmp[nt], af, b0, b1);
+          }
+        }
+        const float2 s = h2_to_f2(sv.x);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          acc[nt][0] = fmaf(s.x, tmp[nt][0], acc[nt][0]);
+          acc[nt][1] = fmaf(s.x, tmp[nt][1], acc[nt][1]);
+          acc[nt][2] = fmaf(s.y, tmp[nt][2], acc[nt][2]);
+          acc[nt][3] = fmaf(s.y, tmp[nt][3], acc[nt][3]);
+        }
+      }
+    }
+  }
+
+  // ---- reduce the four K quarters (fixed order) ---------------------------
+  constexpr int NC = NT * 8;  // activation columns
+  float* myred = red + (kq * 2 + tsel) * 16 * NC;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const int col = nt * 8 + 2 * t;
+    myred[g * NC + col] = acc[nt][0];
+    myred[g * NC + col + 1] = acc[nt][1];
+    myred[(g + 8) * NC + col] = acc[nt][2];
+    myred[(g + 8) * NC + col + 1] = acc[nt][3];
+  }
+  __syncthreads();
+
+  const int r = threadIdx.x & 15, m = threadIdx.x >> 4;
+  if (m >= a.M || m >= NC) return;
+  float va = 0.f, vb = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    va += red[(q * 2 + 0) * 16 * NC + r * NC + m];
+    vb += red[(q * 2 + 1) * 16 * NC + r * NC + m];
+  }
+  const int row0 = t0 * 16 + r, row1 = t1 * 16 + r;
+
+  if (EPI == EPI_STORE) {
+    if (row0 < a.n_rows) a.y[(size_t)m * a.ldy + row0] = __float2half_rn(va);
+    if (row1 < a.n_rows) a.y[(size_t)m * a.ldy + row1] = __float2half_rn(vb);
+  } else if (EPI == EPI_RESID) {
+    if (row0 < a.n_rows) a.resid[(size_t)m * a.ldr + row0] += va;
+    if (row1 < a.n_rows) a.resid[(size_t)m * a.ldr + row1] += vb;
+  } else if (EPI == EPI_SWIGLU) {
+    a.y[(size_t)m * a.ldy + row0] = __float2half_rn(silu(va) * vb);
+  } else {  // EPI_ROPE_KV: row0 is element j < hd/2 of a head, row1 = row0 + hd/2
+    const int hd = a.hd;
+    const int j = row0 % hd;
+    const RowCtx rc = a.rows[m];
+    if (row0 < a.n_q_rows) {
+      const float2 cs = rope_cos_sin(rc.pos, j, hd, a.theta);
+      __half* qo = a.q_out + (size_t)m * a.ldq;
+      qo[row0] = __float2half_rn(va * cs.x - vb * cs.y);
+      qo[row1] = __float2half_rn(vb * cs.x + va * cs.y);
+    } else if (row0 < a.n_q_rows + a.n_kv_rows) {
+      const float2 cs = rope_cos_sin(rc.pos, j, hd, a.theta);
+      const int kvh = (row0 - a.n_q_rows) / hd;
+      __half* dst = a.k_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
+      dst[j] = __float2half_rn(va * cs.x - vb * cs.y);
+      dst[j + hd / 2] = __float2half_rn(vb * cs.x + va * cs.y);
+    } else {
+      const int kvh = (row0 - a.n_q_rows - a.n_kv_rows) / hd;
+      __half* dst = a.v_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
+      dst[j] = __float2half_rn(va);
+      dst[j + hd / 2] = __float2half_rn(vb);
+    }
+  }
+}
+
+// ---- load-time re-layout ----------------------------------------------------
+// Nibble i of packed word j for (tile T, chunk c, lane l = 4g + t) holds, with
+// r0 = 16T + g, r1 = r0 + 8, kb = 64c + 16j:
+//   0:(r0,kb+2t) 1:(r1,kb+2t) 2:(r0,kb+2t+8) 3:(r1,kb+2t+8)
+//   4:(r0,kb+2t+1) 5:(r1,kb+2t+1) 6:(r0,kb+2t+9) 7:(r1,kb+2t+9)
+// so that unpack_a_frag yields the m16n8k16 A fragment.  Rows >= N are zero.
+__global__ void repack_int4_weights_kernel(const uint32_t* __restrict__ qweight, int K, int N,
+                                           int n_tiles, uint4* __restrict__ out) {
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int n_chunks = K >> 6;
+  const size_t total = (size_t)n_tiles * n_chunks * 32;
+  if (idx >= total) return;
+  const int l = (int)(idx & 31);
+  const size_t rest = idx >> 5;
+  const int c = (int)(rest % n_chunks);
+  const int T = (int)(rest / n_chunks);
+  const int g = l >> 2, t = l & 3;
+  const int r0 = T * 16 + g, r1 = r0 + 8;
+  const int kw = K >> 3;
+  auto q = [&](int r, int k) -> uint32_t {
+    if (r >= N) return 0u;
+    return (qweight[(size_t)r * kw + (k >> 3)] >> (4 * (k & 7))) & 0xFu;
+  };
+  uint32_t wd[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int kb = c * 64 + j * 16 + 2 * t;
+    wd[j] = q(r0, kb) | (q(r1, kb) << 4) | (q(r0, kb + 8) << 8) | (q(r1, kb + 8) << 12) |
+            (q(r0, kb + 1) << 16) | (q(r1, kb + 1) << 20) | (q(r0, kb + 9) << 24) |
+            (q(r1, kb + 9) << 28);
+  }
+  out[idx] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+}
+
+// sz[T][group][g] = {(s[r0], s[r1]) fp16 pair, (1024 + z[r0], 1024 + z[r1]) fp16 pair}
+__global__ void repack_int4_scales_kernel(const uint16_t* __restrict__ scales,
+                                          const uint32_t* __restrict__ qzeros, int K, int N,
+                                          int n_tiles, uint2* __restrict__ out) {
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int G = K >> 7;
+  const int zw = (G + 7) >> 3;
+  const size_t total = (size_t)n_tiles * G * 8;
+  if (idx >= total) return;
+  const int g = (int)(idx & 7);
+  const size_t rest = idx >> 3;
+  const int gr = (int)(rest % G);
+  const int T = (int)(rest / G);
+  const int r0 = T * 16 + g, r1 = r0 + 8;
+  auto sc = [&](int r) -> uint32_t { return r < N ? (uint32_t)scales[(size_t)r * G + gr] : 0u; };
+  auto zb = [&](int r) -> uint32_t {
+    const uint32_t z = r < N ? (qzeros[(size_t)r * zw + (gr >> 3)] >> (4 * (gr & 7))) & 0xFu : 0u;
+    return 0x6400u + z;  // fp16 bits of 1024 + z
+  };
+  out[idx] = make_uint2(sc(r0) | (sc(r1) << 16), zb(r0) | (zb(r1) << 16));
+}
+
+}  // namespace tl

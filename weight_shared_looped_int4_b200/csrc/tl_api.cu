@@ -1,0 +1,1006 @@
+// Host runtime behind the C ABI (include/tl.h): model creation and weight
+// re-layout, the KV cache, the prefill / decode / score drivers with the loop
+// over the shared block, and the op entry points.
+//
+// The forward pass follows TinyLoop README, "Why TinyLoop Exists":
+// tokens -> embed -> pre blocks -> shared loop block x L -> output norm -> head.
+// Effective layer l uses pre[l] for l < n_pre and the one loop block after
+// that; its keys and values go to cache slice l of the lane.
+
+#include "../../include/tl.h"
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemv_int4.cuh"
+#include "misc.cuh"
+
+using namespace tl;
+
+// ============================================================================
+// errors
+// ============================================================================
+namespace {
+
+thread_local std::string g_err;
+
+tl_status fail(tl_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+tl_status cuda_fail(cudaError_t e, const char* what) {
+  cudaGetLastError();  // clear a sticky-free launch error
+  return fail(e == cudaErrorMemoryAllocation ? TL_ERR_OOM : TL_ERR_CUDA, "%s: %s", what,
+              cudaGetErrorString(e));
+}
+
+#define TL_CUDA(call)                                   \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess) ok = true;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+// ============================================================================
+// per-kernel event profiler and launch counter
+// ============================================================================
+struct Profiler {
+  unsigned mask = 0;                 // classes being timed (0 = off)
+  std::vector<cudaEvent_t> ev;       // begin/end pairs
+  std::vector<int> cls;              // class of each pair
+  int used = 0;
+  static constexpr int kCapacity = 16384;
+  void destroy() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    ev.clear();
+    cls.clear();
+    used = 0;
+    mask = 0;
+  }
+};
+
+thread_local Profiler* g_prof = nullptr;  // profiler of the model in the current call
+thread_local int g_cls = -1;              // class of the next launch
+std::atomic<unsigned long long> g_launches{0};
+
+struct ProfScope {  // installs a model's profiler for the duration of one API call
+  Profiler* prev;
+  explicit ProfScope(Profiler* p) : prev(g_prof) { g_prof = p; g_cls = -1; }
+  ~ProfScope() { g_prof = prev; g_cls = -1; }
+};
+
+inline void kclass(int c) { g_cls = c; }
+
+// ============================================================================
+// launches (programmatic dependent launch on every kernel of the pass)
+// ============================================================================
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args&&... args) {
+  Profiler* pr = g_prof;
+  const bool timed = pr && g_cls >= 0 && (pr->mask & (1u << g_cls)) && pr->used < Profiler::kCapacity;
+  if (timed) {
+    if ((int)pr->ev.size() < 2 * (pr->used + 1)) {
+      cudaEvent_t a, b;
+      if (cudaEventCreate(&a) != cudaSuccess) return cudaErrorMemoryAllocation;
+      if (cudaEventCreate(&b) != cudaSuccess) return cudaErrorMemoryAllocation;
+      pr->ev.push_back(a);
+      pr->ev.push_back(b);
+      pr->cls.push_back(-1);
+    }
+    cudaEventRecord(pr->ev[2 * pr->used], st);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (timed) {
+    cudaEventRecord(pr->ev[2 * pr->used + 1], st);
+    pr->cls[pr->used] = g_cls;
+    ++pr->used;
+  }
+  return e;
+}
+
+constexpr size_t kMaxDynSmem = 227 * 1024;
+
+// One-time per-device attribute setup for kernels with large dynamic smem.
+std::mutex g_init_mu;
+std::map<int, bool> g_dev_init;
+
+template <int NT, int IN, int EPI>
+cudaError_t set_gemv_attr() {
+  return cudaFuncSetAttribute(gemv_int4_kernel<NT, IN, EPI>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDynSmem);
+}
+
+cudaError_t init_device_kernels(int dev) {
+  std::lock_guard<std::mutex> lk(g_init_mu);
+  if (g_dev_init[dev]) return cudaSuccess;
+  cudaError_t e = cudaSuccess;
+#define SET(NT, IN, EPI) \
+  if (e == cudaSuccess) e = set_gemv_attr<NT, IN, EPI>();
+  SET(1, IN_F16, EPI_STORE) SET(2, IN_F16, EPI_STORE)
+  SET(1, IN_F16, EPI_RESID) SET(2, IN_F16, EPI_RESID)
+  SET(1, IN_NORM, EPI_SWIGLU) SET(2, IN_NORM, EPI_SWIGLU)
+  SET(1, IN_NORM, EPI_ROPE_KV) SET(2, IN_NORM, EPI_ROPE_KV)
+#undef SET
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(head_argmax_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kMaxDynSmem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(head_argmax_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kMaxDynSmem);
+  if (e == cudaSuccess) g_dev_init[dev] = true;
+  return e;
+}
+
+// Largest activation-row count per GEMV launch that fits shared memory.
+int gemv_rows_per_launch(int K) {
+  if (gemv_smem_bytes(K, 2) <= kMaxDynSmem) return 16;
+  if (gemv_smem_bytes(K, 1) <= kMaxDynSmem) return 8;
+  return 0;
+}
+
+cudaError_t launch_gemv(const GemvArgs& a, int grid, int in_mode, int epi, cudaStream_t st) {
+  const int nt = a.M <= 8 ? 1 : 2;
+  const size_t smem = gemv_smem_bytes(a.K, nt);
+  const dim3 g(grid), b(kGemvThreads);
+#define CASE(NT, IN, EPI) \
+  if (nt == NT && in_mode == IN && epi == EPI) return launch(gemv_int4_kernel<NT, IN, EPI>, g, b, smem, st, a);
+  CASE(1, IN_F16, EPI_STORE) CASE(2, IN_F16, EPI_STORE)
+  CASE(1, IN_F16, EPI_RESID) CASE(2, IN_F16, EPI_RESID)
+  CASE(1, IN_NORM, EPI_SWIGLU) CASE(2, IN_NORM, EPI_SWIGLU)
+  CASE(1, IN_NORM, EPI_ROPE_KV) CASE(2, IN_NORM, EPI_ROPE_KV)
+#undef CASE
+  return cudaErrorInvalidValue;
+}
+
+// ============================================================================
+// INT4 weights on the device
+// ============================================================================
+struct Int4Dev {
+  int K = 0, N = 0, n_tiles = 0;
+  uint4* w = nullptr;
+  uint2* sz = nullptr;
+  size_t bytes() const {
+    return (size_t)n_tiles * (K / 64) * 32 * sizeof(uint4) + (size_t)n_tiles * (K / 128) * 8 * sizeof(uint2);
+  }
+  void free_all() {
+    if (w) cudaFree(w);
+    if (sz) cudaFree(sz);
+    w = nullptr;
+    sz = nullptr;
+  }
+};
+
+// Copy one linear in the storage format to the device and re-lay it out.
+// N is padded to whole pairs of 16-row tiles with zero weights.
+tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaStream_t st) {
+  if (!h.qweight || !h.scales || !h.qzeros) return fail(TL_ERR_INVALID_ARG, "null INT4 array");
+  const int G = K / 128, zw = (G + 7) / 8;
+  out->K = K;
+  out->N = N;
+  out->n_tiles = ((N + 31) / 32) * 2;
+  const size_t qb = (size_t)N * (K / 8) * 4, sb = (size_t)N * G * 2, zb = (size_t)N * zw * 4;
+  void *dq = nullptr, *ds = nullptr, *dz = nullptr;
+  tl_status rc = TL_OK;
+  cudaError_t e = cudaMalloc(&dq, qb);
+  if (e == cudaSuccess) e = cudaMalloc(&ds, sb);
+  if (e == cudaSuccess) e = cudaMalloc(&dz, zb);
+  if (e == cudaSuccess) e = cudaMalloc(&out->w, (size_t)out->n_tiles * (K / 64) * 32 * sizeof(uint4));
+  if (e == cudaSuccess) e = cudaMalloc(&out->sz, (size_t)out->n_tiles * G * 8 * sizeof(uint2));
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dq, h.qweight, qb, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(ds, h.scales, sb, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dz, h.qzeros, zb, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) {
+    const size_t tw = (size_t)out->n_tiles * (K / 64) * 32;
+    repack_int4_weights_kernel<<<(unsigned)((tw + 255) / 256), 256, 0, st>>>(
+        (const uint32_t*)dq, K, N, out->n_tiles, out->w);
+    const size_t ts = (size_t)out->n_tiles * G * 8;
+    repack_int4_scales_kernel<<<(unsigned)((ts + 255) / 256), 256, 0, st>>>(
+        (const uint16_t*)ds, (const uint32_t*)dz, K, N, out->n_tiles, out->sz);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    rc = cuda_fail(e, "upload INT4 linear");
+    out->free_all();
+  }
+  if (dq) cudaFree(dq);
+  if (ds) cudaFree(ds);
+  if (dz) cudaFree(dz);
+  return rc;
+}
+
+tl_status upload_f16(const uint16_t* h, size_t n, __half** out, cudaStream_t st) {
+  if (!h) return fail(TL_ERR_INVALID_ARG, "null fp16 array");
+  TL_CUDA(cudaMalloc(out, n * 2));
+  TL_CUDA(cudaMemcpyAsync(*out, h, n * 2, cudaMemcpyHostToDevice, st));
+  return TL_OK;
+}
+
+struct BlockDev {
+  __half* attn_norm = nullptr;
+  __half* ffn_norm = nullptr;
+  Int4Dev qkv, o, gate_up, down;
+  void free_all() {
+    if (attn_norm) cudaFree(attn_norm);
+    if (ffn_norm) cudaFree(ffn_norm);
+    attn_norm = ffn_norm = nullptr;
+    qkv.free_all();
+    o.free_all();
+    gate_up.free_all();
+    down.free_all();
+  }
+  size_t bytes(int d) const { return qkv.bytes() + o.bytes() + gate_up.bytes() + down.bytes() + 4 * (size_t)d; }
+};
+
+// Per-step row description, passed by value to a setup kernel (so no host
+// buffer has to outlive the call).
+struct StepDesc {
+  int n;
+  int lane[kMaxLanes];
+  int pos[kMaxLanes];
+  int tok_index[kMaxLanes];
+  int out_row[kMaxLanes];
+};
+
+__global__ void setup_step_kernel(StepDesc s, RowCtx* rows, int* tok_index, int* out_row) {
+  pdl_trigger();
+  pdl_wait();
+  const int i = threadIdx.x;
+  if (i < s.n) {
+    rows[i].lane = s.lane[i];
+    rows[i].pos = s.pos[i];
+    tok_index[i] = s.tok_index[i];
+    out_row[i] = s.out_row[i];
+  }
+}
+
+__global__ void fill_rows_kernel(RowCtx* rows, int n, int lane, int pos0) {
+  pdl_trigger();
+  pdl_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    rows[i].lane = lane;
+    rows[i].pos = pos0 + i;
+  }
+}
+
+
+template <int HD, int REP>
+cudaError_t launch_decode_attn_t(const DecodeAttnArgs& a, int rows, cudaStream_t st) {
+  return launch(decode_attn_kernel<HD, REP>, dim3(kDecodeMaxSplits, a.Hkv, rows), dim3(kDecodeThreads), 0, st, a);
+}
+
+cudaError_t launch_decode_attn(const DecodeAttnArgs& a, int rows, int hd, int rep, cudaStream_t st) {
+#define C(HD, REP) \
+  if (hd == HD && rep == REP) return launch_decode_attn_t<HD, REP>(a, rows, st);
+  C(64, 1) C(64, 2) C(64, 4) C(64, 8) C(128, 1) C(128, 2) C(128, 4) C(128, 8)
+#undef C
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, int B, int hd, int rep, cudaStream_t st) {
+#define C(HD, REP)                                                                                \
+  if (hd == HD && rep == REP)                                                                     \
+    return launch(prefill_attn_simple_kernel<HD, REP>, dim3(a.T, a.Hkv, B), dim3(REP * 32), 0, st, a);
+  C(64, 1) C(64, 2) C(64, 4) C(64, 8) C(128, 1) C(128, 2) C(128, 4) C(128, 8)
+#undef C
+  return cudaErrorInvalidValue;
+}
+
+bool rep_ok(int rep) { return rep == 1 || rep == 2 || rep == 4 || rep == 8; }
+
+}  // namespace
+
+// ============================================================================
+// model
+// ============================================================================
+struct tl_model {
+  tl_config cfg{};
+  int device = 0;
+  int n_layers_max = 0;
+  std::vector<BlockDev> pre;
+  BlockDev loop;
+  __half* embed = nullptr;
+  __half* out_norm = nullptr;
+  uint4* head_w = nullptr;
+  // KV cache: [max_lanes + 1][n_layers_max][2][Hkv][max_ctx][hd] fp16
+  __half* kv = nullptr;
+  long long plane = 0, layer_stride = 0, lane_stride = 0;
+  // workspaces
+  float* x = nullptr;
+  __half* q = nullptr;
+  __half* o = nullptr;
+  __half* h = nullptr;
+  RowCtx* rows = nullptr;
+  int* tok_index = nullptr;
+  int* out_row = nullptr;
+  float* attn_part = nullptr;
+  unsigned* tickets = nullptr;  // attention [16][Hkv] then head [1]
+  float* head_val = nullptr;
+  int* head_idx = nullptr;
+  int* err_flag = nullptr;
+  int head_grid = 0;
+  cudaStream_t setup_stream = nullptr;
+  std::vector<int> lane_len, lane_loops;
+  size_t weight_bytes = 0, kv_bytes = 0, ws_bytes = 0;
+  Profiler prof;
+
+  unsigned* attn_tickets() const { return tickets; }
+  unsigned* head_ticket() const { return tickets + kMaxLanes * cfg.n_kv_heads; }
+  __half* k_plane(int layer) const { return kv + layer * layer_stride; }
+  __half* v_plane(int layer) const { return kv + layer * layer_stride + plane; }
+  const BlockDev& block(int layer) const { return layer < cfg.n_pre ? pre[layer] : loop; }
+
+  void free_all() {
+    for (auto& b : pre) b.free_all();
+    loop.free_all();
+    void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row,
+                    attn_part, tickets, head_val, head_idx, err_flag};
+    for (void* p : ptrs)
+      if (p) cudaFree(p);
+    if (setup_stream) cudaStreamDestroy(setup_stream);
+    prof.destroy();
+  }
+};
+
+namespace {
+
+tl_status validate_config(const tl_config* c) {
+  if (!c) return fail(TL_ERR_INVALID_ARG, "null config");
+  if (c->d_model < 128 || c->d_model % 128 || c->d_model > 8192)
+    return fail(TL_ERR_UNSUPPORTED, "d_model must be a multiple of 128 in [128, 8192]");
+  if (c->head_dim != 64 && c->head_dim != 128) return fail(TL_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (c->n_q_heads < 1 || c->n_kv_heads < 1 || c->n_q_heads % c->n_kv_heads)
+    return fail(TL_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+  if (!rep_ok(c->n_q_heads / c->n_kv_heads)) return fail(TL_ERR_UNSUPPORTED, "n_q_heads/n_kv_heads must be 1, 2, 4 or 8");
+  if ((c->n_q_heads * c->head_dim) % 128 || c->n_q_heads * c->head_dim > 8192)
+    return fail(TL_ERR_UNSUPPORTED, "n_q_heads*head_dim must be a multiple of 128, <= 8192");
+  if (c->ffn_dim < 128 || c->ffn_dim % 128 || c->ffn_dim > 12288)
+    return fail(TL_ERR_UNSUPPORTED, "ffn_dim must be a multiple of 128 in [128, 12288]");
+  if (c->vocab < 16 || c->vocab % 16) return fail(TL_ERR_UNSUPPORTED, "vocab must be a positive multiple of 16");
+  if (c->n_pre < 0 || c->n_pre > 64) return fail(TL_ERR_INVALID_ARG, "n_pre out of range");
+  if (c->max_loops < 1 || c->max_loops > 256) return fail(TL_ERR_INVALID_ARG, "max_loops out of range");
+  if (c->max_ctx < 1 || c->max_ctx > 8192) return fail(TL_ERR_INVALID_ARG, "max_ctx must be in [1, 8192]");
+  if (c->max_lanes < 1 || c->max_lanes > kMaxLanes) return fail(TL_ERR_INVALID_ARG, "max_lanes must be in [1, 16]");
+  if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return fail(TL_ERR_INVALID_ARG, "bad eps or theta");
+  return TL_OK;
+}
+
+tl_status upload_block(const tl_config& c, const tl_block& hb, BlockDev* b, cudaStream_t st) {
+  const int d = c.d_model, hd = c.head_dim;
+  const int qkv_rows = (c.n_q_heads + 2 * c.n_kv_heads) * hd;
+  tl_status rc;
+  if ((rc = upload_f16(hb.attn_norm, d, &b->attn_norm, st)) != TL_OK) return rc;
+  if ((rc = upload_f16(hb.ffn_norm, d, &b->ffn_norm, st)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.qkv, d, qkv_rows, &b->qkv, st)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.o, c.n_q_heads * hd, d, &b->o, st)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.gate_up, d, 2 * c.ffn_dim, &b->gate_up, st)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.down, c.ffn_dim, d, &b->down, st)) != TL_OK) return rc;
+  return TL_OK;
+}
+
+// ---- one effective layer for M rows (M <= 16) -------------------------------
+// x: fp32 [M][d] residual rows, rows: their lanes/positions, q/o/h buffers.
+tl_status layer_rows(tl_model* m, int layer, int M, float* x, const RowCtx* rows, __half* q,
+                     __half* o, __half* h, bool decode_attn, cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  const BlockDev& b = m->block(layer);
+  const int d = c.d_model, hd = c.head_dim, F = c.ffn_dim;
+  const int qdim = c.n_q_heads * hd;
+  GemvArgs a{};
+  a.M = M;
+  a.eps = c.rms_eps;
+  a.theta = c.rope_theta;
+  a.rows = rows;
+  a.hd = hd;
+
+  // QKV with fused RMSNorm, RoPE and KV write
+  a.w = b.qkv.w; a.sz = b.qkv.sz; a.K = d; a.n_rows = b.qkv.N;
+  a.x = x; a.ldx = d; a.gain = b.attn_norm;
+  a.pair_mode = PAIR_ROPE; a.pair_off = hd / 32;
+  a.q_out = q; a.ldq = qdim; a.n_q_rows = qdim; a.n_kv_rows = c.n_kv_heads * hd;
+  a.k_plane = m->k_plane(layer); a.v_plane = m->v_plane(layer);
+  a.lane_stride = m->lane_stride; a.ctx = c.max_ctx;
+  kclass(TL_KERNEL_QKV);
+  TL_CUDA(launch_gemv(a, (c.n_q_heads + 2 * c.n_kv_heads) * hd / 32, IN_NORM, EPI_ROPE_KV, st));
+  if (decode_attn) {
+    DecodeAttnArgs da{};
+    da.q = q; da.ldq = qdim;
+    da.k = m->k_plane(layer); da.v = m->v_plane(layer);
+    da.lane_stride = m->lane_stride; da.ctx = c.max_ctx;
+    da.rows = rows; da.Hkv = c.n_kv_heads;
+    da.out = o; da.ldo = qdim;
+    da.part = m->attn_part; da.ticket = m->attn_tickets();
+    kclass(TL_KERNEL_ATTN_DECODE);
+    TL_CUDA(launch_decode_attn(da, M, hd, c.n_q_heads / c.n_kv_heads, st));
+  }
+  return TL_OK;
+}
+
+tl_status layer_rows_post(tl_model* m, int layer, int M, float* x, __half* o, __half* h,
+                          cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  const BlockDev& b = m->block(layer);
+  const int d = c.d_model, F = c.ffn_dim;
+  const int qdim = c.n_q_heads * c.head_dim;
+  GemvArgs a{};
+  a.M = M;
+  a.eps = c.rms_eps;
+  // O projection + residual
+  a.w = b.o.w; a.sz = b.o.sz; a.K = qdim; a.n_rows = d;
+  a.xh = o; a.ldx = qdim;
+  a.pair_mode = PAIR_NEIGHBOUR;
+  a.resid = x; a.ldr = d;
+  kclass(TL_KERNEL_O_PROJ);
+  TL_CUDA(launch_gemv(a, b.o.n_tiles / 2, IN_F16, EPI_RESID, st));
+  // gate_up with fused RMSNorm and SwiGLU
+  a.w = b.gate_up.w; a.sz = b.gate_up.sz; a.K = d; a.n_rows = 2 * F;
+  a.x = x; a.ldx = d; a.gain = b.ffn_norm;
+  a.pair_mode = PAIR_OFFSET; a.pair_off = F / 16;
+  a.y = h; a.ldy = F;
+  kclass(TL_KERNEL_GATE_UP);
+  TL_CUDA(launch_gemv(a, F / 16, IN_NORM, EPI_SWIGLU, st));
+  // down + residual
+  a.w = b.down.w; a.sz = b.down.sz; a.K = F; a.n_rows = d;
+  a.xh = h; a.ldx = F;
+  a.pair_mode = PAIR_NEIGHBOUR;
+  a.resid = x; a.ldr = d;
+  kclass(TL_KERNEL_DOWN);
+  TL_CUDA(launch_gemv(a, b.down.n_tiles / 2, IN_F16, EPI_RESID, st));
+  return TL_OK;
+}
+
+tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, float* logits,
+                      int32_t* argmax, cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  HeadArgs ha{};
+  ha.w = m->head_w; ha.V = c.vocab; ha.d = c.d_model;
+  ha.x = x; ha.gain = m->out_norm; ha.eps = c.rms_eps; ha.M = M;
+  ha.out_row = out_row; ha.logits = logits; ha.argmax = argmax;
+  ha.part_val = m->head_val; ha.part_idx = m->head_idx; ha.ticket = m->head_ticket();
+  const int nt = M <= 8 ? 1 : 2;
+  const size_t smem = head_smem_bytes(c.d_model, nt);
+  kclass(TL_KERNEL_HEAD);
+  if (nt == 1) TL_CUDA(launch(head_argmax_kernel<1>, dim3(m->head_grid), dim3(kHeadThreads), smem, st, ha));
+  else TL_CUDA(launch(head_argmax_kernel<2>, dim3(m->head_grid), dim3(kHeadThreads), smem, st, ha));
+  return TL_OK;
+}
+
+// Whole-prompt forward on one lane (positions 0..T-1).
+tl_status forward_prompt(tl_model* m, int lane, const int32_t* d_tokens, int T, int loops,
+                         float* d_logits, int32_t* d_argmax, cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  const int d = c.d_model, qdim = c.n_q_heads * c.head_dim, F = c.ffn_dim;
+  const int n_layers = c.n_pre + loops;
+  kclass(TL_KERNEL_SETUP);
+  TL_CUDA(launch(fill_rows_kernel, dim3((T + 255) / 256), dim3(256), 0, st, m->rows, T, lane, 0));
+  kclass(TL_KERNEL_EMBED);
+  TL_CUDA(launch(embed_kernel, dim3(T), dim3(256), 0, st, (const __half*)m->embed, d, c.vocab,
+                 d_tokens, (const int*)nullptr, m->x, m->err_flag));
+  const int chunk = kMaxLanes;
+  for (int layer = 0; layer < n_layers; ++layer) {
+    for (int r0 = 0; r0 < T; r0 += chunk) {
+      const int M = std::min(chunk, T - r0);
+      tl_status rc = layer_rows(m, layer, M, m->x + (size_t)r0 * d, m->rows + r0,
+                                m->q + (size_t)r0 * qdim, m->o + (size_t)r0 * qdim,
+                                m->h + (size_t)r0 * F, false, st);
+      if (rc != TL_OK) return rc;
+    }
+    PrefillAttnArgs pa{};
+    pa.q = m->q; pa.q_bstride = 0; pa.ldq = qdim;
+    pa.k = m->k_plane(layer) + lane * m->lane_stride;
+    pa.v = m->v_plane(layer) + lane * m->lane_stride;
+    pa.kv_bstride = 0; pa.ctx = c.max_ctx;
+    pa.T = T; pa.pos0 = 0; pa.Hkv = c.n_kv_heads;
+    pa.out = m->o; pa.o_bstride = 0; pa.ldo = qdim;
+    kclass(TL_KERNEL_ATTN_PREFILL);
+    TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, st));
+    for (int r0 = 0; r0 < T; r0 += chunk) {
+      const int M = std::min(chunk, T - r0);
+      tl_status rc = layer_rows_post(m, layer, M, m->x + (size_t)r0 * d, m->o + (size_t)r0 * qdim,
+                                     m->h + (size_t)r0 * F, st);
+      if (rc != TL_OK) return rc;
+    }
+  }
+  if (d_logits || d_argmax)
+    return launch_head(m, m->x + (size_t)(T - 1) * d, 1, nullptr, d_logits, d_argmax, st);
+  return TL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device, tl_model** out) {
+  if (!out) return fail(TL_ERR_INVALID_ARG, "null out");
+  *out = nullptr;
+  tl_status rc = validate_config(cfg);
+  if (rc != TL_OK) return rc;
+  if (!w || !w->embed || !w->out_norm || !w->head || !w->loop || (cfg->n_pre > 0 && !w->pre))
+    return fail(TL_ERR_INVALID_ARG, "null weight pointer");
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)
+    return fail(TL_ERR_INVALID_ARG, "device %d not available", device);
+  DeviceGuard guard(device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device %d", device);
+  TL_CUDA(init_device_kernels(device));
+
+  tl_model* m = new tl_model();
+  m->cfg = *cfg;
+  m->device = device;
+  m->n_layers_max = cfg->n_pre + cfg->max_loops;
+  const tl_config& c = m->cfg;
+  const int d = c.d_model, hd = c.head_dim, qdim = c.n_q_heads * hd;
+  auto bail = [&](tl_status s) {
+    m->free_all();
+    delete m;
+    return s;
+  };
+  if (cudaStreamCreateWithFlags(&m->setup_stream, cudaStreamNonBlocking) != cudaSuccess)
+    return bail(fail(TL_ERR_CUDA, "stream create failed"));
+  cudaStream_t st = m->setup_stream;
+
+  m->pre.resize(c.n_pre);
+  for (int i = 0; i < c.n_pre; ++i)
+    if ((rc = upload_block(c, w->pre[i], &m->pre[i], st)) != TL_OK) return bail(rc);
+  if ((rc = upload_block(c, *w->loop, &m->loop, st)) != TL_OK) return bail(rc);
+  if ((rc = upload_f16(w->embed, (size_t)c.vocab * d, &m->embed, st)) != TL_OK) return bail(rc);
+  if ((rc = upload_f16(w->out_norm, d, &m->out_norm, st)) != TL_OK) return bail(rc);
+  {
+    __half* raw = nullptr;
+    if ((rc = upload_f16(w->head, (size_t)c.vocab * d, &raw, st)) != TL_OK) return bail(rc);
+    const size_t n = (size_t)(c.vocab / 16) * (d / 16) * 32;
+    if (cudaMalloc(&m->head_w, n * sizeof(uint4)) != cudaSuccess) {
+      cudaFree(raw);
+      return bail(fail(TL_ERR_OOM, "head allocation"));
+    }
+    repack_head_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>((const uint32_t*)raw, c.vocab, d, m->head_w);
+    cudaError_t e = cudaStreamSynchronize(st);
+    cudaFree(raw);
+    if (e != cudaSuccess) return bail(cuda_fail(e, "head repack"));
+  }
+  m->weight_bytes = m->loop.bytes(d) + (size_t)c.vocab * d * 4 + 2 * (size_t)d;
+  for (auto& b : m->pre) m->weight_bytes += b.bytes(d);
+
+  // KV cache (one extra private lane for tl_score_last)
+  m->plane = (long long)c.n_kv_heads * c.max_ctx * hd;
+  m->layer_stride = 2 * m->plane;
+  m->lane_stride = (long long)m->n_layers_max * m->layer_stride;
+  m->kv_bytes = (size_t)(c.max_lanes + 1) * m->lane_stride * 2;
+  if (cudaMalloc(&m->kv, m->kv_bytes) != cudaSuccess) return bail(fail(TL_ERR_OOM, "KV cache (%zu bytes)", m->kv_bytes));
+
+  // workspaces
+  const int rows = std::max(c.max_ctx, kMaxLanes);
+  const int rep = c.n_q_heads / c.n_kv_heads;
+  m->head_grid = (c.vocab / 16 + 7) / 8;
+  size_t ws = 0;
+  auto alloc = [&](void** p, size_t bytes) -> bool {
+    ws += bytes;
+    if (cudaMalloc(p, bytes) != cudaSuccess) return false;
+    return cudaMemsetAsync(*p, 0, bytes, st) == cudaSuccess;
+  };
+  bool ok = alloc((void**)&m->x, (size_t)rows * d * 4) && alloc((void**)&m->q, (size_t)rows * qdim * 2) &&
+            alloc((void**)&m->o, (size_t)rows * qdim * 2) && alloc((void**)&m->h, (size_t)rows * c.ffn_dim * 2) &&
+            alloc((void**)&m->rows, (size_t)rows * sizeof(RowCtx)) &&
+            alloc((void**)&m->tok_index, kMaxLanes * 4) && alloc((void**)&m->out_row, kMaxLanes * 4) &&
+            alloc((void**)&m->attn_part, (size_t)kMaxLanes * c.n_kv_heads * kDecodeMaxSplits * rep * (hd + 2) * 4) &&
+            alloc((void**)&m->tickets, (size_t)(kMaxLanes * c.n_kv_heads + 1) * 4) &&
+            alloc((void**)&m->head_val, (size_t)m->head_grid * 16 * 4) &&
+            alloc((void**)&m->head_idx, (size_t)m->head_grid * 16 * 4) && alloc((void**)&m->err_flag, 4);
+  if (!ok) return bail(fail(TL_ERR_OOM, "workspace allocation"));
+  m->ws_bytes = ws;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return bail(fail(TL_ERR_CUDA, "setup sync"));
+  m->lane_len.assign(c.max_lanes + 1, 0);
+  m->lane_loops.assign(c.max_lanes + 1, 0);
+  *out = m;
+  return TL_OK;
+}
+
+void tl_model_destroy(tl_model* m) {
+  if (!m) return;
+  DeviceGuard guard(m->device);
+  cudaDeviceSynchronize();
+  m->free_all();
+  delete m;
+}
+
+tl_status tl_prefill(tl_model* m, int lane, const int32_t* d_tokens, int n_tokens, int loops,
+                     float* d_last_logits, int32_t* d_last_argmax, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (lane < 0 || lane >= c.max_lanes) return fail(TL_ERR_INVALID_ARG, "lane %d out of range", lane);
+  if (!d_tokens) return fail(TL_ERR_INVALID_ARG, "null tokens");
+  if (n_tokens < 1 || n_tokens > c.max_ctx) return fail(TL_ERR_CONTEXT_FULL, "n_tokens %d not in [1, max_ctx]", n_tokens);
+  if (loops < 1 || loops > c.max_loops) return fail(TL_ERR_INVALID_ARG, "loops %d not in [1, max_loops]", loops);
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  ProfScope prof_scope(&m->prof);
+  tl_status rc = forward_prompt(m, lane, d_tokens, n_tokens, loops, d_last_logits, d_last_argmax,
+                                (cudaStream_t)stream);
+  if (rc != TL_OK) {
+    m->lane_len[lane] = 0;
+    return rc;
+  }
+  m->lane_len[lane] = n_tokens;
+  m->lane_loops[lane] = loops;
+  return TL_OK;
+}
+
+tl_status tl_score_last(tl_model* m, const int32_t* d_tokens, int n_tokens, int loops, float* d_logits,
+                        int32_t* d_argmax, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (!d_tokens || !d_logits) return fail(TL_ERR_INVALID_ARG, "null tokens or logits");
+  if (n_tokens < 1 || n_tokens > c.max_ctx) return fail(TL_ERR_CONTEXT_FULL, "n_tokens %d not in [1, max_ctx]", n_tokens);
+  if (loops < 1 || loops > c.max_loops) return fail(TL_ERR_INVALID_ARG, "loops %d not in [1, max_loops]", loops);
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  ProfScope prof_scope(&m->prof);
+  return forward_prompt(m, c.max_lanes, d_tokens, n_tokens, loops, d_logits, d_argmax, (cudaStream_t)stream);
+}
+
+tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, const int32_t* d_tokens,
+                         const int32_t* h_loops, float* d_logits, int32_t* d_argmax, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (n_lanes < 1 || n_lanes > c.max_lanes) return fail(TL_ERR_INVALID_ARG, "n_lanes %d not in [1, max_lanes]", n_lanes);
+  if (!h_lane_ids || !d_tokens || !h_loops) return fail(TL_ERR_INVALID_ARG, "null argument");
+  std::vector<int> order(n_lanes);
+  for (int i = 0; i < n_lanes; ++i) {
+    const int lane = h_lane_ids[i];
+    if (lane < 0 || lane >= c.max_lanes) return fail(TL_ERR_INVALID_ARG, "lane %d out of range", lane);
+    for (int j = 0; j < i; ++j)
+      if (h_lane_ids[j] == lane) return fail(TL_ERR_INVALID_ARG, "lane %d listed twice", lane);
+    if (m->lane_len[lane] == 0) return fail(TL_ERR_NOT_PREFILLED, "lane %d holds no prompt", lane);
+    if (h_loops[i] != m->lane_loops[lane])
+      return fail(TL_ERR_LOOPS_MISMATCH, "lane %d was prefilled with loops=%d, step asks %d", lane,
+                  m->lane_loops[lane], h_loops[i]);
+    if (m->lane_len[lane] >= c.max_ctx) return fail(TL_ERR_CONTEXT_FULL, "lane %d is full", lane);
+    order[i] = i;
+  }
+  // Rows sorted by loop count (descending): the rows still running at layer l
+  // are then a prefix.
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return h_loops[a] > h_loops[b]; });
+  StepDesc sd{};
+  sd.n = n_lanes;
+  for (int s = 0; s < n_lanes; ++s) {
+    const int i = order[s];
+    sd.lane[s] = h_lane_ids[i];
+    sd.pos[s] = m->lane_len[h_lane_ids[i]];
+    sd.tok_index[s] = i;
+    sd.out_row[s] = i;
+  }
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int d = c.d_model, qdim = c.n_q_heads * c.head_dim;
+  ProfScope prof_scope(&m->prof);
+  kclass(TL_KERNEL_SETUP);
+  TL_CUDA(launch(setup_step_kernel, dim3(1), dim3(32), 0, st, sd, m->rows, m->tok_index, m->out_row));
+  kclass(TL_KERNEL_EMBED);
+  TL_CUDA(launch(embed_kernel, dim3(n_lanes), dim3(256), 0, st, (const __half*)m->embed, d, c.vocab, d_tokens,
+                 (const int*)m->tok_index, m->x, m->err_flag));
+  const int max_layers = c.n_pre + h_loops[order[0]];
+  for (int layer = 0; layer < max_layers; ++layer) {
+    int M = 0;
+    while (M < n_lanes && c.n_pre + h_loops[order[M]] > layer) ++M;
+    tl_status rc = layer_rows(m, layer, M, m->x, m->rows, m->q, m->o, m->h, true, st);
+    if (rc == TL_OK) rc = layer_rows_post(m, layer, M, m->x, m->o, m->h, st);
+    if (rc != TL_OK) return rc;
+  }
+  if (d_logits || d_argmax) {
+    tl_status rc = launch_head(m, m->x, n_lanes, m->out_row, d_logits, d_argmax, st);
+    if (rc != TL_OK) return rc;
+  }
+  for (int i = 0; i < n_lanes; ++i) m->lane_len[h_lane_ids[i]] += 1;
+  (void)qdim;
+  return TL_OK;
+}
+
+tl_status tl_model_profile_start(tl_model* m, unsigned class_mask) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  m->prof.mask = class_mask;
+  m->prof.used = 0;
+  return TL_OK;
+}
+
+tl_status tl_model_profile_stop(tl_model* m, int* h_launches, float* h_total_ms) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  DeviceGuard guard(m->device);
+  for (int c = 0; c < TL_KERNEL_CLASSES; ++c) {
+    if (h_launches) h_launches[c] = 0;
+    if (h_total_ms) h_total_ms[c] = 0.f;
+  }
+  for (int i = 0; i < m->prof.used; ++i) {
+    TL_CUDA(cudaEventSynchronize(m->prof.ev[2 * i + 1]));
+    float ms = 0.f;
+    TL_CUDA(cudaEventElapsedTime(&ms, m->prof.ev[2 * i], m->prof.ev[2 * i + 1]));
+    const int c = m->prof.cls[i];
+    if (c < 0 || c >= TL_KERNEL_CLASSES) continue;
+    if (h_launches) h_launches[c] += 1;
+    if (h_total_ms) h_total_ms[c] += ms;
+  }
+  m->prof.mask = 0;
+  m->prof.used = 0;
+  return TL_OK;
+}
+
+unsigned long long tl_kernel_launch_count(void) { return g_launches.load(); }
+
+tl_status tl_lane_length(const tl_model* m, int lane, int* h_length) {
+  if (!m || !h_length) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (lane < 0 || lane >= m->cfg.max_lanes) return fail(TL_ERR_INVALID_ARG, "lane %d out of range", lane);
+  *h_length = m->lane_len[lane];
+  return TL_OK;
+}
+
+tl_status tl_model_info(const tl_model* m, size_t* weight_bytes, size_t* kv_bytes, size_t* workspace_bytes) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  if (weight_bytes) *weight_bytes = m->weight_bytes;
+  if (kv_bytes) *kv_bytes = m->kv_bytes;
+  if (workspace_bytes) *workspace_bytes = m->ws_bytes;
+  return TL_OK;
+}
+
+tl_status tl_check_device_error(tl_model* m, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  DeviceGuard guard(m->device);
+  TL_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  int flag = 0;
+  TL_CUDA(cudaMemcpy(&flag, m->err_flag, 4, cudaMemcpyDeviceToHost));
+  if (flag) {
+    TL_CUDA(cudaMemset(m->err_flag, 0, 4));
+    return fail(TL_ERR_DEVICE_FLAG, "a token id outside [0, vocab) was replaced by 0");
+  }
+  return TL_OK;
+}
+
+// ============================================================================
+// op API
+// ============================================================================
+}  // extern "C"
+
+struct tl_linear {
+  int device = 0;
+  Int4Dev w;
+};
+
+namespace {
+// Library-owned per-device workspace of the op entry points.
+struct OpWorkspace {
+  void* buf = nullptr;
+  size_t bytes = 0;
+};
+std::mutex g_ws_mu;
+std::map<int, OpWorkspace> g_ws;
+
+// Returns a zero-initialised-at-allocation device buffer of at least `bytes`.
+// Growing it synchronises the device.
+tl_status op_workspace(int dev, size_t bytes, void** out) {
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  OpWorkspace& w = g_ws[dev];
+  if (w.bytes < bytes) {
+    if (w.buf) {
+      cudaDeviceSynchronize();
+      cudaFree(w.buf);
+      w.buf = nullptr;
+      w.bytes = 0;
+    }
+    const size_t nb = std::max(bytes, (size_t)1 << 20);
+    TL_CUDA(cudaMalloc(&w.buf, nb));
+    TL_CUDA(cudaMemset(w.buf, 0, nb));
+    w.bytes = nb;
+  }
+  *out = w.buf;
+  return TL_OK;
+}
+}  // namespace
+
+extern "C" {
+
+tl_status tl_linear_create(const tl_int4_linear* w, int K, int N, int device, tl_linear** out) {
+  if (!out || !w) return fail(TL_ERR_INVALID_ARG, "null argument");
+  *out = nullptr;
+  if (K < 128 || K % 128 || K > 12288) return fail(TL_ERR_UNSUPPORTED, "K must be a multiple of 128 in [128, 12288]");
+  if (N < 1 || N > 65536) return fail(TL_ERR_INVALID_ARG, "N must be in [1, 65536]");
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev)
+    return fail(TL_ERR_INVALID_ARG, "device %d not available", device);
+  DeviceGuard guard(device);
+  TL_CUDA(init_device_kernels(device));
+  tl_linear* l = new tl_linear();
+  l->device = device;
+  cudaStream_t st;
+  TL_CUDA(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
+  tl_status rc = upload_int4(*w, K, N, &l->w, st);
+  cudaStreamDestroy(st);
+  if (rc != TL_OK) {
+    delete l;
+    return rc;
+  }
+  *out = l;
+  return TL_OK;
+}
+
+void tl_linear_destroy(tl_linear* l) {
+  if (!l) return;
+  DeviceGuard guard(l->device);
+  cudaDeviceSynchronize();
+  l->w.free_all();
+  delete l;
+}
+
+tl_status tl_linear_forward(tl_linear* l, const uint16_t* d_x, int M, uint16_t* d_y, int path, void* stream) {
+  if (!l || !d_x || !d_y) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (M < 1) return fail(TL_ERR_INVALID_ARG, "M must be >= 1");
+  if (path == TL_PATH_AUTO) path = TL_PATH_GEMV;
+  if (path == TL_PATH_TC) return fail(TL_ERR_UNSUPPORTED, "tensor-core path not built");
+  if (path != TL_PATH_GEMV) return fail(TL_ERR_INVALID_ARG, "unknown path %d", path);
+  DeviceGuard guard(l->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  const int K = l->w.K, N = l->w.N;
+  const int rpl = gemv_rows_per_launch(K);
+  if (!rpl) return fail(TL_ERR_UNSUPPORTED, "K too large for the GEMV");
+  GemvArgs a{};
+  a.w = l->w.w; a.sz = l->w.sz; a.K = K; a.n_rows = N;
+  a.ldx = K; a.pair_mode = PAIR_NEIGHBOUR; a.ldy = N;
+  for (int r0 = 0; r0 < M; r0 += rpl) {
+    a.M = std::min(rpl, M - r0);
+    a.xh = reinterpret_cast<const __half*>(d_x) + (size_t)r0 * K;
+    a.y = reinterpret_cast<__half*>(d_y) + (size_t)r0 * N;
+    TL_CUDA(launch_gemv(a, l->w.n_tiles / 2, IN_F16, EPI_STORE, (cudaStream_t)stream));
+  }
+  return TL_OK;
+}
+
+tl_status tl_op_rmsnorm(const float* d_x, const uint16_t* d_g, int rows, int d, float eps, uint16_t* d_y,
+                        void* stream) {
+  if (!d_x || !d_g || !d_y) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (rows < 1 || d < 4 || d % 4) return fail(TL_ERR_INVALID_ARG, "rows >= 1 and d a multiple of 4 required");
+  TL_CUDA(launch(rmsnorm_kernel, dim3((rows + 7) / 8), dim3(256), 0, (cudaStream_t)stream, d_x,
+                 reinterpret_cast<const __half*>(d_g), rows, d, eps, reinterpret_cast<__half*>(d_y)));
+  return TL_OK;
+}
+
+tl_status tl_op_rope(uint16_t* d_x, int n_tokens, int n_heads, int head_dim, long long token_stride,
+                     long long head_stride, const int32_t* d_positions, float theta, void* stream) {
+  if (!d_x || !d_positions) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (n_tokens < 1 || n_heads < 1 || head_dim < 2 || head_dim % 2 || head_dim > 256 || !(theta > 0.f))
+    return fail(TL_ERR_INVALID_ARG, "bad RoPE shape");
+  const long long n = (long long)n_tokens * n_heads * (head_dim / 2);
+  TL_CUDA(launch(rope_inplace_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, (cudaStream_t)stream,
+                 reinterpret_cast<__half*>(d_x), n_tokens, n_heads, head_dim, token_stride, head_stride,
+                 d_positions, theta));
+  return TL_OK;
+}
+
+tl_status tl_op_gqa_decode(const uint16_t* d_q, const uint16_t* d_k, const uint16_t* d_v, long long batch_stride,
+                           int ctx_stride, const int32_t* h_n_keys, int B, int n_q_heads, int n_kv_heads,
+                           int head_dim, uint16_t* d_out, void* stream) {
+  if (!d_q || !d_k || !d_v || !h_n_keys || !d_out) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (B < 1 || n_kv_heads < 1 || n_q_heads % n_kv_heads || !rep_ok(n_q_heads / n_kv_heads) ||
+      (head_dim != 64 && head_dim != 128))
+    return fail(TL_ERR_UNSUPPORTED, "unsupported attention shape");
+  if (ctx_stride < 1 || ctx_stride > 8192) return fail(TL_ERR_INVALID_ARG, "ctx_stride must be in [1, 8192]");
+  std::vector<RowCtx> rows(B);
+  for (int b = 0; b < B; ++b) {
+    if (h_n_keys[b] < 1 || h_n_keys[b] > ctx_stride) return fail(TL_ERR_INVALID_ARG, "n_keys[%d] out of range", b);
+    rows[b].lane = b;
+    rows[b].pos = h_n_keys[b] - 1;
+  }
+  int dev = 0;
+  TL_CUDA(cudaGetDevice(&dev));
+  const int rep = n_q_heads / n_kv_heads;
+  const size_t rows_b = (size_t)B * sizeof(RowCtx);
+  const size_t part_b = (size_t)B * n_kv_heads * kDecodeMaxSplits * rep * (head_dim + 2) * 4;
+  const size_t tick_b = (size_t)B * n_kv_heads * 4;
+  void* ws = nullptr;
+  tl_status rc = op_workspace(dev, rows_b + part_b + tick_b + 256, &ws);
+  if (rc != TL_OK) return rc;
+  char* base = (char*)ws;
+  RowCtx* d_rows = (RowCtx*)base;
+  float* part = (float*)(base + ((rows_b + 255) / 256) * 256);
+  unsigned* tick = (unsigned*)((char*)part + part_b);
+  cudaStream_t st = (cudaStream_t)stream;
+  TL_CUDA(cudaMemcpyAsync(d_rows, rows.data(), rows_b, cudaMemcpyHostToDevice, st));
+  DecodeAttnArgs a{};
+  a.q = reinterpret_cast<const __half*>(d_q);
+  a.ldq = n_q_heads * head_dim;
+  a.k = reinterpret_cast<const __half*>(d_k);
+  a.v = reinterpret_cast<const __half*>(d_v);
+  a.lane_stride = batch_stride;
+  a.ctx = ctx_stride;
+  a.rows = d_rows;
+  a.Hkv = n_kv_heads;
+  a.out = reinterpret_cast<__half*>(d_out);
+  a.ldo = n_q_heads * head_dim;
+  a.part = part;
+  a.ticket = tick;
+  TL_CUDA(launch_decode_attn(a, B, head_dim, rep, st));
+  return TL_OK;
+}
+
+tl_status tl_op_gqa_prefill(const uint16_t* d_q, const uint16_t* d_k, const uint16_t* d_v, long long batch_stride,
+                            int ctx_stride, int T, int pos0, int B, int n_q_heads, int n_kv_heads, int head_dim,
+                            uint16_t* d_out, void* stream) {
+  if (!d_q || !d_k || !d_v || !d_out) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (B < 1 || T < 1 || pos0 < 0 || n_kv_heads < 1 || n_q_heads % n_kv_heads || !rep_ok(n_q_heads / n_kv_heads) ||
+      (head_dim != 64 && head_dim != 128))
+    return fail(TL_ERR_UNSUPPORTED, "unsupported attention shape");
+  if (pos0 + T > ctx_stride) return fail(TL_ERR_INVALID_ARG, "pos0 + T exceeds ctx_stride");
+  const int qdim = n_q_heads * head_dim;
+  PrefillAttnArgs a{};
+  a.q = reinterpret_cast<const __half*>(d_q);
+  a.q_bstride = (long long)T * qdim;
+  a.ldq = qdim;
+  a.k = reinterpret_cast<const __half*>(d_k);
+  a.v = reinterpret_cast<const __half*>(d_v);
+  a.kv_bstride = batch_stride;
+  a.ctx = ctx_stride;
+  a.T = T;
+  a.pos0 = pos0;
+  a.Hkv = n_kv_heads;
+  a.out = reinterpret_cast<__half*>(d_out);
+  a.o_bstride = (long long)T * qdim;
+  a.ldo = qdim;
+  TL_CUDA(launch_prefill_attn(a, B, head_dim, n_q_heads / n_kv_heads, (cudaStream_t)stream));
+  return TL_OK;
+}
+
+const char* tl_status_string(tl_status s) {
+  switch (s) {
+    case TL_OK: return "TL_OK";
+    case TL_ERR_INVALID_ARG: return "TL_ERR_INVALID_ARG";
+    case TL_ERR_OOM: return "TL_ERR_OOM";
+    case TL_ERR_CUDA: return "TL_ERR_CUDA";
+    case TL_ERR_CONTEXT_FULL: return "TL_ERR_CONTEXT_FULL";
+    case TL_ERR_LOOPS_MISMATCH: return "TL_ERR_LOOPS_MISMATCH";
+    case TL_ERR_NOT_PREFILLED: return "TL_ERR_NOT_PREFILLED";
+    case TL_ERR_DEVICE_FLAG: return "TL_ERR_DEVICE_FLAG";
+    case TL_ERR_UNSUPPORTED: return "TL_ERR_UNSUPPORTED";
+  }
+  return "TL_ERR_UNKNOWN";
+}
+
+const char* tl_last_error(void) { return g_err.c_str(); }
+
+const char* tl_version(void) { return "0.1.0"; }
+
+}  // extern "C"
