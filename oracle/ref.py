@@ -41,7 +41,14 @@ gate rows [0, F) and up rows [F, 2F) of the fused gate_up weight;
 the head is a separate matrix (not tied to the embedding).
 
 Everything is float64; the fp16 inputs (scales, gains, embedding, head,
-activations) are widened exactly.  No fp16 rounding is emulated anywhere.
+activations) are widened exactly.  One precision is fixed by the pages and so
+kept: keys and values are stored in an FP16 KV cache (TinyLoop README, "Python
+API reference": KV cache modes, "FP16 KV"; the workload's "KV cache fp16").  By
+default (``kv_fp16=True``) the rotated keys and the values are rounded to fp16
+(round-to-nearest-even) when they are produced, on the cached and the uncached
+path alike, so attention always reads the stored fp16 values.  With
+``kv_fp16=False`` nothing at all is rounded (used to compare against a float64
+library model).  No other fp16 rounding is emulated.
 """
 
 from __future__ import annotations
@@ -155,6 +162,12 @@ def gqa_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     return out.transpose(2, 0, 1, 3).reshape(T, Hq, hd)
 
 
+def to_fp16_storage(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest fp16 value (ties to even) and widen back to float64:
+    the value an FP16 KV cache holds."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
 def silu(u: np.ndarray) -> np.ndarray:
     return u / (1.0 + np.exp(-u))
 
@@ -229,9 +242,10 @@ class KVCache:
 class LoopedModel:
     """The looped transformer with the weights of a ``tl_synth.ModelWeights``."""
 
-    def __init__(self, weights):
+    def __init__(self, weights, kv_fp16: bool = True):
         sh = weights.shape
         self.shape = sh
+        self.kv_fp16 = kv_fp16
         self.embed = np.asarray(weights.embed, np.float64)
         self.out_norm = np.asarray(weights.out_norm, np.float64)
         self.head = np.asarray(weights.head, np.float64)
@@ -258,6 +272,8 @@ class LoopedModel:
         v = qkv[:, (Hq + Hkv) * hd:].reshape(T, Hkv, hd)
         q = rope(q, positions, sh.rope_theta)
         k = rope(k, positions, sh.rope_theta)
+        if self.kv_fp16:
+            k, v = to_fp16_storage(k), to_fp16_storage(v)
         if cache is not None:
             k_all, v_all = cache.append(layer, k, v)
         else:

@@ -26,6 +26,12 @@ def tiny():
     return w, ref.LoopedModel(w)
 
 
+@pytest.fixture(scope="module")
+def tiny_exact(tiny):
+    # no rounding anywhere: the form compared with the float64 library model
+    return tiny[0], ref.LoopedModel(tiny[0], kv_fp16=False)
+
+
 def test_looped_equals_flattened(tiny):
     _, m = tiny
     toks = tl_synth.make_tokens(1, m.shape.vocab, 17)
@@ -121,8 +127,8 @@ HF_TOL = 2e-5   # float32 internals of the library; logits are O(1)
 
 
 @pytest.mark.parametrize("loops", [1, 4])
-def test_matches_llama_decoder(tiny, loops):
-    _, m = tiny
+def test_matches_llama_decoder(tiny_exact, loops):
+    _, m = tiny_exact
     toks = tl_synth.make_tokens(6, m.shape.vocab, 33)
     hf = _hf_model(m, loops)
     ours = _oracle_all_logits(m, toks, loops)
@@ -181,11 +187,40 @@ MUTATIONS = {
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
-def test_planted_mistake_is_caught(tiny, monkeypatch, name):
-    _, m = tiny
+def test_planted_mistake_is_caught(tiny_exact, monkeypatch, name):
+    _, m = tiny_exact
     toks = tl_synth.make_tokens(6, m.shape.vocab, 33)
     hf = _hf_model(m, 2)
     attr, fn = MUTATIONS[name]
     monkeypatch.setattr(ref, attr, fn)
     err = np.max(np.abs(_oracle_all_logits(m, toks, 2) - _hf_logits(hf, toks)))
     assert err > 100 * HF_TOL, (name, err)
+
+
+# ------------------------------------------------------------ FP16 KV cache ---
+
+def test_kv_cache_holds_fp16_values(tiny, tiny_exact):
+    _, m = tiny
+    _, mx = tiny_exact
+    toks = tl_synth.make_tokens(8, m.shape.vocab, 9)
+    c16, _ = m.prefill(toks, 2)
+    cx, _ = mx.prefill(toks, 2)
+    for layer in range(m.shape.n_pre + 2):
+        k16, kx = c16.k[layer], cx.k[layer]
+        # stored values are fp16 numbers ...
+        assert np.array_equal(k16, k16.astype(np.float16).astype(np.float64))
+        assert np.array_equal(c16.v[layer], c16.v[layer].astype(np.float16).astype(np.float64))
+    # ... and the first layer's keys are exactly the rounded exact keys
+    assert np.array_equal(c16.k[0], cx.k[0].astype(np.float16).astype(np.float64))
+    # rounding the cache changes the result only a little
+    a = m.score_last(toks, 2)
+    b = mx.score_last(toks, 2)
+    assert 0 < np.max(np.abs(a - b)) < 1e-2
+
+
+def test_fp16_storage_rounding():
+    # ties go to even: 2049 lies halfway between fp16 neighbours 2048 and 2050
+    assert ref.to_fp16_storage(np.array([2049.0]))[0] == 2048.0
+    assert ref.to_fp16_storage(np.array([2051.0]))[0] == 2052.0
+    assert ref.to_fp16_storage(np.array([1.0 + 2.0 ** -11]))[0] == 1.0
+    assert ref.to_fp16_storage(np.array([65504.0]))[0] == 65504.0
