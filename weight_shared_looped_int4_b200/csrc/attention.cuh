@@ -32,8 +32,11 @@ __host__ __device__ inline int decode_split_len(int n_keys) {
   return c;
 }
 
+// Queries and outputs are fp32 inside the model (no rounding between the QKV
+// projection, attention and the O projection) and fp16 in the op API.
 struct DecodeAttnArgs {
-  const __half* q;       // [rows][Hq*hd] rotated queries
+  const float* qf;       // [rows][Hq*hd] rotated queries (fp32), or
+  const __half* qh;      // the same in fp16
   int ldq;
   const __half* k;       // K plane of lane 0 (this layer)
   const __half* v;       // V plane of lane 0
@@ -41,13 +44,23 @@ struct DecodeAttnArgs {
   int ctx;
   const RowCtx* rows;    // lane and position of each row; keys 0..pos
   int Hkv;
-  __half* out;           // [rows][Hq*hd]
+  float* of;             // [rows][Hq*hd] output (fp32), or
+  __half* oh;            // the same in fp16
   int ldo;
   float* part;           // [rows][Hkv][kDecodeMaxSplits][REP][hd+2]
   unsigned* ticket;      // [rows][Hkv], zero between launches
 };
 
-template <int HD, int REP>
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__half>(__half v) { return __half2float(v); }
+__device__ __forceinline__ void store_out(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store_out(__half* p, float v) { *p = __float2half_rn(v); }
+
+template <int HD, int REP, bool F32>
 __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const DecodeAttnArgs a) {
   constexpr int DPL = HD / 32;
   constexpr int CMAX = 256;  // largest split length (n_keys <= 8192)
@@ -71,8 +84,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
 
   const __half* kp = a.k + rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;
   const __half* vp = a.v + rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;
-  const __half* qp = a.q + (size_t)row * a.ldq + (size_t)kvh * REP * HD;
-  for (int i = threadIdx.x; i < REP * HD; i += kDecodeThreads) qs[i / HD][i % HD] = __half2float(qp[i]);
+  const size_t qoff = (size_t)row * a.ldq + (size_t)kvh * REP * HD;
+  for (int i = threadIdx.x; i < REP * HD; i += kDecodeThreads)
+    qs[i / HD][i % HD] = F32 ? a.qf[qoff + i] : __half2float(a.qh[qoff + i]);
   __syncthreads();
 
   // scores
@@ -127,11 +141,14 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
     }
   }
 
-  __half* op = a.out + (size_t)row * a.ldo + (size_t)kvh * REP * HD;
+  const size_t ooff = (size_t)row * a.ldo + (size_t)kvh * REP * HD;
   if (nsplit == 1) {
     if (d < HD) {
 #pragma unroll
-      for (int h = 0; h < REP; ++h) op[h * HD + d] = __float2half_rn(acc[h] / ml[h][1]);
+      for (int h = 0; h < REP; ++h) {
+        if (F32) store_out(a.of + ooff + h * HD + d, acc[h] / ml[h][1]);
+        else store_out(a.oh + ooff + h * HD + d, acc[h] / ml[h][1]);
+      }
     }
     return;
   }
@@ -169,7 +186,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
         den = fmaf(w, __ldcg(ps + HD + 1), den);
         num = fmaf(w, __ldcg(ps + d), num);
       }
-      op[h * HD + d] = __float2half_rn(num / den);
+      if (F32) store_out(a.of + ooff + h * HD + d, num / den);
+      else store_out(a.oh + ooff + h * HD + d, num / den);
     }
   }
   if (threadIdx.x == 0) a.ticket[row * a.Hkv + kvh] = 0u;
@@ -177,7 +195,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
 
 // ---- prefill (v1: one warp per query head, online softmax) ----------------
 struct PrefillAttnArgs {
-  const __half* q;        // [B][T][Hq*hd]
+  const float* qf;        // [B][T][Hq*hd] fp32 (model), or
+  const __half* qh;       // fp16 (op API)
   long long q_bstride;    // elements between batch entries
   int ldq;                // elements between tokens
   const __half* k;        // K plane of batch 0: [Hkv][ctx][hd]
@@ -186,12 +205,13 @@ struct PrefillAttnArgs {
   int ctx;
   int T, pos0;
   int Hkv;
-  __half* out;            // [B][T][Hq*hd]
+  float* of;              // [B][T][Hq*hd] fp32 (model), or
+  __half* oh;             // fp16 (op API)
   long long o_bstride;
   int ldo;
 };
 
-template <int HD, int REP>
+template <int HD, int REP, bool F32>
 __global__ void __launch_bounds__(REP * 32) prefill_attn_simple_kernel(const PrefillAttnArgs a) {
   constexpr int DPL = HD / 32;
   const int t = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -200,12 +220,15 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_simple_kernel(const Pre
   pdl_wait();
   const int pos = a.pos0 + t;
   const float scale = 1.0f / sqrtf((float)HD);
-  const __half* qp = a.q + b * a.q_bstride + (size_t)t * a.ldq + (size_t)(kvh * REP + h) * HD + lane * DPL;
+  const size_t qoff = b * a.q_bstride + (size_t)t * a.ldq + (size_t)(kvh * REP + h) * HD + lane * DPL;
   const __half* kp = a.k + b * a.kv_bstride + (size_t)kvh * a.ctx * HD + lane * DPL;
   const __half* vp = a.v + b * a.kv_bstride + (size_t)kvh * a.ctx * HD + lane * DPL;
   float qf[DPL], acc[DPL];
 #pragma unroll
-  for (int d = 0; d < DPL; ++d) { qf[d] = __half2float(qp[d]) * scale; acc[d] = 0.f; }
+  for (int d = 0; d < DPL; ++d) {
+    qf[d] = (F32 ? a.qf[qoff + d] : __half2float(a.qh[qoff + d])) * scale;
+    acc[d] = 0.f;
+  }
   float mx = -INFINITY, l = 0.f;
   for (int j = 0; j <= pos; ++j) {
     float s = 0.f;
@@ -220,9 +243,12 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_simple_kernel(const Pre
     for (int d = 0; d < DPL; ++d) acc[d] = fmaf(p, __half2float(vp[(size_t)j * HD + d]), acc[d] * corr);
     mx = mn;
   }
-  __half* op = a.out + b * a.o_bstride + (size_t)t * a.ldo + (size_t)(kvh * REP + h) * HD + lane * DPL;
+  const size_t ooff = b * a.o_bstride + (size_t)t * a.ldo + (size_t)(kvh * REP + h) * HD + lane * DPL;
 #pragma unroll
-  for (int d = 0; d < DPL; ++d) op[d] = __float2half_rn(acc[d] / l);
+  for (int d = 0; d < DPL; ++d) {
+    if (F32) store_out(a.of + ooff + d, acc[d] / l);
+    else store_out(a.oh + ooff + d, acc[d] / l);
+  }
 }
 
 }  // namespace tl

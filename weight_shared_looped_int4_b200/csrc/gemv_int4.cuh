@@ -20,16 +20,21 @@
 //   result does not depend on how many rows share the launch.
 // * Weight prefetch is issued before griddepcontrol.wait, so it overlaps the
 //   tail of the previous kernel under programmatic dependent launch.
-// * The prologue can fuse the block's RMSNorm (fp32 residual in, fp16 out into
-//   shared memory); the epilogue fuses RoPE + KV-cache write, SwiGLU, or the
-//   residual add.
+// * fp32 activations are split into an fp16 pair x = hi + lo (lo is the fp16
+//   rounding of x - hi) and both halves go through the MMA, so the product
+//   keeps about 22 bits of the activation instead of fp16's 11.  The looped
+//   model amplifies rounding across iterations, and fp16 activations alone
+//   move its logits by several 1e-2.
+// * The prologue can fuse the block's RMSNorm (fp32 residual in, fp16 pair
+//   out into shared memory); the epilogue fuses RoPE + KV-cache write, SwiGLU,
+//   or the residual add.
 #pragma once
 
 #include "common.cuh"
 
 namespace tl {
 
-enum GemvIn { IN_NORM = 0, IN_F16 = 1 };
+enum GemvIn { IN_NORM = 0, IN_F16 = 1, IN_F32 = 2 };
 enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_ROPE_KV = 3 };
 enum PairMode { PAIR_NEIGHBOUR = 0, PAIR_OFFSET = 1, PAIR_ROPE = 2 };
 
@@ -46,7 +51,7 @@ struct GemvArgs {
   int n_rows;          // valid output rows N
   int M;               // activation rows, 1..16
   // input
-  const float* x;      // IN_NORM: fp32 [M][ldx]
+  const float* x;      // IN_NORM / IN_F32: fp32 [M][ldx]
   const __half* xh;    // IN_F16:  fp16 [M][ldx]
   int ldx;
   const __half* gain;  // IN_NORM: RMSNorm gains [K]
@@ -55,12 +60,13 @@ struct GemvArgs {
   int pair_mode;
   int pair_off;        // PAIR_OFFSET: tiles between the two; PAIR_ROPE: hd/32
   // outputs
-  __half* y;           // EPI_STORE / EPI_SWIGLU: fp16 [M][ldy]
+  __half* y;           // EPI_STORE: fp16 [M][ldy]
+  float* yf;           // EPI_SWIGLU: fp32 [M][ldy]
   int ldy;
   float* resid;        // EPI_RESID: fp32 [M][ldr] += y
   int ldr;
   // EPI_ROPE_KV
-  __half* q_out;       // fp16 [M][ldq], rows < n_q_rows
+  float* q_out;        // fp32 [M][ldq], rows < n_q_rows
   int ldq;
   int n_q_rows;        // Hq * hd
   int n_kv_rows;       // Hkv * hd
@@ -76,17 +82,26 @@ struct GemvArgs {
 constexpr int kGemvThreads = 256;
 constexpr int kGemvPrefetch = 8;
 
-__host__ __device__ inline size_t gemv_smem_bytes(int K, int nt) {
-  return (size_t)nt * 8 * (K + 8) * 2 + (size_t)4 * 2 * 16 * nt * 8 * 4;
+// Shared memory: the activation planes (hi, and lo unless IN_F16) of M rows,
+// then the K-quarter reduction buffer.
+__host__ __device__ inline size_t gemv_act_bytes(int K, int M, bool lo) {
+  return (((size_t)M * (K + 8) * 2 * (lo ? 2 : 1)) + 15) / 16 * 16;
+}
+__host__ __device__ inline size_t gemv_smem_bytes(int K, int M, bool lo) {
+  const int nt = M <= 8 ? 1 : 2;
+  return gemv_act_bytes(K, M, lo) + (size_t)4 * 2 * 16 * nt * 8 * 4;
 }
 
 template <int NT, int IN, int EPI>
 __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs a) {
+  constexpr bool LO = (IN != IN_F16);
   extern __shared__ __align__(16) unsigned char smem[];
   const int K = a.K;
+  const int M = a.M;
   const int ldxs = K + 8;
-  __half* xs = reinterpret_cast<__half*>(smem);
-  float* red = reinterpret_cast<float*>(smem + (size_t)NT * 8 * ldxs * 2);
+  __half* xs = reinterpret_cast<__half*>(smem);           // hi plane [M][ldxs]
+  __half* xl = xs + (size_t)M * ldxs;                     // lo plane [M][ldxs]
+  float* red = reinterpret_cast<float*>(smem + gemv_act_bytes(K, M, LO));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -126,44 +141,44 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
 
   pdl_wait();
 
-  // ---- stage the activations (fp16, RMSNorm fused for IN_NORM) -----------
-  if (IN == IN_NORM) {
-    for (int m = warp; m < NT * 8; m += 8) {
+  // ---- stage the activations: fp16 pair (hi, lo) of the fp32 input --------
+  if (IN == IN_F16) {
+    for (int m = warp; m < M; m += 8) {
       __half* dst = xs + m * ldxs;
-      if (m < a.M) {
-        const float* src = a.x + (size_t)m * a.ldx;
+      const __half* src = a.xh + (size_t)m * a.ldx;
+      for (int k = lane * 8; k < K; k += 256)
+        *reinterpret_cast<uint4*>(dst + k) = *reinterpret_cast<const uint4*>(src + k);
+    }
+  } else {
+    for (int m = warp; m < M; m += 8) {
+      const float* src = a.x + (size_t)m * a.ldx;
+      float rs = 1.f;
+      if (IN == IN_NORM) {
         float ss = 0.f;
         for (int k = lane * 4; k < K; k += 128) {
           const float4 v = *reinterpret_cast<const float4*>(src + k);
           ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
         }
         ss = warp_sum(ss);
-        const float rs = 1.0f / sqrtf(ss / (float)K + a.eps);
-        for (int k = lane * 4; k < K; k += 128) {
-          const float4 v = *reinterpret_cast<const float4*>(src + k);
-          const __half2 g01 = *reinterpret_cast<const __half2*>(a.gain + k);
-          const __half2 g23 = *reinterpret_cast<const __half2*>(a.gain + k + 2);
-          const float2 fg01 = __half22float2(g01), fg23 = __half22float2(g23);
-          __half2 o01 = __floats2half2_rn((v.x * rs) * fg01.x, (v.y * rs) * fg01.y);
-          __half2 o23 = __floats2half2_rn((v.z * rs) * fg23.x, (v.w * rs) * fg23.y);
-          uint2 pk;
-          pk.x = *reinterpret_cast<uint32_t*>(&o01);
-          pk.y = *reinterpret_cast<uint32_t*>(&o23);
-          *reinterpret_cast<uint2*>(dst + k) = pk;
-        }
-      } else {
-        for (int k = lane * 4; k < K; k += 128) *reinterpret_cast<uint2*>(dst + k) = make_uint2(0, 0);
+        rs = 1.0f / sqrtf(ss / (float)K + a.eps);
       }
-    }
-  } else {
-    for (int m = warp; m < NT * 8; m += 8) {
-      __half* dst = xs + m * ldxs;
-      if (m < a.M) {
-        const __half* src = a.xh + (size_t)m * a.ldx;
-        for (int k = lane * 8; k < K; k += 256)
-          *reinterpret_cast<uint4*>(dst + k) = *reinterpret_cast<const uint4*>(src + k);
-      } else {
-        for (int k = lane * 8; k < K; k += 256) *reinterpret_cast<uint4*>(dst + k) = make_uint4(0, 0, 0, 0);
+      for (int k = lane * 4; k < K; k += 128) {
+        float4 v = *reinterpret_cast<const float4*>(src + k);
+        if (IN == IN_NORM) {
+          const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
+          const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k + 2));
+          v.x = (v.x * rs) * g01.x; v.y = (v.y * rs) * g01.y;
+          v.z = (v.z * rs) * g23.x; v.w = (v.w * rs) * g23.y;
+        }
+        const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+        const float2 r01 = __half22float2(h01), r23 = __half22float2(h23);
+        const __half2 l01 = __floats2half2_rn(v.x - r01.x, v.y - r01.y);
+        const __half2 l23 = __floats2half2_rn(v.z - r23.x, v.w - r23.y);
+        uint2 ph, pl;
+        ph.x = *reinterpret_cast<const uint32_t*>(&h01); ph.y = *reinterpret_cast<const uint32_t*>(&h23);
+        pl.x = *reinterpret_cast<const uint32_t*>(&l01); pl.y = *reinterpret_cast<const uint32_t*>(&l23);
+        *reinterpret_cast<uint2*>(xs + m * ldxs + k) = ph;
+        *reinterpret_cast<uint2*>(xl + m * ldxs + k) = pl;
       }
     }
   }
@@ -200,10 +215,19 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
           unpack_a_frag(words[j], sv.y, af);
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const __half* xr = xs + (nt * 8 + g) * ldxs + kc + j * 16;
-            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(xr);
-            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(xr + 8);
+            const int row = nt * 8 + g;   // activation row of this lane's B fragment
+            uint32_t b0 = 0, b1 = 0, c0 = 0, c1 = 0;
+            if (row < M) {
+              const size_t off = (size_t)row * ldxs + kc + j * 16;
+              b0 = *reinterpret_cast<const uint32_t*>(xs + off);
+              b1 = *reinterpret_cast<const uint32_t*>(xs + off + 8);
+              if (LO) {
+                c0 = *reinterpret_cast<const uint32_t*>(xl + off);
+                c1 = *reinterpret_cast<const uint32_t*>(xl + off + 8);
+              }
+            }
             mma_f16_16816(tmp[nt], af, b0, b1);
+            if (LO) mma_f16_16816(tmp[nt], af, c0, c1);
           }
         }
         const float2 s = h2_to_f2(sv.x);
@@ -248,16 +272,16 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
     if (row0 < a.n_rows) a.resid[(size_t)m * a.ldr + row0] += va;
     if (row1 < a.n_rows) a.resid[(size_t)m * a.ldr + row1] += vb;
   } else if (EPI == EPI_SWIGLU) {
-    a.y[(size_t)m * a.ldy + row0] = __float2half_rn(silu(va) * vb);
+    a.yf[(size_t)m * a.ldy + row0] = silu(va) * vb;
   } else {  // EPI_ROPE_KV: row0 is element j < hd/2 of a head, row1 = row0 + hd/2
     const int hd = a.hd;
     const int j = row0 % hd;
     const RowCtx rc = a.rows[m];
     if (row0 < a.n_q_rows) {
       const float2 cs = rope_cos_sin(rc.pos, j, hd, a.theta);
-      __half* qo = a.q_out + (size_t)m * a.ldq;
-      qo[row0] = __float2half_rn(va * cs.x - vb * cs.y);
-      qo[row1] = __float2half_rn(vb * cs.x + va * cs.y);
+      float* qo = a.q_out + (size_t)m * a.ldq;
+      qo[row0] = va * cs.x - vb * cs.y;
+      qo[row1] = vb * cs.x + va * cs.y;
     } else if (row0 < a.n_q_rows + a.n_kv_rows) {
       const float2 cs = rope_cos_sin(rc.pos, j, hd, a.theta);
       const int kvh = (row0 - a.n_q_rows) / hd;

@@ -121,20 +121,23 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-__host__ __device__ inline size_t head_smem_bytes(int d, int nt) {
-  return (size_t)nt * 8 * (d + 8) * 2;
+// Activation planes (hi, lo) of M rows.
+__host__ __device__ inline size_t head_smem_bytes(int d, int M) {
+  return (size_t)M * (d + 8) * 2 * 2;
 }
 
 // One warp per 16-row tile over all of K; the CTA's 8 warps take 8
-// consecutive tiles.  The output norm is computed per CTA in the prologue.
+// consecutive tiles.  The output norm is computed per CTA in the prologue and
+// kept as an fp16 pair (hi, lo) like the INT4 GEMV's activations.
 template <int NT>
 __global__ void __launch_bounds__(kHeadThreads) head_argmax_kernel(const HeadArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ float s_val[8][16];
   __shared__ int s_idx[8][16];
   __shared__ int s_last;
-  const int d = a.d, ldxs = d + 8;
+  const int d = a.d, ldxs = d + 8, M = a.M;
   __half* xs = reinterpret_cast<__half*>(smem);
+  __half* xl = xs + (size_t)M * ldxs;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int n_tiles = a.V >> 4;
@@ -150,27 +153,28 @@ __global__ void __launch_bounds__(kHeadThreads) head_argmax_kernel(const HeadArg
     if (has_tile && i < nk) buf[i] = ldg_stream(wp + (size_t)i * 32);
   pdl_wait();
 
-  // output RMSNorm of every row into shared memory (fp16)
-  for (int m = warp; m < NT * 8; m += 8) {
-    __half* dst = xs + m * ldxs;
-    if (m < a.M) {
-      const float* src = a.x + (size_t)m * d;
-      float ss = 0.f;
-      for (int k = lane * 4; k < d; k += 128) {
-        const float4 v = *reinterpret_cast<const float4*>(src + k);
-        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-      }
-      ss = warp_sum(ss);
-      const float rs = 1.0f / sqrtf(ss / (float)d + a.eps);
-      for (int k = lane * 4; k < d; k += 128) {
-        const float4 v = *reinterpret_cast<const float4*>(src + k);
-        const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
-        const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k + 2));
-        *reinterpret_cast<__half2*>(dst + k) = __floats2half2_rn((v.x * rs) * g01.x, (v.y * rs) * g01.y);
-        *reinterpret_cast<__half2*>(dst + k + 2) = __floats2half2_rn((v.z * rs) * g23.x, (v.w * rs) * g23.y);
-      }
-    } else {
-      for (int k = lane * 4; k < d; k += 128) *reinterpret_cast<uint2*>(dst + k) = make_uint2(0, 0);
+  // output RMSNorm of every row into shared memory as an fp16 pair
+  for (int m = warp; m < M; m += 8) {
+    const float* src = a.x + (size_t)m * d;
+    float ss = 0.f;
+    for (int k = lane * 4; k < d; k += 128) {
+      const float4 v = *reinterpret_cast<const float4*>(src + k);
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = warp_sum(ss);
+    const float rs = 1.0f / sqrtf(ss / (float)d + a.eps);
+    for (int k = lane * 4; k < d; k += 128) {
+      float4 v = *reinterpret_cast<const float4*>(src + k);
+      const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
+      const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k + 2));
+      v.x = (v.x * rs) * g01.x; v.y = (v.y * rs) * g01.y;
+      v.z = (v.z * rs) * g23.x; v.w = (v.w * rs) * g23.y;
+      const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+      const float2 r01 = __half22float2(h01), r23 = __half22float2(h23);
+      *reinterpret_cast<__half2*>(xs + m * ldxs + k) = h01;
+      *reinterpret_cast<__half2*>(xs + m * ldxs + k + 2) = h23;
+      *reinterpret_cast<__half2*>(xl + m * ldxs + k) = __floats2half2_rn(v.x - r01.x, v.y - r01.y);
+      *reinterpret_cast<__half2*>(xl + m * ldxs + k + 2) = __floats2half2_rn(v.z - r23.x, v.w - r23.y);
     }
   }
   __syncthreads();
@@ -192,9 +196,17 @@ __global__ void __launch_bounds__(kHeadThreads) head_argmax_kernel(const HeadArg
           const uint32_t af[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            const __half* xr = xs + (nt * 8 + g) * ldxs + kk * 16 + 2 * t;
-            mma_f16_16816(acc[nt], af, *reinterpret_cast<const uint32_t*>(xr),
-                          *reinterpret_cast<const uint32_t*>(xr + 8));
+            const int row = nt * 8 + g;
+            uint32_t b0 = 0, b1 = 0, c0 = 0, c1 = 0;
+            if (row < M) {
+              const size_t off = (size_t)row * ldxs + kk * 16 + 2 * t;
+              b0 = *reinterpret_cast<const uint32_t*>(xs + off);
+              b1 = *reinterpret_cast<const uint32_t*>(xs + off + 8);
+              c0 = *reinterpret_cast<const uint32_t*>(xl + off);
+              c1 = *reinterpret_cast<const uint32_t*>(xl + off + 8);
+            }
+            mma_f16_16816(acc[nt], af, b0, b1);
+            mma_f16_16816(acc[nt], af, c0, c1);
           }
         }
       }
@@ -209,7 +221,7 @@ __global__ void __launch_bounds__(kHeadThreads) head_argmax_kernel(const HeadArg
       const int m = nt * 8 + 2 * t + c;
       const int ra = tile * 16 + g, rb = ra + 8;
       const float va = acc[nt][c], vb = acc[nt][2 + c];
-      if (has_tile && m < a.M && a.logits) {
+      if (has_tile && m < M && a.logits) {
         const int orow = a.out_row ? a.out_row[m] : m;
         a.logits[(size_t)orow * a.V + ra] = va;
         a.logits[(size_t)orow * a.V + rb] = vb;
@@ -230,7 +242,7 @@ __global__ void __launch_bounds__(kHeadThreads) head_argmax_kernel(const HeadArg
   __syncthreads();
 
   if (!a.argmax) return;
-  if (threadIdx.x < a.M) {
+  if (threadIdx.x < M) {
     const int m = threadIdx.x;
     float bv = s_val[0][m];
     int bi = s_idx[0][m];

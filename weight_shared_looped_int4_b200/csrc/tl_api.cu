@@ -135,16 +135,28 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   return e;
 }
 
-constexpr size_t kMaxDynSmem = 227 * 1024;
+constexpr size_t kMaxDynSmem = 220 * 1024;  // budget for dynamic smem per CTA
 
 // One-time per-device attribute setup for kernels with large dynamic smem.
 std::mutex g_init_mu;
 std::map<int, bool> g_dev_init;
 
+// Allow a kernel the opt-in shared memory of the device minus its static part.
+template <typename K>
+cudaError_t allow_max_smem(K* kern, int dev) {
+  int optin = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              optin - (int)fa.sharedSizeBytes);
+}
+
 template <int NT, int IN, int EPI>
-cudaError_t set_gemv_attr() {
-  return cudaFuncSetAttribute(gemv_int4_kernel<NT, IN, EPI>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxDynSmem);
+cudaError_t set_gemv_attr(int dev) {
+  return allow_max_smem(gemv_int4_kernel<NT, IN, EPI>, dev);
 }
 
 cudaError_t init_device_kernels(int dev) {
@@ -152,41 +164,58 @@ cudaError_t init_device_kernels(int dev) {
   if (g_dev_init[dev]) return cudaSuccess;
   cudaError_t e = cudaSuccess;
 #define SET(NT, IN, EPI) \
-  if (e == cudaSuccess) e = set_gemv_attr<NT, IN, EPI>();
+  if (e == cudaSuccess) e = set_gemv_attr<NT, IN, EPI>(dev);
   SET(1, IN_F16, EPI_STORE) SET(2, IN_F16, EPI_STORE)
-  SET(1, IN_F16, EPI_RESID) SET(2, IN_F16, EPI_RESID)
+  SET(1, IN_F32, EPI_RESID) SET(2, IN_F32, EPI_RESID)
   SET(1, IN_NORM, EPI_SWIGLU) SET(2, IN_NORM, EPI_SWIGLU)
   SET(1, IN_NORM, EPI_ROPE_KV) SET(2, IN_NORM, EPI_ROPE_KV)
 #undef SET
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(head_argmax_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kMaxDynSmem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(head_argmax_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kMaxDynSmem);
+  if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<1>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<2>, dev);
   if (e == cudaSuccess) g_dev_init[dev] = true;
   return e;
 }
 
-// Largest activation-row count per GEMV launch that fits shared memory.
-int gemv_rows_per_launch(int K) {
-  if (gemv_smem_bytes(K, 2) <= kMaxDynSmem) return 16;
-  if (gemv_smem_bytes(K, 1) <= kMaxDynSmem) return 8;
-  return 0;
+// Largest activation-row count (<= 16) per GEMV launch that fits shared memory.
+int gemv_rows_per_launch(int K, bool lo) {
+  int M = kMaxLanes;
+  while (M > 0 && gemv_smem_bytes(K, M, lo) > kMaxDynSmem) --M;
+  return M;
 }
 
 cudaError_t launch_gemv(const GemvArgs& a, int grid, int in_mode, int epi, cudaStream_t st) {
   const int nt = a.M <= 8 ? 1 : 2;
-  const size_t smem = gemv_smem_bytes(a.K, nt);
+  const size_t smem = gemv_smem_bytes(a.K, a.M, in_mode != IN_F16);
   const dim3 g(grid), b(kGemvThreads);
 #define CASE(NT, IN, EPI) \
   if (nt == NT && in_mode == IN && epi == EPI) return launch(gemv_int4_kernel<NT, IN, EPI>, g, b, smem, st, a);
   CASE(1, IN_F16, EPI_STORE) CASE(2, IN_F16, EPI_STORE)
-  CASE(1, IN_F16, EPI_RESID) CASE(2, IN_F16, EPI_RESID)
+  CASE(1, IN_F32, EPI_RESID) CASE(2, IN_F32, EPI_RESID)
   CASE(1, IN_NORM, EPI_SWIGLU) CASE(2, IN_NORM, EPI_SWIGLU)
   CASE(1, IN_NORM, EPI_ROPE_KV) CASE(2, IN_NORM, EPI_ROPE_KV)
 #undef CASE
   return cudaErrorInvalidValue;
+}
+
+// Launch a GEMV over `total` activation rows, in chunks of as many rows as
+// fit shared memory; every row-indexed pointer advances with the chunk.
+cudaError_t launch_gemv_rows(GemvArgs a, int total, int in_mode, int epi, int grid, cudaStream_t st) {
+  const int per = gemv_rows_per_launch(a.K, in_mode != IN_F16);
+  if (per < 1) return cudaErrorInvalidValue;
+  for (int r0 = 0; r0 < total; r0 += per) {
+    GemvArgs c = a;
+    c.M = std::min(per, total - r0);
+    if (c.x) c.x += (size_t)r0 * a.ldx;
+    if (c.xh) c.xh += (size_t)r0 * a.ldx;
+    if (c.rows) c.rows += r0;
+    if (c.q_out) c.q_out += (size_t)r0 * a.ldq;
+    if (c.y) c.y += (size_t)r0 * a.ldy;
+    if (c.yf) c.yf += (size_t)r0 * a.ldy;
+    if (c.resid) c.resid += (size_t)r0 * a.ldr;
+    const cudaError_t e = launch_gemv(c, grid, in_mode, epi, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 // ============================================================================
@@ -302,23 +331,26 @@ __global__ void fill_rows_kernel(RowCtx* rows, int n, int lane, int pos0) {
 }
 
 
-template <int HD, int REP>
+template <int HD, int REP, bool F32>
 cudaError_t launch_decode_attn_t(const DecodeAttnArgs& a, int rows, cudaStream_t st) {
-  return launch(decode_attn_kernel<HD, REP>, dim3(kDecodeMaxSplits, a.Hkv, rows), dim3(kDecodeThreads), 0, st, a);
+  return launch(decode_attn_kernel<HD, REP, F32>, dim3(kDecodeMaxSplits, a.Hkv, rows), dim3(kDecodeThreads), 0,
+                st, a);
 }
 
-cudaError_t launch_decode_attn(const DecodeAttnArgs& a, int rows, int hd, int rep, cudaStream_t st) {
-#define C(HD, REP) \
-  if (hd == HD && rep == REP) return launch_decode_attn_t<HD, REP>(a, rows, st);
+cudaError_t launch_decode_attn(const DecodeAttnArgs& a, int rows, int hd, int rep, bool f32, cudaStream_t st) {
+#define C(HD, REP)                                                                                   \
+  if (hd == HD && rep == REP)                                                                        \
+    return f32 ? launch_decode_attn_t<HD, REP, true>(a, rows, st) : launch_decode_attn_t<HD, REP, false>(a, rows, st);
   C(64, 1) C(64, 2) C(64, 4) C(64, 8) C(128, 1) C(128, 2) C(128, 4) C(128, 8)
 #undef C
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, int B, int hd, int rep, cudaStream_t st) {
-#define C(HD, REP)                                                                                \
-  if (hd == HD && rep == REP)                                                                     \
-    return launch(prefill_attn_simple_kernel<HD, REP>, dim3(a.T, a.Hkv, B), dim3(REP * 32), 0, st, a);
+cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, int B, int hd, int rep, bool f32, cudaStream_t st) {
+#define C(HD, REP)                                                                                       \
+  if (hd == HD && rep == REP)                                                                            \
+    return f32 ? launch(prefill_attn_simple_kernel<HD, REP, true>, dim3(a.T, a.Hkv, B), dim3(REP * 32), 0, st, a) \
+               : launch(prefill_attn_simple_kernel<HD, REP, false>, dim3(a.T, a.Hkv, B), dim3(REP * 32), 0, st, a);
   C(64, 1) C(64, 2) C(64, 4) C(64, 8) C(128, 1) C(128, 2) C(128, 4) C(128, 8)
 #undef C
   return cudaErrorInvalidValue;
@@ -344,10 +376,10 @@ struct tl_model {
   __half* kv = nullptr;
   long long plane = 0, layer_stride = 0, lane_stride = 0;
   // workspaces
-  float* x = nullptr;
-  __half* q = nullptr;
-  __half* o = nullptr;
-  __half* h = nullptr;
+  float* x = nullptr;   // residual stream [rows][d]
+  float* q = nullptr;   // rotated queries [rows][Hq*hd]
+  float* o = nullptr;   // attention output [rows][Hq*hd]
+  float* h = nullptr;   // SwiGLU output [rows][F]
   RowCtx* rows = nullptr;
   int* tok_index = nullptr;
   int* out_row = nullptr;
@@ -416,74 +448,74 @@ tl_status upload_block(const tl_config& c, const tl_block& hb, BlockDev* b, cuda
   return TL_OK;
 }
 
-// ---- one effective layer for M rows (M <= 16) -------------------------------
-// x: fp32 [M][d] residual rows, rows: their lanes/positions, q/o/h buffers.
-tl_status layer_rows(tl_model* m, int layer, int M, float* x, const RowCtx* rows, __half* q,
-                     __half* o, __half* h, bool decode_attn, cudaStream_t st) {
+// ---- one effective layer ------------------------------------------------------
+// QKV projection of `M` rows of the residual stream x (RMSNorm fused), RoPE on
+// q and k, k and v written to cache slice `layer` at each row's (lane, pos).
+tl_status run_qkv(tl_model* m, int layer, int M, float* x, const RowCtx* rows, float* q, cudaStream_t st) {
   const tl_config& c = m->cfg;
   const BlockDev& b = m->block(layer);
-  const int d = c.d_model, hd = c.head_dim, F = c.ffn_dim;
-  const int qdim = c.n_q_heads * hd;
+  const int hd = c.head_dim, qdim = c.n_q_heads * hd;
   GemvArgs a{};
-  a.M = M;
   a.eps = c.rms_eps;
   a.theta = c.rope_theta;
   a.rows = rows;
   a.hd = hd;
-
-  // QKV with fused RMSNorm, RoPE and KV write
-  a.w = b.qkv.w; a.sz = b.qkv.sz; a.K = d; a.n_rows = b.qkv.N;
-  a.x = x; a.ldx = d; a.gain = b.attn_norm;
+  a.w = b.qkv.w; a.sz = b.qkv.sz; a.K = c.d_model; a.n_rows = b.qkv.N;
+  a.x = x; a.ldx = c.d_model; a.gain = b.attn_norm;
   a.pair_mode = PAIR_ROPE; a.pair_off = hd / 32;
   a.q_out = q; a.ldq = qdim; a.n_q_rows = qdim; a.n_kv_rows = c.n_kv_heads * hd;
   a.k_plane = m->k_plane(layer); a.v_plane = m->v_plane(layer);
   a.lane_stride = m->lane_stride; a.ctx = c.max_ctx;
   kclass(TL_KERNEL_QKV);
-  TL_CUDA(launch_gemv(a, (c.n_q_heads + 2 * c.n_kv_heads) * hd / 32, IN_NORM, EPI_ROPE_KV, st));
-  if (decode_attn) {
-    DecodeAttnArgs da{};
-    da.q = q; da.ldq = qdim;
-    da.k = m->k_plane(layer); da.v = m->v_plane(layer);
-    da.lane_stride = m->lane_stride; da.ctx = c.max_ctx;
-    da.rows = rows; da.Hkv = c.n_kv_heads;
-    da.out = o; da.ldo = qdim;
-    da.part = m->attn_part; da.ticket = m->attn_tickets();
-    kclass(TL_KERNEL_ATTN_DECODE);
-    TL_CUDA(launch_decode_attn(da, M, hd, c.n_q_heads / c.n_kv_heads, st));
-  }
+  TL_CUDA(launch_gemv_rows(a, M, IN_NORM, EPI_ROPE_KV, (c.n_q_heads + 2 * c.n_kv_heads) * hd / 32, st));
   return TL_OK;
 }
 
-tl_status layer_rows_post(tl_model* m, int layer, int M, float* x, __half* o, __half* h,
+// Single-query attention of M decode rows over their lanes' slice `layer`.
+tl_status run_decode_attn(tl_model* m, int layer, int M, const RowCtx* rows, const float* q, float* o,
                           cudaStream_t st) {
   const tl_config& c = m->cfg;
-  const BlockDev& b = m->block(layer);
-  const int d = c.d_model, F = c.ffn_dim;
   const int qdim = c.n_q_heads * c.head_dim;
+  DecodeAttnArgs da{};
+  da.qf = q; da.ldq = qdim;
+  da.k = m->k_plane(layer); da.v = m->v_plane(layer);
+  da.lane_stride = m->lane_stride; da.ctx = c.max_ctx;
+  da.rows = rows; da.Hkv = c.n_kv_heads;
+  da.of = o; da.ldo = qdim;
+  da.part = m->attn_part; da.ticket = m->attn_tickets();
+  kclass(TL_KERNEL_ATTN_DECODE);
+  TL_CUDA(launch_decode_attn(da, M, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
+  return TL_OK;
+}
+
+// O projection + residual, RMSNorm + gate_up + SwiGLU, down + residual.
+tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float* h, cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  const BlockDev& b = m->block(layer);
+  const int d = c.d_model, F = c.ffn_dim, qdim = c.n_q_heads * c.head_dim;
   GemvArgs a{};
-  a.M = M;
   a.eps = c.rms_eps;
-  // O projection + residual
   a.w = b.o.w; a.sz = b.o.sz; a.K = qdim; a.n_rows = d;
-  a.xh = o; a.ldx = qdim;
+  a.x = o; a.ldx = qdim;
   a.pair_mode = PAIR_NEIGHBOUR;
   a.resid = x; a.ldr = d;
   kclass(TL_KERNEL_O_PROJ);
-  TL_CUDA(launch_gemv(a, b.o.n_tiles / 2, IN_F16, EPI_RESID, st));
-  // gate_up with fused RMSNorm and SwiGLU
-  a.w = b.gate_up.w; a.sz = b.gate_up.sz; a.K = d; a.n_rows = 2 * F;
-  a.x = x; a.ldx = d; a.gain = b.ffn_norm;
-  a.pair_mode = PAIR_OFFSET; a.pair_off = F / 16;
-  a.y = h; a.ldy = F;
+  TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, b.o.n_tiles / 2, st));
+  GemvArgs g{};
+  g.eps = c.rms_eps;
+  g.w = b.gate_up.w; g.sz = b.gate_up.sz; g.K = d; g.n_rows = 2 * F;
+  g.x = x; g.ldx = d; g.gain = b.ffn_norm;
+  g.pair_mode = PAIR_OFFSET; g.pair_off = F / 16;
+  g.yf = h; g.ldy = F;
   kclass(TL_KERNEL_GATE_UP);
-  TL_CUDA(launch_gemv(a, F / 16, IN_NORM, EPI_SWIGLU, st));
-  // down + residual
-  a.w = b.down.w; a.sz = b.down.sz; a.K = F; a.n_rows = d;
-  a.xh = h; a.ldx = F;
-  a.pair_mode = PAIR_NEIGHBOUR;
-  a.resid = x; a.ldr = d;
+  TL_CUDA(launch_gemv_rows(g, M, IN_NORM, EPI_SWIGLU, F / 16, st));
+  GemvArgs dn{};
+  dn.w = b.down.w; dn.sz = b.down.sz; dn.K = F; dn.n_rows = d;
+  dn.x = h; dn.ldx = F;
+  dn.pair_mode = PAIR_NEIGHBOUR;
+  dn.resid = x; dn.ldr = d;
   kclass(TL_KERNEL_DOWN);
-  TL_CUDA(launch_gemv(a, b.down.n_tiles / 2, IN_F16, EPI_RESID, st));
+  TL_CUDA(launch_gemv_rows(dn, M, IN_F32, EPI_RESID, b.down.n_tiles / 2, st));
   return TL_OK;
 }
 
@@ -496,7 +528,7 @@ tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, fl
   ha.out_row = out_row; ha.logits = logits; ha.argmax = argmax;
   ha.part_val = m->head_val; ha.part_idx = m->head_idx; ha.ticket = m->head_ticket();
   const int nt = M <= 8 ? 1 : 2;
-  const size_t smem = head_smem_bytes(c.d_model, nt);
+  const size_t smem = head_smem_bytes(c.d_model, M);
   kclass(TL_KERNEL_HEAD);
   if (nt == 1) TL_CUDA(launch(head_argmax_kernel<1>, dim3(m->head_grid), dim3(kHeadThreads), smem, st, ha));
   else TL_CUDA(launch(head_argmax_kernel<2>, dim3(m->head_grid), dim3(kHeadThreads), smem, st, ha));
@@ -514,30 +546,20 @@ tl_status forward_prompt(tl_model* m, int lane, const int32_t* d_tokens, int T, 
   kclass(TL_KERNEL_EMBED);
   TL_CUDA(launch(embed_kernel, dim3(T), dim3(256), 0, st, (const __half*)m->embed, d, c.vocab,
                  d_tokens, (const int*)nullptr, m->x, m->err_flag));
-  const int chunk = kMaxLanes;
   for (int layer = 0; layer < n_layers; ++layer) {
-    for (int r0 = 0; r0 < T; r0 += chunk) {
-      const int M = std::min(chunk, T - r0);
-      tl_status rc = layer_rows(m, layer, M, m->x + (size_t)r0 * d, m->rows + r0,
-                                m->q + (size_t)r0 * qdim, m->o + (size_t)r0 * qdim,
-                                m->h + (size_t)r0 * F, false, st);
-      if (rc != TL_OK) return rc;
-    }
+    tl_status rc = run_qkv(m, layer, T, m->x, m->rows, m->q, st);
+    if (rc != TL_OK) return rc;
     PrefillAttnArgs pa{};
-    pa.q = m->q; pa.q_bstride = 0; pa.ldq = qdim;
+    pa.qf = m->q; pa.q_bstride = 0; pa.ldq = qdim;
     pa.k = m->k_plane(layer) + lane * m->lane_stride;
     pa.v = m->v_plane(layer) + lane * m->lane_stride;
     pa.kv_bstride = 0; pa.ctx = c.max_ctx;
     pa.T = T; pa.pos0 = 0; pa.Hkv = c.n_kv_heads;
-    pa.out = m->o; pa.o_bstride = 0; pa.ldo = qdim;
+    pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
     kclass(TL_KERNEL_ATTN_PREFILL);
-    TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, st));
-    for (int r0 = 0; r0 < T; r0 += chunk) {
-      const int M = std::min(chunk, T - r0);
-      tl_status rc = layer_rows_post(m, layer, M, m->x + (size_t)r0 * d, m->o + (size_t)r0 * qdim,
-                                     m->h + (size_t)r0 * F, st);
-      if (rc != TL_OK) return rc;
-    }
+    TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
+    rc = run_ffn(m, layer, T, m->x, m->o, m->h, st);
+    if (rc != TL_OK) return rc;
   }
   if (d_logits || d_argmax)
     return launch_head(m, m->x + (size_t)(T - 1) * d, 1, nullptr, d_logits, d_argmax, st);
@@ -616,8 +638,8 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     if (cudaMalloc(p, bytes) != cudaSuccess) return false;
     return cudaMemsetAsync(*p, 0, bytes, st) == cudaSuccess;
   };
-  bool ok = alloc((void**)&m->x, (size_t)rows * d * 4) && alloc((void**)&m->q, (size_t)rows * qdim * 2) &&
-            alloc((void**)&m->o, (size_t)rows * qdim * 2) && alloc((void**)&m->h, (size_t)rows * c.ffn_dim * 2) &&
+  bool ok = alloc((void**)&m->x, (size_t)rows * d * 4) && alloc((void**)&m->q, (size_t)rows * qdim * 4) &&
+            alloc((void**)&m->o, (size_t)rows * qdim * 4) && alloc((void**)&m->h, (size_t)rows * c.ffn_dim * 4) &&
             alloc((void**)&m->rows, (size_t)rows * sizeof(RowCtx)) &&
             alloc((void**)&m->tok_index, kMaxLanes * 4) && alloc((void**)&m->out_row, kMaxLanes * 4) &&
             alloc((void**)&m->attn_part, (size_t)kMaxLanes * c.n_kv_heads * kDecodeMaxSplits * rep * (hd + 2) * 4) &&
@@ -721,8 +743,9 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
   for (int layer = 0; layer < max_layers; ++layer) {
     int M = 0;
     while (M < n_lanes && c.n_pre + h_loops[order[M]] > layer) ++M;
-    tl_status rc = layer_rows(m, layer, M, m->x, m->rows, m->q, m->o, m->h, true, st);
-    if (rc == TL_OK) rc = layer_rows_post(m, layer, M, m->x, m->o, m->h, st);
+    tl_status rc = run_qkv(m, layer, M, m->x, m->rows, m->q, st);
+    if (rc == TL_OK) rc = run_decode_attn(m, layer, M, m->rows, m->q, m->o, st);
+    if (rc == TL_OK) rc = run_ffn(m, layer, M, m->x, m->o, m->h, st);
     if (rc != TL_OK) return rc;
   }
   if (d_logits || d_argmax) {
@@ -803,19 +826,27 @@ struct tl_linear {
 };
 
 namespace {
-// Library-owned per-device workspace of the op entry points.
+// Library-owned per-device workspace of the op entry points: a grow-only
+// scratch buffer (row descriptors, split-KV partials) and a fixed array of
+// tickets that is zeroed once and that every kernel leaves zeroed.
+constexpr int kOpTickets = 65536;
 struct OpWorkspace {
   void* buf = nullptr;
   size_t bytes = 0;
+  unsigned* tickets = nullptr;
 };
 std::mutex g_ws_mu;
 std::map<int, OpWorkspace> g_ws;
 
-// Returns a zero-initialised-at-allocation device buffer of at least `bytes`.
-// Growing it synchronises the device.
-tl_status op_workspace(int dev, size_t bytes, void** out) {
+// Scratch of at least `bytes` (contents undefined) and the ticket array.
+// Growing the scratch synchronises the device.
+tl_status op_workspace(int dev, size_t bytes, void** out, unsigned** tickets) {
   std::lock_guard<std::mutex> lk(g_ws_mu);
   OpWorkspace& w = g_ws[dev];
+  if (!w.tickets) {
+    TL_CUDA(cudaMalloc(&w.tickets, kOpTickets * sizeof(unsigned)));
+    TL_CUDA(cudaMemset(w.tickets, 0, kOpTickets * sizeof(unsigned)));
+  }
   if (w.bytes < bytes) {
     if (w.buf) {
       cudaDeviceSynchronize();
@@ -825,10 +856,10 @@ tl_status op_workspace(int dev, size_t bytes, void** out) {
     }
     const size_t nb = std::max(bytes, (size_t)1 << 20);
     TL_CUDA(cudaMalloc(&w.buf, nb));
-    TL_CUDA(cudaMemset(w.buf, 0, nb));
     w.bytes = nb;
   }
   *out = w.buf;
+  *tickets = w.tickets;
   return TL_OK;
 }
 }  // namespace
@@ -876,17 +907,13 @@ tl_status tl_linear_forward(tl_linear* l, const uint16_t* d_x, int M, uint16_t* 
   DeviceGuard guard(l->device);
   if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
   const int K = l->w.K, N = l->w.N;
-  const int rpl = gemv_rows_per_launch(K);
-  if (!rpl) return fail(TL_ERR_UNSUPPORTED, "K too large for the GEMV");
+  if (gemv_rows_per_launch(K, false) < 1) return fail(TL_ERR_UNSUPPORTED, "K too large for the GEMV");
   GemvArgs a{};
   a.w = l->w.w; a.sz = l->w.sz; a.K = K; a.n_rows = N;
-  a.ldx = K; a.pair_mode = PAIR_NEIGHBOUR; a.ldy = N;
-  for (int r0 = 0; r0 < M; r0 += rpl) {
-    a.M = std::min(rpl, M - r0);
-    a.xh = reinterpret_cast<const __half*>(d_x) + (size_t)r0 * K;
-    a.y = reinterpret_cast<__half*>(d_y) + (size_t)r0 * N;
-    TL_CUDA(launch_gemv(a, l->w.n_tiles / 2, IN_F16, EPI_STORE, (cudaStream_t)stream));
-  }
+  a.xh = reinterpret_cast<const __half*>(d_x); a.ldx = K;
+  a.pair_mode = PAIR_NEIGHBOUR;
+  a.y = reinterpret_cast<__half*>(d_y); a.ldy = N;
+  TL_CUDA(launch_gemv_rows(a, M, IN_F16, EPI_STORE, l->w.n_tiles / 2, (cudaStream_t)stream));
   return TL_OK;
 }
 
@@ -930,18 +957,18 @@ tl_status tl_op_gqa_decode(const uint16_t* d_q, const uint16_t* d_k, const uint1
   const int rep = n_q_heads / n_kv_heads;
   const size_t rows_b = (size_t)B * sizeof(RowCtx);
   const size_t part_b = (size_t)B * n_kv_heads * kDecodeMaxSplits * rep * (head_dim + 2) * 4;
-  const size_t tick_b = (size_t)B * n_kv_heads * 4;
+  if ((long long)B * n_kv_heads > kOpTickets) return fail(TL_ERR_UNSUPPORTED, "B * n_kv_heads > %d", kOpTickets);
   void* ws = nullptr;
-  tl_status rc = op_workspace(dev, rows_b + part_b + tick_b + 256, &ws);
+  unsigned* tick = nullptr;
+  tl_status rc = op_workspace(dev, ((rows_b + 255) / 256) * 256 + part_b, &ws, &tick);
   if (rc != TL_OK) return rc;
   char* base = (char*)ws;
   RowCtx* d_rows = (RowCtx*)base;
   float* part = (float*)(base + ((rows_b + 255) / 256) * 256);
-  unsigned* tick = (unsigned*)((char*)part + part_b);
   cudaStream_t st = (cudaStream_t)stream;
   TL_CUDA(cudaMemcpyAsync(d_rows, rows.data(), rows_b, cudaMemcpyHostToDevice, st));
   DecodeAttnArgs a{};
-  a.q = reinterpret_cast<const __half*>(d_q);
+  a.qh = reinterpret_cast<const __half*>(d_q);
   a.ldq = n_q_heads * head_dim;
   a.k = reinterpret_cast<const __half*>(d_k);
   a.v = reinterpret_cast<const __half*>(d_v);
@@ -949,11 +976,11 @@ tl_status tl_op_gqa_decode(const uint16_t* d_q, const uint16_t* d_k, const uint1
   a.ctx = ctx_stride;
   a.rows = d_rows;
   a.Hkv = n_kv_heads;
-  a.out = reinterpret_cast<__half*>(d_out);
+  a.oh = reinterpret_cast<__half*>(d_out);
   a.ldo = n_q_heads * head_dim;
   a.part = part;
   a.ticket = tick;
-  TL_CUDA(launch_decode_attn(a, B, head_dim, rep, st));
+  TL_CUDA(launch_decode_attn(a, B, head_dim, rep, false, st));
   return TL_OK;
 }
 
@@ -967,7 +994,7 @@ tl_status tl_op_gqa_prefill(const uint16_t* d_q, const uint16_t* d_k, const uint
   if (pos0 + T > ctx_stride) return fail(TL_ERR_INVALID_ARG, "pos0 + T exceeds ctx_stride");
   const int qdim = n_q_heads * head_dim;
   PrefillAttnArgs a{};
-  a.q = reinterpret_cast<const __half*>(d_q);
+  a.qh = reinterpret_cast<const __half*>(d_q);
   a.q_bstride = (long long)T * qdim;
   a.ldq = qdim;
   a.k = reinterpret_cast<const __half*>(d_k);
@@ -977,10 +1004,10 @@ tl_status tl_op_gqa_prefill(const uint16_t* d_q, const uint16_t* d_k, const uint
   a.T = T;
   a.pos0 = pos0;
   a.Hkv = n_kv_heads;
-  a.out = reinterpret_cast<__half*>(d_out);
+  a.oh = reinterpret_cast<__half*>(d_out);
   a.o_bstride = (long long)T * qdim;
   a.ldo = qdim;
-  TL_CUDA(launch_prefill_attn(a, B, head_dim, n_q_heads / n_kv_heads, (cudaStream_t)stream));
+  TL_CUDA(launch_prefill_attn(a, B, head_dim, n_q_heads / n_kv_heads, false, (cudaStream_t)stream));
   return TL_OK;
 }
 
