@@ -268,6 +268,30 @@ tl_status tl_op_gqa_decode(const uint16_t *d_q, const uint16_t *d_k, const uint1
                            int B, int n_q_heads, int n_kv_heads, int head_dim,
                            uint16_t *d_out, void *stream);
 
+/* tl_op_gqa_decode without any allocation.  The pages have no counterpart to
+ * this entry point; it exists for callers that cannot call cudaMalloc, such as
+ * code running inside a stream capture that must not allocate, or a serving
+ * host that plans every device byte up front and owns the allocator.
+ * Same arguments, layout and result as tl_op_gqa_decode, but its scratch (row
+ * descriptors, split-KV partial results and merge tickets) lives in one
+ * fixed 4 MiB device array that every GPU loading this library reserves until
+ * the process exits; nothing is allocated or freed by the call.
+ *   Limits: 1 <= B <= 32, B * n_kv_heads <= 4096, and
+ *   B * n_kv_heads * 32 * (n_q_heads/n_kv_heads) * (head_dim + 2) * 4 bytes
+ *   + 17 KiB <= 4 MiB (e.g. B = 8, 16/4 heads of 128 needs about 2.1 MiB);
+ *   beyond them it returns TL_ERR_UNSUPPORTED and enqueues nothing.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls share the one array and it
+ * keeps the last call's contents (each call re-zeroes what must start at
+ * zero), so calls whose work overlaps on the GPU (different streams without
+ * ordering between them) race and corrupt each other's results: order them on
+ * one stream or with events. */
+tl_status tl_op_gqa_decode_noalloc(const uint16_t *d_q, const uint16_t *d_k, const uint16_t *d_v,
+                                   long long batch_stride, int ctx_stride, const int32_t *h_n_keys,
+                                   int B, int n_q_heads, int n_kv_heads, int head_dim,
+                                   uint16_t *d_out, void *stream);
+
 /* Causal tiled prefill GQA attention (TinyLoop README, "Current Runtime
  * Snapshot", tiled prefill path; tiny-llm feature list, "Tiled Online
  * Softmax", "Causal Masking").  Queries d_q fp16 [B][T][n_q_heads][head_dim]

@@ -31,6 +31,7 @@ __all__ = [
     "tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count", "KERNEL_CLASSES",
     "tl_linear_create", "tl_linear_destroy", "tl_linear_forward",
     "tl_op_rmsnorm", "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill",
+    "tl_op_gqa_decode_noalloc",
     "tl_status_string", "tl_last_error", "tl_version",
     "make_config", "make_weights", "make_int4_linear",
 ]
@@ -96,6 +97,8 @@ def _load():
         "tl_op_gqa_decode": (st, [P, P, P, c_longlong, c_int, P, c_int, c_int, c_int, c_int, P, P]),
         "tl_op_gqa_prefill": (st, [P, P, P, c_longlong, c_int, c_int, c_int, c_int, c_int, c_int,
                                    c_int, P, P]),
+        "tl_op_gqa_decode_noalloc": (st, [P, P, P, c_longlong, c_int, P, c_int, c_int, c_int, c_int,
+                                          P, P]),
         "tl_status_string": (c_char_p, [c_int]),
         "tl_last_error": (c_char_p, []),
         "tl_version": (c_char_p, []),
@@ -128,6 +131,7 @@ EXPORTED = sorted(["tl_model_profile_start", "tl_model_profile_stop", "tl_kernel
                    "tl_score_last", "tl_lane_length", "tl_model_info", "tl_check_device_error",
                    "tl_linear_create", "tl_linear_destroy", "tl_linear_forward", "tl_op_rmsnorm",
                    "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill", "tl_status_string",
+                   "tl_op_gqa_decode_noalloc",
                    "tl_last_error", "tl_version"])
 
 
@@ -310,6 +314,16 @@ def tl_op_gqa_decode(d_q, d_k, d_v, batch_stride, ctx_stride, n_keys, B, n_q_hea
     _check(_L().tl_op_gqa_decode(_ptr(d_q), _ptr(d_k), _ptr(d_v), int(batch_stride), int(ctx_stride),
                                 _i32_host(n_keys), int(B), int(n_q_heads), int(n_kv_heads),
                                 int(head_dim), _ptr(d_out), _stream(stream)))
+
+
+def tl_op_gqa_decode_noalloc(d_q, d_k, d_v, batch_stride, ctx_stride, n_keys, B, n_q_heads,
+                             n_kv_heads, head_dim, d_out, stream=None) -> None:
+    """tl_op_gqa_decode for callers that cannot allocate device memory: the
+    scratch is a fixed 4 MiB array inside the library (see include/tl.h for
+    the limits and the ordering rule).  n_keys is a host sequence of B ints."""
+    _check(_L().tl_op_gqa_decode_noalloc(_ptr(d_q), _ptr(d_k), _ptr(d_v), int(batch_stride),
+                                         int(ctx_stride), _i32_host(n_keys), int(B), int(n_q_heads),
+                                         int(n_kv_heads), int(head_dim), _ptr(d_out), _stream(stream)))
 
 
 def tl_op_gqa_prefill(d_q, d_k, d_v, batch_stride, ctx_stride, T, pos0, B, n_q_heads, n_kv_heads,

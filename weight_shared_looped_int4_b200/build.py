@@ -21,7 +21,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libtl_b200.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-MAIN_SOURCE = os.path.join(CSRC, "tl_api.cu")
+SOURCES = [os.path.join(CSRC, "tl_api.cu"), os.path.join(CSRC, "noalloc.cu")]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -56,7 +56,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not needs_build():
         return LIB_PATH
     tmp = LIB_PATH + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, MAIN_SOURCE]
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-o", tmp, *SOURCES]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), flush=True)

@@ -17,7 +17,6 @@
 #pragma once
 
 #include "common.cuh"
-#include "gemv_int4.cuh"  // RowCtx
 
 namespace tl {
 

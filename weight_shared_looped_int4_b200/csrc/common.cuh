@@ -11,6 +11,13 @@ namespace tl {
 constexpr int kGroup = 128;      // INT4 group size along K
 constexpr int kMaxLanes = 16;    // rows of activations a GEMV launch handles
 
+// Per activation row: which KV-cache lane it reads / writes and at what
+// position.
+struct RowCtx {
+  int lane;
+  int pos;
+};
+
 // ---- programmatic dependent launch -------------------------------------
 // Every kernel of the forward pass calls pdl_trigger() early (so the next
 // kernel may start its weight prefetch) and pdl_wait() before it reads any

@@ -38,12 +38,6 @@ enum GemvIn { IN_NORM = 0, IN_F16 = 1, IN_F32 = 2 };
 enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_ROPE_KV = 3 };
 enum PairMode { PAIR_NEIGHBOUR = 0, PAIR_OFFSET = 1, PAIR_ROPE = 2 };
 
-// Per activation row: which KV-cache lane it writes and at what position.
-struct RowCtx {
-  int lane;
-  int pos;
-};
-
 struct GemvArgs {
   const uint4* w;      // tiled weights  [n_tiles][K/64][32] (see repack)
   const uint2* sz;     // scales / zeros [n_tiles][K/128][8]

@@ -8,6 +8,7 @@
 // that; its keys and values go to cache slice l of the lane.
 
 #include "../../include/tl.h"
+#include "internal.h"
 
 #include <algorithm>
 #include <atomic>
@@ -1027,6 +1028,17 @@ const char* tl_status_string(tl_status s) {
 }
 
 const char* tl_last_error(void) { return g_err.c_str(); }
+
+}  // extern "C"
+
+// Sets the calling thread's last-error text for other translation units of
+// the library (not exported).
+__attribute__((visibility("hidden"))) tl_status tl_internal_set_error(tl_status s, const char* msg) {
+  g_err = msg;
+  return s;
+}
+
+extern "C" {
 
 const char* tl_version(void) { return "0.1.0"; }
 
