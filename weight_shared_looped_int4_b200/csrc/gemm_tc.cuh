@@ -1,0 +1,509 @@
+// INT4 group-wise GEMM on the 5th-generation tensor cores (tcgen05, TMEM)
+// for the prefill linears: Y[t][n] = sum_k X[t][k] * (q[n][k] - z) * s, with
+// groups of 128 along K (TinyLoop README, "Status": INT4 loop / pre linears
+// with zero points; the workload's w = (q - z) * s).
+//
+// Design (ours, sm_100a):
+// * One CTA owns a 128-row weight tile, a 128-token tile and a slice of the K
+//   groups (split-K when the tile grid is smaller than the SM count).
+// * Per K group (128 k) the tensor core computes P = A B^T with A = the exact
+//   fp16 integers q - z of the tile (no scale) and B = the activations split
+//   into an fp16 pair: rows 0..127 of B hold x_hi of the 128 tokens, rows
+//   128..255 hold x_lo (one N = 256 MMA).  P goes to a TMEM buffer; the
+//   epilogue warps read it and accumulate s[n][group] * (P_hi + P_lo) in fp32
+//   registers.  So no weight is rounded and the activation keeps ~22 bits;
+//   fp16 weights or activations move the looped model's logits by ~0.05.
+// * Warp roles (12 warps, 3 per SM sub-partition so each thread may hold 168
+//   registers): warp 0 allocates TMEM and one lane issues tcgen05.mma; warps
+//   1-3 dequantize A from the packed INT4 words straight into the 128-byte
+//   swizzled K-major layout the MMA descriptor reads, and one of them issues
+//   the bulk asynchronous copy of the prepared B tile; warps 4-11 are the
+//   epilogue.  Shared-memory stages and TMEM buffers are double-buffered and
+//   handed over with mbarriers (tcgen05.commit signals MMA completion).
+// * Split-K partials go to a scratch buffer; the last CTA of a tile (atomic
+//   ticket) adds them in split order, so the result is deterministic, and
+//   applies the epilogue: residual add, raw fp32, fp16 store, or RoPE with
+//   the Q output and the K/V cache write.
+// * Every mbarrier wait is bounded; on time-out the kernel records kErrTimeout,
+//   skips the rest of its work and still frees its TMEM.
+#pragma once
+
+#include "common.cuh"
+
+namespace tl {
+
+// ---- tcgen05 wrappers ------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrive on `bar` when all earlier tcgen05 operations of this thread are done.
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 32 consecutive 32-bit columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+// 16 consecutive 32-bit columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// Named barrier among the epilogue warps only.
+__device__ __forceinline__ void epi_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (the canonical layout of a row-major tile whose rows are
+// 128 bytes, written with the 16-byte chunk index XOR (row % 8)).
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(const void* p) {
+  const uint64_t addr = smem_u32(p);
+  uint64_t d = (addr >> 4) & 0x3FFFull;   // start address
+  d |= 1ull << 16;                         // leading byte offset (unused with swizzle)
+  d |= (uint64_t)(1024 >> 4) << 32;        // stride byte offset: 8 rows x 128 B
+  d |= 1ull << 46;                         // descriptor version
+  d |= 2ull << 61;                         // 128-byte swizzle
+  return d;
+}
+// Instruction descriptor of kind::f16: fp16 A and B (K-major), fp32 D.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Byte offset of element pair (row, k..k+1), k even, in a 128-byte-swizzled
+// K-major tile of `rows` rows and 128 k (two 64-wide atoms).
+__host__ __device__ inline uint32_t sw128_offset(int row, int k, int rows) {
+  const int atom = k >> 6, kin = k & 63;
+  const int chunk = kin >> 3, within = (kin & 7) * 2;
+  return (uint32_t)(atom * rows * 128 + row * 128 + ((chunk ^ (row & 7)) << 4) + within);
+}
+
+enum TcEpi { TC_RESID = 0, TC_RAW = 1, TC_STORE = 2, TC_ROPE_KV = 3 };
+
+constexpr int kTcThreads = 384;       // 12 warps
+constexpr int kTcRows = 128;          // weight rows per tile (MMA M)
+constexpr int kTcTokens = 128;        // tokens per tile
+constexpr int kTcEpiThreads = 256;    // warps 4..11
+constexpr int kTcProducers = 96;      // warps 1..3
+
+__host__ __device__ inline int tc_nb(bool lo) { return lo ? 2 * kTcTokens : kTcTokens; }  // B rows (MMA N)
+__host__ __device__ inline size_t tc_a_bytes() { return (size_t)kTcRows * 256; }              // 32 KB
+__host__ __device__ inline size_t tc_b_bytes(bool lo) { return (size_t)tc_nb(lo) * 256; }      // 64 / 32 KB
+__host__ __device__ inline size_t tc_smem_bytes(bool lo) { return 2 * (tc_a_bytes() + tc_b_bytes(lo)) + 1024; }
+
+struct TcGemmArgs {
+  const uint4* w;        // INT4 weights in the GEMV tile layout [n16 tiles][K/64][32] (16 B each)
+  const uint2* sz;       // scales / biased zeros [n16 tiles][K/128][8]
+  int K, N;
+  int n16_tiles;         // 16-row tiles present in w (rows beyond N are zero)
+  const uint8_t* bt;     // prepared activations [token tiles][K/128][2 atoms][NB rows][128 B]
+  int T;                 // tokens
+  int splits;
+  // outputs
+  float* out_f32;        // TC_RESID (+=) / TC_RAW (=): [T][ld_out]
+  __half* out_f16;       // TC_STORE: [T][ld_out]
+  int ld_out;
+  // TC_ROPE_KV
+  float* q_out;          // [T][ldq] rotated queries
+  int ldq;
+  int n_q_rows, n_kv_rows, hd;
+  __half* k_plane;       // K plane [Hkv][ctx][hd] of this lane and layer
+  __half* v_plane;
+  int ctx, pos0;
+  float theta;
+  // split-K
+  float* partial;        // [splits][row tiles][token tiles][128 tokens][128 rows]
+  unsigned* tickets;     // [row tiles][token tiles], zero between launches
+  int* err_flag;
+};
+
+template <int EPI, bool LO>
+__global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGemmArgs a) {
+  constexpr int NB = LO ? 2 * kTcTokens : kTcTokens;
+  constexpr uint32_t NCOL = NB;                    // TMEM columns per buffer
+  constexpr uint32_t A_BYTES = kTcRows * 256;
+  constexpr uint32_t B_BYTES = NB * 256;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  auto sA = [&](int st) { return smem + st * A_BYTES; };
+  auto sB = [&](int st) { return smem + 2 * A_BYTES + st * B_BYTES; };
+  __shared__ __align__(8) uint64_t bar_full[2], bar_empty[2], bar_tfull[2], bar_tempty[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_last;
+  __shared__ int s_fail;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, tt = blockIdx.y, split = blockIdx.z;
+  const int G = a.K >> 7;
+  const int g_begin = split * G / a.splits, g_end = (split + 1) * G / a.splits;
+  const int ng = g_end - g_begin;
+  const int row_tiles = gridDim.x, tok_tiles = gridDim.y;
+
+  if (warp == 0) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar_full[i], kTcProducers);
+      mbar_init(&bar_empty[i], 1);
+      mbar_init(&bar_tfull[i], 1);
+      mbar_init(&bar_tempty[i], kTcEpiThreads);
+    }
+    fence_mbar_init();
+    s_fail = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  pdl_trigger();
+  pdl_wait();
+
+  if (warp == 0) {
+    // ---- MMA issue -------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16_f32(kTcRows, NB);
+      for (int it = 0; it < ng; ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(&bar_full[s], (it >> 1) & 1)) { s_fail = 1; break; }
+        if (it >= 2 && !mbar_wait(&bar_tempty[s], ((it - 2) >> 1) & 1)) { s_fail = 1; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint64_t ad = sw128_kmajor_desc(sA(s) + (j >> 2) * (kTcRows * 128) + (j & 3) * 32);
+          const uint64_t bd = sw128_kmajor_desc(sB(s) + (j >> 2) * (NB * 128) + (j & 3) * 32);
+          tc_mma_f16(tmem + s * NCOL, ad, bd, idesc, j > 0 ? 1u : 0u);
+        }
+        tc_commit(&bar_empty[s]);
+        tc_commit(&bar_tfull[s]);
+      }
+    }
+    __syncwarp();
+  } else if (warp <= 3) {
+    // ---- producers: A dequant (+ B bulk copy by one thread) ------------
+    const int p = threadIdx.x - 32;
+    const int kw = a.K >> 6;  // 64-wide chunks per row
+    for (int it = 0; it < ng; ++it) {
+      const int s = it & 1, g = g_begin + it;
+      if (it >= 2 && !mbar_wait(&bar_empty[s], ((it - 2) >> 1) & 1)) { atomicOr(&s_fail, 1); break; }
+      if (p == 0) {
+        mbar_expect_tx(&bar_full[s], B_BYTES);
+        const uint8_t* src = a.bt + ((size_t)tt * G + g) * B_BYTES;
+        for (uint32_t off = 0; off < B_BYTES; off += 16384)
+          bulk_g2s(sB(s) + off, src + off, 16384, &bar_full[s]);
+      }
+      unsigned char* A = sA(s);
+#pragma unroll
+      for (int i = 0; i < 6; ++i) {
+        const int wi = p + kTcProducers * i;
+        if (wi >= 512) break;
+        const int n16 = wi >> 6, chunk = (wi >> 5) & 1, ln = wi & 31;
+        const int gt = tile * 8 + n16;   // global 16-row tile
+        const int r0 = n16 * 16 + (ln >> 2), t = ln & 3;
+        uint4 wv = make_uint4(0, 0, 0, 0);
+        uint32_t zz = 0x64006400u;  // z = 0 for absent rows (their q are 0 too)
+        if (gt < a.n16_tiles) {
+          wv = ldg_stream(a.w + ((size_t)gt * kw + g * 2 + chunk) * 32 + ln);
+          zz = __ldg(&a.sz[((size_t)gt * G + g) * 8 + (ln >> 2)]).y;
+        }
+        const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t af[4];
+          unpack_a_frag(words[j], zz, af);
+          const int kb = chunk * 64 + j * 16 + 2 * t;
+          *reinterpret_cast<uint32_t*>(A + sw128_offset(r0, kb, kTcRows)) = af[0];
+          *reinterpret_cast<uint32_t*>(A + sw128_offset(r0 + 8, kb, kTcRows)) = af[1];
+          *reinterpret_cast<uint32_t*>(A + sw128_offset(r0, kb + 8, kTcRows)) = af[2];
+          *reinterpret_cast<uint32_t*>(A + sw128_offset(r0 + 8, kb + 8, kTcRows)) = af[3];
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bar_full[s]);
+    }
+  } else {
+    // ---- epilogue: accumulate s * (P_hi + P_lo) per group --------------
+    const int e = warp - 4;
+    const int quad = warp & 3;                 // TMEM lanes this warp may access
+    const int half = e >> 2;                   // tokens [64 half, 64 half + 64)
+    const int row = quad * 32 + lane;          // weight row within the tile
+    const int gt = tile * 8 + (row >> 4);
+    const bool row_ok = gt < a.n16_tiles;
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+    auto scale_of = [&](int g) -> float {
+      if (!row_ok) return 0.f;
+      const uint32_t sp = __ldg(&a.sz[((size_t)gt * G + g) * 8 + (row & 7)]).x;
+      const float2 f = h2_to_f2(sp);
+      return (row & 8) ? f.y : f.x;
+    };
+    float s_next = ng > 0 ? scale_of(g_begin) : 0.f;
+    for (int it = 0; it < ng; ++it) {
+      const int b = it & 1;
+      const float sc = s_next;
+      if (it + 1 < ng) s_next = scale_of(g_begin + it + 1);
+      if (!mbar_wait(&bar_tfull[b], (it >> 1) & 1)) { atomicOr(&s_fail, 1); break; }
+      tc_fence_after();
+      const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + b * NCOL + half * 64;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t hi[16];
+        tmem_ld16(base + c * 16, hi);
+        if (LO) {
+          uint32_t lo[16];
+          tmem_ld16(base + kTcTokens + c * 16, lo);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            acc[c * 16 + i] = fmaf(sc, __uint_as_float(hi[i]) + __uint_as_float(lo[i]), acc[c * 16 + i]);
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[c * 16 + i] = fmaf(sc, __uint_as_float(hi[i]), acc[c * 16 + i]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_tempty[b]);
+    }
+
+    // ---- split-K merge (deterministic) ----------------------------------
+    const int n = tile * kTcRows + row;
+    const int t0 = tt * kTcTokens + half * 64;
+    epi_sync(kTcEpiThreads);
+    const bool failed = s_fail != 0;
+    if (!failed && a.splits > 1) {
+      float* mine = a.partial + (((size_t)split * row_tiles + tile) * tok_tiles + tt) * (kTcTokens * kTcRows);
+#pragma unroll
+      for (int i = 0; i < 64; ++i) mine[(size_t)(half * 64 + i) * kTcRows + row] = acc[i];
+      __threadfence();
+      epi_sync(kTcEpiThreads);
+      if (e == 0 && lane == 0) {
+        unsigned* tk = a.tickets + tile * tok_tiles + tt;
+        s_last = (atomicAdd(tk, 1u) == (unsigned)(a.splits - 1));
+        if (s_last) *tk = 0u;
+      }
+      epi_sync(kTcEpiThreads);
+      if (s_last) {
+        __threadfence();
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+        for (int sp = 0; sp < a.splits; ++sp) {
+          const float* src =
+              a.partial + (((size_t)sp * row_tiles + tile) * tok_tiles + tt) * (kTcTokens * kTcRows);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) acc[i] += __ldcg(src + (size_t)(half * 64 + i) * kTcRows + row);
+        }
+      }
+    } else {
+      if (e == 0 && lane == 0) s_last = 1;
+      epi_sync(kTcEpiThreads);
+    }
+
+    // ---- final epilogue -----------------------------------------------------
+    if (!failed && s_last) {
+      if (EPI == TC_RESID || EPI == TC_RAW || EPI == TC_STORE) {
+        if (n < a.N) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int t = t0 + i;
+            if (t < a.T) {
+              const size_t o = (size_t)t * a.ld_out + n;
+              if (EPI == TC_RESID) a.out_f32[o] += acc[i];
+              else if (EPI == TC_RAW) a.out_f32[o] = acc[i];
+              else a.out_f16[o] = __float2half_rn(acc[i]);
+            }
+          }
+        }
+      } else {
+        // RoPE pairs (j, j + hd/2) sit in different rows of the tile: exchange
+        // through shared memory (the stages are idle now).
+        float* xch = reinterpret_cast<float*>(smem);   // [128 tokens][128 rows]
+#pragma unroll
+        for (int i = 0; i < 64; ++i) xch[(half * 64 + i) * kTcRows + row] = acc[i];
+        epi_sync(kTcEpiThreads);
+        const int hd = a.hd, hh = hd / 2;
+        const int pairs_per_tok = kTcRows / 2;         // 64 (j < hd/2 of each head in the tile)
+        for (int item = threadIdx.x - 4 * 32; item < kTcTokens * pairs_per_tok; item += kTcEpiThreads) {
+          const int tl_ = item / pairs_per_tok, pr = item % pairs_per_tok;
+          const int head_local = pr / hh, j = pr % hh;
+          const int r_a = head_local * hd + j, r_b = r_a + hh;
+          const int t = tt * kTcTokens + tl_;
+          const int na = tile * kTcRows + r_a;
+          if (t >= a.T || na >= a.N) continue;
+          const float va = xch[tl_ * kTcRows + r_a], vb = xch[tl_ * kTcRows + r_b];
+          const int pos = a.pos0 + t;
+          if (na < a.n_q_rows) {
+            const float2 cs = rope_cos_sin(pos, j, hd, a.theta);
+            float* qo = a.q_out + (size_t)t * a.ldq;
+            qo[na] = va * cs.x - vb * cs.y;
+            qo[na + hh] = vb * cs.x + va * cs.y;
+          } else if (na < a.n_q_rows + a.n_kv_rows) {
+            const float2 cs = rope_cos_sin(pos, j, hd, a.theta);
+            const int kvh = (na - a.n_q_rows) / hd;
+            __half* dst = a.k_plane + ((size_t)kvh * a.ctx + pos) * hd;
+            dst[j] = __float2half_rn(va * cs.x - vb * cs.y);
+            dst[j + hh] = __float2half_rn(vb * cs.x + va * cs.y);
+          } else {
+            const int kvh = (na - a.n_q_rows - a.n_kv_rows) / hd;
+            __half* dst = a.v_plane + ((size_t)kvh * a.ctx + pos) * hd;
+            dst[j] = __float2half_rn(va);
+            dst[j + hh] = __float2half_rn(vb);
+          }
+        }
+      }
+    }
+    if (failed && e == 0 && lane == 0) atomicOr(a.err_flag, kErrTimeout);
+  }
+
+  // ---- teardown: every role reaches here; TMEM is always freed -----------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---- activation preparation ---------------------------------------------
+// B tile of token tile tt and K group g: rows 0..127 = fp16 hi of the tokens,
+// rows 128..255 = fp16 lo (when LO), each row 128 k in two 64-wide atoms,
+// 128-byte swizzled; tokens >= T are zero.
+enum PrepMode { PREP_NORM = 0, PREP_F32 = 1, PREP_SWIGLU = 2, PREP_F16 = 3 };
+
+struct PrepArgs {
+  const float* x;        // PREP_NORM / PREP_F32: fp32 [T][ldx]; PREP_SWIGLU: gate_up [T][ldx] (gate | up)
+  const __half* xh;      // PREP_F16: fp16 [T][ldx]
+  int ldx;
+  const __half* gain;    // PREP_NORM
+  float eps;
+  int K, T;
+  int F;                 // PREP_SWIGLU: up columns start at F
+  uint8_t* bt;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(256) prep_b_kernel(const PrepArgs a) {
+  constexpr bool LO = MODE != PREP_F16;
+  constexpr int NB = LO ? 2 * kTcTokens : kTcTokens;
+  __shared__ float s_ss[8];
+  const int tok = blockIdx.x;                    // token index, padded to whole tiles
+  const int tt = tok / kTcTokens, tl_ = tok % kTcTokens;
+  const int G = a.K >> 7;
+  const bool valid = tok < a.T;
+  pdl_trigger();
+  pdl_wait();
+  float rs = 1.f;
+  if (MODE == PREP_NORM && valid) {
+    const float* src = a.x + (size_t)tok * a.ldx;
+    float ss = 0.f;
+    for (int k = threadIdx.x * 4; k < a.K; k += 1024) {
+      const float4 v = *reinterpret_cast<const float4*>(src + k);
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = warp_sum(ss);
+    if ((threadIdx.x & 31) == 0) s_ss[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) tot += s_ss[w];
+    rs = 1.0f / sqrtf(tot / (float)a.K + a.eps);
+  }
+  for (int c8 = threadIdx.x; c8 < a.K / 8; c8 += 256) {
+    const int k = c8 * 8;
+    float v[8];
+    if (!valid) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    } else if (MODE == PREP_F16) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(a.xh + (size_t)tok * a.ldx + k);
+      const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = h2_to_f2(w4[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+      }
+    } else if (MODE == PREP_SWIGLU) {
+      const float* src = a.x + (size_t)tok * a.ldx;
+      const float4 g0 = *reinterpret_cast<const float4*>(src + k), g1 = *reinterpret_cast<const float4*>(src + k + 4);
+      const float4 u0 = *reinterpret_cast<const float4*>(src + a.F + k);
+      const float4 u1 = *reinterpret_cast<const float4*>(src + a.F + k + 4);
+      v[0] = silu(g0.x) * u0.x; v[1] = silu(g0.y) * u0.y; v[2] = silu(g0.z) * u0.z; v[3] = silu(g0.w) * u0.w;
+      v[4] = silu(g1.x) * u1.x; v[5] = silu(g1.y) * u1.y; v[6] = silu(g1.z) * u1.z; v[7] = silu(g1.w) * u1.w;
+    } else {
+      const float* src = a.x + (size_t)tok * a.ldx;
+      const float4 x0 = *reinterpret_cast<const float4*>(src + k), x1 = *reinterpret_cast<const float4*>(src + k + 4);
+      v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+      if (MODE == PREP_NORM) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = (v[i] * rs) * __half2float(a.gain[k + i]);
+      }
+    }
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+      const float2 r = __half22float2(h);
+      const __half2 l = __floats2half2_rn(v[2 * i] - r.x, v[2 * i + 1] - r.y);
+      hw[i] = *reinterpret_cast<const uint32_t*>(&h);
+      lw[i] = *reinterpret_cast<const uint32_t*>(&l);
+    }
+    const int g = k >> 7, kg = k & 127;
+    uint8_t* blk = a.bt + ((size_t)tt * G + g) * (NB * 256);
+    *reinterpret_cast<uint4*>(blk + sw128_offset(tl_, kg, NB)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    if (LO)
+      *reinterpret_cast<uint4*>(blk + sw128_offset(kTcTokens + tl_, kg, NB)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+  }
+}
+
+}  // namespace tl

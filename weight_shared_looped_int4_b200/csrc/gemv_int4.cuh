@@ -13,11 +13,13 @@
 //   so the tensor-core product with the fp16 activation is exact and the MMA
 //   accumulates in fp32.  The fp16 scale is applied in fp32 once per 64-wide
 //   K chunk, so no weight is ever rounded.
-// * Each CTA owns a pair of 16-row tiles (the pair an epilogue needs: RoPE
-//   halves of one head, gate/up rows of SwiGLU, or two neighbours) and all of
-//   K; its 8 warps split (tile, K quarter) and reduce through shared memory in
-//   a fixed order, so results are deterministic and each activation row's
-//   result does not depend on how many rows share the launch.
+// * A CTA owns TPC 16-row tiles and all of K.  With TPC = 2 the two tiles are
+//   the pair an epilogue needs (RoPE halves of one head, gate/up rows of
+//   SwiGLU) and the 8 warps split (tile, K quarter); with TPC = 1 (residual
+//   and plain outputs) the 8 warps split K eight ways, which doubles the CTA
+//   count of the small projections.  Partial sums are reduced through shared
+//   memory in a fixed order, so results are deterministic and each activation
+//   row's result does not depend on how many rows share the launch.
 // * Weight prefetch is issued before griddepcontrol.wait, so it overlaps the
 //   tail of the previous kernel under programmatic dependent launch.
 // * fp32 activations are split into an fp16 pair x = hi + lo (lo is the fp16
@@ -83,28 +85,38 @@ __host__ __device__ inline size_t gemv_act_bytes(int K, int M, bool lo) {
 }
 __host__ __device__ inline size_t gemv_smem_bytes(int K, int M, bool lo) {
   const int nt = M <= 8 ? 1 : 2;
-  return gemv_act_bytes(K, M, lo) + (size_t)4 * 2 * 16 * nt * 8 * 4;
+  return gemv_act_bytes(K, M, lo) + (size_t)8 * 16 * nt * 8 * 4 + 8 * kMaxLanes * 4;
+}
+
+// Tiles per CTA of each epilogue.
+__host__ __device__ constexpr int gemv_tpc(int epi) {
+  return (epi == EPI_ROPE_KV || epi == EPI_SWIGLU) ? 2 : 1;
 }
 
 template <int NT, int IN, int EPI>
-__global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kGemvThreads, 3) gemv_int4_kernel(const GemvArgs a) {
   constexpr bool LO = (IN != IN_F16);
-  extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int TPC = gemv_tpc(EPI);
+  constexpr int KS = 8 / TPC;  // K slices
+  extern __shared__ __align__(128) unsigned char smem[];
   const int K = a.K;
   const int M = a.M;
   const int ldxs = K + 8;
   __half* xs = reinterpret_cast<__half*>(smem);           // hi plane [M][ldxs]
   __half* xl = xs + (size_t)M * ldxs;                     // lo plane [M][ldxs]
-  float* red = reinterpret_cast<float*>(smem + gemv_act_bytes(K, M, LO));
+  constexpr int NC = NT * 8;  // activation columns of the MMA
+  float* red = reinterpret_cast<float*>(smem + gemv_act_bytes(K, M, LO));   // [8][16][NC]
+  float* ssq = red + 8 * 16 * NC;                                           // [16 rows][8 warps]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int tsel = warp & 1, kq = warp >> 1;
+  const int tsel = TPC == 2 ? (warp & 1) : 0;
+  const int kq = TPC == 2 ? (warp >> 1) : warp;
 
   int t0, t1;
-  if (a.pair_mode == PAIR_NEIGHBOUR) {
-    t0 = 2 * blockIdx.x;
-    t1 = t0 + 1;
+  if (TPC == 1) {
+    t0 = blockIdx.x;
+    t1 = t0;
   } else if (a.pair_mode == PAIR_OFFSET) {
     t0 = blockIdx.x;
     t1 = t0 + a.pair_off;
@@ -116,8 +128,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   const int tile = tsel ? t1 : t0;
 
   const int n_chunks = K >> 6;
-  const int c_begin = (n_chunks * kq) >> 2;
-  const int nc = ((n_chunks * (kq + 1)) >> 2) - c_begin;
+  const int c_begin = (n_chunks * kq) / KS;
+  const int nc = (n_chunks * (kq + 1)) / KS - c_begin;
   const uint4* wp = a.w + ((size_t)tile * n_chunks + c_begin) * 32 + lane;
   const uint2* szp = a.sz + (size_t)tile * (K >> 7) * 8 + g;
 
@@ -137,26 +149,40 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
 
   // ---- stage the activations: fp16 pair (hi, lo) of the fp32 input --------
   if (IN == IN_F16) {
-    for (int m = warp; m < M; m += 8) {
+    for (int m = 0; m < M; ++m) {
       __half* dst = xs + m * ldxs;
       const __half* src = a.xh + (size_t)m * a.ldx;
-      for (int k = lane * 8; k < K; k += 256)
+#pragma unroll 4
+      for (int k = threadIdx.x * 8; k < K; k += 8 * kGemvThreads)
         *reinterpret_cast<uint4*>(dst + k) = *reinterpret_cast<const uint4*>(src + k);
     }
   } else {
-    for (int m = warp; m < M; m += 8) {
-      const float* src = a.x + (size_t)m * a.ldx;
-      float rs = 1.f;
-      if (IN == IN_NORM) {
+    // every thread takes float4 columns tid*4 + 1024 i of every row
+    if (IN == IN_NORM) {
+      for (int m = 0; m < M; ++m) {
+        const float* src = a.x + (size_t)m * a.ldx;
         float ss = 0.f;
-        for (int k = lane * 4; k < K; k += 128) {
+#pragma unroll 4
+        for (int k = threadIdx.x * 4; k < K; k += 4 * kGemvThreads) {
           const float4 v = *reinterpret_cast<const float4*>(src + k);
           ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
         }
         ss = warp_sum(ss);
+        if (lane == 0) ssq[m * 8 + warp] = ss;
+      }
+      __syncthreads();
+    }
+    for (int m = 0; m < M; ++m) {
+      const float* src = a.x + (size_t)m * a.ldx;
+      float rs = 1.f;
+      if (IN == IN_NORM) {
+        float ss = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) ss += ssq[m * 8 + w];
         rs = 1.0f / sqrtf(ss / (float)K + a.eps);
       }
-      for (int k = lane * 4; k < K; k += 128) {
+#pragma unroll 4
+      for (int k = threadIdx.x * 4; k < K; k += 4 * kGemvThreads) {
         float4 v = *reinterpret_cast<const float4*>(src + k);
         if (IN == IN_NORM) {
           const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
@@ -236,9 +262,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
     }
   }
 
-  // ---- reduce the four K quarters (fixed order) ---------------------------
-  constexpr int NC = NT * 8;  // activation columns
-  float* myred = red + (kq * 2 + tsel) * 16 * NC;
+  // ---- reduce the K slices (fixed order) ---------------------------------
+  float* myred = red + (kq * TPC + tsel) * 16 * NC;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     const int col = nt * 8 + 2 * t;
@@ -253,18 +278,16 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   if (m >= a.M || m >= NC) return;
   float va = 0.f, vb = 0.f;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    va += red[(q * 2 + 0) * 16 * NC + r * NC + m];
-    vb += red[(q * 2 + 1) * 16 * NC + r * NC + m];
+  for (int q = 0; q < KS; ++q) {
+    va += red[(q * TPC + 0) * 16 * NC + r * NC + m];
+    if (TPC == 2) vb += red[(q * TPC + 1) * 16 * NC + r * NC + m];
   }
   const int row0 = t0 * 16 + r, row1 = t1 * 16 + r;
 
   if (EPI == EPI_STORE) {
     if (row0 < a.n_rows) a.y[(size_t)m * a.ldy + row0] = __float2half_rn(va);
-    if (row1 < a.n_rows) a.y[(size_t)m * a.ldy + row1] = __float2half_rn(vb);
   } else if (EPI == EPI_RESID) {
     if (row0 < a.n_rows) a.resid[(size_t)m * a.ldr + row0] += va;
-    if (row1 < a.n_rows) a.resid[(size_t)m * a.ldr + row1] += vb;
   } else if (EPI == EPI_SWIGLU) {
     a.yf[(size_t)m * a.ldy + row0] = silu(va) * vb;
   } else {  // EPI_ROPE_KV: row0 is element j < hd/2 of a head, row1 = row0 + hd/2

@@ -58,6 +58,19 @@ __global__ void noalloc_setup_kernel(NoAllocRows r, unsigned char* scratch) {
 
 tl_status err(tl_status s, const std::string& m) { return tl_internal_set_error(s, m.c_str()); }
 
+// Allow the attention kernels their dynamic shared memory (once per device,
+// with the scratch address lookup).
+cudaError_t allow_attn_smem() {
+  cudaError_t e = cudaSuccess;
+#define A(HD, REP)                                                                               \
+  if (e == cudaSuccess)                                                                          \
+    e = cudaFuncSetAttribute(decode_attn_kernel<HD, REP, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                             (int)decode_attn_smem_bytes(HD));
+  A(64, 1) A(64, 2) A(64, 4) A(64, 8) A(128, 1) A(128, 2) A(128, 4) A(128, 8)
+#undef A
+  return e;
+}
+
 // Device address of the scratch on the current device (looked up once).
 tl_status scratch_address(void** out) {
   int dev = 0;
@@ -70,6 +83,8 @@ tl_status scratch_address(void** out) {
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p)
       return err(TL_ERR_CUDA, std::string("cudaGetSymbolAddress(scratch): ") + cudaGetErrorString(e));
+    e = allow_attn_smem();
+    if (e != cudaSuccess) return err(TL_ERR_CUDA, std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];
@@ -78,7 +93,7 @@ tl_status scratch_address(void** out) {
 
 template <int HD, int REP>
 cudaError_t launch_attn(const DecodeAttnArgs& a, int rows, cudaStream_t st) {
-  decode_attn_kernel<HD, REP, false><<<dim3(kDecodeMaxSplits, a.Hkv, rows), kDecodeThreads, 0, st>>>(a);
+  decode_attn_kernel<HD, REP, false><<<dim3(kDecodeMaxSplits, a.Hkv, rows), kDecodeThreads, decode_attn_smem_bytes(HD), st>>>(a);
   return cudaGetLastError();
 }
 

@@ -22,6 +22,7 @@
 
 #include "attention.cuh"
 #include "common.cuh"
+#include "gemm_tc.cuh"
 #include "gemv_int4.cuh"
 #include "misc.cuh"
 
@@ -173,6 +174,15 @@ cudaError_t init_device_kernels(int dev) {
 #undef SET
   if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<1>, dev);
   if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<2>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_RESID, true>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_RAW, true>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_ROPE_KV, true>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_STORE, false>, dev);
+#define ATT(HD, REP)                                                                  \
+  if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, true>, dev);   \
+  if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, false>, dev);
+  ATT(64, 1) ATT(64, 2) ATT(64, 4) ATT(64, 8) ATT(128, 1) ATT(128, 2) ATT(128, 4) ATT(128, 8)
+#undef ATT
   if (e == cudaSuccess) g_dev_init[dev] = true;
   return e;
 }
@@ -299,26 +309,47 @@ struct BlockDev {
   size_t bytes(int d) const { return qkv.bytes() + o.bytes() + gate_up.bytes() + down.bytes() + 4 * (size_t)d; }
 };
 
-// Per-step row description, passed by value to a setup kernel (so no host
-// buffer has to outlive the call).
+// Per-step row description, passed by value to the step's first kernel (so
+// no host buffer has to outlive the call).  Rows are the step's lanes in
+// decreasing loop order.
 struct StepDesc {
   int n;
   int lane[kMaxLanes];
   int pos[kMaxLanes];
   int tok_index[kMaxLanes];
   int out_row[kMaxLanes];
+  const int32_t* tokens;
+  float* logits;
+  int32_t* argmax;
 };
 
-__global__ void setup_step_kernel(StepDesc s, RowCtx* rows, int* tok_index, int* out_row) {
+// First kernel of a decode step: publishes the rows' lanes / positions and
+// the output pointers to device memory, then gathers the embeddings.
+__global__ void step_embed_kernel(StepDesc s, const __half* __restrict__ E, int d, int vocab, RowCtx* rows,
+                                  int* out_row, HeadIO* io, float* __restrict__ x, int* err_flag) {
+  const int row = blockIdx.x;
   pdl_trigger();
   pdl_wait();
-  const int i = threadIdx.x;
-  if (i < s.n) {
-    rows[i].lane = s.lane[i];
-    rows[i].pos = s.pos[i];
-    tok_index[i] = s.tok_index[i];
-    out_row[i] = s.out_row[i];
+  if (row == 0) {
+    if (threadIdx.x < s.n) {
+      rows[threadIdx.x].lane = s.lane[threadIdx.x];
+      rows[threadIdx.x].pos = s.pos[threadIdx.x];
+      out_row[threadIdx.x] = s.out_row[threadIdx.x];
+    }
+    if (threadIdx.x == 0) {
+      io->logits = s.logits;
+      io->argmax = s.argmax;
+    }
   }
+  int tok = s.tokens[s.tok_index[row]];
+  if (tok < 0 || tok >= vocab) {
+    if (threadIdx.x == 0) atomicOr(err_flag, kErrToken);
+    tok = 0;
+  }
+  const __half* e = E + (size_t)tok * d;
+  float* xr = x + (size_t)row * d;
+  for (int k = threadIdx.x * 2; k < d; k += blockDim.x * 2)
+    *reinterpret_cast<float2*>(xr + k) = __half22float2(*reinterpret_cast<const __half2*>(e + k));
 }
 
 __global__ void fill_rows_kernel(RowCtx* rows, int n, int lane, int pos0) {
@@ -332,9 +363,65 @@ __global__ void fill_rows_kernel(RowCtx* rows, int n, int lane, int pos0) {
 }
 
 
+// ---- tensor-core INT4 GEMM (prefill / large M) ------------------------------
+struct TcScratch {
+  uint8_t* bt = nullptr;       // prepared activation tiles
+  size_t bt_bytes = 0;
+  float* partial = nullptr;    // split-K partial tiles
+  size_t partial_bytes = 0;
+  unsigned* tickets = nullptr; // >= 4096 entries, zero between launches
+  int* err_flag = nullptr;
+  int n_sm = 148;
+};
+
+constexpr int kTcMinTokens = 32;   // below this the GEMV path is used
+
+size_t tc_bt_bytes(int T, int K, bool lo) {
+  return (size_t)((T + kTcTokens - 1) / kTcTokens) * (K / 128) * tc_b_bytes(lo);
+}
+
+cudaError_t launch_prep(int mode, const PrepArgs& p, cudaStream_t st) {
+  const dim3 g(((p.T + kTcTokens - 1) / kTcTokens) * kTcTokens), b(256);
+  switch (mode) {
+    case PREP_NORM: return launch(prep_b_kernel<PREP_NORM>, g, b, 0, st, p);
+    case PREP_F32: return launch(prep_b_kernel<PREP_F32>, g, b, 0, st, p);
+    case PREP_SWIGLU: return launch(prep_b_kernel<PREP_SWIGLU>, g, b, 0, st, p);
+    case PREP_F16: return launch(prep_b_kernel<PREP_F16>, g, b, 0, st, p);
+  }
+  return cudaErrorInvalidValue;
+}
+
+// Runs prep + GEMM for T tokens.  `ta` carries the epilogue outputs; the
+// weight, activation and scratch fields are filled here.
+cudaError_t launch_tc_linear(const uint4* w, const uint2* sz, int K, int N, int n16_tiles, int prep_mode,
+                             PrepArgs pa, TcGemmArgs ta, int epi, int T, const TcScratch& sc, cudaStream_t st) {
+  const bool lo = prep_mode != PREP_F16;
+  if (tc_bt_bytes(T, K, lo) > sc.bt_bytes) return cudaErrorInvalidValue;
+  pa.K = K;
+  pa.T = T;
+  pa.bt = sc.bt;
+  cudaError_t e = launch_prep(prep_mode, pa, st);
+  if (e != cudaSuccess) return e;
+  const int G = K / 128;
+  const int row_tiles = (N + kTcRows - 1) / kTcRows, tok_tiles = (T + kTcTokens - 1) / kTcTokens;
+  int splits = std::max(1, std::min(G, sc.n_sm / (row_tiles * tok_tiles)));
+  while (splits > 1 && (size_t)splits * row_tiles * tok_tiles * kTcRows * kTcTokens * 4 > sc.partial_bytes) --splits;
+  if (row_tiles * tok_tiles > 4096) return cudaErrorInvalidValue;
+  ta.w = w; ta.sz = sz; ta.K = K; ta.N = N; ta.n16_tiles = n16_tiles;
+  ta.bt = sc.bt; ta.T = T; ta.splits = splits;
+  ta.partial = sc.partial; ta.tickets = sc.tickets; ta.err_flag = sc.err_flag;
+  const dim3 g(row_tiles, tok_tiles, splits), b(kTcThreads);
+  const size_t smem = tc_smem_bytes(lo);
+  if (epi == TC_RESID && lo) return launch(gemm_int4_tc_kernel<TC_RESID, true>, g, b, smem, st, ta);
+  if (epi == TC_RAW && lo) return launch(gemm_int4_tc_kernel<TC_RAW, true>, g, b, smem, st, ta);
+  if (epi == TC_ROPE_KV && lo) return launch(gemm_int4_tc_kernel<TC_ROPE_KV, true>, g, b, smem, st, ta);
+  if (epi == TC_STORE && !lo) return launch(gemm_int4_tc_kernel<TC_STORE, false>, g, b, smem, st, ta);
+  return cudaErrorInvalidValue;
+}
+
 template <int HD, int REP, bool F32>
 cudaError_t launch_decode_attn_t(const DecodeAttnArgs& a, int rows, cudaStream_t st) {
-  return launch(decode_attn_kernel<HD, REP, F32>, dim3(kDecodeMaxSplits, a.Hkv, rows), dim3(kDecodeThreads), 0,
+  return launch(decode_attn_kernel<HD, REP, F32>, dim3(kDecodeMaxSplits, a.Hkv, rows), dim3(kDecodeThreads), decode_attn_smem_bytes(HD),
                 st, a);
 }
 
@@ -390,7 +477,16 @@ struct tl_model {
   int* head_idx = nullptr;
   int* err_flag = nullptr;
   int head_grid = 0;
+  HeadIO* io = nullptr;          // output pointers of the current decode step
+  TcScratch tc;                  // tensor-core GEMM scratch (prefill)
+  float* gu = nullptr;           // raw gate_up output of the prefill [rows][2F]
   cudaStream_t setup_stream = nullptr;
+  cudaStream_t cap_stream = nullptr;   // stream used to capture decode graphs
+  struct Graph {
+    cudaGraphExec_t exec = nullptr;
+    int kernels = 0;
+  };
+  std::map<std::string, Graph> graphs;   // decode step graphs by row pattern
   std::vector<int> lane_len, lane_loops;
   size_t weight_bytes = 0, kv_bytes = 0, ws_bytes = 0;
   Profiler prof;
@@ -404,8 +500,12 @@ struct tl_model {
   void free_all() {
     for (auto& b : pre) b.free_all();
     loop.free_all();
+    for (auto& kv_ : graphs)
+      if (kv_.second.exec) cudaGraphExecDestroy(kv_.second.exec);
+    graphs.clear();
+    if (cap_stream) cudaStreamDestroy(cap_stream);
     void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row,
-                    attn_part, tickets, head_val, head_idx, err_flag};
+                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.partial, tc.tickets, gu};
     for (void* p : ptrs)
       if (p) cudaFree(p);
     if (setup_stream) cudaStreamDestroy(setup_stream);
@@ -501,7 +601,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   a.pair_mode = PAIR_NEIGHBOUR;
   a.resid = x; a.ldr = d;
   kclass(TL_KERNEL_O_PROJ);
-  TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, b.o.n_tiles / 2, st));
+  TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, (b.o.N + 15) / 16, st));
   GemvArgs g{};
   g.eps = c.rms_eps;
   g.w = b.gate_up.w; g.sz = b.gate_up.sz; g.K = d; g.n_rows = 2 * F;
@@ -516,18 +616,70 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   dn.pair_mode = PAIR_NEIGHBOUR;
   dn.resid = x; dn.ldr = d;
   kclass(TL_KERNEL_DOWN);
-  TL_CUDA(launch_gemv_rows(dn, M, IN_F32, EPI_RESID, b.down.n_tiles / 2, st));
+  TL_CUDA(launch_gemv_rows(dn, M, IN_F32, EPI_RESID, (b.down.N + 15) / 16, st));
+  return TL_OK;
+}
+
+// Prefill forms of run_qkv / run_ffn on the tensor cores (positions 0..T-1 of
+// one lane).
+tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  const BlockDev& b = m->block(layer);
+  const int hd = c.head_dim, qdim = c.n_q_heads * hd;
+  PrepArgs pa{};
+  pa.x = m->x; pa.ldx = c.d_model; pa.gain = b.attn_norm; pa.eps = c.rms_eps;
+  TcGemmArgs ta{};
+  ta.q_out = m->q; ta.ldq = qdim; ta.n_q_rows = qdim; ta.n_kv_rows = c.n_kv_heads * hd; ta.hd = hd;
+  ta.k_plane = m->k_plane(layer) + lane * m->lane_stride;
+  ta.v_plane = m->v_plane(layer) + lane * m->lane_stride;
+  ta.ctx = c.max_ctx; ta.pos0 = 0; ta.theta = c.rope_theta;
+  kclass(TL_KERNEL_GEMM_TC);
+  TL_CUDA(launch_tc_linear(b.qkv.w, b.qkv.sz, c.d_model, b.qkv.N, b.qkv.n_tiles, PREP_NORM, pa, ta, TC_ROPE_KV,
+                           T, m->tc, st));
+  return TL_OK;
+}
+
+tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  const BlockDev& b = m->block(layer);
+  const int d = c.d_model, F = c.ffn_dim, qdim = c.n_q_heads * c.head_dim;
+  kclass(TL_KERNEL_GEMM_TC);
+  {  // O projection + residual
+    PrepArgs pa{};
+    pa.x = m->o; pa.ldx = qdim;
+    TcGemmArgs ta{};
+    ta.out_f32 = m->x; ta.ld_out = d;
+    TL_CUDA(launch_tc_linear(b.o.w, b.o.sz, qdim, d, b.o.n_tiles, PREP_F32, pa, ta, TC_RESID, T, m->tc, st));
+  }
+  {  // RMSNorm + gate_up (raw)
+    PrepArgs pa{};
+    pa.x = m->x; pa.ldx = d; pa.gain = b.ffn_norm; pa.eps = c.rms_eps;
+    TcGemmArgs ta{};
+    ta.out_f32 = m->gu; ta.ld_out = 2 * F;
+    TL_CUDA(launch_tc_linear(b.gate_up.w, b.gate_up.sz, d, 2 * F, b.gate_up.n_tiles, PREP_NORM, pa, ta, TC_RAW, T,
+                             m->tc, st));
+  }
+  {  // SwiGLU + down + residual
+    PrepArgs pa{};
+    pa.x = m->gu; pa.ldx = 2 * F; pa.F = F;
+    TcGemmArgs ta{};
+    ta.out_f32 = m->x; ta.ld_out = d;
+    TL_CUDA(launch_tc_linear(b.down.w, b.down.sz, F, d, b.down.n_tiles, PREP_SWIGLU, pa, ta, TC_RESID, T, m->tc,
+                             st));
+  }
   return TL_OK;
 }
 
 tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, float* logits,
-                      int32_t* argmax, cudaStream_t st) {
+                      int32_t* argmax, cudaStream_t st, const HeadIO* io = nullptr) {
   const tl_config& c = m->cfg;
   HeadArgs ha{};
+  ha.io = io;
   ha.w = m->head_w; ha.V = c.vocab; ha.d = c.d_model;
   ha.x = x; ha.gain = m->out_norm; ha.eps = c.rms_eps; ha.M = M;
   ha.out_row = out_row; ha.logits = logits; ha.argmax = argmax;
   ha.part_val = m->head_val; ha.part_idx = m->head_idx; ha.ticket = m->head_ticket();
+  ha.err_flag = m->err_flag;
   const int nt = M <= 8 ? 1 : 2;
   const size_t smem = head_smem_bytes(c.d_model, M);
   kclass(TL_KERNEL_HEAD);
@@ -547,8 +699,9 @@ tl_status forward_prompt(tl_model* m, int lane, const int32_t* d_tokens, int T, 
   kclass(TL_KERNEL_EMBED);
   TL_CUDA(launch(embed_kernel, dim3(T), dim3(256), 0, st, (const __half*)m->embed, d, c.vocab,
                  d_tokens, (const int*)nullptr, m->x, m->err_flag));
+  const bool tc = T >= kTcMinTokens;
   for (int layer = 0; layer < n_layers; ++layer) {
-    tl_status rc = run_qkv(m, layer, T, m->x, m->rows, m->q, st);
+    tl_status rc = tc ? run_qkv_tc(m, layer, lane, T, st) : run_qkv(m, layer, T, m->x, m->rows, m->q, st);
     if (rc != TL_OK) return rc;
     PrefillAttnArgs pa{};
     pa.qf = m->q; pa.q_bstride = 0; pa.ldq = qdim;
@@ -559,7 +712,7 @@ tl_status forward_prompt(tl_model* m, int lane, const int32_t* d_tokens, int T, 
     pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
     kclass(TL_KERNEL_ATTN_PREFILL);
     TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
-    rc = run_ffn(m, layer, T, m->x, m->o, m->h, st);
+    rc = tc ? run_ffn_tc(m, layer, T, st) : run_ffn(m, layer, T, m->x, m->o, m->h, st);
     if (rc != TL_OK) return rc;
   }
   if (d_logits || d_argmax)
@@ -596,7 +749,8 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     delete m;
     return s;
   };
-  if (cudaStreamCreateWithFlags(&m->setup_stream, cudaStreamNonBlocking) != cudaSuccess)
+  if (cudaStreamCreateWithFlags(&m->setup_stream, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess)
     return bail(fail(TL_ERR_CUDA, "stream create failed"));
   cudaStream_t st = m->setup_stream;
 
@@ -632,7 +786,13 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
   // workspaces
   const int rows = std::max(c.max_ctx, kMaxLanes);
   const int rep = c.n_q_heads / c.n_kv_heads;
-  m->head_grid = (c.vocab / 16 + 7) / 8;
+  {
+    int n_sm = 0;
+    if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n_sm < 1) n_sm = 148;
+    // one CTA of 8 warps per SM, never more warps than head tiles
+    m->head_grid = std::min(n_sm, (c.vocab / 16 + 7) / 8);
+    m->tc.n_sm = n_sm;
+  }
   size_t ws = 0;
   auto alloc = [&](void** p, size_t bytes) -> bool {
     ws += bytes;
@@ -646,7 +806,18 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
             alloc((void**)&m->attn_part, (size_t)kMaxLanes * c.n_kv_heads * kDecodeMaxSplits * rep * (hd + 2) * 4) &&
             alloc((void**)&m->tickets, (size_t)(kMaxLanes * c.n_kv_heads + 1) * 4) &&
             alloc((void**)&m->head_val, (size_t)m->head_grid * 16 * 4) &&
-            alloc((void**)&m->head_idx, (size_t)m->head_grid * 16 * 4) && alloc((void**)&m->err_flag, 4);
+            alloc((void**)&m->head_idx, (size_t)m->head_grid * 16 * 4) && alloc((void**)&m->err_flag, 4) &&
+            alloc((void**)&m->io, sizeof(HeadIO));
+  if (ok) {
+    const int kmax = std::max(std::max(d, qdim), c.ffn_dim);
+    const int tok_pad = ((rows + kTcTokens - 1) / kTcTokens) * kTcTokens;
+    m->tc.bt_bytes = tc_bt_bytes(rows, kmax, true);
+    m->tc.partial_bytes = (size_t)160 * kTcRows * kTcTokens * 4;
+    m->tc.err_flag = m->err_flag;
+    ok = alloc((void**)&m->tc.bt, m->tc.bt_bytes) && alloc((void**)&m->tc.partial, m->tc.partial_bytes) &&
+         alloc((void**)&m->tc.tickets, 4096 * sizeof(unsigned)) &&
+         alloc((void**)&m->gu, (size_t)tok_pad * 2 * c.ffn_dim * 4);
+  }
   if (!ok) return bail(fail(TL_ERR_OOM, "workspace allocation"));
   m->ws_bytes = ws;
   if (cudaStreamSynchronize(st) != cudaSuccess) return bail(fail(TL_ERR_CUDA, "setup sync"));
@@ -730,31 +901,66 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
     sd.tok_index[s] = i;
     sd.out_row[s] = i;
   }
+  sd.tokens = d_tokens;
+  sd.logits = d_logits;
+  sd.argmax = d_argmax;
   DeviceGuard guard(m->device);
   if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
   cudaStream_t st = (cudaStream_t)stream;
-  const int d = c.d_model, qdim = c.n_q_heads * c.head_dim;
   ProfScope prof_scope(&m->prof);
-  kclass(TL_KERNEL_SETUP);
-  TL_CUDA(launch(setup_step_kernel, dim3(1), dim3(32), 0, st, sd, m->rows, m->tok_index, m->out_row));
   kclass(TL_KERNEL_EMBED);
-  TL_CUDA(launch(embed_kernel, dim3(n_lanes), dim3(256), 0, st, (const __half*)m->embed, d, c.vocab, d_tokens,
-                 (const int*)m->tok_index, m->x, m->err_flag));
+  TL_CUDA(launch(step_embed_kernel, dim3(n_lanes), dim3(256), 0, st, sd, (const __half*)m->embed, c.d_model,
+                 c.vocab, m->rows, m->out_row, m->io, m->x, m->err_flag));
+  // rows still running at each effective layer
   const int max_layers = c.n_pre + h_loops[order[0]];
+  std::vector<int> active(max_layers);
   for (int layer = 0; layer < max_layers; ++layer) {
     int M = 0;
     while (M < n_lanes && c.n_pre + h_loops[order[M]] > layer) ++M;
-    tl_status rc = run_qkv(m, layer, M, m->x, m->rows, m->q, st);
-    if (rc == TL_OK) rc = run_decode_attn(m, layer, M, m->rows, m->q, m->o, st);
-    if (rc == TL_OK) rc = run_ffn(m, layer, M, m->x, m->o, m->h, st);
-    if (rc != TL_OK) return rc;
+    active[layer] = M;
   }
-  if (d_logits || d_argmax) {
-    tl_status rc = launch_head(m, m->x, n_lanes, m->out_row, d_logits, d_argmax, st);
+  auto body = [&](cudaStream_t s) -> tl_status {
+    for (int layer = 0; layer < max_layers; ++layer) {
+      const int M = active[layer];
+      tl_status rc = run_qkv(m, layer, M, m->x, m->rows, m->q, s);
+      if (rc == TL_OK) rc = run_decode_attn(m, layer, M, m->rows, m->q, m->o, s);
+      if (rc == TL_OK) rc = run_ffn(m, layer, M, m->x, m->o, m->h, s);
+      if (rc != TL_OK) return rc;
+    }
+    return launch_head(m, m->x, n_lanes, m->out_row, nullptr, nullptr, s, m->io);
+  };
+  if (m->prof.mask) {  // profiling times every launch: run eagerly
+    tl_status rc = body(st);
     if (rc != TL_OK) return rc;
+  } else {
+    std::string key = std::to_string(n_lanes);
+    for (int a : active) key += "," + std::to_string(a);
+    auto it = m->graphs.find(key);
+    if (it == m->graphs.end()) {
+      // capture the layers and the head once for this row pattern
+      tl_model::Graph gr;
+      const unsigned long long before = g_launches.load();
+      Profiler* saved = g_prof;
+      g_prof = nullptr;
+      cudaError_t e = cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal);
+      if (e != cudaSuccess) { g_prof = saved; return cuda_fail(e, "cudaStreamBeginCapture"); }
+      tl_status rc = body(m->cap_stream);
+      cudaGraph_t graph = nullptr;
+      e = cudaStreamEndCapture(m->cap_stream, &graph);
+      g_prof = saved;
+      gr.kernels = (int)(g_launches.load() - before);
+      g_launches.fetch_sub(gr.kernels);   // counted when the graph runs
+      if (rc != TL_OK) { if (graph) cudaGraphDestroy(graph); return rc; }
+      if (e != cudaSuccess) { if (graph) cudaGraphDestroy(graph); return cuda_fail(e, "cudaStreamEndCapture"); }
+      e = cudaGraphInstantiate(&gr.exec, graph, 0);
+      cudaGraphDestroy(graph);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGraphInstantiate");
+      it = m->graphs.emplace(key, gr).first;
+    }
+    TL_CUDA(cudaGraphLaunch(it->second.exec, st));
+    g_launches.fetch_add(it->second.kernels);
   }
   for (int i = 0; i < n_lanes; ++i) m->lane_len[h_lane_ids[i]] += 1;
-  (void)qdim;
   return TL_OK;
 }
 
@@ -811,6 +1017,7 @@ tl_status tl_check_device_error(tl_model* m, void* stream) {
   TL_CUDA(cudaMemcpy(&flag, m->err_flag, 4, cudaMemcpyDeviceToHost));
   if (flag) {
     TL_CUDA(cudaMemset(m->err_flag, 0, 4));
+    if (flag & kErrTimeout) return fail(TL_ERR_DEVICE_FLAG, "a kernel's bounded wait gave up (results invalid)");
     return fail(TL_ERR_DEVICE_FLAG, "a token id outside [0, vocab) was replaced by 0");
   }
   return TL_OK;
@@ -838,6 +1045,18 @@ struct OpWorkspace {
 };
 std::mutex g_ws_mu;
 std::map<int, OpWorkspace> g_ws;
+
+// A zeroed per-device fault flag for the op entry points.
+std::map<int, int*> g_op_err;
+int* op_err_flag(int dev) {
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  int*& f = g_op_err[dev];
+  if (!f) {
+    if (cudaMalloc(&f, sizeof(int)) != cudaSuccess) { f = nullptr; return nullptr; }
+    if (cudaMemset(f, 0, sizeof(int)) != cudaSuccess) return nullptr;
+  }
+  return f;
+}
 
 // Scratch of at least `bytes` (contents undefined) and the ticket array.
 // Growing the scratch synchronises the device.
@@ -902,19 +1121,45 @@ void tl_linear_destroy(tl_linear* l) {
 tl_status tl_linear_forward(tl_linear* l, const uint16_t* d_x, int M, uint16_t* d_y, int path, void* stream) {
   if (!l || !d_x || !d_y) return fail(TL_ERR_INVALID_ARG, "null argument");
   if (M < 1) return fail(TL_ERR_INVALID_ARG, "M must be >= 1");
-  if (path == TL_PATH_AUTO) path = TL_PATH_GEMV;
-  if (path == TL_PATH_TC) return fail(TL_ERR_UNSUPPORTED, "tensor-core path not built");
-  if (path != TL_PATH_GEMV) return fail(TL_ERR_INVALID_ARG, "unknown path %d", path);
+  if (path == TL_PATH_AUTO) path = M <= kMaxLanes ? TL_PATH_GEMV : TL_PATH_TC;
+  if (path != TL_PATH_GEMV && path != TL_PATH_TC) return fail(TL_ERR_INVALID_ARG, "unknown path %d", path);
   DeviceGuard guard(l->device);
   if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
   const int K = l->w.K, N = l->w.N;
+  if (path == TL_PATH_TC) {
+    if ((N + kTcRows - 1) / kTcRows * ((M + kTcTokens - 1) / kTcTokens) > 4096)
+      return fail(TL_ERR_UNSUPPORTED, "too many tiles for the tensor-core path");
+    TcScratch sc;
+    const size_t bt = tc_bt_bytes(M, K, false), part = (size_t)160 * kTcRows * kTcTokens * 4;
+    void* ws = nullptr;
+    unsigned* tick = nullptr;
+    tl_status rc = op_workspace(l->device, bt + part + 256, &ws, &tick);
+    if (rc != TL_OK) return rc;
+    sc.bt = (uint8_t*)ws;
+    sc.bt_bytes = bt;
+    sc.partial = (float*)((char*)ws + ((bt + 255) / 256) * 256);
+    sc.partial_bytes = part;
+    sc.tickets = tick + kOpTickets / 2;    // the second half of the op tickets
+    sc.err_flag = op_err_flag(l->device);
+    if (!sc.err_flag) return fail(TL_ERR_OOM, "op error flag");
+    int n_sm = 148;
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, l->device);
+    sc.n_sm = n_sm;
+    PrepArgs pa{};
+    pa.xh = reinterpret_cast<const __half*>(d_x); pa.ldx = K;
+    TcGemmArgs ta{};
+    ta.out_f16 = reinterpret_cast<__half*>(d_y); ta.ld_out = N;
+    TL_CUDA(launch_tc_linear(l->w.w, l->w.sz, K, N, l->w.n_tiles, PREP_F16, pa, ta, TC_STORE, M, sc,
+                             (cudaStream_t)stream));
+    return TL_OK;
+  }
   if (gemv_rows_per_launch(K, false) < 1) return fail(TL_ERR_UNSUPPORTED, "K too large for the GEMV");
   GemvArgs a{};
   a.w = l->w.w; a.sz = l->w.sz; a.K = K; a.n_rows = N;
   a.xh = reinterpret_cast<const __half*>(d_x); a.ldx = K;
   a.pair_mode = PAIR_NEIGHBOUR;
   a.y = reinterpret_cast<__half*>(d_y); a.ldy = N;
-  TL_CUDA(launch_gemv_rows(a, M, IN_F16, EPI_STORE, l->w.n_tiles / 2, (cudaStream_t)stream));
+  TL_CUDA(launch_gemv_rows(a, M, IN_F16, EPI_STORE, (N + 15) / 16, (cudaStream_t)stream));
   return TL_OK;
 }
 
@@ -955,6 +1200,7 @@ tl_status tl_op_gqa_decode(const uint16_t* d_q, const uint16_t* d_k, const uint1
   }
   int dev = 0;
   TL_CUDA(cudaGetDevice(&dev));
+  TL_CUDA(init_device_kernels(dev));
   const int rep = n_q_heads / n_kv_heads;
   const size_t rows_b = (size_t)B * sizeof(RowCtx);
   const size_t part_b = (size_t)B * n_kv_heads * kDecodeMaxSplits * rep * (head_dim + 2) * 4;
