@@ -270,7 +270,6 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   if (threadIdx.x == 0) a.ticket[row * a.Hkv + kvh] = 0u;
 }
 
-// ---- prefill (v1: one warp per query head, online softmax) ----------------
 struct PrefillAttnArgs {
   const float* qf;        // [B][T][Hq*hd] fp32 (model), or
   const __half* qh;       // fp16 (op API)
@@ -287,6 +286,204 @@ struct PrefillAttnArgs {
   long long o_bstride;
   int ldo;
 };
+
+// ---- prefill: tiled, tensor cores (m16n8k16), online softmax --------------
+// One CTA per (16-query tile, kv head, batch entry); warp w handles q head
+// kv_head * REP + w for the 16 queries, so each K/V block staged in shared
+// memory serves all REP heads of the group.  S = Q K^T and O += P V run on the
+// tensor cores; Q and P are split into fp16 pairs (hi, lo) and both halves are
+// multiplied (K and V are fp16 already), so the result keeps ~fp32 accuracy.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((unsigned)__cvta_generic_to_shared(p)));
+}
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// (hi, lo) fp16 pairs of two floats.
+__device__ __forceinline__ void split_h2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 r = __half22float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_h2(a - r.x, b - r.y);
+}
+
+constexpr int kPfKeys = 64;   // keys per staged block
+constexpr int kPfPad = 8;     // fp16 padding per staged row
+
+__host__ __device__ inline size_t prefill_attn_smem_bytes(int hd) {
+  return (size_t)2 * kPfKeys * (hd + kPfPad) * 2;
+}
+
+template <int HD, int REP, bool F32>
+__global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const PrefillAttnArgs a) {
+  constexpr int KC = HD / 16;        // k16 chunks of a head
+  constexpr int NT = HD / 8;         // n8 tiles of the output
+  constexpr int LD = HD + kPfPad;
+  constexpr int NTHR = REP * 32;
+  extern __shared__ __align__(128) unsigned char psm[];
+  __half* ks = reinterpret_cast<__half*>(psm);             // [64][LD]
+  __half* vs = ks + kPfKeys * LD;                          // [64][LD]
+
+  const int qt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int h = kvh * REP + warp;
+  const int q0 = qt * 16;
+  pdl_trigger();
+  pdl_wait();
+
+  // Q fragments (hi, lo) of rows q0+g and q0+g+8, scaled by 1/sqrt(hd)
+  const float scale = 1.0f / sqrtf((float)HD);
+  uint32_t qa[KC][4], ql[KC][4];
+  {
+    const int r0 = min(q0 + g, a.T - 1), r1 = min(q0 + g + 8, a.T - 1);
+    const size_t base0 = b * a.q_bstride + (size_t)r0 * a.ldq + (size_t)h * HD;
+    const size_t base1 = b * a.q_bstride + (size_t)r1 * a.ldq + (size_t)h * HD;
+    auto ld2 = [&](size_t off) -> float2 {
+      if (F32) return *reinterpret_cast<const float2*>(a.qf + off);
+      return __half22float2(*reinterpret_cast<const __half2*>(a.qh + off));
+    };
+#pragma unroll
+    for (int c = 0; c < KC; ++c) {
+      const int d0 = c * 16 + 2 * t;
+      float2 v;
+      v = ld2(base0 + d0);     split_h2(v.x * scale, v.y * scale, qa[c][0], ql[c][0]);
+      v = ld2(base1 + d0);     split_h2(v.x * scale, v.y * scale, qa[c][1], ql[c][1]);
+      v = ld2(base0 + d0 + 8); split_h2(v.x * scale, v.y * scale, qa[c][2], ql[c][2]);
+      v = ld2(base1 + d0 + 8); split_h2(v.x * scale, v.y * scale, qa[c][3], ql[c][3]);
+    }
+  }
+
+  float o[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[n][i] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const int pq0 = a.pos0 + q0 + g, pq1 = pq0 + 8;   // query positions of this thread's rows
+  const int last_key = a.pos0 + min(q0 + 15, a.T - 1);
+  const int nblk = last_key / kPfKeys + 1;
+  const __half* kp = a.k + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
+  const __half* vp = a.v + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
+
+  for (int kb = 0; kb < nblk; ++kb) {
+    const int j0 = kb * kPfKeys;
+    __syncthreads();  // the previous block is no longer read
+    for (int c = threadIdx.x; c < kPfKeys * HD / 8; c += NTHR) {
+      const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
+      const bool ok = j0 + key <= last_key;
+      const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
+      cp_async16(ks + key * LD + off, kp + src, ok ? 16 : 0);
+      cp_async16(vs + key * LD + off, vp + src, ok ? 16 : 0);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+
+    // S = Q K^T for 64 keys: 8 n8 tiles
+    float sc[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sc[n][i] = 0.f;
+#pragma unroll
+      for (int c = 0; c < KC; ++c) {
+        const __half* kr = ks + (n * 8 + g) * LD + c * 16 + 2 * t;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 8);
+        mma_f16_16816(sc[n], qa[c], b0, b1);
+        mma_f16_16816(sc[n], ql[c], b0, b1);
+      }
+    }
+    // causal mask and online softmax (rows g and g+8 of the tile)
+    float mx0 = m0, mx1 = m1;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      const int key = j0 + n * 8 + 2 * t;
+      if (key > pq0) sc[n][0] = -INFINITY;
+      if (key + 1 > pq0) sc[n][1] = -INFINITY;
+      if (key > pq1) sc[n][2] = -INFINITY;
+      if (key + 1 > pq1) sc[n][3] = -INFINITY;
+      mx0 = fmaxf(mx0, fmaxf(sc[n][0], sc[n][1]));
+      mx1 = fmaxf(mx1, fmaxf(sc[n][2], sc[n][3]));
+    }
+#pragma unroll
+    for (int o_ = 1; o_ < 4; o_ <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o_));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o_));
+    }
+    const float c0 = (m0 == -INFINITY) ? 0.f : expf(m0 - mx0);
+    const float c1 = (m1 == -INFINITY) ? 0.f : expf(m1 - mx1);
+    m0 = mx0;
+    m1 = mx1;
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      sc[n][0] = (mx0 == -INFINITY) ? 0.f : expf(sc[n][0] - mx0);
+      sc[n][1] = (mx0 == -INFINITY) ? 0.f : expf(sc[n][1] - mx0);
+      sc[n][2] = (mx1 == -INFINITY) ? 0.f : expf(sc[n][2] - mx1);
+      sc[n][3] = (mx1 == -INFINITY) ? 0.f : expf(sc[n][3] - mx1);
+      s0 += sc[n][0] + sc[n][1];
+      s1 += sc[n][2] + sc[n][3];
+    }
+#pragma unroll
+    for (int o_ = 1; o_ < 4; o_ <<= 1) {
+      s0 += __shfl_xor_sync(0xffffffffu, s0, o_);
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o_);
+    }
+    l0 = l0 * c0 + s0;
+    l1 = l1 * c1 + s1;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      o[n][0] *= c0; o[n][1] *= c0;
+      o[n][2] *= c1; o[n][3] *= c1;
+    }
+    // O += P V: P as A fragments (hi, lo) straight from the S accumulators
+#pragma unroll
+    for (int kc = 0; kc < 4; ++kc) {
+      uint32_t pa[4], pl[4];
+      split_h2(sc[2 * kc][0], sc[2 * kc][1], pa[0], pl[0]);
+      split_h2(sc[2 * kc][2], sc[2 * kc][3], pa[1], pl[1]);
+      split_h2(sc[2 * kc + 1][0], sc[2 * kc + 1][1], pa[2], pl[2]);
+      split_h2(sc[2 * kc + 1][2], sc[2 * kc + 1][3], pa[3], pl[3]);
+#pragma unroll
+      for (int n2 = 0; n2 < NT / 2; ++n2) {
+        // V rows kc*16 .. +15, dims n2*16 .. +15 -> B fragments of two n8 tiles
+        const int key = kc * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int dim = n2 * 16 + (lane >> 4) * 8;
+        uint32_t vb[4];
+        ldmatrix_x4_trans(vb, vs + key * LD + dim);
+        mma_f16_16816(o[2 * n2], pa, vb[0], vb[1]);
+        mma_f16_16816(o[2 * n2], pl, vb[0], vb[1]);
+        mma_f16_16816(o[2 * n2 + 1], pa, vb[2], vb[3]);
+        mma_f16_16816(o[2 * n2 + 1], pl, vb[2], vb[3]);
+      }
+    }
+  }
+
+  // normalise and store rows q0+g, q0+g+8
+  const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+  const int r0 = q0 + g, r1 = q0 + g + 8;
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    const int d = n * 8 + 2 * t;
+    if (r0 < a.T) {
+      const size_t off = b * a.o_bstride + (size_t)r0 * a.ldo + (size_t)h * HD + d;
+      if (F32) { a.of[off] = o[n][0] * inv0; a.of[off + 1] = o[n][1] * inv0; }
+      else *reinterpret_cast<uint32_t*>(a.oh + off) = pack_h2(o[n][0] * inv0, o[n][1] * inv0);
+    }
+    if (r1 < a.T) {
+      const size_t off = b * a.o_bstride + (size_t)r1 * a.ldo + (size_t)h * HD + d;
+      if (F32) { a.of[off] = o[n][2] * inv1; a.of[off + 1] = o[n][3] * inv1; }
+      else *reinterpret_cast<uint32_t*>(a.oh + off) = pack_h2(o[n][2] * inv1, o[n][3] * inv1);
+    }
+  }
+}
+
+// ---- prefill (v1: one warp per query head, online softmax) ----------------
 
 template <int HD, int REP, bool F32>
 __global__ void __launch_bounds__(REP * 32) prefill_attn_simple_kernel(const PrefillAttnArgs a) {

@@ -88,6 +88,9 @@ struct Profiler {
 
 thread_local Profiler* g_prof = nullptr;  // profiler of the model in the current call
 thread_local int g_cls = -1;              // class of the next launch
+// L2 access-policy window of the next launches (the loop block's weights while
+// a loop iteration runs; num_bytes == 0 means none).
+thread_local cudaAccessPolicyWindow g_window = {};
 std::atomic<unsigned long long> g_launches{0};
 
 struct ProfScope {  // installs a model's profiler for the duration of one API call
@@ -122,11 +125,16 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (g_window.num_bytes) {
+    attr[1].id = cudaLaunchAttributeAccessPolicyWindow;
+    attr[1].val.accessPolicyWindow = g_window;
+    cfg.numAttrs = 2;
+  }
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
   if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
   if (timed) {
@@ -180,7 +188,9 @@ cudaError_t init_device_kernels(int dev) {
   if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_STORE, false>, dev);
 #define ATT(HD, REP)                                                                  \
   if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, true>, dev);   \
-  if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, false>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, false>, dev);  \
+  if (e == cudaSuccess) e = allow_max_smem(prefill_attn_mma_kernel<HD, REP, true>, dev); \
+  if (e == cudaSuccess) e = allow_max_smem(prefill_attn_mma_kernel<HD, REP, false>, dev);
   ATT(64, 1) ATT(64, 2) ATT(64, 4) ATT(64, 8) ATT(128, 1) ATT(128, 2) ATT(128, 4) ATT(128, 8)
 #undef ATT
   if (e == cudaSuccess) g_dev_init[dev] = true;
@@ -236,20 +246,35 @@ struct Int4Dev {
   int K = 0, N = 0, n_tiles = 0;
   uint4* w = nullptr;
   uint2* sz = nullptr;
-  size_t bytes() const {
-    return (size_t)n_tiles * (K / 64) * 32 * sizeof(uint4) + (size_t)n_tiles * (K / 128) * 8 * sizeof(uint2);
-  }
+  bool owned = true;   // false when w / sz live in a block's arena
+  static size_t w_bytes(int K, int N) { return (size_t)(((N + 31) / 32) * 2) * (K / 64) * 32 * sizeof(uint4); }
+  static size_t sz_bytes(int K, int N) { return (size_t)(((N + 31) / 32) * 2) * (K / 128) * 8 * sizeof(uint2); }
+  size_t bytes() const { return w_bytes(K, N) + sz_bytes(K, N); }
   void free_all() {
-    if (w) cudaFree(w);
-    if (sz) cudaFree(sz);
+    if (owned) {
+      if (w) cudaFree(w);
+      if (sz) cudaFree(sz);
+    }
     w = nullptr;
     sz = nullptr;
   }
 };
 
+// A bump allocator over one device allocation (256-byte aligned pieces).
+struct Arena {
+  char* base = nullptr;
+  size_t size = 0, used = 0;
+  void* take(size_t bytes) {
+    const size_t off = (used + 255) & ~size_t(255);
+    if (off + bytes > size) return nullptr;
+    used = off + bytes;
+    return base + off;
+  }
+};
+
 // Copy one linear in the storage format to the device and re-lay it out.
 // N is padded to whole pairs of 16-row tiles with zero weights.
-tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaStream_t st) {
+tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaStream_t st, Arena* arena = nullptr) {
   if (!h.qweight || !h.scales || !h.qzeros) return fail(TL_ERR_INVALID_ARG, "null INT4 array");
   const int G = K / 128, zw = (G + 7) / 8;
   out->K = K;
@@ -261,8 +286,15 @@ tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaS
   cudaError_t e = cudaMalloc(&dq, qb);
   if (e == cudaSuccess) e = cudaMalloc(&ds, sb);
   if (e == cudaSuccess) e = cudaMalloc(&dz, zb);
-  if (e == cudaSuccess) e = cudaMalloc(&out->w, (size_t)out->n_tiles * (K / 64) * 32 * sizeof(uint4));
-  if (e == cudaSuccess) e = cudaMalloc(&out->sz, (size_t)out->n_tiles * G * 8 * sizeof(uint2));
+  if (arena) {
+    out->owned = false;
+    out->w = (uint4*)arena->take(Int4Dev::w_bytes(K, N));
+    out->sz = (uint2*)arena->take(Int4Dev::sz_bytes(K, N));
+    if (e == cudaSuccess && (!out->w || !out->sz)) e = cudaErrorMemoryAllocation;
+  } else {
+    if (e == cudaSuccess) e = cudaMalloc(&out->w, Int4Dev::w_bytes(K, N));
+    if (e == cudaSuccess) e = cudaMalloc(&out->sz, Int4Dev::sz_bytes(K, N));
+  }
   if (e == cudaSuccess) e = cudaMemcpyAsync(dq, h.qweight, qb, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(ds, h.scales, sb, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(dz, h.qzeros, zb, cudaMemcpyHostToDevice, st);
@@ -297,6 +329,7 @@ struct BlockDev {
   __half* attn_norm = nullptr;
   __half* ffn_norm = nullptr;
   Int4Dev qkv, o, gate_up, down;
+  Arena arena;   // one allocation holding the four linears (an L2 window)
   void free_all() {
     if (attn_norm) cudaFree(attn_norm);
     if (ffn_norm) cudaFree(ffn_norm);
@@ -305,6 +338,8 @@ struct BlockDev {
     o.free_all();
     gate_up.free_all();
     down.free_all();
+    if (arena.base) cudaFree(arena.base);
+    arena = Arena{};
   }
   size_t bytes(int d) const { return qkv.bytes() + o.bytes() + gate_up.bytes() + down.bytes() + 4 * (size_t)d; }
 };
@@ -435,10 +470,12 @@ cudaError_t launch_decode_attn(const DecodeAttnArgs& a, int rows, int hd, int re
 }
 
 cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, int B, int hd, int rep, bool f32, cudaStream_t st) {
+  const dim3 grid((a.T + 15) / 16, a.Hkv, B);
+  const size_t smem = prefill_attn_smem_bytes(hd);
 #define C(HD, REP)                                                                                       \
   if (hd == HD && rep == REP)                                                                            \
-    return f32 ? launch(prefill_attn_simple_kernel<HD, REP, true>, dim3(a.T, a.Hkv, B), dim3(REP * 32), 0, st, a) \
-               : launch(prefill_attn_simple_kernel<HD, REP, false>, dim3(a.T, a.Hkv, B), dim3(REP * 32), 0, st, a);
+    return f32 ? launch(prefill_attn_mma_kernel<HD, REP, true>, grid, dim3(REP * 32), smem, st, a)       \
+               : launch(prefill_attn_mma_kernel<HD, REP, false>, grid, dim3(REP * 32), smem, st, a);
   C(64, 1) C(64, 2) C(64, 4) C(64, 8) C(128, 1) C(128, 2) C(128, 4) C(128, 8)
 #undef C
   return cudaErrorInvalidValue;
@@ -479,6 +516,8 @@ struct tl_model {
   int head_grid = 0;
   HeadIO* io = nullptr;          // output pointers of the current decode step
   TcScratch tc;                  // tensor-core GEMM scratch (prefill)
+  cudaAccessPolicyWindow loop_window = {};  // keeps the loop block's weights in L2
+  size_t l2_persist_bytes = 0;
   float* gu = nullptr;           // raw gate_up output of the prefill [rows][2F]
   cudaStream_t setup_stream = nullptr;
   cudaStream_t cap_stream = nullptr;   // stream used to capture decode graphs
@@ -542,17 +581,33 @@ tl_status upload_block(const tl_config& c, const tl_block& hb, BlockDev* b, cuda
   tl_status rc;
   if ((rc = upload_f16(hb.attn_norm, d, &b->attn_norm, st)) != TL_OK) return rc;
   if ((rc = upload_f16(hb.ffn_norm, d, &b->ffn_norm, st)) != TL_OK) return rc;
-  if ((rc = upload_int4(hb.qkv, d, qkv_rows, &b->qkv, st)) != TL_OK) return rc;
-  if ((rc = upload_int4(hb.o, c.n_q_heads * hd, d, &b->o, st)) != TL_OK) return rc;
-  if ((rc = upload_int4(hb.gate_up, d, 2 * c.ffn_dim, &b->gate_up, st)) != TL_OK) return rc;
-  if ((rc = upload_int4(hb.down, c.ffn_dim, d, &b->down, st)) != TL_OK) return rc;
+  const int qdim = c.n_q_heads * hd;
+  size_t total = 0;
+  const int shapes[4][2] = {{d, qkv_rows}, {qdim, d}, {d, 2 * c.ffn_dim}, {c.ffn_dim, d}};
+  for (auto& sh : shapes) total += Int4Dev::w_bytes(sh[0], sh[1]) + Int4Dev::sz_bytes(sh[0], sh[1]) + 512;
+  if (cudaMalloc(&b->arena.base, total) != cudaSuccess) return fail(TL_ERR_OOM, "block weights (%zu bytes)", total);
+  b->arena.size = total;
+  if ((rc = upload_int4(hb.qkv, d, qkv_rows, &b->qkv, st, &b->arena)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.o, qdim, d, &b->o, st, &b->arena)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.gate_up, d, 2 * c.ffn_dim, &b->gate_up, st, &b->arena)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.down, c.ffn_dim, d, &b->down, st, &b->arena)) != TL_OK) return rc;
   return TL_OK;
 }
+
+// Launches of a loop-block layer carry the L2 window of the loop weights.
+struct WindowScope {
+  cudaAccessPolicyWindow prev;
+  WindowScope(const tl_model* m, int layer) : prev(g_window) {
+    if (layer >= m->cfg.n_pre) g_window = m->loop_window;
+  }
+  ~WindowScope() { g_window = prev; }
+};
 
 // ---- one effective layer ------------------------------------------------------
 // QKV projection of `M` rows of the residual stream x (RMSNorm fused), RoPE on
 // q and k, k and v written to cache slice `layer` at each row's (lane, pos).
 tl_status run_qkv(tl_model* m, int layer, int M, float* x, const RowCtx* rows, float* q, cudaStream_t st) {
+  WindowScope window_scope(m, layer);
   const tl_config& c = m->cfg;
   const BlockDev& b = m->block(layer);
   const int hd = c.head_dim, qdim = c.n_q_heads * hd;
@@ -591,6 +646,7 @@ tl_status run_decode_attn(tl_model* m, int layer, int M, const RowCtx* rows, con
 
 // O projection + residual, RMSNorm + gate_up + SwiGLU, down + residual.
 tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float* h, cudaStream_t st) {
+  WindowScope window_scope(m, layer);
   const tl_config& c = m->cfg;
   const BlockDev& b = m->block(layer);
   const int d = c.d_model, F = c.ffn_dim, qdim = c.n_q_heads * c.head_dim;
@@ -623,6 +679,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
 // Prefill forms of run_qkv / run_ffn on the tensor cores (positions 0..T-1 of
 // one lane).
 tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, cudaStream_t st) {
+  WindowScope window_scope(m, layer);
   const tl_config& c = m->cfg;
   const BlockDev& b = m->block(layer);
   const int hd = c.head_dim, qdim = c.n_q_heads * hd;
@@ -640,6 +697,7 @@ tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, cudaStream_t st) {
 }
 
 tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
+  WindowScope window_scope(m, layer);
   const tl_config& c = m->cfg;
   const BlockDev& b = m->block(layer);
   const int d = c.d_model, F = c.ffn_dim, qdim = c.n_q_heads * c.head_dim;
@@ -773,6 +831,27 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     cudaFree(raw);
     if (e != cudaSuccess) return bail(cuda_fail(e, "head repack"));
   }
+  {  // L2 residency of the loop block: persisting window over its arena
+    int max_persist = 0, max_window = 0;
+    cudaDeviceGetAttribute(&max_persist, cudaDevAttrMaxPersistingL2CacheSize, device);
+    cudaDeviceGetAttribute(&max_window, cudaDevAttrMaxAccessPolicyWindowSize, device);
+    const size_t want = m->loop.arena.used;
+    if (max_persist > 0 && max_window > 0 && want > 0) {
+      const size_t carve = std::min((size_t)max_persist, want);
+      size_t cur = 0;
+      cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize);
+      if (cur < carve) cudaDeviceSetLimit(cudaLimitPersistingL2CacheSize, carve);
+      cudaDeviceGetLimit(&cur, cudaLimitPersistingL2CacheSize);
+      const size_t win = std::min(want, (size_t)max_window);
+      m->loop_window.base_ptr = m->loop.arena.base;
+      m->loop_window.num_bytes = win;
+      m->loop_window.hitRatio = std::min(1.0f, (float)cur / (float)win);
+      m->loop_window.hitProp = cudaAccessPropertyPersisting;
+      m->loop_window.missProp = cudaAccessPropertyStreaming;
+      m->l2_persist_bytes = cur;
+    }
+    cudaGetLastError();
+  }
   m->weight_bytes = m->loop.bytes(d) + (size_t)c.vocab * d * 4 + 2 * (size_t)d;
   for (auto& b : m->pre) m->weight_bytes += b.bytes(d);
 
@@ -831,6 +910,7 @@ void tl_model_destroy(tl_model* m) {
   if (!m) return;
   DeviceGuard guard(m->device);
   cudaDeviceSynchronize();
+  if (m->loop_window.num_bytes) cudaCtxResetPersistingL2Cache();
   m->free_all();
   delete m;
 }
@@ -1239,6 +1319,9 @@ tl_status tl_op_gqa_prefill(const uint16_t* d_q, const uint16_t* d_k, const uint
       (head_dim != 64 && head_dim != 128))
     return fail(TL_ERR_UNSUPPORTED, "unsupported attention shape");
   if (pos0 + T > ctx_stride) return fail(TL_ERR_INVALID_ARG, "pos0 + T exceeds ctx_stride");
+  int dev = 0;
+  TL_CUDA(cudaGetDevice(&dev));
+  TL_CUDA(init_device_kernels(dev));
   const int qdim = n_q_heads * head_dim;
   PrefillAttnArgs a{};
   a.qh = reinterpret_cast<const __half*>(d_q);
