@@ -205,6 +205,54 @@ def run_reference(args):
     return 0
 
 
+def run_ncu_case(args):
+    """A small eager run of the same model for kernel profilers (no timing
+    output): `decode` = prefill of the prompt + --decode-steps greedy steps,
+    `prefill` = two prefills of the prompt."""
+    import torch
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    shape = tl_synth.LOOPED_LM
+    w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM)
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, shape.vocab, PROMPT + 1)
+    steps = args.decode_steps
+    cfg = tl.make_config(shape, max_loops=LOOPS, max_ctx=PROMPT + max(steps, 1), max_lanes=1)
+    tw, keep = tl.make_weights(w)
+    m = tl.tl_model_create(cfg, tw, 0)
+    del keep
+    tl.tl_model_set_graphs(m, False)
+    d_prompt = torch.as_tensor(prompt, device="cuda:0")
+    hist = torch.zeros(steps + 1, dtype=torch.int32, device="cuda:0")
+    hp = hist.data_ptr()
+    for _ in range(2 if args.ncu_case == "prefill" else 1):
+        tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS)
+    if args.ncu_case == "decode":
+        hist[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
+        for i in range(steps):
+            tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1))
+    torch.cuda.synchronize()
+    tl.tl_check_device_error(m)
+    tl.tl_model_destroy(m)
+    print(json.dumps({"ncu_case": args.ncu_case, "decode_steps": steps, "ok": True}))
+    return 0
+
+
+def l2_read_probe(dev, mbytes=24, reps=200):
+    """Read bandwidth of an L2-resident buffer (GB/s): torch sum over a tensor
+    the size of the loop block, repeated; a reference for the loop-layer bytes."""
+    import torch
+    x = torch.ones(mbytes * (1 << 20) // 2, dtype=torch.float16, device=dev)
+    for _ in range(10):
+        x.sum()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        x.sum()
+    b.record()
+    b.synchronize()
+    return x.numel() * 2 * reps / (a.elapsed_time(b) * 1e6)
+
+
 def run_ours(args):
     import torch
     import tl_synth
@@ -225,14 +273,17 @@ def run_ours(args):
     shape = tl_synth.LOOPED_LM
     w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM)
     prompt = tl_synth.make_tokens(tl_synth.SEED_LM, shape.vocab, PROMPT + 1)
-    cfg = tl.make_config(shape, max_loops=LOOPS, max_ctx=PROMPT + STEPS_DECODE, max_lanes=1)
+    n_dec = args.decode_steps
+    cfg = tl.make_config(shape, max_loops=LOOPS, max_ctx=PROMPT + n_dec, max_lanes=1)
     tw, keep = tl.make_weights(w)
     m = tl.tl_model_create(cfg, tw, local)
     del keep
+    if args.no_graphs:
+        tl.tl_model_set_graphs(m, False)
 
     st = torch.cuda.Stream(device=dev)
     d_prompt = torch.as_tensor(prompt, device=dev)
-    hist = torch.zeros(STEPS_DECODE + 1, dtype=torch.int32, device=dev)
+    hist = torch.zeros(n_dec + 1, dtype=torch.int32, device=dev)
     hp = hist.data_ptr()
 
     def step(ev=None):
@@ -243,7 +294,7 @@ def run_ours(args):
             if ev:
                 ev[1].record(st)
             hist[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
-            for i in range(STEPS_DECODE):
+            for i in range(n_dec):
                 tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1), st)
             if ev:
                 ev[2].record(st)
@@ -277,15 +328,15 @@ def run_ours(args):
     if pg:
         pg.all_reduce(stats, op=pg.ReduceOp.MAX)
     total_ms, prefill_sum, decode_sum = (float(v) for v in stats.cpu())
-    tokens = world * STEPS_DECODE * args.steps
+    tokens = world * n_dec * args.steps
     value = tokens / (decode_sum / 1e3)
     generated = hist[1:].cpu().numpy().copy()
 
     # ---- end to end: pinned host prompt in, generated tokens out, per step --
     h_prompt = torch.from_numpy(prompt.copy()).pin_memory()
-    h_out = torch.empty(STEPS_DECODE, dtype=torch.int32).pin_memory()
+    h_out = torch.empty(n_dec, dtype=torch.int32).pin_memory()
     e2e_ms = []
-    for i in range(args.warmup + args.steps):
+    for i in range(0 if args.no_e2e else args.warmup + args.steps):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(st):
             a.record(st)
@@ -296,49 +347,72 @@ def run_ours(args):
         b.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
+    e2e = torch.tensor([sum(e2e_ms) if e2e_ms else float("nan")], dtype=torch.float64, device=dev)
     if pg:
         pg.all_reduce(e2e, op=pg.ReduceOp.MAX)
-    e2e_value = world * STEPS_DECODE * args.steps / (float(e2e.item()) / 1e3)
-    assert np.array_equal(h_out.numpy(), generated), "end-to-end run diverged from the timed run"
+    e2e_value = world * n_dec * args.steps / (float(e2e.item()) / 1e3) if e2e_ms else None
+    if e2e_ms:
+        assert np.array_equal(h_out.numpy(), generated), "end-to-end run diverged from the timed run"
 
     # ---- per-kernel profile of one decode phase (separate from the timing) -
-    with torch.cuda.stream(st):
-        tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS, None, None, st)
-        hist[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
-        st.synchronize()
-        tl.tl_model_profile_start(m)
-        for i in range(STEPS_DECODE):
-            tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1), st)
-        prof = tl.tl_model_profile_stop(m)
     peaks = load_peaks()
-    mean_keys = PROMPT + (STEPS_DECODE + 1) / 2
-    per_class = {}
-    for name, (n, ms) in prof.items():
-        avg_us = 1e3 * ms / n
-        b = BYTES_PER_LAUNCH.get(name)
-        if name == "attn_decode":
-            b = _attn_bytes_per_launch(mean_keys)
-        per_class[name] = {"launches": n, "total_ms": round(ms, 4), "avg_us": round(avg_us, 3),
-                           "gbs": round(b / (avg_us * 1e3), 1) if b else None}
-    dom = max(per_class, key=lambda k: per_class[k]["total_ms"])
-    dom_b = BYTES_PER_LAUNCH.get(dom) or (_attn_bytes_per_launch(mean_keys) if dom == "attn_decode" else None)
-    achieved = dom_b / (per_class[dom]["avg_us"] * 1e3) if dom_b else None
-    roofline = {
-        "kernel": dom, "bound": "hbm", "achieved": round(achieved, 1) if achieved else None,
-        "peak": peaks["hbm_gbs"], "unit": "GB/s",
-        "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
-        "traffic": None, "peak_source": peaks["source"],
-        "bytes_per_launch": dom_b,
-    }
+    per_class, roofline = {}, None
+    mean_keys = PROMPT + (n_dec + 1) / 2
+    if not args.no_profile:
+        with torch.cuda.stream(st):
+            tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS, None, None, st)
+            hist[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
+            st.synchronize()
+            tl.tl_model_profile_start(m)
+            for i in range(n_dec):
+                tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1), st)
+            prof = tl.tl_model_profile_stop(m)
+        for name, (n, ms) in prof.items():
+            avg_us = 1e3 * ms / n
+            b = BYTES_PER_LAUNCH.get(name)
+            if name == "attn_decode":
+                b = _attn_bytes_per_launch(mean_keys)
+            per_class[name] = {"launches": n, "total_ms": round(ms, 4), "avg_us": round(avg_us, 3),
+                               "gbs": round(b / (avg_us * 1e3), 1) if b else None}
+        dom = max(per_class, key=lambda k: per_class[k]["total_ms"])
+        dom_b = BYTES_PER_LAUNCH.get(dom) or (_attn_bytes_per_launch(mean_keys) if dom == "attn_decode" else None)
+        achieved = dom_b / (per_class[dom]["avg_us"] * 1e3) if dom_b else None
+        roofline = {
+            "kernel": dom, "bound": "hbm", "achieved": round(achieved, 1) if achieved else None,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
+            "traffic": None, "peak_source": peaks["source"],
+            "bytes_per_launch": dom_b,
+            "timing": "CUDA events around each launch of one extra decode phase (eager), after the timed region",
+        }
+    # whole-token byte roofline: HBM bytes (pre blocks, head, KV) at the
+    # measured copy bandwidth + the loop block's L2-resident re-reads at the
+    # measured L2 read bandwidth
+    l2_gbs = l2_read_probe(dev)
+    layer_bytes = sum(BYTES_PER_LAUNCH[k] for k in ("qkv", "o_proj", "gate_up", "down"))
+    hbm_bytes = 2 * layer_bytes + BYTES_PER_LAUNCH["head"] + 10 * _attn_bytes_per_launch(mean_keys)
+    l2_bytes = LOOPS * layer_bytes
+    t_roof_us = hbm_bytes / (peaks["hbm_gbs"] * 1e3) + l2_bytes / (l2_gbs * 1e3)
+    t_tok_us = 1e3 * decode_sum / (args.steps * n_dec)
+    roof_step = {"hbm_bytes_per_token": int(hbm_bytes), "l2_bytes_per_token": int(l2_bytes),
+                 "l2_read_gbs_measured": round(l2_gbs, 1), "roofline_us_per_token": round(t_roof_us, 2),
+                 "achieved_us_per_token": round(t_tok_us, 2), "frac": round(t_roof_us / t_tok_us, 4)}
+    # prefill: dense-equivalent flops of the linears + attention vs tensor peak
+    per_layer_flops = 2 * PROMPT * (D * (HQ + 2 * HKV) * HD + HQ * HD * D + D * 2 * F + F * D)
+    attn_flops = 4 * HQ * HD * PROMPT * (PROMPT + 1) / 2
+    pf_flops = (2 + LOOPS) * (per_layer_flops + attn_flops)
+    pf_ms = prefill_sum / args.steps
+    roof_prefill = {"flops": int(pf_flops), "achieved_tflops": round(pf_flops / (pf_ms * 1e9), 2),
+                    "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"] + " bf16 (fp16 assumed equal)",
+                    "frac": round(pf_flops / (pf_ms * 1e9) / peaks["bf16_tflops"], 4)}
 
     # ---- CPU oracle baseline (rank 0, bounded sample) -----------------------
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
-        n_dec = 4
-        p_s, d_s, _ = oracle_sample(w, prompt, n_dec)
-        cpu = {"value": n_dec / d_s, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"oracle prefill of the 128-token prompt ({p_s:.2f} s) + {n_dec} cached "
+        n_or = 4
+        p_s, d_s, _ = oracle_sample(w, prompt, n_or)
+        cpu = {"value": n_or / d_s, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"oracle prefill of the 128-token prompt ({p_s:.2f} s) + {n_or} cached "
                          f"greedy decode steps at L=8 ({d_s:.2f} s), float64 NumPy"}
 
     tl.tl_model_destroy(m)
@@ -348,16 +422,19 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total_ms / args.steps, 4),
             "prefill_ms": round(prefill_sum / args.steps, 4),
-            "decode_ms_per_token": round(decode_sum / (args.steps * STEPS_DECODE), 5),
+            "decode_ms_per_token": round(decode_sum / (args.steps * n_dec), 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (INT4 weights)",
             "data": "synthetic (seeded random weights and token ids)",
-            "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": PROMPT + STEPS_DECODE,
+            "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": PROMPT + n_dec,
+                       "decode_steps": n_dec, "cuda_graphs": not args.no_graphs,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: each step streams ~333 MB of weights"},
             "roofline": roofline,
+            "roofline_decode_token": roof_step,
+            "roofline_prefill": roof_prefill,
             "kernels_decode": per_class,
             "cpu_baseline": cpu,
-            "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
+            "e2e": {"value": round(e2e_value, 2) if e2e_value else None, "unit": UNIT,
                     "h2d_bytes_per_step": int(h_prompt.numel() * 4),
                     "d2h_bytes_per_step": int(h_out.numel() * 4)},
             "gpu_launches": int(launches),
@@ -377,11 +454,21 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=STEPS_DECODE,
+                    help="greedy decode steps per step (the workload uses 128)")
+    ap.add_argument("--no-graphs", action="store_true",
+                    help="launch decode kernels one by one instead of as CUDA graphs")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-profile", action="store_true")
+    ap.add_argument("--ncu-case", choices=["none", "decode", "prefill"], default="none",
+                    help="run a small eager case for kernel profilers and exit")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args)
+    if args.ncu_case != "none":
+        return run_ncu_case(args)
     return run_ours(args)
 
 

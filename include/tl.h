@@ -209,6 +209,11 @@ tl_status tl_model_profile_start(tl_model *m, unsigned class_mask);
  *   h_launches int [TL_KERNEL_CLASSES] or NULL, h_total_ms float [..] or NULL */
 tl_status tl_model_profile_stop(tl_model *m, int *h_launches, float *h_total_ms);
 
+/* Decode steps run as one captured CUDA graph per row pattern (lanes and
+ * loop counts) by default; enable = 0 launches their kernels one by one
+ * (same kernels, same results; useful under a kernel profiler). */
+tl_status tl_model_set_graphs(tl_model *m, int enable);
+
 /* Number of kernels this library has launched in the process so far. */
 unsigned long long tl_kernel_launch_count(void);
 

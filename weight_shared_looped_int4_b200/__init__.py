@@ -29,6 +29,7 @@ __all__ = [
     "tl_model_create", "tl_model_destroy", "tl_prefill", "tl_decode_step", "tl_score_last",
     "tl_lane_length", "tl_model_info", "tl_check_device_error",
     "tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count", "KERNEL_CLASSES",
+    "tl_model_set_graphs",
     "tl_linear_create", "tl_linear_destroy", "tl_linear_forward",
     "tl_op_rmsnorm", "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill",
     "tl_op_gqa_decode_noalloc",
@@ -89,6 +90,7 @@ def _load():
         "tl_model_profile_start": (st, [P, ctypes.c_uint]),
         "tl_model_profile_stop": (st, [P, POINTER(c_int), POINTER(c_float)]),
         "tl_kernel_launch_count": (ctypes.c_ulonglong, []),
+        "tl_model_set_graphs": (st, [P, c_int]),
         "tl_linear_create": (st, [POINTER(tl_int4_linear), c_int, c_int, c_int, POINTER(c_void_p)]),
         "tl_linear_destroy": (None, [P]),
         "tl_linear_forward": (st, [P, P, c_int, P, c_int, P]),
@@ -127,6 +129,7 @@ def __getattr__(name):
 
 # names every header declaration must have in the library (checked by tests)
 EXPORTED = sorted(["tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count",
+                   "tl_model_set_graphs",
                    "tl_model_create", "tl_model_destroy", "tl_prefill", "tl_decode_step",
                    "tl_score_last", "tl_lane_length", "tl_model_info", "tl_check_device_error",
                    "tl_linear_create", "tl_linear_destroy", "tl_linear_forward", "tl_op_rmsnorm",
@@ -276,6 +279,10 @@ def tl_model_profile_stop(model):
     total = (c_float * n)()
     _check(_L().tl_model_profile_stop(model, launches, total))
     return {KERNEL_CLASSES[i]: (launches[i], total[i]) for i in range(n) if launches[i]}
+
+
+def tl_model_set_graphs(model, enable: bool) -> None:
+    _check(_L().tl_model_set_graphs(model, 1 if enable else 0))
 
 
 def tl_kernel_launch_count() -> int:

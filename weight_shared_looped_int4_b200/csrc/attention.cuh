@@ -21,20 +21,24 @@
 namespace tl {
 
 constexpr int kDecodeMaxSplits = 32;
-constexpr int kDecodeThreads = 256;
-constexpr int kDecodeSub = 64;      // keys per shared-memory sub-chunk
+constexpr int kDecodeThreads = 512;
+constexpr int kDecodeSub = 256;     // largest split, staged in shared memory at once
 constexpr int kKeyPad = 8;          // fp16 padding per staged key row (bank spread)
 
-// Keys per split: 64, doubled until at most kDecodeMaxSplits splits are
-// needed (so <= 8192 keys fit).  Depends only on the row's own key count.
+// Keys per split: kDecodeSub (256), so contexts up to 8192 keys need at most
+// kDecodeMaxSplits splits and up to 256 keys need no merge.  (Splits of 64
+// keys spread short contexts over more CTAs but measured slower at batch 1:
+// the ticketed merge costs more than the shorter scan saves.)  The length
+// depends only on the row's own key count, never on the batch.
 __host__ __device__ inline int decode_split_len(int n_keys) {
   int c = kDecodeSub;
   while (c * kDecodeMaxSplits < n_keys) c <<= 1;
   return c;
 }
 
-__host__ __device__ inline size_t decode_attn_smem_bytes(int hd) {
-  return (size_t)2 * 2 * kDecodeSub * (hd + kKeyPad) * 2;  // K and V, double buffered
+__host__ __device__ inline size_t decode_attn_smem_bytes(int hd, int rep) {
+  (void)rep;
+  return (size_t)2 * kDecodeSub * (hd + kKeyPad) * 2;  // K and V of one split
 }
 
 // Queries and outputs are fp32 inside the model (no rounding between the QKV
@@ -74,30 +78,46 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// One CTA per (row, kv head, key split).  The split's keys are streamed in
-// sub-chunks of kDecodeSub keys; K and V of the next sub-chunk are copied into
-// shared memory (cp.async, double buffered) while the current one is used, and
-// the softmax runs online across sub-chunks.  Up to 256 keys there is one
-// split and no merge step.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"((unsigned)__cvta_generic_to_shared(p)));
+}
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// (hi, lo) fp16 pairs of two floats.
+__device__ __forceinline__ void split_h2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 r = __half22float2(h);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = pack_h2(a - r.x, b - r.y);
+}
+
+// One CTA (16 warps) per (row, kv head, split of up to 256 keys).  All keys of the
+// split are copied into shared memory at once (cp.async).  On the tensor
+// cores, with the REP query heads of the group as the MMA rows: warp w scores
+// keys 16w..16w+15 (S = Q K^T), one warp per head takes the softmax over the
+// split, then warp w computes output dims 8w..8w+7 over all keys (O = P V).
+// Q and P are split into fp16 pairs (hi, lo).  Splits are merged by the last
+// CTA of the (row, kv head) to finish (see above).
 template <int HD, int REP, bool F32>
 __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const DecodeAttnArgs a) {
-  constexpr int DPL = HD / 32;
   constexpr int SUB = kDecodeSub;
-  constexpr int NW = kDecodeThreads / 32;
-  constexpr int CHUNKS = SUB * HD / 8;   // 16-byte pieces of one K (or V) sub-chunk
-  constexpr int KH = kDecodeThreads / HD; // key interleave of the P V step
+  constexpr int KC = HD / 16;
   constexpr int LDK = HD + kKeyPad;
+  constexpr int CHUNKS = SUB * HD / 8;      // 16-byte pieces of K (or V)
   extern __shared__ __align__(128) unsigned char dsm[];
-  __half (*ks)[SUB][LDK] = reinterpret_cast<__half (*)[SUB][LDK]>(dsm);
-  __half (*vs)[SUB][LDK] = reinterpret_cast<__half (*)[SUB][LDK]>(dsm + (size_t)2 * SUB * LDK * 2);
-  __shared__ __align__(16) float qs[REP][HD];
-  __shared__ float sc[REP][SUB];
-  __shared__ float s_m[REP], s_l[REP], s_corr[REP];
-  __shared__ float s_acc[KH][REP][HD];
+  __half* ks = reinterpret_cast<__half*>(dsm);                 // [SUB][LDK]
+  __half* vs = ks + (size_t)SUB * LDK;                         // [SUB][LDK]
+  __shared__ __align__(16) float sc[REP][SUB + 4];
+  __shared__ float s_m[REP], s_l[REP];
   __shared__ int s_last;
 
   const int split = blockIdx.x, kvh = blockIdx.y, row = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
   pdl_trigger();
   pdl_wait();
 
@@ -107,124 +127,117 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   const int nsplit = (n + C - 1) / C;
   if (split >= nsplit) return;
   const int j0 = split * C, j1 = min(n, j0 + C), nk = j1 - j0;
-  const int nsub = (nk + SUB - 1) / SUB;
   const float scale = 1.0f / sqrtf((float)HD);
 
   const __half* kp = a.k + rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;
   const __half* vp = a.v + rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;
+  for (int c = threadIdx.x; c < CHUNKS; c += kDecodeThreads) {
+    const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
+    const bool ok = key < nk;
+    const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
+    cp_async16(ks + key * LDK + off, kp + src, ok ? 16 : 0);
+    cp_async16(vs + key * LDK + off, vp + src, ok ? 16 : 0);
+  }
+  cp_async_commit();
 
-  auto issue = [&](int sb, int b) {
-    const int jb = j0 + sb * SUB;
-    for (int c = threadIdx.x; c < CHUNKS; c += kDecodeThreads) {
-      const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
-      const bool ok = jb + key < j1;
-      const size_t src = ok ? (size_t)(jb + key) * HD + off : 0;
-      cp_async16(&ks[b][key][off], kp + src, ok ? 16 : 0);
-      cp_async16(&vs[b][key][off], vp + src, ok ? 16 : 0);
-    }
-    cp_async_commit();
-  };
-  issue(0, 0);
-
+  // Q fragments (hi, lo): MMA row g is q head g of the group (zero beyond REP)
   const size_t qoff = (size_t)row * a.ldq + (size_t)kvh * REP * HD;
-  for (int i = threadIdx.x; i < REP * HD; i += kDecodeThreads)
-    qs[i / HD][i % HD] = F32 ? a.qf[qoff + i] : __half2float(a.qh[qoff + i]);
-  if (threadIdx.x < REP) { s_m[threadIdx.x] = -INFINITY; s_l[threadIdx.x] = 0.f; }
-
-  const int d = threadIdx.x % HD, kh = threadIdx.x / HD;
-  float acc[REP];
+  uint32_t qa[KC][2], ql[KC][2];
 #pragma unroll
-  for (int h = 0; h < REP; ++h) acc[h] = 0.f;
-
-  for (int sb = 0; sb < nsub; ++sb) {
-    const int b = sb & 1;
-    if (sb + 1 < nsub) {
-      issue(sb + 1, b ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int kc = min(SUB, nk - sb * SUB);
-
-    // scores of this sub-chunk: thread (key j, head h) takes one dot product
-    // (K row from shared memory, q broadcast), no shuffles
-    for (int item = threadIdx.x; item < REP * SUB; item += kDecodeThreads) {
-      const int jj = item % SUB, h = item / SUB;
-      if (jj < kc) {
-        const float4* qv = reinterpret_cast<const float4*>(qs[h]);
-        const uint4* kr = reinterpret_cast<const uint4*>(&ks[b][jj][0]);
-        float p = 0.f;
-#pragma unroll 4
-        for (int c8 = 0; c8 < HD / 8; ++c8) {
-          const uint4 raw = kr[c8];
-          const float4 qa = qv[2 * c8], qb = qv[2 * c8 + 1];
-          const float2 k01 = h2_to_f2(raw.x), k23 = h2_to_f2(raw.y);
-          const float2 k45 = h2_to_f2(raw.z), k67 = h2_to_f2(raw.w);
-          p = fmaf(qa.x, k01.x, p); p = fmaf(qa.y, k01.y, p);
-          p = fmaf(qa.z, k23.x, p); p = fmaf(qa.w, k23.y, p);
-          p = fmaf(qb.x, k45.x, p); p = fmaf(qb.y, k45.y, p);
-          p = fmaf(qb.z, k67.x, p); p = fmaf(qb.w, k67.y, p);
-        }
-        sc[h][jj] = p * scale;
+  for (int c = 0; c < KC; ++c) {
+    float2 v0 = make_float2(0.f, 0.f), v1 = make_float2(0.f, 0.f);
+    if (g < REP) {
+      const size_t o = qoff + (size_t)g * HD + c * 16 + 2 * t;
+      if (F32) {
+        v0 = *reinterpret_cast<const float2*>(a.qf + o);
+        v1 = *reinterpret_cast<const float2*>(a.qf + o + 8);
+      } else {
+        v0 = __half22float2(*reinterpret_cast<const __half2*>(a.qh + o));
+        v1 = __half22float2(*reinterpret_cast<const __half2*>(a.qh + o + 8));
       }
     }
-    __syncthreads();
-
-    // online softmax update (one warp per head)
-    for (int h = warp; h < REP; h += NW) {
-      float mx = -INFINITY;
-      for (int j = lane; j < kc; j += 32) mx = fmaxf(mx, sc[h][j]);
-      mx = warp_max(mx);
-      const float m_new = fmaxf(s_m[h], mx);
-      float sum = 0.f;
-      for (int j = lane; j < kc; j += 32) {
-        const float e = expf(sc[h][j] - m_new);
-        sc[h][j] = e;
-        sum += e;
-      }
-      sum = warp_sum(sum);
-      if (lane == 0) {
-        const float corr = expf(s_m[h] - m_new);
-        s_corr[h] = corr;
-        s_l[h] = s_l[h] * corr + sum;
-        s_m[h] = m_new;
-      }
-    }
-    __syncthreads();
-
-    // P V: thread (d, kh) takes keys kh, kh + KH, ...
-#pragma unroll
-    for (int h = 0; h < REP; ++h) acc[h] *= s_corr[h];
-    for (int jj = kh; jj < kc; jj += KH) {
-      const float vv = __half2float(vs[b][jj][d]);
-#pragma unroll
-      for (int h = 0; h < REP; ++h) acc[h] = fmaf(sc[h][jj], vv, acc[h]);
-    }
-    __syncthreads();
+    split_h2(v0.x * scale, v0.y * scale, qa[c][0], ql[c][0]);
+    split_h2(v1.x * scale, v1.y * scale, qa[c][1], ql[c][1]);
   }
-
-  // combine the key interleave
-#pragma unroll
-  for (int h = 0; h < REP; ++h) s_acc[kh][h][d] = acc[h];
+  cp_async_wait<0>();
   __syncthreads();
-  if (threadIdx.x < HD) {
+
+  // S for keys kb .. kb+15 of this warp (two n8 tiles) -> shared memory
+  const int kb = warp * 16;
+  if (kb < nk) {
 #pragma unroll
-    for (int h = 0; h < REP; ++h) {
-      float v = 0.f;
+    for (int nt = 0; nt < 2; ++nt) {
+      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < KH; ++q) v += s_acc[q][h][d];
-      acc[h] = v;
+      for (int c = 0; c < KC; ++c) {
+        const __half* kr = ks + (kb + nt * 8 + g) * LDK + c * 16 + 2 * t;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kr);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 8);
+        const uint32_t ah[4] = {qa[c][0], 0u, qa[c][1], 0u};
+        const uint32_t al[4] = {ql[c][0], 0u, ql[c][1], 0u};
+        mma_f16_16816(acc0, ah, b0, b1);
+        mma_f16_16816(acc1, al, b0, b1);
+      }
+      if (g < REP) {
+        const int key = kb + nt * 8 + 2 * t;
+        sc[g][key] = key < nk ? acc0[0] + acc1[0] : -INFINITY;
+        sc[g][key + 1] = key + 1 < nk ? acc0[1] + acc1[1] : -INFINITY;
+      }
     }
   }
+  __syncthreads();
 
+  // softmax over the split: warp h takes head h (unnormalised exp in place)
+  if (warp < REP) {
+    const int h = warp;
+    float mx = -INFINITY;
+    for (int j = lane; j < nk; j += 32) mx = fmaxf(mx, sc[h][j]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+    for (int j = lane; j < nk; j += 32) {
+      const float e = expf(sc[h][j] - mx);
+      sc[h][j] = e;
+      sum += e;
+    }
+    // keys nk .. end of their last 16-key chunk read as zero probability
+    for (int j = nk + lane; j < ((nk + 15) & ~15); j += 32) sc[h][j] = 0.f;
+    sum = warp_sum(sum);
+    if (lane == 0) { s_m[h] = mx; s_l[h] = sum; }
+  }
+  __syncthreads();
+
+  // O = P V: warp w takes output dims 8w .. 8w+7 over all keys of the split
+  const int dt = warp;
+  float o[4] = {0.f, 0.f, 0.f, 0.f}, o2[4] = {0.f, 0.f, 0.f, 0.f};
+  if (dt < HD / 8) {
+    const int nch = (nk + 15) >> 4;
+    for (int c = 0; c < nch; ++c) {
+      uint32_t pa[4] = {0u, 0u, 0u, 0u}, pl[4] = {0u, 0u, 0u, 0u};
+      if (g < REP) {
+        const float2 p0 = *reinterpret_cast<const float2*>(&sc[g][c * 16 + 2 * t]);
+        const float2 p1 = *reinterpret_cast<const float2*>(&sc[g][c * 16 + 8 + 2 * t]);
+        split_h2(p0.x, p0.y, pa[0], pl[0]);
+        split_h2(p1.x, p1.y, pa[2], pl[2]);
+      }
+      uint32_t vb[4];
+      // rows (keys) c*16 .. +15 at dims 8 dt .. +7: two 8x8 transposed tiles
+      const int key = c * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      ldmatrix_x4_trans(vb, vs + key * LDK + dt * 8);
+      mma_f16_16816(o, pa, vb[0], vb[1]);
+      mma_f16_16816(o2, pl, vb[0], vb[1]);
+    }
+  }
   const size_t ooff = (size_t)row * a.ldo + (size_t)kvh * REP * HD;
   if (nsplit == 1) {
-    if (threadIdx.x < HD) {
-#pragma unroll
-      for (int h = 0; h < REP; ++h) {
-        if (F32) store_out(a.of + ooff + h * HD + d, acc[h] / s_l[h]);
-        else store_out(a.oh + ooff + h * HD + d, acc[h] / s_l[h]);
+    if (dt < HD / 8 && g < REP) {
+      const float inv = 1.f / s_l[g];
+      const int dd = g * HD + dt * 8 + 2 * t;
+      if (F32) {
+        store_out(a.of + ooff + dd, (o[0] + o2[0]) * inv);
+        store_out(a.of + ooff + dd + 1, (o[1] + o2[1]) * inv);
+      } else {
+        store_out(a.oh + ooff + dd, (o[0] + o2[0]) * inv);
+        store_out(a.oh + ooff + dd + 1, (o[1] + o2[1]) * inv);
       }
     }
     return;
@@ -233,9 +246,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   constexpr int PSTRIDE = REP * (HD + 2);
   float* pbase = a.part + ((size_t)row * a.Hkv + kvh) * kDecodeMaxSplits * PSTRIDE;
   float* pme = pbase + (size_t)split * PSTRIDE;
-  if (threadIdx.x < HD) {
-#pragma unroll
-    for (int h = 0; h < REP; ++h) pme[h * (HD + 2) + d] = acc[h];
+  if (dt < HD / 8 && g < REP) {
+    pme[g * (HD + 2) + dt * 8 + 2 * t] = o[0] + o2[0];
+    pme[g * (HD + 2) + dt * 8 + 2 * t + 1] = o[1] + o2[1];
   }
   if (threadIdx.x < REP) {
     pme[threadIdx.x * (HD + 2) + HD] = s_m[threadIdx.x];
@@ -251,7 +264,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   if (!s_last) return;
   __threadfence();
 
-  if (threadIdx.x < HD) {
+  const int d = threadIdx.x;
+  if (d < HD) {
 #pragma unroll
     for (int h = 0; h < REP; ++h) {
       float mx = -INFINITY;
@@ -293,23 +307,6 @@ struct PrefillAttnArgs {
 // memory serves all REP heads of the group.  S = Q K^T and O += P V run on the
 // tensor cores; Q and P are split into fp16 pairs (hi, lo) and both halves are
 // multiplied (K and V are fp16 already), so the result keeps ~fp32 accuracy.
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], const void* p) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"((unsigned)__cvta_generic_to_shared(p)));
-}
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  const __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-// (hi, lo) fp16 pairs of two floats.
-__device__ __forceinline__ void split_h2(float a, float b, uint32_t& hi, uint32_t& lo) {
-  const __half2 h = __floats2half2_rn(a, b);
-  const float2 r = __half22float2(h);
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = pack_h2(a - r.x, b - r.y);
-}
-
 constexpr int kPfKeys = 64;   // keys per staged block
 constexpr int kPfPad = 8;     // fp16 padding per staged row
 

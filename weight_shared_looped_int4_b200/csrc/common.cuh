@@ -83,6 +83,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }
+// Bounded wait that gives up at once when another thread of the CTA already
+// gave up (*fail != 0), so a stuck pipeline costs at most one time-out per
+// thread and threads that share later barriers keep the same control flow.
+__device__ __forceinline__ bool mbar_wait_or_fail(uint64_t* bar, unsigned parity, int* fail) {
+  if (*reinterpret_cast<volatile int*>(fail)) return false;
+  if (mbar_wait(bar, parity)) return true;
+  atomicOr(fail, 1);
+  return false;
+}
 // Global -> shared bulk copy of `bytes` (multiple of 16, both addresses 16-byte
 // aligned); completion is signalled on `bar` as transaction bytes.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
@@ -160,12 +169,19 @@ __device__ __forceinline__ float warp_max(float v) {
 __device__ __forceinline__ float silu(float u) { return u / (1.0f + expf(-u)); }
 
 // RoPE angle of pair j at position p: p * theta^(-2j/hd), evaluated in double
-// precision and returned as (cos, sin) in float.
+// precision and returned as (cos, sin) in float.  The model keeps a table of
+// these values per (position, j), built once at load.
 __device__ __forceinline__ float2 rope_cos_sin(int pos, int j, int hd, float theta) {
   const double inv_freq = exp(-(2.0 * (double)j / (double)hd) * log((double)theta));
   double s, c;
   sincos((double)pos * inv_freq, &s, &c);
   return make_float2((float)c, (float)s);
+}
+
+// (cos, sin) of pair j at position p from a [positions][hd/2] table when
+// given, else computed.
+__device__ __forceinline__ float2 rope_cs(const float2* tab, int pos, int j, int hd, float theta) {
+  return tab ? tab[(size_t)pos * (hd >> 1) + j] : rope_cos_sin(pos, j, hd, theta);
 }
 
 }  // namespace tl

@@ -157,6 +157,7 @@ struct TcGemmArgs {
   __half* v_plane;
   int ctx, pos0;
   float theta;
+  const float2* rope_tab;  // (cos, sin) [positions][hd/2], or NULL
   // split-K
   float* partial;        // [splits][row tiles][token tiles][128 tokens][128 rows]
   unsigned* tickets;     // [row tiles][token tiles], zero between launches
@@ -214,8 +215,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
       const uint32_t idesc = idesc_f16_f32(kTcRows, NB);
       for (int it = 0; it < ng; ++it) {
         const int s = it & 1;
-        if (!mbar_wait(&bar_full[s], (it >> 1) & 1)) { s_fail = 1; break; }
-        if (it >= 2 && !mbar_wait(&bar_tempty[s], ((it - 2) >> 1) & 1)) { s_fail = 1; break; }
+        if (!mbar_wait_or_fail(&bar_full[s], (it >> 1) & 1, &s_fail)) break;
+        if (it >= 2 && !mbar_wait_or_fail(&bar_tempty[s], ((it - 2) >> 1) & 1, &s_fail)) break;
         tc_fence_after();
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -234,7 +235,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     const int kw = a.K >> 6;  // 64-wide chunks per row
     for (int it = 0; it < ng; ++it) {
       const int s = it & 1, g = g_begin + it;
-      if (it >= 2 && !mbar_wait(&bar_empty[s], ((it - 2) >> 1) & 1)) { atomicOr(&s_fail, 1); break; }
+      if (it >= 2 && !mbar_wait_or_fail(&bar_empty[s], ((it - 2) >> 1) & 1, &s_fail)) break;
       if (p == 0) {
         mbar_expect_tx(&bar_full[s], B_BYTES);
         const uint8_t* src = a.bt + ((size_t)tt * G + g) * B_BYTES;
@@ -292,7 +293,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
       const int b = it & 1;
       const float sc = s_next;
       if (it + 1 < ng) s_next = scale_of(g_begin + it + 1);
-      if (!mbar_wait(&bar_tfull[b], (it >> 1) & 1)) { atomicOr(&s_fail, 1); break; }
+      // on a time-out the loop keeps its shape (no further waits) so the
+      // epilogue barriers below still match across the epilogue warps
+      mbar_wait_or_fail(&bar_tfull[b], (it >> 1) & 1, &s_fail);
       tc_fence_after();
       const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16) + b * NCOL + half * 64;
 #pragma unroll
@@ -383,12 +386,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
           const float va = xch[tl_ * kTcRows + r_a], vb = xch[tl_ * kTcRows + r_b];
           const int pos = a.pos0 + t;
           if (na < a.n_q_rows) {
-            const float2 cs = rope_cos_sin(pos, j, hd, a.theta);
+            const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
             float* qo = a.q_out + (size_t)t * a.ldq;
             qo[na] = va * cs.x - vb * cs.y;
             qo[na + hh] = vb * cs.x + va * cs.y;
           } else if (na < a.n_q_rows + a.n_kv_rows) {
-            const float2 cs = rope_cos_sin(pos, j, hd, a.theta);
+            const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
             const int kvh = (na - a.n_q_rows) / hd;
             __half* dst = a.k_plane + ((size_t)kvh * a.ctx + pos) * hd;
             dst[j] = __float2half_rn(va * cs.x - vb * cs.y);

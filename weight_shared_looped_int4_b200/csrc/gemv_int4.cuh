@@ -73,19 +73,24 @@ struct GemvArgs {
   int ctx;
   const RowCtx* rows;  // per activation row
   float theta;
+  const float2* rope_tab;  // (cos, sin) [positions][hd/2], or NULL
+  int* err_flag;       // device fault flags (a bounded wait gave up)
 };
 
 constexpr int kGemvThreads = 256;
-constexpr int kGemvPrefetch = 8;
 
-// Shared memory: the activation planes (hi, and lo unless IN_F16) of M rows,
-// then the K-quarter reduction buffer.
+// Shared memory of a CTA: its weight tiles and scales (bulk-copied), the
+// activation planes (hi, and lo unless IN_F16) of M rows, the K-slice
+// reduction buffer and the RMSNorm partial sums.
 __host__ __device__ inline size_t gemv_act_bytes(int K, int M, bool lo) {
   return (((size_t)M * (K + 8) * 2 * (lo ? 2 : 1)) + 15) / 16 * 16;
 }
-__host__ __device__ inline size_t gemv_smem_bytes(int K, int M, bool lo) {
-  const int nt = M <= 8 ? 1 : 2;
-  return gemv_act_bytes(K, M, lo) + (size_t)8 * 16 * nt * 8 * 4 + 8 * kMaxLanes * 4;
+__host__ __device__ inline size_t gemv_w_bytes(int K) { return (size_t)(K >> 6) * 512; }
+__host__ __device__ inline size_t gemv_sz_bytes(int K) { return (size_t)(K >> 7) * 64; }
+__host__ __device__ inline size_t gemv_smem_bytes(int K, int M, bool lo, int tpc) {
+  const int nc = M <= 8 ? 8 : 16;
+  return (size_t)tpc * (gemv_w_bytes(K) + gemv_sz_bytes(K)) + gemv_act_bytes(K, M, lo) +
+         (size_t)8 * 16 * nc * 4 + 16 * 8 * 4;
 }
 
 // Tiles per CTA of each epilogue.
@@ -93,20 +98,35 @@ __host__ __device__ constexpr int gemv_tpc(int epi) {
   return (epi == EPI_ROPE_KV || epi == EPI_SWIGLU) ? 2 : 1;
 }
 
+// MMA column layouts.  NT = 0: one MMA per k16 tile; with the fp16 pair the
+// B columns are (row m hi, row m lo) for m < 4, otherwise columns are rows
+// m < 8.  NT = 1: rows m < 8, hi and lo in two MMAs.  NT = 2: rows m < 16.
+__host__ __device__ inline int gemv_nt(int M, bool lo) {
+  if (M <= (lo ? 4 : 8)) return 0;
+  return M <= 8 ? 1 : 2;
+}
+
 template <int NT, int IN, int EPI>
-__global__ void __launch_bounds__(kGemvThreads, 3) gemv_int4_kernel(const GemvArgs a) {
+__global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs a) {
   constexpr bool LO = (IN != IN_F16);
   constexpr int TPC = gemv_tpc(EPI);
-  constexpr int KS = 8 / TPC;  // K slices
+  constexpr int KS = 8 / TPC;                 // K slices
+  constexpr int NC = NT == 2 ? 16 : 8;        // reduction columns
+  constexpr int NTILES = NT == 2 ? 2 : 1;     // n8 tiles of the MMA
   extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t wbar;
+  __shared__ int s_ok;
   const int K = a.K;
   const int M = a.M;
   const int ldxs = K + 8;
-  __half* xs = reinterpret_cast<__half*>(smem);           // hi plane [M][ldxs]
-  __half* xl = xs + (size_t)M * ldxs;                     // lo plane [M][ldxs]
-  constexpr int NC = NT * 8;  // activation columns of the MMA
-  float* red = reinterpret_cast<float*>(smem + gemv_act_bytes(K, M, LO));   // [8][16][NC]
-  float* ssq = red + 8 * 16 * NC;                                           // [16 rows][8 warps]
+  const int n_chunks = K >> 6;
+  const size_t wt_bytes = gemv_w_bytes(K), sz_bytes = gemv_sz_bytes(K);
+  unsigned char* sw = smem;                                       // [TPC][chunks][32][16 B]
+  unsigned char* ssz = smem + TPC * wt_bytes;                     // [TPC][groups][8][8 B]
+  __half* xs = reinterpret_cast<__half*>(ssz + TPC * sz_bytes);   // hi plane [M][ldxs]
+  __half* xl = xs + (size_t)M * ldxs;                             // lo plane [M][ldxs]
+  float* red = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(xs) + gemv_act_bytes(K, M, LO));
+  float* ssq = red + 8 * 16 * NC;                                 // [16 rows][8 warps]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -125,23 +145,23 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_int4_kernel(const GemvAr
     t0 = head * 2 * a.pair_off + j16;
     t1 = t0 + a.pair_off;
   }
-  const int tile = tsel ? t1 : t0;
-
-  const int n_chunks = K >> 6;
-  const int c_begin = (n_chunks * kq) / KS;
-  const int nc = (n_chunks * (kq + 1)) / KS - c_begin;
-  const uint4* wp = a.w + ((size_t)tile * n_chunks + c_begin) * 32 + lane;
-  const uint2* szp = a.sz + (size_t)tile * (K >> 7) * 8 + g;
 
   pdl_trigger();
-
-  uint4 buf[kGemvPrefetch];
-  uint2 szb[kGemvPrefetch];
-#pragma unroll
-  for (int i = 0; i < kGemvPrefetch; ++i) {
-    if (i < nc) {
-      buf[i] = ldg_stream(wp + (size_t)i * 32);
-      szb[i] = __ldg(szp + ((c_begin + i) >> 1) * 8);
+  // The weights do not depend on earlier kernels: start their bulk copies
+  // before waiting for the previous kernel.
+  if (threadIdx.x == 0) {
+    mbar_init(&wbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&wbar, (unsigned)(TPC * (wt_bytes + sz_bytes)));
+    for (int ts = 0; ts < TPC; ++ts) {
+      const int tile = ts ? t1 : t0;
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
+      for (size_t off = 0; off < wt_bytes; off += 32768) {
+        const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
+        bulk_g2s(sw + ts * wt_bytes + off, src + off, n, &wbar);
+      }
+      bulk_g2s(ssz + ts * sz_bytes, reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes,
+               (unsigned)sz_bytes, &wbar);
     }
   }
 
@@ -202,80 +222,102 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_int4_kernel(const GemvAr
       }
     }
   }
+  if (threadIdx.x == 0) {
+    s_ok = mbar_wait(&wbar, 0) ? 1 : 0;
+    if (!s_ok) atomicOr(a.err_flag, kErrTimeout);
+  }
   __syncthreads();
+  if (!s_ok) return;  // uniform: every thread read the same flag after the barrier
 
-  // ---- main loop: 64-wide K chunks, 4 MMAs each ---------------------------
-  float acc[NT][4];
+  // ---- main loop: 64-wide K chunks from shared memory, 4 k16 tiles each ----
+  const int c_begin = (n_chunks * kq) / KS;
+  const int nc = (n_chunks * (kq + 1)) / KS - c_begin;
+  const unsigned char* wbase = sw + tsel * wt_bytes + (size_t)lane * 16;
+  const unsigned char* sbase = ssz + tsel * sz_bytes + (size_t)g * 8;
+  // B-fragment source of this lane: activation row and plane
+  int brow, bplane;
+  if (NT == 0 && LO) { brow = g >> 1; bplane = g & 1; }
+  else { brow = g; bplane = 0; }
+  const __half* bsrc = (bplane ? xl : xs) + (size_t)brow * ldxs + 2 * t;
+
+  float acc[NTILES][4];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int nt = 0; nt < NTILES; ++nt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
 
-  for (int base = 0; base < nc; base += kGemvPrefetch) {
+#pragma unroll 2
+  for (int ci = 0; ci < nc; ++ci) {
+    const int c = c_begin + ci;
+    const uint4 wv = *reinterpret_cast<const uint4*>(wbase + (size_t)c * 512);
+    const uint2 sv = *reinterpret_cast<const uint2*>(sbase + (size_t)(c >> 1) * 64);
+    const int kc = c * 64;
+    float tmp[NTILES][4];
 #pragma unroll
-    for (int i = 0; i < kGemvPrefetch; ++i) {
-      const int ci = base + i;
-      if (ci < nc) {
-        const uint4 wv = buf[i];
-        const uint2 sv = szb[i];
-        if (ci + kGemvPrefetch < nc) {
-          buf[i] = ldg_stream(wp + (size_t)(ci + kGemvPrefetch) * 32);
-          szb[i] = __ldg(szp + ((c_begin + ci + kGemvPrefetch) >> 1) * 8);
+    for (int nt = 0; nt < NTILES; ++nt)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) tmp[nt][q] = 0.f;
+    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t af[4];
+      unpack_a_frag(words[j], sv.y, af);
+      const int ko = kc + j * 16;
+      if (NT == 0) {
+        uint32_t b0 = 0, b1 = 0;
+        if (brow < M) {
+          b0 = *reinterpret_cast<const uint32_t*>(bsrc + ko);
+          b1 = *reinterpret_cast<const uint32_t*>(bsrc + ko + 8);
         }
-        const int kc = (c_begin + ci) * 64 + 2 * t;
-        float tmp[NT][4];
+        mma_f16_16816(tmp[0], af, b0, b1);
+      } else {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) tmp[nt][q] = 0.f;
-        const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t af[4];
-          unpack_a_frag(words[j], sv.y, af);
-#pragma unroll
-          for (int nt = 0; nt < NT; ++nt) {
-            const int row = nt * 8 + g;   // activation row of this lane's B fragment
-            uint32_t b0 = 0, b1 = 0, c0 = 0, c1 = 0;
-            if (row < M) {
-              const size_t off = (size_t)row * ldxs + kc + j * 16;
-              b0 = *reinterpret_cast<const uint32_t*>(xs + off);
-              b1 = *reinterpret_cast<const uint32_t*>(xs + off + 8);
-              if (LO) {
-                c0 = *reinterpret_cast<const uint32_t*>(xl + off);
-                c1 = *reinterpret_cast<const uint32_t*>(xl + off + 8);
-              }
+        for (int nt = 0; nt < NTILES; ++nt) {
+          const int row = nt * 8 + g;
+          uint32_t b0 = 0, b1 = 0, c0 = 0, c1 = 0;
+          if (row < M) {
+            const size_t off = (size_t)row * ldxs + ko + 2 * t;
+            b0 = *reinterpret_cast<const uint32_t*>(xs + off);
+            b1 = *reinterpret_cast<const uint32_t*>(xs + off + 8);
+            if (LO) {
+              c0 = *reinterpret_cast<const uint32_t*>(xl + off);
+              c1 = *reinterpret_cast<const uint32_t*>(xl + off + 8);
             }
-            mma_f16_16816(tmp[nt], af, b0, b1);
-            if (LO) mma_f16_16816(tmp[nt], af, c0, c1);
           }
-        }
-        const float2 s = h2_to_f2(sv.x);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          acc[nt][0] = fmaf(s.x, tmp[nt][0], acc[nt][0]);
-          acc[nt][1] = fmaf(s.x, tmp[nt][1], acc[nt][1]);
-          acc[nt][2] = fmaf(s.y, tmp[nt][2], acc[nt][2]);
-          acc[nt][3] = fmaf(s.y, tmp[nt][3], acc[nt][3]);
+          mma_f16_16816(tmp[nt], af, b0, b1);
+          if (LO) mma_f16_16816(tmp[nt], af, c0, c1);
         }
       }
+    }
+    const float2 s = h2_to_f2(sv.x);
+#pragma unroll
+    for (int nt = 0; nt < NTILES; ++nt) {
+      acc[nt][0] = fmaf(s.x, tmp[nt][0], acc[nt][0]);
+      acc[nt][1] = fmaf(s.x, tmp[nt][1], acc[nt][1]);
+      acc[nt][2] = fmaf(s.y, tmp[nt][2], acc[nt][2]);
+      acc[nt][3] = fmaf(s.y, tmp[nt][3], acc[nt][3]);
     }
   }
 
   // ---- reduce the K slices (fixed order) ---------------------------------
   float* myred = red + (kq * TPC + tsel) * 16 * NC;
+  if (NT == 0 && LO) {  // columns (2m, 2m+1) = (hi, lo) parts of row m = t
+    myred[g * NC + t] = acc[0][0] + acc[0][1];
+    myred[(g + 8) * NC + t] = acc[0][2] + acc[0][3];
+  } else {
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const int col = nt * 8 + 2 * t;
-    myred[g * NC + col] = acc[nt][0];
-    myred[g * NC + col + 1] = acc[nt][1];
-    myred[(g + 8) * NC + col] = acc[nt][2];
-    myred[(g + 8) * NC + col + 1] = acc[nt][3];
+    for (int nt = 0; nt < NTILES; ++nt) {
+      const int col = nt * 8 + 2 * t;
+      myred[g * NC + col] = acc[nt][0];
+      myred[g * NC + col + 1] = acc[nt][1];
+      myred[(g + 8) * NC + col] = acc[nt][2];
+      myred[(g + 8) * NC + col + 1] = acc[nt][3];
+    }
   }
   __syncthreads();
 
   const int r = threadIdx.x & 15, m = threadIdx.x >> 4;
-  if (m >= a.M || m >= NC) return;
+  if (m >= M || m >= NC) return;
   float va = 0.f, vb = 0.f;
 #pragma unroll
   for (int q = 0; q < KS; ++q) {
@@ -295,12 +337,12 @@ __global__ void __launch_bounds__(kGemvThreads, 3) gemv_int4_kernel(const GemvAr
     const int j = row0 % hd;
     const RowCtx rc = a.rows[m];
     if (row0 < a.n_q_rows) {
-      const float2 cs = rope_cos_sin(rc.pos, j, hd, a.theta);
+      const float2 cs = rope_cs(a.rope_tab, rc.pos, j, hd, a.theta);
       float* qo = a.q_out + (size_t)m * a.ldq;
       qo[row0] = va * cs.x - vb * cs.y;
       qo[row1] = vb * cs.x + va * cs.y;
     } else if (row0 < a.n_q_rows + a.n_kv_rows) {
-      const float2 cs = rope_cos_sin(rc.pos, j, hd, a.theta);
+      const float2 cs = rope_cs(a.rope_tab, rc.pos, j, hd, a.theta);
       const int kvh = (row0 - a.n_q_rows) / hd;
       __half* dst = a.k_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
       dst[j] = __float2half_rn(va * cs.x - vb * cs.y);

@@ -55,6 +55,13 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const __half* __rest
   }
 }
 
+// ---- RoPE table of a model: (cos, sin) [positions][hd/2] --------------------
+__global__ void rope_table_kernel(float2* tab, int n_pos, int hd, float theta) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const int half = hd >> 1;
+  if (i < n_pos * half) tab[i] = rope_cos_sin(i / half, i % half, hd, theta);
+}
+
 // ---- RoPE in place: one thread per (token, head, pair) ---------------------
 __global__ void rope_inplace_kernel(__half* x, int n_tokens, int n_heads, int hd,
                                     long long token_stride, long long head_stride,
@@ -123,93 +130,110 @@ struct HeadArgs {
   int* err_flag;        // device fault flags
 };
 
-constexpr int kHeadThreads = 256;
-constexpr int kHeadChunk = 4096;   // bytes per bulk copy: 8 k16-tiles of one 16-row tile
+constexpr int kHeadWarps = 8;                      // compute warps
+constexpr int kHeadThreads = (kHeadWarps + 1) * 32;  // + one producer warp
+constexpr int kHeadStageMax = 16384;                  // bytes per bulk-copy stage
+constexpr size_t kHeadSmemBudget = 200 * 1024;
 
 __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-// Ring stages per warp: deeper when the activation planes are small.
-__host__ __device__ inline int head_stages(int M) { return M <= 8 ? 4 : 2; }
-
-// Dynamic shared memory: per-warp rings, then the activation planes (hi, lo).
+// Stage size: 16 KB, or one whole row tile when the tile is smaller.
+__host__ __device__ inline int head_stage_bytes(int d) {
+  const int tile = (d / 16) * 512;
+  return tile < kHeadStageMax ? tile : kHeadStageMax;
+}
+__host__ __device__ inline size_t head_act_bytes(int d, int M) { return (size_t)M * (d + 8) * 2 * 2; }
+__host__ __device__ inline int head_stages(int d, int M) {
+  const size_t rest = kHeadSmemBudget - head_act_bytes(d, M);
+  int s = (int)(rest / head_stage_bytes(d));
+  return s > 12 ? 12 : s;
+}
+// Dynamic shared memory: the stage ring, the activation planes (hi, lo), the
+// cross-warp reduction buffer.
 __host__ __device__ inline size_t head_smem_bytes(int d, int M) {
-  return (size_t)8 * head_stages(M) * kHeadChunk + (size_t)M * (d + 8) * 2 * 2;
+  return (size_t)head_stages(d, M) * head_stage_bytes(d) + head_act_bytes(d, M) +
+         (size_t)kHeadWarps * 16 * 16 * 4;
 }
 
-// One CTA per SM.  Global warp w takes 16-row tiles w, w + W, w + 2W, ...
-// (W = warps in the grid) over all of K.  Its tiles stream through a private
-// ring of S shared-memory stages, each filled by one 4 KB bulk asynchronous
-// copy (the TMA engine) that completes on an mbarrier, so a warp keeps S * 4 KB
-// in flight without spending registers on it; the first copies are issued
-// before griddepcontrol.wait.  The output norm is computed by every CTA in the
-// prologue and kept as an fp16 pair (hi, lo) like the INT4 GEMV's activations.
-// Each warp keeps its best (value, index) per row; CTAs combine warps, and the
-// last CTA to finish (atomic ticket) combines CTAs.  Ties go to the lowest
-// index, so the result does not depend on the order of combination.  Every
-// wait is bounded: on time-out the kernel sets kErrTimeout and stops.
+// One CTA per SM takes a contiguous range of 16-row tiles (balanced to +-1
+// tile).  A producer warp streams the range through a ring of shared-memory
+// stages with bulk asynchronous copies (the TMA engine), so up to ~190 KB per
+// SM is in flight without spending registers; the first stages are requested
+// before griddepcontrol.wait.  The 8 compute warps split each stage along K
+// (MMA with the fp16 pair of the normalised activations) and combine at the
+// end of every tile through shared memory, in warp order.  The output norm is
+// computed by every CTA in the prologue.  Each row keeps its best (value,
+// index); the last CTA to finish (atomic ticket) combines the CTAs.  Ties go
+// to the lowest index.  Every wait is bounded (kErrTimeout on give-up).
 template <int NT>
 __global__ void __launch_bounds__(kHeadThreads, 1) head_argmax_kernel(const HeadArgs a) {
-  constexpr int S = NT == 1 ? 4 : 2;
+  constexpr int NC = NT * 8;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ __align__(8) uint64_t bars[8][4];
-  __shared__ float s_val[8][16];
-  __shared__ int s_idx[8][16];
-  __shared__ float s_ss[16][8];
-  __shared__ int s_last;
+  __shared__ __align__(8) uint64_t full[12], empty[12];
+  __shared__ float s_ss[16][kHeadWarps];
+  __shared__ float s_val[16][16];
+  __shared__ int s_idx[16][16];
+  __shared__ int s_last, s_fail;
   const int d = a.d, ldxs = d + 8, M = a.M;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  unsigned char* ring = smem + (size_t)warp * S * kHeadChunk;
-  __half* xs = reinterpret_cast<__half*>(smem + (size_t)8 * S * kHeadChunk);
-  __half* xl = xs + (size_t)M * ldxs;
-  const int n_tiles = a.V >> 4;
+  const int SB = head_stage_bytes(d);
+  const int S = head_stages(d, M);
   const int nk = d >> 4;                      // k16-tiles per row tile
-  const int cpt = nk / 8;                     // 4 KB chunks per row tile
-  const int GW = gridDim.x * 8;
-  const int gw = blockIdx.x * 8 + warp;
-  const int my_tiles = gw < n_tiles ? (n_tiles - 1 - gw) / GW + 1 : 0;
-  const int nf = my_tiles * cpt;              // chunks this warp streams
-  uint64_t* bar = bars[warp];
-  auto chunk_src = [&](int f) {
-    const int tile = gw + (f / cpt) * GW;
-    return reinterpret_cast<const unsigned char*>(a.w) + ((size_t)tile * cpt + (f % cpt)) * kHeadChunk;
-  };
+  const int spt = (nk * 512) / SB;            // stages per row tile
+  const int k16_per_stage = SB / 512;
+  const int k16_per_warp = k16_per_stage / kHeadWarps;
+  unsigned char* ring = smem;
+  __half* xs = reinterpret_cast<__half*>(smem + (size_t)S * SB);
+  __half* xl = xs + (size_t)M * ldxs;
+  float* red = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(xs) + head_act_bytes(d, M));
+  const int n_tiles = a.V >> 4;
+  const int tb = (int)((long)blockIdx.x * n_tiles / gridDim.x);
+  const int te = (int)((long)(blockIdx.x + 1) * n_tiles / gridDim.x);
+  const int nf = (te - tb) * spt;             // stages this CTA streams
 
   pdl_trigger();
-  if (lane == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&bar[s], 1);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kHeadWarps);
+    }
     fence_mbar_init();
-    for (int s = 0; s < S && s < nf; ++s) {
-      mbar_arrive_expect_tx(&bar[s], kHeadChunk);
-      bulk_g2s(ring + s * kHeadChunk, chunk_src(s), kHeadChunk, &bar[s]);
+    s_fail = 0;
+  }
+  __syncthreads();
+  const unsigned char* wsrc = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tb * spt * SB;
+  if (warp == kHeadWarps && lane == 0) {  // first stages before the dependency wait
+    for (int f = 0; f < S && f < nf; ++f) {
+      mbar_arrive_expect_tx(&full[f], SB);
+      bulk_g2s(ring + (size_t)f * SB, wsrc + (size_t)f * SB, SB, &full[f]);
     }
   }
-  __syncwarp();
   pdl_wait();
 
   // output RMSNorm of every row into shared memory as an fp16 pair
   for (int m = 0; m < M; ++m) {
     const float* src = a.x + (size_t)m * d;
     float ss = 0.f;
-#pragma unroll 4
-    for (int k = threadIdx.x * 4; k < d; k += 4 * kHeadThreads) {
-      const float4 v = *reinterpret_cast<const float4*>(src + k);
-      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    if (warp < kHeadWarps) {
+      for (int k = threadIdx.x * 4; k < d; k += 4 * kHeadWarps * 32) {
+        const float4 v = *reinterpret_cast<const float4*>(src + k);
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) s_ss[m][warp] = ss;
     }
-    ss = warp_sum(ss);
-    if (lane == 0) s_ss[m][warp] = ss;
   }
   __syncthreads();
-  for (int m = 0; m < M; ++m) {
+  for (int m = 0; m < M && warp < kHeadWarps; ++m) {
     const float* src = a.x + (size_t)m * d;
     float ss = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) ss += s_ss[m][w];
+    for (int w = 0; w < kHeadWarps; ++w) ss += s_ss[m][w];
     const float rs = 1.0f / sqrtf(ss / (float)d + a.eps);
-#pragma unroll 4
-    for (int k = threadIdx.x * 4; k < d; k += 4 * kHeadThreads) {
+    for (int k = threadIdx.x * 4; k < d; k += 4 * kHeadWarps * 32) {
       float4 v = *reinterpret_cast<const float4*>(src + k);
       const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
       const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k + 2));
@@ -225,107 +249,104 @@ __global__ void __launch_bounds__(kHeadThreads, 1) head_argmax_kernel(const Head
   }
   __syncthreads();
 
-  float acc[NT][4];
-  float bv[NT][2];
-  int bi[NT][2];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-    bv[nt][0] = bv[nt][1] = -INFINITY;
-    bi[nt][0] = bi[nt][1] = 0x7fffffff;
-  }
-
   float* const logits = a.io ? a.io->logits : a.logits;
   int32_t* const argmax = a.io ? a.io->argmax : a.argmax;
-  bool ok = true;
-  for (int f = 0; f < nf && ok; ++f) {
-    const int s = f % S;
-    if (!mbar_wait(&bar[s], (unsigned)((f / S) & 1))) {
-      ok = false;
-      if (lane == 0) atomicOr(a.err_flag, kErrTimeout);
-      break;
-    }
-    const unsigned char* stage = ring + s * kHeadChunk;
-    const int kk0 = (f % cpt) * 8;   // first k16-tile of this chunk within the row tile
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(stage + (j * 32 + lane) * 16);
-      const uint32_t af[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const int row = nt * 8 + g;
-        uint32_t b0 = 0, b1 = 0, c0 = 0, c1 = 0;
-        if (row < M) {
-          const size_t off = (size_t)row * ldxs + (kk0 + j) * 16 + 2 * t;
-          b0 = *reinterpret_cast<const uint32_t*>(xs + off);
-          b1 = *reinterpret_cast<const uint32_t*>(xs + off + 8);
-          c0 = *reinterpret_cast<const uint32_t*>(xl + off);
-          c1 = *reinterpret_cast<const uint32_t*>(xl + off + 8);
-        }
-        mma_f16_16816(acc[nt], af, b0, b1);
-        mma_f16_16816(acc[nt], af, c0, c1);
-      }
-    }
-    __syncwarp();
-    if (lane == 0 && f + S < nf) {  // refill this stage
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&bar[s], kHeadChunk);
-      bulk_g2s(ring + s * kHeadChunk, chunk_src(f + S), kHeadChunk, &bar[s]);
-    }
-    if ((f + 1) % cpt == 0) {  // row tile done: logits and running best
-      const int tile = gw + (f / cpt) * GW;
-      const int ra = tile * 16 + g, rb = ra + 8;
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int m = nt * 8 + 2 * t + c;
-          const float va = acc[nt][c], vb = acc[nt][2 + c];
-          if (m < M && logits) {
-            const int orow = a.out_row ? a.out_row[m] : m;
-            logits[(size_t)orow * a.V + ra] = va;
-            logits[(size_t)orow * a.V + rb] = vb;
-          }
-          if (better(va, ra, bv[nt][c], bi[nt][c])) { bv[nt][c] = va; bi[nt][c] = ra; }
-          if (better(vb, rb, bv[nt][c], bi[nt][c])) { bv[nt][c] = vb; bi[nt][c] = rb; }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) acc[nt][q] = 0.f;
-      }
-    }
-  }
-  if (!ok) {  // drain the copies still in flight (bounded), then stop
-    if (lane == 0)
-      for (int s = 0; s < S; ++s) (void)mbar_try_wait(&bar[s], 0);
-    return;
-  }
 
-  // best per row across the lanes of the warp, then across warps
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      float v = bv[nt][c];
-      int ix = bi[nt][c];
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, ix, o);
-        if (better(ov, oi, v, ix)) { v = ov; ix = oi; }
+  if (warp == kHeadWarps) {
+    // ---- producer: refill each stage once all compute warps released it ----
+    if (lane == 0) {
+      int s = 0;
+      unsigned par = 0;   // parity of the release being waited for
+      for (int f = S; f < nf; ++f) {
+        if (!mbar_wait_or_fail(&empty[s], par, &s_fail)) break;
+        mbar_arrive_expect_tx(&full[s], SB);
+        bulk_g2s(ring + (size_t)s * SB, wsrc + (size_t)f * SB, SB, &full[s]);
+        if (++s == S) { s = 0; par ^= 1u; }
       }
-      if (g == 0) { s_val[warp][nt * 8 + 2 * t + c] = v; s_idx[warp][nt * 8 + 2 * t + c] = ix; }
     }
+  } else {
+    // ---- compute warps ------------------------------------------------------
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+    // rows of the logits this thread finalises: (r, m) = (tid % 16, tid / 16)
+    const int fr = threadIdx.x & 15, fm = threadIdx.x >> 4;
+    float best_v = -INFINITY;
+    int best_i = 0x7fffffff;
+    int s = 0, part = 0, tile = tb;
+    unsigned par = 0;
+    for (int f = 0; f < nf; ++f) {
+      // on a time-out the loop keeps its shape (no further waits) so the
+      // tile-end barriers below still match across the compute warps
+      mbar_wait_or_fail(&full[s], par, &s_fail);
+      const unsigned char* stage = ring + (size_t)s * SB;
+      for (int jj = 0; jj < k16_per_warp; ++jj) {
+        const int j = warp * k16_per_warp + jj;          // k16-tile within the stage
+        const int kk = part * k16_per_stage + j;         // k16-tile within the row tile
+        const uint4 wv = *reinterpret_cast<const uint4*>(stage + (size_t)(j * 32 + lane) * 16);
+        const uint32_t af[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int row = nt * 8 + g;
+          uint32_t b0 = 0, b1 = 0, c0 = 0, c1 = 0;
+          if (row < M) {
+            const size_t off = (size_t)row * ldxs + kk * 16 + 2 * t;
+            b0 = *reinterpret_cast<const uint32_t*>(xs + off);
+            b1 = *reinterpret_cast<const uint32_t*>(xs + off + 8);
+            c0 = *reinterpret_cast<const uint32_t*>(xl + off);
+            c1 = *reinterpret_cast<const uint32_t*>(xl + off + 8);
+          }
+          mma_f16_16816(acc[nt], af, b0, b1);
+          mma_f16_16816(acc[nt], af, c0, c1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      if (++s == S) { s = 0; par ^= 1u; }
+      if (part == spt - 1) {  // row tile done: combine the warps, logits, best
+        float* myred = red + warp * 16 * 16;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int col = nt * 8 + 2 * t;
+          myred[g * 16 + col] = acc[nt][0];
+          myred[g * 16 + col + 1] = acc[nt][1];
+          myred[(g + 8) * 16 + col] = acc[nt][2];
+          myred[(g + 8) * 16 + col + 1] = acc[nt][3];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(kHeadWarps * 32) : "memory");
+        if (fm < M && fm < NC) {
+          float v = 0.f;
+#pragma unroll
+          for (int w = 0; w < kHeadWarps; ++w) v += red[w * 256 + fr * 16 + fm];
+          const int row = tile * 16 + fr;
+          if (logits) logits[(size_t)(a.out_row ? a.out_row[fm] : fm) * a.V + row] = v;
+          if (better(v, row, best_v, best_i)) { best_v = v; best_i = row; }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(kHeadWarps * 32) : "memory");
+        part = 0;
+        ++tile;
+      } else {
+        ++part;
+      }
+    }
+    if (fm < 16) { s_val[fm][fr] = best_v; s_idx[fm][fr] = best_i; }
   }
   __syncthreads();
-
+  if (s_fail) {
+    if (threadIdx.x == 0) atomicOr(a.err_flag, kErrTimeout);
+    return;
+  }
   if (!argmax) return;
   if (threadIdx.x < M) {
     const int m = threadIdx.x;
-    float v = s_val[0][m];
-    int ix = s_idx[0][m];
-    for (int w = 1; w < 8; ++w)
-      if (better(s_val[w][m], s_idx[w][m], v, ix)) { v = s_val[w][m]; ix = s_idx[w][m]; }
+    float v = s_val[m][0];
+    int ix = s_idx[m][0];
+    for (int r = 1; r < 16; ++r)
+      if (better(s_val[m][r], s_idx[m][r], v, ix)) { v = s_val[m][r]; ix = s_idx[m][r]; }
     a.part_val[blockIdx.x * 16 + m] = v;
     a.part_idx[blockIdx.x * 16 + m] = ix;
   }

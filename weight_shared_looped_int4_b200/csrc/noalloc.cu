@@ -65,7 +65,7 @@ cudaError_t allow_attn_smem() {
 #define A(HD, REP)                                                                               \
   if (e == cudaSuccess)                                                                          \
     e = cudaFuncSetAttribute(decode_attn_kernel<HD, REP, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                             (int)decode_attn_smem_bytes(HD));
+                             (int)decode_attn_smem_bytes(HD, REP));
   A(64, 1) A(64, 2) A(64, 4) A(64, 8) A(128, 1) A(128, 2) A(128, 4) A(128, 8)
 #undef A
   return e;
@@ -93,7 +93,7 @@ tl_status scratch_address(void** out) {
 
 template <int HD, int REP>
 cudaError_t launch_attn(const DecodeAttnArgs& a, int rows, cudaStream_t st) {
-  decode_attn_kernel<HD, REP, false><<<dim3(kDecodeMaxSplits, a.Hkv, rows), kDecodeThreads, decode_attn_smem_bytes(HD), st>>>(a);
+  decode_attn_kernel<HD, REP, false><<<dim3(kDecodeMaxSplits, a.Hkv, rows), kDecodeThreads, decode_attn_smem_bytes(HD, REP), st>>>(a);
   return cudaGetLastError();
 }
 

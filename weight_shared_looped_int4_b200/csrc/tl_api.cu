@@ -175,10 +175,9 @@ cudaError_t init_device_kernels(int dev) {
   cudaError_t e = cudaSuccess;
 #define SET(NT, IN, EPI) \
   if (e == cudaSuccess) e = set_gemv_attr<NT, IN, EPI>(dev);
-  SET(1, IN_F16, EPI_STORE) SET(2, IN_F16, EPI_STORE)
-  SET(1, IN_F32, EPI_RESID) SET(2, IN_F32, EPI_RESID)
-  SET(1, IN_NORM, EPI_SWIGLU) SET(2, IN_NORM, EPI_SWIGLU)
-  SET(1, IN_NORM, EPI_ROPE_KV) SET(2, IN_NORM, EPI_ROPE_KV)
+#define SET3(IN, EPI) SET(0, IN, EPI) SET(1, IN, EPI) SET(2, IN, EPI)
+  SET3(IN_F16, EPI_STORE) SET3(IN_F32, EPI_RESID) SET3(IN_NORM, EPI_SWIGLU) SET3(IN_NORM, EPI_ROPE_KV)
+#undef SET3
 #undef SET
   if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<1>, dev);
   if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<2>, dev);
@@ -198,22 +197,22 @@ cudaError_t init_device_kernels(int dev) {
 }
 
 // Largest activation-row count (<= 16) per GEMV launch that fits shared memory.
-int gemv_rows_per_launch(int K, bool lo) {
+int gemv_rows_per_launch(int K, bool lo, int tpc) {
   int M = kMaxLanes;
-  while (M > 0 && gemv_smem_bytes(K, M, lo) > kMaxDynSmem) --M;
+  while (M > 0 && gemv_smem_bytes(K, M, lo, tpc) > kMaxDynSmem) --M;
   return M;
 }
 
 cudaError_t launch_gemv(const GemvArgs& a, int grid, int in_mode, int epi, cudaStream_t st) {
-  const int nt = a.M <= 8 ? 1 : 2;
-  const size_t smem = gemv_smem_bytes(a.K, a.M, in_mode != IN_F16);
+  const bool lo = in_mode != IN_F16;
+  const int nt = gemv_nt(a.M, lo);
+  const size_t smem = gemv_smem_bytes(a.K, a.M, lo, gemv_tpc(epi));
   const dim3 g(grid), b(kGemvThreads);
 #define CASE(NT, IN, EPI) \
   if (nt == NT && in_mode == IN && epi == EPI) return launch(gemv_int4_kernel<NT, IN, EPI>, g, b, smem, st, a);
-  CASE(1, IN_F16, EPI_STORE) CASE(2, IN_F16, EPI_STORE)
-  CASE(1, IN_F32, EPI_RESID) CASE(2, IN_F32, EPI_RESID)
-  CASE(1, IN_NORM, EPI_SWIGLU) CASE(2, IN_NORM, EPI_SWIGLU)
-  CASE(1, IN_NORM, EPI_ROPE_KV) CASE(2, IN_NORM, EPI_ROPE_KV)
+#define CASE3(IN, EPI) CASE(0, IN, EPI) CASE(1, IN, EPI) CASE(2, IN, EPI)
+  CASE3(IN_F16, EPI_STORE) CASE3(IN_F32, EPI_RESID) CASE3(IN_NORM, EPI_SWIGLU) CASE3(IN_NORM, EPI_ROPE_KV)
+#undef CASE3
 #undef CASE
   return cudaErrorInvalidValue;
 }
@@ -221,7 +220,7 @@ cudaError_t launch_gemv(const GemvArgs& a, int grid, int in_mode, int epi, cudaS
 // Launch a GEMV over `total` activation rows, in chunks of as many rows as
 // fit shared memory; every row-indexed pointer advances with the chunk.
 cudaError_t launch_gemv_rows(GemvArgs a, int total, int in_mode, int epi, int grid, cudaStream_t st) {
-  const int per = gemv_rows_per_launch(a.K, in_mode != IN_F16);
+  const int per = gemv_rows_per_launch(a.K, in_mode != IN_F16, gemv_tpc(epi));
   if (per < 1) return cudaErrorInvalidValue;
   for (int r0 = 0; r0 < total; r0 += per) {
     GemvArgs c = a;
@@ -456,7 +455,7 @@ cudaError_t launch_tc_linear(const uint4* w, const uint2* sz, int K, int N, int 
 
 template <int HD, int REP, bool F32>
 cudaError_t launch_decode_attn_t(const DecodeAttnArgs& a, int rows, cudaStream_t st) {
-  return launch(decode_attn_kernel<HD, REP, F32>, dim3(kDecodeMaxSplits, a.Hkv, rows), dim3(kDecodeThreads), decode_attn_smem_bytes(HD),
+  return launch(decode_attn_kernel<HD, REP, F32>, dim3(kDecodeMaxSplits, a.Hkv, rows), dim3(kDecodeThreads), decode_attn_smem_bytes(HD, REP),
                 st, a);
 }
 
@@ -519,6 +518,7 @@ struct tl_model {
   cudaAccessPolicyWindow loop_window = {};  // keeps the loop block's weights in L2
   size_t l2_persist_bytes = 0;
   float* gu = nullptr;           // raw gate_up output of the prefill [rows][2F]
+  float2* rope_tab = nullptr;    // RoPE (cos, sin) [max_ctx][hd/2]
   cudaStream_t setup_stream = nullptr;
   cudaStream_t cap_stream = nullptr;   // stream used to capture decode graphs
   struct Graph {
@@ -526,6 +526,7 @@ struct tl_model {
     int kernels = 0;
   };
   std::map<std::string, Graph> graphs;   // decode step graphs by row pattern
+  bool use_graphs = true;
   std::vector<int> lane_len, lane_loops;
   size_t weight_bytes = 0, kv_bytes = 0, ws_bytes = 0;
   Profiler prof;
@@ -544,7 +545,8 @@ struct tl_model {
     graphs.clear();
     if (cap_stream) cudaStreamDestroy(cap_stream);
     void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row,
-                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.partial, tc.tickets, gu};
+                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.partial, tc.tickets, gu,
+                    rope_tab};
     for (void* p : ptrs)
       if (p) cudaFree(p);
     if (setup_stream) cudaStreamDestroy(setup_stream);
@@ -622,6 +624,8 @@ tl_status run_qkv(tl_model* m, int layer, int M, float* x, const RowCtx* rows, f
   a.q_out = q; a.ldq = qdim; a.n_q_rows = qdim; a.n_kv_rows = c.n_kv_heads * hd;
   a.k_plane = m->k_plane(layer); a.v_plane = m->v_plane(layer);
   a.lane_stride = m->lane_stride; a.ctx = c.max_ctx;
+  a.rope_tab = m->rope_tab;
+  a.err_flag = m->err_flag;
   kclass(TL_KERNEL_QKV);
   TL_CUDA(launch_gemv_rows(a, M, IN_NORM, EPI_ROPE_KV, (c.n_q_heads + 2 * c.n_kv_heads) * hd / 32, st));
   return TL_OK;
@@ -656,6 +660,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   a.x = o; a.ldx = qdim;
   a.pair_mode = PAIR_NEIGHBOUR;
   a.resid = x; a.ldr = d;
+  a.err_flag = m->err_flag;
   kclass(TL_KERNEL_O_PROJ);
   TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, (b.o.N + 15) / 16, st));
   GemvArgs g{};
@@ -664,6 +669,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   g.x = x; g.ldx = d; g.gain = b.ffn_norm;
   g.pair_mode = PAIR_OFFSET; g.pair_off = F / 16;
   g.yf = h; g.ldy = F;
+  g.err_flag = m->err_flag;
   kclass(TL_KERNEL_GATE_UP);
   TL_CUDA(launch_gemv_rows(g, M, IN_NORM, EPI_SWIGLU, F / 16, st));
   GemvArgs dn{};
@@ -671,6 +677,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   dn.x = h; dn.ldx = F;
   dn.pair_mode = PAIR_NEIGHBOUR;
   dn.resid = x; dn.ldr = d;
+  dn.err_flag = m->err_flag;
   kclass(TL_KERNEL_DOWN);
   TL_CUDA(launch_gemv_rows(dn, M, IN_F32, EPI_RESID, (b.down.N + 15) / 16, st));
   return TL_OK;
@@ -689,7 +696,7 @@ tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, cudaStream_t st) {
   ta.q_out = m->q; ta.ldq = qdim; ta.n_q_rows = qdim; ta.n_kv_rows = c.n_kv_heads * hd; ta.hd = hd;
   ta.k_plane = m->k_plane(layer) + lane * m->lane_stride;
   ta.v_plane = m->v_plane(layer) + lane * m->lane_stride;
-  ta.ctx = c.max_ctx; ta.pos0 = 0; ta.theta = c.rope_theta;
+  ta.ctx = c.max_ctx; ta.pos0 = 0; ta.theta = c.rope_theta; ta.rope_tab = m->rope_tab;
   kclass(TL_KERNEL_GEMM_TC);
   TL_CUDA(launch_tc_linear(b.qkv.w, b.qkv.sz, c.d_model, b.qkv.N, b.qkv.n_tiles, PREP_NORM, pa, ta, TC_ROPE_KV,
                            T, m->tc, st));
@@ -868,8 +875,8 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
   {
     int n_sm = 0;
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n_sm < 1) n_sm = 148;
-    // one CTA of 8 warps per SM, never more warps than head tiles
-    m->head_grid = std::min(n_sm, (c.vocab / 16 + 7) / 8);
+    // one CTA per SM, never more CTAs than head tiles
+    m->head_grid = std::min(n_sm, c.vocab / 16);
     m->tc.n_sm = n_sm;
   }
   size_t ws = 0;
@@ -895,7 +902,13 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     m->tc.err_flag = m->err_flag;
     ok = alloc((void**)&m->tc.bt, m->tc.bt_bytes) && alloc((void**)&m->tc.partial, m->tc.partial_bytes) &&
          alloc((void**)&m->tc.tickets, 4096 * sizeof(unsigned)) &&
-         alloc((void**)&m->gu, (size_t)tok_pad * 2 * c.ffn_dim * 4);
+         alloc((void**)&m->gu, (size_t)tok_pad * 2 * c.ffn_dim * 4) &&
+         alloc((void**)&m->rope_tab, (size_t)c.max_ctx * (hd / 2) * sizeof(float2));
+    if (ok) {
+      const int n = c.max_ctx * (hd / 2);
+      rope_table_kernel<<<(n + 255) / 256, 256, 0, st>>>(m->rope_tab, c.max_ctx, hd, c.rope_theta);
+      ok = cudaGetLastError() == cudaSuccess;
+    }
   }
   if (!ok) return bail(fail(TL_ERR_OOM, "workspace allocation"));
   m->ws_bytes = ws;
@@ -1009,7 +1022,7 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
     }
     return launch_head(m, m->x, n_lanes, m->out_row, nullptr, nullptr, s, m->io);
   };
-  if (m->prof.mask) {  // profiling times every launch: run eagerly
+  if (m->prof.mask || !m->use_graphs) {  // profiling times every launch: run eagerly
     tl_status rc = body(st);
     if (rc != TL_OK) return rc;
   } else {
@@ -1073,6 +1086,12 @@ tl_status tl_model_profile_stop(tl_model* m, int* h_launches, float* h_total_ms)
 }
 
 unsigned long long tl_kernel_launch_count(void) { return g_launches.load(); }
+
+tl_status tl_model_set_graphs(tl_model* m, int enable) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  m->use_graphs = enable != 0;
+  return TL_OK;
+}
 
 tl_status tl_lane_length(const tl_model* m, int lane, int* h_length) {
   if (!m || !h_length) return fail(TL_ERR_INVALID_ARG, "null argument");
@@ -1233,8 +1252,10 @@ tl_status tl_linear_forward(tl_linear* l, const uint16_t* d_x, int M, uint16_t* 
                              (cudaStream_t)stream));
     return TL_OK;
   }
-  if (gemv_rows_per_launch(K, false) < 1) return fail(TL_ERR_UNSUPPORTED, "K too large for the GEMV");
+  if (gemv_rows_per_launch(K, false, gemv_tpc(EPI_STORE)) < 1) return fail(TL_ERR_UNSUPPORTED, "K too large for the GEMV");
   GemvArgs a{};
+  a.err_flag = op_err_flag(l->device);
+  if (!a.err_flag) return fail(TL_ERR_OOM, "op error flag");
   a.w = l->w.w; a.sz = l->w.sz; a.K = K; a.n_rows = N;
   a.xh = reinterpret_cast<const __half*>(d_x); a.ldx = K;
   a.pair_mode = PAIR_NEIGHBOUR;
