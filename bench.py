@@ -57,6 +57,9 @@ BYTES_PER_LAUNCH = {
 }
 
 
+DECODE_PATHS = {"auto": 0, "layered": 1, "fused": 2}
+
+
 def _attn_bytes_per_launch(mean_keys):
     return 2 * HKV * HD * 2 * mean_keys + 2 * HQ * HD * 2
 
@@ -221,6 +224,7 @@ def run_ncu_case(args):
     m = tl.tl_model_create(cfg, tw, 0)
     del keep
     tl.tl_model_set_graphs(m, False)
+    tl.tl_model_set_decode_path(m, DECODE_PATHS[args.decode_path])
     d_prompt = torch.as_tensor(prompt, device="cuda:0")
     hist = torch.zeros(steps + 1, dtype=torch.int32, device="cuda:0")
     hp = hist.data_ptr()
@@ -237,20 +241,86 @@ def run_ncu_case(args):
     return 0
 
 
-def l2_read_probe(dev, mbytes=24, reps=200):
-    """Read bandwidth of an L2-resident buffer (GB/s): torch sum over a tensor
-    the size of the loop block, repeated; a reference for the loop-layer bytes."""
+PHASES = ["qkv", "attention", "o_proj", "gate_up", "down"]
+
+
+def run_trace(args):
+    """Phase timeline (globaltimer) of the single-kernel decode step at the
+    workload's mid-decode context: per phase, the time from the previous
+    barrier's release to the last CTA's arrival (work) and from that arrival
+    to the last release (barrier), averaged over the effective layers."""
     import torch
-    x = torch.ones(mbytes * (1 << 20) // 2, dtype=torch.float16, device=dev)
-    for _ in range(10):
-        x.sum()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(reps):
-        x.sum()
-    b.record()
-    b.synchronize()
-    return x.numel() * 2 * reps / (a.elapsed_time(b) * 1e6)
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    shape = tl_synth.LOOPED_LM
+    w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM)
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, shape.vocab, PROMPT + 1)
+    cfg = tl.make_config(shape, max_loops=LOOPS, max_ctx=PROMPT + 64, max_lanes=1)
+    tw, keep = tl.make_weights(w)
+    m = tl.tl_model_create(cfg, tw, 0)
+    del keep
+    tl.tl_model_set_decode_path(m, DECODE_PATHS["fused"])
+    d_prompt = torch.as_tensor(prompt, device="cuda:0")
+    tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS)
+    G = tl.tl_model_trace_grid(m)
+    n_bar = 5 * (2 + LOOPS)
+    buf = torch.zeros((4 + 5 * n_bar) * G, dtype=torch.int64, device="cuda:0")
+    tok = torch.zeros(2, dtype=torch.int32, device="cuda:0")
+    tok[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
+    for i in range(8):   # warm, then keep the last step's timeline
+        if i == 7:
+            tl.tl_model_set_trace(m, buf, buf.numel())
+        tl.tl_decode_step(m, [0], tok, [LOOPS], None, tok)
+    torch.cuda.synchronize()
+    tl.tl_check_device_error(m)
+    tl.tl_model_destroy(m)
+    t = buf.cpu().numpy().reshape(-1, G).astype(np.float64)
+    t0 = t[0].min()
+    t = (t - t0) / 1e3   # us from the first CTA's start
+    slot = lambda s: t[s]
+    stats = {p: ({"load": [], "scores": [], "softmax_pv": [], "finish": []} if p == "attention" else
+                 {"stage": [], "first_weights_wait": [], "items": [], "epilogue": []}) for p in PHASES}
+    for p in PHASES:
+        stats[p].update({"work_max": [], "work_median": []})
+    barrier = []
+    prev = slot(0)
+    for k in range(n_bar):
+        p = PHASES[k % 5]
+        arr, rel = slot(1 + 5 * k), slot(2 + 5 * k)
+        st = stats[p]
+        st["work_max"].append(float(arr.max() - prev.max()))
+        st["work_median"].append(float(np.median(arr - prev)))
+        if p == "attention":
+            ld, sc_, pv = slot(3 + 5 * k), slot(4 + 5 * k), slot(5 + 5 * k)
+            has = ld > 0   # CTAs with an attention unit
+            st["load"].append(float(np.median((ld - prev)[has])))
+            st["scores"].append(float(np.median((sc_ - ld)[has])))
+            st["softmax_pv"].append(float(np.median((pv - sc_)[has])))
+            st["finish"].append(float(np.median((arr - pv)[has])))
+        else:
+            staged, ready, done = slot(3 + 5 * k), slot(4 + 5 * k), slot(5 + 5 * k)
+            has = ready > 0   # CTAs with weight items in this phase
+            st["stage"].append(float(np.median((staged - prev)[has])))
+            st["first_weights_wait"].append(float(np.median(np.maximum(ready - staged, 0)[has])))
+            st["items"].append(float(np.median((done - np.maximum(ready, staged))[has])))
+            st["epilogue"].append(float(np.median((arr - done)[has])))
+        barrier.append(float(rel.max() - arr.max()))
+        prev = rel
+    hs, hd_, end = slot(1 + 5 * n_bar), slot(2 + 5 * n_bar), slot(3 + 5 * n_bar)
+    mean = lambda v: round(statistics.mean(v), 2) if v else None
+    out = {"trace": "single-kernel decode step, LM L=8, context %d" % (PROMPT + 8), "grid": G,
+           "total_us": round(float(end.max()), 2),
+           "start_skew_us": round(float(t[0].max()), 2),
+           "per_layer_us": {p: {k: mean(v) for k, v in st.items()} for p, st in stats.items()},
+           "barrier_us_mean": round(statistics.mean(barrier), 3),
+           "barrier_us_max": round(max(barrier), 3),
+           "head_us": {"stage": round(float(np.median(hs - prev)), 2),
+                       "tiles_median": round(float(np.median(hd_ - hs)), 2),
+                       "tiles_max": round(float((hd_ - hs).max()), 2),
+                       "total": round(float(end.max() - prev.max()), 2)},
+           "layers": 2 + LOOPS, "barriers": n_bar}
+    print(json.dumps(out))
+    return 0
 
 
 def run_ours(args):
@@ -280,6 +350,7 @@ def run_ours(args):
     del keep
     if args.no_graphs:
         tl.tl_model_set_graphs(m, False)
+    tl.tl_model_set_decode_path(m, DECODE_PATHS[args.decode_path])
 
     st = torch.cuda.Stream(device=dev)
     d_prompt = torch.as_tensor(prompt, device=dev)
@@ -354,10 +425,27 @@ def run_ours(args):
     if e2e_ms:
         assert np.array_equal(h_out.numpy(), generated), "end-to-end run diverged from the timed run"
 
-    # ---- per-kernel profile of one decode phase (separate from the timing) -
+    # ---- per-token byte roofline ------------------------------------------
+    # HBM bytes (pre blocks, head, KV reads) at the measured HBM copy bandwidth
+    # + the loop block's re-reads (L2-resident) at the measured L2 read
+    # bandwidth (library probe over a buffer the size of the loop block).
     peaks = load_peaks()
-    per_class, roofline = {}, None
     mean_keys = PROMPT + (n_dec + 1) / 2
+    layer_bytes = sum(BYTES_PER_LAUNCH[k] for k in ("qkv", "o_proj", "gate_up", "down"))
+    hbm_bytes = 2 * layer_bytes + BYTES_PER_LAUNCH["head"] + 10 * _attn_bytes_per_launch(mean_keys)
+    l2_bytes = LOOPS * layer_bytes
+    probe = torch.empty(24 << 20, dtype=torch.uint8, device=dev)
+    l2_gbs = tl.tl_probe_read_bandwidth(probe, probe.numel(), 2000, st)
+    del probe
+    t_roof_us = hbm_bytes / (peaks["hbm_gbs"] * 1e3) + l2_bytes / (l2_gbs * 1e3)
+    t_tok_us = 1e3 * decode_sum / (args.steps * n_dec)
+    roof_step = {"hbm_bytes_per_token": int(hbm_bytes), "l2_bytes_per_token": int(l2_bytes),
+                 "hbm_gbs": peaks["hbm_gbs"], "l2_read_gbs_measured": round(l2_gbs, 1),
+                 "roofline_us_per_token": round(t_roof_us, 2),
+                 "achieved_us_per_token": round(t_tok_us, 2), "frac": round(t_roof_us / t_tok_us, 4)}
+
+    # ---- per-kernel profile of one decode phase (separate from the timing) -
+    per_class, roofline = {}, None
     if not args.no_profile:
         with torch.cuda.stream(st):
             tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS, None, None, st)
@@ -367,36 +455,41 @@ def run_ours(args):
             for i in range(n_dec):
                 tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1), st)
             prof = tl.tl_model_profile_stop(m)
+        step_bytes = hbm_bytes + l2_bytes
+
+        def bytes_of(name):
+            if name == "attn_decode":
+                return _attn_bytes_per_launch(mean_keys)
+            if name == "decode_fused":
+                return step_bytes
+            return BYTES_PER_LAUNCH.get(name)
+
         for name, (n, ms) in prof.items():
             avg_us = 1e3 * ms / n
-            b = BYTES_PER_LAUNCH.get(name)
-            if name == "attn_decode":
-                b = _attn_bytes_per_launch(mean_keys)
+            b = bytes_of(name)
             per_class[name] = {"launches": n, "total_ms": round(ms, 4), "avg_us": round(avg_us, 3),
                                "gbs": round(b / (avg_us * 1e3), 1) if b else None}
         dom = max(per_class, key=lambda k: per_class[k]["total_ms"])
-        dom_b = BYTES_PER_LAUNCH.get(dom) or (_attn_bytes_per_launch(mean_keys) if dom == "attn_decode" else None)
-        achieved = dom_b / (per_class[dom]["avg_us"] * 1e3) if dom_b else None
+        dom_b = bytes_of(dom)
+        avg_us = per_class[dom]["avg_us"]
+        if dom == "decode_fused":
+            # one launch = one token: HBM and L2 bytes against the blend of the
+            # two measured bandwidths (peak = bytes / roofline time)
+            peak = step_bytes / (t_roof_us * 1e3)
+            peak_src = (f"blend: {peaks['source']} HBM {peaks['hbm_gbs']} GB/s for {int(hbm_bytes)} B + "
+                        f"measured L2 read {round(l2_gbs, 1)} GB/s for {int(l2_bytes)} B")
+        else:
+            peak = peaks["hbm_gbs"]
+            peak_src = peaks["source"] + " HBM copy"
+        achieved = dom_b / (avg_us * 1e3) if dom_b else None
         roofline = {
             "kernel": dom, "bound": "hbm", "achieved": round(achieved, 1) if achieved else None,
-            "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4) if achieved else None,
-            "traffic": None, "peak_source": peaks["source"],
-            "bytes_per_launch": dom_b,
-            "timing": "CUDA events around each launch of one extra decode phase (eager), after the timed region",
+            "peak": round(peak, 1), "unit": "GB/s",
+            "frac": round(achieved / peak, 4) if achieved else None,
+            "traffic": None, "peak_source": peak_src,
+            "bytes_per_launch": int(dom_b) if dom_b else None,
+            "timing": "CUDA events around each launch of one extra decode phase, after the timed region",
         }
-    # whole-token byte roofline: HBM bytes (pre blocks, head, KV) at the
-    # measured copy bandwidth + the loop block's L2-resident re-reads at the
-    # measured L2 read bandwidth
-    l2_gbs = l2_read_probe(dev)
-    layer_bytes = sum(BYTES_PER_LAUNCH[k] for k in ("qkv", "o_proj", "gate_up", "down"))
-    hbm_bytes = 2 * layer_bytes + BYTES_PER_LAUNCH["head"] + 10 * _attn_bytes_per_launch(mean_keys)
-    l2_bytes = LOOPS * layer_bytes
-    t_roof_us = hbm_bytes / (peaks["hbm_gbs"] * 1e3) + l2_bytes / (l2_gbs * 1e3)
-    t_tok_us = 1e3 * decode_sum / (args.steps * n_dec)
-    roof_step = {"hbm_bytes_per_token": int(hbm_bytes), "l2_bytes_per_token": int(l2_bytes),
-                 "l2_read_gbs_measured": round(l2_gbs, 1), "roofline_us_per_token": round(t_roof_us, 2),
-                 "achieved_us_per_token": round(t_tok_us, 2), "frac": round(t_roof_us / t_tok_us, 4)}
     # prefill: dense-equivalent flops of the linears + attention vs tensor peak
     per_layer_flops = 2 * PROMPT * (D * (HQ + 2 * HKV) * HD + HQ * HD * D + D * 2 * F + F * D)
     attn_flops = 4 * HQ * HD * PROMPT * (PROMPT + 1) / 2
@@ -426,7 +519,8 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (INT4 weights)",
             "data": "synthetic (seeded random weights and token ids)",
             "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": PROMPT + n_dec,
-                       "decode_steps": n_dec, "cuda_graphs": not args.no_graphs,
+                       "decode_steps": n_dec, "decode_path": args.decode_path,
+                       "cuda_graphs": not args.no_graphs,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": "inputs larger than L2: each step streams ~333 MB of weights"},
             "roofline": roofline,
@@ -457,9 +551,14 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=STEPS_DECODE,
                     help="greedy decode steps per step (the workload uses 128)")
     ap.add_argument("--no-graphs", action="store_true",
-                    help="launch decode kernels one by one instead of as CUDA graphs")
+                    help="layered decode path: launch kernels one by one instead of as CUDA graphs")
+    ap.add_argument("--decode-path", choices=["auto", "fused", "layered"], default="auto",
+                    help="single-kernel decode step (fused), one kernel per op (layered), or the "
+                         "library's default (auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-profile", action="store_true")
+    ap.add_argument("--trace", action="store_true",
+                    help="print the phase timeline of one single-kernel decode step and exit")
     ap.add_argument("--ncu-case", choices=["none", "decode", "prefill"], default="none",
                     help="run a small eager case for kernel profilers and exit")
     args = ap.parse_args()
@@ -469,6 +568,8 @@ def main():
         return run_reference(args)
     if args.ncu_case != "none":
         return run_ncu_case(args)
+    if args.trace:
+        return run_trace(args)
     return run_ours(args)
 
 

@@ -193,7 +193,8 @@ typedef enum {
   TL_KERNEL_GEMM_TC = 8,      /* tensor-core INT4 GEMM (prefill linears) */
   TL_KERNEL_NORM = 9,         /* stand-alone RMSNorm */
   TL_KERNEL_SETUP = 10,       /* per-call row bookkeeping */
-  TL_KERNEL_CLASSES = 11
+  TL_KERNEL_DECODE_FUSED = 11,/* a whole decode step in one persistent kernel */
+  TL_KERNEL_CLASSES = 12
 } tl_kernel_class;
 
 /* Per-kernel timing (the counterpart of the pages' phase timings, TinyLoop
@@ -213,6 +214,43 @@ tl_status tl_model_profile_stop(tl_model *m, int *h_launches, float *h_total_ms)
  * loop counts) by default; enable = 0 launches their kernels one by one
  * (same kernels, same results; useful under a kernel profiler). */
 tl_status tl_model_set_graphs(tl_model *m, int enable);
+
+/* How tl_decode_step runs a step (the same computation either way: the
+ * cached single-token forward of TinyLoop README, "Architecture"):
+ *   TL_DECODE_LAYERED  one kernel per projection / attention / head
+ *                      (replayed as a CUDA graph unless disabled above);
+ *   TL_DECODE_FUSED    the whole step as ONE persistent cooperative kernel
+ *                      (one CTA per SM, grid-wide barriers between the
+ *                      phases, weights streamed through shared memory);
+ *                      steps it cannot take return TL_ERR_UNSUPPORTED;
+ *   TL_DECODE_AUTO     (default) the faster of the two as measured on
+ *                      B200 for the 400M model at batch 1: LAYERED.
+ * FUSED needs <= 4 lanes per step, head_dim 64 or 128, n_pre <= 8,
+ * d_model, n_q_heads * head_dim and ffn_dim <= 5760, and a device with
+ * cooperative launch; set_decode_path returns TL_ERR_UNSUPPORTED for a model
+ * it cannot run. */
+typedef enum {
+  TL_DECODE_AUTO = 0,
+  TL_DECODE_LAYERED = 1,
+  TL_DECODE_FUSED = 2
+} tl_decode_path;
+tl_status tl_model_set_decode_path(tl_model *m, int path);
+
+/* Phase timeline of single-kernel decode steps (the counterpart of the pages'
+ * per-phase timings, TinyLoop README, "Quick CLI Tour", Benchmark with
+ * TINYLOOP_CUDA_PROFILE=1).  While d_buf (device memory, n_entries uint64,
+ * owned by the caller) is set, every TL_DECODE_FUSED step writes %globaltimer
+ * nanoseconds there, G = tl_model_trace_grid(m) entries per event (slot s
+ * = entries [s G, (s + 1) G), one per CTA): slot 0 kernel start; for grid
+ * barrier k (5 per effective layer: after QKV, attention, O, gate_up, down)
+ * slot 1 + 5k arrival and 2 + 5k release, and for the GEMV phase before it
+ * 3 + 5k activations staged, 4 + 5k first weight item arrived (not written
+ * by CTAs without items), 5 + 5k items consumed (none of the three for
+ * attention); after B barriers, slot 1 + 5B head activations staged,
+ * 2 + 5B head tiles done, 3 + 5B end.  Entries past n_entries are skipped.
+ * d_buf = NULL turns it off.  Steps overwrite the same entries. */
+tl_status tl_model_set_trace(tl_model *m, unsigned long long *d_buf, long long n_entries);
+int tl_model_trace_grid(const tl_model *m);
 
 /* Number of kernels this library has launched in the process so far. */
 unsigned long long tl_kernel_launch_count(void);
@@ -321,6 +359,17 @@ const char *tl_last_error(void);
 
 /* Library version, e.g. "0.1.0". */
 const char *tl_version(void);
+
+/* Measurement helper with no counterpart in the pages: read bandwidth of a
+ * device buffer.  Streams the `bytes` (a multiple of 16, >= 16) of d_buf with
+ * 16-byte loads that skip L1 (one CTA per SM x 4, 512 threads, 4 loads in
+ * flight per thread), `reps` times (1..100000) after 3 untimed passes, on
+ * `stream`, timed with CUDA events; writes GB/s (bytes x reps / time) to
+ * *h_gbs and synchronises the stream.  A buffer well under the L2 size (e.g.
+ * the 24 MB loop block) measures L2 read bandwidth, one well over it HBM.
+ * The buffer is only read. */
+tl_status tl_probe_read_bandwidth(const void *d_buf, size_t bytes, int reps, void *stream,
+                                  double *h_gbs);
 
 #ifdef __cplusplus
 }

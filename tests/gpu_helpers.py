@@ -69,6 +69,10 @@ class GpuModel:
             tl.tl_model_destroy(self.handle)
             self.handle = None
 
+    def set_path(self, path):
+        """Decode path of tl_decode_step (tl.DECODE_AUTO / _LAYERED / _FUSED)."""
+        tl.tl_model_set_decode_path(self.handle, path)
+
     def score_last(self, tokens, loops):
         V = self.shape.vocab
         d_tok = torch.as_tensor(np.asarray(tokens, np.int32), device=DEV)

@@ -11,6 +11,9 @@ Workloads:
 Decoding is teacher-forced with the oracle's tokens, so an allowed near-tie
 argmax flip cannot change later steps.  Bounds: logits max-abs <= 2e-2, argmax
 exact unless the oracle's top-2 margin is < 1e-3.
+
+Decode tests run on both decode paths: the single persistent kernel per step
+("fused") and one kernel per projection / attention / head ("layered").
 """
 
 import numpy as np
@@ -39,8 +42,19 @@ def _max_abs(a, b):
     return float(np.max(np.abs(np.asarray(a) - np.asarray(b))))
 
 
-def test_tiny_prefill_decode(tiny):
+@pytest.fixture(params=[tl.DECODE_FUSED, tl.DECODE_LAYERED], ids=["fused", "layered"])
+def path(request):
+    return request.param
+
+
+def _use(gm, path):
+    gm.set_path(path)
+    return gm
+
+
+def test_tiny_prefill_decode(tiny, path):
     w, om, gm = tiny
+    _use(gm, path)
     L, P, steps = 4, 32, 8
     prompt = tl_synth.make_tokens(tl_synth.SEED_TINY, w.shape.vocab, P + 1)
     # oracle: logits at positions P .. P+steps-1 (prefill of P+1 ids = first decode step)
@@ -70,9 +84,10 @@ def test_tiny_score_last(tiny):
         check_argmax(am, expect, "score_last")
 
 
-def test_tiny_cached_equals_uncached_on_gpu(tiny):
+def test_tiny_cached_equals_uncached_on_gpu(tiny, path):
     # Decode step i must agree with a fresh uncached forward of the prefix.
     w, om, gm = tiny
+    _use(gm, path)
     prompt = tl_synth.make_tokens(55, w.shape.vocab, 20)
     gm.prefill_lane(1, prompt[:12], 4, logits=False)
     seq = list(prompt[:12])
@@ -102,10 +117,11 @@ def test_tiny_looped_equals_flattened_on_gpu(tiny):
         fm.close()
 
 
-def test_tiny_per_lane_loops_independent(tiny):
+def test_tiny_per_lane_loops_independent(tiny, path):
     # Lanes with loops 4, 8, 16 decoded together give bitwise the results of
     # decoding each lane alone.
     w, om, gm = tiny
+    _use(gm, path)
     loops = [4, 16, 8]
     prompts = tl_synth.make_lane_prompts(7, w.shape.vocab, 3, 10)
     nxt = [5, 6, 7]
@@ -123,8 +139,34 @@ def test_tiny_per_lane_loops_independent(tiny):
         assert _max_abs(alone[0], expect) <= LOGIT_MAX_ABS
 
 
+def test_tiny_paths_agree_and_auto(tiny):
+    # Both decode paths on the same step: same argmax, logits within rounding
+    # of each other; asking FUSED for more than 4 lanes is refused and AUTO
+    # takes any lane count.
+    w, om, gm = tiny
+    prompts = tl_synth.make_lane_prompts(21, w.shape.vocab, 6, 9)
+    res = {}
+    for p in (tl.DECODE_FUSED, tl.DECODE_LAYERED):
+        gm.set_path(p)
+        for lane in range(6):
+            gm.prefill_lane(lane, prompts[lane, :8], 4, logits=False)
+        res[p] = gm.decode([0, 1], [int(prompts[0, 8]), int(prompts[1, 8])], [4, 4])
+    assert np.array_equal(res[tl.DECODE_FUSED][1], res[tl.DECODE_LAYERED][1])
+    assert _max_abs(res[tl.DECODE_FUSED][0], res[tl.DECODE_LAYERED][0]) <= 1e-3
+    gm.set_path(tl.DECODE_FUSED)
+    with pytest.raises(tl.TLError) as e:
+        gm.decode(list(range(5)), [1] * 5, [4] * 5)
+    assert e.value.status == tl.TL_ERR_UNSUPPORTED
+    gm.set_path(tl.DECODE_AUTO)
+    lg, _ = gm.decode(list(range(5)), [int(p[8]) for p in prompts[:5]], [4] * 5)
+    for lane in range(2, 5):   # lanes 0, 1 already took one step above
+        cache, _ = om.prefill(prompts[lane, :8], 4)
+        assert _max_abs(lg[lane], om.decode(cache, int(prompts[lane, 8]), 4)) <= LOGIT_MAX_ABS
+
+
 def test_tiny_errors(tiny):
     w, om, gm = tiny
+    gm.set_path(tl.DECODE_AUTO)
     gm.prefill_lane(5, [1, 2, 3], 4, logits=False)
     with pytest.raises(tl.TLError) as e:
         gm.decode([5], [1], [8])
@@ -147,8 +189,9 @@ def test_tiny_errors(tiny):
     tl.tl_check_device_error(gm.handle)   # cleared
 
 
-def test_tiny_context_full(tiny):
+def test_tiny_context_full(tiny, path):
     w, om, gm = tiny
+    _use(gm, path)
     gm.prefill_lane(6, list(range(255)), 1, logits=False)
     gm.decode([6], [1], [1])
     with pytest.raises(tl.TLError) as e:
@@ -164,15 +207,23 @@ def lm():
     w = tl_synth.make_model_weights(tl_synth.LOOPED_LM, tl_synth.SEED_LM)
     om = ref.LoopedModel(w)
     gm = GpuModel(w, max_loops=16, max_ctx=2048, max_lanes=16)
+    om.memo = {}   # oracle results shared by the two decode paths
     yield w, om, gm
     gm.close()
 
 
-def test_lm_prefill_then_decode(lm):
+def _memo(om, key, fn):
+    if key not in om.memo:
+        om.memo[key] = fn()
+    return om.memo[key]
+
+
+def test_lm_prefill_then_decode(lm, path):
     w, om, gm = lm
+    _use(gm, path)
     L, P, steps = 8, 128, 6
     prompt = tl_synth.make_tokens(tl_synth.SEED_LM, w.shape.vocab, P + 1)
-    o_tokens, o_logits = om.generate_greedy(prompt, L, steps)
+    o_tokens, o_logits = _memo(om, "greedy", lambda: om.generate_greedy(prompt, L, steps))
     gm.prefill_lane(0, prompt[:P], L, logits=False)
     fed = int(prompt[P])
     for i in range(steps):
@@ -193,10 +244,11 @@ def test_lm_score_last(lm):
         check_argmax(am, expect, f"L={L}")
 
 
-def test_lm_lanes_per_lane_loops(lm):
+def test_lm_lanes_per_lane_loops(lm, path):
     # Lanes with loops drawn from {4, 8, 16}, prompts of 512 ids; two lanes
-    # are checked against the oracle, all against their solo runs.
+    # are checked against the oracle.
     w, om, gm = lm
+    _use(gm, path)
     n_lanes, P = 4, 512
     loops = [int(v) for v in tl_synth.make_lane_loops(tl_synth.SEED_LSWEEP, n_lanes)]
     prompts = tl_synth.make_lane_prompts(tl_synth.SEED_LSWEEP, w.shape.vocab, n_lanes, P + 1)
@@ -205,6 +257,7 @@ def test_lm_lanes_per_lane_loops(lm):
         gm.prefill_lane(i, prompts[i, :P], loops[i], logits=False)
     together, am = gm.decode(lanes, [int(p[P]) for p in prompts], loops)
     for i in (0, n_lanes - 1):
-        expect = om.score_last(prompts[i, :P + 1], loops[i])   # = decode step at position P
+        # = decode step at position P
+        expect = _memo(om, ("lane", i), lambda: om.score_last(prompts[i, :P + 1], loops[i]))
         assert _max_abs(together[i], expect) <= LOGIT_MAX_ABS
         check_argmax(int(am[i]), expect, f"lane {i}")

@@ -17,7 +17,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from ctypes import POINTER, c_char_p, c_float, c_int, c_int32, c_longlong, c_size_t, c_void_p
+from ctypes import POINTER, c_char_p, c_double, c_float, c_int, c_int32, c_longlong, c_size_t, c_void_p
 
 from .build import LIB_PATH
 
@@ -29,7 +29,8 @@ __all__ = [
     "tl_model_create", "tl_model_destroy", "tl_prefill", "tl_decode_step", "tl_score_last",
     "tl_lane_length", "tl_model_info", "tl_check_device_error",
     "tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count", "KERNEL_CLASSES",
-    "tl_model_set_graphs",
+    "tl_model_set_graphs", "tl_model_set_decode_path", "DECODE_AUTO", "DECODE_LAYERED", "DECODE_FUSED",
+    "tl_probe_read_bandwidth", "tl_model_set_trace", "tl_model_trace_grid",
     "tl_linear_create", "tl_linear_destroy", "tl_linear_forward",
     "tl_op_rmsnorm", "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill",
     "tl_op_gqa_decode_noalloc",
@@ -91,6 +92,10 @@ def _load():
         "tl_model_profile_stop": (st, [P, POINTER(c_int), POINTER(c_float)]),
         "tl_kernel_launch_count": (ctypes.c_ulonglong, []),
         "tl_model_set_graphs": (st, [P, c_int]),
+        "tl_model_set_decode_path": (st, [P, c_int]),
+        "tl_model_set_trace": (st, [P, P, c_longlong]),
+        "tl_model_trace_grid": (c_int, [P]),
+        "tl_probe_read_bandwidth": (st, [P, c_size_t, c_int, P, POINTER(c_double)]),
         "tl_linear_create": (st, [POINTER(tl_int4_linear), c_int, c_int, c_int, POINTER(c_void_p)]),
         "tl_linear_destroy": (None, [P]),
         "tl_linear_forward": (st, [P, P, c_int, P, c_int, P]),
@@ -129,7 +134,8 @@ def __getattr__(name):
 
 # names every header declaration must have in the library (checked by tests)
 EXPORTED = sorted(["tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count",
-                   "tl_model_set_graphs",
+                   "tl_model_set_graphs", "tl_model_set_decode_path", "tl_probe_read_bandwidth",
+                   "tl_model_set_trace", "tl_model_trace_grid",
                    "tl_model_create", "tl_model_destroy", "tl_prefill", "tl_decode_step",
                    "tl_score_last", "tl_lane_length", "tl_model_info", "tl_check_device_error",
                    "tl_linear_create", "tl_linear_destroy", "tl_linear_forward", "tl_op_rmsnorm",
@@ -265,10 +271,13 @@ def tl_check_device_error(model, stream=None) -> None:
 
 
 KERNEL_CLASSES = ["embed", "qkv", "attn_decode", "o_proj", "gate_up", "down", "head",
-                  "attn_prefill", "gemm_tc", "norm", "setup"]
+                  "attn_prefill", "gemm_tc", "norm", "setup", "decode_fused"]
+
+# tl_decode_path
+DECODE_AUTO, DECODE_LAYERED, DECODE_FUSED = 0, 1, 2
 
 
-def tl_model_profile_start(model, class_mask: int = (1 << 11) - 1) -> None:
+def tl_model_profile_start(model, class_mask: int = (1 << 12) - 1) -> None:
     _check(_L().tl_model_profile_start(model, int(class_mask)))
 
 
@@ -283,6 +292,28 @@ def tl_model_profile_stop(model):
 
 def tl_model_set_graphs(model, enable: bool) -> None:
     _check(_L().tl_model_set_graphs(model, 1 if enable else 0))
+
+
+def tl_probe_read_bandwidth(buf, nbytes: int, reps: int = 200, stream=None) -> float:
+    """GB/s of repeated 16-byte L2-path reads over `nbytes` of a device buffer."""
+    out = c_double(0.0)
+    _check(_L().tl_probe_read_bandwidth(_ptr(buf), int(nbytes), int(reps), _stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def tl_model_set_trace(model, buf=None, n_entries: int = 0) -> None:
+    """Phase timeline of fused decode steps into a device uint64 buffer (None = off)."""
+    _check(_L().tl_model_set_trace(model, _ptr(buf) if buf is not None else None,
+                                   int(n_entries if buf is not None else 0)))
+
+
+def tl_model_trace_grid(model) -> int:
+    return int(_L().tl_model_trace_grid(model))
+
+
+def tl_model_set_decode_path(model, path: int) -> None:
+    """DECODE_AUTO (default), DECODE_LAYERED or DECODE_FUSED (see include/tl.h)."""
+    _check(_L().tl_model_set_decode_path(model, int(path)))
 
 
 def tl_kernel_launch_count() -> int:

@@ -22,6 +22,7 @@
 
 #include "attention.cuh"
 #include "common.cuh"
+#include "decode_fused.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_int4.cuh"
 #include "misc.cuh"
@@ -104,9 +105,12 @@ inline void kclass(int c) { g_cls = c; }
 // ============================================================================
 // launches (programmatic dependent launch on every kernel of the pass)
 // ============================================================================
+// Launch with event profiling and launch counting.  Ordinary kernels get
+// programmatic dependent launch (and the current L2 access-policy window);
+// `coop` launches are cooperative (all CTAs co-resident) and get neither.
 template <typename... KArgs, typename... Args>
-cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                   Args&&... args) {
+cudaError_t launch_impl(bool coop, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                        Args&&... args) {
   Profiler* pr = g_prof;
   const bool timed = pr && g_cls >= 0 && (pr->mask & (1u << g_cls)) && pr->used < Profiler::kCapacity;
   if (timed) {
@@ -126,11 +130,16 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (coop) {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (g_window.num_bytes) {
+  if (!coop && g_window.num_bytes) {
     attr[1].id = cudaLaunchAttributeAccessPolicyWindow;
     attr[1].val.accessPolicyWindow = g_window;
     cfg.numAttrs = 2;
@@ -143,6 +152,12 @@ cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, c
     ++pr->used;
   }
   return e;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   Args&&... args) {
+  return launch_impl(false, kern, grid, block, smem, st, std::forward<Args>(args)...);
 }
 
 constexpr size_t kMaxDynSmem = 220 * 1024;  // budget for dynamic smem per CTA
@@ -179,6 +194,8 @@ cudaError_t init_device_kernels(int dev) {
   SET3(IN_F16, EPI_STORE) SET3(IN_F32, EPI_RESID) SET3(IN_NORM, EPI_SWIGLU) SET3(IN_NORM, EPI_ROPE_KV)
 #undef SET3
 #undef SET
+  if (e == cudaSuccess) e = allow_max_smem(decode_fused_kernel<64>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(decode_fused_kernel<128>, dev);
   if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<1>, dev);
   if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<2>, dev);
   if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_RESID, true>, dev);
@@ -527,6 +544,17 @@ struct tl_model {
   };
   std::map<std::string, Graph> graphs;   // decode step graphs by row pattern
   bool use_graphs = true;
+  int decode_path = TL_DECODE_AUTO;
+  // single-kernel decode step
+  bool fused_ok = false;          // the model's shapes and the device allow it
+  int fused_grid = 0;             // one CTA per SM
+  int fused_smem_max = 0;         // dynamic shared memory the kernel may use
+  FusedArgs fused{};              // model part of the arguments
+  unsigned* fused_bar = nullptr;  // grid-barrier words [4]
+  float* fused_val = nullptr;     // per-CTA best logit [grid][4]
+  int* fused_idx = nullptr;
+  unsigned long long* trace = nullptr;  // caller's phase-timeline buffer (device), or NULL
+  long long trace_cap = 0;
   std::vector<int> lane_len, lane_loops;
   size_t weight_bytes = 0, kv_bytes = 0, ws_bytes = 0;
   Profiler prof;
@@ -546,7 +574,7 @@ struct tl_model {
     if (cap_stream) cudaStreamDestroy(cap_stream);
     void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row,
                     attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.partial, tc.tickets, gu,
-                    rope_tab};
+                    rope_tab, fused_bar, fused_val, fused_idx};
     for (void* p : ptrs)
       if (p) cudaFree(p);
     if (setup_stream) cudaStreamDestroy(setup_stream);
@@ -555,6 +583,27 @@ struct tl_model {
 };
 
 namespace {
+
+// Shared-memory plan of the single-kernel decode step for `rows` rows: the
+// largest ring (<= kFusedMaxSlots slots) that fits beside the activation
+// planes and the reduction buffer.  False if not even two slots fit.
+bool fused_plan(const tl_model* m, int rows, FusedArgs* f, size_t* smem) {
+  const tl_config& c = m->cfg;
+  const int qdim = c.n_q_heads * c.head_dim;
+  const int kmax = std::max(std::max(c.d_model, qdim), c.ffn_dim);
+  if (kmax > kFusedStageV4 * 4 * kFusedCompute) return false;
+  const int area = fused_area_bytes(rows, kmax, c.n_q_heads / c.n_kv_heads, c.head_dim);
+  const int red = fused_red_bytes(*f, m->fused_grid);
+  const int xown = fused_xown_bytes(*f, m->fused_grid);
+  const long avail = (long)m->fused_smem_max - area - red - xown;
+  const long ns = std::min<long>(kFusedMaxSlots, avail / kFusedSlotBytes);
+  if (ns < 2) return false;
+  f->n_slots = (int)ns;
+  f->area_bytes = area;
+  f->red_bytes = red;
+  *smem = (size_t)ns * kFusedSlotBytes + area + red + xown;
+  return true;
+}
 
 tl_status validate_config(const tl_config* c) {
   if (!c) return fail(TL_ERR_INVALID_ARG, "null config");
@@ -911,6 +960,54 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     }
   }
   if (!ok) return bail(fail(TL_ERR_OOM, "workspace allocation"));
+  {  // single-kernel decode step: shapes, device support, resources
+    // attention partials share the layered path's buffer, which holds
+    // kMaxLanes x Hkv x kDecodeMaxSplits x rep x (hd + 2) floats
+    static_assert(kFusedMaxSplits == kDecodeMaxSplits && 2 * kFusedMaxRows <= kMaxLanes,
+                  "fused partials ([4 rows][..][hd + 4]) must fit the layered path's buffer");
+    int coop = 0;
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, device);
+    if (coop && (hd == 64 || hd == 128) && c.n_pre < kFusedMaxBlocks && rep_ok(rep)) {
+      FusedArgs& f = m->fused;
+      for (int i = 0; i <= c.n_pre; ++i) {
+        const BlockDev& b = i < c.n_pre ? m->pre[i] : m->loop;
+        f.blk[i].lin[FP_QKV] = {b.qkv.w, b.qkv.sz};
+        f.blk[i].lin[FP_O] = {b.o.w, b.o.sz};
+        f.blk[i].lin[FP_GU] = {b.gate_up.w, b.gate_up.sz};
+        f.blk[i].lin[FP_DOWN] = {b.down.w, b.down.sz};
+        f.blk[i].attn_norm = b.attn_norm;
+        f.blk[i].ffn_norm = b.ffn_norm;
+      }
+      f.n_pre = c.n_pre;
+      f.d = d; f.qdim = qdim; f.F = c.ffn_dim; f.V = c.vocab; f.hd = hd; f.Hkv = c.n_kv_heads; f.rep = rep;
+      f.eps = c.rms_eps; f.theta = c.rope_theta;
+      f.embed = m->embed; f.out_norm = m->out_norm; f.head_w = m->head_w;
+      f.kv = m->kv; f.plane = m->plane; f.layer_stride = m->layer_stride; f.lane_stride = m->lane_stride;
+      f.ctx = c.max_ctx; f.rope_tab = m->rope_tab;
+      f.x = m->x; f.q = m->q; f.o = m->o; f.h = m->h;
+      f.attn_part = m->attn_part; f.attn_ticket = m->attn_tickets(); f.head_ticket = m->head_ticket();
+      f.err_flag = m->err_flag;
+      m->fused_grid = m->tc.n_sm;
+      ok = alloc((void**)&m->fused_bar, 4 * sizeof(unsigned)) &&
+           alloc((void**)&m->fused_val, (size_t)m->fused_grid * kFusedMaxRows * 4) &&
+           alloc((void**)&m->fused_idx, (size_t)m->fused_grid * kFusedMaxRows * 4);
+      if (!ok) return bail(fail(TL_ERR_OOM, "workspace allocation"));
+      f.bar = m->fused_bar; f.head_val = m->fused_val; f.head_idx = m->fused_idx;
+      void (*kern)(const FusedArgs) = hd == 64 ? decode_fused_kernel<64> : decode_fused_kernel<128>;
+      cudaFuncAttributes fa{};
+      int optin = 0, nb = 0;
+      size_t smem = 0;
+      FusedArgs probe = f;
+      if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess &&
+          cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) == cudaSuccess) {
+        m->fused_smem_max = optin - (int)fa.sharedSizeBytes;
+        if (fused_plan(m, kFusedMaxRows, &probe, &smem) &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kFusedThreads, smem) == cudaSuccess)
+          m->fused_ok = nb >= 1;
+      }
+    }
+    cudaGetLastError();
+  }
   m->ws_bytes = ws;
   if (cudaStreamSynchronize(st) != cudaSuccess) return bail(fail(TL_ERR_CUDA, "setup sync"));
   m->lane_len.assign(c.max_lanes + 1, 0);
@@ -1001,6 +1098,37 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
   if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
   cudaStream_t st = (cudaStream_t)stream;
   ProfScope prof_scope(&m->prof);
+  // AUTO takes the layered path: on the 400M model at batch 1 its graph
+  // replay currently measures faster than the single-kernel step.
+  const bool fused = m->decode_path == TL_DECODE_FUSED;
+  if (fused) {
+    if (!m->fused_ok || n_lanes > kFusedMaxRows)
+      return fail(TL_ERR_UNSUPPORTED, "single-kernel decode needs <= %d lanes and a supported model/device",
+                  kFusedMaxRows);
+    FusedArgs f = m->fused;
+    f.M = n_lanes;
+    for (int s = 0; s < n_lanes; ++s) {
+      f.lane[s] = sd.lane[s];
+      f.pos[s] = sd.pos[s];
+      f.loops[s] = h_loops[order[s]];
+      f.tok_index[s] = sd.tok_index[s];
+      f.out_row[s] = sd.out_row[s];
+    }
+    f.tokens = d_tokens;
+    f.logits = d_logits;
+    f.argmax = d_argmax;
+    f.trace = m->trace;
+    f.trace_cap = m->trace_cap;
+    size_t smem = 0;
+    if (!fused_plan(m, n_lanes, &f, &smem)) return fail(TL_ERR_UNSUPPORTED, "single-kernel decode: no shared-memory plan");
+    kclass(TL_KERNEL_DECODE_FUSED);
+    if (c.head_dim == 64)
+      TL_CUDA(launch_impl(true, decode_fused_kernel<64>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
+    else
+      TL_CUDA(launch_impl(true, decode_fused_kernel<128>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
+    for (int i = 0; i < n_lanes; ++i) m->lane_len[h_lane_ids[i]] += 1;
+    return TL_OK;
+  }
   kclass(TL_KERNEL_EMBED);
   TL_CUDA(launch(step_embed_kernel, dim3(n_lanes), dim3(256), 0, st, sd, (const __half*)m->embed, c.d_model,
                  c.vocab, m->rows, m->out_row, m->io, m->x, m->err_flag));
@@ -1092,6 +1220,26 @@ tl_status tl_model_set_graphs(tl_model* m, int enable) {
   m->use_graphs = enable != 0;
   return TL_OK;
 }
+
+tl_status tl_model_set_decode_path(tl_model* m, int path) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  if (path != TL_DECODE_AUTO && path != TL_DECODE_LAYERED && path != TL_DECODE_FUSED)
+    return fail(TL_ERR_INVALID_ARG, "unknown decode path %d", path);
+  if (path == TL_DECODE_FUSED && !m->fused_ok)
+    return fail(TL_ERR_UNSUPPORTED, "single-kernel decode is not available for this model/device");
+  m->decode_path = path;
+  return TL_OK;
+}
+
+tl_status tl_model_set_trace(tl_model* m, unsigned long long* d_buf, long long n_entries) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  if (d_buf && n_entries < 1) return fail(TL_ERR_INVALID_ARG, "n_entries must be >= 1");
+  m->trace = d_buf;
+  m->trace_cap = d_buf ? n_entries : 0;
+  return TL_OK;
+}
+
+int tl_model_trace_grid(const tl_model* m) { return m ? m->fused_grid : 0; }
 
 tl_status tl_lane_length(const tl_model* m, int lane, int* h_length) {
   if (!m || !h_length) return fail(TL_ERR_INVALID_ARG, "null argument");
@@ -1388,8 +1536,72 @@ __attribute__((visibility("hidden"))) tl_status tl_internal_set_error(tl_status 
   return s;
 }
 
+namespace {
+// Read-bandwidth probe: 4 independent 16-byte L2 loads in flight per thread.
+__global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict__ p, size_t n16,
+                                                         unsigned* __restrict__ sink) {
+  const size_t stride = (size_t)gridDim.x * blockDim.x;
+  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  unsigned acc = 0;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    const uint4 a = __ldcg(p + i), b = __ldcg(p + i + stride);
+    const uint4 c = __ldcg(p + i + 2 * stride), d = __ldcg(p + i + 3 * stride);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w ^ b.x ^ b.y ^ b.z ^ b.w ^ c.x ^ c.y ^ c.z ^ c.w ^ d.x ^ d.y ^ d.z ^ d.w;
+  }
+  for (; i < n16; i += stride) {
+    const uint4 a = __ldcg(p + i);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w;
+  }
+  if (acc == 0x9E3779B9u) *sink = acc;  // keeps the loads; practically never taken
+}
+}  // namespace
+
 extern "C" {
 
 const char* tl_version(void) { return "0.1.0"; }
+
+tl_status tl_probe_read_bandwidth(const void* d_buf, size_t bytes, int reps, void* stream, double* h_gbs) {
+  if (!d_buf || !h_gbs) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (bytes < 16 || bytes % 16 || ((uintptr_t)d_buf & 15))
+    return fail(TL_ERR_INVALID_ARG, "bytes must be a positive multiple of 16 on a 16-byte boundary");
+  if (reps < 1 || reps > 100000) return fail(TL_ERR_INVALID_ARG, "reps must be in [1, 100000]");
+  cudaPointerAttributes pa{};
+  if (cudaPointerGetAttributes(&pa, d_buf) != cudaSuccess || pa.type != cudaMemoryTypeDevice) {
+    cudaGetLastError();
+    return fail(TL_ERR_INVALID_ARG, "d_buf is not device memory");
+  }
+  DeviceGuard guard(pa.device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  int n_sm = 0;
+  TL_CUDA(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, pa.device));
+  cudaStream_t st = (cudaStream_t)stream;
+  unsigned* sink = nullptr;
+  TL_CUDA(cudaMalloc(&sink, sizeof(unsigned)));
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  cudaError_t e = cudaEventCreate(&e0);
+  if (e == cudaSuccess) e = cudaEventCreate(&e1);
+  const dim3 grid(n_sm * 4), block(512);
+  const uint4* p = (const uint4*)d_buf;
+  const size_t n16 = bytes / 16;
+  for (int i = 0; i < 3 && e == cudaSuccess; ++i) {
+    read_probe_kernel<<<grid, block, 0, st>>>(p, n16, sink);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaEventRecord(e0, st);
+  for (int i = 0; i < reps && e == cudaSuccess; ++i) {
+    read_probe_kernel<<<grid, block, 0, st>>>(p, n16, sink);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaEventRecord(e1, st);
+  if (e == cudaSuccess) e = cudaEventSynchronize(e1);
+  float ms = 0.f;
+  if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, e0, e1);
+  if (e0) cudaEventDestroy(e0);
+  if (e1) cudaEventDestroy(e1);
+  cudaFree(sink);
+  if (e != cudaSuccess) return cuda_fail(e, "read probe");
+  *h_gbs = (double)bytes * reps / ((double)ms * 1e6);
+  return TL_OK;
+}
 
 }  // extern "C"
