@@ -39,6 +39,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "misc.cuh"
 
 namespace tl {
 
@@ -112,6 +113,12 @@ struct FusedArgs {
   // head tiles done, 3 + 5B end.  Entries >= trace_cap are not written.
   unsigned long long* trace;
   long long trace_cap;
+  // head-only mode (no layers: output norm + head + argmax of the rows of x),
+  // used by the per-layer path; outputs may come from device memory so that a
+  // captured graph does not depend on them
+  int head_only;
+  const HeadIO* io;          // if set, logits / argmax pointers are read here
+  const int* out_row_dev;    // if set, output slots are read here
 };
 
 // ---- the fixed work sequence (shared by the producer and the consumers) ----
@@ -134,7 +141,7 @@ __host__ __device__ inline int fused_tile(const FusedArgs& a, int ph, int u, int
   if (ph == FP_GU) return u + (ti ? a.F / 16 : 0);
   return u;
 }
-__host__ __device__ inline int fused_layers(const FusedArgs& a) { return a.n_pre + a.loops[0]; }
+__host__ __device__ inline int fused_layers(const FusedArgs& a) { return a.head_only ? 0 : a.n_pre + a.loops[0]; }
 __device__ __forceinline__ int fused_active(const FusedArgs& a, int layer) {
   int n = 0;
   while (n < a.M && a.n_pre + a.loops[n] > layer) ++n;
@@ -836,11 +843,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
     int item = 0;
     unsigned target = 0;
     __half* xs = reinterpret_cast<__half*>(area);
-    for (int e = tid; e < a.M * (a.hd / 2); e += kFusedCompute) {
+    pdl_wait();   // head-only launches follow the kernel that wrote x
+    for (int e = tid; e < (a.head_only ? 0 : a.M * (a.hd / 2)); e += kFusedCompute) {
       const int m = e / (a.hd / 2), j = e % (a.hd / 2);
       rope_s[e] = rope_cs(a.rope_tab, a.pos[m], j, a.hd, a.theta);
     }
-    {  // the residual stream of this CTA's rows starts as the tokens' embeddings
+    if (!a.head_only) {  // the residual stream of this CTA's rows starts as the tokens' embeddings
       const int n_own = (fused_units(a, FP_O) - c + P - 1) / P;
       for (int e = tid; e < n_own * 16 * a.M; e += kFusedCompute) {
         const int ul = e / (16 * a.M), rem = e % (16 * a.M), r = rem & 15, m = rem >> 4;
@@ -907,6 +915,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
     const int fr = tid & 15, fm = tid >> 4;
     float best_v = -INFINITY;
     int best_i = 0x7fffffff;
+    float* const logits = a.io ? a.io->logits : a.logits;
+    int32_t* const argmax = a.io ? a.io->argmax : a.argmax;
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
     for (int tile = tb; tile < te; ++tile) {
       for (int kk = 0; kk < d; kk += ki) {
@@ -940,7 +950,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
 #pragma unroll
         for (int w = 0; w < kFusedWarps; ++w) v += red[((size_t)(tile & 1) * kFusedWarps + w) * 64 + fr * 4 + fm];
         const int row = tile * 16 + fr;
-        if (a.logits) a.logits[(size_t)a.out_row[fm] * a.V + row] = v;
+        if (logits) logits[(size_t)(a.out_row_dev ? a.out_row_dev[fm] : a.out_row[fm]) * a.V + row] = v;
         if (fused_better(v, row, best_v, best_i)) { best_v = v; best_i = row; }
       }
     }
@@ -961,7 +971,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
     fused_sync();
     if (s_last) {
       __threadfence();
-      if (a.argmax) {
+      if (argmax) {
         // every CTA's best per row, loaded in one round, reduced by warps
         float v[kFusedMaxRows];
         int ix[kFusedMaxRows];
@@ -993,7 +1003,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
           int bi = s_wi[tid][0];
           for (int w = 1; w < kFusedWarps; ++w)
             if (fused_better(s_wv[tid][w], s_wi[tid][w], bv, bi)) { bv = s_wv[tid][w]; bi = s_wi[tid][w]; }
-          a.argmax[a.out_row[tid]] = bi;
+          argmax[a.out_row_dev ? a.out_row_dev[tid] : a.out_row[tid]] = bi;
         }
       }
       if (tid == 0) *a.head_ticket = 0u;

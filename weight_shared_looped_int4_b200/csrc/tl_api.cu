@@ -787,6 +787,28 @@ tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
 tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, float* logits,
                       int32_t* argmax, cudaStream_t st, const HeadIO* io = nullptr) {
   const tl_config& c = m->cfg;
+  if (m->fused_ok && M <= kFusedMaxRows) {
+    // the persistent step kernel in head-only mode: one CTA per SM streams
+    // its head tiles through a bulk-copy ring (15 compute warps)
+    FusedArgs f = m->fused;
+    f.head_only = 1;
+    f.M = M;
+    f.x = const_cast<float*>(x);
+    for (int i = 0; i < M; ++i) f.out_row[i] = i;
+    f.out_row_dev = out_row;
+    f.io = io;
+    f.logits = logits;
+    f.argmax = argmax;
+    size_t smem = 0;
+    if (fused_plan(m, M, &f, &smem)) {
+      kclass(TL_KERNEL_HEAD);
+      if (c.head_dim == 64)
+        TL_CUDA(launch(decode_fused_kernel<64>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
+      else
+        TL_CUDA(launch(decode_fused_kernel<128>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
+      return TL_OK;
+    }
+  }
   HeadArgs ha{};
   ha.io = io;
   ha.w = m->head_w; ha.V = c.vocab; ha.d = c.d_model;
