@@ -13,17 +13,20 @@
 //   epilogue warps read it and accumulate s[n][group] * (P_hi + P_lo) in fp32
 //   registers.  So no weight is rounded and the activation keeps ~22 bits;
 //   fp16 weights or activations move the looped model's logits by ~0.05.
-// * Warp roles (12 warps, 3 per SM sub-partition so each thread may hold 168
-//   registers): warp 0 allocates TMEM and one lane issues tcgen05.mma; warps
-//   1-3 dequantize A from the packed INT4 words straight into the 128-byte
-//   swizzled K-major layout the MMA descriptor reads, and one of them issues
-//   the bulk asynchronous copy of the prepared B tile; warps 4-11 are the
-//   epilogue.  Shared-memory stages and TMEM buffers are double-buffered and
-//   handed over with mbarriers (tcgen05.commit signals MMA completion).
-// * Split-K partials go to a scratch buffer; the last CTA of a tile (atomic
-//   ticket) adds them in split order, so the result is deterministic, and
-//   applies the epilogue: residual add, raw fp32, fp16 store, or RoPE with
-//   the Q output and the K/V cache write.
+// * Warp roles (16 warps): warp 0 allocates TMEM and one lane issues
+//   tcgen05.mma; one lane of warp 1 issues the bulk asynchronous copies (raw
+//   INT4 words + scales/zeros a few groups ahead, the prepared B atoms per
+//   stage); warps 2-7 dequantize A from the raw ring straight into the
+//   128-byte swizzled K-major layout the MMA descriptor reads (the
+//   dequantisation, not the tensor core, paces this GEMM); warps 8-15 are the
+//   epilogue.  Stages of 64 k (4 deep), the raw ring (3 groups) and the TMEM
+//   buffers (2 groups) are handed over with mbarriers (tcgen05.commit signals
+//   MMA completion).
+// * Split-K partials go to a scratch buffer; a merge kernel (one CTA per 8
+//   tokens of a tile, all loads in flight) adds them in split order, so the
+//   result is deterministic, and applies the epilogue: residual add, raw
+//   fp32, fp16 store, or RoPE with the Q output and the K/V cache write.
+//   Without a split the GEMM applies the epilogue itself.
 // * Every mbarrier wait is bounded; on time-out the kernel records kErrTimeout,
 //   skips the rest of its work and still frees its TMEM.
 #pragma once
@@ -123,16 +126,23 @@ __host__ __device__ inline uint32_t sw128_offset(int row, int k, int rows) {
 
 enum TcEpi { TC_RESID = 0, TC_RAW = 1, TC_STORE = 2, TC_ROPE_KV = 3 };
 
-constexpr int kTcThreads = 384;       // 12 warps
+constexpr int kTcThreads = 512;       // 16 warps
 constexpr int kTcRows = 128;          // weight rows per tile (MMA M)
 constexpr int kTcTokens = 128;        // tokens per tile
-constexpr int kTcEpiThreads = 256;    // warps 4..11
-constexpr int kTcProducers = 96;      // warps 1..3
+constexpr int kTcEpiThreads = 256;    // warps 8..15
+constexpr int kTcUnpack = 192;        // warps 2..7
+constexpr int kTcEpiWarp0 = 8;
+
+constexpr int kTcStages = 4;          // half-group (64 k) operand stages
+constexpr int kTcRaw = 3;             // raw INT4 group stages
+constexpr int kTcRawBytes = 8 * 1024 + 8 * 64;   // 8 16-row tiles x (2 chunks of 512 B + 64 B of scales/zeros)
 
 __host__ __device__ inline int tc_nb(bool lo) { return lo ? 2 * kTcTokens : kTcTokens; }  // B rows (MMA N)
-__host__ __device__ inline size_t tc_a_bytes() { return (size_t)kTcRows * 256; }              // 32 KB
-__host__ __device__ inline size_t tc_b_bytes(bool lo) { return (size_t)tc_nb(lo) * 256; }      // 64 / 32 KB
-__host__ __device__ inline size_t tc_smem_bytes(bool lo) { return 2 * (tc_a_bytes() + tc_b_bytes(lo)) + 1024; }
+__host__ __device__ inline size_t tc_b_bytes(bool lo) { return (size_t)tc_nb(lo) * 256; }      // B of one group: 64 / 32 KB
+// Stage = one 64-wide K atom: A 128 rows x 128 B (16 KB), B NB rows x 128 B.
+__host__ __device__ inline size_t tc_smem_bytes(bool lo) {
+  return (size_t)kTcStages * ((size_t)kTcRows * 128 + (size_t)tc_nb(lo) * 128) + (size_t)kTcRaw * kTcRawBytes + 1024;
+}
 
 struct TcGemmArgs {
   const uint4* w;        // INT4 weights in the GEMV tile layout [n16 tiles][K/64][32] (16 B each)
@@ -165,14 +175,16 @@ template <int EPI, bool LO>
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGemmArgs a) {
   constexpr int NB = LO ? 2 * kTcTokens : kTcTokens;
   constexpr uint32_t NCOL = NB;                    // TMEM columns per buffer
-  constexpr uint32_t A_BYTES = kTcRows * 256;
-  constexpr uint32_t B_BYTES = NB * 256;
+  constexpr uint32_t A_BYTES = kTcRows * 128;      // one 64-k atom of A
+  constexpr uint32_t B_BYTES = NB * 128;           // one 64-k atom of B
   extern __shared__ __align__(128) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   auto sA = [&](int st) { return smem + st * A_BYTES; };
-  auto sB = [&](int st) { return smem + 2 * A_BYTES + st * B_BYTES; };
-  __shared__ __align__(8) uint64_t bar_full[2], bar_empty[2], bar_tfull[2], bar_tempty[2];
+  auto sB = [&](int st) { return smem + kTcStages * A_BYTES + st * B_BYTES; };
+  auto sR = [&](int r) { return smem + kTcStages * (A_BYTES + B_BYTES) + r * kTcRawBytes; };
+  __shared__ __align__(8) uint64_t bar_full[kTcStages], bar_empty[kTcStages], bar_tfull[2], bar_tempty[2];
+  __shared__ __align__(8) uint64_t raw_full[kTcRaw], raw_empty[kTcRaw];
   __shared__ uint32_t s_tmem;
   __shared__ int s_last;
   __shared__ int s_fail;
@@ -182,18 +194,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   const int G = a.K >> 7;
   const int g_begin = split * G / a.splits, g_end = (split + 1) * G / a.splits;
   const int ng = g_end - g_begin;
+  const int nh = 2 * ng;                             // half-group steps
   const int row_tiles = gridDim.x, tok_tiles = gridDim.y;
+  // CTAs walk their K groups from different starting points so that they do
+  // not all fetch the same activation atom at the same time (the epilogue
+  // adds the groups in this fixed order: deterministic)
+  const int rot = ng > 0 ? tile % ng : 0;
+  auto gmap = [&](int it) { return g_begin + (it + rot) % ng; };
 
   if (warp == 0) {
     tmem_alloc(&s_tmem, 512);
     tmem_relinquish();
   }
   if (threadIdx.x == 32) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar_full[i], kTcProducers);
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(&bar_full[i], kTcUnpack + 1);   // + the copy lane's arrive with the B bytes
       mbar_init(&bar_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&bar_tfull[i], 1);
       mbar_init(&bar_tempty[i], kTcEpiThreads);
+    }
+    for (int i = 0; i < kTcRaw; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], kTcUnpack);
     }
     fence_mbar_init();
     s_fail = 0;
@@ -204,73 +228,117 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   const uint32_t tmem = s_tmem;
 
   pdl_trigger();
-  pdl_wait();
 
   if (warp == 0) {
-    // ---- MMA issue -------------------------------------------------------
+    pdl_wait();
+    // ---- MMA issue: 4 k16 steps per 64-k stage, a group = 2 stages into one
+    // TMEM buffer (double-buffered across groups) ----------------------------
     if (lane == 0) {
       const uint32_t idesc = idesc_f16_f32(kTcRows, NB);
-      for (int it = 0; it < ng; ++it) {
-        const int s = it & 1;
-        if (!mbar_wait_or_fail(&bar_full[s], (it >> 1) & 1, &s_fail)) break;
-        if (it >= 2 && !mbar_wait_or_fail(&bar_tempty[s], ((it - 2) >> 1) & 1, &s_fail)) break;
+      for (int h = 0; h < nh; ++h) {
+        const int s = h % kTcStages, it = h >> 1, half = h & 1, b = it & 1;
+        if (!mbar_wait_or_fail(&bar_full[s], (unsigned)(h / kTcStages) & 1u, &s_fail)) break;
+        if (half == 0 && it >= 2 && !mbar_wait_or_fail(&bar_tempty[b], (unsigned)((it - 2) >> 1) & 1u, &s_fail))
+          break;
         tc_fence_after();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint64_t ad = sw128_kmajor_desc(sA(s) + (j >> 2) * (kTcRows * 128) + (j & 3) * 32);
-          const uint64_t bd = sw128_kmajor_desc(sB(s) + (j >> 2) * (NB * 128) + (j & 3) * 32);
-          tc_mma_f16(tmem + s * NCOL, ad, bd, idesc, j > 0 ? 1u : 0u);
+        for (int j = 0; j < 4; ++j) {
+          const uint64_t ad = sw128_kmajor_desc(sA(s) + j * 32);
+          const uint64_t bd = sw128_kmajor_desc(sB(s) + j * 32);
+          tc_mma_f16(tmem + b * NCOL, ad, bd, idesc, (half | j) ? 1u : 0u);
         }
         tc_commit(&bar_empty[s]);
-        tc_commit(&bar_tfull[s]);
+        if (half) tc_commit(&bar_tfull[b]);
       }
     }
     __syncwarp();
-  } else if (warp <= 3) {
-    // ---- producers: A dequant (+ B bulk copy by one thread) ------------
-    const int p = threadIdx.x - 32;
-    const int kw = a.K >> 6;  // 64-wide chunks per row
-    for (int it = 0; it < ng; ++it) {
-      const int s = it & 1, g = g_begin + it;
-      if (it >= 2 && !mbar_wait_or_fail(&bar_empty[s], ((it - 2) >> 1) & 1, &s_fail)) break;
-      if (p == 0) {
-        mbar_expect_tx(&bar_full[s], B_BYTES);
-        const uint8_t* src = a.bt + ((size_t)tt * G + g) * B_BYTES;
-        for (uint32_t off = 0; off < B_BYTES; off += 16384)
-          bulk_g2s(sB(s) + off, src + off, 16384, &bar_full[s]);
+  } else if (warp == 1) {
+    // ---- copy issuer (one lane) ----------------------------------------------
+    // Keeps kTcRaw groups of raw INT4 words and scales/zeros in flight (bulk
+    // copies; the weights do not depend on earlier kernels, so the first ones
+    // go out before the dependency wait) and issues each stage's B atom as
+    // soon as the MMA has released the stage.
+    if (lane == 0) {
+      const int kw = a.K >> 6;  // 64-wide chunks per row
+      int g_issued = 0;
+      auto issue_raw = [&](int it) {
+        const int r = it % kTcRaw, g = gmap(it);
+        unsigned char* dst = sR(r);
+        mbar_arrive_expect_tx(&raw_full[r], kTcRawBytes);
+        for (int n16 = 0; n16 < 8; ++n16) {
+          int gt = tile * 8 + n16;
+          if (gt >= a.n16_tiles) gt = a.n16_tiles - 1;   // absent rows: any valid tile (their A is zeroed)
+          bulk_g2s(dst + n16 * 1024, reinterpret_cast<const unsigned char*>(a.w) + ((size_t)gt * kw + g * 2) * 512,
+                   1024, &raw_full[r]);
+          bulk_g2s(dst + 8192 + n16 * 64, reinterpret_cast<const unsigned char*>(a.sz) + ((size_t)gt * G + g) * 64,
+                   64, &raw_full[r]);
+        }
+      };
+      for (; g_issued < ng && g_issued < kTcRaw; ++g_issued) issue_raw(g_issued);
+      pdl_wait();
+      for (int h = 0; h < nh; ++h) {
+        const int s = h % kTcStages, it = h >> 1, half = h & 1, g = gmap(it);
+        if (h >= kTcStages && !mbar_wait_or_fail(&bar_empty[s], (unsigned)((h / kTcStages) - 1) & 1u, &s_fail))
+          break;
+        // arrive with the expected bytes: the stage cannot complete before
+        // this arrival, so the unpackers' arrivals cannot race past the copy
+        mbar_arrive_expect_tx(&bar_full[s], B_BYTES);
+        bulk_g2s(sB(s), a.bt + (((size_t)tt * G + g) * 2 + half) * B_BYTES, B_BYTES, &bar_full[s]);
+        if (half) {
+          // top up the raw ring: group g_issued reuses the slot of g_issued - kTcRaw
+          for (; g_issued < ng && g_issued < it + kTcRaw; ++g_issued)
+            if (mbar_wait_or_fail(&raw_empty[g_issued % kTcRaw], (unsigned)((g_issued / kTcRaw) - 1) & 1u,
+                                  &s_fail))
+              issue_raw(g_issued);
+        }
       }
+      // a CTA that gave up waits (bounded) for its raw copies still in flight
+      if (*reinterpret_cast<volatile int*>(&s_fail))
+        for (int it = g_issued - kTcRaw < 0 ? 0 : g_issued - kTcRaw; it < g_issued; ++it)
+          mbar_wait(&raw_full[it % kTcRaw], (unsigned)(it / kTcRaw) & 1u);
+    }
+    __syncwarp();
+  } else if (warp < kTcEpiWarp0) {
+    // ---- unpackers: A from the raw ring into the 128-byte swizzled K-major
+    // layout the MMA descriptor reads --------------------------------------------
+    const int p = threadIdx.x - 64;
+    for (int h = 0; h < nh; ++h) {
+      const int s = h % kTcStages, it = h >> 1, half = h & 1, r = it % kTcRaw;
+      if (h >= kTcStages && !mbar_wait_or_fail(&bar_empty[s], (unsigned)((h / kTcStages) - 1) & 1u, &s_fail))
+        break;
+      if (!mbar_wait_or_fail(&raw_full[r], (unsigned)(it / kTcRaw) & 1u, &s_fail)) break;
+      const unsigned char* raw = sR(r);
       unsigned char* A = sA(s);
-#pragma unroll
-      for (int i = 0; i < 6; ++i) {
-        const int wi = p + kTcProducers * i;
-        if (wi >= 512) break;
-        const int n16 = wi >> 6, chunk = (wi >> 5) & 1, ln = wi & 31;
-        const int gt = tile * 8 + n16;   // global 16-row tile
+      for (int wi = p; wi < 256; wi += kTcUnpack) {
+        const int n16 = wi >> 5, ln = wi & 31;
+        const int gt = tile * 8 + n16;
         const int r0 = n16 * 16 + (ln >> 2), t = ln & 3;
         uint4 wv = make_uint4(0, 0, 0, 0);
         uint32_t zz = 0x64006400u;  // z = 0 for absent rows (their q are 0 too)
         if (gt < a.n16_tiles) {
-          wv = ldg_stream(a.w + ((size_t)gt * kw + g * 2 + chunk) * 32 + ln);
-          zz = __ldg(&a.sz[((size_t)gt * G + g) * 8 + (ln >> 2)]).y;
+          wv = *reinterpret_cast<const uint4*>(raw + n16 * 1024 + half * 512 + ln * 16);
+          zz = reinterpret_cast<const uint2*>(raw + 8192 + n16 * 64)[ln >> 2].y;
         }
         const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t af[4];
           unpack_a_frag(words[j], zz, af);
-          const int kb = chunk * 64 + j * 16 + 2 * t;
+          const int kb = j * 16 + 2 * t;
           *reinterpret_cast<uint32_t*>(A + sw128_offset(r0, kb, kTcRows)) = af[0];
           *reinterpret_cast<uint32_t*>(A + sw128_offset(r0 + 8, kb, kTcRows)) = af[1];
           *reinterpret_cast<uint32_t*>(A + sw128_offset(r0, kb + 8, kTcRows)) = af[2];
           *reinterpret_cast<uint32_t*>(A + sw128_offset(r0 + 8, kb + 8, kTcRows)) = af[3];
         }
       }
+      if (half) mbar_arrive(&raw_empty[r]);
       fence_proxy_async_smem();
       mbar_arrive(&bar_full[s]);
     }
   } else {
     // ---- epilogue: accumulate s * (P_hi + P_lo) per group --------------
-    const int e = warp - 4;
+    pdl_wait();   // it reads / writes what earlier kernels wrote
+    const int e = warp - kTcEpiWarp0;
     const int quad = warp & 3;                 // TMEM lanes this warp may access
     const int half = e >> 2;                   // tokens [64 half, 64 half + 64)
     const int row = quad * 32 + lane;          // weight row within the tile
@@ -285,11 +353,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
       const float2 f = h2_to_f2(sp);
       return (row & 8) ? f.y : f.x;
     };
-    float s_next = ng > 0 ? scale_of(g_begin) : 0.f;
+    float s_next = ng > 0 ? scale_of(gmap(0)) : 0.f;
     for (int it = 0; it < ng; ++it) {
       const int b = it & 1;
       const float sc = s_next;
-      if (it + 1 < ng) s_next = scale_of(g_begin + it + 1);
+      if (it + 1 < ng) s_next = scale_of(gmap(it + 1));
       // on a time-out the loop keeps its shape (no further waits) so the
       // epilogue barriers below still match across the epilogue warps
       mbar_wait_or_fail(&bar_tfull[b], (it >> 1) & 1, &s_fail);
@@ -316,38 +384,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
       mbar_arrive(&bar_tempty[b]);
     }
 
-    // ---- split-K merge (deterministic) ----------------------------------
+    // ---- split-K: partial sums to scratch, merged by tc_merge_kernel --------
     const int n = tile * kTcRows + row;
     const int t0 = tt * kTcTokens + half * 64;
     epi_sync(kTcEpiThreads);
     const bool failed = s_fail != 0;
-    if (!failed && a.splits > 1) {
+    if (a.splits > 1) {
       float* mine = a.partial + (((size_t)split * row_tiles + tile) * tok_tiles + tt) * (kTcTokens * kTcRows);
 #pragma unroll
       for (int i = 0; i < 64; ++i) mine[(size_t)(half * 64 + i) * kTcRows + row] = acc[i];
-      __threadfence();
-      epi_sync(kTcEpiThreads);
-      if (e == 0 && lane == 0) {
-        unsigned* tk = a.tickets + tile * tok_tiles + tt;
-        s_last = (atomicAdd(tk, 1u) == (unsigned)(a.splits - 1));
-        if (s_last) *tk = 0u;
-      }
-      epi_sync(kTcEpiThreads);
-      if (s_last) {
-        __threadfence();
-#pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = 0.f;
-        for (int sp = 0; sp < a.splits; ++sp) {
-          const float* src =
-              a.partial + (((size_t)sp * row_tiles + tile) * tok_tiles + tt) * (kTcTokens * kTcRows);
-#pragma unroll
-          for (int i = 0; i < 64; ++i) acc[i] += __ldcg(src + (size_t)(half * 64 + i) * kTcRows + row);
-        }
-      }
+      if (e == 0 && lane == 0) s_last = 0;
     } else {
       if (e == 0 && lane == 0) s_last = 1;
-      epi_sync(kTcEpiThreads);
     }
+    epi_sync(kTcEpiThreads);
 
     // ---- final epilogue -----------------------------------------------------
     if (!failed && s_last) {
@@ -373,7 +423,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
         epi_sync(kTcEpiThreads);
         const int hd = a.hd, hh = hd / 2;
         const int pairs_per_tok = kTcRows / 2;         // 64 (j < hd/2 of each head in the tile)
-        for (int item = threadIdx.x - 4 * 32; item < kTcTokens * pairs_per_tok; item += kTcEpiThreads) {
+        for (int item = threadIdx.x - kTcEpiWarp0 * 32; item < kTcTokens * pairs_per_tok; item += kTcEpiThreads) {
           const int tl_ = item / pairs_per_tok, pr = item % pairs_per_tok;
           const int head_local = pr / hh, j = pr % hh;
           const int r_a = head_local * hd + j, r_b = r_a + hh;
@@ -411,6 +461,87 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---- split-K merge + epilogue ------------------------------------------------
+// One CTA per (row tile, token tile, 8-token slice): sums the split partials
+// of its 8 x 128 outputs in split order (all loads of a batch of 8 splits in
+// flight), then applies the GEMM's epilogue.  Deterministic; the partials
+// are [split][row tile][token tile][128 tokens][128 rows].
+constexpr int kTcMergeTok = 8;
+template <int EPI>
+__global__ void __launch_bounds__(256) tc_merge_kernel(const TcGemmArgs a) {
+  __shared__ float xch[kTcMergeTok][kTcRows];
+  const int tile = blockIdx.x, tt = blockIdx.y, slice = blockIdx.z;
+  const int row_tiles = gridDim.x, tok_tiles = gridDim.y;
+  const int tl_ = threadIdx.x >> 5, r4 = (threadIdx.x & 31) * 4;   // token in the slice, 4 rows
+  const int tok = slice * kTcMergeTok + tl_;                       // token within the tile
+  pdl_trigger();
+  pdl_wait();
+  float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+  const size_t split_stride = (size_t)row_tiles * tok_tiles * kTcTokens * kTcRows;
+  const float* base = a.partial + ((size_t)tile * tok_tiles + tt) * (kTcTokens * kTcRows) + (size_t)tok * kTcRows + r4;
+  for (int sp0 = 0; sp0 < a.splits; sp0 += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[i] = sp0 + i < a.splits ? __ldcg(reinterpret_cast<const float4*>(base + (size_t)(sp0 + i) * split_stride))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (sp0 + i < a.splits) {
+        sum.x += v[i].x; sum.y += v[i].y; sum.z += v[i].z; sum.w += v[i].w;
+      }
+    }
+  }
+  const int t = tt * kTcTokens + tok;
+  if (EPI == TC_RESID || EPI == TC_RAW || EPI == TC_STORE) {
+    const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
+    if (t < a.T) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int n = tile * kTcRows + r4 + i;
+        if (n < a.N) {
+          const size_t o = (size_t)t * a.ld_out + n;
+          if (EPI == TC_RESID) a.out_f32[o] += vals[i];
+          else if (EPI == TC_RAW) a.out_f32[o] = vals[i];
+          else a.out_f16[o] = __float2half_rn(vals[i]);
+        }
+      }
+    }
+  } else {
+    *reinterpret_cast<float4*>(&xch[tl_][r4]) = sum;
+    __syncthreads();
+    const int hd = a.hd, hh = hd / 2;
+    const int pairs = kTcRows / 2;
+    for (int item = threadIdx.x; item < kTcMergeTok * pairs; item += 256) {
+      const int ti = item / pairs, pr = item % pairs;
+      const int head_local = pr / hh, j = pr % hh;
+      const int r_a = head_local * hd + j, r_b = r_a + hh;
+      const int tq = tt * kTcTokens + slice * kTcMergeTok + ti;
+      const int na = tile * kTcRows + r_a;
+      if (tq >= a.T || na >= a.N) continue;
+      const float va = xch[ti][r_a], vb = xch[ti][r_b];
+      const int pos = a.pos0 + tq;
+      if (na < a.n_q_rows) {
+        const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
+        float* qo = a.q_out + (size_t)tq * a.ldq;
+        qo[na] = va * cs.x - vb * cs.y;
+        qo[na + hh] = vb * cs.x + va * cs.y;
+      } else if (na < a.n_q_rows + a.n_kv_rows) {
+        const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
+        const int kvh = (na - a.n_q_rows) / hd;
+        __half* dst = a.k_plane + ((size_t)kvh * a.ctx + pos) * hd;
+        dst[j] = __float2half_rn(va * cs.x - vb * cs.y);
+        dst[j + hh] = __float2half_rn(vb * cs.x + va * cs.y);
+      } else {
+        const int kvh = (na - a.n_q_rows - a.n_kv_rows) / hd;
+        __half* dst = a.v_plane + ((size_t)kvh * a.ctx + pos) * hd;
+        dst[j] = __float2half_rn(va);
+        dst[j + hh] = __float2half_rn(vb);
+      }
+    }
   }
 }
 

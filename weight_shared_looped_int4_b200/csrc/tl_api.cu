@@ -463,11 +463,17 @@ cudaError_t launch_tc_linear(const uint4* w, const uint2* sz, int K, int N, int 
   ta.partial = sc.partial; ta.tickets = sc.tickets; ta.err_flag = sc.err_flag;
   const dim3 g(row_tiles, tok_tiles, splits), b(kTcThreads);
   const size_t smem = tc_smem_bytes(lo);
-  if (epi == TC_RESID && lo) return launch(gemm_int4_tc_kernel<TC_RESID, true>, g, b, smem, st, ta);
-  if (epi == TC_RAW && lo) return launch(gemm_int4_tc_kernel<TC_RAW, true>, g, b, smem, st, ta);
-  if (epi == TC_ROPE_KV && lo) return launch(gemm_int4_tc_kernel<TC_ROPE_KV, true>, g, b, smem, st, ta);
-  if (epi == TC_STORE && !lo) return launch(gemm_int4_tc_kernel<TC_STORE, false>, g, b, smem, st, ta);
-  return cudaErrorInvalidValue;
+  if (epi == TC_RESID && lo) e = launch(gemm_int4_tc_kernel<TC_RESID, true>, g, b, smem, st, ta);
+  else if (epi == TC_RAW && lo) e = launch(gemm_int4_tc_kernel<TC_RAW, true>, g, b, smem, st, ta);
+  else if (epi == TC_ROPE_KV && lo) e = launch(gemm_int4_tc_kernel<TC_ROPE_KV, true>, g, b, smem, st, ta);
+  else if (epi == TC_STORE && !lo) e = launch(gemm_int4_tc_kernel<TC_STORE, false>, g, b, smem, st, ta);
+  else return cudaErrorInvalidValue;
+  if (e != cudaSuccess || splits == 1) return e;
+  const dim3 mg(row_tiles, tok_tiles, kTcTokens / kTcMergeTok);
+  if (epi == TC_RESID) return launch(tc_merge_kernel<TC_RESID>, mg, dim3(256), 0, st, ta);
+  if (epi == TC_RAW) return launch(tc_merge_kernel<TC_RAW>, mg, dim3(256), 0, st, ta);
+  if (epi == TC_ROPE_KV) return launch(tc_merge_kernel<TC_ROPE_KV>, mg, dim3(256), 0, st, ta);
+  return launch(tc_merge_kernel<TC_STORE>, mg, dim3(256), 0, st, ta);
 }
 
 template <int HD, int REP, bool F32>
