@@ -135,7 +135,12 @@ constexpr int kTcEpiWarp0 = 8;
 
 constexpr int kTcStages = 4;          // half-group (64 k) operand stages
 constexpr int kTcRaw = 3;             // raw INT4 group stages
-constexpr int kTcRawBytes = 8 * 1024 + 8 * 64;   // 8 16-row tiles x (2 chunks of 512 B + 64 B of scales/zeros)
+// Tensor-core weight layout, one block per (128-row tile, K group): 128 rows
+// x 16 words of 8 nibbles (k = 8j .. 8j + 7 of the group, in the order
+// k0 k2 k4 k6 at bits 0, 4, 8, 12 and k1 k3 k5 k7 at bits 16, 20, 24, 28, so
+// that the 1024-bias unpacking yields the pairs (k0, k1) .. (k6, k7) in
+// order), then 128 fp16 biased zeros 1024 + z.  Rows >= N are zero.
+constexpr int kTcRawBytes = kTcRows * 64 + kTcRows * 2;   // 8448 B
 
 __host__ __device__ inline int tc_nb(bool lo) { return lo ? 2 * kTcTokens : kTcTokens; }  // B rows (MMA N)
 __host__ __device__ inline size_t tc_b_bytes(bool lo) { return (size_t)tc_nb(lo) * 256; }      // B of one group: 64 / 32 KB
@@ -145,8 +150,8 @@ __host__ __device__ inline size_t tc_smem_bytes(bool lo) {
 }
 
 struct TcGemmArgs {
-  const uint4* w;        // INT4 weights in the GEMV tile layout [n16 tiles][K/64][32] (16 B each)
-  const uint2* sz;       // scales / biased zeros [n16 tiles][K/128][8]
+  const uint8_t* wtc;    // INT4 weights in the tensor-core layout [N/128][K/128][kTcRawBytes]
+  const uint2* sz;       // scales / biased zeros [n16 tiles][K/128][8] (GEMV layout; the epilogue's scales)
   int K, N;
   int n16_tiles;         // 16-row tiles present in w (rows beyond N are zero)
   const uint8_t* bt;     // prepared activations [token tiles][K/128][2 atoms][NB rows][128 B]
@@ -259,20 +264,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     // go out before the dependency wait) and issues each stage's B atom as
     // soon as the MMA has released the stage.
     if (lane == 0) {
-      const int kw = a.K >> 6;  // 64-wide chunks per row
       int g_issued = 0;
       auto issue_raw = [&](int it) {
         const int r = it % kTcRaw, g = gmap(it);
-        unsigned char* dst = sR(r);
         mbar_arrive_expect_tx(&raw_full[r], kTcRawBytes);
-        for (int n16 = 0; n16 < 8; ++n16) {
-          int gt = tile * 8 + n16;
-          if (gt >= a.n16_tiles) gt = a.n16_tiles - 1;   // absent rows: any valid tile (their A is zeroed)
-          bulk_g2s(dst + n16 * 1024, reinterpret_cast<const unsigned char*>(a.w) + ((size_t)gt * kw + g * 2) * 512,
-                   1024, &raw_full[r]);
-          bulk_g2s(dst + 8192 + n16 * 64, reinterpret_cast<const unsigned char*>(a.sz) + ((size_t)gt * G + g) * 64,
-                   64, &raw_full[r]);
-        }
+        bulk_g2s(sR(r), a.wtc + ((size_t)tile * G + g) * kTcRawBytes, kTcRawBytes, &raw_full[r]);
       };
       for (; g_issued < ng && g_issued < kTcRaw; ++g_issued) issue_raw(g_issued);
       pdl_wait();
@@ -309,26 +305,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
       if (!mbar_wait_or_fail(&raw_full[r], (unsigned)(it / kTcRaw) & 1u, &s_fail)) break;
       const unsigned char* raw = sR(r);
       unsigned char* A = sA(s);
-      for (int wi = p; wi < 256; wi += kTcUnpack) {
-        const int n16 = wi >> 5, ln = wi & 31;
-        const int gt = tile * 8 + n16;
-        const int r0 = n16 * 16 + (ln >> 2), t = ln & 3;
-        uint4 wv = make_uint4(0, 0, 0, 0);
-        uint32_t zz = 0x64006400u;  // z = 0 for absent rows (their q are 0 too)
-        if (gt < a.n16_tiles) {
-          wv = *reinterpret_cast<const uint4*>(raw + n16 * 1024 + half * 512 + ln * 16);
-          zz = reinterpret_cast<const uint2*>(raw + 8192 + n16 * 64)[ln >> 2].y;
-        }
+      // item = (row, 4 consecutive 8-k chunks of this 64-k atom): one 16-byte
+      // load of 32 nibbles, four 16-byte stores of exact fp16 q - z
+      for (int wi = p; wi < 2 * kTcRows; wi += kTcUnpack) {
+        const int row = wi >> 1, qd = wi & 1;
+        const uint4 wv = *reinterpret_cast<const uint4*>(raw + row * 64 + (half * 8 + qd * 4) * 4);
+        const uint32_t zb = *reinterpret_cast<const uint16_t*>(raw + kTcRows * 64 + row * 2);
+        const uint32_t zz = zb | (zb << 16);
         const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t af[4];
-          unpack_a_frag(words[j], zz, af);
-          const int kb = j * 16 + 2 * t;
-          *reinterpret_cast<uint32_t*>(A + sw128_offset(r0, kb, kTcRows)) = af[0];
-          *reinterpret_cast<uint32_t*>(A + sw128_offset(r0 + 8, kb, kTcRows)) = af[1];
-          *reinterpret_cast<uint32_t*>(A + sw128_offset(r0, kb + 8, kTcRows)) = af[2];
-          *reinterpret_cast<uint32_t*>(A + sw128_offset(r0 + 8, kb + 8, kTcRows)) = af[3];
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t w = words[i];
+          uint4 o;
+          o.x = h2_sub(nib_pair_to_h2_biased(w), zz);
+          o.y = h2_sub(nib_pair_to_h2_biased(w >> 4), zz);
+          o.z = h2_sub(nib_pair_to_h2_biased(w >> 8), zz);
+          o.w = h2_sub(nib_pair_to_h2_biased(w >> 12), zz);
+          const int c = qd * 4 + i;   // 16-byte chunk (8 k) within the 128-byte row
+          *reinterpret_cast<uint4*>(A + row * 128 + ((c ^ (row & 7)) << 4)) = o;
         }
       }
       if (half) mbar_arrive(&raw_empty[r]);
@@ -462,6 +456,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// ---- load-time re-layout for the tensor-core path -------------------------------
+// One thread per 8-nibble word (and, for j == 0, the row's biased zero) of
+// the tensor-core layout, from the storage format (qweight [N][K/8] words,
+// element k in bits 4 (k % 8); qzeros [N][ceil(G/8)] words).
+__global__ void repack_int4_tc_kernel(const uint32_t* __restrict__ qweight, const uint32_t* __restrict__ qzeros,
+                                      int K, int N, uint8_t* __restrict__ out) {
+  const int G = K >> 7, zw = (G + 7) >> 3;
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int row_tiles = (N + kTcRows - 1) / kTcRows;
+  const size_t total = (size_t)row_tiles * G * kTcRows * 16;
+  if (idx >= total) return;
+  const int j = (int)(idx & 15);
+  const int r = (int)((idx >> 4) % kTcRows);
+  const size_t blk = (idx >> 4) / kTcRows;          // rt * G + g
+  const int g = (int)(blk % G), rt = (int)(blk / G);
+  const int n = rt * kTcRows + r;
+  uint8_t* base = out + blk * kTcRawBytes;
+  uint32_t word = 0, z = 0;
+  if (n < N) {
+    const uint32_t src = qweight[(size_t)n * (K >> 3) + g * 16 + j];   // k = 128 g + 8 j + i at bits 4 i
+    // destination nibble slot of k_i: i even -> 4 (i / 2), i odd -> 16 + 4 (i / 2)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) word |= ((src >> (4 * i)) & 0xFu) << ((i & 1) * 16 + 4 * (i >> 1));
+    z = (qzeros[(size_t)n * zw + (g >> 3)] >> (4 * (g & 7))) & 0xFu;
+  }
+  reinterpret_cast<uint32_t*>(base)[r * 16 + j] = word;
+  if (j == 0) reinterpret_cast<uint16_t*>(base + kTcRows * 64)[r] = (uint16_t)(0x6400u + z);
 }
 
 // ---- split-K merge + epilogue ------------------------------------------------

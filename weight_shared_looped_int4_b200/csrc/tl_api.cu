@@ -262,17 +262,21 @@ struct Int4Dev {
   int K = 0, N = 0, n_tiles = 0;
   uint4* w = nullptr;
   uint2* sz = nullptr;
+  uint8_t* tc = nullptr;   // tensor-core layout (prefill), always owned
   bool owned = true;   // false when w / sz live in a block's arena
+  static size_t tc_bytes(int K, int N) { return (size_t)((N + kTcRows - 1) / kTcRows) * (K / 128) * kTcRawBytes; }
   static size_t w_bytes(int K, int N) { return (size_t)(((N + 31) / 32) * 2) * (K / 64) * 32 * sizeof(uint4); }
   static size_t sz_bytes(int K, int N) { return (size_t)(((N + 31) / 32) * 2) * (K / 128) * 8 * sizeof(uint2); }
-  size_t bytes() const { return w_bytes(K, N) + sz_bytes(K, N); }
+  size_t bytes() const { return w_bytes(K, N) + sz_bytes(K, N) + (tc ? tc_bytes(K, N) : 0); }
   void free_all() {
     if (owned) {
       if (w) cudaFree(w);
       if (sz) cudaFree(sz);
     }
+    if (tc) cudaFree(tc);
     w = nullptr;
     sz = nullptr;
+    tc = nullptr;
   }
 };
 
@@ -311,6 +315,7 @@ tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaS
     if (e == cudaSuccess) e = cudaMalloc(&out->w, Int4Dev::w_bytes(K, N));
     if (e == cudaSuccess) e = cudaMalloc(&out->sz, Int4Dev::sz_bytes(K, N));
   }
+  if (e == cudaSuccess) e = cudaMalloc(&out->tc, Int4Dev::tc_bytes(K, N));
   if (e == cudaSuccess) e = cudaMemcpyAsync(dq, h.qweight, qb, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(ds, h.scales, sb, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(dz, h.qzeros, zb, cudaMemcpyHostToDevice, st);
@@ -321,6 +326,9 @@ tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaS
     const size_t ts = (size_t)out->n_tiles * G * 8;
     repack_int4_scales_kernel<<<(unsigned)((ts + 255) / 256), 256, 0, st>>>(
         (const uint16_t*)ds, (const uint32_t*)dz, K, N, out->n_tiles, out->sz);
+    const size_t tt = (size_t)((N + kTcRows - 1) / kTcRows) * G * kTcRows * 16;
+    repack_int4_tc_kernel<<<(unsigned)((tt + 255) / 256), 256, 0, st>>>((const uint32_t*)dq, (const uint32_t*)dz, K,
+                                                                       N, out->tc);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
@@ -444,7 +452,7 @@ cudaError_t launch_prep(int mode, const PrepArgs& p, cudaStream_t st) {
 
 // Runs prep + GEMM for T tokens.  `ta` carries the epilogue outputs; the
 // weight, activation and scratch fields are filled here.
-cudaError_t launch_tc_linear(const uint4* w, const uint2* sz, int K, int N, int n16_tiles, int prep_mode,
+cudaError_t launch_tc_linear(const uint8_t* wtc, const uint2* sz, int K, int N, int n16_tiles, int prep_mode,
                              PrepArgs pa, TcGemmArgs ta, int epi, int T, const TcScratch& sc, cudaStream_t st) {
   const bool lo = prep_mode != PREP_F16;
   if (tc_bt_bytes(T, K, lo) > sc.bt_bytes) return cudaErrorInvalidValue;
@@ -458,7 +466,7 @@ cudaError_t launch_tc_linear(const uint4* w, const uint2* sz, int K, int N, int 
   int splits = std::max(1, std::min(G, sc.n_sm / (row_tiles * tok_tiles)));
   while (splits > 1 && (size_t)splits * row_tiles * tok_tiles * kTcRows * kTcTokens * 4 > sc.partial_bytes) --splits;
   if (row_tiles * tok_tiles > 4096) return cudaErrorInvalidValue;
-  ta.w = w; ta.sz = sz; ta.K = K; ta.N = N; ta.n16_tiles = n16_tiles;
+  ta.wtc = wtc; ta.sz = sz; ta.K = K; ta.N = N; ta.n16_tiles = n16_tiles;
   ta.bt = sc.bt; ta.T = T; ta.splits = splits;
   ta.partial = sc.partial; ta.tickets = sc.tickets; ta.err_flag = sc.err_flag;
   const dim3 g(row_tiles, tok_tiles, splits), b(kTcThreads);
@@ -753,7 +761,7 @@ tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, cudaStream_t st) {
   ta.v_plane = m->v_plane(layer) + lane * m->lane_stride;
   ta.ctx = c.max_ctx; ta.pos0 = 0; ta.theta = c.rope_theta; ta.rope_tab = m->rope_tab;
   kclass(TL_KERNEL_GEMM_TC);
-  TL_CUDA(launch_tc_linear(b.qkv.w, b.qkv.sz, c.d_model, b.qkv.N, b.qkv.n_tiles, PREP_NORM, pa, ta, TC_ROPE_KV,
+  TL_CUDA(launch_tc_linear(b.qkv.tc, b.qkv.sz, c.d_model, b.qkv.N, b.qkv.n_tiles, PREP_NORM, pa, ta, TC_ROPE_KV,
                            T, m->tc, st));
   return TL_OK;
 }
@@ -769,14 +777,14 @@ tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
     pa.x = m->o; pa.ldx = qdim;
     TcGemmArgs ta{};
     ta.out_f32 = m->x; ta.ld_out = d;
-    TL_CUDA(launch_tc_linear(b.o.w, b.o.sz, qdim, d, b.o.n_tiles, PREP_F32, pa, ta, TC_RESID, T, m->tc, st));
+    TL_CUDA(launch_tc_linear(b.o.tc, b.o.sz, qdim, d, b.o.n_tiles, PREP_F32, pa, ta, TC_RESID, T, m->tc, st));
   }
   {  // RMSNorm + gate_up (raw)
     PrepArgs pa{};
     pa.x = m->x; pa.ldx = d; pa.gain = b.ffn_norm; pa.eps = c.rms_eps;
     TcGemmArgs ta{};
     ta.out_f32 = m->gu; ta.ld_out = 2 * F;
-    TL_CUDA(launch_tc_linear(b.gate_up.w, b.gate_up.sz, d, 2 * F, b.gate_up.n_tiles, PREP_NORM, pa, ta, TC_RAW, T,
+    TL_CUDA(launch_tc_linear(b.gate_up.tc, b.gate_up.sz, d, 2 * F, b.gate_up.n_tiles, PREP_NORM, pa, ta, TC_RAW, T,
                              m->tc, st));
   }
   {  // SwiGLU + down + residual
@@ -784,7 +792,7 @@ tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
     pa.x = m->gu; pa.ldx = 2 * F; pa.F = F;
     TcGemmArgs ta{};
     ta.out_f32 = m->x; ta.ld_out = d;
-    TL_CUDA(launch_tc_linear(b.down.w, b.down.sz, F, d, b.down.n_tiles, PREP_SWIGLU, pa, ta, TC_RESID, T, m->tc,
+    TL_CUDA(launch_tc_linear(b.down.tc, b.down.sz, F, d, b.down.n_tiles, PREP_SWIGLU, pa, ta, TC_RESID, T, m->tc,
                              st));
   }
   return TL_OK;
@@ -1424,7 +1432,7 @@ tl_status tl_linear_forward(tl_linear* l, const uint16_t* d_x, int M, uint16_t* 
     pa.xh = reinterpret_cast<const __half*>(d_x); pa.ldx = K;
     TcGemmArgs ta{};
     ta.out_f16 = reinterpret_cast<__half*>(d_y); ta.ld_out = N;
-    TL_CUDA(launch_tc_linear(l->w.w, l->w.sz, K, N, l->w.n_tiles, PREP_F16, pa, ta, TC_STORE, M, sc,
+    TL_CUDA(launch_tc_linear(l->w.tc, l->w.sz, K, N, l->w.n_tiles, PREP_F16, pa, ta, TC_STORE, M, sc,
                              (cudaStream_t)stream));
     return TL_OK;
   }
