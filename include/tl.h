@@ -320,8 +320,8 @@ tl_status tl_op_gqa_decode(const uint16_t *d_q, const uint16_t *d_k, const uint1
  * fixed 4 MiB device array that every GPU loading this library reserves until
  * the process exits; nothing is allocated or freed by the call.
  *   Limits: 1 <= B <= 32, B * n_kv_heads <= 4096, and
- *   B * n_kv_heads * 32 * (n_q_heads/n_kv_heads) * (head_dim + 2) * 4 bytes
- *   + 17 KiB <= 4 MiB (e.g. B = 8, 16/4 heads of 128 needs about 2.1 MiB);
+ *   B * n_kv_heads * 32 * (n_q_heads/n_kv_heads) * (head_dim + 4) * 4 bytes
+ *   + 17 KiB <= 4 MiB (e.g. B = 8, 16/4 heads of 128 needs about 2.2 MiB);
  *   beyond them it returns TL_ERR_UNSUPPORTED and enqueues nothing.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it; make that

@@ -36,6 +36,10 @@ __host__ __device__ inline int decode_split_len(int n_keys) {
   return c;
 }
 
+// Partial results of a split: REP x (hd unnormalised sums, max, sum of
+// weights, 2 pad) floats, so every head's block starts 16-byte aligned.
+constexpr int kPartPad = 4;
+
 __host__ __device__ inline size_t decode_attn_smem_bytes(int hd, int rep) {
   (void)rep;
   return (size_t)2 * kDecodeSub * (hd + kKeyPad) * 2;  // K and V of one split
@@ -56,7 +60,7 @@ struct DecodeAttnArgs {
   float* of;             // [rows][Hq*hd] output (fp32), or
   __half* oh;            // the same in fp16
   int ldo;
-  float* part;           // [rows][Hkv][kDecodeMaxSplits][REP][hd+2]
+  float* part;           // [rows][Hkv][kDecodeMaxSplits][REP][hd + kPartPad]
   unsigned* ticket;      // [rows][Hkv], zero between launches
 };
 
@@ -243,16 +247,17 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
     return;
   }
 
-  constexpr int PSTRIDE = REP * (HD + 2);
+  constexpr int HS = HD + kPartPad;
+  constexpr int PSTRIDE = REP * HS;
   float* pbase = a.part + ((size_t)row * a.Hkv + kvh) * kDecodeMaxSplits * PSTRIDE;
   float* pme = pbase + (size_t)split * PSTRIDE;
   if (dt < HD / 8 && g < REP) {
-    pme[g * (HD + 2) + dt * 8 + 2 * t] = o[0] + o2[0];
-    pme[g * (HD + 2) + dt * 8 + 2 * t + 1] = o[1] + o2[1];
+    pme[g * HS + dt * 8 + 2 * t] = o[0] + o2[0];
+    pme[g * HS + dt * 8 + 2 * t + 1] = o[1] + o2[1];
   }
   if (threadIdx.x < REP) {
-    pme[threadIdx.x * (HD + 2) + HD] = s_m[threadIdx.x];
-    pme[threadIdx.x * (HD + 2) + HD + 1] = s_l[threadIdx.x];
+    pme[threadIdx.x * HS + HD] = s_m[threadIdx.x];
+    pme[threadIdx.x * HS + HD + 1] = s_l[threadIdx.x];
   }
   __threadfence();
   __syncthreads();
@@ -264,22 +269,27 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   if (!s_last) return;
   __threadfence();
 
-  const int d = threadIdx.x;
-  if (d < HD) {
-#pragma unroll
-    for (int h = 0; h < REP; ++h) {
-      float mx = -INFINITY;
-      for (int s = 0; s < nsplit; ++s) mx = fmaxf(mx, __ldcg(pbase + (size_t)s * PSTRIDE + h * (HD + 2) + HD));
-      float num = 0.f, den = 0.f;
-      for (int s = 0; s < nsplit; ++s) {
-        const float* ps = pbase + (size_t)s * PSTRIDE + h * (HD + 2);
-        const float w = expf(__ldcg(ps + HD) - mx);
-        den = fmaf(w, __ldcg(ps + HD + 1), den);
-        num = fmaf(w, __ldcg(ps + d), num);
-      }
-      if (F32) store_out(a.of + ooff + h * HD + d, num / den);
-      else store_out(a.oh + ooff + h * HD + d, num / den);
+  // (max, sum of weights) of every split and head in one round of loads,
+  // then each (head, dim) output from independent loads in split order
+  float* mls = &sc[0][0];   // >= 2 * kDecodeMaxSplits * REP floats
+  for (int e = threadIdx.x; e < nsplit * REP * 2; e += kDecodeThreads) {
+    const int sp = e / (REP * 2), rem = e % (REP * 2);
+    mls[e] = __ldcg(pbase + (size_t)sp * PSTRIDE + (rem >> 1) * HS + HD + (rem & 1));
+  }
+  __syncthreads();
+  for (int oi = threadIdx.x; oi < REP * HD; oi += kDecodeThreads) {
+    const int h = oi / HD, d = oi % HD;
+    float mx = -INFINITY;
+    for (int sp = 0; sp < nsplit; ++sp) mx = fmaxf(mx, mls[(sp * REP + h) * 2]);
+    float num = 0.f, den = 0.f;
+#pragma unroll 8
+    for (int sp = 0; sp < nsplit; ++sp) {
+      const float w = expf(mls[(sp * REP + h) * 2] - mx);
+      den = fmaf(w, mls[(sp * REP + h) * 2 + 1], den);
+      num = fmaf(w, __ldcg(pbase + (size_t)sp * PSTRIDE + h * HS + d), num);
     }
+    if (F32) store_out(a.of + ooff + h * HD + d, num / den);
+    else store_out(a.oh + ooff + h * HD + d, num / den);
   }
   if (threadIdx.x == 0) a.ticket[row * a.Hkv + kvh] = 0u;
 }

@@ -112,7 +112,7 @@ extern "C" tl_status tl_op_gqa_decode_noalloc(const uint16_t* d_q, const uint16_
   if (B < 1 || B > kNoAllocMaxRows)
     return err(TL_ERR_UNSUPPORTED, "B must be in [1, 32] for the no-allocation variant");
   if (B * n_kv_heads > kNoAllocTickets) return err(TL_ERR_UNSUPPORTED, "B * n_kv_heads exceeds 4096");
-  const size_t part_bytes = (size_t)B * n_kv_heads * kDecodeMaxSplits * rep * (head_dim + 2) * sizeof(float);
+  const size_t part_bytes = (size_t)B * n_kv_heads * kDecodeMaxSplits * rep * (head_dim + kPartPad) * sizeof(float);
   if (kPartOffset + part_bytes > kNoAllocScratchBytes)
     return err(TL_ERR_UNSUPPORTED,
                "shape needs " + std::to_string(kPartOffset + part_bytes) +

@@ -974,7 +974,7 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
             alloc((void**)&m->o, (size_t)rows * qdim * 4) && alloc((void**)&m->h, (size_t)rows * c.ffn_dim * 4) &&
             alloc((void**)&m->rows, (size_t)rows * sizeof(RowCtx)) &&
             alloc((void**)&m->tok_index, kMaxLanes * 4) && alloc((void**)&m->out_row, kMaxLanes * 4) &&
-            alloc((void**)&m->attn_part, (size_t)kMaxLanes * c.n_kv_heads * kDecodeMaxSplits * rep * (hd + 2) * 4) &&
+            alloc((void**)&m->attn_part, (size_t)kMaxLanes * c.n_kv_heads * kDecodeMaxSplits * rep * (hd + kPartPad) * 4) &&
             alloc((void**)&m->tickets, (size_t)(kMaxLanes * c.n_kv_heads + 1) * 4) &&
             alloc((void**)&m->head_val, (size_t)m->head_grid * 16 * 4) &&
             alloc((void**)&m->head_idx, (size_t)m->head_grid * 16 * 4) && alloc((void**)&m->err_flag, 4) &&
@@ -998,7 +998,7 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
   if (!ok) return bail(fail(TL_ERR_OOM, "workspace allocation"));
   {  // single-kernel decode step: shapes, device support, resources
     // attention partials share the layered path's buffer, which holds
-    // kMaxLanes x Hkv x kDecodeMaxSplits x rep x (hd + 2) floats
+    // kMaxLanes x Hkv x kDecodeMaxSplits x rep x (hd + kPartPad) floats
     static_assert(kFusedMaxSplits == kDecodeMaxSplits && 2 * kFusedMaxRows <= kMaxLanes,
                   "fused partials ([4 rows][..][hd + 4]) must fit the layered path's buffer");
     int coop = 0;
@@ -1488,7 +1488,7 @@ tl_status tl_op_gqa_decode(const uint16_t* d_q, const uint16_t* d_k, const uint1
   TL_CUDA(init_device_kernels(dev));
   const int rep = n_q_heads / n_kv_heads;
   const size_t rows_b = (size_t)B * sizeof(RowCtx);
-  const size_t part_b = (size_t)B * n_kv_heads * kDecodeMaxSplits * rep * (head_dim + 2) * 4;
+  const size_t part_b = (size_t)B * n_kv_heads * kDecodeMaxSplits * rep * (head_dim + kPartPad) * 4;
   if ((long long)B * n_kv_heads > kOpTickets) return fail(TL_ERR_UNSUPPORTED, "B * n_kv_heads > %d", kOpTickets);
   void* ws = nullptr;
   unsigned* tick = nullptr;
