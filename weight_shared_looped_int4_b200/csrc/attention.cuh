@@ -490,46 +490,4 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const Prefil
   }
 }
 
-// ---- prefill (v1: one warp per query head, online softmax) ----------------
-
-template <int HD, int REP, bool F32>
-__global__ void __launch_bounds__(REP * 32) prefill_attn_simple_kernel(const PrefillAttnArgs a) {
-  constexpr int DPL = HD / 32;
-  const int t = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_trigger();
-  pdl_wait();
-  const int pos = a.pos0 + t;
-  const float scale = 1.0f / sqrtf((float)HD);
-  const size_t qoff = b * a.q_bstride + (size_t)t * a.ldq + (size_t)(kvh * REP + h) * HD + lane * DPL;
-  const __half* kp = a.k + b * a.kv_bstride + (size_t)kvh * a.ctx * HD + lane * DPL;
-  const __half* vp = a.v + b * a.kv_bstride + (size_t)kvh * a.ctx * HD + lane * DPL;
-  float qf[DPL], acc[DPL];
-#pragma unroll
-  for (int d = 0; d < DPL; ++d) {
-    qf[d] = (F32 ? a.qf[qoff + d] : __half2float(a.qh[qoff + d])) * scale;
-    acc[d] = 0.f;
-  }
-  float mx = -INFINITY, l = 0.f;
-  for (int j = 0; j <= pos; ++j) {
-    float s = 0.f;
-#pragma unroll
-    for (int d = 0; d < DPL; ++d) s = fmaf(qf[d], __half2float(kp[(size_t)j * HD + d]), s);
-    s = warp_sum(s);
-    const float mn = fmaxf(mx, s);
-    const float corr = expf(mx - mn);
-    const float p = expf(s - mn);
-    l = l * corr + p;
-#pragma unroll
-    for (int d = 0; d < DPL; ++d) acc[d] = fmaf(p, __half2float(vp[(size_t)j * HD + d]), acc[d] * corr);
-    mx = mn;
-  }
-  const size_t ooff = b * a.o_bstride + (size_t)t * a.ldo + (size_t)(kvh * REP + h) * HD + lane * DPL;
-#pragma unroll
-  for (int d = 0; d < DPL; ++d) {
-    if (F32) store_out(a.of + ooff + d, acc[d] / l);
-    else store_out(a.oh + ooff + d, acc[d] / l);
-  }
-}
-
 }  // namespace tl
