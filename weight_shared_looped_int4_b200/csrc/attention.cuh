@@ -309,10 +309,12 @@ struct PrefillAttnArgs {
   __half* oh;             // fp16 (op API)
   long long o_bstride;
   int ldo;
+  int rep;                // query heads per kv head (the kernel's REP heads are a slice of a group)
 };
 
 // ---- prefill: tiled, tensor cores (m16n8k16), online softmax --------------
-// One CTA per (16-query tile, kv head, batch entry); warp w handles q head
+// One CTA per (16-query tile, slice of REP query heads of one kv group, batch
+// entry; short prompts use smaller slices for more CTAs); warp w handles q head
 // kv_head * REP + w for the 16 queries, so each K/V block staged in shared
 // memory serves all REP heads of the group.  S = Q K^T and O += P V run on the
 // tensor cores; Q and P are split into fp16 pairs (hi, lo) and both halves are
@@ -334,10 +336,11 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const Prefil
   __half* ks = reinterpret_cast<__half*>(psm);             // [64][LD]
   __half* vs = ks + kPfKeys * LD;                          // [64][LD]
 
-  const int qt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int qt = blockIdx.x, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int h = kvh * REP + warp;
+  const int h = blockIdx.y * REP + warp;   // REP divides the group size a.rep
+  const int kvh = h / a.rep;
   const int q0 = qt * 16;
   pdl_trigger();
   pdl_wait();

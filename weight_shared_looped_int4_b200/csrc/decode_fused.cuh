@@ -53,7 +53,7 @@ constexpr int kFusedMaxBlocks = 9;                      // up to 8 pre blocks + 
 constexpr int kFusedItemK = 2048;                       // K of one INT4 ring item
 constexpr int kFusedSlotW = 16384;                      // weight bytes of a slot
 constexpr int kFusedSlotBytes = kFusedSlotW + 1024;     // + scales / zeros
-constexpr int kFusedMaxSlots = 12;
+constexpr int kFusedMaxSlots = 13;
 constexpr int kFusedMaxSplits = 32;                     // key splits per (row, kv head)
 constexpr int kFusedMaxKeys = 256;                      // keys per attention unit
 constexpr long long kFusedWaitNs = 500LL * 1000 * 1000; // grid-barrier time limit

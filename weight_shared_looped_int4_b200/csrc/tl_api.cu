@@ -499,11 +499,17 @@ cudaError_t launch_decode_attn(const DecodeAttnArgs& a, int rows, int hd, int re
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_prefill_attn(const PrefillAttnArgs& a, int B, int hd, int rep, bool f32, cudaStream_t st) {
-  const dim3 grid((a.T + 15) / 16, a.Hkv, B);
+cudaError_t launch_prefill_attn(PrefillAttnArgs a, int B, int hd, int rep, bool f32, cudaStream_t st) {
+  // query heads per CTA: the whole group, halved while the grid would leave
+  // SMs idle (short prompts); each CTA stages its kv head's keys itself
+  int hpc = rep;
+  const int qtiles = (a.T + 15) / 16;
+  while (hpc > 1 && (long)qtiles * (a.Hkv * rep / hpc) * B < 148) hpc /= 2;
+  a.rep = rep;
+  const dim3 grid(qtiles, a.Hkv * rep / hpc, B);
   const size_t smem = prefill_attn_smem_bytes(hd);
 #define C(HD, REP)                                                                                       \
-  if (hd == HD && rep == REP)                                                                            \
+  if (hd == HD && hpc == REP)                                                                            \
     return f32 ? launch(prefill_attn_mma_kernel<HD, REP, true>, grid, dim3(REP * 32), smem, st, a)       \
                : launch(prefill_attn_mma_kernel<HD, REP, false>, grid, dim3(REP * 32), smem, st, a);
   C(64, 1) C(64, 2) C(64, 4) C(64, 8) C(128, 1) C(128, 2) C(128, 4) C(128, 8)
@@ -601,14 +607,17 @@ namespace {
 // Shared-memory plan of the single-kernel decode step for `rows` rows: the
 // largest ring (<= kFusedMaxSlots slots) that fits beside the activation
 // planes and the reduction buffer.  False if not even two slots fit.
+// Head-only launches need only the d-wide activation planes and the head's
+// double reduction buffer, which leaves room for more ring slots.
 bool fused_plan(const tl_model* m, int rows, FusedArgs* f, size_t* smem) {
   const tl_config& c = m->cfg;
   const int qdim = c.n_q_heads * c.head_dim;
-  const int kmax = std::max(std::max(c.d_model, qdim), c.ffn_dim);
+  const int kmax = f->head_only ? c.d_model : std::max(std::max(c.d_model, qdim), c.ffn_dim);
   if (kmax > kFusedStageV4 * 4 * kFusedCompute) return false;
-  const int area = fused_area_bytes(rows, kmax, c.n_q_heads / c.n_kv_heads, c.head_dim);
-  const int red = fused_red_bytes(*f, m->fused_grid);
-  const int xown = fused_xown_bytes(*f, m->fused_grid);
+  const int area = f->head_only ? (2 * rows * (c.d_model + 8) * 2 + 127) / 128 * 128
+                                : fused_area_bytes(rows, kmax, c.n_q_heads / c.n_kv_heads, c.head_dim);
+  const int red = f->head_only ? 2 * kFusedWarps * 64 * 4 : fused_red_bytes(*f, m->fused_grid);
+  const int xown = f->head_only ? 0 : fused_xown_bytes(*f, m->fused_grid);
   const long avail = (long)m->fused_smem_max - area - red - xown;
   const long ns = std::min<long>(kFusedMaxSlots, avail / kFusedSlotBytes);
   if (ns < 2) return false;
