@@ -1,0 +1,428 @@
+// Decode: RMSNorm + QKV INT4 linear + RoPE + KV write + GQA attention of one
+// effective layer in ONE kernel, one thread-block cluster per kv head.
+//
+// What it computes is steps a2-a5 of a decode step (TinyLoop README,
+// "Status": fused RMSNorm + RoPE, GQA with a per-layer KV cache): the same
+// arithmetic as gemv_int4_kernel<.., IN_NORM, EPI_ROPE_KV> followed by
+// decode_attn_kernel (exact integer q - z MMA operands with (hi, lo) fp16
+// activations, fp32 scales and q, fp16 keys/values, fp32 softmax).
+//
+// Why a cluster: attention for kv head g needs exactly the QKV rows of its
+// group (rep query heads, the key head and the value head: (rep + 2) hd
+// rows).  A cluster of kQaCluster CTAs computes those rows, exchanges q and
+// the new key/value through distributed shared memory, synchronises with the
+// hardware cluster barrier and runs the attention over the lane's cache with
+// the keys split across its CTAs; the split results are merged in the rank-0
+// CTA's shared memory.  That removes a kernel boundary (and its global round
+// trips) per layer.
+//
+// CTA c of cluster g: GEMV of RoPE pair units u = c, c + kQaCluster, ...
+// (tiles j and j + hd/32 of one head), weights bulk-copied into shared memory
+// before the programmatic-launch wait; 8 warps split K, each warp's B
+// fragments are loaded once per chunk and reused for every tile.
+#pragma once
+
+#include "attention.cuh"
+#include "common.cuh"
+
+namespace tl {
+
+constexpr int kQaCluster = 16;         // non-portable cluster size (B200 GPCs hold 16 CTAs of this size)
+constexpr int kQaThreads = 256;
+constexpr int kQaWarps = kQaThreads / 32;
+constexpr int kQaMaxRows = 2;
+constexpr int kQaMaxUnits = 2;        // RoPE pair units per CTA
+constexpr int kQaChunk = 64;          // keys per staged chunk
+
+struct QkvAttnArgs {
+  const uint4* w;        // QKV weights, GEMV tile layout [n16 tiles][K/64][32]
+  const uint2* sz;       // [n16 tiles][K/128][8]
+  int K;                 // d_model
+  const float* x;        // residual stream [M][K]
+  const __half* gain;    // attention RMSNorm gains
+  float eps;
+  int M;                 // rows (lanes), <= kQaMaxRows
+  const RowCtx* rows;    // lane and position of each row
+  int hd, rep, Hkv;
+  const float2* rope_tab;
+  float theta;
+  __half* k_plane;       // this layer's K plane of lane 0 [Hkv][ctx][hd]
+  __half* v_plane;
+  long long lane_stride;
+  int ctx;
+  float* o;              // attention output [M][Hq*hd] fp32
+  int* err_flag;
+};
+
+__host__ __device__ inline int qa_units(int rep, int hd) { return (rep + 2) * hd / 32; }
+__host__ __device__ inline int qa_units_per_cta(int rep, int hd) {
+  return (qa_units(rep, hd) + kQaCluster - 1) / kQaCluster;
+}
+// Shared memory: weight tiles (reused for key/value chunks), partial results
+// of every rank (used in rank 0), activation planes, reduction buffer, q and
+// the new key/value of every row.
+struct QaLayout {
+  size_t w, part, act, red, q, kv, total;
+};
+__host__ __device__ inline QaLayout qa_layout(int K, int M, int rep, int hd) {
+  QaLayout L;
+  const size_t tile = (size_t)(K / 64) * 512 + (size_t)(K / 128) * 64;
+  size_t wbytes = (size_t)2 * qa_units_per_cta(rep, hd) * tile;
+  const size_t chunk = (size_t)2 * kQaChunk * hd * 2;
+  if (wbytes < chunk) wbytes = chunk;
+  L.w = 0;
+  L.part = (wbytes + 127) / 128 * 128;
+  L.act = L.part + ((size_t)kQaCluster * M * rep * (hd + kPartPad) * 4 + 127) / 128 * 128;
+  L.red = L.act + ((size_t)M * (K + 8) * 2 * 2 + 127) / 128 * 128;
+  L.q = L.red + (size_t)kQaWarps * 2 * kQaMaxUnits * 64 * 4;
+  L.kv = L.q + (size_t)M * rep * hd * 4;
+  L.total = L.kv + (size_t)2 * M * hd * 4 + 128;   // + scores and softmax state
+  L.total += (size_t)(rep * kQaChunk + 4 * rep) * 4;
+  return L;
+}
+
+__device__ __forceinline__ unsigned qa_cluster_rank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void qa_cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared-memory address of `p` in the CTA of cluster rank `rank`.
+__device__ __forceinline__ unsigned qa_peer(const void* p, unsigned rank) {
+  unsigned out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+  return out;
+}
+__device__ __forceinline__ void qa_st_peer(unsigned addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnArgs a) {
+  constexpr int DPL = HD / 32;
+  constexpr int ROW16 = HD / 8;
+  extern __shared__ __align__(128) unsigned char qsm[];
+  __shared__ __align__(8) uint64_t wbar;
+  __shared__ int s_ok;
+  __shared__ float s_ss[kQaMaxRows][kQaWarps];
+  const int K = a.K, M = a.M, rep = a.rep;
+  const QaLayout L = qa_layout(K, M, rep, HD);
+  unsigned char* wsm = qsm + L.w;
+  float* part = reinterpret_cast<float*>(qsm + L.part);     // [rank][m][h][hd + kPartPad]
+  __half* xs = reinterpret_cast<__half*>(qsm + L.act);
+  __half* xl = xs + (size_t)M * (K + 8);
+  float* red = reinterpret_cast<float*>(qsm + L.red);       // [warp][tile][16][4]
+  float* qb = reinterpret_cast<float*>(qsm + L.q);          // [m][rep * hd]
+  float* knew = reinterpret_cast<float*>(qsm + L.kv);       // [m][hd]
+  float* vnew = knew + (size_t)M * HD;                       // [m][hd]
+  float* sc = vnew + (size_t)M * HD;                         // [rep][kQaChunk]
+  float* ml = sc + rep * kQaChunk;                           // [rep][4]: max, sum, rescale
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, t4 = lane & 3;
+  const unsigned crank = qa_cluster_rank();
+  const int c = (int)crank, grp = blockIdx.y;
+  const int U = qa_units(rep, HD), hp = HD / 32;
+  const int qdim = a.Hkv * rep * HD, kvdim = a.Hkv * HD;
+  const size_t wt_bytes = (size_t)(K / 64) * 512, sz_bytes = (size_t)(K / 128) * 64;
+  int nu = 0, units[kQaMaxUnits];
+  for (int u = c; u < U && nu < kQaMaxUnits; u += kQaCluster) units[nu++] = u;
+  // group-local unit -> global 16-row tile of the QKV output: group heads are
+  // rep query heads, then the key head, then the value head
+  auto unit_tile = [&](int u, int second) -> int {
+    const int hh = u / hp, j = u % hp;
+    const int row_base = hh < rep ? (grp * rep + hh) * HD : (hh == rep ? qdim + grp * HD : qdim + kvdim + grp * HD);
+    return row_base / 16 + j + (second ? hp : 0);
+  };
+
+  pdl_trigger();
+  if (tid == 0) {
+    mbar_init(&wbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&wbar, (unsigned)(2 * nu * (wt_bytes + sz_bytes)));
+    for (int i = 0; i < 2 * nu; ++i) {
+      const int tile = unit_tile(units[i >> 1], i & 1);
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
+      for (size_t off = 0; off < wt_bytes; off += 32768) {
+        const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
+        bulk_g2s(wsm + i * wt_bytes + off, src + off, n, &wbar);
+      }
+      bulk_g2s(wsm + 2 * nu * wt_bytes + i * sz_bytes,
+               reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes, (unsigned)sz_bytes, &wbar);
+    }
+  }
+  // every rank of the cluster must be running before any distributed
+  // shared-memory write reaches it (the first ones come after the GEMV)
+  qa_cluster_sync();
+  pdl_wait();
+
+  // ---- RMSNorm of the rows into the (hi, lo) planes -------------------------
+  for (int m = 0; m < M; ++m) {
+    const float* src = a.x + (size_t)m * K;
+    float ss = 0.f;
+    for (int k = tid * 4; k < K; k += 4 * kQaThreads) {
+      const float4 v = *reinterpret_cast<const float4*>(src + k);
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) s_ss[m][warp] = ss;
+  }
+  __syncthreads();
+  for (int m = 0; m < M; ++m) {
+    const float* src = a.x + (size_t)m * K;
+    float ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < kQaWarps; ++w) ss += s_ss[m][w];
+    const float rs = 1.0f / sqrtf(ss / (float)K + a.eps);
+    for (int k = tid * 4; k < K; k += 4 * kQaThreads) {
+      float4 v = *reinterpret_cast<const float4*>(src + k);
+      const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
+      const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k + 2));
+      v.x = (v.x * rs) * g01.x; v.y = (v.y * rs) * g01.y;
+      v.z = (v.z * rs) * g23.x; v.w = (v.w * rs) * g23.y;
+      const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+      const float2 r01 = __half22float2(h01), r23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(v.x - r01.x, v.y - r01.y);
+      const __half2 l23 = __floats2half2_rn(v.z - r23.x, v.w - r23.y);
+      uint2 ph, pl;
+      ph.x = *reinterpret_cast<const uint32_t*>(&h01); ph.y = *reinterpret_cast<const uint32_t*>(&h23);
+      pl.x = *reinterpret_cast<const uint32_t*>(&l01); pl.y = *reinterpret_cast<const uint32_t*>(&l23);
+      *reinterpret_cast<uint2*>(xs + (size_t)m * (K + 8) + k) = ph;
+      *reinterpret_cast<uint2*>(xl + (size_t)m * (K + 8) + k) = pl;
+    }
+  }
+  if (tid == 0) {
+    s_ok = mbar_wait(&wbar, 0) ? 1 : 0;
+    if (!s_ok) atomicOr(a.err_flag, kErrTimeout);
+  }
+  __syncthreads();
+  const bool ok = s_ok != 0;   // on a time-out the control flow stays the same (cluster barriers)
+
+  // ---- GEMV of this CTA's tiles: warps split K, B fragments shared --------
+  {
+    const int nck = K / 64;
+    const int c0 = warp * nck / kQaWarps, c1 = (warp + 1) * nck / kQaWarps;
+    const int brow = g8 >> 1;
+    const __half* bsrc = ((g8 & 1) ? xl : xs) + (size_t)brow * (K + 8) + 2 * t4;
+    const bool bok = brow < M;
+    float acc[2 * kQaMaxUnits][4];
+#pragma unroll
+    for (int i = 0; i < 2 * kQaMaxUnits; ++i)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
+    for (int ci = c0; ok && ci < c1; ++ci) {
+      uint32_t bf[4][2];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bf[j][0] = bok ? *reinterpret_cast<const uint32_t*>(bsrc + ci * 64 + j * 16) : 0u;
+        bf[j][1] = bok ? *reinterpret_cast<const uint32_t*>(bsrc + ci * 64 + j * 16 + 8) : 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 2 * kQaMaxUnits; ++i) {
+        if (i < 2 * nu) {
+          const uint4 wv = *reinterpret_cast<const uint4*>(wsm + i * wt_bytes + (size_t)ci * 512 + lane * 16);
+          const uint2 sv =
+              *reinterpret_cast<const uint2*>(wsm + 2 * nu * wt_bytes + i * sz_bytes + (size_t)(ci >> 1) * 64 + g8 * 8);
+          const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
+          float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t af[4];
+            unpack_a_frag(words[j], sv.y, af);
+            if (j & 1) mma_f16_16816(t1, af, bf[j][0], bf[j][1]);
+            else mma_f16_16816(t0, af, bf[j][0], bf[j][1]);
+          }
+          const float2 s2 = h2_to_f2(sv.x);
+          acc[i][0] = fmaf(s2.x, t0[0] + t1[0], acc[i][0]);
+          acc[i][1] = fmaf(s2.x, t0[1] + t1[1], acc[i][1]);
+          acc[i][2] = fmaf(s2.y, t0[2] + t1[2], acc[i][2]);
+          acc[i][3] = fmaf(s2.y, t0[3] + t1[3], acc[i][3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 2 * kQaMaxUnits; ++i) {
+      if (i < 2 * nu) {
+        float* r = red + ((size_t)warp * 2 * kQaMaxUnits + i) * 64;
+        r[g8 * 4 + t4] = acc[i][0] + acc[i][1];        // tile row g8, activation row t4 (hi + lo)
+        r[(g8 + 8) * 4 + t4] = acc[i][2] + acc[i][3];  // tile row g8 + 8
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- epilogue: RoPE; q to every rank, k / v to the cache and every rank --
+  for (int e = tid; e < nu * 16 * M; e += kQaThreads) {
+    const int ul = e / (16 * M), rem = e % (16 * M), r = rem & 15, m = rem >> 4;
+    float va = 0.f, vb = 0.f;
+#pragma unroll
+    for (int w = 0; w < kQaWarps; ++w) {
+      va += red[((size_t)w * 2 * kQaMaxUnits + 2 * ul) * 64 + r * 4 + m];
+      vb += red[((size_t)w * 2 * kQaMaxUnits + 2 * ul + 1) * 64 + r * 4 + m];
+    }
+    const int u = units[ul], hh = u / hp, j = (u % hp) * 16 + r;   // element j < hd/2 of group head hh
+    const RowCtx rc = a.rows[m];
+    float e0 = va, e1 = vb;                                          // elements j and j + hd/2
+    if (hh <= rep) {                                                 // query or key: rotate
+      const float2 cs = rope_cs(a.rope_tab, rc.pos, j, HD, a.theta);
+      e0 = va * cs.x - vb * cs.y;
+      e1 = vb * cs.x + va * cs.y;
+    }
+    float* dst_s;
+    if (hh < rep) {
+      dst_s = qb + (size_t)m * rep * HD + hh * HD;
+    } else {
+      __half* cache = (hh == rep ? a.k_plane : a.v_plane) + rc.lane * a.lane_stride +
+                      ((size_t)grp * a.ctx + rc.pos) * HD;
+      const __half h0 = __float2half_rn(e0), h1 = __float2half_rn(e1);
+      if (ok) { cache[j] = h0; cache[j + HD / 2] = h1; }
+      e0 = __half2float(h0);    // attention reads the stored (fp16) key / value
+      e1 = __half2float(h1);
+      dst_s = (hh == rep ? knew : vnew) + (size_t)m * HD;
+    }
+    for (unsigned rk = 0; rk < kQaCluster; ++rk) {
+      qa_st_peer(qa_peer(dst_s + j, rk), e0);
+      qa_st_peer(qa_peer(dst_s + j + HD / 2, rk), e1);
+    }
+  }
+  qa_cluster_sync();   // #1: q and the new key / value are in every rank
+
+  // ---- attention over this rank's key split, per row -------------------------
+  const float scale = 1.0f / sqrtf((float)HD);
+  __half* ks = reinterpret_cast<__half*>(wsm);            // [kQaChunk][HD]
+  __half* vs = ks + kQaChunk * HD;
+  for (int m = 0; m < M; ++m) {
+    const RowCtx rc = a.rows[m];
+    const int n = rc.pos + 1;
+    const int C = (n + kQaCluster - 1) / kQaCluster;
+    const int j0 = min(n, c * C), j1 = min(n, j0 + C);
+    const __half* kb = a.k_plane + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
+    const __half* vb = a.v_plane + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
+    const float* qrow = qb + (size_t)m * rep * HD;
+    float acc2[4] = {0.f, 0.f, 0.f, 0.f};    // (head, dim) = tid + i * 256, rep * HD <= 1024
+    if (tid < rep) { ml[4 * tid] = -INFINITY; ml[4 * tid + 1] = 0.f; ml[4 * tid + 2] = 0.f; }
+    __syncthreads();
+    for (int jc = j0; jc < j1; jc += kQaChunk) {
+      const int nk = min(kQaChunk, j1 - jc);
+      // chunk into shared memory; the row's newest key / value come from the cluster
+      for (int e = tid; e < 2 * kQaChunk * ROW16; e += kQaThreads) {
+        const int kv = e / (kQaChunk * ROW16), rem = e % (kQaChunk * ROW16);
+        const int key = rem / ROW16, pc = rem % ROW16;
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (key < nk) {
+          const int jj = jc + key;
+          if (jj == rc.pos) {
+            const float* s = (kv ? vnew : knew) + (size_t)m * HD + pc * 8;
+            __half2 h[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(s[2 * q], s[2 * q + 1]);
+            val = *reinterpret_cast<uint4*>(h);
+          } else {
+            val = __ldcg(reinterpret_cast<const uint4*>((kv ? vb : kb) + (size_t)jj * HD) + pc);
+          }
+        }
+        reinterpret_cast<uint4*>(ks)[e] = val;
+      }
+      __syncthreads();
+      for (int jj = warp; jj < nk; jj += kQaWarps) {
+        const __half* kp = ks + jj * HD + lane * DPL;
+        float kf[DPL];
+        if constexpr (DPL == 4) {
+          const uint2 u2 = *reinterpret_cast<const uint2*>(kp);
+          const float2 f01 = h2_to_f2(u2.x), f23 = h2_to_f2(u2.y);
+          kf[0] = f01.x; kf[1] = f01.y; kf[2] = f23.x; kf[3] = f23.y;
+        } else {
+          const float2 f01 = h2_to_f2(*reinterpret_cast<const unsigned*>(kp));
+          kf[0] = f01.x; kf[1] = f01.y;
+        }
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          if (h < rep) {
+            float dot = 0.f;
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) dot = fmaf(qrow[h * HD + lane * DPL + i], kf[i], dot);
+            dot = warp_sum(dot);
+            if (lane == 0) sc[h * kQaChunk + jj] = dot * scale;
+          }
+        }
+      }
+      __syncthreads();
+      if (warp < rep) {
+        float* sh = sc + warp * kQaChunk;
+        float mx = -INFINITY;
+        for (int jj = lane; jj < nk; jj += 32) mx = fmaxf(mx, sh[jj]);
+        mx = warp_max(mx);
+        const float m_old = ml[4 * warp], m_new = fmaxf(m_old, mx);
+        float sum = 0.f;
+        for (int jj = lane; jj < nk; jj += 32) {
+          const float p = expf(sh[jj] - m_new);
+          sh[jj] = p;
+          sum += p;
+        }
+        sum = warp_sum(sum);
+        if (lane == 0) {
+          const float alpha = expf(m_old - m_new);
+          ml[4 * warp] = m_new;
+          ml[4 * warp + 1] = ml[4 * warp + 1] * alpha + sum;
+          ml[4 * warp + 2] = alpha;
+        }
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int oi = tid + i * kQaThreads;
+        if (oi < rep * HD) {
+          const int h = oi / HD, dim = oi % HD;
+          const float* ph = sc + h * kQaChunk;
+          float v = acc2[i] * ml[4 * h + 2];
+#pragma unroll 8
+          for (int jj = 0; jj < nk; ++jj) v = fmaf(ph[jj], __half2float(vs[jj * HD + dim]), v);
+          acc2[i] = v;
+        }
+      }
+      __syncthreads();   // the chunk buffers are reused
+    }
+    // partial (sums, max, sum of weights) of this rank into rank 0
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int oi = tid + i * kQaThreads;
+      if (oi < rep * HD) {
+        const int h = oi / HD, dim = oi % HD;
+        float* pp = part + (((size_t)c * M + m) * rep + h) * (HD + kPartPad);
+        qa_st_peer(qa_peer(pp + dim, 0), acc2[i]);
+        if (dim == 0) {
+          qa_st_peer(qa_peer(pp + HD, 0), ml[4 * h]);
+          qa_st_peer(qa_peer(pp + HD + 1, 0), ml[4 * h + 1]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+  qa_cluster_sync();   // #2: every rank's partials are in rank 0
+
+  // ---- rank 0 merges the ranks in order --------------------------------------
+  if (c == 0) {
+    for (int e = tid; e < M * rep * HD; e += kQaThreads) {
+      const int m = e / (rep * HD), oi = e % (rep * HD), h = oi / HD, dim = oi % HD;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int rk = 0; rk < kQaCluster; ++rk)
+        mx = fmaxf(mx, part[(((size_t)rk * M + m) * rep + h) * (HD + kPartPad) + HD]);
+      float num = 0.f, den = 0.f;
+#pragma unroll
+      for (int rk = 0; rk < kQaCluster; ++rk) {
+        const float* pp = part + (((size_t)rk * M + m) * rep + h) * (HD + kPartPad);
+        const float l = pp[HD + 1];
+        if (l > 0.f) {   // ranks without keys contribute nothing
+          const float w = expf(pp[HD] - mx);
+          num = fmaf(w, pp[dim], num);
+          den = fmaf(w, l, den);
+        }
+      }
+      if (ok) a.o[(size_t)m * (a.Hkv * rep * HD) + (size_t)(grp * rep + h) * HD + dim] = num / den;
+    }
+  }
+}
+
+}  // namespace tl

@@ -26,6 +26,7 @@
 #include "gemm_tc.cuh"
 #include "gemv_int4.cuh"
 #include "misc.cuh"
+#include "qkv_attn.cuh"
 
 using namespace tl;
 
@@ -109,8 +110,8 @@ inline void kclass(int c) { g_cls = c; }
 // programmatic dependent launch (and the current L2 access-policy window);
 // `coop` launches are cooperative (all CTAs co-resident) and get neither.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_impl(bool coop, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                        Args&&... args) {
+cudaError_t launch_impl(bool coop, unsigned cluster_x, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                        cudaStream_t st, Args&&... args) {
   Profiler* pr = g_prof;
   const bool timed = pr && g_cls >= 0 && (pr->mask & (1u << g_cls)) && pr->used < Profiler::kCapacity;
   if (timed) {
@@ -129,7 +130,7 @@ cudaError_t launch_impl(bool coop, void (*kern)(KArgs...), dim3 grid, dim3 block
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   if (coop) {
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
@@ -140,9 +141,16 @@ cudaError_t launch_impl(bool coop, void (*kern)(KArgs...), dim3 grid, dim3 block
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (!coop && g_window.num_bytes) {
-    attr[1].id = cudaLaunchAttributeAccessPolicyWindow;
-    attr[1].val.accessPolicyWindow = g_window;
-    cfg.numAttrs = 2;
+    attr[cfg.numAttrs].id = cudaLaunchAttributeAccessPolicyWindow;
+    attr[cfg.numAttrs].val.accessPolicyWindow = g_window;
+    ++cfg.numAttrs;
+  }
+  if (cluster_x) {
+    attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+    attr[cfg.numAttrs].val.clusterDim.x = cluster_x;
+    attr[cfg.numAttrs].val.clusterDim.y = 1;
+    attr[cfg.numAttrs].val.clusterDim.z = 1;
+    ++cfg.numAttrs;
   }
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
   if (e == cudaSuccess) g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -157,7 +165,7 @@ cudaError_t launch_impl(bool coop, void (*kern)(KArgs...), dim3 grid, dim3 block
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                    Args&&... args) {
-  return launch_impl(false, kern, grid, block, smem, st, std::forward<Args>(args)...);
+  return launch_impl(false, 0u, kern, grid, block, smem, st, std::forward<Args>(args)...);
 }
 
 constexpr size_t kMaxDynSmem = 220 * 1024;  // budget for dynamic smem per CTA
@@ -194,6 +202,12 @@ cudaError_t init_device_kernels(int dev) {
   SET3(IN_F16, EPI_STORE) SET3(IN_F32, EPI_RESID) SET3(IN_NORM, EPI_SWIGLU) SET3(IN_NORM, EPI_ROPE_KV)
 #undef SET3
 #undef SET
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<64>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<128>, dev);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qkv_attn_kernel<64>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qkv_attn_kernel<128>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess) e = allow_max_smem(decode_fused_kernel<64>, dev);
   if (e == cudaSuccess) e = allow_max_smem(decode_fused_kernel<128>, dev);
   if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<1>, dev);
@@ -564,6 +578,8 @@ struct tl_model {
   };
   std::map<std::string, Graph> graphs;   // decode step graphs by row pattern
   bool use_graphs = true;
+  bool use_qkv_attn = true;       // clustered QKV + attention kernel for <= kQaMaxRows rows
+  int qa_smem_max = 0;            // dynamic shared memory it may use
   int decode_path = TL_DECODE_AUTO;
   // single-kernel decode step
   bool fused_ok = false;          // the model's shapes and the device allow it
@@ -717,6 +733,46 @@ tl_status run_decode_attn(tl_model* m, int layer, int M, const RowCtx* rows, con
   da.part = m->attn_part; da.ticket = m->attn_tickets();
   kclass(TL_KERNEL_ATTN_DECODE);
   TL_CUDA(launch_decode_attn(da, M, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
+  return TL_OK;
+}
+
+// QKV projection + RoPE + KV write + attention of M <= kQaMaxRows decode rows
+// in one clustered kernel (see qkv_attn.cuh), when the shapes allow it.
+// A model-level choice (shapes and device only, never the row count), so a
+// lane's arithmetic does not depend on which lanes share the step.
+bool qkv_attn_ok(const tl_model* m) {
+  const tl_config& c = m->cfg;
+  const int rep = c.n_q_heads / c.n_kv_heads;
+  if (!m->use_qkv_attn || (c.head_dim != 64 && c.head_dim != 128)) return false;
+  if (qa_units_per_cta(rep, c.head_dim) > kQaMaxUnits || rep * c.head_dim > 4 * kQaThreads) return false;
+  return qa_layout(c.d_model, kQaMaxRows, rep, c.head_dim).total <= (size_t)m->qa_smem_max;
+}
+
+// Rows are taken kQaMaxRows per launch; each row's result is independent of
+// the others in its launch.
+tl_status run_qkv_attn(tl_model* m, int layer, int M, const RowCtx* rows, cudaStream_t st) {
+  WindowScope window_scope(m, layer);
+  const tl_config& c = m->cfg;
+  const BlockDev& b = m->block(layer);
+  const int qdim = c.n_q_heads * c.head_dim;
+  kclass(TL_KERNEL_QKV);
+  for (int r0 = 0; r0 < M; r0 += kQaMaxRows) {
+    QkvAttnArgs a{};
+    a.w = b.qkv.w; a.sz = b.qkv.sz; a.K = c.d_model;
+    a.x = m->x + (size_t)r0 * c.d_model; a.gain = b.attn_norm; a.eps = c.rms_eps;
+    a.M = std::min(kQaMaxRows, M - r0); a.rows = rows + r0;
+    a.hd = c.head_dim; a.rep = c.n_q_heads / c.n_kv_heads; a.Hkv = c.n_kv_heads;
+    a.rope_tab = m->rope_tab; a.theta = c.rope_theta;
+    a.k_plane = m->k_plane(layer); a.v_plane = m->v_plane(layer);
+    a.lane_stride = m->lane_stride; a.ctx = c.max_ctx;
+    a.o = m->o + (size_t)r0 * qdim; a.err_flag = m->err_flag;
+    const size_t smem = qa_layout(c.d_model, a.M, a.rep, c.head_dim).total;
+    const dim3 grid(kQaCluster, c.n_kv_heads);
+    if (c.head_dim == 64)
+      TL_CUDA(launch_impl(false, (unsigned)kQaCluster, qkv_attn_kernel<64>, grid, dim3(kQaThreads), smem, st, a));
+    else
+      TL_CUDA(launch_impl(false, (unsigned)kQaCluster, qkv_attn_kernel<128>, grid, dim3(kQaThreads), smem, st, a));
+  }
   return TL_OK;
 }
 
@@ -1053,6 +1109,32 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     }
     cudaGetLastError();
   }
+  {
+    cudaFuncAttributes fa{};
+    int optin = 0;
+    if (cudaFuncGetAttributes(&fa, hd == 64 ? qkv_attn_kernel<64> : qkv_attn_kernel<128>) == cudaSuccess &&
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) == cudaSuccess)
+      m->qa_smem_max = optin - (int)fa.sharedSizeBytes;
+    // the clustered kernel is used only if a cluster of its size fits the GPU
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(kQaCluster, c.n_kv_heads);
+    lc.blockDim = dim3(kQaThreads);
+    lc.dynamicSmemBytes = qa_layout(d, kQaMaxRows, rep, hd).total;
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeClusterDimension;
+    la[0].val.clusterDim.x = kQaCluster;
+    la[0].val.clusterDim.y = 1;
+    la[0].val.clusterDim.z = 1;
+    lc.attrs = la;
+    lc.numAttrs = 1;
+    int n_clusters = 0;
+    if (lc.dynamicSmemBytes > (size_t)m->qa_smem_max ||
+        cudaOccupancyMaxActiveClusters(&n_clusters, hd == 64 ? qkv_attn_kernel<64> : qkv_attn_kernel<128>, &lc) !=
+            cudaSuccess ||
+        n_clusters < 1)
+      m->use_qkv_attn = false;
+    cudaGetLastError();
+  }
   m->ws_bytes = ws;
   if (cudaStreamSynchronize(st) != cudaSuccess) return bail(fail(TL_ERR_CUDA, "setup sync"));
   m->lane_len.assign(c.max_lanes + 1, 0);
@@ -1168,9 +1250,9 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
     if (!fused_plan(m, n_lanes, &f, &smem)) return fail(TL_ERR_UNSUPPORTED, "single-kernel decode: no shared-memory plan");
     kclass(TL_KERNEL_DECODE_FUSED);
     if (c.head_dim == 64)
-      TL_CUDA(launch_impl(true, decode_fused_kernel<64>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
+      TL_CUDA(launch_impl(true, 0u, decode_fused_kernel<64>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
     else
-      TL_CUDA(launch_impl(true, decode_fused_kernel<128>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
+      TL_CUDA(launch_impl(true, 0u, decode_fused_kernel<128>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
     for (int i = 0; i < n_lanes; ++i) m->lane_len[h_lane_ids[i]] += 1;
     return TL_OK;
   }
@@ -1188,8 +1270,13 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
   auto body = [&](cudaStream_t s) -> tl_status {
     for (int layer = 0; layer < max_layers; ++layer) {
       const int M = active[layer];
-      tl_status rc = run_qkv(m, layer, M, m->x, m->rows, m->q, s);
-      if (rc == TL_OK) rc = run_decode_attn(m, layer, M, m->rows, m->q, m->o, s);
+      tl_status rc = TL_OK;
+      if (qkv_attn_ok(m)) {
+        rc = run_qkv_attn(m, layer, M, m->rows, s);
+      } else {
+        rc = run_qkv(m, layer, M, m->x, m->rows, m->q, s);
+        if (rc == TL_OK) rc = run_decode_attn(m, layer, M, m->rows, m->q, m->o, s);
+      }
       if (rc == TL_OK) rc = run_ffn(m, layer, M, m->x, m->o, m->h, s);
       if (rc != TL_OK) return rc;
     }
