@@ -157,28 +157,43 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   qa_cluster_sync();
   pdl_wait();
 
-  // ---- RMSNorm of the rows into the (hi, lo) planes -------------------------
-  for (int m = 0; m < M; ++m) {
-    const float* src = a.x + (size_t)m * K;
+  // ---- RMSNorm of the rows into the (hi, lo) planes: every thread loads its
+  // columns of every row (and the gains) at once and keeps them in registers
+  constexpr int V4 = 4;                       // float4 columns per thread and row: K <= 4096
+  float4 xv[kQaMaxRows][V4];
+  uint2 gv[V4];
+#pragma unroll
+  for (int i = 0; i < V4; ++i) {
+    const int k = tid * 4 + i * 4 * kQaThreads;
+    gv[i] = k < K ? *reinterpret_cast<const uint2*>(a.gain + k) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int m = 0; m < kQaMaxRows; ++m)
+      xv[m][i] = (m < M && k < K) ? *reinterpret_cast<const float4*>(a.x + (size_t)m * K + k)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int m = 0; m < kQaMaxRows; ++m) {
     float ss = 0.f;
-    for (int k = tid * 4; k < K; k += 4 * kQaThreads) {
-      const float4 v = *reinterpret_cast<const float4*>(src + k);
-      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-    }
+#pragma unroll
+    for (int i = 0; i < V4; ++i)
+      ss += xv[m][i].x * xv[m][i].x + xv[m][i].y * xv[m][i].y + xv[m][i].z * xv[m][i].z + xv[m][i].w * xv[m][i].w;
     ss = warp_sum(ss);
     if (lane == 0) s_ss[m][warp] = ss;
   }
   __syncthreads();
-  for (int m = 0; m < M; ++m) {
-    const float* src = a.x + (size_t)m * K;
+#pragma unroll
+  for (int m = 0; m < kQaMaxRows; ++m) {
+    if (m >= M) continue;
     float ss = 0.f;
 #pragma unroll
     for (int w = 0; w < kQaWarps; ++w) ss += s_ss[m][w];
     const float rs = 1.0f / sqrtf(ss / (float)K + a.eps);
-    for (int k = tid * 4; k < K; k += 4 * kQaThreads) {
-      float4 v = *reinterpret_cast<const float4*>(src + k);
-      const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
-      const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k + 2));
+#pragma unroll
+    for (int i = 0; i < V4; ++i) {
+      const int k = tid * 4 + i * 4 * kQaThreads;
+      if (k >= K) continue;
+      float4 v = xv[m][i];
+      const float2 g01 = h2_to_f2(gv[i].x), g23 = h2_to_f2(gv[i].y);
       v.x = (v.x * rs) * g01.x; v.y = (v.y * rs) * g01.y;
       v.z = (v.z * rs) * g23.x; v.w = (v.w * rs) * g23.y;
       const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);

@@ -743,7 +743,7 @@ tl_status run_decode_attn(tl_model* m, int layer, int M, const RowCtx* rows, con
 bool qkv_attn_ok(const tl_model* m) {
   const tl_config& c = m->cfg;
   const int rep = c.n_q_heads / c.n_kv_heads;
-  if (!m->use_qkv_attn || (c.head_dim != 64 && c.head_dim != 128)) return false;
+  if (!m->use_qkv_attn || (c.head_dim != 64 && c.head_dim != 128) || c.d_model > 4 * 4 * kQaThreads) return false;
   if (qa_units_per_cta(rep, c.head_dim) > kQaMaxUnits || rep * c.head_dim > 4 * kQaThreads) return false;
   return qa_layout(c.d_model, kQaMaxRows, rep, c.head_dim).total <= (size_t)m->qa_smem_max;
 }
