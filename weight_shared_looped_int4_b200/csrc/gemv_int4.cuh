@@ -176,6 +176,56 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
       for (int k = threadIdx.x * 8; k < K; k += 8 * kGemvThreads)
         *reinterpret_cast<uint4*>(dst + k) = *reinterpret_cast<const uint4*>(src + k);
     }
+  } else if (IN == IN_NORM && M <= 4 && K <= 8 * kGemvThreads) {
+    // few short rows: one pass, the row values and gains stay in registers
+    // (one round trip to L2 instead of two)
+    float4 xv[4][2];
+    uint2 gv[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int k = threadIdx.x * 4 + i * 4 * kGemvThreads;
+      gv[i] = k < K ? *reinterpret_cast<const uint2*>(a.gain + k) : make_uint2(0u, 0u);
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        xv[m][i] = (m < M && k < K) ? *reinterpret_cast<const float4*>(a.x + (size_t)m * a.ldx + k)
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        ss += xv[m][i].x * xv[m][i].x + xv[m][i].y * xv[m][i].y + xv[m][i].z * xv[m][i].z + xv[m][i].w * xv[m][i].w;
+      ss = warp_sum(ss);
+      if (lane == 0 && m < M) ssq[m * 8 + warp] = ss;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      if (m >= M) continue;
+      float ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) ss += ssq[m * 8 + w];
+      const float rs = 1.0f / sqrtf(ss / (float)K + a.eps);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int k = threadIdx.x * 4 + i * 4 * kGemvThreads;
+        if (k >= K) continue;
+        float4 v = xv[m][i];
+        const float2 g01 = h2_to_f2(gv[i].x), g23 = h2_to_f2(gv[i].y);
+        v.x = (v.x * rs) * g01.x; v.y = (v.y * rs) * g01.y;
+        v.z = (v.z * rs) * g23.x; v.w = (v.w * rs) * g23.y;
+        const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+        const float2 r01 = __half22float2(h01), r23 = __half22float2(h23);
+        const __half2 l01 = __floats2half2_rn(v.x - r01.x, v.y - r01.y);
+        const __half2 l23 = __floats2half2_rn(v.z - r23.x, v.w - r23.y);
+        uint2 ph, pl;
+        ph.x = *reinterpret_cast<const uint32_t*>(&h01); ph.y = *reinterpret_cast<const uint32_t*>(&h23);
+        pl.x = *reinterpret_cast<const uint32_t*>(&l01); pl.y = *reinterpret_cast<const uint32_t*>(&l23);
+        *reinterpret_cast<uint2*>(xs + m * ldxs + k) = ph;
+        *reinterpret_cast<uint2*>(xl + m * ldxs + k) = pl;
+      }
+    }
   } else {
     // every thread takes float4 columns tid*4 + 1024 i of every row
     if (IN == IN_NORM) {
