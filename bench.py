@@ -274,6 +274,7 @@ def run_trace(args):
     torch.cuda.synchronize()
     tl.tl_check_device_error(m)
     tl.tl_model_destroy(m)
+    tw, keep = tl.make_weights(w)   # for the second model below
     t = buf.cpu().numpy().reshape(-1, G).astype(np.float64)
     t0 = t[0].min()
     t = (t - t0) / 1e3   # us from the first CTA's start
@@ -319,6 +320,27 @@ def run_trace(args):
                        "tiles_max": round(float((hd_ - hs).max()), 2),
                        "total": round(float(end.max() - prev.max()), 2)},
            "layers": 2 + LOOPS, "barriers": n_bar}
+    # the per-op path's head (the persistent kernel in head-only mode), in a
+    # captured decode graph
+    m = tl.tl_model_create(cfg, tw, 0)
+    tl.tl_model_set_decode_path(m, DECODE_PATHS["layered"])
+    tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS)
+    hbuf = torch.zeros(4 * G, dtype=torch.int64, device="cuda:0")
+    tl.tl_model_set_trace(m, hbuf, hbuf.numel())
+    tok[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
+    heads = []
+    for i in range(8):
+        tl.tl_decode_step(m, [0], tok, [LOOPS], None, tok)
+        torch.cuda.synchronize()
+        h = hbuf.cpu().numpy().reshape(4, G).astype(np.float64) / 1e3
+        heads.append((float(h[1].max() - h[0].min()), float(np.median(h[2] - h[1])), float(h[2].max() - h[1].min()),
+                      float(h[3].max() - h[0].min())))
+    tl.tl_model_destroy(m)
+    hs = heads[2:]
+    out["layered_head_us"] = {"start_to_staged": round(statistics.mean(x[0] for x in hs), 2),
+                              "tiles_median": round(statistics.mean(x[1] for x in hs), 2),
+                              "tiles_span": round(statistics.mean(x[2] for x in hs), 2),
+                              "total": round(statistics.mean(x[3] for x in hs), 2)}
     print(json.dumps(out))
     return 0
 

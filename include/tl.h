@@ -248,7 +248,10 @@ tl_status tl_model_set_decode_path(tl_model *m, int path);
  * by CTAs without items), 5 + 5k items consumed (none of the three for
  * attention); after B barriers, slot 1 + 5B head activations staged,
  * 2 + 5B head tiles done, 3 + 5B end.  Entries past n_entries are skipped.
- * d_buf = NULL turns it off.  Steps overwrite the same entries. */
+ * d_buf = NULL turns it off.  Steps overwrite the same entries.  Head-only
+ * launches of the layered path (output norm + head + argmax) write slots 0
+ * (start), 1 (activations staged), 2 (head tiles done), 3 (end); a decode
+ * graph captured while a buffer is set keeps writing to that buffer. */
 tl_status tl_model_set_trace(tl_model *m, unsigned long long *d_buf, long long n_entries);
 int tl_model_trace_grid(const tl_model *m);
 

@@ -878,6 +878,8 @@ tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, fl
     f.io = io;
     f.logits = logits;
     f.argmax = argmax;
+    f.trace = m->trace;   // head-only timeline: start, staged, tiles done, end
+    f.trace_cap = m->trace_cap;
     size_t smem = 0;
     if (fused_plan(m, M, &f, &smem)) {
       kclass(TL_KERNEL_HEAD);
