@@ -36,6 +36,9 @@ __host__ __device__ inline int decode_split_len(int n_keys) {
   return c;
 }
 
+// Tokens per tile of the tcgen05 GEMM's prepared B operand (its kTcTokens).
+constexpr int kTcTokensB = 128;
+
 // Partial results of a split: REP x (hd unnormalised sums, max, sum of
 // weights, 2 pad) floats, so every head's block starts 16-byte aligned.
 constexpr int kPartPad = 4;
@@ -310,6 +313,11 @@ struct PrefillAttnArgs {
   long long o_bstride;
   int ldo;
   int rep;                // query heads per kv head (the kernel's REP heads are a slice of a group)
+  // model prefill: the output goes straight into the O projection's prepared
+  // B tiles ([token tiles][K/128][2 atoms][256 rows][128 B], fp16 hi rows
+  // then lo rows, 128-byte swizzled; K = Hq * hd) instead of `of`
+  uint8_t* bt;
+  int bt_groups;
 };
 
 // ---- prefill: tiled, tensor cores (m16n8k16), online softmax --------------
@@ -477,6 +485,27 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const Prefil
   // normalise and store rows q0+g, q0+g+8
   const float inv0 = 1.f / l0, inv1 = 1.f / l1;
   const int r0 = q0 + g, r1 = q0 + g + 8;
+  if (F32 && a.bt) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int k = h * HD + n * 8 + 2 * t;     // column of the O projection's input
+      const int grp = k >> 7, kg = k & 127;
+#pragma unroll
+      for (int half_ = 0; half_ < 2; ++half_) {
+        const int r = half_ ? r1 : r0;
+        if (r < a.T) {
+          const float inv = half_ ? inv1 : inv0;
+          uint32_t hw, lw;
+          split_h2(o[n][2 * half_] * inv, o[n][2 * half_ + 1] * inv, hw, lw);
+          const int tt = r / kTcTokensB, tl_ = r % kTcTokensB;
+          uint8_t* blk = a.bt + ((size_t)tt * a.bt_groups + grp) * (2 * kTcTokensB * 256);
+          *reinterpret_cast<uint32_t*>(blk + sw128_offset(tl_, kg, 2 * kTcTokensB)) = hw;
+          *reinterpret_cast<uint32_t*>(blk + sw128_offset(kTcTokensB + tl_, kg, 2 * kTcTokensB)) = lw;
+        }
+      }
+    }
+    return;
+  }
 #pragma unroll
   for (int n = 0; n < NT; ++n) {
     const int d = n * 8 + 2 * t;

@@ -157,6 +157,15 @@ __device__ __forceinline__ void unpack_a_frag(uint32_t w, uint32_t zz, uint32_t 
   a[3] = h2_sub(nib_pair_to_h2_biased(w >> 12), zhi);  // row g+8, k 2t+8..2t+9
 }
 
+// Byte offset of element pair (row, k..k+1), k even, in a 128-byte-swizzled
+// K-major tile of `rows` rows and 128 k (two 64-wide atoms): the operand
+// layout of the tcgen05 GEMM's B tiles and A stages.
+__host__ __device__ inline uint32_t sw128_offset(int row, int k, int rows) {
+  const int atom = k >> 6, kin = k & 63;
+  const int chunk = kin >> 3, within = (kin & 7) * 2;
+  return (uint32_t)(atom * rows * 128 + row * 128 + ((chunk ^ (row & 7)) << 4) + within);
+}
+
 // ---- reductions -----------------------------------------------------------
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

@@ -31,6 +31,7 @@
 //   skips the rest of its work and still frees its TMEM.
 #pragma once
 
+#include "attention.cuh"
 #include "common.cuh"
 
 namespace tl {
@@ -116,19 +117,14 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-// Byte offset of element pair (row, k..k+1), k even, in a 128-byte-swizzled
-// K-major tile of `rows` rows and 128 k (two 64-wide atoms).
-__host__ __device__ inline uint32_t sw128_offset(int row, int k, int rows) {
-  const int atom = k >> 6, kin = k & 63;
-  const int chunk = kin >> 3, within = (kin & 7) * 2;
-  return (uint32_t)(atom * rows * 128 + row * 128 + ((chunk ^ (row & 7)) << 4) + within);
-}
 
 enum TcEpi { TC_RESID = 0, TC_RAW = 1, TC_STORE = 2, TC_ROPE_KV = 3 };
 
 constexpr int kTcThreads = 512;       // 16 warps
 constexpr int kTcRows = 128;          // weight rows per tile (MMA M)
 constexpr int kTcTokens = 128;        // tokens per tile
+static_assert(kTcTokens == kTcTokensB, "the prefill attention writes B tiles of this many tokens");
+static_assert(kTcTokens == kTcTokensB, "the prefill attention writes B tiles of this many tokens");
 constexpr int kTcEpiThreads = 256;    // warps 8..15
 constexpr int kTcUnpack = 192;        // warps 2..7
 constexpr int kTcEpiWarp0 = 8;
@@ -572,7 +568,9 @@ __global__ void __launch_bounds__(256) tc_merge_kernel(const TcGemmArgs a) {
 // B tile of token tile tt and K group g: rows 0..127 = fp16 hi of the tokens,
 // rows 128..255 = fp16 lo (when LO), each row 128 k in two 64-wide atoms,
 // 128-byte swizzled; tokens >= T are zero.
-enum PrepMode { PREP_NORM = 0, PREP_F32 = 1, PREP_SWIGLU = 2, PREP_F16 = 3 };
+// PREP_NONE: the B tiles were written by the producing kernel (the prefill
+// attention writes the O projection's).
+enum PrepMode { PREP_NORM = 0, PREP_F32 = 1, PREP_SWIGLU = 2, PREP_F16 = 3, PREP_NONE = 4 };
 
 struct PrepArgs {
   const float* x;        // PREP_NORM / PREP_F32: fp32 [T][ldx]; PREP_SWIGLU: gate_up [T][ldx] (gate | up)

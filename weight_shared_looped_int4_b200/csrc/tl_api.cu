@@ -454,6 +454,7 @@ size_t tc_bt_bytes(int T, int K, bool lo) {
 }
 
 cudaError_t launch_prep(int mode, const PrepArgs& p, cudaStream_t st) {
+  if (mode == PREP_NONE) return cudaSuccess;
   const dim3 g(((p.T + kTcTokens - 1) / kTcTokens) * kTcTokens), b(256);
   switch (mode) {
     case PREP_NORM: return launch(prep_b_kernel<PREP_NORM>, g, b, 0, st, p);
@@ -837,12 +838,11 @@ tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
   const BlockDev& b = m->block(layer);
   const int d = c.d_model, F = c.ffn_dim, qdim = c.n_q_heads * c.head_dim;
   kclass(TL_KERNEL_GEMM_TC);
-  {  // O projection + residual
+  {  // O projection + residual (the prefill attention wrote its B tiles)
     PrepArgs pa{};
-    pa.x = m->o; pa.ldx = qdim;
     TcGemmArgs ta{};
     ta.out_f32 = m->x; ta.ld_out = d;
-    TL_CUDA(launch_tc_linear(b.o.tc, b.o.sz, qdim, d, b.o.n_tiles, PREP_F32, pa, ta, TC_RESID, T, m->tc, st));
+    TL_CUDA(launch_tc_linear(b.o.tc, b.o.sz, qdim, d, b.o.n_tiles, PREP_NONE, pa, ta, TC_RESID, T, m->tc, st));
   }
   {  // RMSNorm + gate_up (raw)
     PrepArgs pa{};
@@ -927,6 +927,10 @@ tl_status forward_prompt(tl_model* m, int lane, const int32_t* d_tokens, int T, 
     pa.kv_bstride = 0; pa.ctx = c.max_ctx;
     pa.T = T; pa.pos0 = 0; pa.Hkv = c.n_kv_heads;
     pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
+    if (tc) {   // straight into the O projection's B tiles
+      pa.bt = m->tc.bt;
+      pa.bt_groups = qdim / 128;
+    }
     kclass(TL_KERNEL_ATTN_PREFILL);
     TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
     rc = tc ? run_ffn_tc(m, layer, T, st) : run_ffn(m, layer, T, m->x, m->o, m->h, st);
