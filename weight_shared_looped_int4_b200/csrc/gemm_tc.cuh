@@ -118,7 +118,10 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 }
 
 
-enum TcEpi { TC_RESID = 0, TC_RAW = 1, TC_STORE = 2, TC_ROPE_KV = 3 };
+// TC_SWIGLU_B: the gate_up projection with its tensor-core rows interleaved
+// (tile t = gate rows 64t.. and up rows F + 64t..): silu(gate) * up is written
+// straight into the down projection's prepared B tiles.
+enum TcEpi { TC_RESID = 0, TC_RAW = 1, TC_STORE = 2, TC_ROPE_KV = 3, TC_SWIGLU_B = 4 };
 
 constexpr int kTcThreads = 512;       // 16 warps
 constexpr int kTcRows = 128;          // weight rows per tile (MMA M)
@@ -128,6 +131,33 @@ static_assert(kTcTokens == kTcTokensB, "the prefill attention writes B tiles of 
 constexpr int kTcEpiThreads = 256;    // warps 8..15
 constexpr int kTcUnpack = 192;        // warps 2..7
 constexpr int kTcEpiWarp0 = 8;
+
+// Original row of tensor-core row p when the layout interleaves gate / up
+// (perm_F = F; 0 = no interleave).
+__host__ __device__ inline int tc_row_orig(int p, int perm_F) {
+  if (!perm_F) return p;
+  const int rt = p / kTcRows, r = p % kTcRows;
+  return r < kTcRows / 2 ? rt * (kTcRows / 2) + r : perm_F + rt * (kTcRows / 2) + r - kTcRows / 2;
+}
+
+// silu(gate) * up of token `tl_` (within token tile tt) and interleaved pair
+// column j of row tile `tile`, pairs (j, j+1), as hi/lo fp16 into the down
+// projection's B tile (K index 64 tile + j).
+__device__ __forceinline__ void tc_swiglu_store(uint8_t* bt, int groups, int tt, int tile, int tl_, int j, float g0,
+                                                float g1, float u0, float u1) {
+  const float h0 = silu(g0) * u0, h1 = silu(g1) * u1;
+  uint32_t hw, lw;
+  const __half2 hh = __floats2half2_rn(h0, h1);
+  const float2 rr = __half22float2(hh);
+  const __half2 ll = __floats2half2_rn(h0 - rr.x, h1 - rr.y);
+  hw = *reinterpret_cast<const uint32_t*>(&hh);
+  lw = *reinterpret_cast<const uint32_t*>(&ll);
+  const int k = tile * 64 + j, grp = k >> 7, kg = k & 127;
+  uint8_t* blk = bt + ((size_t)tt * groups + grp) * (2 * 128 * 256);
+  *reinterpret_cast<uint32_t*>(blk + sw128_offset(tl_, kg, 256)) = hw;
+  *reinterpret_cast<uint32_t*>(blk + sw128_offset(128 + tl_, kg, 256)) = lw;
+}
+
 
 constexpr int kTcStages = 4;          // half-group (64 k) operand stages
 constexpr int kTcRaw = 3;             // raw INT4 group stages
@@ -167,6 +197,10 @@ struct TcGemmArgs {
   float theta;
   const float2* rope_tab;  // (cos, sin) [positions][hd/2], or NULL
   // split-K
+  // TC_SWIGLU_B
+  int perm_F;            // interleaved gate/up rows (the scales are looked up by original row)
+  uint8_t* bt_out;       // the down projection's B tiles
+  int bt_out_groups;     // its K / 128
   float* partial;        // [splits][row tiles][token tiles][128 tokens][128 rows]
   unsigned* tickets;     // [row tiles][token tiles], zero between launches
   int* err_flag;
@@ -332,16 +366,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     const int quad = warp & 3;                 // TMEM lanes this warp may access
     const int half = e >> 2;                   // tokens [64 half, 64 half + 64)
     const int row = quad * 32 + lane;          // weight row within the tile
-    const int gt = tile * 8 + (row >> 4);
+    const int orow = tc_row_orig(tile * kTcRows + row, a.perm_F);   // row in the GEMV layout
+    const int gt = orow >> 4;
     const bool row_ok = gt < a.n16_tiles;
     float acc[64];
 #pragma unroll
     for (int i = 0; i < 64; ++i) acc[i] = 0.f;
     auto scale_of = [&](int g) -> float {
       if (!row_ok) return 0.f;
-      const uint32_t sp = __ldg(&a.sz[((size_t)gt * G + g) * 8 + (row & 7)]).x;
+      const uint32_t sp = __ldg(&a.sz[((size_t)gt * G + g) * 8 + (orow & 7)]).x;
       const float2 f = h2_to_f2(sp);
-      return (row & 8) ? f.y : f.x;
+      return (orow & 8) ? f.y : f.x;
     };
     float s_next = ng > 0 ? scale_of(gmap(0)) : 0.f;
     for (int it = 0; it < ng; ++it) {
@@ -404,6 +439,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
             }
           }
         }
+      } else if (EPI == TC_SWIGLU_B) {
+        // gate rows 0..63 and up rows 64..127 of the tile: exchange through
+        // shared memory, then write pairs of SwiGLU outputs
+        float* xch = reinterpret_cast<float*>(smem);   // [128 tokens][128 rows]
+#pragma unroll
+        for (int i = 0; i < 64; ++i) xch[(half * 64 + i) * kTcRows + row] = acc[i];
+        epi_sync(kTcEpiThreads);
+        for (int item = threadIdx.x - kTcEpiWarp0 * 32; item < kTcTokens * 32; item += kTcEpiThreads) {
+          const int tl_ = item >> 5, j = (item & 31) * 2;
+          if (tt * kTcTokens + tl_ >= a.T) continue;
+          const float* xr = xch + tl_ * kTcRows;
+          tc_swiglu_store(a.bt_out, a.bt_out_groups, tt, tile, tl_, j, xr[j], xr[j + 1], xr[64 + j], xr[65 + j]);
+        }
       } else {
         // RoPE pairs (j, j + hd/2) sit in different rows of the tile: exchange
         // through shared memory (the stages are idle now).
@@ -457,9 +505,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
 // ---- load-time re-layout for the tensor-core path -------------------------------
 // One thread per 8-nibble word (and, for j == 0, the row's biased zero) of
 // the tensor-core layout, from the storage format (qweight [N][K/8] words,
-// element k in bits 4 (k % 8); qzeros [N][ceil(G/8)] words).
+// element k in bits 4 (k % 8); qzeros [N][ceil(G/8)] words).  perm_F != 0
+// interleaves gate and up rows per 128-row tile (see tc_row_orig).
 __global__ void repack_int4_tc_kernel(const uint32_t* __restrict__ qweight, const uint32_t* __restrict__ qzeros,
-                                      int K, int N, uint8_t* __restrict__ out) {
+                                      int K, int N, int perm_F, uint8_t* __restrict__ out) {
   const int G = K >> 7, zw = (G + 7) >> 3;
   const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int row_tiles = (N + kTcRows - 1) / kTcRows;
@@ -469,7 +518,7 @@ __global__ void repack_int4_tc_kernel(const uint32_t* __restrict__ qweight, cons
   const int r = (int)((idx >> 4) % kTcRows);
   const size_t blk = (idx >> 4) / kTcRows;          // rt * G + g
   const int g = (int)(blk % G), rt = (int)(blk / G);
-  const int n = rt * kTcRows + r;
+  const int n = tc_row_orig(rt * kTcRows + r, perm_F);
   uint8_t* base = out + blk * kTcRawBytes;
   uint32_t word = 0, z = 0;
   if (n < N) {
@@ -515,6 +564,18 @@ __global__ void __launch_bounds__(256) tc_merge_kernel(const TcGemmArgs a) {
     }
   }
   const int t = tt * kTcTokens + tok;
+  if (EPI == TC_SWIGLU_B) {
+    *reinterpret_cast<float4*>(&xch[tl_][r4]) = sum;
+    __syncthreads();
+    for (int item = threadIdx.x; item < kTcMergeTok * 32; item += 256) {
+      const int ti = item >> 5, j = (item & 31) * 2;
+      const int tq = slice * kTcMergeTok + ti;      // token within the tile
+      if (tt * kTcTokens + tq >= a.T) continue;
+      tc_swiglu_store(a.bt_out, a.bt_out_groups, tt, tile, tq, j, xch[ti][j], xch[ti][j + 1], xch[ti][64 + j],
+                      xch[ti][65 + j]);
+    }
+    return;
+  }
   if (EPI == TC_RESID || EPI == TC_RAW || EPI == TC_STORE) {
     const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
     if (t < a.T) {

@@ -216,6 +216,7 @@ cudaError_t init_device_kernels(int dev) {
   if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_RAW, true>, dev);
   if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_ROPE_KV, true>, dev);
   if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_STORE, false>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_SWIGLU_B, true>, dev);
 #define ATT(HD, REP)                                                                  \
   if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, true>, dev);   \
   if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, false>, dev);  \
@@ -308,7 +309,10 @@ struct Arena {
 
 // Copy one linear in the storage format to the device and re-lay it out.
 // N is padded to whole pairs of 16-row tiles with zero weights.
-tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaStream_t st, Arena* arena = nullptr) {
+// perm_F != 0: the tensor-core copy interleaves gate rows [0, F) and up rows
+// [F, 2F) per 128-row tile (for the fused SwiGLU epilogue).
+tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaStream_t st, Arena* arena = nullptr,
+                      int perm_F = 0) {
   if (!h.qweight || !h.scales || !h.qzeros) return fail(TL_ERR_INVALID_ARG, "null INT4 array");
   const int G = K / 128, zw = (G + 7) / 8;
   out->K = K;
@@ -342,7 +346,7 @@ tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaS
         (const uint16_t*)ds, (const uint32_t*)dz, K, N, out->n_tiles, out->sz);
     const size_t tt = (size_t)((N + kTcRows - 1) / kTcRows) * G * kTcRows * 16;
     repack_int4_tc_kernel<<<(unsigned)((tt + 255) / 256), 256, 0, st>>>((const uint32_t*)dq, (const uint32_t*)dz, K,
-                                                                       N, out->tc);
+                                                                       N, perm_F, out->tc);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
@@ -439,6 +443,7 @@ __global__ void fill_rows_kernel(RowCtx* rows, int n, int lane, int pos0) {
 // ---- tensor-core INT4 GEMM (prefill / large M) ------------------------------
 struct TcScratch {
   uint8_t* bt = nullptr;       // prepared activation tiles
+  uint8_t* bt2 = nullptr;      // the down projection's tiles, written by the gate_up epilogue
   size_t bt_bytes = 0;
   float* partial = nullptr;    // split-K partial tiles
   size_t partial_bytes = 0;
@@ -467,8 +472,11 @@ cudaError_t launch_prep(int mode, const PrepArgs& p, cudaStream_t st) {
 
 // Runs prep + GEMM for T tokens.  `ta` carries the epilogue outputs; the
 // weight, activation and scratch fields are filled here.
+// `b_tiles`: where the GEMM reads its prepared B tiles (default: the scratch
+// the prep kernel writes).
 cudaError_t launch_tc_linear(const uint8_t* wtc, const uint2* sz, int K, int N, int n16_tiles, int prep_mode,
-                             PrepArgs pa, TcGemmArgs ta, int epi, int T, const TcScratch& sc, cudaStream_t st) {
+                             PrepArgs pa, TcGemmArgs ta, int epi, int T, const TcScratch& sc, cudaStream_t st,
+                             const uint8_t* b_tiles = nullptr) {
   const bool lo = prep_mode != PREP_F16;
   if (tc_bt_bytes(T, K, lo) > sc.bt_bytes) return cudaErrorInvalidValue;
   pa.K = K;
@@ -482,7 +490,7 @@ cudaError_t launch_tc_linear(const uint8_t* wtc, const uint2* sz, int K, int N, 
   while (splits > 1 && (size_t)splits * row_tiles * tok_tiles * kTcRows * kTcTokens * 4 > sc.partial_bytes) --splits;
   if (row_tiles * tok_tiles > 4096) return cudaErrorInvalidValue;
   ta.wtc = wtc; ta.sz = sz; ta.K = K; ta.N = N; ta.n16_tiles = n16_tiles;
-  ta.bt = sc.bt; ta.T = T; ta.splits = splits;
+  ta.bt = b_tiles ? b_tiles : sc.bt; ta.T = T; ta.splits = splits;
   ta.partial = sc.partial; ta.tickets = sc.tickets; ta.err_flag = sc.err_flag;
   const dim3 g(row_tiles, tok_tiles, splits), b(kTcThreads);
   const size_t smem = tc_smem_bytes(lo);
@@ -490,12 +498,14 @@ cudaError_t launch_tc_linear(const uint8_t* wtc, const uint2* sz, int K, int N, 
   else if (epi == TC_RAW && lo) e = launch(gemm_int4_tc_kernel<TC_RAW, true>, g, b, smem, st, ta);
   else if (epi == TC_ROPE_KV && lo) e = launch(gemm_int4_tc_kernel<TC_ROPE_KV, true>, g, b, smem, st, ta);
   else if (epi == TC_STORE && !lo) e = launch(gemm_int4_tc_kernel<TC_STORE, false>, g, b, smem, st, ta);
+  else if (epi == TC_SWIGLU_B && lo) e = launch(gemm_int4_tc_kernel<TC_SWIGLU_B, true>, g, b, smem, st, ta);
   else return cudaErrorInvalidValue;
   if (e != cudaSuccess || splits == 1) return e;
   const dim3 mg(row_tiles, tok_tiles, kTcTokens / kTcMergeTok);
   if (epi == TC_RESID) return launch(tc_merge_kernel<TC_RESID>, mg, dim3(256), 0, st, ta);
   if (epi == TC_RAW) return launch(tc_merge_kernel<TC_RAW>, mg, dim3(256), 0, st, ta);
   if (epi == TC_ROPE_KV) return launch(tc_merge_kernel<TC_ROPE_KV>, mg, dim3(256), 0, st, ta);
+  if (epi == TC_SWIGLU_B) return launch(tc_merge_kernel<TC_SWIGLU_B>, mg, dim3(256), 0, st, ta);
   return launch(tc_merge_kernel<TC_STORE>, mg, dim3(256), 0, st, ta);
 }
 
@@ -610,7 +620,7 @@ struct tl_model {
     graphs.clear();
     if (cap_stream) cudaStreamDestroy(cap_stream);
     void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row,
-                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.partial, tc.tickets, gu,
+                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.bt2, tc.partial, tc.tickets, gu,
                     rope_tab, fused_bar, fused_val, fused_idx};
     for (void* p : ptrs)
       if (p) cudaFree(p);
@@ -680,7 +690,7 @@ tl_status upload_block(const tl_config& c, const tl_block& hb, BlockDev* b, cuda
   b->arena.size = total;
   if ((rc = upload_int4(hb.qkv, d, qkv_rows, &b->qkv, st, &b->arena)) != TL_OK) return rc;
   if ((rc = upload_int4(hb.o, qdim, d, &b->o, st, &b->arena)) != TL_OK) return rc;
-  if ((rc = upload_int4(hb.gate_up, d, 2 * c.ffn_dim, &b->gate_up, st, &b->arena)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.gate_up, d, 2 * c.ffn_dim, &b->gate_up, st, &b->arena, c.ffn_dim)) != TL_OK) return rc;
   if ((rc = upload_int4(hb.down, c.ffn_dim, d, &b->down, st, &b->arena)) != TL_OK) return rc;
   return TL_OK;
 }
@@ -844,21 +854,21 @@ tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
     ta.out_f32 = m->x; ta.ld_out = d;
     TL_CUDA(launch_tc_linear(b.o.tc, b.o.sz, qdim, d, b.o.n_tiles, PREP_NONE, pa, ta, TC_RESID, T, m->tc, st));
   }
-  {  // RMSNorm + gate_up (raw)
+  {  // RMSNorm + gate_up; its epilogue writes silu(gate) * up as the down
+     // projection's B tiles (the tensor-core rows interleave gate and up)
     PrepArgs pa{};
     pa.x = m->x; pa.ldx = d; pa.gain = b.ffn_norm; pa.eps = c.rms_eps;
     TcGemmArgs ta{};
-    ta.out_f32 = m->gu; ta.ld_out = 2 * F;
-    TL_CUDA(launch_tc_linear(b.gate_up.tc, b.gate_up.sz, d, 2 * F, b.gate_up.n_tiles, PREP_NORM, pa, ta, TC_RAW, T,
-                             m->tc, st));
+    ta.perm_F = F; ta.bt_out = m->tc.bt2; ta.bt_out_groups = F / 128;
+    TL_CUDA(launch_tc_linear(b.gate_up.tc, b.gate_up.sz, d, 2 * F, b.gate_up.n_tiles, PREP_NORM, pa, ta,
+                             TC_SWIGLU_B, T, m->tc, st));
   }
-  {  // SwiGLU + down + residual
+  {  // down + residual
     PrepArgs pa{};
-    pa.x = m->gu; pa.ldx = 2 * F; pa.F = F;
     TcGemmArgs ta{};
     ta.out_f32 = m->x; ta.ld_out = d;
-    TL_CUDA(launch_tc_linear(b.down.tc, b.down.sz, F, d, b.down.n_tiles, PREP_SWIGLU, pa, ta, TC_RESID, T, m->tc,
-                             st));
+    TL_CUDA(launch_tc_linear(b.down.tc, b.down.sz, F, d, b.down.n_tiles, PREP_NONE, pa, ta, TC_RESID, T, m->tc, st,
+                             m->tc.bt2));
   }
   return TL_OK;
 }
@@ -1056,7 +1066,8 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     m->tc.bt_bytes = tc_bt_bytes(rows, kmax, true);
     m->tc.partial_bytes = (size_t)160 * kTcRows * kTcTokens * 4;
     m->tc.err_flag = m->err_flag;
-    ok = alloc((void**)&m->tc.bt, m->tc.bt_bytes) && alloc((void**)&m->tc.partial, m->tc.partial_bytes) &&
+    ok = alloc((void**)&m->tc.bt, m->tc.bt_bytes) && alloc((void**)&m->tc.bt2, m->tc.bt_bytes) &&
+         alloc((void**)&m->tc.partial, m->tc.partial_bytes) &&
          alloc((void**)&m->tc.tickets, 4096 * sizeof(unsigned)) &&
          alloc((void**)&m->gu, (size_t)tok_pad * 2 * c.ffn_dim * 4) &&
          alloc((void**)&m->rope_tab, (size_t)c.max_ctx * (hd / 2) * sizeof(float2));
