@@ -630,17 +630,17 @@ __global__ void __launch_bounds__(256) tc_merge_kernel(const TcGemmArgs a) {
 // rows 128..255 = fp16 lo (when LO), each row 128 k in two 64-wide atoms,
 // 128-byte swizzled; tokens >= T are zero.
 // PREP_NONE: the B tiles were written by the producing kernel (the prefill
-// attention writes the O projection's).
-enum PrepMode { PREP_NORM = 0, PREP_F32 = 1, PREP_SWIGLU = 2, PREP_F16 = 3, PREP_NONE = 4 };
+// attention writes the O projection's, the gate_up epilogue the down
+// projection's).
+enum PrepMode { PREP_NORM = 0, PREP_F16 = 3, PREP_NONE = 4 };
 
 struct PrepArgs {
-  const float* x;        // PREP_NORM / PREP_F32: fp32 [T][ldx]; PREP_SWIGLU: gate_up [T][ldx] (gate | up)
+  const float* x;        // PREP_NORM: fp32 [T][ldx]
   const __half* xh;      // PREP_F16: fp16 [T][ldx]
   int ldx;
   const __half* gain;    // PREP_NORM
   float eps;
   int K, T;
-  int F;                 // PREP_SWIGLU: up columns start at F
   uint8_t* bt;
 };
 
@@ -686,13 +686,6 @@ __global__ void __launch_bounds__(256) prep_b_kernel(const PrepArgs a) {
         v[2 * i] = f.x;
         v[2 * i + 1] = f.y;
       }
-    } else if (MODE == PREP_SWIGLU) {
-      const float* src = a.x + (size_t)tok * a.ldx;
-      const float4 g0 = *reinterpret_cast<const float4*>(src + k), g1 = *reinterpret_cast<const float4*>(src + k + 4);
-      const float4 u0 = *reinterpret_cast<const float4*>(src + a.F + k);
-      const float4 u1 = *reinterpret_cast<const float4*>(src + a.F + k + 4);
-      v[0] = silu(g0.x) * u0.x; v[1] = silu(g0.y) * u0.y; v[2] = silu(g0.z) * u0.z; v[3] = silu(g0.w) * u0.w;
-      v[4] = silu(g1.x) * u1.x; v[5] = silu(g1.y) * u1.y; v[6] = silu(g1.z) * u1.z; v[7] = silu(g1.w) * u1.w;
     } else {
       const float* src = a.x + (size_t)tok * a.ldx;
       const float4 x0 = *reinterpret_cast<const float4*>(src + k), x1 = *reinterpret_cast<const float4*>(src + k + 4);

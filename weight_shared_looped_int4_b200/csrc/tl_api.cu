@@ -463,8 +463,6 @@ cudaError_t launch_prep(int mode, const PrepArgs& p, cudaStream_t st) {
   const dim3 g(((p.T + kTcTokens - 1) / kTcTokens) * kTcTokens), b(256);
   switch (mode) {
     case PREP_NORM: return launch(prep_b_kernel<PREP_NORM>, g, b, 0, st, p);
-    case PREP_F32: return launch(prep_b_kernel<PREP_F32>, g, b, 0, st, p);
-    case PREP_SWIGLU: return launch(prep_b_kernel<PREP_SWIGLU>, g, b, 0, st, p);
     case PREP_F16: return launch(prep_b_kernel<PREP_F16>, g, b, 0, st, p);
   }
   return cudaErrorInvalidValue;
@@ -579,7 +577,6 @@ struct tl_model {
   TcScratch tc;                  // tensor-core GEMM scratch (prefill)
   cudaAccessPolicyWindow loop_window = {};  // keeps the loop block's weights in L2
   size_t l2_persist_bytes = 0;
-  float* gu = nullptr;           // raw gate_up output of the prefill [rows][2F]
   float2* rope_tab = nullptr;    // RoPE (cos, sin) [max_ctx][hd/2]
   cudaStream_t setup_stream = nullptr;
   cudaStream_t cap_stream = nullptr;   // stream used to capture decode graphs
@@ -620,7 +617,7 @@ struct tl_model {
     graphs.clear();
     if (cap_stream) cudaStreamDestroy(cap_stream);
     void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row,
-                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.bt2, tc.partial, tc.tickets, gu,
+                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.bt2, tc.partial, tc.tickets,
                     rope_tab, fused_bar, fused_val, fused_idx};
     for (void* p : ptrs)
       if (p) cudaFree(p);
@@ -1062,14 +1059,12 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
             alloc((void**)&m->io, sizeof(HeadIO));
   if (ok) {
     const int kmax = std::max(std::max(d, qdim), c.ffn_dim);
-    const int tok_pad = ((rows + kTcTokens - 1) / kTcTokens) * kTcTokens;
     m->tc.bt_bytes = tc_bt_bytes(rows, kmax, true);
     m->tc.partial_bytes = (size_t)160 * kTcRows * kTcTokens * 4;
     m->tc.err_flag = m->err_flag;
     ok = alloc((void**)&m->tc.bt, m->tc.bt_bytes) && alloc((void**)&m->tc.bt2, m->tc.bt_bytes) &&
          alloc((void**)&m->tc.partial, m->tc.partial_bytes) &&
          alloc((void**)&m->tc.tickets, 4096 * sizeof(unsigned)) &&
-         alloc((void**)&m->gu, (size_t)tok_pad * 2 * c.ffn_dim * 4) &&
          alloc((void**)&m->rope_tab, (size_t)c.max_ctx * (hd / 2) * sizeof(float2));
     if (ok) {
       const int n = c.max_ctx * (hd / 2);
