@@ -479,11 +479,17 @@ def run_ours(args):
             prof = tl.tl_model_profile_stop(m)
         step_bytes = hbm_bytes + l2_bytes
 
+        # with the clustered QKV + attention kernel (no separate attention
+        # launches) the "qkv" class also reads the KV cache
+        attn_in_qkv = "attn_decode" not in prof
+
         def bytes_of(name):
             if name == "attn_decode":
                 return _attn_bytes_per_launch(mean_keys)
             if name == "decode_fused":
                 return step_bytes
+            if name == "qkv" and attn_in_qkv:
+                return BYTES_PER_LAUNCH["qkv"] + _attn_bytes_per_launch(mean_keys)
             return BYTES_PER_LAUNCH.get(name)
 
         for name, (n, ms) in prof.items():

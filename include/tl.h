@@ -183,7 +183,7 @@ tl_status tl_check_device_error(tl_model *m, void *stream);
 /* Kernel families, for the per-kernel profiler. */
 typedef enum {
   TL_KERNEL_EMBED = 0,        /* embedding gather */
-  TL_KERNEL_QKV = 1,          /* RMSNorm + QKV INT4 linear + RoPE + KV write */
+  TL_KERNEL_QKV = 1,          /* RMSNorm + QKV INT4 linear + RoPE + KV write (+ attention: clustered kernel) */
   TL_KERNEL_ATTN_DECODE = 2,  /* single-query cached-decode attention */
   TL_KERNEL_O_PROJ = 3,       /* O INT4 linear + residual */
   TL_KERNEL_GATE_UP = 4,      /* RMSNorm + gate_up INT4 linear + SwiGLU */
