@@ -325,22 +325,69 @@ def run_trace(args):
     m = tl.tl_model_create(cfg, tw, 0)
     tl.tl_model_set_decode_path(m, DECODE_PATHS["layered"])
     tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS)
-    hbuf = torch.zeros(4 * G, dtype=torch.int64, device="cuda:0")
+    n_rec = 4 * (2 + LOOPS)   # layer launches: QKV + attention, O, gate_up, down
+    hbuf = torch.zeros(4 * G + 6 * n_rec, dtype=torch.int64, device="cuda:0")
     tl.tl_model_set_trace(m, hbuf, hbuf.numel())
     tok[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
-    heads = []
+    heads, recs = [], []
     for i in range(8):
+        hbuf.zero_()   # the layer records take the max over CTAs
         tl.tl_decode_step(m, [0], tok, [LOOPS], None, tok)
         torch.cuda.synchronize()
-        h = hbuf.cpu().numpy().reshape(4, G).astype(np.float64) / 1e3
+        raw = hbuf.cpu().numpy()
+        h = raw[:4 * G].reshape(4, G).astype(np.float64) / 1e3
         heads.append((float(h[1].max() - h[0].min()), float(np.median(h[2] - h[1])), float(h[2].max() - h[1].min()),
                       float(h[3].max() - h[0].min())))
+        last_h = h
+        r = raw[4 * G:].reshape(n_rec, 6).view(np.uint64).copy()
+        r[:, 0] = ~r[:, 0]   # the first start is stored complemented
+        recs.append((r.astype(np.float64) / 1e3, float(h[0].min()), float(h[3].max())))
     tl.tl_model_destroy(m)
     hs = heads[2:]
     out["layered_head_us"] = {"start_to_staged": round(statistics.mean(x[0] for x in hs), 2),
                               "tiles_median": round(statistics.mean(x[1] for x in hs), 2),
                               "tiles_span": round(statistics.mean(x[2] for x in hs), 2),
                               "total": round(statistics.mean(x[3] for x in hs), 2)}
+    # per layer kernel, in the captured graph: its share of the step's critical
+    # path (previous launch's last CTA end -> its own last CTA end), how long
+    # its CTAs waited for the previous kernel's end, and its phases after that
+    names = ("qkv_attn", "o_proj", "gate_up", "down")
+    acc = {n: {"critical_path": [], "started_before_prev_end": [], "release_after_prev_end": [],
+               "phase1": [], "phase2": [], "phase3": []} for n in names}
+    step_us, head_tail = [], []
+    for r, h_start, h_end in recs[2:]:
+        step_us.append(h_end - r[0, 0])
+        head_tail.append(h_end - r[-1, 5])
+        for i in range(1, n_rec):
+            a = acc[names[i % 4]]
+            prev_end = r[i - 1, 5]
+            a["critical_path"].append(r[i, 5] - prev_end)
+            a["started_before_prev_end"].append(prev_end - r[i, 1])
+            a["release_after_prev_end"].append(r[i, 2] - prev_end)
+            rel = r[i, 2]
+            if i % 4 == 0:   # clustered: GEMV + exchange, attention + exchange, merge
+                a["phase1"].append(r[i, 3] - rel)
+                a["phase2"].append(r[i, 4] - r[i, 3])
+            else:            # GEMV: weights-ready wait after release, main loop, epilogue
+                a["phase1"].append(max(r[i, 3] - rel, 0.0))
+                a["phase2"].append(r[i, 4] - max(r[i, 3], rel))
+            a["phase3"].append(r[i, 5] - r[i, 4])
+    r, h_start, h_end = recs[-1]
+    out["layered_last_step_per_launch"] = [
+        [round(float(v), 2) for v in (r[i, 5] - (r[i - 1, 5] if i else r[i, 0]), r[i, 2] - r[i, 1],
+                                      r[i, 3] - r[i, 2], r[i, 4] - r[i, 3], r[i, 5] - r[i, 4])]
+        for i in range(n_rec)]
+    out["layered_step_us"] = round(statistics.mean(step_us), 2)
+    out["layered_head_after_last_down_us"] = round(statistics.mean(head_tail), 2)
+    d_end = r[-1, 5]
+    out["layered_head_last_step_vs_down_end_us"] = {
+        "first_start": round(float(last_h[0].min() - d_end), 2), "median_start": round(float(np.median(last_h[0]) - d_end), 2),
+        "last_start": round(float(last_h[0].max() - d_end), 2), "median_staged": round(float(np.median(last_h[1]) - d_end), 2),
+        "last_staged": round(float(last_h[1].max() - d_end), 2), "last_end": round(float(last_h[3].max() - d_end), 2)}
+    out["layered_kernels_us"] = {n: {k: round(statistics.mean(v), 2) for k, v in a.items()} for n, a in acc.items()}
+    out["layered_phases"] = {"qkv_attn": "phase1 RMSNorm+QKV GEMV+RoPE+exchange, phase2 attention+exchange, "
+                                         "phase3 merge",
+                             "gemv": "phase1 wait for weights after release, phase2 main loop, phase3 epilogue"}
     print(json.dumps(out))
     return 0
 

@@ -47,6 +47,28 @@ __device__ __forceinline__ uint2 ldg_stream2(const uint2* p) {
   return r;
 }
 
+// ---- launch timeline ---------------------------------------------------------
+__device__ __forceinline__ long long globaltimer_ns() {
+  long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Per-launch timeline of a layer kernel: `tr` holds kTraceEvents entries of
+// one launch (zeroed by the caller), or is NULL.  Thread 0 of every CTA
+// stamps event e >= 1 as the latest %globaltimer over the CTAs; event 0 holds
+// the earliest start, complemented (so that both use atomicMax).
+constexpr int kTraceEvents = 6;   // first start, last start, released, mid 1, mid 2, end
+__device__ __forceinline__ void trace_start(unsigned long long* tr) {
+  if (tr && threadIdx.x == 0) {
+    const unsigned long long t = (unsigned long long)globaltimer_ns();
+    atomicMax(tr, ~t);
+    atomicMax(tr + 1, t);
+  }
+}
+__device__ __forceinline__ void trace_mark(unsigned long long* tr, int e) {
+  if (tr && threadIdx.x == 0) atomicMax(tr + e, (unsigned long long)globaltimer_ns());
+}
+
 // ---- bulk asynchronous copies (TMA engine) with mbarrier completion --------
 __device__ __forceinline__ unsigned smem_u32(const void* p) {
   return (unsigned)__cvta_generic_to_shared(p);

@@ -174,11 +174,6 @@ __device__ __forceinline__ void fused_split(int n, int P, int Hkv, int& C, int& 
 
 // ---- primitives -------------------------------------------------------------
 __device__ __forceinline__ void fused_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kFusedCompute) : "memory"); }
-__device__ __forceinline__ long long globaltimer_ns() {
-  long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -75,6 +75,8 @@ struct GemvArgs {
   float theta;
   const float2* rope_tab;  // (cos, sin) [positions][hd/2], or NULL
   int* err_flag;       // device fault flags (a bounded wait gave up)
+  unsigned long long* trace;  // launch timeline (kTraceEvents entries) or NULL:
+                              // released, weights arrived, main loop done
 };
 
 constexpr int kGemvThreads = 256;
@@ -146,6 +148,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
     t1 = t0 + a.pair_off;
   }
 
+  trace_start(a.trace);
   pdl_trigger();
   // The weights do not depend on earlier kernels: start their bulk copies
   // before waiting for the previous kernel.
@@ -166,6 +169,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   }
 
   pdl_wait();
+  trace_mark(a.trace, 2);
 
   // ---- stage the activations: fp16 pair (hi, lo) of the fp32 input --------
   if (IN == IN_F16) {
@@ -275,6 +279,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   if (threadIdx.x == 0) {
     s_ok = mbar_wait(&wbar, 0) ? 1 : 0;
     if (!s_ok) atomicOr(a.err_flag, kErrTimeout);
+    trace_mark(a.trace, 3);
   }
   __syncthreads();
   if (!s_ok) return;  // uniform: every thread read the same flag after the barrier
@@ -349,6 +354,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
     }
   }
 
+  trace_mark(a.trace, 4);
   // ---- reduce the K slices (fixed order) ---------------------------------
   float* myred = red + (kq * TPC + tsel) * 16 * NC;
   if (NT == 0 && LO) {  // columns (2m, 2m+1) = (hi, lo) parts of row m = t
@@ -404,6 +410,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
       dst[j + hd / 2] = __float2half_rn(vb);
     }
   }
+  trace_mark(a.trace, 5);
 }
 
 // ---- load-time re-layout ----------------------------------------------------

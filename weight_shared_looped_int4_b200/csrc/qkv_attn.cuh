@@ -52,6 +52,8 @@ struct QkvAttnArgs {
   int ctx;
   float* o;              // attention output [M][Hq*hd] fp32
   int* err_flag;
+  unsigned long long* trace;  // launch timeline (kTraceEvents entries) or NULL:
+                              // released, q/k/v exchanged, partials exchanged
 };
 
 __host__ __device__ inline int qa_units(int rep, int hd) { return (rep + 2) * hd / 32; }
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     return row_base / 16 + j + (second ? hp : 0);
   };
 
+  trace_start(a.trace);
   pdl_trigger();
   if (tid == 0) {
     mbar_init(&wbar, 1);
@@ -156,6 +159,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   // shared-memory write reaches it (the first ones come after the GEMV)
   qa_cluster_sync();
   pdl_wait();
+  trace_mark(a.trace, 2);
 
   // ---- RMSNorm of the rows into the (hi, lo) planes: every thread loads its
   // columns of every row (and the gains) at once and keeps them in registers
@@ -302,6 +306,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     }
   }
   qa_cluster_sync();   // #1: q and the new key / value are in every rank
+  trace_mark(a.trace, 3);
 
   // ---- attention over this rank's key split, per row -------------------------
   const float scale = 1.0f / sqrtf((float)HD);
@@ -415,6 +420,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     __syncthreads();
   }
   qa_cluster_sync();   // #2: every rank's partials are in rank 0
+  trace_mark(a.trace, 4);
 
   // ---- rank 0 merges the ranks in order --------------------------------------
   if (c == 0) {
@@ -438,6 +444,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       if (ok) a.o[(size_t)m * (a.Hkv * rep * HD) + (size_t)(grp * rep + h) * HD + dim] = num / den;
     }
   }
+  trace_mark(a.trace, 5);
 }
 
 }  // namespace tl

@@ -599,6 +599,7 @@ struct tl_model {
   int* fused_idx = nullptr;
   unsigned long long* trace = nullptr;  // caller's phase-timeline buffer (device), or NULL
   long long trace_cap = 0;
+  long long trace_i = -1;         // next layer-launch record of a layered decode step (-1: none)
   std::vector<int> lane_len, lane_loops;
   size_t weight_bytes = 0, kv_bytes = 0, ws_bytes = 0;
   Profiler prof;
@@ -701,6 +702,14 @@ struct WindowScope {
   ~WindowScope() { g_window = prev; }
 };
 
+// Timeline entries of the next layer launch of a traced layered decode step
+// (kTraceEvents per launch after the head-only launch's 4 slots), or NULL.
+unsigned long long* next_trace(tl_model* m) {
+  if (!m->trace || m->trace_i < 0) return nullptr;
+  const long long base = 4LL * m->fused_grid + (long long)kTraceEvents * m->trace_i++;
+  return base + kTraceEvents <= m->trace_cap ? m->trace + base : nullptr;
+}
+
 // ---- one effective layer ------------------------------------------------------
 // QKV projection of `M` rows of the residual stream x (RMSNorm fused), RoPE on
 // q and k, k and v written to cache slice `layer` at each row's (lane, pos).
@@ -722,6 +731,7 @@ tl_status run_qkv(tl_model* m, int layer, int M, float* x, const RowCtx* rows, f
   a.lane_stride = m->lane_stride; a.ctx = c.max_ctx;
   a.rope_tab = m->rope_tab;
   a.err_flag = m->err_flag;
+  a.trace = next_trace(m);
   kclass(TL_KERNEL_QKV);
   TL_CUDA(launch_gemv_rows(a, M, IN_NORM, EPI_ROPE_KV, (c.n_q_heads + 2 * c.n_kv_heads) * hd / 32, st));
   return TL_OK;
@@ -774,6 +784,7 @@ tl_status run_qkv_attn(tl_model* m, int layer, int M, const RowCtx* rows, cudaSt
     a.k_plane = m->k_plane(layer); a.v_plane = m->v_plane(layer);
     a.lane_stride = m->lane_stride; a.ctx = c.max_ctx;
     a.o = m->o + (size_t)r0 * qdim; a.err_flag = m->err_flag;
+    a.trace = next_trace(m);
     const size_t smem = qa_layout(c.d_model, a.M, a.rep, c.head_dim).total;
     const dim3 grid(kQaCluster, c.n_kv_heads);
     if (c.head_dim == 64)
@@ -797,6 +808,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   a.pair_mode = PAIR_NEIGHBOUR;
   a.resid = x; a.ldr = d;
   a.err_flag = m->err_flag;
+  a.trace = next_trace(m);
   kclass(TL_KERNEL_O_PROJ);
   TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, (b.o.N + 15) / 16, st));
   GemvArgs g{};
@@ -806,6 +818,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   g.pair_mode = PAIR_OFFSET; g.pair_off = F / 16;
   g.yf = h; g.ldy = F;
   g.err_flag = m->err_flag;
+  g.trace = next_trace(m);
   kclass(TL_KERNEL_GATE_UP);
   TL_CUDA(launch_gemv_rows(g, M, IN_NORM, EPI_SWIGLU, F / 16, st));
   GemvArgs dn{};
@@ -814,6 +827,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   dn.pair_mode = PAIR_NEIGHBOUR;
   dn.resid = x; dn.ldr = d;
   dn.err_flag = m->err_flag;
+  dn.trace = next_trace(m);
   kclass(TL_KERNEL_DOWN);
   TL_CUDA(launch_gemv_rows(dn, M, IN_F32, EPI_RESID, (b.down.N + 15) / 16, st));
   return TL_OK;
@@ -1280,6 +1294,8 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
     active[layer] = M;
   }
   auto body = [&](cudaStream_t s) -> tl_status {
+    m->trace_i = 0;   // layer launches of this step take timeline records 0, 1, ...
+    struct TraceOff { tl_model* m; ~TraceOff() { m->trace_i = -1; } } trace_off{m};
     for (int layer = 0; layer < max_layers; ++layer) {
       const int M = active[layer];
       tl_status rc = TL_OK;
