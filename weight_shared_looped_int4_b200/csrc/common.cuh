@@ -19,10 +19,11 @@ struct RowCtx {
 };
 
 // ---- programmatic dependent launch -------------------------------------
-// Every kernel of the forward pass calls pdl_trigger() early (so the next
-// kernel may start its weight prefetch) and pdl_wait() before it reads any
-// activation the previous kernel wrote.  Every kernel waits, so completion is
-// transitive along the stream.
+// Kernels of the forward pass call pdl_trigger() (most at their start, so the
+// next kernel may start its weight prefetch; the decode GEMVs where their
+// caller says, the clustered QKV + attention kernel never) and pdl_wait()
+// before they read anything an earlier kernel wrote.  Every kernel waits, so
+// completion is transitive along the stream.
 __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }

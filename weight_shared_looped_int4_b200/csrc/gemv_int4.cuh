@@ -21,7 +21,8 @@
 //   memory in a fixed order, so results are deterministic and each activation
 //   row's result does not depend on how many rows share the launch.
 // * Weight prefetch is issued before griddepcontrol.wait, so it overlaps the
-//   tail of the previous kernel under programmatic dependent launch.
+//   tail of the previous kernel under programmatic dependent launch (the
+//   caller picks where the kernel releases its own dependent: PdlTrigger).
 // * fp32 activations are split into an fp16 pair x = hi + lo (lo is the fp16
 //   rounding of x - hi) and both halves go through the MMA, so the product
 //   keeps about 22 bits of the activation instead of fp16's 11.  The looped
@@ -39,6 +40,12 @@ namespace tl {
 enum GemvIn { IN_NORM = 0, IN_F16 = 1, IN_F32 = 2 };
 enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_ROPE_KV = 3 };
 enum PairMode { PAIR_NEIGHBOUR = 0, PAIR_OFFSET = 1, PAIR_ROPE = 2 };
+// When the kernel lets the next kernel of the stream launch (programmatic
+// dependent launch).  A dependent launched early prefetches its weights
+// during this kernel, but its CTAs land wherever this kernel's leave room,
+// several on one SM at times; measured on the decode step, the gate_up ->
+// down hand-off is faster with the trigger after the main loop.
+enum PdlTrigger { TRIGGER_AT_START = 0, TRIGGER_AFTER_LOOP = 1 };
 
 struct GemvArgs {
   const uint4* w;      // tiled weights  [n_tiles][K/64][32] (see repack)
@@ -77,6 +84,7 @@ struct GemvArgs {
   int* err_flag;       // device fault flags (a bounded wait gave up)
   unsigned long long* trace;  // launch timeline (kTraceEvents entries) or NULL:
                               // released, weights arrived, main loop done
+  int trigger;                // PdlTrigger
 };
 
 constexpr int kGemvThreads = 256;
@@ -149,7 +157,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   }
 
   trace_start(a.trace);
-  pdl_trigger();
+  if (a.trigger == TRIGGER_AT_START) pdl_trigger();
   // The weights do not depend on earlier kernels: start their bulk copies
   // before waiting for the previous kernel.
   if (threadIdx.x == 0) {
@@ -355,6 +363,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   }
 
   trace_mark(a.trace, 4);
+  if (a.trigger == TRIGGER_AFTER_LOOP) pdl_trigger();
   // ---- reduce the K slices (fixed order) ---------------------------------
   float* myred = red + (kq * TPC + tsel) * 16 * NC;
   if (NT == 0 && LO) {  // columns (2m, 2m+1) = (hi, lo) parts of row m = t

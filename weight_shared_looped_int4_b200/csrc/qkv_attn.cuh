@@ -12,9 +12,16 @@
 // rows).  A cluster of kQaCluster CTAs computes those rows, exchanges q and
 // the new key/value through distributed shared memory, synchronises with the
 // hardware cluster barrier and runs the attention over the lane's cache with
-// the keys split across its CTAs; the split results are merged in the rank-0
-// CTA's shared memory.  That removes a kernel boundary (and its global round
-// trips) per layer.
+// the keys split across its CTAs.  Each rank sends its split's running max
+// and weight sum to every rank and each slice of its weighted value sums to
+// the rank that owns that slice of the head dimension, so after the second
+// cluster barrier every rank merges hd / kQaCluster dimensions of every head.
+// That removes a kernel boundary (and its global round trips) per layer.
+//
+// The lane's cached keys and values (positions before the new one) do not
+// depend on this step: once the row table is read, one thread bulk-copies the
+// first chunk of the rank's key split into shared memory, and the copy runs
+// under the RMSNorm, the GEMV and the first exchange.
 //
 // CTA c of cluster g: GEMV of RoPE pair units u = c, c + kQaCluster, ...
 // (tiles j and j + hd/32 of one head), weights bulk-copied into shared memory
@@ -33,6 +40,8 @@ constexpr int kQaWarps = kQaThreads / 32;
 constexpr int kQaMaxRows = 2;
 constexpr int kQaMaxUnits = 2;        // RoPE pair units per CTA
 constexpr int kQaChunk = 64;          // keys per staged chunk
+static_assert(kQaMaxUnits * 16 * kQaMaxRows <= kQaThreads, "one epilogue element per thread");
+static_assert(kQaMaxRows * 8 * 8 <= kQaThreads, "one merged (row, head, dimension) per thread");
 
 struct QkvAttnArgs {
   const uint4* w;        // QKV weights, GEMV tile layout [n16 tiles][K/64][32]
@@ -60,21 +69,22 @@ __host__ __device__ inline int qa_units(int rep, int hd) { return (rep + 2) * hd
 __host__ __device__ inline int qa_units_per_cta(int rep, int hd) {
   return (qa_units(rep, hd) + kQaCluster - 1) / kQaCluster;
 }
-// Shared memory: weight tiles (reused for key/value chunks), partial results
-// of every rank (used in rank 0), activation planes, reduction buffer, q and
-// the new key/value of every row.
+// Shared memory: weight tiles, one key/value chunk per row (the prefetched
+// first chunk, then later chunks), the partials this rank merges, activation
+// planes, reduction buffer, q and the new key/value of every row, scores.
 struct QaLayout {
-  size_t w, part, act, red, q, kv, total;
+  size_t w, kvc, pml, pv, act, red, q, kv, total;
 };
 __host__ __device__ inline QaLayout qa_layout(int K, int M, int rep, int hd) {
   QaLayout L;
   const size_t tile = (size_t)(K / 64) * 512 + (size_t)(K / 128) * 64;
-  size_t wbytes = (size_t)2 * qa_units_per_cta(rep, hd) * tile;
-  const size_t chunk = (size_t)2 * kQaChunk * hd * 2;
-  if (wbytes < chunk) wbytes = chunk;
+  const size_t wbytes = (size_t)2 * qa_units_per_cta(rep, hd) * tile;
+  const size_t chunk = (size_t)2 * kQaChunk * hd * 2;   // keys then values, fp16
   L.w = 0;
-  L.part = (wbytes + 127) / 128 * 128;
-  L.act = L.part + ((size_t)kQaCluster * M * rep * (hd + kPartPad) * 4 + 127) / 128 * 128;
+  L.kvc = (wbytes + 127) / 128 * 128;
+  L.pml = L.kvc + (size_t)M * chunk;
+  L.pv = L.pml + ((size_t)kQaCluster * M * rep * 8 + 127) / 128 * 128;
+  L.act = L.pv + ((size_t)kQaCluster * M * rep * (hd / kQaCluster) * 4 + 127) / 128 * 128;
   L.red = L.act + ((size_t)M * (K + 8) * 2 * 2 + 127) / 128 * 128;
   L.q = L.red + (size_t)kQaWarps * 2 * kQaMaxUnits * 64 * 4;
   L.kv = L.q + (size_t)M * rep * hd * 4;
@@ -100,19 +110,25 @@ __device__ __forceinline__ unsigned qa_peer(const void* p, unsigned rank) {
 __device__ __forceinline__ void qa_st_peer(unsigned addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
+__device__ __forceinline__ void qa_st_peer2(unsigned addr, float x, float y) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnArgs a) {
   constexpr int DPL = HD / 32;
   constexpr int ROW16 = HD / 8;
+  constexpr int SW = HD / kQaCluster;   // head dimensions merged by each rank
   extern __shared__ __align__(128) unsigned char qsm[];
-  __shared__ __align__(8) uint64_t wbar;
-  __shared__ int s_ok;
+  __shared__ __align__(8) uint64_t wbar, kvbar;
+  __shared__ int s_ok, s_kv_ok;
   __shared__ float s_ss[kQaMaxRows][kQaWarps];
   const int K = a.K, M = a.M, rep = a.rep;
   const QaLayout L = qa_layout(K, M, rep, HD);
   unsigned char* wsm = qsm + L.w;
-  float* part = reinterpret_cast<float*>(qsm + L.part);     // [rank][m][h][hd + kPartPad]
+  __half* kvc = reinterpret_cast<__half*>(qsm + L.kvc);     // [m][keys, values][kQaChunk][hd]
+  float2* pml = reinterpret_cast<float2*>(qsm + L.pml);     // [rank][m][h]: (max, sum of weights)
+  float* pv = reinterpret_cast<float*>(qsm + L.pv);         // [rank][m][h][SW]: this rank's dims
   __half* xs = reinterpret_cast<__half*>(qsm + L.act);
   __half* xl = xs + (size_t)M * (K + 8);
   float* red = reinterpret_cast<float*>(qsm + L.red);       // [warp][tile][16][4]
@@ -128,8 +144,8 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   const int U = qa_units(rep, HD), hp = HD / 32;
   const int qdim = a.Hkv * rep * HD, kvdim = a.Hkv * HD;
   const size_t wt_bytes = (size_t)(K / 64) * 512, sz_bytes = (size_t)(K / 128) * 64;
-  int nu = 0, units[kQaMaxUnits];
-  for (int u = c; u < U && nu < kQaMaxUnits; u += kQaCluster) units[nu++] = u;
+  // this CTA's units: c, c + kQaCluster, ... (nu of them)
+  const int nu = c < U ? min(kQaMaxUnits, (U - 1 - c) / kQaCluster + 1) : 0;
   // group-local unit -> global 16-row tile of the QKV output: group heads are
   // rep query heads, then the key head, then the value head
   auto unit_tile = [&](int u, int second) -> int {
@@ -139,13 +155,17 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   };
 
   trace_start(a.trace);
-  pdl_trigger();
+  // No early trigger: the next kernel (the O projection) launches when this
+  // one completes.  Launched early, its CTAs and, through its own trigger,
+  // gate_up's crowd onto the SMs this kernel leaves free; the decode step
+  // measured faster without.
   if (tid == 0) {
     mbar_init(&wbar, 1);
+    mbar_init(&kvbar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(&wbar, (unsigned)(2 * nu * (wt_bytes + sz_bytes)));
     for (int i = 0; i < 2 * nu; ++i) {
-      const int tile = unit_tile(units[i >> 1], i & 1);
+      const int tile = unit_tile(c + (i >> 1) * kQaCluster, i & 1);
       const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
       for (size_t off = 0; off < wt_bytes; off += 32768) {
         const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
@@ -160,6 +180,43 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   qa_cluster_sync();
   pdl_wait();
   trace_mark(a.trace, 2);
+  RowCtx rcs[kQaMaxRows];
+#pragma unroll
+  for (int m = 0; m < kQaMaxRows; ++m) rcs[m] = m < M ? a.rows[m] : RowCtx{0, 0};
+  // the first chunk of this rank's key split of every row, minus the new key
+  if (tid == 0) {
+    unsigned bytes = 0;
+    int lo[kQaMaxRows], cnt[kQaMaxRows];
+#pragma unroll
+    for (int m = 0; m < kQaMaxRows; ++m) {
+      cnt[m] = 0;
+      lo[m] = 0;
+      if (m < M) {
+        const int n = rcs[m].pos + 1, C = (n + kQaCluster - 1) / kQaCluster;
+        lo[m] = min(n, c * C);
+        const int hi = min(min(n, lo[m] + C), lo[m] + kQaChunk);
+        cnt[m] = max(0, min(hi, rcs[m].pos) - lo[m]);
+        bytes += 2u * (unsigned)cnt[m] * HD * 2u;
+      }
+    }
+    mbar_arrive_expect_tx(&kvbar, bytes);
+#pragma unroll
+    for (int m = 0; m < kQaMaxRows; ++m) {
+      if (cnt[m] > 0) {
+        const size_t src = (size_t)rcs[m].lane * a.lane_stride + ((size_t)grp * a.ctx + lo[m]) * HD;
+        __half* dst = kvc + (size_t)m * 2 * kQaChunk * HD;
+        bulk_g2s(dst, a.k_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
+        bulk_g2s(dst + kQaChunk * HD, a.v_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
+      }
+    }
+  }
+  // RoPE (cos, sin) of this thread's epilogue element (loaded under the GEMV)
+  float2 cs_pre = make_float2(1.f, 0.f);
+  if (tid < nu * 16 * M) {
+    const int ul = tid / (16 * M), rem = tid % (16 * M), r = rem & 15, m = rem >> 4;
+    const int u = c + ul * kQaCluster, hh = u / hp, j = (u % hp) * 16 + r;
+    if (hh <= rep) cs_pre = rope_cs(a.rope_tab, rcs[m].pos, j, HD, a.theta);
+  }
 
   // ---- RMSNorm of the rows into the (hi, lo) planes: every thread loads its
   // columns of every row (and the gains) at once and keeps them in registers
@@ -272,7 +329,8 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   __syncthreads();
 
   // ---- epilogue: RoPE; q to every rank, k / v to the cache and every rank --
-  for (int e = tid; e < nu * 16 * M; e += kQaThreads) {
+  if (tid < nu * 16 * M) {   // nu * 16 * M <= 64: one element per thread
+    const int e = tid;
     const int ul = e / (16 * M), rem = e % (16 * M), r = rem & 15, m = rem >> 4;
     float va = 0.f, vb = 0.f;
 #pragma unroll
@@ -280,11 +338,14 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       va += red[((size_t)w * 2 * kQaMaxUnits + 2 * ul) * 64 + r * 4 + m];
       vb += red[((size_t)w * 2 * kQaMaxUnits + 2 * ul + 1) * 64 + r * 4 + m];
     }
-    const int u = units[ul], hh = u / hp, j = (u % hp) * 16 + r;   // element j < hd/2 of group head hh
-    const RowCtx rc = a.rows[m];
+    const int u = c + ul * kQaCluster, hh = u / hp, j = (u % hp) * 16 + r;   // element j < hd/2 of group head hh
+    RowCtx rc = rcs[0];
+#pragma unroll
+    for (int q = 1; q < kQaMaxRows; ++q)
+      if (m == q) rc = rcs[q];
     float e0 = va, e1 = vb;                                          // elements j and j + hd/2
     if (hh <= rep) {                                                 // query or key: rotate
-      const float2 cs = rope_cs(a.rope_tab, rc.pos, j, HD, a.theta);
+      const float2 cs = cs_pre;
       e0 = va * cs.x - vb * cs.y;
       e1 = vb * cs.x + va * cs.y;
     }
@@ -310,39 +371,62 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
 
   // ---- attention over this rank's key split, per row -------------------------
   const float scale = 1.0f / sqrtf((float)HD);
-  __half* ks = reinterpret_cast<__half*>(wsm);            // [kQaChunk][HD]
-  __half* vs = ks + kQaChunk * HD;
+  if (tid == 0) {   // the prefetched chunks (published by the barrier after the state reset)
+    s_kv_ok = mbar_wait(&kvbar, 0) ? 1 : 0;
+    if (!s_kv_ok) atomicOr(a.err_flag, kErrTimeout);
+  }
   for (int m = 0; m < M; ++m) {
-    const RowCtx rc = a.rows[m];
+    RowCtx rc = rcs[0];
+#pragma unroll
+    for (int q = 1; q < kQaMaxRows; ++q)
+      if (m == q) rc = rcs[q];
     const int n = rc.pos + 1;
     const int C = (n + kQaCluster - 1) / kQaCluster;
     const int j0 = min(n, c * C), j1 = min(n, j0 + C);
     const __half* kb = a.k_plane + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
     const __half* vb = a.v_plane + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
+    __half* ks = kvc + (size_t)m * 2 * kQaChunk * HD;      // [kQaChunk][HD]
+    __half* vs = ks + kQaChunk * HD;
     const float* qrow = qb + (size_t)m * rep * HD;
     float acc2[4] = {0.f, 0.f, 0.f, 0.f};    // (head, dim) = tid + i * 256, rep * HD <= 1024
     if (tid < rep) { ml[4 * tid] = -INFINITY; ml[4 * tid + 1] = 0.f; ml[4 * tid + 2] = 0.f; }
     __syncthreads();
     for (int jc = j0; jc < j1; jc += kQaChunk) {
       const int nk = min(kQaChunk, j1 - jc);
-      // chunk into shared memory; the row's newest key / value come from the cluster
-      for (int e = tid; e < 2 * kQaChunk * ROW16; e += kQaThreads) {
-        const int kv = e / (kQaChunk * ROW16), rem = e % (kQaChunk * ROW16);
-        const int key = rem / ROW16, pc = rem % ROW16;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (key < nk) {
-          const int jj = jc + key;
-          if (jj == rc.pos) {
-            const float* s = (kv ? vnew : knew) + (size_t)m * HD + pc * 8;
+      if (jc == j0) {
+        // prefetched: every cached key of the chunk; the row's new key / value
+        // (the last key of the context) come from the cluster exchange
+        if (rc.pos < jc + nk) {
+          const int key = rc.pos - jc;
+          for (int e = tid; e < 2 * ROW16; e += kQaThreads) {
+            const int kv = e / ROW16, pc = e % ROW16;
+            const float* src = (kv ? vnew : knew) + (size_t)m * HD + pc * 8;
             __half2 h[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(s[2 * q], s[2 * q + 1]);
-            val = *reinterpret_cast<uint4*>(h);
-          } else {
-            val = __ldcg(reinterpret_cast<const uint4*>((kv ? vb : kb) + (size_t)jj * HD) + pc);
+            for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(src[2 * q], src[2 * q + 1]);
+            reinterpret_cast<uint4*>((kv ? vs : ks) + (size_t)key * HD)[pc] = *reinterpret_cast<uint4*>(h);
           }
         }
-        reinterpret_cast<uint4*>(ks)[e] = val;
+      } else {
+        // later chunks (splits longer than kQaChunk keys): plain loads
+        for (int e = tid; e < 2 * kQaChunk * ROW16; e += kQaThreads) {
+          const int kv = e / (kQaChunk * ROW16), rem = e % (kQaChunk * ROW16);
+          const int key = rem / ROW16, pc = rem % ROW16;
+          uint4 val = make_uint4(0, 0, 0, 0);
+          if (key < nk) {
+            const int jj = jc + key;
+            if (jj == rc.pos) {
+              const float* src = (kv ? vnew : knew) + (size_t)m * HD + pc * 8;
+              __half2 h[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(src[2 * q], src[2 * q + 1]);
+              val = *reinterpret_cast<uint4*>(h);
+            } else {
+              val = __ldcg(reinterpret_cast<const uint4*>((kv ? vb : kb) + (size_t)jj * HD) + pc);
+            }
+          }
+          reinterpret_cast<uint4*>(ks)[e] = val;
+        }
       }
       __syncthreads();
       for (int jj = warp; jj < nk; jj += kQaWarps) {
@@ -403,46 +487,43 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       }
       __syncthreads();   // the chunk buffers are reused
     }
-    // partial (sums, max, sum of weights) of this rank into rank 0
+    // this split's (max, sum of weights) to every rank, each slice of its
+    // weighted value sums to the rank that merges those dimensions
+    if (tid < rep * kQaCluster) {
+      const int h = tid / kQaCluster, rk = tid % kQaCluster;
+      qa_st_peer2(qa_peer(pml + ((size_t)c * M + m) * rep + h, (unsigned)rk), ml[4 * h], ml[4 * h + 1]);
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int oi = tid + i * kQaThreads;
       if (oi < rep * HD) {
         const int h = oi / HD, dim = oi % HD;
-        float* pp = part + (((size_t)c * M + m) * rep + h) * (HD + kPartPad);
-        qa_st_peer(qa_peer(pp + dim, 0), acc2[i]);
-        if (dim == 0) {
-          qa_st_peer(qa_peer(pp + HD, 0), ml[4 * h]);
-          qa_st_peer(qa_peer(pp + HD + 1, 0), ml[4 * h + 1]);
-        }
+        qa_st_peer(qa_peer(pv + (((size_t)c * M + m) * rep + h) * SW + dim % SW, (unsigned)(dim / SW)), acc2[i]);
       }
     }
-    __syncthreads();
+    __syncthreads();   // ml is reset for the next row
   }
-  qa_cluster_sync();   // #2: every rank's partials are in rank 0
+  qa_cluster_sync();   // #2: every rank holds every split's partials of its dimensions
   trace_mark(a.trace, 4);
 
-  // ---- rank 0 merges the ranks in order --------------------------------------
-  if (c == 0) {
-    for (int e = tid; e < M * rep * HD; e += kQaThreads) {
-      const int m = e / (rep * HD), oi = e % (rep * HD), h = oi / HD, dim = oi % HD;
-      float mx = -INFINITY;
+  // ---- each rank merges its SW dimensions of every (row, head), ranks in order
+  if (tid < M * rep * SW) {
+    const int m = tid / (rep * SW), rem = tid % (rep * SW), h = rem / SW, dd = rem % SW;
+    float mx = -INFINITY;
 #pragma unroll
-      for (int rk = 0; rk < kQaCluster; ++rk)
-        mx = fmaxf(mx, part[(((size_t)rk * M + m) * rep + h) * (HD + kPartPad) + HD]);
-      float num = 0.f, den = 0.f;
+    for (int rk = 0; rk < kQaCluster; ++rk) mx = fmaxf(mx, pml[((size_t)rk * M + m) * rep + h].x);
+    float num = 0.f, den = 0.f;
 #pragma unroll
-      for (int rk = 0; rk < kQaCluster; ++rk) {
-        const float* pp = part + (((size_t)rk * M + m) * rep + h) * (HD + kPartPad);
-        const float l = pp[HD + 1];
-        if (l > 0.f) {   // ranks without keys contribute nothing
-          const float w = expf(pp[HD] - mx);
-          num = fmaf(w, pp[dim], num);
-          den = fmaf(w, l, den);
-        }
+    for (int rk = 0; rk < kQaCluster; ++rk) {
+      const float2 st = pml[((size_t)rk * M + m) * rep + h];
+      if (st.y > 0.f) {   // ranks without keys contribute nothing
+        const float w = expf(st.x - mx);
+        num = fmaf(w, pv[(((size_t)rk * M + m) * rep + h) * SW + dd], num);
+        den = fmaf(w, st.y, den);
       }
-      if (ok) a.o[(size_t)m * (a.Hkv * rep * HD) + (size_t)(grp * rep + h) * HD + dim] = num / den;
     }
+    if (ok && s_kv_ok)
+      a.o[(size_t)m * (a.Hkv * rep * HD) + (size_t)(grp * rep + h) * HD + c * SW + dd] = num / den;
   }
   trace_mark(a.trace, 5);
 }

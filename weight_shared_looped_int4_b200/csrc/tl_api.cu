@@ -809,6 +809,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   a.resid = x; a.ldr = d;
   a.err_flag = m->err_flag;
   a.trace = next_trace(m);
+  a.trigger = TRIGGER_AT_START;
   kclass(TL_KERNEL_O_PROJ);
   TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, (b.o.N + 15) / 16, st));
   GemvArgs g{};
@@ -819,6 +820,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   g.yf = h; g.ldy = F;
   g.err_flag = m->err_flag;
   g.trace = next_trace(m);
+  g.trigger = TRIGGER_AFTER_LOOP;
   kclass(TL_KERNEL_GATE_UP);
   TL_CUDA(launch_gemv_rows(g, M, IN_NORM, EPI_SWIGLU, F / 16, st));
   GemvArgs dn{};
@@ -828,6 +830,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   dn.resid = x; dn.ldr = d;
   dn.err_flag = m->err_flag;
   dn.trace = next_trace(m);
+  dn.trigger = TRIGGER_AT_START;
   kclass(TL_KERNEL_DOWN);
   TL_CUDA(launch_gemv_rows(dn, M, IN_F32, EPI_RESID, (b.down.N + 15) / 16, st));
   return TL_OK;
