@@ -326,7 +326,7 @@ def run_trace(args):
     tl.tl_model_set_decode_path(m, DECODE_PATHS["layered"])
     tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS)
     n_rec = 4 * (2 + LOOPS)   # layer launches: QKV + attention, O, gate_up, down
-    hbuf = torch.zeros(4 * G + 6 * n_rec, dtype=torch.int64, device="cuda:0")
+    hbuf = torch.zeros(4 * G + 12 * n_rec, dtype=torch.int64, device="cuda:0")
     tl.tl_model_set_trace(m, hbuf, hbuf.numel())
     tok[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
     heads, recs = [], []
@@ -339,7 +339,7 @@ def run_trace(args):
         heads.append((float(h[1].max() - h[0].min()), float(np.median(h[2] - h[1])), float(h[2].max() - h[1].min()),
                       float(h[3].max() - h[0].min())))
         last_h = h
-        r = raw[4 * G:].reshape(n_rec, 6).view(np.uint64).copy()
+        r = raw[4 * G:].reshape(n_rec, 12).view(np.uint64).copy()
         r[:, 0] = ~r[:, 0]   # the first start is stored complemented
         recs.append((r.astype(np.float64) / 1e3, float(h[0].min()), float(h[3].max())))
     tl.tl_model_destroy(m)
@@ -353,7 +353,7 @@ def run_trace(args):
     # its CTAs waited for the previous kernel's end, and its phases after that
     names = ("qkv_attn", "o_proj", "gate_up", "down")
     acc = {n: {"critical_path": [], "started_before_prev_end": [], "release_after_prev_end": [],
-               "phase1": [], "phase2": [], "phase3": []} for n in names}
+               "phase1": [], "phase2": [], "phase3": [], "phase1a": [], "phase2a": []} for n in names}
     step_us, head_tail = [], []
     for r, h_start, h_end in recs[2:]:
         step_us.append(h_end - r[0, 0])
@@ -368,9 +368,17 @@ def run_trace(args):
             if i % 4 == 0:   # clustered: GEMV + exchange, attention + exchange, merge
                 a["phase1"].append(r[i, 3] - rel)
                 a["phase2"].append(r[i, 4] - r[i, 3])
+                a["phase1a"].append(r[i, 6] - rel)        # to the last arrival at barrier 1
+                a["phase2a"].append(r[i, 7] - r[i, 3])    # to the last arrival at barrier 2
+                for key, v in (("norm", r[i, 8] - rel), ("weights", r[i, 9] - r[i, 8]),
+                               ("gemv", r[i, 10] - r[i, 9]), ("epilogue", r[i, 6] - r[i, 10]),
+                               ("keys_after_barrier1", r[i, 11] - r[i, 3])):
+                    a.setdefault("p1_" + key, []).append(v)
             else:            # GEMV: weights-ready wait after release, main loop, epilogue
                 a["phase1"].append(max(r[i, 3] - rel, 0.0))
                 a["phase2"].append(r[i, 4] - max(r[i, 3], rel))
+                a["phase1a"].append(r[i, 6] - rel)        # activations staged
+                a["phase2a"].append(0.0)
             a["phase3"].append(r[i, 5] - r[i, 4])
     r, h_start, h_end = recs[-1]
     out["layered_last_step_per_launch"] = [
@@ -385,9 +393,11 @@ def run_trace(args):
         "last_start": round(float(last_h[0].max() - d_end), 2), "median_staged": round(float(np.median(last_h[1]) - d_end), 2),
         "last_staged": round(float(last_h[1].max() - d_end), 2), "last_end": round(float(last_h[3].max() - d_end), 2)}
     out["layered_kernels_us"] = {n: {k: round(statistics.mean(v), 2) for k, v in a.items()} for n, a in acc.items()}
-    out["layered_phases"] = {"qkv_attn": "phase1 RMSNorm+QKV GEMV+RoPE+exchange, phase2 attention+exchange, "
+    out["layered_phases"] = {"qkv_attn": "phase1 RMSNorm+QKV GEMV+RoPE+exchange (phase1a: up to the last "
+                                         "arrival at its barrier), phase2 attention+exchange (phase2a: likewise), "
                                          "phase3 merge",
-                             "gemv": "phase1 wait for weights after release, phase2 main loop, phase3 epilogue"}
+                             "gemv": "phase1 release to weights ready (phase1a: activations staged), "
+                                     "phase2 main loop, phase3 epilogue"}
     print(json.dumps(out))
     return 0
 

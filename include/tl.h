@@ -252,13 +252,16 @@ tl_status tl_model_set_decode_path(tl_model *m, int path);
  * launches of the layered path (output norm + head + argmax) write slots 0
  * (start), 1 (activations staged), 2 (head tiles done), 3 (end).  Each layer
  * launch of a layered step (per effective layer: QKV (+ attention), O,
- * gate_up, down, in launch order; launch i) writes 6 entries from
- * 4 G + 6 i, each an atomic maximum over its CTAs (thread 0), so the caller
+ * gate_up, down, in launch order; launch i) writes 12 entries from
+ * 4 G + 12 i, each an atomic maximum over its CTAs (thread 0), so the caller
  * zeroes them before the step: 0 the earliest CTA start, stored complemented
  * (~t); 1 the latest CTA start; 2 the latest return from the wait for the
  * previous kernel; 3 and 4 GEMV: weights arrived, main loop done; clustered
  * QKV + attention: q/k/v exchanged, attention partials exchanged; 5 the
- * latest CTA end.  A decode graph captured while a buffer is set keeps
+ * latest CTA end; 6 and 7 GEMV: activations staged, unused; clustered:
+ * arrival at the q/k/v and at the partials exchange barrier; 8 to 11
+ * clustered only: rows normalised, weights arrived, GEMV reduced, cached
+ * keys arrived.  A decode graph captured while a buffer is set keeps
  * writing to that buffer. */
 tl_status tl_model_set_trace(tl_model *m, unsigned long long *d_buf, long long n_entries);
 int tl_model_trace_grid(const tl_model *m);

@@ -58,7 +58,7 @@ __device__ __forceinline__ long long globaltimer_ns() {
 // one launch (zeroed by the caller), or is NULL.  Thread 0 of every CTA
 // stamps event e >= 1 as the latest %globaltimer over the CTAs; event 0 holds
 // the earliest start, complemented (so that both use atomicMax).
-constexpr int kTraceEvents = 6;   // first start, last start, released, mid 1, mid 2, end
+constexpr int kTraceEvents = 12;  // first start, last start, released, mid 1, mid 2, end, extra 6 .. 11
 __device__ __forceinline__ void trace_start(unsigned long long* tr) {
   if (tr && threadIdx.x == 0) {
     const unsigned long long t = (unsigned long long)globaltimer_ns();

@@ -83,7 +83,8 @@ struct GemvArgs {
   const float2* rope_tab;  // (cos, sin) [positions][hd/2], or NULL
   int* err_flag;       // device fault flags (a bounded wait gave up)
   unsigned long long* trace;  // launch timeline (kTraceEvents entries) or NULL:
-                              // released, weights arrived, main loop done
+                              // released, weights arrived, main loop done,
+                              // (6) activations staged
   int trigger;                // PdlTrigger
 };
 
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
     }
   }
   if (threadIdx.x == 0) {
+    trace_mark(a.trace, 6);
     s_ok = mbar_wait(&wbar, 0) ? 1 : 0;
     if (!s_ok) atomicOr(a.err_flag, kErrTimeout);
     trace_mark(a.trace, 3);

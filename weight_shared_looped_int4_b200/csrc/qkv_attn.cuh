@@ -62,7 +62,10 @@ struct QkvAttnArgs {
   float* o;              // attention output [M][Hq*hd] fp32
   int* err_flag;
   unsigned long long* trace;  // launch timeline (kTraceEvents entries) or NULL:
-                              // released, q/k/v exchanged, partials exchanged
+                              // released, q/k/v exchanged, partials exchanged,
+                              // (6, 7) arrival at the two exchange barriers,
+                              // (8) rows normalised, (9) weights arrived,
+                              // (10) GEMV reduced, (11) key prefetch arrived
 };
 
 __host__ __device__ inline int qa_units(int rep, int hd) { return (rep + 2) * hd / 32; }
@@ -121,7 +124,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   constexpr int SW = HD / kQaCluster;   // head dimensions merged by each rank
   extern __shared__ __align__(128) unsigned char qsm[];
   __shared__ __align__(8) uint64_t wbar, kvbar;
-  __shared__ int s_ok, s_kv_ok;
+  __shared__ int s_ok;
   __shared__ float s_ss[kQaMaxRows][kQaWarps];
   const int K = a.K, M = a.M, rep = a.rep;
   const QaLayout L = qa_layout(K, M, rep, HD);
@@ -136,7 +139,6 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   float* knew = reinterpret_cast<float*>(qsm + L.kv);       // [m][hd]
   float* vnew = knew + (size_t)M * HD;                       // [m][hd]
   float* sc = vnew + (size_t)M * HD;                         // [rep][kQaChunk]
-  float* ml = sc + rep * kQaChunk;                           // [rep][4]: max, sum, rescale
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, t4 = lane & 3;
   const unsigned crank = qa_cluster_rank();
@@ -183,6 +185,21 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   RowCtx rcs[kQaMaxRows];
 #pragma unroll
   for (int m = 0; m < kQaMaxRows; ++m) rcs[m] = m < M ? a.rows[m] : RowCtx{0, 0};
+  // ---- RMSNorm of the rows into the (hi, lo) planes: every thread loads its
+  // columns of every row (and the gains) at once and keeps them in registers
+  constexpr int V4 = 4;                       // float4 columns per thread and row: K <= 4096
+  float4 xv[kQaMaxRows][V4];
+  uint2 gv[V4];
+#pragma unroll
+  for (int i = 0; i < V4; ++i) {
+    const int k = tid * 4 + i * 4 * kQaThreads;
+    gv[i] = k < K ? *reinterpret_cast<const uint2*>(a.gain + k) : make_uint2(0u, 0u);
+#pragma unroll
+    for (int m = 0; m < kQaMaxRows; ++m)
+      xv[m][i] = (m < M && k < K) ? *reinterpret_cast<const float4*>(a.x + (size_t)m * K + k)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // (issued after the row loads above, so that they overlap)
   // the first chunk of this rank's key split of every row, minus the new key
   if (tid == 0) {
     unsigned bytes = 0;
@@ -218,20 +235,6 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     if (hh <= rep) cs_pre = rope_cs(a.rope_tab, rcs[m].pos, j, HD, a.theta);
   }
 
-  // ---- RMSNorm of the rows into the (hi, lo) planes: every thread loads its
-  // columns of every row (and the gains) at once and keeps them in registers
-  constexpr int V4 = 4;                       // float4 columns per thread and row: K <= 4096
-  float4 xv[kQaMaxRows][V4];
-  uint2 gv[V4];
-#pragma unroll
-  for (int i = 0; i < V4; ++i) {
-    const int k = tid * 4 + i * 4 * kQaThreads;
-    gv[i] = k < K ? *reinterpret_cast<const uint2*>(a.gain + k) : make_uint2(0u, 0u);
-#pragma unroll
-    for (int m = 0; m < kQaMaxRows; ++m)
-      xv[m][i] = (m < M && k < K) ? *reinterpret_cast<const float4*>(a.x + (size_t)m * K + k)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-  }
 #pragma unroll
   for (int m = 0; m < kQaMaxRows; ++m) {
     float ss = 0.f;
@@ -269,8 +272,10 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     }
   }
   if (tid == 0) {
+    trace_mark(a.trace, 8);
     s_ok = mbar_wait(&wbar, 0) ? 1 : 0;
     if (!s_ok) atomicOr(a.err_flag, kErrTimeout);
+    trace_mark(a.trace, 9);
   }
   __syncthreads();
   const bool ok = s_ok != 0;   // on a time-out the control flow stays the same (cluster barriers)
@@ -327,6 +332,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     }
   }
   __syncthreads();
+  trace_mark(a.trace, 10);
 
   // ---- epilogue: RoPE; q to every rank, k / v to the cache and every rank --
   if (tid < nu * 16 * M) {   // nu * 16 * M <= 64: one element per thread
@@ -366,15 +372,15 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       qa_st_peer(qa_peer(dst_s + j + HD / 2, rk), e1);
     }
   }
+  trace_mark(a.trace, 6);
   qa_cluster_sync();   // #1: q and the new key / value are in every rank
   trace_mark(a.trace, 3);
 
-  // ---- attention over this rank's key split, per row -------------------------
+  // ---- attention over this rank's key split, per row: warp h < rep takes
+  // query head h (scores, online softmax and P V stay inside the warp) ------
   const float scale = 1.0f / sqrtf((float)HD);
-  if (tid == 0) {   // the prefetched chunks (published by the barrier after the state reset)
-    s_kv_ok = mbar_wait(&kvbar, 0) ? 1 : 0;
-    if (!s_kv_ok) atomicOr(a.err_flag, kErrTimeout);
-  }
+  const bool head_warp = warp < rep;
+  float* sh = sc + (head_warp ? warp : 0) * kQaChunk;   // this warp's scores / weights
   for (int m = 0; m < M; ++m) {
     RowCtx rc = rcs[0];
 #pragma unroll
@@ -387,122 +393,121 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     const __half* vb = a.v_plane + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
     __half* ks = kvc + (size_t)m * 2 * kQaChunk * HD;      // [kQaChunk][HD]
     __half* vs = ks + kQaChunk * HD;
-    const float* qrow = qb + (size_t)m * rep * HD;
-    float acc2[4] = {0.f, 0.f, 0.f, 0.f};    // (head, dim) = tid + i * 256, rep * HD <= 1024
-    if (tid < rep) { ml[4 * tid] = -INFINITY; ml[4 * tid + 1] = 0.f; ml[4 * tid + 2] = 0.f; }
-    __syncthreads();
+    // this lane's DPL dimensions of q (head `warp`) and of the new key / value
+    float qv[DPL], kn[DPL], vn[DPL], o[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      qv[i] = head_warp ? qb[((size_t)m * rep + warp) * HD + lane * DPL + i] : 0.f;
+      kn[i] = knew[(size_t)m * HD + lane * DPL + i];
+      vn[i] = vnew[(size_t)m * HD + lane * DPL + i];
+      o[i] = 0.f;
+    }
+    float m_run = -INFINITY, l_run = 0.f;
+    if (head_warp && j0 < j1 && !mbar_wait(&kvbar, 0) && lane == 0) atomicOr(a.err_flag, kErrTimeout);
+    trace_mark(a.trace, 11);
     for (int jc = j0; jc < j1; jc += kQaChunk) {
       const int nk = min(kQaChunk, j1 - jc);
-      if (jc == j0) {
-        // prefetched: every cached key of the chunk; the row's new key / value
-        // (the last key of the context) come from the cluster exchange
-        if (rc.pos < jc + nk) {
-          const int key = rc.pos - jc;
-          for (int e = tid; e < 2 * ROW16; e += kQaThreads) {
-            const int kv = e / ROW16, pc = e % ROW16;
-            const float* src = (kv ? vnew : knew) + (size_t)m * HD + pc * 8;
-            __half2 h[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(src[2 * q], src[2 * q + 1]);
-            reinterpret_cast<uint4*>((kv ? vs : ks) + (size_t)key * HD)[pc] = *reinterpret_cast<uint4*>(h);
-          }
-        }
-      } else {
-        // later chunks (splits longer than kQaChunk keys): plain loads
+      if (jc != j0) {
+        // later chunks (splits longer than kQaChunk keys): plain loads by
+        // every thread; the new key is read from registers, not from here
+        __syncthreads();   // the previous chunk is consumed
         for (int e = tid; e < 2 * kQaChunk * ROW16; e += kQaThreads) {
           const int kv = e / (kQaChunk * ROW16), rem = e % (kQaChunk * ROW16);
-          const int key = rem / ROW16, pc = rem % ROW16;
+          const int key = rem / ROW16, pc = rem % ROW16, jj = jc + key;
           uint4 val = make_uint4(0, 0, 0, 0);
-          if (key < nk) {
-            const int jj = jc + key;
-            if (jj == rc.pos) {
-              const float* src = (kv ? vnew : knew) + (size_t)m * HD + pc * 8;
-              __half2 h[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(src[2 * q], src[2 * q + 1]);
-              val = *reinterpret_cast<uint4*>(h);
-            } else {
-              val = __ldcg(reinterpret_cast<const uint4*>((kv ? vb : kb) + (size_t)jj * HD) + pc);
-            }
-          }
+          if (key < nk && jj != rc.pos) val = __ldcg(reinterpret_cast<const uint4*>((kv ? vb : kb) + (size_t)jj * HD) + pc);
           reinterpret_cast<uint4*>(ks)[e] = val;
         }
+        __syncthreads();
       }
-      __syncthreads();
-      for (int jj = warp; jj < nk; jj += kQaWarps) {
-        const __half* kp = ks + jj * HD + lane * DPL;
-        float kf[DPL];
-        if constexpr (DPL == 4) {
-          const uint2 u2 = *reinterpret_cast<const uint2*>(kp);
-          const float2 f01 = h2_to_f2(u2.x), f23 = h2_to_f2(u2.y);
-          kf[0] = f01.x; kf[1] = f01.y; kf[2] = f23.x; kf[3] = f23.y;
-        } else {
-          const float2 f01 = h2_to_f2(*reinterpret_cast<const unsigned*>(kp));
-          kf[0] = f01.x; kf[1] = f01.y;
-        }
+      if (head_warp) {
+        // scores, eight keys at a time (independent butterfly reductions)
+        for (int j8 = 0; j8 < nk; j8 += 8) {
+          float p[8];
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          if (h < rep) {
-            float dot = 0.f;
+          for (int u = 0; u < 8; ++u) {
+            const int jj = j8 + u;
+            float d = 0.f;
+            if (jj < nk) {
+              float kf[DPL];
+              if (jc + jj == rc.pos) {
 #pragma unroll
-            for (int i = 0; i < DPL; ++i) dot = fmaf(qrow[h * HD + lane * DPL + i], kf[i], dot);
-            dot = warp_sum(dot);
-            if (lane == 0) sc[h * kQaChunk + jj] = dot * scale;
+                for (int i = 0; i < DPL; ++i) kf[i] = kn[i];
+              } else if constexpr (DPL == 4) {
+                const uint2 u2 = *reinterpret_cast<const uint2*>(ks + jj * HD + lane * 4);
+                const float2 f01 = h2_to_f2(u2.x), f23 = h2_to_f2(u2.y);
+                kf[0] = f01.x; kf[1] = f01.y; kf[2] = f23.x; kf[3] = f23.y;
+              } else {
+                const float2 f01 = h2_to_f2(*reinterpret_cast<const unsigned*>(ks + jj * HD + lane * 2));
+                kf[0] = f01.x; kf[1] = f01.y;
+              }
+#pragma unroll
+              for (int i = 0; i < DPL; ++i) d = fmaf(qv[i], kf[i], d);
+            }
+            p[u] = d;
           }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) p[u] += __shfl_xor_sync(0xffffffffu, p[u], off);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (lane == u && j8 + u < nk) sh[j8 + u] = p[u] * scale;
         }
-      }
-      __syncthreads();
-      if (warp < rep) {
-        float* sh = sc + warp * kQaChunk;
+        __syncwarp();
+        // online softmax over the chunk
         float mx = -INFINITY;
         for (int jj = lane; jj < nk; jj += 32) mx = fmaxf(mx, sh[jj]);
         mx = warp_max(mx);
-        const float m_old = ml[4 * warp], m_new = fmaxf(m_old, mx);
+        const float m_new = fmaxf(m_run, mx);
         float sum = 0.f;
         for (int jj = lane; jj < nk; jj += 32) {
-          const float p = expf(sh[jj] - m_new);
-          sh[jj] = p;
-          sum += p;
+          const float e = expf(sh[jj] - m_new);
+          sh[jj] = e;
+          sum += e;
         }
         sum = warp_sum(sum);
-        if (lane == 0) {
-          const float alpha = expf(m_old - m_new);
-          ml[4 * warp] = m_new;
-          ml[4 * warp + 1] = ml[4 * warp + 1] * alpha + sum;
-          ml[4 * warp + 2] = alpha;
-        }
-      }
-      __syncthreads();
+        const float alpha = expf(m_run - m_new);
+        l_run = l_run * alpha + sum;
+        m_run = m_new;
+        __syncwarp();
+        // P V over the lane's dimensions
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int oi = tid + i * kQaThreads;
-        if (oi < rep * HD) {
-          const int h = oi / HD, dim = oi % HD;
-          const float* ph = sc + h * kQaChunk;
-          float v = acc2[i] * ml[4 * h + 2];
-#pragma unroll 8
-          for (int jj = 0; jj < nk; ++jj) v = fmaf(ph[jj], __half2float(vs[jj * HD + dim]), v);
-          acc2[i] = v;
+        for (int i = 0; i < DPL; ++i) o[i] *= alpha;
+#pragma unroll 4
+        for (int jj = 0; jj < nk; ++jj) {
+          const float pj = sh[jj];
+          float vf[DPL];
+          if (jc + jj == rc.pos) {
+#pragma unroll
+            for (int i = 0; i < DPL; ++i) vf[i] = vn[i];
+          } else if constexpr (DPL == 4) {
+            const uint2 u2 = *reinterpret_cast<const uint2*>(vs + jj * HD + lane * 4);
+            const float2 f01 = h2_to_f2(u2.x), f23 = h2_to_f2(u2.y);
+            vf[0] = f01.x; vf[1] = f01.y; vf[2] = f23.x; vf[3] = f23.y;
+          } else {
+            const float2 f01 = h2_to_f2(*reinterpret_cast<const unsigned*>(vs + jj * HD + lane * 2));
+            vf[0] = f01.x; vf[1] = f01.y;
+          }
+#pragma unroll
+          for (int i = 0; i < DPL; ++i) o[i] = fmaf(pj, vf[i], o[i]);
         }
+        __syncwarp();   // sh is rewritten by the next chunk
       }
-      __syncthreads();   // the chunk buffers are reused
     }
     // this split's (max, sum of weights) to every rank, each slice of its
     // weighted value sums to the rank that merges those dimensions
-    if (tid < rep * kQaCluster) {
-      const int h = tid / kQaCluster, rk = tid % kQaCluster;
-      qa_st_peer2(qa_peer(pml + ((size_t)c * M + m) * rep + h, (unsigned)rk), ml[4 * h], ml[4 * h + 1]);
-    }
+    if (head_warp) {
+      if (lane < kQaCluster)
+        qa_st_peer2(qa_peer(pml + ((size_t)c * M + m) * rep + warp, (unsigned)lane), m_run, l_run);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int oi = tid + i * kQaThreads;
-      if (oi < rep * HD) {
-        const int h = oi / HD, dim = oi % HD;
-        qa_st_peer(qa_peer(pv + (((size_t)c * M + m) * rep + h) * SW + dim % SW, (unsigned)(dim / SW)), acc2[i]);
+      for (int i = 0; i < DPL; ++i) {
+        const int dim = lane * DPL + i;
+        qa_st_peer(qa_peer(pv + (((size_t)c * M + m) * rep + warp) * SW + dim % SW, (unsigned)(dim / SW)), o[i]);
       }
     }
-    __syncthreads();   // ml is reset for the next row
   }
+  trace_mark(a.trace, 7);
   qa_cluster_sync();   // #2: every rank holds every split's partials of its dimensions
   trace_mark(a.trace, 4);
 
@@ -522,7 +527,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
         den = fmaf(w, st.y, den);
       }
     }
-    if (ok && s_kv_ok)
+    if (ok)
       a.o[(size_t)m * (a.Hkv * rep * HD) + (size_t)(grp * rep + h) * HD + c * SW + dd] = num / den;
   }
   trace_mark(a.trace, 5);

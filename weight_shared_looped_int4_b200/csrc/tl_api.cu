@@ -895,6 +895,7 @@ tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, fl
     // its head tiles through a bulk-copy ring (15 compute warps)
     FusedArgs f = m->fused;
     f.head_only = 1;
+    f.head_early = getenv("TL_HEAD_EARLY") ? atoi(getenv("TL_HEAD_EARLY")) : 0;
     f.M = M;
     f.x = const_cast<float*>(x);
     for (int i = 0; i < M; ++i) f.out_row[i] = i;
@@ -933,7 +934,7 @@ tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, fl
 tl_status forward_prompt(tl_model* m, int lane, const int32_t* d_tokens, int T, int loops,
                          float* d_logits, int32_t* d_argmax, cudaStream_t st) {
   const tl_config& c = m->cfg;
-  const int d = c.d_model, qdim = c.n_q_heads * c.head_dim, F = c.ffn_dim;
+  const int d = c.d_model, qdim = c.n_q_heads * c.head_dim;
   const int n_layers = c.n_pre + loops;
   kclass(TL_KERNEL_SETUP);
   TL_CUDA(launch(fill_rows_kernel, dim3((T + 255) / 256), dim3(256), 0, st, m->rows, T, lane, 0));
