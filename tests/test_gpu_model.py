@@ -164,6 +164,33 @@ def test_tiny_paths_agree_and_auto(tiny):
         assert _max_abs(lg[lane], om.decode(cache, int(prompts[lane, 8]), 4)) <= LOGIT_MAX_ABS
 
 
+def test_width_not_multiple_of_512(path):
+    # d_model 640: the head's k items (512 wide at d_model 2048) must divide
+    # d_model, so the head streams 128-wide items here; prefill on the tensor
+    # cores (40 tokens), then greedy decode teacher-forced with the oracle.
+    need_gpu()
+    shape = tl_synth.ModelShape(d_model=640, n_q_heads=10, n_kv_heads=5, head_dim=64,
+                                ffn_dim=1280, vocab=1024, n_pre=1)
+    w = tl_synth.make_model_weights(shape, 640)
+    om = ref.LoopedModel(w)
+    gm = GpuModel(w, max_loops=4, max_ctx=64, max_lanes=1)
+    try:
+        _use(gm, path)
+        L, P, steps = 3, 40, 3
+        prompt = tl_synth.make_tokens(641, shape.vocab, P + 1)
+        o_tokens, o_logits = om.generate_greedy(prompt, L, steps)
+        gm.prefill_lane(0, prompt[:P], L, logits=False)
+        fed = int(prompt[P])
+        for i in range(steps):
+            glg, gam = gm.decode([0], [fed], [L])
+            err = _max_abs(glg[0], o_logits[i])
+            assert err <= LOGIT_MAX_ABS, (i, err)
+            check_argmax(int(gam[0]), o_logits[i], f"step {i}")
+            fed = o_tokens[i]
+    finally:
+        gm.close()
+
+
 def test_tiny_errors(tiny):
     w, om, gm = tiny
     gm.set_path(tl.DECODE_AUTO)

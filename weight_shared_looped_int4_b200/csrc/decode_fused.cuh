@@ -117,7 +117,6 @@ struct FusedArgs {
   // used by the per-layer path; outputs may come from device memory so that a
   // captured graph does not depend on them
   int head_only;
-  int head_early;            // head-only: ring slots issued before the activations are staged (0: all)
   const HeadIO* io;          // if set, logits / argmax pointers are read here
   const int* out_row_dev;    // if set, output slots are read here
 };
@@ -148,7 +147,13 @@ __device__ __forceinline__ int fused_active(const FusedArgs& a, int layer) {
   while (n < a.M && a.n_pre + a.loops[n] > layer) ++n;
   return n;
 }
-__host__ __device__ inline int fused_head_item_k(int d) { return d < 512 ? d : 512; }
+// k columns of a head item: at most 512 and a divisor of d (d is a multiple
+// of 128), so that items never run past a tile's row.
+__host__ __device__ inline int fused_head_item_k(int d) {
+  int k = d < 512 ? d : 512;
+  while (d % k) k -= 128;
+  return k;
+}
 
 // ---- attention key splits -------------------------------------------------
 constexpr int kFusedChunk = 64;
@@ -239,7 +244,7 @@ __device__ __forceinline__ void fused_grid_sync(const FusedArgs& a, unsigned& ta
 
 // ---- producer -----------------------------------------------------------------
 __device__ void fused_producer(const FusedArgs& a, unsigned char* ring, uint64_t* full, uint64_t* empty,
-                               int* s_fail, const int* s_staged) {
+                               int* s_fail) {
   const uint64_t keep = l2_evict_last(), stream = l2_evict_first();
   const int P = gridDim.x, c = blockIdx.x, NS = a.n_slots;
   int item = 0;
@@ -284,15 +289,9 @@ __device__ void fused_producer(const FusedArgs& a, unsigned char* ring, uint64_t
     const size_t tile_bytes = (size_t)(a.d >> 4) * 512;
     const unsigned char* hw = reinterpret_cast<const unsigned char*>(a.head_w);
     for (int tile = tb; tile < te; ++tile)
-      for (int kk = 0; kk < a.d; kk += ki) {
-        if (a.head_only && a.head_early > 0 && item == a.head_early) {
-          // keep the weight stream from queueing ahead of the activation load:
-          // pause until the rows are staged (a pacing hint: on a time-out go on)
-          for (long i = 0; i < kMaxSpin && !*reinterpret_cast<const volatile int*>(s_staged); ++i) __nanosleep(64);
-        }
+      for (int kk = 0; kk < a.d; kk += ki)
         issue(hw + (size_t)tile * tile_bytes + (size_t)(kk >> 4) * 512, (unsigned)(ki >> 4) * 512, nullptr, 0,
               stream);
-      }
   }
   // On a give-up, wait (bounded) for the copies still in flight before the
   // CTA may exit.
@@ -819,7 +818,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
   __shared__ float2 rope_s[kFusedMaxRows * 64];   // (cos, sin) of each row's position, hd <= 128
   __shared__ float s_wv[kFusedMaxRows][kFusedWarps];
   __shared__ int s_wi[kFusedMaxRows][kFusedWarps];
-  __shared__ int s_fail, s_last, s_staged;
+  __shared__ int s_fail, s_last;
   const int NS = a.n_slots;
   unsigned char* ring = smem;
   unsigned char* area = smem + (size_t)NS * kFusedSlotBytes;
@@ -835,12 +834,11 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
     }
     fence_mbar_init();
     s_fail = 0;
-    s_staged = 0;
   }
   __syncthreads();
 
   if (warp == kFusedWarps) {
-    if (lane == 0) fused_producer(a, ring, full, empty, &s_fail, &s_staged);
+    if (lane == 0) fused_producer(a, ring, full, empty, &s_fail);
   } else {
     const int P = gridDim.x, c = blockIdx.x;
     int item = 0;
@@ -908,7 +906,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
     const int d = a.d, M = a.M, ldx = d + 8;
     __half* xl = xs + (size_t)M * ldx;
     fused_stage(a, FS_NORM, a.x, d, a.out_norm, d, M, xs, xl, ssq);
-    if (tid == 0) *reinterpret_cast<volatile int*>(&s_staged) = 1;
     const long long th = 5 * (long long)(target / P);
     if (tid == 0) fused_trace(a, th + 1);
     const int nt = a.V >> 4, tb = (int)((long)c * nt / P), te = (int)((long)(c + 1) * nt / P);

@@ -895,7 +895,6 @@ tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, fl
     // its head tiles through a bulk-copy ring (15 compute warps)
     FusedArgs f = m->fused;
     f.head_only = 1;
-    f.head_early = getenv("TL_HEAD_EARLY") ? atoi(getenv("TL_HEAD_EARLY")) : 0;
     f.M = M;
     f.x = const_cast<float*>(x);
     for (int i = 0; i < M; ++i) f.out_row[i] = i;
