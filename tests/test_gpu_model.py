@@ -191,6 +191,31 @@ def test_width_not_multiple_of_512(path):
         gm.close()
 
 
+def test_width_not_multiple_of_512_five_lanes():
+    # The same width with five lanes in one step: beyond the single-kernel
+    # head's four rows, the standalone head kernel takes the step; its stages
+    # must divide the 640-wide rows too.
+    need_gpu()
+    shape = tl_synth.ModelShape(d_model=640, n_q_heads=10, n_kv_heads=5, head_dim=64,
+                                ffn_dim=1280, vocab=1024, n_pre=1)
+    w = tl_synth.make_model_weights(shape, 640)
+    om = ref.LoopedModel(w)
+    gm = GpuModel(w, max_loops=4, max_ctx=64, max_lanes=5)
+    try:
+        gm.set_path(tl.DECODE_AUTO)
+        prompts = tl_synth.make_lane_prompts(642, shape.vocab, 5, 9)
+        for lane in range(5):
+            gm.prefill_lane(lane, prompts[lane, :8], 2, logits=False)
+        lg, am = gm.decode(list(range(5)), [int(p[8]) for p in prompts], [2] * 5)
+        for lane in range(5):
+            cache, _ = om.prefill(prompts[lane, :8], 2)
+            o = om.decode(cache, int(prompts[lane, 8]), 2)
+            assert _max_abs(lg[lane], o) <= LOGIT_MAX_ABS, lane
+            check_argmax(int(am[lane]), o, f"lane {lane}")
+    finally:
+        gm.close()
+
+
 def test_tiny_errors(tiny):
     w, om, gm = tiny
     gm.set_path(tl.DECODE_AUTO)

@@ -140,9 +140,14 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
 }
 
 // Stage size: 16 KB, or one whole row tile when the tile is smaller.
+// Bytes per stage: at most kHeadStageMax, a divisor of the tile's bytes and a
+// multiple of kHeadWarps k16 blocks (the tile, 32 d bytes, is a multiple of
+// 4096 since d is a multiple of 128).
 __host__ __device__ inline int head_stage_bytes(int d) {
   const int tile = (d / 16) * 512;
-  return tile < kHeadStageMax ? tile : kHeadStageMax;
+  int sb = tile < kHeadStageMax ? tile : kHeadStageMax;
+  while (tile % sb) sb -= 512 * kHeadWarps;
+  return sb;
 }
 __host__ __device__ inline size_t head_act_bytes(int d, int M) { return (size_t)M * (d + 8) * 2 * 2; }
 __host__ __device__ inline int head_stages(int d, int M) {
