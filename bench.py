@@ -57,6 +57,15 @@ BYTES_PER_LAUNCH = {
 }
 
 
+# DRAM bytes (read + write) of one launch of each decode kernel class, from the
+# `ncu --set full` capture summarised in profiles/decode_launches_lm_L8_layered.md
+# (cold cache, first decode step: NCU_KEYS cached keys for the QKV + attention
+# kernel).  Valid for the kernels as captured; the QKV class's cache part is
+# rescaled to the bench's mean context.
+NCU_TRAFFIC = {"qkv": 3683328, "o_proj": 2262528, "gate_up": 12306944, "down": 6176000,
+               "head": 131194368 + 6204160}
+NCU_KEYS = 133
+
 DECODE_PATHS = {"auto": 0, "layered": 1, "fused": 2}
 
 
@@ -567,11 +576,15 @@ def run_ours(args):
             peak = peaks["hbm_gbs"]
             peak_src = peaks["source"] + " HBM copy"
         achieved = dom_b / (avg_us * 1e3) if dom_b else None
+        traffic = NCU_TRAFFIC.get(dom) if attn_in_qkv else None
+        if traffic is not None and dom == "qkv":
+            kv = lambda n: 2 * HKV * HD * 2 * n
+            traffic = traffic - kv(NCU_KEYS) + kv(mean_keys)
         roofline = {
             "kernel": dom, "bound": "hbm", "achieved": round(achieved, 1) if achieved else None,
             "peak": round(peak, 1), "unit": "GB/s",
             "frac": round(achieved / peak, 4) if achieved else None,
-            "traffic": None, "peak_source": peak_src,
+            "traffic": int(traffic) if traffic is not None else None, "peak_source": peak_src,
             "bytes_per_launch": int(dom_b) if dom_b else None,
             "timing": "CUDA events around each launch of one extra decode phase, after the timed region",
         }
