@@ -66,6 +66,18 @@ NCU_TRAFFIC = {"qkv": 3683328, "o_proj": 2262528, "gate_up": 12306944, "down": 6
                "head": 131194368 + 6204160}
 NCU_KEYS = 133
 
+
+
+def roofline_traffic(kernel_class, mean_keys):
+    """ncu DRAM bytes of one launch of a decode kernel class at the bench's
+    mean context (None where no capture covers it)."""
+    traffic = NCU_TRAFFIC.get(kernel_class)
+    if traffic is not None and kernel_class == "qkv":
+        kv = lambda n: 2 * HKV * HD * 2 * n
+        traffic = traffic - kv(NCU_KEYS) + kv(mean_keys)
+    return int(traffic) if traffic is not None else None
+
+
 DECODE_PATHS = {"auto": 0, "layered": 1, "fused": 2}
 
 
@@ -576,15 +588,12 @@ def run_ours(args):
             peak = peaks["hbm_gbs"]
             peak_src = peaks["source"] + " HBM copy"
         achieved = dom_b / (avg_us * 1e3) if dom_b else None
-        traffic = NCU_TRAFFIC.get(dom) if attn_in_qkv else None
-        if traffic is not None and dom == "qkv":
-            kv = lambda n: 2 * HKV * HD * 2 * n
-            traffic = traffic - kv(NCU_KEYS) + kv(mean_keys)
+        traffic = roofline_traffic(dom, mean_keys) if attn_in_qkv else None
         roofline = {
             "kernel": dom, "bound": "hbm", "achieved": round(achieved, 1) if achieved else None,
             "peak": round(peak, 1), "unit": "GB/s",
             "frac": round(achieved / peak, 4) if achieved else None,
-            "traffic": int(traffic) if traffic is not None else None, "peak_source": peak_src,
+            "traffic": traffic, "peak_source": peak_src,
             "bytes_per_launch": int(dom_b) if dom_b else None,
             "timing": "CUDA events around each launch of one extra decode phase, after the timed region",
         }
