@@ -164,6 +164,31 @@ def test_tiny_paths_agree_and_auto(tiny):
         assert _max_abs(lg[lane], om.decode(cache, int(prompts[lane, 8]), 4)) <= LOGIT_MAX_ABS
 
 
+def test_tiny_long_context(path):
+    # A 1100-token context: the clustered decode kernel's key split exceeds
+    # one 64-key chunk (later chunks are loaded inside the kernel), and the
+    # single-kernel step uses its long-context splits with a ticketed merge.
+    need_gpu()
+    w = tl_synth.make_model_weights(tl_synth.TINY_LM, tl_synth.SEED_TINY)
+    om = ref.LoopedModel(w)
+    gm = GpuModel(w, max_loops=2, max_ctx=1104, max_lanes=1)
+    try:
+        _use(gm, path)
+        L, P, steps = 2, 1100, 2
+        prompt = tl_synth.make_tokens(1100, w.shape.vocab, P + 1)
+        o_tokens, o_logits = om.generate_greedy(prompt, L, steps)
+        gm.prefill_lane(0, prompt[:P], L, logits=False)
+        fed = int(prompt[P])
+        for i in range(steps):
+            glg, gam = gm.decode([0], [fed], [L])
+            err = _max_abs(glg[0], o_logits[i])
+            assert err <= LOGIT_MAX_ABS, (i, err)
+            check_argmax(int(gam[0]), o_logits[i], f"step {i}")
+            fed = o_tokens[i]
+    finally:
+        gm.close()
+
+
 def test_width_not_multiple_of_512(path):
     # d_model 640: the head's k items (512 wide at d_model 2048) must divide
     # d_model, so the head streams 128-wide items here; prefill on the tensor
