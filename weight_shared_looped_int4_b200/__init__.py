@@ -302,7 +302,11 @@ def tl_probe_read_bandwidth(buf, nbytes: int, reps: int = 200, stream=None) -> f
 
 
 def tl_model_set_trace(model, buf=None, n_entries: int = 0) -> None:
-    """Phase timeline of fused decode steps into a device uint64 buffer (None = off)."""
+    """Phase timeline of decode steps into a device uint64 buffer (None = off).
+
+    Single-kernel steps stamp per-CTA phase times; per-op steps stamp, per
+    layer launch, maxima over its CTAs (the caller zeroes the buffer before
+    the step) after the head's per-CTA slots.  Layout in include/tl.h."""
     _check(_L().tl_model_set_trace(model, _ptr(buf) if buf is not None else None,
                                    int(n_entries if buf is not None else 0)))
 
