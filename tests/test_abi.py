@@ -69,6 +69,16 @@ def test_null_arguments_rejected_on_host():
     assert e.value.status == tl.TL_ERR_INVALID_ARG
 
 
+def test_model_controls_reject_a_null_model_on_host():
+    for call in (lambda: tl.tl_model_set_trace(None, None, 0),
+                 lambda: tl.tl_model_set_decode_path(None, tl.DECODE_LAYERED),
+                 lambda: tl.tl_model_set_graphs(None, True)):
+        with pytest.raises(tl.TLError) as e:
+            call()
+        assert e.value.status == tl.TL_ERR_INVALID_ARG
+    assert tl.tl_model_trace_grid(None) == 0
+
+
 def test_unsupported_shapes_rejected_on_host():
     x = np.zeros(8, np.uint32)
     lin = type("L", (), {"qweight": x, "scales": x, "qzeros": x})
