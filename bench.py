@@ -57,10 +57,9 @@ BYTES_PER_LAUNCH = {
 }
 
 
-# DRAM bytes (read + write) of one launch of each decode kernel class, from the
-# `ncu --set full` capture summarised in profiles/decode_launches_lm_L8_layered.md
-# (cold cache, first decode step: NCU_KEYS cached keys for the QKV + attention
-# kernel).  Valid for the kernels as captured; the QKV class's cache part is
+# DRAM bytes (read + write) of one launch of each decode kernel class, from an
+# `ncu --set full` capture of `bench.py --ncu-case decode` (cold cache, first
+# decode step: NCU_KEYS cached keys for the QKV + attention kernel).  Valid for the kernels as captured; the QKV class's cache part is
 # rescaled to the bench's mean context.
 NCU_TRAFFIC = {"qkv": 3683328, "o_proj": 2262528, "gate_up": 12306944, "down": 6176000,
                "head": 131194368 + 6204160}
@@ -81,6 +80,14 @@ def roofline_traffic(kernel_class, mean_keys):
 DECODE_PATHS = {"auto": 0, "layered": 1, "fused": 2}
 
 
+def bench_config(world, n_dec, decode_path, graphs):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": WORKLOAD, "global_batch": world, "seq_len": PROMPT + n_dec,
+            "decode_steps": n_dec, "decode_path": decode_path, "cuda_graphs": graphs,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2: each step streams ~333 MB of weights"}
+
+
 def _attn_bytes_per_launch(mean_keys):
     return 2 * HKV * HD * 2 * mean_keys + 2 * HQ * HD * 2
 
@@ -94,6 +101,22 @@ def load_peaks():
                 "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
             "source": "fallback"}
+
+
+def probe_read_bandwidths(tl, torch, dev, st):
+    """Measured read bandwidths: L2 (a buffer of half the L2 size, 200 sweeps
+    in one launch after warm sweeps) and HBM (a 4 GiB buffer, 3 sweeps).
+    Returns (l2_gbs, l2_buffer_bytes, hbm_read_gbs)."""
+    l2_size = torch.cuda.get_device_properties(dev).L2_cache_size
+    nbytes = (l2_size // 2) // (1 << 20) * (1 << 20)
+    buf = torch.ones(nbytes, dtype=torch.uint8, device=dev)
+    l2_gbs = tl.tl_probe_read_bandwidth(buf, nbytes, 200, st)
+    del buf
+    big = torch.ones(4 << 30, dtype=torch.uint8, device=dev)
+    hbm_gbs = tl.tl_probe_read_bandwidth(big, big.numel(), 3, st)
+    del big
+    torch.cuda.empty_cache()
+    return l2_gbs, nbytes, hbm_gbs
 
 
 # ------------------------------------------------------------------ clocks ---
@@ -219,8 +242,7 @@ def run_reference(args):
         "prefill_ms": 1e3 * statistics.mean(pre),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded random weights and token ids)",
-        "config": {"workload": WORKLOAD, "global_batch": 1, "seq_len": PROMPT + STEPS_DECODE,
-                   "parallelism": "cpu oracle, rank 0 only"},
+        "config": bench_config(world, STEPS_DECODE, "auto", True),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -534,13 +556,13 @@ def run_ours(args):
     layer_bytes = sum(BYTES_PER_LAUNCH[k] for k in ("qkv", "o_proj", "gate_up", "down"))
     hbm_bytes = 2 * layer_bytes + BYTES_PER_LAUNCH["head"] + 10 * _attn_bytes_per_launch(mean_keys)
     l2_bytes = LOOPS * layer_bytes
-    probe = torch.empty(24 << 20, dtype=torch.uint8, device=dev)
-    l2_gbs = tl.tl_probe_read_bandwidth(probe, probe.numel(), 2000, st)
-    del probe
+    l2_gbs, l2_probe_bytes, hbm_read_gbs = probe_read_bandwidths(tl, torch, dev, st)
     t_roof_us = hbm_bytes / (peaks["hbm_gbs"] * 1e3) + l2_bytes / (l2_gbs * 1e3)
     t_tok_us = 1e3 * decode_sum / (args.steps * n_dec)
     roof_step = {"hbm_bytes_per_token": int(hbm_bytes), "l2_bytes_per_token": int(l2_bytes),
                  "hbm_gbs": peaks["hbm_gbs"], "l2_read_gbs_measured": round(l2_gbs, 1),
+                 "l2_probe": f"{l2_probe_bytes >> 20} MiB buffer (half the L2), 200 sweeps in one launch",
+                 "hbm_plain_read_gbs_measured": round(hbm_read_gbs, 1),
                  "roofline_us_per_token": round(t_roof_us, 2),
                  "achieved_us_per_token": round(t_tok_us, 2), "frac": round(t_roof_us / t_tok_us, 4)}
 
@@ -610,10 +632,18 @@ def run_ours(args):
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         n_or = 4
-        p_s, d_s, _ = oracle_sample(w, prompt, n_or)
+        p_s, d_s, om = oracle_sample(w, prompt, n_or)
         cpu = {"value": n_or / d_s, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                "sample": f"oracle prefill of the 128-token prompt ({p_s:.2f} s) + {n_or} cached "
                          f"greedy decode steps at L=8 ({d_s:.2f} s), float64 NumPy"}
+        try:   # the same sample on one BLAS thread
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1, user_api="blas"):
+                p1, d1, _ = oracle_sample(w, prompt, n_or, om)
+            cpu["value_1thread"] = n_or / d1
+            cpu["prefill_s_1thread"] = round(p1, 3)
+        except ImportError:
+            pass
 
     tl.tl_model_destroy(m)
     if rank == 0:
@@ -625,11 +655,7 @@ def run_ours(args):
             "decode_ms_per_token": round(decode_sum / (args.steps * n_dec), 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16/fp32 (INT4 weights)",
             "data": "synthetic (seeded random weights and token ids)",
-            "config": {"workload": WORKLOAD, "global_batch": world, "seq_len": PROMPT + n_dec,
-                       "decode_steps": n_dec, "decode_path": args.decode_path,
-                       "cuda_graphs": not args.no_graphs,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": "inputs larger than L2: each step streams ~333 MB of weights"},
+            "config": bench_config(world, n_dec, args.decode_path, not args.no_graphs),
             "roofline": roofline,
             "roofline_decode_token": roof_step,
             "roofline_prefill": roof_prefill,
@@ -646,6 +672,345 @@ def run_ours(args):
         pg.barrier()
         pg.destroy_process_group()
     return 0
+
+
+# ------------------------------------------------------- other workloads ---
+# `--workload tiny|linear|attention|lsweep|peaks` times the kernels on the
+# shapes of the other workloads (one JSON line each, rank 0, one GPU).  The
+# headline line above stays the 400M-LM L=8 step.
+
+def _dev_setup():
+    import torch
+    torch.cuda.set_device(0)
+    return torch, torch.device("cuda", 0), torch.cuda.Stream(device=0)
+
+
+def _l2_flusher(torch, dev):
+    """Writes a buffer twice the L2 size (on the current stream): between
+    timed repetitions, so each starts with a cold L2."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    buf = torch.empty(2 * l2 // 4, dtype=torch.float32, device=dev)
+    return lambda: buf.fill_(1.0)
+
+
+def _time_reps(torch, st, fn, reps, flush=None):
+    """Median ms of `reps` CUDA-event-timed calls of fn() on stream st (flush()
+    runs between them, outside the events)."""
+    out = []
+    with torch.cuda.stream(st):
+        for _ in range(reps):
+            if flush:
+                flush()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            b.synchronize()
+            out.append(a.elapsed_time(b))
+    return statistics.median(out)
+
+
+def tensor_peak_probe(torch, dev):
+    """Dense fp16 and bf16 tensor-core throughput of torch.matmul (cuBLAS) at
+    8192^3, TFLOP/s, 20 timed reps after 5 warm-ups."""
+    n = 8192
+    res = {}
+    for name, dt in (("fp16", torch.float16), ("bf16", torch.bfloat16)):
+        a = torch.randn(n, n, device=dev, dtype=dt)
+        b = torch.randn(n, n, device=dev, dtype=dt)
+        for _ in range(5):
+            torch.matmul(a, b)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(20):
+            torch.matmul(a, b)
+        e1.record()
+        e1.synchronize()
+        res[name] = round(2 * n ** 3 * 20 / (e0.elapsed_time(e1) * 1e9), 1)
+        del a, b
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_workload_peaks(args):
+    torch, dev, st = _dev_setup()
+    import weight_shared_looped_int4_b200 as tl
+    with ClockSampler(0) as clocks:
+        tc = tensor_peak_probe(torch, dev)
+        l2, l2_bytes, hbm = probe_read_bandwidths(tl, torch, dev, st)
+    print(json.dumps({"workload": "peaks", "tensor_tflops_torch_matmul_8192": tc,
+                      "l2_read_gbs": round(l2, 1), "l2_probe_bytes": l2_bytes,
+                      "hbm_plain_read_gbs": round(hbm, 1), "measured_peaks_file": load_peaks(),
+                      "clocks": clocks.summary()}))
+    return 0
+
+
+def run_workload_linear(args):
+    """INT4 group-128 linear sweep: M in {1,4,16,128} x the four (K, N), the
+    library's default path per M, L2-cold (flushed) and L2-warm; torch fp16
+    matmul on the dequantized weight as the comparator (context only)."""
+    torch, dev, st = _dev_setup()
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    peaks = load_peaks()
+    flush = _l2_flusher(torch, dev)
+    rows = []
+    launches0 = tl.tl_kernel_launch_count()
+    with ClockSampler(0) as clocks:
+        tc_peak = tensor_peak_probe(torch, dev)
+        for K, N in tl_synth.LINEAR_SWEEP_KN:
+            rng = np.random.default_rng(tl_synth.SEED_LINEAR + K + N)
+            lin = tl_synth.make_int4_linear(rng, N, K)
+            h = tl.tl_linear_create(lin, K, N, 0)
+            # fp16 comparator: the same weights dequantized on the device by torch
+            q = torch.from_numpy(lin.qweight.view(np.int32)).to(dev)
+            nib = torch.stack([(q >> (4 * j)) & 15 for j in range(8)], dim=-1).reshape(N, -1)[:, :K]
+            zw = torch.from_numpy(lin.qzeros.view(np.int32)).to(dev)
+            z = torch.stack([(zw >> (4 * j)) & 15 for j in range(8)], dim=-1).reshape(N, -1)[:, :K // 128]
+            sc = torch.from_numpy(lin.scales.view(np.float16)).to(dev).float()
+            w16 = ((nib.view(N, K // 128, 128) - z[:, :, None]).float() * sc[:, :, None]).reshape(N, K).half()
+            del q, nib, zw, z, sc
+            for M in tl_synth.LINEAR_SWEEP_M:
+                x = torch.from_numpy(tl_synth.make_activations(tl_synth.SEED_LINEAR * 7 + M, M, K)).to(dev)
+                y = torch.empty((M, N), dtype=torch.float16, device=dev)
+                fn = lambda: tl.tl_linear_forward(h, x, M, y, tl.TL_PATH_AUTO, st)
+                for _ in range(5):
+                    fn()
+                cold = _time_reps(torch, st, fn, 30, flush)
+                warm = _time_reps(torch, st, fn, 50)
+                tfn = lambda: torch.matmul(x, w16.t())
+                for _ in range(3):
+                    with torch.cuda.stream(st):
+                        tfn()
+                t_cold = _time_reps(torch, st, tfn, 20, flush)
+                nbytes = _int4_bytes(K, N) + 2 * M * K + 2 * M * N
+                flops = 2 * M * K * N
+                t_hbm = nbytes / (peaks["hbm_gbs"] * 1e3)          # us
+                t_tc = flops / (peaks["bf16_tflops"] * 1e6)         # us
+                bound = "hbm" if t_hbm >= t_tc else "tensor"
+                t_roof = max(t_hbm, t_tc)
+                rows.append({"M": M, "K": K, "N": N, "path": "gemv" if M <= 16 else "tcgen05",
+                             "us_l2_cold": round(1e3 * cold, 2), "us_l2_warm": round(1e3 * warm, 2),
+                             "bytes": nbytes, "flops": flops, "bound": bound,
+                             "achieved_cold": round(nbytes / (cold * 1e6), 1) if bound == "hbm"
+                             else round(flops / (cold * 1e9), 1),
+                             "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+                             "roofline_us": round(t_roof, 3),
+                             "frac_cold": round(t_roof / (1e3 * cold), 4),
+                             "frac_warm": round(t_roof / (1e3 * warm), 4),
+                             "torch_fp16_dequantized_us_l2_cold": round(1e3 * t_cold, 2)})
+            tl.tl_linear_destroy(h)
+            del w16
+    print(json.dumps({"workload": "INT4 g128 linear sweep (fp16 x, fp32 acc, fp16 y)",
+                      "metric": "per-shape us and fraction of roofline", "peaks": peaks,
+                      "tensor_tflops_torch_matmul_8192": tc_peak,
+                      "timing": "median of 30 (cold: 2xL2 buffer written between reps) / 50 (warm) CUDA-event reps",
+                      "results": rows, "gpu_launches": tl.tl_kernel_launch_count() - launches0,
+                      "clocks": clocks.summary()}))
+    return 0
+
+
+def run_workload_attention(args):
+    """GQA attention, D 2048, 16 Q / 4 KV heads of 128: single-query decode
+    over S in {128,1024,4096,8192} and causal prefill at T in {128,512,2048},
+    batch 1 and 8; fp16 N(0,1) inputs; RoPE by the in-place op (timed apart)."""
+    torch, dev, st = _dev_setup()
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    peaks = load_peaks()
+    flush = _l2_flusher(torch, dev)
+    dec, pre = [], []
+    launches0 = tl.tl_kernel_launch_count()
+    with ClockSampler(0) as clocks:
+        for B in (1, 8):
+            for S in (128, 1024, 4096, 8192):
+                q, k, v = tl_synth.make_qkv(tl_synth.SEED_ATTN + S + B, B, S, HQ, HKV, HD, T_q=1)
+                kc = torch.from_numpy(np.ascontiguousarray(k.transpose(0, 2, 1, 3))).to(dev)
+                vc = torch.from_numpy(np.ascontiguousarray(v.transpose(0, 2, 1, 3))).to(dev)
+                qd = torch.from_numpy(np.ascontiguousarray(q[:, 0])).to(dev)
+                out = torch.empty((B, HQ, HD), dtype=torch.float16, device=dev)
+                pos = torch.full((B,), S - 1, dtype=torch.int32, device=dev)
+                fn = lambda: tl.tl_op_gqa_decode(qd, kc, vc, HKV * S * HD, S, [S] * B, B, HQ, HKV, HD, out, st)
+                rope = lambda: tl.tl_op_rope(qd, B, HQ, HD, HQ * HD, HD, pos, 1e4, st)
+                for _ in range(5):
+                    fn()
+                cold = _time_reps(torch, st, fn, 30, flush)
+                warm = _time_reps(torch, st, fn, 50)
+                t_rope = _time_reps(torch, st, rope, 20)
+                nbytes = B * (2 * HKV * S * HD * 2 + 2 * HQ * HD * 2)
+                t_roof = nbytes / (peaks["hbm_gbs"] * 1e3)
+                dec.append({"B": B, "S": S, "us_l2_cold": round(1e3 * cold, 2), "us_l2_warm": round(1e3 * warm, 2),
+                            "bytes": nbytes, "gbs_cold": round(nbytes / (cold * 1e6), 1),
+                            "frac_cold": round(t_roof / (1e3 * cold), 4), "rope_q_us": round(1e3 * t_rope, 2)})
+                del kc, vc
+        for B in (1, 8):
+            for T in (128, 512, 2048):
+                q, k, v = tl_synth.make_qkv(tl_synth.SEED_ATTN + 7 * T + B, B, T, HQ, HKV, HD)
+                kc = torch.from_numpy(np.ascontiguousarray(k.transpose(0, 2, 1, 3))).to(dev)
+                vc = torch.from_numpy(np.ascontiguousarray(v.transpose(0, 2, 1, 3))).to(dev)
+                qd = torch.from_numpy(np.ascontiguousarray(q)).to(dev)
+                out = torch.empty((B, T, HQ, HD), dtype=torch.float16, device=dev)
+                fn = lambda: tl.tl_op_gqa_prefill(qd, kc, vc, HKV * T * HD, T, T, 0, B, HQ, HKV, HD, out, st)
+                for _ in range(3):
+                    fn()
+                cold = _time_reps(torch, st, fn, 20, flush)
+                flops = B * 4 * HQ * HD * T * (T + 1) / 2
+                t_roof = flops / (peaks["bf16_tflops"] * 1e6)
+                pre.append({"B": B, "T": T, "us_l2_cold": round(1e3 * cold, 2), "flops": int(flops),
+                            "tflops": round(flops / (cold * 1e9), 2), "frac": round(t_roof / (1e3 * cold), 4)})
+                del kc, vc, qd, out
+    print(json.dumps({"workload": "GQA attention D2048 16q/4kv hd128 (fp16 KV)",
+                      "metric": "per-case us and fraction of roofline", "peaks": peaks,
+                      "decode": dec, "prefill": pre,
+                      "context_h100_from_pages": {"decode_K128_D2048_16heads_ms": 0.092,
+                                                  "prefill_T128_ms": [0.143, 0.087]},
+                      "timing": "median of CUDA-event reps; decode cold = 2xL2 buffer written between reps",
+                      "gpu_launches": tl.tl_kernel_launch_count() - launches0,
+                      "clocks": clocks.summary()}))
+    return 0
+
+
+def _lm_model(tl, tl_synth, max_loops, max_ctx, max_lanes):
+    shape = tl_synth.LOOPED_LM
+    w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM)
+    cfg = tl.make_config(shape, max_loops=max_loops, max_ctx=max_ctx, max_lanes=max_lanes)
+    tw, keep = tl.make_weights(w)
+    m = tl.tl_model_create(cfg, tw, 0)
+    del keep
+    return w, m
+
+
+def _decode_roofline_us(n_rows_kv, loops_list, l2_gbs, peaks):
+    """Byte roofline of one decode step (us): pre blocks + head + KV reads
+    from HBM, the loop block once per iteration of the longest lane from L2."""
+    layer = sum(BYTES_PER_LAUNCH[k] for k in ("qkv", "o_proj", "gate_up", "down"))
+    hbm = 2 * layer + BYTES_PER_LAUNCH["head"] + n_rows_kv
+    l2 = max(loops_list) * layer
+    return hbm / (peaks["hbm_gbs"] * 1e3) + l2 / (l2_gbs * 1e3), hbm, l2
+
+
+def run_workload_lsweep(args):
+    """The 400M LM swept over loops L in {1,2,4,8,16}: prefill of a 512-token
+    prompt (no logits) and 256 greedy decode steps at batch 1; then 1/4/16
+    lanes with per-lane loops drawn from {4,8,16}, 512-token prompts each,
+    256 decode steps (max context 2048)."""
+    torch, dev, st = _dev_setup()
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    peaks = load_peaks()
+    P, n_dec = 512, args.decode_steps if args.decode_steps != STEPS_DECODE else 256
+    w, m = _lm_model(tl, tl_synth, 16, 2048, 16)
+    l2_gbs, _, _ = probe_read_bandwidths(tl, torch, dev, st)
+    prompts = tl_synth.make_lane_prompts(tl_synth.SEED_LSWEEP, w.shape.vocab, 16, P + 1)
+    d_prompts = torch.as_tensor(prompts, device=dev)
+    hist = torch.zeros((n_dec + 1, 16), dtype=torch.int32, device=dev)
+    hp = hist.data_ptr()
+    per_layer_flops = 2 * P * (D * (HQ + 2 * HKV) * HD + HQ * HD * D + D * 2 * F + F * D)
+    attn_flops = 4 * HQ * HD * P * (P + 1) / 2
+    sweep, lanes_res = [], []
+    launches0 = tl.tl_kernel_launch_count()
+
+    def decode_run(lanes, loops):
+        n = len(lanes)
+        for i, lane in enumerate(lanes):
+            tl.tl_prefill(m, lane, d_prompts[lane], P, loops[i], None, None, st)
+        with torch.cuda.stream(st):
+            hist[0, :n].copy_(d_prompts[:n, P])
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for i in range(n_dec):
+            tl.tl_decode_step(m, lanes, hp + 64 * i, loops, None, hp + 64 * (i + 1), st)
+        b.record(st)
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    with ClockSampler(0) as clocks:
+        for L in (1, 2, 4, 8, 16):
+            fn = lambda: tl.tl_prefill(m, 0, d_prompts[0], P, L, None, None, st)
+            for _ in range(3):
+                fn()
+            pf = _time_reps(torch, st, fn, 10)
+            flops = (2 + L) * (per_layer_flops + attn_flops)
+            decode_run([0], [L])          # warm (graph capture)
+            ms = decode_run([0], [L])
+            kv = (2 + L) * 2 * HKV * HD * 2 * (P + n_dec / 2)
+            t_roof, _, _ = _decode_roofline_us(kv, [L], l2_gbs, peaks)
+            us_tok = 1e3 * ms / n_dec
+            sweep.append({"L": L, "prefill_T512_ms": round(pf, 4), "prefill_flops": int(flops),
+                          "prefill_tflops": round(flops / (pf * 1e9), 2),
+                          "prefill_frac": round(flops / (pf * 1e9) / peaks["bf16_tflops"], 4),
+                          "decode_tok_s": round(n_dec / (ms / 1e3), 1), "decode_us_per_step": round(us_tok, 2),
+                          "decode_roofline_us": round(t_roof, 2), "decode_frac": round(t_roof / us_tok, 4)})
+        for n in (1, 4, 16):
+            loops = [int(v) for v in tl_synth.make_lane_loops(tl_synth.SEED_LSWEEP, n)]
+            lanes = list(range(n))
+            decode_run(lanes, loops)      # warm (graph capture)
+            ms = decode_run(lanes, loops)
+            kv = sum((2 + L) * 2 * HKV * HD * 2 * (P + n_dec / 2) for L in loops)
+            t_roof, _, _ = _decode_roofline_us(kv, loops, l2_gbs, peaks)
+            us_step = 1e3 * ms / n_dec
+            lanes_res.append({"lanes": n, "loops": loops, "decode_tok_s": round(n * n_dec / (ms / 1e3), 1),
+                              "us_per_step": round(us_step, 2), "roofline_us_per_step": round(t_roof, 2),
+                              "frac": round(t_roof / us_step, 4)})
+    tl.tl_check_device_error(m)
+    tl.tl_model_destroy(m)
+    print(json.dumps({"workload": "400M looped LM, L sweep and per-lane loops (prompts 512, ctx 2048)",
+                      "metric": "prefill ms (T=512) and decode tok/s per L; decode tok/s per lane count",
+                      "decode_steps": n_dec, "peaks": peaks, "l2_read_gbs": round(l2_gbs, 1),
+                      "loops_sweep": sweep, "lanes": lanes_res,
+                      "gpu_launches": tl.tl_kernel_launch_count() - launches0,
+                      "clocks": clocks.summary()}))
+    return 0
+
+
+def run_workload_tiny(args):
+    """Tiny looped LM (d 256, 4/2 heads of 64, F 1024, V 512, 1 pre block,
+    L = 4): 32-token prompt prefill, then 8 greedy decode steps, batch 1."""
+    torch, dev, st = _dev_setup()
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    shape = tl_synth.TINY_LM
+    w = tl_synth.make_model_weights(shape, tl_synth.SEED_TINY)
+    cfg = tl.make_config(shape, max_loops=4, max_ctx=64, max_lanes=1)
+    tw, keep = tl.make_weights(w)
+    m = tl.tl_model_create(cfg, tw, 0)
+    del keep
+    P, L, n_dec = 32, 4, 8
+    prompt = tl_synth.make_tokens(tl_synth.SEED_TINY, shape.vocab, P + 1)
+    d_prompt = torch.as_tensor(prompt, device=dev)
+    hist = torch.zeros(n_dec + 1, dtype=torch.int32, device=dev)
+    hp = hist.data_ptr()
+    pre_ms, dec_ms = [], []
+    with ClockSampler(0) as clocks:
+        for it in range(args.warmup + args.steps):
+            a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            with torch.cuda.stream(st):
+                a.record(st)
+                tl.tl_prefill(m, 0, d_prompt, P, L, None, None, st)
+                b.record(st)
+                hist[0:1].copy_(d_prompt[P:P + 1])
+                for i in range(n_dec):
+                    tl.tl_decode_step(m, [0], hp + 4 * i, [L], None, hp + 4 * (i + 1), st)
+                c.record(st)
+            c.synchronize()
+            if it >= args.warmup:
+                pre_ms.append(a.elapsed_time(b))
+                dec_ms.append(b.elapsed_time(c))
+    tl.tl_model_destroy(m)
+    print(json.dumps({"workload": "tiny looped LM d256 4q/2kv hd64 F1024 V512 n_pre1 L4; prompt 32 + 8 greedy steps",
+                      "prefill_ms": round(statistics.median(pre_ms), 4),
+                      "decode_tok_s": round(n_dec / (statistics.median(dec_ms) / 1e3), 1),
+                      "decode_us_per_token": round(1e3 * statistics.median(dec_ms) / n_dec, 2),
+                      "roofline": None,
+                      "note": "0.51 MB per block pass: launch/latency bound, no roofline claim",
+                      "clocks": clocks.summary()}))
+    return 0
+
+
+WORKLOADS = {"tiny": run_workload_tiny, "linear": run_workload_linear,
+             "attention": run_workload_attention, "lsweep": run_workload_lsweep,
+             "peaks": run_workload_peaks}
 
 
 def main():
@@ -666,6 +1031,9 @@ def main():
     ap.add_argument("--no-profile", action="store_true")
     ap.add_argument("--trace", action="store_true",
                     help="print the phase timeline of one single-kernel decode step and exit")
+    ap.add_argument("--workload", choices=["lm"] + sorted(WORKLOADS), default="lm",
+                    help="lm (default): the 400M-LM L=8 step; others time the kernels on the "
+                         "shapes of the other workloads and print their own JSON line")
     ap.add_argument("--ncu-case", choices=["none", "decode", "prefill"], default="none",
                     help="run a small eager case for kernel profilers and exit")
     args = ap.parse_args()
@@ -677,6 +1045,8 @@ def main():
         return run_ncu_case(args)
     if args.trace:
         return run_trace(args)
+    if args.workload != "lm":
+        return WORKLOADS[args.workload](args)
     return run_ours(args)
 
 

@@ -160,12 +160,91 @@ tl_status tl_decode_step(tl_model *m, int n_lanes, const int32_t *h_lane_ids,
                          const int32_t *d_tokens, const int32_t *h_loops,
                          float *d_logits, int32_t *d_argmax, void *stream);
 
+/* Append n_tokens tokens to a prefilled lane: positions length(lane) ..
+ * length(lane) + n_tokens - 1 through the lane's n_pre + loops layers,
+ * attending to everything the lane holds (a chunk of a longer prompt --
+ * TinyLoop docs, "Async API", "Constructor": prefill_chunk -- or the verify
+ * pass of speculative decoding).  The lane's length grows by n_tokens.
+ *   d_tokens  int32 [n_tokens]
+ *   d_logits  fp32 [n_tokens][vocab] logits of EVERY appended position, or NULL
+ *   d_argmax  int32 [n_tokens] greedy token of every position, or NULL
+ * Per-position outputs need n_tokens <= 16 (else TL_ERR_UNSUPPORTED);
+ * TL_ERR_NOT_PREFILLED for an empty lane, TL_ERR_CONTEXT_FULL past max_ctx. */
+tl_status tl_extend(tl_model *m, int lane, const int32_t *d_tokens, int n_tokens, float *d_logits,
+                    int32_t *d_argmax, void *stream);
+
+/* Counters of one tl_generate_speculative call. */
+typedef struct {
+  int rounds;    /* draft + verify rounds */
+  int drafted;   /* draft tokens proposed */
+  int accepted;  /* draft tokens the verifier agreed with */
+} tl_spec_stats;
+
+/* Greedy self-speculative generation on a prefilled lane (TinyLoop docs,
+ * "Async API", "Speculative decode": draft_loops, verify_loops, draft_ahead;
+ * TinyLoop README, "Why TinyLoop Exists", item 3: draft and verify reuse the
+ * same weights; "Quick CLI Tour", Speculate).  The verifier runs the lane's
+ * prefill loops; the draft model is the same network cut after draft_loops
+ * loop iterations, so its keys and values are the verifier's first slices.
+ * Each round: k = min(draft_ahead, tokens still to produce) cached greedy
+ * draft steps with draft_loops from the next input token, then one pass of
+ * those k inputs through all the lane's loops (tl_extend's computation)
+ * giving the verifier's greedy token at each; drafts are accepted while they
+ * equal the verifier's tokens, the verifier's token replaces the first
+ * rejected draft, and the lane's length is rolled back to the accepted
+ * positions.  The output therefore equals max_tokens plain greedy decode
+ * steps at the lane's loops (up to rounding at near-ties).
+ *   d_first_token  int32 [1] the token fed at position length(lane), as for
+ *                  tl_decode_step
+ *   max_tokens     tokens to produce (>= 1, length(lane) + max_tokens <= max_ctx)
+ *   draft_loops    1 <= draft_loops <= the lane's loops
+ *   draft_ahead    1 <= draft_ahead <= 16
+ *   d_out_tokens   int32 [max_tokens] the generated tokens
+ *   h_stats        HOST, or NULL
+ * On return the lane holds length + max_tokens positions, as after
+ * max_tokens decode steps.  Synchronises `stream` once per round (the
+ * accepted count decides the next round on the host). */
+tl_status tl_generate_speculative(tl_model *m, int lane, const int32_t *d_first_token, int max_tokens,
+                                  int draft_loops, int draft_ahead, int32_t *d_out_tokens,
+                                  tl_spec_stats *h_stats, void *stream);
+
 /* Stateless uncached forward (TinyLoop docs, "Async API", "Scoring",
  * score_last): logits [vocab] of the last of n_tokens tokens.  Touches no
  * lane (it uses a private scratch slice).  d_logits must not be NULL;
  * d_argmax may be NULL. */
 tl_status tl_score_last(tl_model *m, const int32_t *d_tokens, int n_tokens, int loops,
                         float *d_logits, int32_t *d_argmax, void *stream);
+
+/* Logit lens (TinyLoop docs, "Async API", "Scoring", score_logit_lens:
+ * [loops, vocab]): a stateless uncached forward like tl_score_last that
+ * applies the output norm and head to the last position after EVERY loop
+ * iteration.  Row i of d_logits (fp32 [loops][vocab]) holds the logits after
+ * iteration i + 1, which equal tl_score_last with loops = i + 1; d_argmax
+ * (int32 [loops], or NULL) their greedy tokens. */
+tl_status tl_score_logit_lens(tl_model *m, const int32_t *d_tokens, int n_tokens, int loops,
+                              float *d_logits, int32_t *d_argmax, void *stream);
+
+/* Token-stable early exit (TinyLoop README, "Runtime Flags",
+ * TINYLOOP_TOKEN_EXIT=N): a stateless uncached forward of the last position
+ * that stops iterating the loop block once the greedy token after the last
+ * stable_n iterations has been the same, or after max_loops iterations.
+ * d_logits fp32 [vocab] (and d_argmax int32 [1], or NULL) receive the
+ * logits of the exit iteration, which equal tl_score_last with that many
+ * loops; *h_loops_used (HOST) the iterations run.  Synchronises `stream`
+ * after every iteration. */
+tl_status tl_score_early_exit(tl_model *m, const int32_t *d_tokens, int n_tokens, int max_loops,
+                              int stable_n, float *d_logits, int32_t *d_argmax, int *h_loops_used,
+                              void *stream);
+
+/* Prefix cache (TinyLoop README, "Python Quick Start": build_prefix_cache /
+ * generate_from_prefix_cache; "Python API reference", Prefix cache): copy
+ * the keys and values of positions 0 .. n_tokens - 1 of every slice of
+ * src_lane (n_pre + its loops layers) into dst_lane, which then holds
+ * n_tokens positions with src_lane's loops, as if it had been prefilled with
+ * the same first n_tokens tokens.  A lane prefilled with a shared prompt is
+ * the prefix cache; forks continue from it without recomputing it.
+ * 1 <= n_tokens <= length(src_lane); the lanes differ. */
+tl_status tl_lane_fork(tl_model *m, int src_lane, int dst_lane, int n_tokens, void *stream);
 
 /* Tokens currently held by a lane (0 if never prefilled). */
 tl_status tl_lane_length(const tl_model *m, int lane, int *h_length);
@@ -266,6 +345,18 @@ tl_status tl_model_set_decode_path(tl_model *m, int path);
 tl_status tl_model_set_trace(tl_model *m, unsigned long long *d_buf, long long n_entries);
 int tl_model_trace_grid(const tl_model *m);
 
+/* Test hook with no counterpart in the pages: exercises the bounded waits.
+ * With extra_arrivals = 1, every grid barrier of the following
+ * TL_DECODE_FUSED steps waits for one CTA more than the step launches, so
+ * the first barrier's wait runs out after its time limit (0.5 s of
+ * %globaltimer), the CTA that gives up tells the others to stop waiting, the
+ * step finishes with invalid results and tl_check_device_error() returns
+ * TL_ERR_DEVICE_FLAG ("a kernel's bounded wait gave up").  The barrier words
+ * are reset at the end of the launch as usual, so after
+ * tl_model_set_wait_test(m, 0) the next steps are correct again (re-prefill
+ * the lanes whose caches the invalid step wrote).  Other paths ignore it. */
+tl_status tl_model_set_wait_test(tl_model *m, int extra_arrivals);
+
 /* Number of kernels this library has launched in the process so far. */
 unsigned long long tl_kernel_launch_count(void);
 
@@ -327,19 +418,22 @@ tl_status tl_op_gqa_decode(const uint16_t *d_q, const uint16_t *d_k, const uint1
 
 /* tl_op_gqa_decode without any allocation.  The pages have no counterpart to
  * this entry point; it exists for callers that cannot call cudaMalloc, such as
- * code running inside a stream capture that must not allocate, or a serving
- * host that plans every device byte up front and owns the allocator.
+ * a serving host that plans every device byte up front and owns the
+ * allocator, or a plug-in running inside another runtime whose allocator owns
+ * the device memory.
  * Same arguments, layout and result as tl_op_gqa_decode, but its scratch (row
  * descriptors, split-KV partial results and merge tickets) lives in one
  * fixed 4 MiB device array that every GPU loading this library reserves until
  * the process exits; nothing is allocated or freed by the call.
  *   Limits: 1 <= B <= 32, B * n_kv_heads <= 4096, and
  *   B * n_kv_heads * 32 * (n_q_heads/n_kv_heads) * (head_dim + 4) * 4 bytes
- *   + 17 KiB <= 4 MiB (e.g. B = 8, 16/4 heads of 128 needs about 2.2 MiB);
+ *   + 17 KiB <= 4 MiB (e.g. B = 8, 16/4 heads of 128 needs about 2.1 MiB);
  *   beyond them it returns TL_ERR_UNSUPPORTED and enqueues nothing.
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  All calls share the one array and it
+ * (cudaGetSymbolAddress, with that device current) and caches it for the
+ * life of the process (a cudaDeviceReset makes the cached address stale; do
+ * not call this entry point on a device after resetting it); make that first
+ * call before any stream capture.  All calls share the one array and it
  * keeps the last call's contents (each call re-zeroes what must start at
  * zero), so calls whose work overlaps on the GPU (different streams without
  * ordering between them) race and corrupt each other's results: order them on
@@ -375,13 +469,14 @@ const char *tl_last_error(void);
 const char *tl_version(void);
 
 /* Measurement helper with no counterpart in the pages: read bandwidth of a
- * device buffer.  Streams the `bytes` (a multiple of 16, >= 16) of d_buf with
- * 16-byte loads that skip L1 (one CTA per SM x 4, 512 threads, 4 loads in
- * flight per thread), `reps` times (1..100000) after 3 untimed passes, on
- * `stream`, timed with CUDA events; writes GB/s (bytes x reps / time) to
- * *h_gbs and synchronises the stream.  A buffer well under the L2 size (e.g.
- * the 24 MB loop block) measures L2 read bandwidth, one well over it HBM.
- * The buffer is only read. */
+ * device buffer.  One launch (one CTA per SM x 4, 512 threads, 8 independent
+ * 16-byte loads in flight per thread, loads that skip L1) sweeps the `bytes`
+ * (a multiple of 16, >= 16) of d_buf `reps` times (1..100000), after one
+ * untimed launch of 3 sweeps, on `stream`; it is timed with CUDA events and
+ * *h_gbs = bytes x reps / time in GB/s; the stream is synchronised.  Because
+ * the sweeps repeat inside one launch, launch overhead does not count.  A
+ * buffer of about half the L2 size measures L2 read bandwidth, one well over
+ * it HBM read bandwidth.  The buffer is only read. */
 tl_status tl_probe_read_bandwidth(const void *d_buf, size_t bytes, int reps, void *stream,
                                   double *h_gbs);
 

@@ -29,7 +29,14 @@ What it computes, step by step, in the order the pages give it:
   uncached recompute (TinyLoop README, "Current Runtime Snapshot" quality notes
   and "Quick CLI Tour", Generate);
 * greedy decoding = argmax, lowest index on ties (TinyLoop docs, "Async API",
-  "Generation", temperature 0).
+  "Generation", temperature 0);
+* around that pass: the logit lens (the head after every loop iteration;
+  TinyLoop docs, "Async API", "Scoring", score_logit_lens), token-stable early
+  exit (TinyLoop README, "Runtime Flags", TINYLOOP_TOKEN_EXIT), greedy
+  self-speculative decoding with a draft that runs fewer loops of the same
+  block (TinyLoop docs, "Async API", "Speculative decode"; TinyLoop README,
+  "Why TinyLoop Exists", item 3) and forking a cached prefix (TinyLoop README,
+  "Python Quick Start", build_prefix_cache / generate_from_prefix_cache).
 
 Readings taken where the pages are silent (each is listed with its reason in
 the design notes): Llama-style pre-norm block with no Q/K norm; iteration i+1
@@ -230,6 +237,18 @@ class KVCache:
     def length(self) -> int:
         return 0 if self.k[0] is None else self.k[0].shape[0]
 
+    def fork(self, n: int) -> "KVCache":
+        """A new cache holding copies of this one's first ``n`` positions in
+        every slice (the prefix cache: TinyLoop README, "Python Quick Start",
+        build_prefix_cache / generate_from_prefix_cache)."""
+        if not 1 <= n <= self.length:
+            raise ValueError("fork length out of range")
+        out = KVCache(len(self.k))
+        for layer in range(len(self.k)):
+            out.k[layer] = self.k[layer][:n].copy()
+            out.v[layer] = self.v[layer][:n].copy()
+        return out
+
     def append(self, layer: int, k: np.ndarray, v: np.ndarray):
         if self.k[layer] is None:
             self.k[layer], self.v[layer] = k, v
@@ -314,6 +333,75 @@ class LoopedModel:
     def score_last(self, tokens, loops: int) -> np.ndarray:
         """Logits [V] of the last position, no cache (a stateless forward)."""
         return self.logits(self.forward(tokens, loops)[-1])
+
+    def score_logit_lens(self, tokens, loops: int) -> np.ndarray:
+        """Logit lens [loops][V] (TinyLoop docs, "Async API", "Scoring",
+        score_logit_lens): output norm + head of the last position after each
+        loop iteration, no cache."""
+        tokens = np.asarray(tokens, dtype=np.int64)
+        positions = np.arange(tokens.shape[0])
+        x = self.embed[tokens]
+        for layer, blk in enumerate(self.pre):
+            x = self.block(blk, x, positions, None, layer)
+        rows = []
+        for i in range(loops):
+            x = self.block(self.loop, x, positions, None, self.shape.n_pre + i)
+            rows.append(self.logits(x[-1]))
+        return np.asarray(rows)
+
+    def score_early_exit(self, tokens, max_loops: int, stable_n: int):
+        """Token-stable early exit (TinyLoop README, "Runtime Flags",
+        TINYLOOP_TOKEN_EXIT=N): iterate the loop block on the last position's
+        stream until the greedy token of the last ``stable_n`` iterations is
+        the same (or ``max_loops`` iterations ran).  Returns (logits of the
+        exit iteration, iterations run)."""
+        if stable_n < 1:
+            raise ValueError("stable_n must be >= 1")
+        tokens = np.asarray(tokens, dtype=np.int64)
+        positions = np.arange(tokens.shape[0])
+        x = self.embed[tokens]
+        for layer, blk in enumerate(self.pre):
+            x = self.block(blk, x, positions, None, layer)
+        history = []
+        for i in range(max_loops):
+            x = self.block(self.loop, x, positions, None, self.shape.n_pre + i)
+            logits = self.logits(x[-1])
+            history.append(greedy(logits))
+            if len(history) >= stable_n and len(set(history[-stable_n:])) == 1:
+                break
+        return logits, len(history)
+
+    def generate_speculative(self, prompt, draft_loops: int, verify_loops: int, draft_ahead: int,
+                             max_tokens: int):
+        """Greedy self-speculative decoding (TinyLoop docs, "Async API",
+        "Speculative decode"; TinyLoop README, "Why TinyLoop Exists" item 3):
+        the draft model is the same network run with ``draft_loops``
+        iterations.  Each round drafts k = min(draft_ahead, tokens left)
+        tokens greedily, then the ``verify_loops`` model scores the sequence
+        extended by the drafts; drafts are kept while they equal the
+        verifier's greedy tokens and the verifier's token replaces the first
+        rejected one.  Written without a cache (the cache changes no value).
+        Returns (tokens, {"rounds", "drafted", "accepted"})."""
+        seq = [int(t) for t in prompt]
+        out = []
+        stats = {"rounds": 0, "drafted": 0, "accepted": 0}
+        while len(out) < max_tokens:
+            k = min(draft_ahead, max_tokens - len(out))
+            drafts = []
+            for _ in range(k):
+                drafts.append(greedy(self.score_last(seq + drafts, draft_loops)))
+            h = self.forward(seq + drafts[:k - 1], verify_loops)
+            ver = [greedy(self.logits(h[len(seq) - 1 + i])) for i in range(k)]
+            acc = 0
+            while acc < k and drafts[acc] == ver[acc]:
+                acc += 1
+            emit = min(acc + 1, k)
+            out += ver[:emit]
+            seq += ver[:emit]
+            stats["rounds"] += 1
+            stats["drafted"] += k
+            stats["accepted"] += acc
+        return out, stats
 
     def new_cache(self, loops: int) -> KVCache:
         return KVCache(self.shape.n_pre + loops)

@@ -266,6 +266,40 @@ def test_tiny_errors(tiny):
     tl.tl_check_device_error(gm.handle)   # cleared
 
 
+def test_tiny_bounded_wait_times_out(tiny):
+    # A grid barrier made to expect one CTA more than the step launches: its
+    # bounded wait (0.5 s) runs out, the step ends instead of hanging, the
+    # device flag reports it, and the next steps on the same model are
+    # correct again.
+    import time
+    w, om, gm = tiny
+    gm.set_path(tl.DECODE_FUSED)
+    prompt = tl_synth.make_tokens(77, w.shape.vocab, 12)
+    tl.tl_check_device_error(gm.handle)
+    gm.prefill_lane(9, prompt[:10], 2, logits=False)
+    tl.tl_model_set_wait_test(gm.handle, 1)
+    try:
+        t0 = time.perf_counter()
+        gm.decode([9], [int(prompt[10])], [2])
+        waited = time.perf_counter() - t0
+    finally:
+        tl.tl_model_set_wait_test(gm.handle, 0)
+    assert 0.3 < waited < 30.0, waited
+    with pytest.raises(tl.TLError) as e:
+        tl.tl_check_device_error(gm.handle)
+    assert e.value.status == tl.TL_ERR_DEVICE_FLAG
+    assert "wait" in str(e.value)
+    tl.tl_check_device_error(gm.handle)   # cleared
+    gm.prefill_lane(9, prompt[:10], 2, logits=False)
+    cache, _ = om.prefill(prompt[:10], 2)
+    for i in (10, 11):
+        glg, gam = gm.decode([9], [int(prompt[i])], [2])
+        expect = om.decode(cache, int(prompt[i]), 2)
+        assert _max_abs(glg[0], expect) <= LOGIT_MAX_ABS
+        check_argmax(int(gam[0]), expect, f"after the wait test, position {i}")
+    tl.tl_check_device_error(gm.handle)
+
+
 def test_tiny_context_full(tiny, path):
     w, om, gm = tiny
     _use(gm, path)
@@ -296,9 +330,12 @@ def _memo(om, key, fn):
 
 
 def test_lm_prefill_then_decode(lm, path):
+    # The whole benchmarked sequence: a 128-token prompt prefilled with no
+    # logits, then all 128 greedy decode steps, every step's logits and argmax
+    # checked (teacher-forced with the oracle's tokens).
     w, om, gm = lm
     _use(gm, path)
-    L, P, steps = 8, 128, 6
+    L, P, steps = 8, 128, 128
     prompt = tl_synth.make_tokens(tl_synth.SEED_LM, w.shape.vocab, P + 1)
     o_tokens, o_logits = _memo(om, "greedy", lambda: om.generate_greedy(prompt, L, steps))
     gm.prefill_lane(0, prompt[:P], L, logits=False)
@@ -338,3 +375,65 @@ def test_lm_lanes_per_lane_loops(lm, path):
         expect = _memo(om, ("lane", i), lambda: om.score_last(prompts[i, :P + 1], loops[i]))
         assert _max_abs(together[i], expect) <= LOGIT_MAX_ABS
         check_argmax(int(am[i]), expect, f"lane {i}")
+
+
+def test_lm_loops_sweep(lm):
+    # Loops L in {1, 2, 4, 8, 16} on one lane: a 512-token prompt prefilled
+    # with last-position logits, then two cached decode steps.
+    w, om, gm = lm
+    gm.set_path(tl.DECODE_AUTO)
+    P = 512
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LSWEEP, w.shape.vocab, P + 2)
+    for L in (1, 2, 4, 8, 16):
+        cache, o_pre = om.prefill(prompt[:P], L)
+        lg, am = gm.prefill_lane(7, prompt[:P], L)
+        assert _max_abs(lg, o_pre) <= LOGIT_MAX_ABS, (L, "prefill")
+        check_argmax(am, o_pre, f"L={L} prefill")
+        for i in range(2):
+            expect = om.decode(cache, int(prompt[P + i]), L)
+            glg, gam = gm.decode([7], [int(prompt[P + i])], [L])
+            err = _max_abs(glg[0], expect)
+            assert err <= LOGIT_MAX_ABS, (L, i, err)
+            check_argmax(int(gam[0]), expect, f"L={L} step {i}")
+
+
+def test_lm_sixteen_lanes_every_lane(lm):
+    # All 16 lanes in one decode step, per-lane loops drawn from {4, 8, 16},
+    # ragged prompt lengths; every lane is compared with its own single-lane
+    # oracle run, on two consecutive steps.
+    w, om, gm = lm
+    gm.set_path(tl.DECODE_AUTO)
+    n = 16
+    loops = [int(v) for v in tl_synth.make_lane_loops(tl_synth.SEED_LSWEEP + 16, n)]
+    prompts = tl_synth.make_lane_prompts(tl_synth.SEED_LSWEEP + 16, w.shape.vocab, n, 100)
+    lens = [40 + 4 * i for i in range(n)]       # 40 .. 100 tokens
+    caches = []
+    for i in range(n):
+        gm.prefill_lane(i, prompts[i, :lens[i]], loops[i], logits=False)
+        caches.append(om.prefill(prompts[i, :lens[i]], loops[i])[0])
+    fed = [int(prompts[i, lens[i] - 1]) ^ 1 for i in range(n)]   # any in-range ids
+    for step in range(2):
+        lg, am = gm.decode(list(range(n)), fed, loops)
+        for i in range(n):
+            expect = om.decode(caches[i], fed[i], loops[i])
+            err = _max_abs(lg[i], expect)
+            assert err <= LOGIT_MAX_ABS, (step, i, loops[i], err)
+            check_argmax(int(am[i]), expect, f"step {step} lane {i}")
+        fed = [int((t * 7 + 3) % w.shape.vocab) for t in fed]
+
+
+def test_lm_long_context(lm):
+    # One lane decoding at the end of the 2048-token context: a 2040-token
+    # prompt at L = 2, then decode steps up to position 2047 (the last slot).
+    w, om, gm = lm
+    gm.set_path(tl.DECODE_AUTO)
+    L, P = 2, 2040
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LSWEEP + 2048, w.shape.vocab, 2048)
+    cache, _ = om.prefill(prompt[:P], L)
+    gm.prefill_lane(8, prompt[:P], L, logits=False)
+    for pos in range(P, 2048):
+        expect = om.decode(cache, int(prompt[pos]), L)
+        glg, gam = gm.decode([8], [int(prompt[pos])], [L])
+        err = _max_abs(glg[0], expect)
+        assert err <= LOGIT_MAX_ABS, (pos, err)
+        check_argmax(int(gam[0]), expect, f"position {pos}")

@@ -31,6 +31,8 @@ __all__ = [
     "tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count", "KERNEL_CLASSES",
     "tl_model_set_graphs", "tl_model_set_decode_path", "DECODE_AUTO", "DECODE_LAYERED", "DECODE_FUSED",
     "tl_probe_read_bandwidth", "tl_model_set_trace", "tl_model_trace_grid",
+    "tl_model_set_wait_test", "tl_extend", "tl_generate_speculative", "tl_score_logit_lens",
+    "tl_score_early_exit", "tl_lane_fork", "tl_spec_stats",
     "tl_linear_create", "tl_linear_destroy", "tl_linear_forward",
     "tl_op_rmsnorm", "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill",
     "tl_op_gqa_decode_noalloc",
@@ -72,6 +74,10 @@ class tl_weights(ctypes.Structure):
                 ("pre", POINTER(tl_block)), ("loop", POINTER(tl_block))]
 
 
+class tl_spec_stats(ctypes.Structure):
+    _fields_ = [("rounds", c_int), ("drafted", c_int), ("accepted", c_int)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -95,6 +101,12 @@ def _load():
         "tl_model_set_decode_path": (st, [P, c_int]),
         "tl_model_set_trace": (st, [P, P, c_longlong]),
         "tl_model_trace_grid": (c_int, [P]),
+        "tl_model_set_wait_test": (st, [P, c_int]),
+        "tl_extend": (st, [P, c_int, P, c_int, P, P, P]),
+        "tl_generate_speculative": (st, [P, c_int, P, c_int, c_int, c_int, P, POINTER(tl_spec_stats), P]),
+        "tl_score_logit_lens": (st, [P, P, c_int, c_int, P, P, P]),
+        "tl_score_early_exit": (st, [P, P, c_int, c_int, c_int, P, P, POINTER(c_int), P]),
+        "tl_lane_fork": (st, [P, c_int, c_int, c_int, P]),
         "tl_probe_read_bandwidth": (st, [P, c_size_t, c_int, P, POINTER(c_double)]),
         "tl_linear_create": (st, [POINTER(tl_int4_linear), c_int, c_int, c_int, POINTER(c_void_p)]),
         "tl_linear_destroy": (None, [P]),
@@ -135,7 +147,9 @@ def __getattr__(name):
 # names every header declaration must have in the library (checked by tests)
 EXPORTED = sorted(["tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count",
                    "tl_model_set_graphs", "tl_model_set_decode_path", "tl_probe_read_bandwidth",
-                   "tl_model_set_trace", "tl_model_trace_grid",
+                   "tl_model_set_trace", "tl_model_trace_grid", "tl_model_set_wait_test",
+                   "tl_extend", "tl_generate_speculative", "tl_score_logit_lens", "tl_score_early_exit",
+                   "tl_lane_fork",
                    "tl_model_create", "tl_model_destroy", "tl_prefill", "tl_decode_step",
                    "tl_score_last", "tl_lane_length", "tl_model_info", "tl_check_device_error",
                    "tl_linear_create", "tl_linear_destroy", "tl_linear_forward", "tl_op_rmsnorm",
@@ -254,6 +268,39 @@ def tl_score_last(model, d_tokens, n_tokens, loops, d_logits, d_argmax=None, str
                              _ptr(d_argmax), _stream(stream)))
 
 
+def tl_extend(model, lane, d_tokens, n_tokens, d_logits=None, d_argmax=None, stream=None) -> None:
+    _check(_L().tl_extend(model, int(lane), _ptr(d_tokens), int(n_tokens), _ptr(d_logits), _ptr(d_argmax),
+                         _stream(stream)))
+
+
+def tl_generate_speculative(model, lane, d_first_token, max_tokens, draft_loops, draft_ahead, d_out_tokens,
+                            stream=None) -> dict:
+    """Returns the round counters {rounds, drafted, accepted}."""
+    stats = tl_spec_stats()
+    _check(_L().tl_generate_speculative(model, int(lane), _ptr(d_first_token), int(max_tokens), int(draft_loops),
+                                       int(draft_ahead), _ptr(d_out_tokens), ctypes.byref(stats),
+                                       _stream(stream)))
+    return {"rounds": stats.rounds, "drafted": stats.drafted, "accepted": stats.accepted}
+
+
+def tl_score_logit_lens(model, d_tokens, n_tokens, loops, d_logits, d_argmax=None, stream=None) -> None:
+    _check(_L().tl_score_logit_lens(model, _ptr(d_tokens), int(n_tokens), int(loops), _ptr(d_logits),
+                                   _ptr(d_argmax), _stream(stream)))
+
+
+def tl_score_early_exit(model, d_tokens, n_tokens, max_loops, stable_n, d_logits, d_argmax=None,
+                        stream=None) -> int:
+    """Returns the loop iterations run."""
+    used = c_int(0)
+    _check(_L().tl_score_early_exit(model, _ptr(d_tokens), int(n_tokens), int(max_loops), int(stable_n),
+                                   _ptr(d_logits), _ptr(d_argmax), ctypes.byref(used), _stream(stream)))
+    return used.value
+
+
+def tl_lane_fork(model, src_lane, dst_lane, n_tokens, stream=None) -> None:
+    _check(_L().tl_lane_fork(model, int(src_lane), int(dst_lane), int(n_tokens), _stream(stream)))
+
+
 def tl_lane_length(model, lane) -> int:
     out = c_int()
     _check(_L().tl_lane_length(model, int(lane), ctypes.byref(out)))
@@ -313,6 +360,12 @@ def tl_model_set_trace(model, buf=None, n_entries: int = 0) -> None:
 
 def tl_model_trace_grid(model) -> int:
     return int(_L().tl_model_trace_grid(model))
+
+
+def tl_model_set_wait_test(model, extra_arrivals: int) -> None:
+    """Test hook: 1 makes the next single-kernel steps' grid barriers run out
+    of time (see tl.h); 0 restores normal steps."""
+    _check(_L().tl_model_set_wait_test(model, int(extra_arrivals)))
 
 
 def tl_model_set_decode_path(model, path: int) -> None:

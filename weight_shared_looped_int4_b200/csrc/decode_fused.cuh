@@ -100,6 +100,7 @@ struct FusedArgs {
   int* head_idx;
   unsigned* head_ticket;             // zero between launches
   unsigned* bar;                     // [0] arrivals, [1] exits, [2] give-up; zero between launches
+  unsigned bar_extra;                // arrivals every grid barrier expects beyond the grid (0; 1 = wait test)
   int* err_flag;
   // shared-memory plan
   int n_slots;                       // ring slots
@@ -842,7 +843,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) decode_fused_kernel(const __
   } else {
     const int P = gridDim.x, c = blockIdx.x;
     int item = 0;
-    unsigned target = 0;
+    unsigned target = a.bar_extra;   // > 0 only under the wait test: no barrier can complete
     __half* xs = reinterpret_cast<__half*>(area);
     pdl_wait();   // head-only launches follow the kernel that wrote x
     for (int e = tid; e < (a.head_only ? 0 : a.M * (a.hd / 2)); e += kFusedCompute) {

@@ -3,17 +3,18 @@
 // call itself allocates nothing.
 //
 // Who needs it: callers that must not call cudaMalloc from inside their own
-// code, e.g. code running under a CUDA graph capture that forbids allocation,
-// a host that pre-plans every device byte before serving starts, or an
-// environment whose allocator is owned by someone else and must not be
-// bypassed.  tl_op_gqa_decode allocates (and may grow) its workspace on first
-// use; this variant never does.
+// code, e.g. a host that pre-plans every device byte before serving starts,
+// or a plug-in running inside another runtime whose allocator owns the
+// device memory and must not be bypassed.  tl_op_gqa_decode allocates (and
+// may grow) its workspace on first use; this variant never does.
 //
 // The scratch is the file-scope array below.  Every GPU that loads this
 // library reserves it for the life of the process.  In host code the name
 // g_noalloc_scratch is only a stand-in for the device array, not a device
 // address: the device address is looked up once per device with
-// cudaGetSymbolAddress (with that device current) and cached.
+// cudaGetSymbolAddress (with that device current) and cached for the life of
+// the process.  The cache is not refreshed if the device's context is torn
+// down (cudaDeviceReset): a call after that would use a stale address.
 #include <mutex>
 #include <string>
 
@@ -111,7 +112,7 @@ extern "C" tl_status tl_op_gqa_decode_noalloc(const uint16_t* d_q, const uint16_
   if (ctx_stride < 1 || ctx_stride > 8192) return err(TL_ERR_INVALID_ARG, "ctx_stride must be in [1, 8192]");
   if (B < 1 || B > kNoAllocMaxRows)
     return err(TL_ERR_UNSUPPORTED, "B must be in [1, 32] for the no-allocation variant");
-  if (B * n_kv_heads > kNoAllocTickets) return err(TL_ERR_UNSUPPORTED, "B * n_kv_heads exceeds 4096");
+  if ((long long)B * n_kv_heads > kNoAllocTickets) return err(TL_ERR_UNSUPPORTED, "B * n_kv_heads exceeds 4096");
   const size_t part_bytes = (size_t)B * n_kv_heads * kDecodeMaxSplits * rep * (head_dim + kPartPad) * sizeof(float);
   if (kPartOffset + part_bytes > kNoAllocScratchBytes)
     return err(TL_ERR_UNSUPPORTED,

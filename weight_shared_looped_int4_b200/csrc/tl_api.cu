@@ -572,6 +572,7 @@ struct tl_model {
   float* head_val = nullptr;
   int* head_idx = nullptr;
   int* err_flag = nullptr;
+  int32_t* spec_tok = nullptr;    // speculative decode / early exit tokens [2 kMaxLanes + 2]
   int head_grid = 0;
   HeadIO* io = nullptr;          // output pointers of the current decode step
   TcScratch tc;                  // tensor-core GEMM scratch (prefill)
@@ -617,7 +618,7 @@ struct tl_model {
       if (kv_.second.exec) cudaGraphExecDestroy(kv_.second.exec);
     graphs.clear();
     if (cap_stream) cudaStreamDestroy(cap_stream);
-    void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row,
+    void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row, spec_tok,
                     attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.bt2, tc.partial, tc.tickets,
                     rope_tab, fused_bar, fused_val, fused_idx};
     for (void* p : ptrs)
@@ -836,9 +837,9 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   return TL_OK;
 }
 
-// Prefill forms of run_qkv / run_ffn on the tensor cores (positions 0..T-1 of
-// one lane).
-tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, cudaStream_t st) {
+// Prefill forms of run_qkv / run_ffn on the tensor cores (positions
+// pos0..pos0+T-1 of one lane).
+tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, int pos0, cudaStream_t st) {
   WindowScope window_scope(m, layer);
   const tl_config& c = m->cfg;
   const BlockDev& b = m->block(layer);
@@ -849,7 +850,7 @@ tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, cudaStream_t st) {
   ta.q_out = m->q; ta.ldq = qdim; ta.n_q_rows = qdim; ta.n_kv_rows = c.n_kv_heads * hd; ta.hd = hd;
   ta.k_plane = m->k_plane(layer) + lane * m->lane_stride;
   ta.v_plane = m->v_plane(layer) + lane * m->lane_stride;
-  ta.ctx = c.max_ctx; ta.pos0 = 0; ta.theta = c.rope_theta; ta.rope_tab = m->rope_tab;
+  ta.ctx = c.max_ctx; ta.pos0 = pos0; ta.theta = c.rope_theta; ta.rope_tab = m->rope_tab;
   kclass(TL_KERNEL_GEMM_TC);
   TL_CUDA(launch_tc_linear(b.qkv.tc, b.qkv.sz, c.d_model, b.qkv.N, b.qkv.n_tiles, PREP_NORM, pa, ta, TC_ROPE_KV,
                            T, m->tc, st));
@@ -895,6 +896,7 @@ tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, fl
     // its head tiles through a bulk-copy ring (15 compute warps)
     FusedArgs f = m->fused;
     f.head_only = 1;
+    f.bar_extra = 0;   // the wait test applies to full fused steps only
     f.M = M;
     f.x = const_cast<float*>(x);
     for (int i = 0; i < M; ++i) f.out_row[i] = i;
@@ -929,27 +931,38 @@ tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, fl
   return TL_OK;
 }
 
-// Whole-prompt forward on one lane (positions 0..T-1).
-tl_status forward_prompt(tl_model* m, int lane, const int32_t* d_tokens, int T, int loops,
-                         float* d_logits, int32_t* d_argmax, cudaStream_t st) {
+// What a forward pass over a lane's tokens produces besides the KV cache.
+struct FwdOut {
+  float* logits = nullptr;       // last position [V] (or every position [T][V] with all_rows)
+  int32_t* argmax = nullptr;     // last position [1] (or [T])
+  bool all_rows = false;         // head on every position (T <= kMaxLanes)
+  float* lens_logits = nullptr;  // logit lens: last position after each loop iteration [loops][V]
+  int32_t* lens_argmax = nullptr;
+};
+
+// Forward of T tokens on one lane at positions pos0..pos0+T-1 through
+// n_pre + loops effective layers, attending to the lane's cached keys
+// 0..pos0+t (a whole prompt when pos0 = 0, an appended chunk otherwise).
+tl_status forward_tokens(tl_model* m, int lane, const int32_t* d_tokens, int T, int loops, int pos0,
+                         const FwdOut& out, cudaStream_t st) {
   const tl_config& c = m->cfg;
   const int d = c.d_model, qdim = c.n_q_heads * c.head_dim;
   const int n_layers = c.n_pre + loops;
   kclass(TL_KERNEL_SETUP);
-  TL_CUDA(launch(fill_rows_kernel, dim3((T + 255) / 256), dim3(256), 0, st, m->rows, T, lane, 0));
+  TL_CUDA(launch(fill_rows_kernel, dim3((T + 255) / 256), dim3(256), 0, st, m->rows, T, lane, pos0));
   kclass(TL_KERNEL_EMBED);
   TL_CUDA(launch(embed_kernel, dim3(T), dim3(256), 0, st, (const __half*)m->embed, d, c.vocab,
                  d_tokens, (const int*)nullptr, m->x, m->err_flag));
   const bool tc = T >= kTcMinTokens;
   for (int layer = 0; layer < n_layers; ++layer) {
-    tl_status rc = tc ? run_qkv_tc(m, layer, lane, T, st) : run_qkv(m, layer, T, m->x, m->rows, m->q, st);
+    tl_status rc = tc ? run_qkv_tc(m, layer, lane, T, pos0, st) : run_qkv(m, layer, T, m->x, m->rows, m->q, st);
     if (rc != TL_OK) return rc;
     PrefillAttnArgs pa{};
     pa.qf = m->q; pa.q_bstride = 0; pa.ldq = qdim;
     pa.k = m->k_plane(layer) + lane * m->lane_stride;
     pa.v = m->v_plane(layer) + lane * m->lane_stride;
     pa.kv_bstride = 0; pa.ctx = c.max_ctx;
-    pa.T = T; pa.pos0 = 0; pa.Hkv = c.n_kv_heads;
+    pa.T = T; pa.pos0 = pos0; pa.Hkv = c.n_kv_heads;
     pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
     if (tc) {   // straight into the O projection's B tiles
       pa.bt = m->tc.bt;
@@ -959,10 +972,39 @@ tl_status forward_prompt(tl_model* m, int lane, const int32_t* d_tokens, int T, 
     TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
     rc = tc ? run_ffn_tc(m, layer, T, st) : run_ffn(m, layer, T, m->x, m->o, m->h, st);
     if (rc != TL_OK) return rc;
+    if ((out.lens_logits || out.lens_argmax) && layer >= c.n_pre) {
+      const int i = layer - c.n_pre;   // loop iteration i + 1 done
+      rc = launch_head(m, m->x + (size_t)(T - 1) * d, 1, nullptr,
+                       out.lens_logits ? out.lens_logits + (size_t)i * c.vocab : nullptr,
+                       out.lens_argmax ? out.lens_argmax + i : nullptr, st);
+      if (rc != TL_OK) return rc;
+    }
   }
-  if (d_logits || d_argmax)
-    return launch_head(m, m->x + (size_t)(T - 1) * d, 1, nullptr, d_logits, d_argmax, st);
+  if (out.logits || out.argmax) {
+    if (out.all_rows) return launch_head(m, m->x, T, nullptr, out.logits, out.argmax, st);
+    return launch_head(m, m->x + (size_t)(T - 1) * d, 1, nullptr, out.logits, out.argmax, st);
+  }
   return TL_OK;
+}
+
+tl_status decode_impl(tl_model* m, int n_lanes, const int32_t* h_lane_ids, const int32_t* d_tokens,
+                      const int32_t* h_loops, float* d_logits, int32_t* d_argmax, cudaStream_t st);
+
+// Copy positions [0, n) of every KV slice of `layers` layers from one lane to
+// another: runs of n * head_dim fp16 per (layer, K|V, kv head), 16 bytes per
+// thread, one CTA row per run (grid.y), the positions of a run over grid.x.
+__global__ void kv_copy_kernel(__half* __restrict__ kv, long long lane_stride, long long layer_stride,
+                               long long plane, int Hkv, int ctx, int hd, int src, int dst, int n) {
+  pdl_trigger();
+  pdl_wait();
+  const int run = blockIdx.y;                  // (layer * 2 + kv) * Hkv + head
+  const int head = run % Hkv, kvsel = (run / Hkv) & 1, layer = run / (2 * Hkv);
+  const size_t off = (size_t)layer * layer_stride + (size_t)kvsel * plane + (size_t)head * ctx * hd;
+  const uint4* s4 = reinterpret_cast<const uint4*>(kv + (size_t)src * lane_stride + off);
+  uint4* d4 = reinterpret_cast<uint4*>(kv + (size_t)dst * lane_stride + off);
+  const size_t n16 = (size_t)n * hd / 8;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
+    d4[i] = __ldcs(s4 + i);
 }
 
 }  // namespace
@@ -1073,6 +1115,7 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
             alloc((void**)&m->tickets, (size_t)(kMaxLanes * c.n_kv_heads + 1) * 4) &&
             alloc((void**)&m->head_val, (size_t)m->head_grid * 16 * 4) &&
             alloc((void**)&m->head_idx, (size_t)m->head_grid * 16 * 4) && alloc((void**)&m->err_flag, 4) &&
+            alloc((void**)&m->spec_tok, (2 * kMaxLanes + 2) * 4) &&
             alloc((void**)&m->io, sizeof(HeadIO));
   if (ok) {
     const int kmax = std::max(std::max(d, qdim), c.ffn_dim);
@@ -1192,8 +1235,10 @@ tl_status tl_prefill(tl_model* m, int lane, const int32_t* d_tokens, int n_token
   DeviceGuard guard(m->device);
   if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
   ProfScope prof_scope(&m->prof);
-  tl_status rc = forward_prompt(m, lane, d_tokens, n_tokens, loops, d_last_logits, d_last_argmax,
-                                (cudaStream_t)stream);
+  FwdOut out;
+  out.logits = d_last_logits;
+  out.argmax = d_last_argmax;
+  tl_status rc = forward_tokens(m, lane, d_tokens, n_tokens, loops, 0, out, (cudaStream_t)stream);
   if (rc != TL_OK) {
     m->lane_len[lane] = 0;
     return rc;
@@ -1213,7 +1258,10 @@ tl_status tl_score_last(tl_model* m, const int32_t* d_tokens, int n_tokens, int 
   DeviceGuard guard(m->device);
   if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
   ProfScope prof_scope(&m->prof);
-  return forward_prompt(m, c.max_lanes, d_tokens, n_tokens, loops, d_logits, d_argmax, (cudaStream_t)stream);
+  FwdOut out;
+  out.logits = d_logits;
+  out.argmax = d_argmax;
+  return forward_tokens(m, c.max_lanes, d_tokens, n_tokens, loops, 0, out, (cudaStream_t)stream);
 }
 
 tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, const int32_t* d_tokens,
@@ -1222,7 +1270,6 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
   const tl_config& c = m->cfg;
   if (n_lanes < 1 || n_lanes > c.max_lanes) return fail(TL_ERR_INVALID_ARG, "n_lanes %d not in [1, max_lanes]", n_lanes);
   if (!h_lane_ids || !d_tokens || !h_loops) return fail(TL_ERR_INVALID_ARG, "null argument");
-  std::vector<int> order(n_lanes);
   for (int i = 0; i < n_lanes; ++i) {
     const int lane = h_lane_ids[i];
     if (lane < 0 || lane >= c.max_lanes) return fail(TL_ERR_INVALID_ARG, "lane %d out of range", lane);
@@ -1233,8 +1280,27 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
       return fail(TL_ERR_LOOPS_MISMATCH, "lane %d was prefilled with loops=%d, step asks %d", lane,
                   m->lane_loops[lane], h_loops[i]);
     if (m->lane_len[lane] >= c.max_ctx) return fail(TL_ERR_CONTEXT_FULL, "lane %d is full", lane);
-    order[i] = i;
   }
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  ProfScope prof_scope(&m->prof);
+  return decode_impl(m, n_lanes, h_lane_ids, d_tokens, h_loops, d_logits, d_argmax, (cudaStream_t)stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// One decode step of validated rows: lane h_lane_ids[i] feeds d_tokens[i] at
+// its current length through n_pre + h_loops[i] layers (h_loops[i] may be
+// below the lane's prefill loops: a draft step reads and writes only the
+// first slices, which a longer pass computes identically); each lane's
+// length grows by one.
+tl_status decode_impl(tl_model* m, int n_lanes, const int32_t* h_lane_ids, const int32_t* d_tokens,
+                      const int32_t* h_loops, float* d_logits, int32_t* d_argmax, cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  std::vector<int> order(n_lanes);
+  for (int i = 0; i < n_lanes; ++i) order[i] = i;
   // Rows sorted by loop count (descending): the rows still running at layer l
   // are then a prefix.
   std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return h_loops[a] > h_loops[b]; });
@@ -1250,10 +1316,6 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
   sd.tokens = d_tokens;
   sd.logits = d_logits;
   sd.argmax = d_argmax;
-  DeviceGuard guard(m->device);
-  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
-  cudaStream_t st = (cudaStream_t)stream;
-  ProfScope prof_scope(&m->prof);
   // AUTO takes the layered path: on the 400M model at batch 1 its graph
   // replay currently measures faster than the single-kernel step.
   const bool fused = m->decode_path == TL_DECODE_FUSED;
@@ -1348,6 +1410,199 @@ tl_status tl_decode_step(tl_model* m, int n_lanes, const int32_t* h_lane_ids, co
   return TL_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+tl_status tl_extend(tl_model* m, int lane, const int32_t* d_tokens, int n_tokens, float* d_logits,
+                    int32_t* d_argmax, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (lane < 0 || lane >= c.max_lanes) return fail(TL_ERR_INVALID_ARG, "lane %d out of range", lane);
+  if (!d_tokens) return fail(TL_ERR_INVALID_ARG, "null tokens");
+  if (m->lane_len[lane] == 0) return fail(TL_ERR_NOT_PREFILLED, "lane %d holds no prompt", lane);
+  if (n_tokens < 1) return fail(TL_ERR_INVALID_ARG, "n_tokens must be >= 1");
+  if ((d_logits || d_argmax) && n_tokens > kMaxLanes)
+    return fail(TL_ERR_UNSUPPORTED, "per-position logits need n_tokens <= %d", kMaxLanes);
+  const int pos0 = m->lane_len[lane];
+  if (n_tokens > c.max_ctx - pos0) return fail(TL_ERR_CONTEXT_FULL, "lane %d: %d + %d tokens exceed max_ctx", lane,
+                                               pos0, n_tokens);
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  ProfScope prof_scope(&m->prof);
+  FwdOut out;
+  out.logits = d_logits;
+  out.argmax = d_argmax;
+  out.all_rows = true;
+  tl_status rc = forward_tokens(m, lane, d_tokens, n_tokens, m->lane_loops[lane], pos0, out, (cudaStream_t)stream);
+  if (rc != TL_OK) return rc;
+  m->lane_len[lane] = pos0 + n_tokens;
+  return TL_OK;
+}
+
+tl_status tl_generate_speculative(tl_model* m, int lane, const int32_t* d_first_token, int max_tokens,
+                                  int draft_loops, int draft_ahead, int32_t* d_out_tokens, tl_spec_stats* h_stats,
+                                  void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (lane < 0 || lane >= c.max_lanes) return fail(TL_ERR_INVALID_ARG, "lane %d out of range", lane);
+  if (!d_first_token || !d_out_tokens) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (m->lane_len[lane] == 0) return fail(TL_ERR_NOT_PREFILLED, "lane %d holds no prompt", lane);
+  const int verify_loops = m->lane_loops[lane];
+  if (draft_loops < 1 || draft_loops > verify_loops)
+    return fail(TL_ERR_INVALID_ARG, "draft_loops %d not in [1, the lane's loops %d]", draft_loops, verify_loops);
+  if (draft_ahead < 1 || draft_ahead > kMaxLanes)
+    return fail(TL_ERR_INVALID_ARG, "draft_ahead %d not in [1, %d]", draft_ahead, kMaxLanes);
+  if (max_tokens < 1) return fail(TL_ERR_INVALID_ARG, "max_tokens must be >= 1");
+  const int p_start = m->lane_len[lane];
+  if (max_tokens > c.max_ctx - p_start)
+    return fail(TL_ERR_CONTEXT_FULL, "lane %d: %d + %d tokens exceed max_ctx", lane, p_start, max_tokens);
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  ProfScope prof_scope(&m->prof);
+  cudaStream_t st = (cudaStream_t)stream;
+  // Per round on the device: seq = [next input, draft 1 .. draft k] and the
+  // verifier's greedy tokens ver[0 .. k-1] (ver[i] follows seq[0..i]).
+  int32_t* seq = m->spec_tok;
+  int32_t* ver = m->spec_tok + kMaxLanes + 1;
+  TL_CUDA(cudaMemcpyAsync(seq, d_first_token, 4, cudaMemcpyDeviceToDevice, st));
+  tl_spec_stats stats{};
+  int produced = 0;
+  std::vector<int32_t> h(2 * kMaxLanes + 2);
+  while (produced < max_tokens) {
+    const int p = m->lane_len[lane];
+    const int k = std::min(draft_ahead, max_tokens - produced);
+    // draft: k cached greedy steps with draft_loops (first slices only)
+    const int32_t lane_id = lane, dl = draft_loops;
+    for (int i = 0; i < k; ++i) {
+      tl_status rc = decode_impl(m, 1, &lane_id, seq + i, &dl, nullptr, seq + i + 1, st);
+      if (rc != TL_OK) return rc;
+    }
+    // verify: the k inputs seq[0..k-1] at positions p..p+k-1 with the
+    // lane's loops, one greedy token per position
+    FwdOut out;
+    out.argmax = ver;
+    out.all_rows = true;
+    tl_status rc = forward_tokens(m, lane, seq, k, verify_loops, p, out, st);
+    if (rc != TL_OK) return rc;
+    TL_CUDA(cudaMemcpyAsync(h.data(), seq, (size_t)(2 * kMaxLanes + 2) * 4, cudaMemcpyDeviceToHost, st));
+    TL_CUDA(cudaStreamSynchronize(st));
+    // accept drafts while they equal the verifier's tokens; the verifier's
+    // token at the first mismatch is emitted in place of the draft
+    int acc = 0;
+    while (acc < k && h[1 + acc] == h[kMaxLanes + 1 + acc]) ++acc;
+    const int emit = std::min(acc + 1, k);
+    TL_CUDA(cudaMemcpyAsync(d_out_tokens + produced, ver, (size_t)emit * 4, cudaMemcpyDeviceToDevice, st));
+    TL_CUDA(cudaMemcpyAsync(seq, ver + emit - 1, 4, cudaMemcpyDeviceToDevice, st));
+    produced += emit;
+    m->lane_len[lane] = p + emit;   // roll back the rejected drafts' positions
+    stats.rounds += 1;
+    stats.drafted += k;
+    stats.accepted += acc;
+  }
+  if (h_stats) *h_stats = stats;
+  return TL_OK;
+}
+
+tl_status tl_score_logit_lens(tl_model* m, const int32_t* d_tokens, int n_tokens, int loops, float* d_logits,
+                              int32_t* d_argmax, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (!d_tokens || !d_logits) return fail(TL_ERR_INVALID_ARG, "null tokens or logits");
+  if (n_tokens < 1 || n_tokens > c.max_ctx) return fail(TL_ERR_CONTEXT_FULL, "n_tokens %d not in [1, max_ctx]", n_tokens);
+  if (loops < 1 || loops > c.max_loops) return fail(TL_ERR_INVALID_ARG, "loops %d not in [1, max_loops]", loops);
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  ProfScope prof_scope(&m->prof);
+  FwdOut out;
+  out.lens_logits = d_logits;
+  out.lens_argmax = d_argmax;
+  return forward_tokens(m, c.max_lanes, d_tokens, n_tokens, loops, 0, out, (cudaStream_t)stream);
+}
+
+tl_status tl_score_early_exit(tl_model* m, const int32_t* d_tokens, int n_tokens, int max_loops, int stable_n,
+                              float* d_logits, int32_t* d_argmax, int* h_loops_used, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (!d_tokens || !d_logits || !h_loops_used) return fail(TL_ERR_INVALID_ARG, "null argument");
+  if (n_tokens < 1 || n_tokens > c.max_ctx) return fail(TL_ERR_CONTEXT_FULL, "n_tokens %d not in [1, max_ctx]", n_tokens);
+  if (max_loops < 1 || max_loops > c.max_loops) return fail(TL_ERR_INVALID_ARG, "max_loops %d not in [1, max_loops]", max_loops);
+  if (stable_n < 1) return fail(TL_ERR_INVALID_ARG, "stable_n must be >= 1");
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  ProfScope prof_scope(&m->prof);
+  cudaStream_t st = (cudaStream_t)stream;
+  const int lane = c.max_lanes;   // the private scratch lane, as tl_score_last
+  const int d = c.d_model, qdim = c.n_q_heads * c.head_dim, T = n_tokens;
+  const bool tc = T >= kTcMinTokens;
+  kclass(TL_KERNEL_SETUP);
+  TL_CUDA(launch(fill_rows_kernel, dim3((T + 255) / 256), dim3(256), 0, st, m->rows, T, lane, 0));
+  kclass(TL_KERNEL_EMBED);
+  TL_CUDA(launch(embed_kernel, dim3(T), dim3(256), 0, st, (const __half*)m->embed, d, c.vocab, d_tokens,
+                 (const int*)nullptr, m->x, m->err_flag));
+  int32_t* am = m->spec_tok;   // device argmax of the current iteration
+  int prev = -1, run = 0;
+  for (int layer = 0; layer < c.n_pre + max_loops; ++layer) {
+    tl_status rc = tc ? run_qkv_tc(m, layer, lane, T, 0, st) : run_qkv(m, layer, T, m->x, m->rows, m->q, st);
+    if (rc != TL_OK) return rc;
+    PrefillAttnArgs pa{};
+    pa.qf = m->q; pa.q_bstride = 0; pa.ldq = qdim;
+    pa.k = m->k_plane(layer) + lane * m->lane_stride;
+    pa.v = m->v_plane(layer) + lane * m->lane_stride;
+    pa.kv_bstride = 0; pa.ctx = c.max_ctx;
+    pa.T = T; pa.pos0 = 0; pa.Hkv = c.n_kv_heads;
+    pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
+    if (tc) {
+      pa.bt = m->tc.bt;
+      pa.bt_groups = qdim / 128;
+    }
+    kclass(TL_KERNEL_ATTN_PREFILL);
+    TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
+    rc = tc ? run_ffn_tc(m, layer, T, st) : run_ffn(m, layer, T, m->x, m->o, m->h, st);
+    if (rc != TL_OK) return rc;
+    if (layer < c.n_pre) continue;
+    // output norm + head after this iteration; stop once the greedy token
+    // has been the same for stable_n consecutive iterations
+    rc = launch_head(m, m->x + (size_t)(T - 1) * d, 1, nullptr, d_logits, am, st);
+    if (rc != TL_OK) return rc;
+    int32_t tok = 0;
+    TL_CUDA(cudaMemcpyAsync(&tok, am, 4, cudaMemcpyDeviceToHost, st));
+    TL_CUDA(cudaStreamSynchronize(st));
+    run = tok == prev ? run + 1 : 1;
+    prev = tok;
+    *h_loops_used = layer - c.n_pre + 1;
+    if (run >= stable_n) break;
+  }
+  if (d_argmax) TL_CUDA(cudaMemcpyAsync(d_argmax, am, 4, cudaMemcpyDeviceToDevice, st));
+  return TL_OK;
+}
+
+tl_status tl_lane_fork(tl_model* m, int src_lane, int dst_lane, int n_tokens, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (src_lane < 0 || src_lane >= c.max_lanes || dst_lane < 0 || dst_lane >= c.max_lanes)
+    return fail(TL_ERR_INVALID_ARG, "lane out of range");
+  if (src_lane == dst_lane) return fail(TL_ERR_INVALID_ARG, "source and destination lanes are the same");
+  if (m->lane_len[src_lane] == 0) return fail(TL_ERR_NOT_PREFILLED, "lane %d holds no prompt", src_lane);
+  if (n_tokens < 1 || n_tokens > m->lane_len[src_lane])
+    return fail(TL_ERR_INVALID_ARG, "n_tokens %d not in [1, length of lane %d = %d]", n_tokens, src_lane,
+                m->lane_len[src_lane]);
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  ProfScope prof_scope(&m->prof);
+  const int layers = c.n_pre + m->lane_loops[src_lane];
+  const int runs = layers * 2 * c.n_kv_heads;
+  const int per_run16 = n_tokens * c.head_dim / 8;
+  const int gx = std::max(1, std::min((per_run16 + 255) / 256, std::max(1, 4 * m->tc.n_sm / runs)));
+  kclass(TL_KERNEL_SETUP);
+  TL_CUDA(launch(kv_copy_kernel, dim3(gx, runs), dim3(256), 0, (cudaStream_t)stream, m->kv,
+                 m->lane_stride, m->layer_stride, m->plane, c.n_kv_heads, c.max_ctx, c.head_dim, src_lane, dst_lane,
+                 n_tokens));
+  m->lane_len[dst_lane] = n_tokens;
+  m->lane_loops[dst_lane] = m->lane_loops[src_lane];
+  return TL_OK;
+}
+
 tl_status tl_model_profile_start(tl_model* m, unsigned class_mask) {
   if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
   m->prof.mask = class_mask;
@@ -1403,6 +1658,13 @@ tl_status tl_model_set_trace(tl_model* m, unsigned long long* d_buf, long long n
 }
 
 int tl_model_trace_grid(const tl_model* m) { return m ? m->fused_grid : 0; }
+
+tl_status tl_model_set_wait_test(tl_model* m, int extra_arrivals) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  if (extra_arrivals < 0 || extra_arrivals > 1) return fail(TL_ERR_INVALID_ARG, "extra_arrivals must be 0 or 1");
+  m->fused.bar_extra = (unsigned)extra_arrivals;
+  return TL_OK;
+}
 
 tl_status tl_lane_length(const tl_model* m, int lane, int* h_length) {
   if (!m || !h_length) return fail(TL_ERR_INVALID_ARG, "null argument");
@@ -1700,20 +1962,35 @@ __attribute__((visibility("hidden"))) tl_status tl_internal_set_error(tl_status 
 }
 
 namespace {
-// Read-bandwidth probe: 4 independent 16-byte L2 loads in flight per thread.
-__global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict__ p, size_t n16,
+// Read-bandwidth probe: `passes` sweeps over the buffer inside one launch, 8
+// independent 16-byte loads in flight per thread.  The loads are volatile
+// (ld.global.cg: L2, not L1), so no pass can be folded into another.
+__device__ __forceinline__ uint4 probe_ld(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict__ p, size_t n16, int passes,
                                                          unsigned* __restrict__ sink) {
   const size_t stride = (size_t)gridDim.x * blockDim.x;
-  size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   unsigned acc = 0;
-  for (; i + 3 * stride < n16; i += 4 * stride) {
-    const uint4 a = __ldcg(p + i), b = __ldcg(p + i + stride);
-    const uint4 c = __ldcg(p + i + 2 * stride), d = __ldcg(p + i + 3 * stride);
-    acc ^= a.x ^ a.y ^ a.z ^ a.w ^ b.x ^ b.y ^ b.z ^ b.w ^ c.x ^ c.y ^ c.z ^ c.w ^ d.x ^ d.y ^ d.z ^ d.w;
-  }
-  for (; i < n16; i += stride) {
-    const uint4 a = __ldcg(p + i);
-    acc ^= a.x ^ a.y ^ a.z ^ a.w;
+  for (int pass = 0; pass < passes; ++pass) {
+    size_t i = i0;
+    for (; i + 7 * stride < n16; i += 8 * stride) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = probe_ld(p + i + u * stride);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+    }
+    for (; i < n16; i += stride) {
+      const uint4 a = probe_ld(p + i);
+      acc ^= a.x ^ a.y ^ a.z ^ a.w;
+    }
   }
   if (acc == 0x9E3779B9u) *sink = acc;  // keeps the loads; practically never taken
 }
@@ -1721,7 +1998,7 @@ __global__ void __launch_bounds__(512) read_probe_kernel(const uint4* __restrict
 
 extern "C" {
 
-const char* tl_version(void) { return "0.1.0"; }
+const char* tl_version(void) { return "0.2.0"; }
 
 tl_status tl_probe_read_bandwidth(const void* d_buf, size_t bytes, int reps, void* stream, double* h_gbs) {
   if (!d_buf || !h_gbs) return fail(TL_ERR_INVALID_ARG, "null argument");
@@ -1746,13 +2023,14 @@ tl_status tl_probe_read_bandwidth(const void* d_buf, size_t bytes, int reps, voi
   const dim3 grid(n_sm * 4), block(512);
   const uint4* p = (const uint4*)d_buf;
   const size_t n16 = bytes / 16;
-  for (int i = 0; i < 3 && e == cudaSuccess; ++i) {
-    read_probe_kernel<<<grid, block, 0, st>>>(p, n16, sink);
+  // warm: 3 untimed passes (brings an L2-sized buffer into L2)
+  if (e == cudaSuccess) {
+    read_probe_kernel<<<grid, block, 0, st>>>(p, n16, 3, sink);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaEventRecord(e0, st);
-  for (int i = 0; i < reps && e == cudaSuccess; ++i) {
-    read_probe_kernel<<<grid, block, 0, st>>>(p, n16, sink);
+  if (e == cudaSuccess) {
+    read_probe_kernel<<<grid, block, 0, st>>>(p, n16, reps, sink);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaEventRecord(e1, st);
