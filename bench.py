@@ -1008,9 +1008,91 @@ def run_workload_tiny(args):
     return 0
 
 
+def run_workload_next(args):
+    """The 400M LM around the forward pass: greedy self-speculative decoding
+    (draft 2 or 4 loops, verify 8, look-ahead 4) against plain greedy decode,
+    the logit lens and early exit against score_last, and forking a cached
+    512-token prefix against prefilling it again."""
+    torch, dev, st = _dev_setup()
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    peaks = load_peaks()
+    w, m = _lm_model(tl, tl_synth, 16, 1024, 4)
+    P, n = 128, 128
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, w.shape.vocab, 1024)
+    d_prompt = torch.as_tensor(prompt, device=dev)
+    out = torch.zeros(n, dtype=torch.int32, device=dev)
+    hist = torch.zeros(n + 1, dtype=torch.int32, device=dev)
+    hp = hist.data_ptr()
+    res = {}
+    launches0 = tl.tl_kernel_launch_count()
+
+    def ev_ms(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    with ClockSampler(0) as clocks:
+        def plain():
+            for i in range(n):
+                tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1), st)
+        for rep in range(3):
+            tl.tl_prefill(m, 0, d_prompt, P, LOOPS, None, None, st)
+            with torch.cuda.stream(st):
+                hist[0:1].copy_(d_prompt[P:P + 1])
+            t_plain = ev_ms(plain)
+        greedy_tokens = hist[1:].cpu().numpy().copy()
+        res["plain_decode_tok_s"] = round(n / (t_plain / 1e3), 1)
+        for draft in (2, 4):
+            for rep in range(3):
+                tl.tl_prefill(m, 0, d_prompt, P, LOOPS, None, None, st)
+                stats = {}
+                t = ev_ms(lambda: stats.update(tl.tl_generate_speculative(m, 0, d_prompt[P:], n, draft, 4, out, st)))
+            same = int(np.sum(out.cpu().numpy() == greedy_tokens))
+            res[f"speculative_draft{draft}_ahead4"] = {
+                "tok_s": round(n / (t / 1e3), 1), "rounds": stats["rounds"], "drafted": stats["drafted"],
+                "accepted": stats["accepted"], "acceptance": round(stats["accepted"] / stats["drafted"], 4),
+                "tokens_equal_to_plain_greedy": same}
+        d_tok = d_prompt[:P]
+        lg = torch.empty((LOOPS, V), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            tl.tl_score_last(m, d_tok, P, LOOPS, lg[0], None, st)
+        t_sl = statistics.median(ev_ms(lambda: tl.tl_score_last(m, d_tok, P, LOOPS, lg[0], None, st))
+                                 for _ in range(10))
+        t_lens = statistics.median(ev_ms(lambda: tl.tl_score_logit_lens(m, d_tok, P, LOOPS, lg, None, st))
+                                   for _ in range(10))
+        used = []
+        t_exit = statistics.median(ev_ms(lambda: used.append(
+            tl.tl_score_early_exit(m, d_tok, P, 16, 2, lg[0], None, st))) for _ in range(10))
+        res["score_last_T128_L8_ms"] = round(t_sl, 4)
+        res["logit_lens_T128_L8_ms"] = round(t_lens, 4)
+        res["early_exit_T128_max16_stable2"] = {"ms": round(t_exit, 4), "loops_used": used[-1]}
+        PF = 512
+        tl.tl_prefill(m, 1, d_prompt, PF, LOOPS, None, None, st)
+        t_pf = statistics.median(ev_ms(lambda: tl.tl_prefill(m, 1, d_prompt, PF, LOOPS, None, None, st))
+                                 for _ in range(5))
+        for _ in range(3):
+            tl.tl_lane_fork(m, 1, 2, PF, st)
+        t_fork = statistics.median(ev_ms(lambda: tl.tl_lane_fork(m, 1, 2, PF, st)) for _ in range(20))
+        fork_bytes = 2 * (2 + LOOPS) * 2 * HKV * PF * HD * 2    # read + write
+        res["prefix_512_L8"] = {"prefill_ms": round(t_pf, 4), "fork_ms": round(t_fork, 4),
+                                "fork_gbs": round(fork_bytes / (t_fork * 1e6), 1),
+                                "fork_frac_of_hbm": round(fork_bytes / (t_fork * 1e6) / peaks["hbm_gbs"], 4),
+                                "speedup_vs_prefill": round(t_pf / t_fork, 1)}
+    tl.tl_check_device_error(m)
+    tl.tl_model_destroy(m)
+    print(json.dumps({"workload": "400M looped LM: speculative decode, logit lens, early exit, prefix fork",
+                      "results": res, "peaks": peaks,
+                      "gpu_launches": tl.tl_kernel_launch_count() - launches0, "clocks": clocks.summary()}))
+    return 0
+
+
 WORKLOADS = {"tiny": run_workload_tiny, "linear": run_workload_linear,
              "attention": run_workload_attention, "lsweep": run_workload_lsweep,
-             "peaks": run_workload_peaks}
+             "peaks": run_workload_peaks, "next": run_workload_next}
 
 
 def main():

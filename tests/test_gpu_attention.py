@@ -106,9 +106,12 @@ def test_prefill_attention(T, B):
     _prefill_case(T, B, 0, HQ, HKV, HD, seed=tl_synth.SEED_ATTN + 7 * T + B, sample=sample)
 
 
-@pytest.mark.parametrize("T,pos0,hq,hkv,hd", [(1, 0, 4, 2, 64), (37, 0, 4, 2, 64), (50, 77, 16, 4, 128),
-                                              (130, 5, 8, 8, 64), (65, 0, 8, 1, 128)])
+@pytest.mark.parametrize("T,pos0,hq,hkv,hd", [(1, 0, 4, 2, 64), (17, 3, 16, 4, 128), (37, 0, 4, 2, 64),
+                                              (50, 77, 16, 4, 128), (130, 5, 8, 8, 64), (65, 0, 8, 1, 128),
+                                              (300, 1000, 16, 4, 128)])
 def test_prefill_attention_ragged(T, pos0, hq, hkv, hd):
+    # below 32 queries the 16-query mma.sync kernel runs, from 32 on the
+    # tcgen05 kernel (128-query tiles): ragged tiles, offsets, GQA ratios
     _prefill_case(T, 2, pos0, hq, hkv, hd, seed=T + pos0)
 
 

@@ -318,6 +318,7 @@ struct PrefillAttnArgs {
   // then lo rows, 128-byte swizzled; K = Hq * hd) instead of `of`
   uint8_t* bt;
   int bt_groups;
+  int* err_flag;          // device fault flags (a bounded wait gave up), or NULL
 };
 
 // ---- prefill: tiled, tensor cores (m16n8k16), online softmax --------------

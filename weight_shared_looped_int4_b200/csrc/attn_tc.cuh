@@ -1,0 +1,320 @@
+// Causal tiled prefill GQA attention on the 5th-generation tensor cores
+// (tcgen05, TMEM accumulators) -- the tiled prefill path of TinyLoop README,
+// "Current Runtime Snapshot" (full prefill attention, tiled), with the GQA
+// head mapping of "Status" and the tiled online softmax / causal masking of
+// the tiny-llm feature list.
+//
+// Design (ours, sm_100a):
+// * One CTA per (128-query tile, query head, batch entry); 8 warps.  The
+//   queries are the MMA rows (M = 128): S = Q K^T over a block of 64 keys
+//   (N = 64) and O_blk = P V (N = head_dim), both into TMEM.
+// * Q (fp32 or fp16 in memory) is scaled by 1/sqrt(hd) and split into an fp16
+//   pair (hi, lo); S accumulates Q_hi K^T + Q_lo K^T.  P is split the same
+//   way and O_blk accumulates P_hi V + P_lo V.  K and V are fp16 already, so
+//   the products keep ~fp32 accuracy (as the other attention kernels).
+// * Operands in shared memory, 128-byte swizzled: Q and P K-major (rows of
+//   64 consecutive k), K K-major (a key's head dims are the MMA's K), V
+//   MN-major (a key's head dims are the MMA's N: 64-wide dim chunks LBO apart,
+//   groups of 8 keys SBO apart), so K and V rows are copied as they lie in the
+//   cache, 16 bytes per cp.async, double-buffered one block ahead.
+// * Softmax: warp w reads TMEM lanes 32 (w % 4) .. (its query rows) and half
+//   w / 4 of the columns; the two warps of a row exchange the row maximum and
+//   sum through shared memory.  The online rescaling is applied to the
+//   running output held in registers (O_acc = O_acc c + O_blk), so TMEM never
+//   needs a read-modify-write.
+// * Every mbarrier wait is bounded; a CTA that gives up records kErrTimeout
+//   and still frees its TMEM.
+#pragma once
+
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+
+namespace tl {
+
+constexpr int kAtQ = 128;        // queries per CTA (MMA M)
+constexpr int kAtKeys = 64;      // keys per block (MMA N of S, K of P V)
+constexpr int kAtThreads = 256;  // 8 warps
+
+// Shared-memory plan (bytes) for head_dim HD.
+template <int HD>
+struct AtLayout {
+  static constexpr int KA = HD / 64;                       // 64-wide atoms of a head
+  static constexpr int Q_BYTES = KA * kAtQ * 128;          // one of hi / lo
+  static constexpr int K_BYTES = KA * kAtKeys * 128;       // one key block
+  static constexpr int V_BYTES = KA * kAtKeys * 128;
+  static constexpr int P_BYTES = kAtQ * 128;               // one of hi / lo (64 keys)
+  static constexpr int q_hi = 0, q_lo = Q_BYTES;
+  static constexpr int k0 = 2 * Q_BYTES;                   // [2 buffers]
+  static constexpr int v0 = k0 + 2 * K_BYTES;              // [2 buffers]
+  static constexpr int p_hi = v0 + 2 * V_BYTES, p_lo = p_hi + P_BYTES;
+  static constexpr int total = p_lo + P_BYTES;
+};
+template <int HD>
+__host__ __device__ constexpr size_t attn_tc_smem_bytes() {
+  return (size_t)AtLayout<HD>::total + 1024;   // + alignment slack
+}
+
+// Shared-memory descriptor of an MN-major operand, 128-byte swizzle: rows of
+// 64 consecutive N elements (128 B), 8 rows (8 consecutive K) per 1024-byte
+// swizzle atom; `lbo` bytes between 64-wide N chunks, `sbo` bytes between
+// groups of 8 K.
+__device__ __forceinline__ uint64_t sw128_mnmajor_desc(const void* p, uint32_t lbo, uint32_t sbo) {
+  const uint64_t addr = smem_u32(p);
+  uint64_t d = (addr >> 4) & 0x3FFFull;
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= 1ull << 46;
+  d |= 2ull << 61;
+  return d;
+}
+// kind::f16 instruction descriptor with B MN-major (bit 16).
+__host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
+  return idesc_f16_f32(M, N) | (1u << 16);
+}
+
+template <int HD, bool F32>
+__global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const PrefillAttnArgs a) {
+  using Lay = AtLayout<HD>;
+  constexpr int KA = Lay::KA;
+  constexpr int HALF = HD / 2;                 // output columns per warp
+  extern __shared__ __align__(128) unsigned char at_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(at_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_fail;
+  __shared__ float x_max[2][kAtQ], x_sum[2][kAtQ];
+
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3, ch = warp >> 2;   // TMEM lane quarter, column half
+  const int r = quad * 32 + lane;              // this thread's query row in the tile
+  const int kvh = h / a.rep;
+  const int q0 = qt * kAtQ;
+  const int t_row = q0 + r;                    // token of the row
+  const int pos = a.pos0 + t_row;              // its position (keys 0..pos)
+  const int last_key = a.pos0 + min(q0 + kAtQ - 1, a.T - 1);
+  const int nblk = last_key / kAtKeys + 1;
+  const __half* kp = a.k + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
+  const __half* vp = a.v + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
+
+  if (warp == 0) {
+    tmem_alloc(&s_tmem, 256);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 32) {
+    mbar_init(&mma_bar, 1);
+    fence_mbar_init();
+    s_fail = 0;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint32_t t_s = tmem, t_o = tmem + 128;   // S: 64 columns, O_blk: HD columns
+  pdl_trigger();
+  pdl_wait();
+
+  // ---- K / V block j into buffer j % 2 (cp.async, zeros past last_key) ----
+  auto load_kv = [&](int j) {
+    unsigned char* ks = sm + Lay::k0 + (j & 1) * Lay::K_BYTES;
+    unsigned char* vs = sm + Lay::v0 + (j & 1) * Lay::V_BYTES;
+    const int j0 = j * kAtKeys;
+    for (int c = threadIdx.x; c < kAtKeys * HD / 8; c += kAtThreads) {
+      const int key = c / (HD / 8), c16 = c % (HD / 8);       // 16-byte chunk of the key's row
+      const bool ok = j0 + key <= last_key;
+      const size_t src = ok ? (size_t)(j0 + key) * HD + c16 * 8 : 0;
+      const int atom = c16 >> 3, j16 = c16 & 7;
+      // K: K-major, [atom][64 keys][128 B]
+      cp_async16(ks + atom * kAtKeys * 128 + key * 128 + ((j16 ^ (key & 7)) << 4), kp + src, ok ? 16 : 0);
+      // V: MN-major, [dim chunk][8-key group][8 keys][128 B]
+      cp_async16(vs + atom * (kAtKeys * 128) + (key >> 3) * 1024 + (key & 7) * 128 + ((j16 ^ (key & 7)) << 4),
+                 vp + src, ok ? 16 : 0);
+    }
+    cp_async_commit();
+  };
+  load_kv(0);
+
+  // ---- Q tile: scale, split into (hi, lo), K-major swizzled ----------------
+  {
+    const float scale = 1.0f / sqrtf((float)HD);
+    for (int c = threadIdx.x; c < kAtQ * HD / 8; c += kAtThreads) {
+      const int row = c / (HD / 8), c16 = c % (HD / 8);
+      const int t = q0 + row;
+      float v[8];
+      if (t < a.T) {
+        const size_t off = b * a.q_bstride + (size_t)t * a.ldq + (size_t)h * HD + c16 * 8;
+        if (F32) {
+          const float4 x0 = *reinterpret_cast<const float4*>(a.qf + off);
+          const float4 x1 = *reinterpret_cast<const float4*>(a.qf + off + 4);
+          v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+        } else {
+          const uint4 raw = *reinterpret_cast<const uint4*>(a.qh + off);
+          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = h2_to_f2(w4[i]);
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+      }
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) split_h2(v[2 * i] * scale, v[2 * i + 1] * scale, hw[i], lw[i]);
+      const int atom = c16 >> 3, j16 = c16 & 7;
+      const int o = atom * kAtQ * 128 + row * 128 + ((j16 ^ (row & 7)) << 4);
+      *reinterpret_cast<uint4*>(sm + Lay::q_hi + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(sm + Lay::q_lo + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+  }
+
+  float o_acc[HALF];
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) o_acc[i] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  unsigned phase = 0;
+  const uint32_t idesc_s = idesc_f16_f32(kAtQ, kAtKeys);
+  const uint32_t idesc_o = idesc_f16_f32_bmn(kAtQ, HD);
+
+  for (int j = 0; j < nblk; ++j) {
+    if (j + 1 < nblk) {
+      load_kv(j + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    fence_proxy_async_smem();   // cp.async / st.shared writes -> the tensor core's reads
+    __syncthreads();
+    const unsigned char* ks = sm + Lay::k0 + (j & 1) * Lay::K_BYTES;
+    const unsigned char* vs = sm + Lay::v0 + (j & 1) * Lay::V_BYTES;
+    // ---- S = Q_hi K^T + Q_lo K^T ---------------------------------------------
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const unsigned char* qs = sm + (pass ? Lay::q_lo : Lay::q_hi);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const int atom = kk >> 2, within = (kk & 3) * 32;
+          const uint64_t ad = sw128_kmajor_desc(qs + atom * kAtQ * 128 + within);
+          const uint64_t bd = sw128_kmajor_desc(ks + atom * kAtKeys * 128 + within);
+          tc_mma_f16(t_s, ad, bd, idesc_s, (pass | kk) ? 1u : 0u);
+        }
+      }
+      tc_commit(&mma_bar);
+    }
+    mbar_wait_or_fail(&mma_bar, phase, &s_fail);
+    phase ^= 1u;
+    tc_fence_after();
+    // ---- softmax of this thread's 32 scores (row r, keys ch*32 ..) ----------
+    float s[32];
+    {
+      uint32_t raw[32];
+      tmem_ld32(t_s + ((uint32_t)(quad * 32) << 16) + ch * 32, raw);
+      tmem_ld_wait();
+      const int k0 = j * kAtKeys + ch * 32;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[i] = (k0 + i <= pos) ? __uint_as_float(raw[i]) : -INFINITY;
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, s[i]);
+    x_max[ch][r] = mx;
+    __syncthreads();
+    const float m_new = fmaxf(m_run, fmaxf(mx, x_max[ch ^ 1][r]));
+    const float c = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      s[i] = (m_new == -INFINITY || s[i] == -INFINITY) ? 0.f : expf(s[i] - m_new);
+      sum += s[i];
+    }
+    m_run = m_new;
+    x_sum[ch][r] = sum;
+    // P (hi, lo) of keys ch*32 .. ch*32+31 of row r: 16-byte chunks 4 ch .. 4 ch + 3
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) split_h2(s[q * 8 + 2 * i], s[q * 8 + 2 * i + 1], hw[i], lw[i]);
+      const int j16 = ch * 4 + q;
+      const int o = r * 128 + ((j16 ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(sm + Lay::p_hi + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(sm + Lay::p_lo + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    l_run = l_run * c + sum + x_sum[ch ^ 1][r];
+    // ---- O_blk = P_hi V + P_lo V ---------------------------------------------
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+        const unsigned char* ps = sm + (pass ? Lay::p_lo : Lay::p_hi);
+#pragma unroll
+        for (int kk = 0; kk < kAtKeys / 16; ++kk) {
+          const uint64_t ad = sw128_kmajor_desc(ps + kk * 32);
+          const uint64_t bd = sw128_mnmajor_desc(vs + kk * 2 * 1024, kAtKeys * 128, 1024);
+          tc_mma_f16(t_o, ad, bd, idesc_o, (pass | kk) ? 1u : 0u);
+        }
+      }
+      tc_commit(&mma_bar);
+    }
+    mbar_wait_or_fail(&mma_bar, phase, &s_fail);
+    phase ^= 1u;
+    tc_fence_after();
+    // ---- O_acc = O_acc c + O_blk (row r, columns ch * HALF ..) ---------------
+#pragma unroll
+    for (int c0 = 0; c0 < HALF; c0 += 32) {
+      uint32_t raw[32];
+      tmem_ld32(t_o + ((uint32_t)(quad * 32) << 16) + ch * HALF + c0, raw);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o_acc[c0 + i] = fmaf(o_acc[c0 + i], c, __uint_as_float(raw[i]));
+    }
+    tc_fence_before();
+    __syncthreads();   // S / O_blk / P / this K-V buffer are free for the next block
+  }
+
+  // ---- normalise and store row r, columns ch * HALF .. --------------------
+  if (t_row < a.T) {
+    const float inv = 1.f / l_run;
+    if (F32 && a.bt) {
+      const int tt = t_row / kTcTokensB, tl_ = t_row % kTcTokensB;
+#pragma unroll
+      for (int i = 0; i < HALF; i += 2) {
+        const int k = h * HD + ch * HALF + i;   // column of the O projection's input
+        const int grp = k >> 7, kg = k & 127;
+        uint32_t hw, lw;
+        split_h2(o_acc[i] * inv, o_acc[i + 1] * inv, hw, lw);
+        uint8_t* blk = a.bt + ((size_t)tt * a.bt_groups + grp) * (2 * kTcTokensB * 256);
+        *reinterpret_cast<uint32_t*>(blk + sw128_offset(tl_, kg, 2 * kTcTokensB)) = hw;
+        *reinterpret_cast<uint32_t*>(blk + sw128_offset(kTcTokensB + tl_, kg, 2 * kTcTokensB)) = lw;
+      }
+    } else {
+      const size_t off = b * a.o_bstride + (size_t)t_row * a.ldo + (size_t)h * HD + ch * HALF;
+#pragma unroll
+      for (int i = 0; i < HALF; i += 2) {
+        if (F32) {
+          *reinterpret_cast<float2*>(a.of + off + i) = make_float2(o_acc[i] * inv, o_acc[i + 1] * inv);
+        } else {
+          *reinterpret_cast<uint32_t*>(a.oh + off + i) = pack_h2(o_acc[i] * inv, o_acc[i + 1] * inv);
+        }
+      }
+    }
+  }
+  if (threadIdx.x == 0 && s_fail && a.err_flag) atomicOr(a.err_flag, kErrTimeout);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace tl

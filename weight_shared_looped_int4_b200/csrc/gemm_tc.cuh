@@ -201,10 +201,104 @@ struct TcGemmArgs {
   int perm_F;            // interleaved gate/up rows (the scales are looked up by original row)
   uint8_t* bt_out;       // the down projection's B tiles
   int bt_out_groups;     // its K / 128
+  int cluster;           // 1: the splits of a tile form a thread-block cluster and
+                         // reduce in distributed shared memory (no partial buffer)
   float* partial;        // [splits][row tiles][token tiles][128 tokens][128 rows]
   unsigned* tickets;     // [row tiles][token tiles], zero between launches
   int* err_flag;
 };
+
+// Final epilogue of `ntok` tokens of token tile tt (tile-local tokens tok0 ..
+// tok0 + ntok - 1) of row tile `tile`, whose sums are xch[ntok][kTcRows] in
+// shared memory; threads tid = 0 .. nthr - 1 share the work.
+template <int EPI>
+__device__ void tc_epilogue_tokens(const TcGemmArgs& a, const float* xch, int tile, int tt, int tok0, int ntok,
+                                   int tid, int nthr) {
+  if (EPI == TC_RESID || EPI == TC_RAW || EPI == TC_STORE) {
+    for (int item = tid; item < ntok * kTcRows; item += nthr) {
+      const int ti = item / kTcRows, r = item % kTcRows;
+      const int t = tt * kTcTokens + tok0 + ti, n = tile * kTcRows + r;
+      if (t >= a.T || n >= a.N) continue;
+      const float v = xch[ti * kTcRows + r];
+      const size_t o = (size_t)t * a.ld_out + n;
+      if (EPI == TC_RESID) a.out_f32[o] += v;
+      else if (EPI == TC_RAW) a.out_f32[o] = v;
+      else a.out_f16[o] = __float2half_rn(v);
+    }
+  } else if (EPI == TC_SWIGLU_B) {
+    for (int item = tid; item < ntok * 32; item += nthr) {
+      const int ti = item >> 5, j = (item & 31) * 2;
+      const int tq = tok0 + ti;
+      if (tt * kTcTokens + tq >= a.T) continue;
+      const float* xr = xch + ti * kTcRows;
+      tc_swiglu_store(a.bt_out, a.bt_out_groups, tt, tile, tq, j, xr[j], xr[j + 1], xr[64 + j], xr[65 + j]);
+    }
+  } else {
+    const int hd = a.hd, hh = hd / 2;
+    const int pairs = kTcRows / 2;
+    for (int item = tid; item < ntok * pairs; item += nthr) {
+      const int ti = item / pairs, pr = item % pairs;
+      const int head_local = pr / hh, j = pr % hh;
+      const int r_a = head_local * hd + j, r_b = r_a + hh;
+      const int t = tt * kTcTokens + tok0 + ti;
+      const int na = tile * kTcRows + r_a;
+      if (t >= a.T || na >= a.N) continue;
+      const float va = xch[ti * kTcRows + r_a], vb = xch[ti * kTcRows + r_b];
+      const int pos = a.pos0 + t;
+      if (na < a.n_q_rows) {
+        const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
+        float* qo = a.q_out + (size_t)t * a.ldq;
+        qo[na] = va * cs.x - vb * cs.y;
+        qo[na + hh] = vb * cs.x + va * cs.y;
+      } else if (na < a.n_q_rows + a.n_kv_rows) {
+        const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
+        const int kvh = (na - a.n_q_rows) / hd;
+        __half* dst = a.k_plane + ((size_t)kvh * a.ctx + pos) * hd;
+        dst[j] = __float2half_rn(va * cs.x - vb * cs.y);
+        dst[j + hh] = __float2half_rn(vb * cs.x + va * cs.y);
+      } else {
+        const int kvh = (na - a.n_q_rows - a.n_kv_rows) / hd;
+        __half* dst = a.v_plane + ((size_t)kvh * a.ctx + pos) * hd;
+        dst[j] = __float2half_rn(va);
+        dst[j + hh] = __float2half_rn(vb);
+      }
+    }
+  }
+}
+
+// Split-K reduction inside the thread-block cluster that holds the splits of
+// one (row tile, token tile): each rank's partial tile P [128 tokens][128
+// rows] fp32 sits at the start of its shared memory; rank r sums tokens
+// [r * 128 / S, (r + 1) * 128 / S) over the ranks in rank (= split) order --
+// deterministic -- into a slice buffer behind P and applies the epilogue.
+// Called by all threads of every CTA of the cluster.
+template <int EPI>
+__device__ void tc_cluster_reduce(const TcGemmArgs& a, unsigned char* smem, int tile, int tt) {
+  const int S = a.splits;
+  cluster_sync_all();   // every rank's partial tile is complete
+  const int r = (int)cluster_rank();
+  const int tok0 = r * kTcTokens / S, ntok = (r + 1) * kTcTokens / S - tok0;
+  const float* P = reinterpret_cast<const float*>(smem);
+  float* xs = reinterpret_cast<float*>(smem + (size_t)kTcTokens * kTcRows * 4);   // [ntok][kTcRows]
+  for (int item = threadIdx.x; item < ntok * (kTcRows / 4); item += kTcThreads) {
+    const int ti = item / (kTcRows / 4), r4 = (item % (kTcRows / 4)) * 4;
+    const float* src = P + (size_t)(tok0 + ti) * kTcRows + r4;
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < S; s0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (s0 + i < S) v[i] = ld_cluster_f4(cluster_map(src, (unsigned)(s0 + i)));
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (s0 + i < S) { sum.x += v[i].x; sum.y += v[i].y; sum.z += v[i].z; sum.w += v[i].w; }
+    }
+    *reinterpret_cast<float4*>(xs + ti * kTcRows + r4) = sum;
+  }
+  __syncthreads();
+  tc_epilogue_tokens<EPI>(a, xs, tile, tt, tok0, ntok, threadIdx.x, kTcThreads);
+  cluster_sync_all();   // no rank leaves while another still reads its partial tile
+}
 
 template <int EPI, bool LO>
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGemmArgs a) {
@@ -414,7 +508,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     const int t0 = tt * kTcTokens + half * 64;
     epi_sync(kTcEpiThreads);
     const bool failed = s_fail != 0;
-    if (a.splits > 1) {
+    if (a.splits > 1 && a.cluster) {
+      // partial tile into this CTA's shared memory (the operand stages are
+      // idle: the last MMA has completed), reduced across the cluster below
+      float* P = reinterpret_cast<float*>(smem);   // [128 tokens][128 rows]
+#pragma unroll
+      for (int i = 0; i < 64; ++i) P[(half * 64 + i) * kTcRows + row] = acc[i];
+      if (e == 0 && lane == 0) s_last = 0;
+    } else if (a.splits > 1) {
       float* mine = a.partial + (((size_t)split * row_tiles + tile) * tok_tiles + tt) * (kTcTokens * kTcRows);
 #pragma unroll
       for (int i = 0; i < 64; ++i) mine[(size_t)(half * 64 + i) * kTcRows + row] = acc[i];
@@ -496,6 +597,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   // ---- teardown: every role reaches here; TMEM is always freed -----------
   tc_fence_before();
   __syncthreads();
+  if (a.splits > 1 && a.cluster) tc_cluster_reduce<EPI>(a, smem, tile, tt);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

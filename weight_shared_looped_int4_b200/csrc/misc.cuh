@@ -375,4 +375,196 @@ __global__ void __launch_bounds__(kHeadThreads, 1) head_argmax_kernel(const Head
   if (threadIdx.x == 0) *a.ticket = 0u;
 }
 
+// ---- output norm + head + argmax for up to 4 rows, direct loads -----------
+// One CTA per SM, 16 warps.  Warp w of CTA c owns the 16-row head tiles
+// c * 16 + w, then every P * 16 after that, and streams each whole tile
+// (64 KB at d = 2048, in A-fragment order: lane l's 16-byte word of k16
+// chunk j is exactly its m16n8k16 A operand) with plain 16-byte loads, eight
+// in flight per lane, marked L2 evict-first (the head is read once per token
+// and must not push the loop block out of L2).  The first loads go out
+// before the wait on the previous kernel.  The B operand is the normalised
+// activation as fp16 (hi, lo) pairs from shared memory (columns 2t / 2t + 1
+// = hi / lo of row t), so lane (g, t) ends a tile holding the logits of
+// vocabulary rows g and g + 8 for row t: no cross-warp reduction per tile.
+// The greedy argmax (lowest index on ties) is reduced per warp, per CTA and
+// by the last CTA (ticket).  Timeline (when `trace` is set, G = grid entries
+// per slot): slot 0 start, 1 activations staged, 2 tiles done, 3 end.
+constexpr int kHdWarps = 16;
+constexpr int kHdThreads = kHdWarps * 32;
+constexpr int kHdMaxRows = 4;
+constexpr int kHdUnroll = 8;
+
+__host__ __device__ inline size_t head_direct_smem(int d) { return (size_t)2 * kHdMaxRows * (d + 8) * 2; }
+
+__device__ __forceinline__ uint4 ldg_evict_first(const uint4* p, uint64_t pol) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p), "l"(pol));
+  return r;
+}
+
+__global__ void __launch_bounds__(kHdThreads, 1) head_direct_kernel(const HeadArgs a, unsigned long long* trace,
+                                                                    long long trace_cap) {
+  extern __shared__ __align__(16) unsigned char hsm[];
+  __shared__ float s_ss[kHdMaxRows][kHdWarps];
+  __shared__ float s_bv[kHdMaxRows][kHdWarps];
+  __shared__ int s_bi[kHdMaxRows][kHdWarps];
+  __shared__ int s_last;
+  const int d = a.d, M = a.M, ldx = d + 8;
+  __half* xs = reinterpret_cast<__half*>(hsm);      // hi [kHdMaxRows][ldx]
+  __half* xl = xs + (size_t)kHdMaxRows * ldx;       // lo
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x, P = gridDim.x;
+  const int g = lane >> 2, t = lane & 3;
+  const int nt = a.V >> 4, nk16 = d >> 4;
+  auto stamp = [&](int slot) {
+    if (trace && threadIdx.x == 0) {
+      const long long i = (long long)slot * P + c;
+      if (i < trace_cap) trace[i] = (unsigned long long)globaltimer_ns();
+    }
+  };
+  stamp(0);
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  const int stride = P * kHdWarps;
+  int tile = c * kHdWarps + warp;
+  uint4 wv[kHdUnroll];
+  if (tile < nt) {   // the weights do not depend on earlier kernels
+    const uint4* wt = a.w + (size_t)tile * nk16 * 32 + lane;
+#pragma unroll
+    for (int u = 0; u < kHdUnroll; ++u) wv[u] = ldg_evict_first(wt + u * 32, pol);
+  }
+  pdl_trigger();
+  pdl_wait();
+  float* const logits = a.io ? a.io->logits : a.logits;
+  int32_t* const argmax = a.io ? a.io->argmax : a.argmax;
+
+  // RMSNorm of the M rows, staged as fp16 (hi, lo); rows >= M are zero
+  for (int m = 0; m < M; ++m) {
+    float ss = 0.f;
+    for (int k = threadIdx.x * 4; k < d; k += kHdThreads * 4) {
+      const float4 v = *reinterpret_cast<const float4*>(a.x + (size_t)m * d + k);
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) s_ss[m][warp] = ss;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kHdMaxRows * (d / 2); e += kHdThreads) {
+    const int m = e / (d / 2), k = (e % (d / 2)) * 2;
+    uint32_t hw = 0, lw = 0;
+    if (m < M) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kHdWarps; ++w) tot += s_ss[m][w];
+      const float rs = 1.0f / sqrtf(tot / (float)d + a.eps);
+      const float2 xv = *reinterpret_cast<const float2*>(a.x + (size_t)m * d + k);
+      const float2 gv = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
+      const __half2 h = __floats2half2_rn(xv.x * rs * gv.x, xv.y * rs * gv.y);
+      const float2 r = __half22float2(h);
+      const __half2 l = __floats2half2_rn(xv.x * rs * gv.x - r.x, xv.y * rs * gv.y - r.y);
+      hw = *reinterpret_cast<const uint32_t*>(&h);
+      lw = *reinterpret_cast<const uint32_t*>(&l);
+    }
+    *reinterpret_cast<uint32_t*>(xs + (size_t)m * ldx + k) = hw;
+    *reinterpret_cast<uint32_t*>(xl + (size_t)m * ldx + k) = lw;
+  }
+  __syncthreads();
+  stamp(1);
+
+  const __half* bsrc = ((g & 1) ? xl : xs) + (size_t)(g >> 1) * ldx + 2 * t;
+  float best_v = -INFINITY;
+  int best_i = 0x7fffffff;
+  bool have = tile < nt;   // wv holds the first words of `tile`
+  for (; tile < nt; tile += stride) {
+    const uint4* wt = a.w + (size_t)tile * nk16 * 32 + lane;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int j0 = 0; j0 < nk16; j0 += kHdUnroll) {
+      if (!have) {
+#pragma unroll
+        for (int u = 0; u < kHdUnroll; ++u) wv[u] = ldg_evict_first(wt + (size_t)(j0 + u) * 32, pol);
+      }
+      have = false;
+      uint4 nv[kHdUnroll];
+      const bool more = j0 + kHdUnroll < nk16;
+      if (more) {   // next batch in flight while this one multiplies
+#pragma unroll
+        for (int u = 0; u < kHdUnroll; ++u) nv[u] = ldg_evict_first(wt + (size_t)(j0 + kHdUnroll + u) * 32, pol);
+      }
+#pragma unroll
+      for (int u = 0; u < kHdUnroll; ++u) {
+        const uint32_t af[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(bsrc + (j0 + u) * 16);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(bsrc + (j0 + u) * 16 + 8);
+        if (u & 1) mma_f16_16816(acc2, af, b0, b1);
+        else mma_f16_16816(acc, af, b0, b1);
+      }
+      if (more) {
+#pragma unroll
+        for (int u = 0; u < kHdUnroll; ++u) wv[u] = nv[u];
+        have = true;
+      }
+    }
+    have = false;
+    // lane (g, t): columns 2t (hi) and 2t + 1 (lo) of row t
+    const float v0 = (acc[0] + acc2[0]) + (acc[1] + acc2[1]);
+    const float v1 = (acc[2] + acc2[2]) + (acc[3] + acc2[3]);
+    if (t < M) {
+      const int r0 = tile * 16 + g, r1 = r0 + 8;
+      if (logits) {
+        const size_t o = (size_t)(a.out_row ? a.out_row[t] : t) * a.V;
+        logits[o + r0] = v0;
+        logits[o + r1] = v1;
+      }
+      if (better(v0, r0, best_v, best_i)) { best_v = v0; best_i = r0; }
+      if (better(v1, r1, best_v, best_i)) { best_v = v1; best_i = r1; }
+    }
+  }
+  // best per row: lanes of equal t, then warps, then CTAs
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, best_v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, best_i, o);
+    if (better(ov, oi, best_v, best_i)) { best_v = ov; best_i = oi; }
+  }
+  if (lane < kHdMaxRows) { s_bv[lane][warp] = best_v; s_bi[lane][warp] = best_i; }
+  __syncthreads();
+  stamp(2);
+  if (threadIdx.x < M) {
+    const int m = threadIdx.x;
+    float v = s_bv[m][0];
+    int ix = s_bi[m][0];
+    for (int w = 1; w < kHdWarps; ++w)
+      if (better(s_bv[m][w], s_bi[m][w], v, ix)) { v = s_bv[m][w]; ix = s_bi[m][w]; }
+    a.part_val[c * 16 + m] = v;
+    a.part_idx[c * 16 + m] = ix;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(a.ticket, 1u) == (unsigned)(P - 1);
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    if (argmax && warp < M) {
+      float v = -INFINITY;
+      int ix = 0x7fffffff;
+      for (int cc = lane; cc < P; cc += 32) {
+        const float pv = __ldcg(a.part_val + cc * 16 + warp);
+        const int pi = __ldcg(a.part_idx + cc * 16 + warp);
+        if (better(pv, pi, v, ix)) { v = pv; ix = pi; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, ix, o);
+        if (better(ov, oi, v, ix)) { v = ov; ix = oi; }
+      }
+      if (lane == 0) argmax[a.out_row ? a.out_row[warp] : warp] = ix;
+    }
+    if (threadIdx.x == 0) *a.ticket = 0u;
+  }
+  stamp(3);
+}
+
 }  // namespace tl

@@ -18,9 +18,11 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 #include <vector>
 
 #include "attention.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "decode_fused.cuh"
 #include "gemm_tc.cuh"
@@ -110,7 +112,7 @@ inline void kclass(int c) { g_cls = c; }
 // programmatic dependent launch (and the current L2 access-policy window);
 // `coop` launches are cooperative (all CTAs co-resident) and get neither.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_impl(bool coop, unsigned cluster_x, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+cudaError_t launch_impl(bool coop, dim3 cluster, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                         cudaStream_t st, Args&&... args) {
   Profiler* pr = g_prof;
   const bool timed = pr && g_cls >= 0 && (pr->mask & (1u << g_cls)) && pr->used < Profiler::kCapacity;
@@ -145,11 +147,11 @@ cudaError_t launch_impl(bool coop, unsigned cluster_x, void (*kern)(KArgs...), d
     attr[cfg.numAttrs].val.accessPolicyWindow = g_window;
     ++cfg.numAttrs;
   }
-  if (cluster_x) {
+  if (cluster.x * cluster.y * cluster.z > 1) {
     attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
-    attr[cfg.numAttrs].val.clusterDim.x = cluster_x;
-    attr[cfg.numAttrs].val.clusterDim.y = 1;
-    attr[cfg.numAttrs].val.clusterDim.z = 1;
+    attr[cfg.numAttrs].val.clusterDim.x = cluster.x;
+    attr[cfg.numAttrs].val.clusterDim.y = cluster.y;
+    attr[cfg.numAttrs].val.clusterDim.z = cluster.z;
     ++cfg.numAttrs;
   }
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
@@ -165,7 +167,7 @@ cudaError_t launch_impl(bool coop, unsigned cluster_x, void (*kern)(KArgs...), d
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                    Args&&... args) {
-  return launch_impl(false, 0u, kern, grid, block, smem, st, std::forward<Args>(args)...);
+  return launch_impl(false, dim3(1, 1, 1), kern, grid, block, smem, st, std::forward<Args>(args)...);
 }
 
 constexpr size_t kMaxDynSmem = 220 * 1024;  // budget for dynamic smem per CTA
@@ -217,6 +219,25 @@ cudaError_t init_device_kernels(int dev) {
   if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_ROPE_KV, true>, dev);
   if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_STORE, false>, dev);
   if (e == cudaSuccess) e = allow_max_smem(gemm_int4_tc_kernel<TC_SWIGLU_B, true>, dev);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_attn_tc_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)attn_tc_smem_bytes<128>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_attn_tc_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)attn_tc_smem_bytes<128>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_attn_tc_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)attn_tc_smem_bytes<64>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_attn_tc_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)attn_tc_smem_bytes<64>());
+  if (e == cudaSuccess) e = allow_max_smem(head_direct_kernel, dev);
+  // split-K clusters of up to 16 CTAs
+#define NP(EPI, LO)   \
+  if (e == cudaSuccess) \
+    e = cudaFuncSetAttribute(gemm_int4_tc_kernel<EPI, LO>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  NP(TC_RESID, true) NP(TC_RAW, true) NP(TC_ROPE_KV, true) NP(TC_STORE, false) NP(TC_SWIGLU_B, true)
+#undef NP
 #define ATT(HD, REP)                                                                  \
   if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, true>, dev);   \
   if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, false>, dev);  \
@@ -458,6 +479,41 @@ size_t tc_bt_bytes(int T, int K, bool lo) {
   return (size_t)((T + kTcTokens - 1) / kTcTokens) * (K / 128) * tc_b_bytes(lo);
 }
 
+using TcKernel = void (*)(const TcGemmArgs);
+constexpr int kTcMaxCluster = 16;   // non-portable cluster size limit
+
+// Whether `clusters` clusters of S CTAs of a GEMM variant can be resident on
+// the current device at once (cached per device, kernel and S).
+bool tc_clusters_fit(TcKernel kern, int S, int clusters, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const auto key = std::make_tuple(dev, (const void*)kern, S);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(1, 1, S);
+    lc.blockDim = dim3(kTcThreads);
+    lc.dynamicSmemBytes = smem;
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeClusterDimension;
+    la[0].val.clusterDim.x = 1;
+    la[0].val.clusterDim.y = 1;
+    la[0].val.clusterDim.z = S;
+    lc.attrs = la;
+    lc.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &lc) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    it = cache.emplace(key, n).first;
+  }
+  return it->second >= clusters;
+}
+
 cudaError_t launch_prep(int mode, const PrepArgs& p, cudaStream_t st) {
   if (mode == PREP_NONE) return cudaSuccess;
   const dim3 g(((p.T + kTcTokens - 1) / kTcTokens) * kTcTokens), b(256);
@@ -484,21 +540,37 @@ cudaError_t launch_tc_linear(const uint8_t* wtc, const uint2* sz, int K, int N, 
   if (e != cudaSuccess) return e;
   const int G = K / 128;
   const int row_tiles = (N + kTcRows - 1) / kTcRows, tok_tiles = (T + kTcTokens - 1) / kTcTokens;
-  int splits = std::max(1, std::min(G, sc.n_sm / (row_tiles * tok_tiles)));
-  while (splits > 1 && (size_t)splits * row_tiles * tok_tiles * kTcRows * kTcTokens * 4 > sc.partial_bytes) --splits;
   if (row_tiles * tok_tiles > 4096) return cudaErrorInvalidValue;
+  TcKernel kern = nullptr;
+  if (epi == TC_RESID && lo) kern = gemm_int4_tc_kernel<TC_RESID, true>;
+  else if (epi == TC_RAW && lo) kern = gemm_int4_tc_kernel<TC_RAW, true>;
+  else if (epi == TC_ROPE_KV && lo) kern = gemm_int4_tc_kernel<TC_ROPE_KV, true>;
+  else if (epi == TC_STORE && !lo) kern = gemm_int4_tc_kernel<TC_STORE, false>;
+  else if (epi == TC_SWIGLU_B && lo) kern = gemm_int4_tc_kernel<TC_SWIGLU_B, true>;
+  else return cudaErrorInvalidValue;
+  const size_t smem = tc_smem_bytes(lo);
+  // Split K when the tiles alone leave SMs idle.  Preferred: the splits of a
+  // tile run as one thread-block cluster and reduce in distributed shared
+  // memory (as many splits as keep every cluster resident in one wave);
+  // otherwise partial sums go to global scratch and a merge kernel adds them.
+  int splits = std::max(1, std::min(G, sc.n_sm / (row_tiles * tok_tiles)));
+  bool cluster = false;
+  if (splits > 1) {
+    int S = std::min(splits, kTcMaxCluster);
+    while (S > 1 && !tc_clusters_fit(kern, S, row_tiles * tok_tiles, smem)) --S;
+    if (S > 1) {
+      splits = S;
+      cluster = true;
+    }
+  }
+  if (!cluster)
+    while (splits > 1 && (size_t)splits * row_tiles * tok_tiles * kTcRows * kTcTokens * 4 > sc.partial_bytes) --splits;
   ta.wtc = wtc; ta.sz = sz; ta.K = K; ta.N = N; ta.n16_tiles = n16_tiles;
-  ta.bt = b_tiles ? b_tiles : sc.bt; ta.T = T; ta.splits = splits;
+  ta.bt = b_tiles ? b_tiles : sc.bt; ta.T = T; ta.splits = splits; ta.cluster = cluster ? 1 : 0;
   ta.partial = sc.partial; ta.tickets = sc.tickets; ta.err_flag = sc.err_flag;
   const dim3 g(row_tiles, tok_tiles, splits), b(kTcThreads);
-  const size_t smem = tc_smem_bytes(lo);
-  if (epi == TC_RESID && lo) e = launch(gemm_int4_tc_kernel<TC_RESID, true>, g, b, smem, st, ta);
-  else if (epi == TC_RAW && lo) e = launch(gemm_int4_tc_kernel<TC_RAW, true>, g, b, smem, st, ta);
-  else if (epi == TC_ROPE_KV && lo) e = launch(gemm_int4_tc_kernel<TC_ROPE_KV, true>, g, b, smem, st, ta);
-  else if (epi == TC_STORE && !lo) e = launch(gemm_int4_tc_kernel<TC_STORE, false>, g, b, smem, st, ta);
-  else if (epi == TC_SWIGLU_B && lo) e = launch(gemm_int4_tc_kernel<TC_SWIGLU_B, true>, g, b, smem, st, ta);
-  else return cudaErrorInvalidValue;
-  if (e != cudaSuccess || splits == 1) return e;
+  e = launch_impl(false, cluster ? dim3(1, 1, splits) : dim3(1, 1, 1), kern, g, b, smem, st, ta);
+  if (e != cudaSuccess || splits == 1 || cluster) return e;
   const dim3 mg(row_tiles, tok_tiles, kTcTokens / kTcMergeTok);
   if (epi == TC_RESID) return launch(tc_merge_kernel<TC_RESID>, mg, dim3(256), 0, st, ta);
   if (epi == TC_RAW) return launch(tc_merge_kernel<TC_RAW>, mg, dim3(256), 0, st, ta);
@@ -522,13 +594,27 @@ cudaError_t launch_decode_attn(const DecodeAttnArgs& a, int rows, int hd, int re
   return cudaErrorInvalidValue;
 }
 
+constexpr int kAtMinTokens = 32;   // prefill attention on tcgen05 from this many queries
+
 cudaError_t launch_prefill_attn(PrefillAttnArgs a, int B, int hd, int rep, bool f32, cudaStream_t st) {
-  // query heads per CTA: the whole group, halved while the grid would leave
-  // SMs idle (short prompts); each CTA stages its kv head's keys itself
+  a.rep = rep;
+  if (a.T >= kAtMinTokens) {
+    // tensor cores (tcgen05): one CTA per (128-query tile, query head, batch entry)
+    const dim3 grid((a.T + kAtQ - 1) / kAtQ, a.Hkv * rep, B);
+    if (hd == 128)
+      return f32 ? launch(prefill_attn_tc_kernel<128, true>, grid, dim3(kAtThreads), attn_tc_smem_bytes<128>(), st, a)
+                 : launch(prefill_attn_tc_kernel<128, false>, grid, dim3(kAtThreads), attn_tc_smem_bytes<128>(), st, a);
+    if (hd == 64)
+      return f32 ? launch(prefill_attn_tc_kernel<64, true>, grid, dim3(kAtThreads), attn_tc_smem_bytes<64>(), st, a)
+                 : launch(prefill_attn_tc_kernel<64, false>, grid, dim3(kAtThreads), attn_tc_smem_bytes<64>(), st, a);
+    return cudaErrorInvalidValue;
+  }
+  // short passes (decode-sized verify / append chunks): 16-query tiles on
+  // mma.sync; query heads per CTA: the whole group, halved while the grid
+  // would leave SMs idle; each CTA stages its kv head's keys itself
   int hpc = rep;
   const int qtiles = (a.T + 15) / 16;
   while (hpc > 1 && (long)qtiles * (a.Hkv * rep / hpc) * B < 148) hpc /= 2;
-  a.rep = rep;
   const dim3 grid(qtiles, a.Hkv * rep / hpc, B);
   const size_t smem = prefill_attn_smem_bytes(hd);
 #define C(HD, REP)                                                                                       \
@@ -574,6 +660,7 @@ struct tl_model {
   int* err_flag = nullptr;
   int32_t* spec_tok = nullptr;    // speculative decode / early exit tokens [2 kMaxLanes + 2]
   int head_grid = 0;
+  int hd_grid = 0;                // CTAs of the direct-load head (one per SM)
   HeadIO* io = nullptr;          // output pointers of the current decode step
   TcScratch tc;                  // tensor-core GEMM scratch (prefill)
   cudaAccessPolicyWindow loop_window = {};  // keeps the loop block's weights in L2
@@ -789,9 +876,9 @@ tl_status run_qkv_attn(tl_model* m, int layer, int M, const RowCtx* rows, cudaSt
     const size_t smem = qa_layout(c.d_model, a.M, a.rep, c.head_dim).total;
     const dim3 grid(kQaCluster, c.n_kv_heads);
     if (c.head_dim == 64)
-      TL_CUDA(launch_impl(false, (unsigned)kQaCluster, qkv_attn_kernel<64>, grid, dim3(kQaThreads), smem, st, a));
+      TL_CUDA(launch_impl(false, dim3(kQaCluster, 1, 1), qkv_attn_kernel<64>, grid, dim3(kQaThreads), smem, st, a));
     else
-      TL_CUDA(launch_impl(false, (unsigned)kQaCluster, qkv_attn_kernel<128>, grid, dim3(kQaThreads), smem, st, a));
+      TL_CUDA(launch_impl(false, dim3(kQaCluster, 1, 1), qkv_attn_kernel<128>, grid, dim3(kQaThreads), smem, st, a));
   }
   return TL_OK;
 }
@@ -891,30 +978,19 @@ tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
 tl_status launch_head(tl_model* m, const float* x, int M, const int* out_row, float* logits,
                       int32_t* argmax, cudaStream_t st, const HeadIO* io = nullptr) {
   const tl_config& c = m->cfg;
-  if (m->fused_ok && M <= kFusedMaxRows) {
-    // the persistent step kernel in head-only mode: one CTA per SM streams
-    // its head tiles through a bulk-copy ring (15 compute warps)
-    FusedArgs f = m->fused;
-    f.head_only = 1;
-    f.bar_extra = 0;   // the wait test applies to full fused steps only
-    f.M = M;
-    f.x = const_cast<float*>(x);
-    for (int i = 0; i < M; ++i) f.out_row[i] = i;
-    f.out_row_dev = out_row;
-    f.io = io;
-    f.logits = logits;
-    f.argmax = argmax;
-    f.trace = m->trace;   // head-only timeline: start, staged, tiles done, end
-    f.trace_cap = m->trace_cap;
-    size_t smem = 0;
-    if (fused_plan(m, M, &f, &smem)) {
-      kclass(TL_KERNEL_HEAD);
-      if (c.head_dim == 64)
-        TL_CUDA(launch(decode_fused_kernel<64>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
-      else
-        TL_CUDA(launch(decode_fused_kernel<128>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
-      return TL_OK;
-    }
+  if (M <= kHdMaxRows) {
+    // one CTA per SM; each warp streams whole head tiles with direct loads
+    HeadArgs ha{};
+    ha.io = io;
+    ha.w = m->head_w; ha.V = c.vocab; ha.d = c.d_model;
+    ha.x = x; ha.gain = m->out_norm; ha.eps = c.rms_eps; ha.M = M;
+    ha.out_row = out_row; ha.logits = logits; ha.argmax = argmax;
+    ha.part_val = m->head_val; ha.part_idx = m->head_idx; ha.ticket = m->head_ticket();
+    ha.err_flag = m->err_flag;
+    kclass(TL_KERNEL_HEAD);
+    TL_CUDA(launch(head_direct_kernel, dim3(m->hd_grid), dim3(kHdThreads), head_direct_smem(c.d_model), st, ha,
+                   m->trace, m->trace_cap));
+    return TL_OK;
   }
   HeadArgs ha{};
   ha.io = io;
@@ -964,6 +1040,7 @@ tl_status forward_tokens(tl_model* m, int lane, const int32_t* d_tokens, int T, 
     pa.kv_bstride = 0; pa.ctx = c.max_ctx;
     pa.T = T; pa.pos0 = pos0; pa.Hkv = c.n_kv_heads;
     pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
+    pa.err_flag = m->err_flag;
     if (tc) {   // straight into the O projection's B tiles
       pa.bt = m->tc.bt;
       pa.bt_groups = qdim / 128;
@@ -1099,6 +1176,8 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n_sm < 1) n_sm = 148;
     // one CTA per SM, never more CTAs than head tiles
     m->head_grid = std::min(n_sm, c.vocab / 16);
+    m->hd_grid = n_sm;
+    m->fused_grid = n_sm;   // one CTA per SM; also the timeline's entries per slot
     m->tc.n_sm = n_sm;
   }
   size_t ws = 0;
@@ -1113,8 +1192,9 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
             alloc((void**)&m->tok_index, kMaxLanes * 4) && alloc((void**)&m->out_row, kMaxLanes * 4) &&
             alloc((void**)&m->attn_part, (size_t)kMaxLanes * c.n_kv_heads * kDecodeMaxSplits * rep * (hd + kPartPad) * 4) &&
             alloc((void**)&m->tickets, (size_t)(kMaxLanes * c.n_kv_heads + 1) * 4) &&
-            alloc((void**)&m->head_val, (size_t)m->head_grid * 16 * 4) &&
-            alloc((void**)&m->head_idx, (size_t)m->head_grid * 16 * 4) && alloc((void**)&m->err_flag, 4) &&
+            alloc((void**)&m->head_val, (size_t)std::max(m->head_grid, m->hd_grid) * 16 * 4) &&
+            alloc((void**)&m->head_idx, (size_t)std::max(m->head_grid, m->hd_grid) * 16 * 4) &&
+            alloc((void**)&m->err_flag, 4) &&
             alloc((void**)&m->spec_tok, (2 * kMaxLanes + 2) * 4) &&
             alloc((void**)&m->io, sizeof(HeadIO));
   if (ok) {
@@ -1341,9 +1421,9 @@ tl_status decode_impl(tl_model* m, int n_lanes, const int32_t* h_lane_ids, const
     if (!fused_plan(m, n_lanes, &f, &smem)) return fail(TL_ERR_UNSUPPORTED, "single-kernel decode: no shared-memory plan");
     kclass(TL_KERNEL_DECODE_FUSED);
     if (c.head_dim == 64)
-      TL_CUDA(launch_impl(true, 0u, decode_fused_kernel<64>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
+      TL_CUDA(launch_impl(true, dim3(1, 1, 1), decode_fused_kernel<64>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
     else
-      TL_CUDA(launch_impl(true, 0u, decode_fused_kernel<128>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
+      TL_CUDA(launch_impl(true, dim3(1, 1, 1), decode_fused_kernel<128>, dim3(m->fused_grid), dim3(kFusedThreads), smem, st, f));
     for (int i = 0; i < n_lanes; ++i) m->lane_len[h_lane_ids[i]] += 1;
     return TL_OK;
   }
@@ -1552,6 +1632,7 @@ tl_status tl_score_early_exit(tl_model* m, const int32_t* d_tokens, int n_tokens
     pa.kv_bstride = 0; pa.ctx = c.max_ctx;
     pa.T = T; pa.pos0 = 0; pa.Hkv = c.n_kv_heads;
     pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
+    pa.err_flag = m->err_flag;
     if (tc) {
       pa.bt = m->tc.bt;
       pa.bt_groups = qdim / 128;
@@ -1931,6 +2012,7 @@ tl_status tl_op_gqa_prefill(const uint16_t* d_q, const uint16_t* d_k, const uint
   a.oh = reinterpret_cast<__half*>(d_out);
   a.o_bstride = (long long)T * qdim;
   a.ldo = qdim;
+  a.err_flag = op_err_flag(dev);
   TL_CUDA(launch_prefill_attn(a, B, head_dim, n_q_heads / n_kv_heads, false, (cudaStream_t)stream));
   return TL_OK;
 }
