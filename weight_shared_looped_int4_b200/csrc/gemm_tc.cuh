@@ -201,6 +201,17 @@ struct TcGemmArgs {
   int perm_F;            // interleaved gate/up rows (the scales are looked up by original row)
   uint8_t* bt_out;       // the down projection's B tiles
   int bt_out_groups;     // its K / 128
+  // RMSNorm hand-off between consecutive GEMMs (prefill).  Producer side
+  // (TC_RESID): besides the residual, write the next GEMM's B tiles of
+  // x * g_next (fp16 hi / lo) and, per token, this row tile's sum of x^2.
+  uint8_t* bt_next;      // [token tiles][K/128][2 atoms][256 rows][128 B], K = N of this GEMM
+  const __half* g_next;  // [N] gains of the next RMSNorm
+  float* ss_out;         // [row tiles][ss_ld] sums of squares
+  // Consumer side: every output of token t is scaled by
+  // rsqrt(sum_p ss_in[p][t] / ss_k + eps) (the RMSNorm of its B rows).
+  const float* ss_in;    // [ss_parts][ss_ld], or NULL
+  int ss_parts, ss_ld;
+  float ss_k, ss_eps;
   int cluster;           // 1: the splits of a tile form a thread-block cluster and
                          // reduce in distributed shared memory (no partial buffer)
   float* partial;        // [splits][row tiles][token tiles][128 tokens][128 rows]
@@ -211,15 +222,49 @@ struct TcGemmArgs {
 // Final epilogue of `ntok` tokens of token tile tt (tile-local tokens tok0 ..
 // tok0 + ntok - 1) of row tile `tile`, whose sums are xch[ntok][kTcRows] in
 // shared memory; threads tid = 0 .. nthr - 1 share the work.
+// rs_tok: per tile-local token factor applied to every value first (the
+// consumer side of the RMSNorm hand-off), or NULL.
 template <int EPI>
 __device__ void tc_epilogue_tokens(const TcGemmArgs& a, const float* xch, int tile, int tt, int tok0, int ntok,
-                                   int tid, int nthr) {
+                                   int tid, int nthr, const float* rs_tok = nullptr) {
+  if (EPI == TC_RESID && a.bt_next) {
+    // one warp per token: the new residual of the tile's 128 rows, the next
+    // GEMM's B tile entries of x * g_next and the token's sum of x^2 here
+    const int warp = tid >> 5, lane = tid & 31, nw = nthr >> 5;
+    const int grp = tile;   // this row tile is one K group of the next GEMM
+    for (int ti = warp; ti < ntok; ti += nw) {
+      const int tl_ = tok0 + ti, t = tt * kTcTokens + tl_;
+      if (t >= a.T) continue;   // warp-uniform
+      const float f = rs_tok ? rs_tok[tl_] : 1.f;
+      float ss = 0.f;
+      uint8_t* blk = a.bt_next + ((size_t)tt * (a.N / kTcRows) + grp) * (2 * kTcTokens * 256);
+#pragma unroll
+      for (int pr = 0; pr < 2; ++pr) {
+        const int r = (lane + 32 * pr) * 2;   // rows r, r + 1
+        const int n = tile * kTcRows + r;
+        float2* xo = reinterpret_cast<float2*>(a.out_f32 + (size_t)t * a.ld_out + n);
+        float2 xv = *xo;
+        xv.x += xch[ti * kTcRows + r] * f;
+        xv.y += xch[ti * kTcRows + r + 1] * f;
+        *xo = xv;
+        ss += xv.x * xv.x + xv.y * xv.y;
+        const float2 gv = __half22float2(*reinterpret_cast<const __half2*>(a.g_next + n));
+        uint32_t hw, lw;
+        split_h2(xv.x * gv.x, xv.y * gv.y, hw, lw);
+        *reinterpret_cast<uint32_t*>(blk + sw128_offset(tl_, r, 2 * kTcTokens)) = hw;
+        *reinterpret_cast<uint32_t*>(blk + sw128_offset(kTcTokens + tl_, r, 2 * kTcTokens)) = lw;
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) a.ss_out[(size_t)tile * a.ss_ld + t] = ss;
+    }
+    return;
+  }
   if (EPI == TC_RESID || EPI == TC_RAW || EPI == TC_STORE) {
     for (int item = tid; item < ntok * kTcRows; item += nthr) {
       const int ti = item / kTcRows, r = item % kTcRows;
       const int t = tt * kTcTokens + tok0 + ti, n = tile * kTcRows + r;
       if (t >= a.T || n >= a.N) continue;
-      const float v = xch[ti * kTcRows + r];
+      const float v = xch[ti * kTcRows + r] * (rs_tok ? rs_tok[tok0 + ti] : 1.f);
       const size_t o = (size_t)t * a.ld_out + n;
       if (EPI == TC_RESID) a.out_f32[o] += v;
       else if (EPI == TC_RAW) a.out_f32[o] = v;
@@ -231,7 +276,9 @@ __device__ void tc_epilogue_tokens(const TcGemmArgs& a, const float* xch, int ti
       const int tq = tok0 + ti;
       if (tt * kTcTokens + tq >= a.T) continue;
       const float* xr = xch + ti * kTcRows;
-      tc_swiglu_store(a.bt_out, a.bt_out_groups, tt, tile, tq, j, xr[j], xr[j + 1], xr[64 + j], xr[65 + j]);
+      const float f = rs_tok ? rs_tok[tq] : 1.f;
+      tc_swiglu_store(a.bt_out, a.bt_out_groups, tt, tile, tq, j, xr[j] * f, xr[j + 1] * f, xr[64 + j] * f,
+                      xr[65 + j] * f);
     }
   } else {
     const int hd = a.hd, hh = hd / 2;
@@ -243,7 +290,8 @@ __device__ void tc_epilogue_tokens(const TcGemmArgs& a, const float* xch, int ti
       const int t = tt * kTcTokens + tok0 + ti;
       const int na = tile * kTcRows + r_a;
       if (t >= a.T || na >= a.N) continue;
-      const float va = xch[ti * kTcRows + r_a], vb = xch[ti * kTcRows + r_b];
+      const float f = rs_tok ? rs_tok[tok0 + ti] : 1.f;
+      const float va = xch[ti * kTcRows + r_a] * f, vb = xch[ti * kTcRows + r_b] * f;
       const int pos = a.pos0 + t;
       if (na < a.n_q_rows) {
         const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
@@ -266,6 +314,21 @@ __device__ void tc_epilogue_tokens(const TcGemmArgs& a, const float* xch, int ti
   }
 }
 
+// Consumer side of the RMSNorm hand-off: rs[i] for the tile-local tokens
+// i = tid, tid + nthr, ... of token tile tt (1 where no sums are given).
+__device__ __forceinline__ void tc_token_scales(const TcGemmArgs& a, int tt, float* rs, int tid, int nthr) {
+  for (int i = tid; i < kTcTokens; i += nthr) {
+    float f = 1.f;
+    const int t = tt * kTcTokens + i;
+    if (a.ss_in && t < a.T) {
+      float tot = 0.f;
+      for (int p = 0; p < a.ss_parts; ++p) tot += a.ss_in[(size_t)p * a.ss_ld + t];
+      f = 1.0f / sqrtf(tot / a.ss_k + a.ss_eps);
+    }
+    rs[i] = f;
+  }
+}
+
 // Split-K reduction inside the thread-block cluster that holds the splits of
 // one (row tile, token tile): each rank's partial tile P [128 tokens][128
 // rows] fp32 sits at the start of its shared memory; rank r sums tokens
@@ -273,7 +336,7 @@ __device__ void tc_epilogue_tokens(const TcGemmArgs& a, const float* xch, int ti
 // deterministic -- into a slice buffer behind P and applies the epilogue.
 // Called by all threads of every CTA of the cluster.
 template <int EPI>
-__device__ void tc_cluster_reduce(const TcGemmArgs& a, unsigned char* smem, int tile, int tt) {
+__device__ void tc_cluster_reduce(const TcGemmArgs& a, unsigned char* smem, int tile, int tt, const float* rs_tok) {
   const int S = a.splits;
   cluster_sync_all();   // every rank's partial tile is complete
   const int r = (int)cluster_rank();
@@ -296,7 +359,7 @@ __device__ void tc_cluster_reduce(const TcGemmArgs& a, unsigned char* smem, int 
     *reinterpret_cast<float4*>(xs + ti * kTcRows + r4) = sum;
   }
   __syncthreads();
-  tc_epilogue_tokens<EPI>(a, xs, tile, tt, tok0, ntok, threadIdx.x, kTcThreads);
+  tc_epilogue_tokens<EPI>(a, xs, tile, tt, tok0, ntok, threadIdx.x, kTcThreads, rs_tok);
   cluster_sync_all();   // no rank leaves while another still reads its partial tile
 }
 
@@ -317,6 +380,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   __shared__ uint32_t s_tmem;
   __shared__ int s_last;
   __shared__ int s_fail;
+  __shared__ float s_rs[kTcTokens];   // per-token factor (RMSNorm hand-off), 1 without it
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, tt = blockIdx.y, split = blockIdx.z;
@@ -506,8 +570,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     // ---- split-K: partial sums to scratch, merged by tc_merge_kernel --------
     const int n = tile * kTcRows + row;
     const int t0 = tt * kTcTokens + half * 64;
+    const int etid = threadIdx.x - kTcEpiWarp0 * 32;
+    tc_token_scales(a, tt, s_rs, etid, kTcEpiThreads);
     epi_sync(kTcEpiThreads);
     const bool failed = s_fail != 0;
+    // the direct epilogue below writes from registers; the hand-off needs
+    // whole token rows, so it goes through shared memory like RoPE / SwiGLU
+    const bool via_smem = a.bt_next || a.ss_in;
     if (a.splits > 1 && a.cluster) {
       // partial tile into this CTA's shared memory (the operand stages are
       // idle: the last MMA has completed), reduced across the cluster below
@@ -526,7 +595,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     epi_sync(kTcEpiThreads);
 
     // ---- final epilogue -----------------------------------------------------
-    if (!failed && s_last) {
+    if (!failed && s_last && via_smem) {
+      float* xch = reinterpret_cast<float*>(smem);   // [128 tokens][128 rows]
+#pragma unroll
+      for (int i = 0; i < 64; ++i) xch[(half * 64 + i) * kTcRows + row] = acc[i];
+      epi_sync(kTcEpiThreads);
+      tc_epilogue_tokens<EPI>(a, xch, tile, tt, 0, kTcTokens, etid, kTcEpiThreads, s_rs);
+    } else if (!failed && s_last) {
       if (EPI == TC_RESID || EPI == TC_RAW || EPI == TC_STORE) {
         if (n < a.N) {
 #pragma unroll
@@ -597,7 +672,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   // ---- teardown: every role reaches here; TMEM is always freed -----------
   tc_fence_before();
   __syncthreads();
-  if (a.splits > 1 && a.cluster) tc_cluster_reduce<EPI>(a, smem, tile, tt);
+  if (a.splits > 1 && a.cluster) tc_cluster_reduce<EPI>(a, smem, tile, tt, s_rs);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -642,13 +717,15 @@ __global__ void repack_int4_tc_kernel(const uint32_t* __restrict__ qweight, cons
 constexpr int kTcMergeTok = 8;
 template <int EPI>
 __global__ void __launch_bounds__(256) tc_merge_kernel(const TcGemmArgs a) {
-  __shared__ float xch[kTcMergeTok][kTcRows];
+  __shared__ __align__(16) float xch[kTcMergeTok][kTcRows];
+  __shared__ float s_rs[kTcTokens];
   const int tile = blockIdx.x, tt = blockIdx.y, slice = blockIdx.z;
   const int row_tiles = gridDim.x, tok_tiles = gridDim.y;
   const int tl_ = threadIdx.x >> 5, r4 = (threadIdx.x & 31) * 4;   // token in the slice, 4 rows
   const int tok = slice * kTcMergeTok + tl_;                       // token within the tile
   pdl_trigger();
   pdl_wait();
+  tc_token_scales(a, tt, s_rs, threadIdx.x, 256);
   float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
   const size_t split_stride = (size_t)row_tiles * tok_tiles * kTcTokens * kTcRows;
   const float* base = a.partial + ((size_t)tile * tok_tiles + tt) * (kTcTokens * kTcRows) + (size_t)tok * kTcRows + r4;
@@ -665,66 +742,9 @@ __global__ void __launch_bounds__(256) tc_merge_kernel(const TcGemmArgs a) {
       }
     }
   }
-  const int t = tt * kTcTokens + tok;
-  if (EPI == TC_SWIGLU_B) {
-    *reinterpret_cast<float4*>(&xch[tl_][r4]) = sum;
-    __syncthreads();
-    for (int item = threadIdx.x; item < kTcMergeTok * 32; item += 256) {
-      const int ti = item >> 5, j = (item & 31) * 2;
-      const int tq = slice * kTcMergeTok + ti;      // token within the tile
-      if (tt * kTcTokens + tq >= a.T) continue;
-      tc_swiglu_store(a.bt_out, a.bt_out_groups, tt, tile, tq, j, xch[ti][j], xch[ti][j + 1], xch[ti][64 + j],
-                      xch[ti][65 + j]);
-    }
-    return;
-  }
-  if (EPI == TC_RESID || EPI == TC_RAW || EPI == TC_STORE) {
-    const float vals[4] = {sum.x, sum.y, sum.z, sum.w};
-    if (t < a.T) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int n = tile * kTcRows + r4 + i;
-        if (n < a.N) {
-          const size_t o = (size_t)t * a.ld_out + n;
-          if (EPI == TC_RESID) a.out_f32[o] += vals[i];
-          else if (EPI == TC_RAW) a.out_f32[o] = vals[i];
-          else a.out_f16[o] = __float2half_rn(vals[i]);
-        }
-      }
-    }
-  } else {
-    *reinterpret_cast<float4*>(&xch[tl_][r4]) = sum;
-    __syncthreads();
-    const int hd = a.hd, hh = hd / 2;
-    const int pairs = kTcRows / 2;
-    for (int item = threadIdx.x; item < kTcMergeTok * pairs; item += 256) {
-      const int ti = item / pairs, pr = item % pairs;
-      const int head_local = pr / hh, j = pr % hh;
-      const int r_a = head_local * hd + j, r_b = r_a + hh;
-      const int tq = tt * kTcTokens + slice * kTcMergeTok + ti;
-      const int na = tile * kTcRows + r_a;
-      if (tq >= a.T || na >= a.N) continue;
-      const float va = xch[ti][r_a], vb = xch[ti][r_b];
-      const int pos = a.pos0 + tq;
-      if (na < a.n_q_rows) {
-        const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
-        float* qo = a.q_out + (size_t)tq * a.ldq;
-        qo[na] = va * cs.x - vb * cs.y;
-        qo[na + hh] = vb * cs.x + va * cs.y;
-      } else if (na < a.n_q_rows + a.n_kv_rows) {
-        const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
-        const int kvh = (na - a.n_q_rows) / hd;
-        __half* dst = a.k_plane + ((size_t)kvh * a.ctx + pos) * hd;
-        dst[j] = __float2half_rn(va * cs.x - vb * cs.y);
-        dst[j + hh] = __float2half_rn(vb * cs.x + va * cs.y);
-      } else {
-        const int kvh = (na - a.n_q_rows - a.n_kv_rows) / hd;
-        __half* dst = a.v_plane + ((size_t)kvh * a.ctx + pos) * hd;
-        dst[j] = __float2half_rn(va);
-        dst[j + hh] = __float2half_rn(vb);
-      }
-    }
-  }
+  *reinterpret_cast<float4*>(&xch[tl_][r4]) = sum;
+  __syncthreads();
+  tc_epilogue_tokens<EPI>(a, &xch[0][0], tile, tt, slice * kTcMergeTok, kTcMergeTok, threadIdx.x, 256, s_rs);
 }
 
 // ---- activation preparation ---------------------------------------------

@@ -465,6 +465,10 @@ __global__ void fill_rows_kernel(RowCtx* rows, int n, int lane, int pos0) {
 struct TcScratch {
   uint8_t* bt = nullptr;       // prepared activation tiles
   uint8_t* bt2 = nullptr;      // the down projection's tiles, written by the gate_up epilogue
+  uint8_t* bt3 = nullptr;      // gate_up's tiles (x * ffn gains), written by the O epilogue
+  float* ss_attn = nullptr;    // per (d row tile, token) sums of x^2 for the next attention RMSNorm
+  float* ss_ffn = nullptr;     // ... for the FFN RMSNorm
+  int ss_ld = 0;               // tokens per row of ss_*
   size_t bt_bytes = 0;
   float* partial = nullptr;    // split-K partial tiles
   size_t partial_bytes = 0;
@@ -706,7 +710,8 @@ struct tl_model {
     graphs.clear();
     if (cap_stream) cudaStreamDestroy(cap_stream);
     void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row, spec_tok,
-                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.bt2, tc.partial, tc.tickets,
+                    attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.bt2, tc.bt3, tc.ss_attn,
+                    tc.ss_ffn, tc.partial, tc.tickets,
                     rope_tab, fused_bar, fused_val, fused_idx};
     for (void* p : ptrs)
       if (p) cudaFree(p);
@@ -926,49 +931,70 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
 
 // Prefill forms of run_qkv / run_ffn on the tensor cores (positions
 // pos0..pos0+T-1 of one lane).
+// RMSNorm hand-off: for layer > 0 the previous layer's down projection has
+// already written this layer's B tiles (x * attn gains) and the per-token
+// sums of squares, so the QKV GEMM scales each token by its norm factor in
+// the epilogue instead of running a prep kernel; the O projection does the
+// same for the FFN's norm.
 tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, int pos0, cudaStream_t st) {
   WindowScope window_scope(m, layer);
   const tl_config& c = m->cfg;
   const BlockDev& b = m->block(layer);
   const int hd = c.head_dim, qdim = c.n_q_heads * hd;
+  const bool handed = layer > 0;
   PrepArgs pa{};
   pa.x = m->x; pa.ldx = c.d_model; pa.gain = b.attn_norm; pa.eps = c.rms_eps;
   TcGemmArgs ta{};
+  if (handed) {
+    ta.ss_in = m->tc.ss_attn; ta.ss_parts = c.d_model / kTcRows; ta.ss_ld = m->tc.ss_ld;
+    ta.ss_k = (float)c.d_model; ta.ss_eps = c.rms_eps;
+  }
   ta.q_out = m->q; ta.ldq = qdim; ta.n_q_rows = qdim; ta.n_kv_rows = c.n_kv_heads * hd; ta.hd = hd;
   ta.k_plane = m->k_plane(layer) + lane * m->lane_stride;
   ta.v_plane = m->v_plane(layer) + lane * m->lane_stride;
   ta.ctx = c.max_ctx; ta.pos0 = pos0; ta.theta = c.rope_theta; ta.rope_tab = m->rope_tab;
   kclass(TL_KERNEL_GEMM_TC);
-  TL_CUDA(launch_tc_linear(b.qkv.tc, b.qkv.sz, c.d_model, b.qkv.N, b.qkv.n_tiles, PREP_NORM, pa, ta, TC_ROPE_KV,
-                           T, m->tc, st));
+  TL_CUDA(launch_tc_linear(b.qkv.tc, b.qkv.sz, c.d_model, b.qkv.N, b.qkv.n_tiles, handed ? PREP_NONE : PREP_NORM,
+                           pa, ta, TC_ROPE_KV, T, m->tc, st));
   return TL_OK;
 }
 
-tl_status run_ffn_tc(tl_model* m, int layer, int T, cudaStream_t st) {
+// O + residual, gate_up + SwiGLU, down + residual of `layer`; the down
+// projection also hands the next layer's attention RMSNorm over when
+// `next_layer` >= 0 (its gains).
+tl_status run_ffn_tc(tl_model* m, int layer, int T, int next_layer, cudaStream_t st) {
   WindowScope window_scope(m, layer);
   const tl_config& c = m->cfg;
   const BlockDev& b = m->block(layer);
   const int d = c.d_model, F = c.ffn_dim, qdim = c.n_q_heads * c.head_dim;
   kclass(TL_KERNEL_GEMM_TC);
-  {  // O projection + residual (the prefill attention wrote its B tiles)
+  {  // O projection + residual (the prefill attention wrote its B tiles);
+     // hands the FFN RMSNorm over to gate_up
     PrepArgs pa{};
     TcGemmArgs ta{};
     ta.out_f32 = m->x; ta.ld_out = d;
+    ta.bt_next = m->tc.bt3; ta.g_next = b.ffn_norm; ta.ss_out = m->tc.ss_ffn; ta.ss_ld = m->tc.ss_ld;
     TL_CUDA(launch_tc_linear(b.o.tc, b.o.sz, qdim, d, b.o.n_tiles, PREP_NONE, pa, ta, TC_RESID, T, m->tc, st));
   }
-  {  // RMSNorm + gate_up; its epilogue writes silu(gate) * up as the down
-     // projection's B tiles (the tensor-core rows interleave gate and up)
+  {  // gate_up (B = x * ffn gains, each token scaled by its norm factor);
+     // its epilogue writes silu(gate) * up as the down projection's B tiles
+     // (the tensor-core rows interleave gate and up)
     PrepArgs pa{};
-    pa.x = m->x; pa.ldx = d; pa.gain = b.ffn_norm; pa.eps = c.rms_eps;
     TcGemmArgs ta{};
+    ta.ss_in = m->tc.ss_ffn; ta.ss_parts = d / kTcRows; ta.ss_ld = m->tc.ss_ld;
+    ta.ss_k = (float)d; ta.ss_eps = c.rms_eps;
     ta.perm_F = F; ta.bt_out = m->tc.bt2; ta.bt_out_groups = F / 128;
-    TL_CUDA(launch_tc_linear(b.gate_up.tc, b.gate_up.sz, d, 2 * F, b.gate_up.n_tiles, PREP_NORM, pa, ta,
-                             TC_SWIGLU_B, T, m->tc, st));
+    TL_CUDA(launch_tc_linear(b.gate_up.tc, b.gate_up.sz, d, 2 * F, b.gate_up.n_tiles, PREP_NONE, pa, ta,
+                             TC_SWIGLU_B, T, m->tc, st, m->tc.bt3));
   }
-  {  // down + residual
+  {  // down + residual (+ the next layer's attention RMSNorm hand-off)
     PrepArgs pa{};
     TcGemmArgs ta{};
     ta.out_f32 = m->x; ta.ld_out = d;
+    if (next_layer >= 0) {
+      ta.bt_next = m->tc.bt; ta.g_next = m->block(next_layer).attn_norm; ta.ss_out = m->tc.ss_attn;
+      ta.ss_ld = m->tc.ss_ld;
+    }
     TL_CUDA(launch_tc_linear(b.down.tc, b.down.sz, F, d, b.down.n_tiles, PREP_NONE, pa, ta, TC_RESID, T, m->tc, st,
                              m->tc.bt2));
   }
@@ -1047,7 +1073,8 @@ tl_status forward_tokens(tl_model* m, int lane, const int32_t* d_tokens, int T, 
     }
     kclass(TL_KERNEL_ATTN_PREFILL);
     TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
-    rc = tc ? run_ffn_tc(m, layer, T, st) : run_ffn(m, layer, T, m->x, m->o, m->h, st);
+    rc = tc ? run_ffn_tc(m, layer, T, layer + 1 < n_layers ? layer + 1 : -1, st)
+            : run_ffn(m, layer, T, m->x, m->o, m->h, st);
     if (rc != TL_OK) return rc;
     if ((out.lens_logits || out.lens_argmax) && layer >= c.n_pre) {
       const int i = layer - c.n_pre;   // loop iteration i + 1 done
@@ -1202,7 +1229,11 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     m->tc.bt_bytes = tc_bt_bytes(rows, kmax, true);
     m->tc.partial_bytes = (size_t)160 * kTcRows * kTcTokens * 4;
     m->tc.err_flag = m->err_flag;
+    m->tc.ss_ld = (rows + kTcTokens - 1) / kTcTokens * kTcTokens;
+    const size_t ss_bytes = (size_t)(d / kTcRows) * m->tc.ss_ld * 4;
     ok = alloc((void**)&m->tc.bt, m->tc.bt_bytes) && alloc((void**)&m->tc.bt2, m->tc.bt_bytes) &&
+         alloc((void**)&m->tc.bt3, m->tc.bt_bytes) && alloc((void**)&m->tc.ss_attn, ss_bytes) &&
+         alloc((void**)&m->tc.ss_ffn, ss_bytes) &&
          alloc((void**)&m->tc.partial, m->tc.partial_bytes) &&
          alloc((void**)&m->tc.tickets, 4096 * sizeof(unsigned)) &&
          alloc((void**)&m->rope_tab, (size_t)c.max_ctx * (hd / 2) * sizeof(float2));
@@ -1639,7 +1670,8 @@ tl_status tl_score_early_exit(tl_model* m, const int32_t* d_tokens, int n_tokens
     }
     kclass(TL_KERNEL_ATTN_PREFILL);
     TL_CUDA(launch_prefill_attn(pa, 1, c.head_dim, c.n_q_heads / c.n_kv_heads, true, st));
-    rc = tc ? run_ffn_tc(m, layer, T, st) : run_ffn(m, layer, T, m->x, m->o, m->h, st);
+    rc = tc ? run_ffn_tc(m, layer, T, layer + 1 < c.n_pre + max_loops ? layer + 1 : -1, st)
+            : run_ffn(m, layer, T, m->x, m->o, m->h, st);
     if (rc != TL_OK) return rc;
     if (layer < c.n_pre) continue;
     // output norm + head after this iteration; stop once the greedy token
