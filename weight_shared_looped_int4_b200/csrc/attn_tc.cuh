@@ -5,23 +5,28 @@
 // the tiny-llm feature list.
 //
 // Design (ours, sm_100a):
-// * One CTA per (128-query tile, query head, batch entry); 8 warps.  The
-//   queries are the MMA rows (M = 128): S = Q K^T over a block of 64 keys
-//   (N = 64) and O_blk = P V (N = head_dim), both into TMEM.
+// * One CTA per (128-query tile, query head, batch entry).  The queries are
+//   the MMA rows (M = 128): S = Q K^T over a block of 64 keys (N = 64) and
+//   O_j = P_j V_j (N = head_dim), both in TMEM, double-buffered.
 // * Q (fp32 or fp16 in memory) is scaled by 1/sqrt(hd) and split into an fp16
 //   pair (hi, lo); S accumulates Q_hi K^T + Q_lo K^T.  P is split the same
-//   way and O_blk accumulates P_hi V + P_lo V.  K and V are fp16 already, so
+//   way and O_j accumulates P_hi V + P_lo V.  K and V are fp16 already, so
 //   the products keep ~fp32 accuracy (as the other attention kernels).
-// * Operands in shared memory, 128-byte swizzled: Q and P K-major (rows of
-//   64 consecutive k), K K-major (a key's head dims are the MMA's K), V
-//   MN-major (a key's head dims are the MMA's N: 64-wide dim chunks LBO apart,
-//   groups of 8 keys SBO apart), so K and V rows are copied as they lie in the
-//   cache, 16 bytes per cp.async, double-buffered one block ahead.
-// * Softmax: warp w reads TMEM lanes 32 (w % 4) .. (its query rows) and half
-//   w / 4 of the columns; the two warps of a row exchange the row maximum and
-//   sum through shared memory.  The online rescaling is applied to the
-//   running output held in registers (O_acc = O_acc c + O_blk), so TMEM never
-//   needs a read-modify-write.
+// * Operands in shared memory, 128-byte swizzled: Q and P K-major, K K-major
+//   (a key's head dims are the MMA's K), V MN-major (a key's head dims are
+//   the MMA's N: 64-wide dim chunks LBO apart, groups of 8 keys SBO apart),
+//   so K and V rows are copied as they lie in the cache.
+// * Warp roles, all handing over through mbarriers, so loads, MMAs, softmax
+//   and the output update of different key blocks overlap:
+//     warp 0       one lane issues the MMAs: S_j, then O_{j-1} (the softmax of
+//                  block j runs while O_{j-1} is computed);
+//     warp 1       loads K/V blocks (cp.async, completion tracked by an
+//                  mbarrier), two blocks ahead;
+//     warps 2-5    softmax: one thread per query row reads its 64 scores from
+//                  TMEM, masks, keeps the running max / sum, writes P (hi, lo)
+//                  and the rescale factor of the block;
+//     warps 6-9    output: one thread per query row keeps O in registers and
+//                  applies O = O c_j + O_j as each O_j lands in TMEM.
 // * Every mbarrier wait is bounded; a CTA that gives up records kErrTimeout
 //   and still frees its TMEM.
 #pragma once
@@ -34,7 +39,9 @@ namespace tl {
 
 constexpr int kAtQ = 128;        // queries per CTA (MMA M)
 constexpr int kAtKeys = 64;      // keys per block (MMA N of S, K of P V)
-constexpr int kAtThreads = 256;  // 8 warps
+constexpr int kAtWarps = 10;
+constexpr int kAtThreads = kAtWarps * 32;
+constexpr int kAtSoftWarp0 = 2, kAtOutWarp0 = 6;
 
 // Shared-memory plan (bytes) for head_dim HD.
 template <int HD>
@@ -47,8 +54,8 @@ struct AtLayout {
   static constexpr int q_hi = 0, q_lo = Q_BYTES;
   static constexpr int k0 = 2 * Q_BYTES;                   // [2 buffers]
   static constexpr int v0 = k0 + 2 * K_BYTES;              // [2 buffers]
-  static constexpr int p_hi = v0 + 2 * V_BYTES, p_lo = p_hi + P_BYTES;
-  static constexpr int total = p_lo + P_BYTES;
+  static constexpr int p0 = v0 + 2 * V_BYTES;              // [2 buffers][hi, lo]
+  static constexpr int total = p0 + 4 * P_BYTES;
 };
 template <int HD>
 __host__ __device__ constexpr size_t attn_tc_smem_bytes() {
@@ -72,70 +79,52 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(const void* p, uint32_t l
 __host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
   return idesc_f16_f32(M, N) | (1u << 16);
 }
+// Arrive on `bar` once all of this thread's earlier cp.async copies landed.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 template <int HD, bool F32>
 __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const PrefillAttnArgs a) {
   using Lay = AtLayout<HD>;
   constexpr int KA = Lay::KA;
-  constexpr int HALF = HD / 2;                 // output columns per warp
   extern __shared__ __align__(128) unsigned char at_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(at_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t mma_bar;
+  __shared__ __align__(8) uint64_t kv_full[2], s_full[2], p_full[2], o_full[2], o_empty[2], blk_done[2];
   __shared__ uint32_t s_tmem;
   __shared__ int s_fail;
-  __shared__ float x_max[2][kAtQ], x_sum[2][kAtQ];
+  __shared__ float cfac[2][kAtQ];   // rescale factor of block j for each row
+  __shared__ float lfin[kAtQ];      // final row sums
 
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int quad = warp & 3, ch = warp >> 2;   // TMEM lane quarter, column half
-  const int r = quad * 32 + lane;              // this thread's query row in the tile
   const int kvh = h / a.rep;
   const int q0 = qt * kAtQ;
-  const int t_row = q0 + r;                    // token of the row
-  const int pos = a.pos0 + t_row;              // its position (keys 0..pos)
   const int last_key = a.pos0 + min(q0 + kAtQ - 1, a.T - 1);
   const int nblk = last_key / kAtKeys + 1;
   const __half* kp = a.k + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
   const __half* vp = a.v + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
 
   if (warp == 0) {
-    tmem_alloc(&s_tmem, 256);
+    tmem_alloc(&s_tmem, 512);
     tmem_relinquish();
   }
   if (threadIdx.x == 32) {
-    mbar_init(&mma_bar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&kv_full[i], 32);          // the loader warp's lanes (cp.async completion)
+      mbar_init(&s_full[i], 1);            // tcgen05.commit
+      mbar_init(&p_full[i], 128);          // softmax threads
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 128);         // output threads
+      mbar_init(&blk_done[i], 1);
+    }
     fence_mbar_init();
     s_fail = 0;
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = s_tmem;
-  const uint32_t t_s = tmem, t_o = tmem + 128;   // S: 64 columns, O_blk: HD columns
   pdl_trigger();
   pdl_wait();
 
-  // ---- K / V block j into buffer j % 2 (cp.async, zeros past last_key) ----
-  auto load_kv = [&](int j) {
-    unsigned char* ks = sm + Lay::k0 + (j & 1) * Lay::K_BYTES;
-    unsigned char* vs = sm + Lay::v0 + (j & 1) * Lay::V_BYTES;
-    const int j0 = j * kAtKeys;
-    for (int c = threadIdx.x; c < kAtKeys * HD / 8; c += kAtThreads) {
-      const int key = c / (HD / 8), c16 = c % (HD / 8);       // 16-byte chunk of the key's row
-      const bool ok = j0 + key <= last_key;
-      const size_t src = ok ? (size_t)(j0 + key) * HD + c16 * 8 : 0;
-      const int atom = c16 >> 3, j16 = c16 & 7;
-      // K: K-major, [atom][64 keys][128 B]
-      cp_async16(ks + atom * kAtKeys * 128 + key * 128 + ((j16 ^ (key & 7)) << 4), kp + src, ok ? 16 : 0);
-      // V: MN-major, [dim chunk][8-key group][8 keys][128 B]
-      cp_async16(vs + atom * (kAtKeys * 128) + (key >> 3) * 1024 + (key & 7) * 128 + ((j16 ^ (key & 7)) << 4),
-                 vp + src, ok ? 16 : 0);
-    }
-    cp_async_commit();
-  };
-  load_kv(0);
-
-  // ---- Q tile: scale, split into (hi, lo), K-major swizzled ----------------
+  // ---- Q tile (all threads): scale, split into (hi, lo), K-major swizzled --
   {
     const float scale = 1.0f / sqrtf((float)HD);
     for (int c = threadIdx.x; c < kAtQ * HD / 8; c += kAtThreads) {
@@ -171,149 +160,198 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
       *reinterpret_cast<uint4*>(sm + Lay::q_lo + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
   }
-
-  float o_acc[HALF];
-#pragma unroll
-  for (int i = 0; i < HALF; ++i) o_acc[i] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
-  unsigned phase = 0;
-  const uint32_t idesc_s = idesc_f16_f32(kAtQ, kAtKeys);
-  const uint32_t idesc_o = idesc_f16_f32_bmn(kAtQ, HD);
-
-  for (int j = 0; j < nblk; ++j) {
-    if (j + 1 < nblk) {
-      load_kv(j + 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    fence_proxy_async_smem();   // cp.async / st.shared writes -> the tensor core's reads
-    __syncthreads();
-    const unsigned char* ks = sm + Lay::k0 + (j & 1) * Lay::K_BYTES;
-    const unsigned char* vs = sm + Lay::v0 + (j & 1) * Lay::V_BYTES;
-    // ---- S = Q_hi K^T + Q_lo K^T ---------------------------------------------
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        const unsigned char* qs = sm + (pass ? Lay::q_lo : Lay::q_hi);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const int atom = kk >> 2, within = (kk & 3) * 32;
-          const uint64_t ad = sw128_kmajor_desc(qs + atom * kAtQ * 128 + within);
-          const uint64_t bd = sw128_kmajor_desc(ks + atom * kAtKeys * 128 + within);
-          tc_mma_f16(t_s, ad, bd, idesc_s, (pass | kk) ? 1u : 0u);
-        }
-      }
-      tc_commit(&mma_bar);
-    }
-    mbar_wait_or_fail(&mma_bar, phase, &s_fail);
-    phase ^= 1u;
-    tc_fence_after();
-    // ---- softmax of this thread's 32 scores (row r, keys ch*32 ..) ----------
-    float s[32];
-    {
-      uint32_t raw[32];
-      tmem_ld32(t_s + ((uint32_t)(quad * 32) << 16) + ch * 32, raw);
-      tmem_ld_wait();
-      const int k0 = j * kAtKeys + ch * 32;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) s[i] = (k0 + i <= pos) ? __uint_as_float(raw[i]) : -INFINITY;
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) mx = fmaxf(mx, s[i]);
-    x_max[ch][r] = mx;
-    __syncthreads();
-    const float m_new = fmaxf(m_run, fmaxf(mx, x_max[ch ^ 1][r]));
-    const float c = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
-    float sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      s[i] = (m_new == -INFINITY || s[i] == -INFINITY) ? 0.f : expf(s[i] - m_new);
-      sum += s[i];
-    }
-    m_run = m_new;
-    x_sum[ch][r] = sum;
-    // P (hi, lo) of keys ch*32 .. ch*32+31 of row r: 16-byte chunks 4 ch .. 4 ch + 3
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) split_h2(s[q * 8 + 2 * i], s[q * 8 + 2 * i + 1], hw[i], lw[i]);
-      const int j16 = ch * 4 + q;
-      const int o = r * 128 + ((j16 ^ (r & 7)) << 4);
-      *reinterpret_cast<uint4*>(sm + Lay::p_hi + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(sm + Lay::p_lo + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    l_run = l_run * c + sum + x_sum[ch ^ 1][r];
-    // ---- O_blk = P_hi V + P_lo V ---------------------------------------------
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int pass = 0; pass < 2; ++pass) {
-        const unsigned char* ps = sm + (pass ? Lay::p_lo : Lay::p_hi);
-#pragma unroll
-        for (int kk = 0; kk < kAtKeys / 16; ++kk) {
-          const uint64_t ad = sw128_kmajor_desc(ps + kk * 32);
-          const uint64_t bd = sw128_mnmajor_desc(vs + kk * 2 * 1024, kAtKeys * 128, 1024);
-          tc_mma_f16(t_o, ad, bd, idesc_o, (pass | kk) ? 1u : 0u);
-        }
-      }
-      tc_commit(&mma_bar);
-    }
-    mbar_wait_or_fail(&mma_bar, phase, &s_fail);
-    phase ^= 1u;
-    tc_fence_after();
-    // ---- O_acc = O_acc c + O_blk (row r, columns ch * HALF ..) ---------------
-#pragma unroll
-    for (int c0 = 0; c0 < HALF; c0 += 32) {
-      uint32_t raw[32];
-      tmem_ld32(t_o + ((uint32_t)(quad * 32) << 16) + ch * HALF + c0, raw);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o_acc[c0 + i] = fmaf(o_acc[c0 + i], c, __uint_as_float(raw[i]));
-    }
-    tc_fence_before();
-    __syncthreads();   // S / O_blk / P / this K-V buffer are free for the next block
-  }
-
-  // ---- normalise and store row r, columns ch * HALF .. --------------------
-  if (t_row < a.T) {
-    const float inv = 1.f / l_run;
-    if (F32 && a.bt) {
-      const int tt = t_row / kTcTokensB, tl_ = t_row % kTcTokensB;
-#pragma unroll
-      for (int i = 0; i < HALF; i += 2) {
-        const int k = h * HD + ch * HALF + i;   // column of the O projection's input
-        const int grp = k >> 7, kg = k & 127;
-        uint32_t hw, lw;
-        split_h2(o_acc[i] * inv, o_acc[i + 1] * inv, hw, lw);
-        uint8_t* blk = a.bt + ((size_t)tt * a.bt_groups + grp) * (2 * kTcTokensB * 256);
-        *reinterpret_cast<uint32_t*>(blk + sw128_offset(tl_, kg, 2 * kTcTokensB)) = hw;
-        *reinterpret_cast<uint32_t*>(blk + sw128_offset(kTcTokensB + tl_, kg, 2 * kTcTokensB)) = lw;
-      }
-    } else {
-      const size_t off = b * a.o_bstride + (size_t)t_row * a.ldo + (size_t)h * HD + ch * HALF;
-#pragma unroll
-      for (int i = 0; i < HALF; i += 2) {
-        if (F32) {
-          *reinterpret_cast<float2*>(a.of + off + i) = make_float2(o_acc[i] * inv, o_acc[i + 1] * inv);
-        } else {
-          *reinterpret_cast<uint32_t*>(a.oh + off + i) = pack_h2(o_acc[i] * inv, o_acc[i + 1] * inv);
-        }
-      }
-    }
-  }
-  if (threadIdx.x == 0 && s_fail && a.err_flag) atomicOr(a.err_flag, kErrTimeout);
+  fence_proxy_async_smem();   // Q (st.shared) -> the tensor core's reads
   tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  auto t_s = [&](int buf) { return tmem + (uint32_t)(buf * 64); };          // S_j: 64 columns
+  auto t_o = [&](int buf) { return tmem + 128u + (uint32_t)(buf * 128); };  // O_j: HD columns
+
+  if (warp == 0) {
+    // ---- MMA issue --------------------------------------------------------
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_f16_f32(kAtQ, kAtKeys);
+      const uint32_t idesc_o = idesc_f16_f32_bmn(kAtQ, HD);
+      auto issue_o = [&](int j) {   // O_j = P_j V_j into O buffer j % 2
+        const int bb = j & 1;
+        mbar_wait_or_fail(&p_full[bb], (unsigned)(j >> 1) & 1u, &s_fail);
+        if (j >= 2) mbar_wait_or_fail(&o_empty[bb], (unsigned)((j - 2) >> 1) & 1u, &s_fail);
+        tc_fence_after();
+        const unsigned char* vs = sm + Lay::v0 + bb * Lay::V_BYTES;
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+          const unsigned char* ps = sm + Lay::p0 + (bb * 2 + pass) * Lay::P_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kAtKeys / 16; ++kk) {
+            const uint64_t ad = sw128_kmajor_desc(ps + kk * 32);
+            const uint64_t bd = sw128_mnmajor_desc(vs + kk * 2 * 1024, kAtKeys * 128, 1024);
+            tc_mma_f16(t_o(bb), ad, bd, idesc_o, (pass | kk) ? 1u : 0u);
+          }
+        }
+        tc_commit(&o_full[bb]);
+        tc_commit(&blk_done[bb]);   // K_j, V_j and P_j are no longer read
+      };
+      for (int j = 0; j < nblk; ++j) {
+        const int bb = j & 1;
+        mbar_wait_or_fail(&kv_full[bb], (unsigned)(j >> 1) & 1u, &s_fail);
+        fence_proxy_async_smem();   // the cp.async data -> the tensor core's reads
+        // S buffer bb was last read by the softmax of block j - 2
+        if (j >= 2) mbar_wait_or_fail(&p_full[bb], (unsigned)((j - 2) >> 1) & 1u, &s_fail);
+        tc_fence_after();
+        const unsigned char* ks = sm + Lay::k0 + bb * Lay::K_BYTES;
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+          const unsigned char* qs = sm + (pass ? Lay::q_lo : Lay::q_hi);
+#pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            const int atom = kk >> 2, within = (kk & 3) * 32;
+            const uint64_t ad = sw128_kmajor_desc(qs + atom * kAtQ * 128 + within);
+            const uint64_t bd = sw128_kmajor_desc(ks + atom * kAtKeys * 128 + within);
+            tc_mma_f16(t_s(bb), ad, bd, idesc_s, (pass | kk) ? 1u : 0u);
+          }
+        }
+        tc_commit(&s_full[bb]);
+        if (j >= 1) issue_o(j - 1);
+      }
+      issue_o(nblk - 1);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---- K / V loader: block j into buffer j % 2 (zeros past last_key) ----
+    for (int j = 0; j < nblk; ++j) {
+      const int bb = j & 1;
+      if (j >= 2) mbar_wait_or_fail(&blk_done[bb], (unsigned)((j - 2) >> 1) & 1u, &s_fail);
+      unsigned char* ks = sm + Lay::k0 + bb * Lay::K_BYTES;
+      unsigned char* vs = sm + Lay::v0 + bb * Lay::V_BYTES;
+      const int j0 = j * kAtKeys;
+      for (int c = lane; c < kAtKeys * HD / 8; c += 32) {
+        const int key = c / (HD / 8), c16 = c % (HD / 8);
+        const bool ok = j0 + key <= last_key;
+        const size_t src = ok ? (size_t)(j0 + key) * HD + c16 * 8 : 0;
+        const int atom = c16 >> 3, j16 = c16 & 7;
+        cp_async16(ks + atom * kAtKeys * 128 + key * 128 + ((j16 ^ (key & 7)) << 4), kp + src, ok ? 16 : 0);
+        cp_async16(vs + atom * (kAtKeys * 128) + (key >> 3) * 1024 + (key & 7) * 128 + ((j16 ^ (key & 7)) << 4),
+                   vp + src, ok ? 16 : 0);
+      }
+      cp_async_mbar_arrive(&kv_full[bb]);
+    }
+    cp_async_wait<0>();   // nothing of this warp in flight at exit
+  } else if (warp < kAtOutWarp0) {
+    // ---- softmax: thread = query row r ---------------------------------------
+    const int quad = warp & 3, r = quad * 32 + lane;
+    const int pos = a.pos0 + q0 + r;
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int j = 0; j < nblk; ++j) {
+      const int bb = j & 1;
+      mbar_wait_or_fail(&s_full[bb], (unsigned)(j >> 1) & 1u, &s_fail);
+      tc_fence_after();
+      float s[64];
+      {
+        uint32_t raw[32];
+        const int k0 = j * kAtKeys;
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          tmem_ld32(t_s(bb) + ((uint32_t)(quad * 32) << 16) + c0, raw);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c0 + i] = (k0 + c0 + i <= pos) ? __uint_as_float(raw[i]) : -INFINITY;
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
+      const float m_new = fmaxf(m_run, mx);
+      const float c = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        s[i] = (m_new == -INFINITY || s[i] == -INFINITY) ? 0.f : expf(s[i] - m_new);
+        sum += s[i];
+      }
+      m_run = m_new;
+      l_run = l_run * c + sum;
+      // P buffer bb was last read by O_{j-2}, cfac[bb] by the output warps'
+      // update of block j - 2
+      if (j >= 2) {
+        mbar_wait_or_fail(&blk_done[bb], (unsigned)((j - 2) >> 1) & 1u, &s_fail);
+        mbar_wait_or_fail(&o_empty[bb], (unsigned)((j - 2) >> 1) & 1u, &s_fail);
+      }
+      unsigned char* ph = sm + Lay::p0 + (bb * 2) * Lay::P_BYTES;
+      unsigned char* pl = ph + Lay::P_BYTES;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split_h2(s[q * 8 + 2 * i], s[q * 8 + 2 * i + 1], hw[i], lw[i]);
+        const int o = r * 128 + ((q ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(ph + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(pl + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      cfac[bb][r] = c;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[bb]);
+    }
+    lfin[r] = l_run;
+  } else {
+    // ---- output: thread = query row r, O kept in registers ------------------
+    const int quad = warp & 3, r = quad * 32 + lane;
+    float o_acc[HD];
+#pragma unroll
+    for (int i = 0; i < HD; ++i) o_acc[i] = 0.f;
+    for (int j = 0; j < nblk; ++j) {
+      const int bb = j & 1;
+      // cfac of block j first: p_full cannot move on to block j + 2 before
+      // this warp releases o_empty for block j, so the phase is unambiguous
+      mbar_wait_or_fail(&p_full[bb], (unsigned)(j >> 1) & 1u, &s_fail);
+      mbar_wait_or_fail(&o_full[bb], (unsigned)(j >> 1) & 1u, &s_fail);
+      tc_fence_after();
+      const float c = cfac[bb][r];
+#pragma unroll
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        uint32_t raw[32];
+        tmem_ld32(t_o(bb) + ((uint32_t)(quad * 32) << 16) + c0, raw);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o_acc[c0 + i] = fmaf(o_acc[c0 + i], c, __uint_as_float(raw[i]));
+      }
+      tc_fence_before();
+      mbar_arrive(&o_empty[bb]);
+    }
+    asm volatile("bar.sync 1, 256;" ::: "memory");   // softmax (lfin) and output warps
+    const int t_row = q0 + r;
+    if (t_row < a.T) {
+      const float inv = 1.f / lfin[r];
+      if (F32 && a.bt) {
+        const int tt = t_row / kTcTokensB, tl_ = t_row % kTcTokensB;
+#pragma unroll
+        for (int i = 0; i < HD; i += 2) {
+          const int k = h * HD + i;   // column of the O projection's input
+          const int grp = k >> 7, kg = k & 127;
+          uint32_t hw, lw;
+          split_h2(o_acc[i] * inv, o_acc[i + 1] * inv, hw, lw);
+          uint8_t* blk = a.bt + ((size_t)tt * a.bt_groups + grp) * (2 * kTcTokensB * 256);
+          *reinterpret_cast<uint32_t*>(blk + sw128_offset(tl_, kg, 2 * kTcTokensB)) = hw;
+          *reinterpret_cast<uint32_t*>(blk + sw128_offset(kTcTokensB + tl_, kg, 2 * kTcTokensB)) = lw;
+        }
+      } else {
+        const size_t off = b * a.o_bstride + (size_t)t_row * a.ldo + (size_t)h * HD;
+#pragma unroll
+        for (int i = 0; i < HD; i += 2) {
+          if (F32) *reinterpret_cast<float2*>(a.of + off + i) = make_float2(o_acc[i] * inv, o_acc[i + 1] * inv);
+          else *reinterpret_cast<uint32_t*>(a.oh + off + i) = pack_h2(o_acc[i] * inv, o_acc[i + 1] * inv);
+        }
+      }
+    }
+  }
+  if (warp >= kAtSoftWarp0 && warp < kAtOutWarp0) asm volatile("bar.arrive 1, 256;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && s_fail && a.err_flag) atomicOr(a.err_flag, kErrTimeout);
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
