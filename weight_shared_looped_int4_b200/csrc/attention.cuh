@@ -138,11 +138,19 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
 
   const __half* kp = a.k + rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;
   const __half* vp = a.v + rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;
+  // keys first, values in a second group: the scores and the softmax run
+  // while the values are still arriving
   for (int c = threadIdx.x; c < CHUNKS; c += kDecodeThreads) {
     const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
     const bool ok = key < nk;
     const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
     cp_async16(ks + key * LDK + off, kp + src, ok ? 16 : 0);
+  }
+  cp_async_commit();
+  for (int c = threadIdx.x; c < CHUNKS; c += kDecodeThreads) {
+    const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
+    const bool ok = key < nk;
+    const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
     cp_async16(vs + key * LDK + off, vp + src, ok ? 16 : 0);
   }
   cp_async_commit();
@@ -166,7 +174,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
     split_h2(v0.x * scale, v0.y * scale, qa[c][0], ql[c][0]);
     split_h2(v1.x * scale, v1.y * scale, qa[c][1], ql[c][1]);
   }
-  cp_async_wait<0>();
+  cp_async_wait<1>();   // the keys
   __syncthreads();
 
   // S for keys kb .. kb+15 of this warp (two n8 tiles) -> shared memory
@@ -211,6 +219,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
     sum = warp_sum(sum);
     if (lane == 0) { s_m[h] = mx; s_l[h] = sum; }
   }
+  cp_async_wait<0>();   // the values
   __syncthreads();
 
   // O = P V: warp w takes output dims 8w .. 8w+7 over all keys of the split
