@@ -79,10 +79,6 @@ __device__ __forceinline__ uint64_t sw128_mnmajor_desc(const void* p, uint32_t l
 __host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
   return idesc_f16_f32(M, N) | (1u << 16);
 }
-// Arrive on `bar` once all of this thread's earlier cp.async copies landed.
-__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 
 template <int HD, bool F32>
 __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const PrefillAttnArgs a) {
@@ -234,7 +230,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
         cp_async16(vs + atom * (kAtKeys * 128) + (key >> 3) * 1024 + (key & 7) * 128 + ((j16 ^ (key & 7)) << 4),
                    vp + src, ok ? 16 : 0);
       }
-      cp_async_mbar_arrive(&kv_full[bb]);
+      cp_async_mbar_arrive_noinc(&kv_full[bb]);
     }
     cp_async_wait<0>();   // nothing of this warp in flight at exit
   } else if (warp < kAtOutWarp0) {
