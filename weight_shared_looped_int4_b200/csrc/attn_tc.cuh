@@ -8,8 +8,9 @@
 // * One CTA per (128-query tile, query head, batch entry).  The queries are
 //   the MMA rows (M = 128): S = Q K^T over a block of 64 keys (N = 64) and
 //   O_j = P_j V_j (N = head_dim), both in TMEM, double-buffered.
-// * Q (fp32 or fp16 in memory) is scaled by 1/sqrt(hd) and split into an fp16
-//   pair (hi, lo); S accumulates Q_hi K^T + Q_lo K^T.  P is split the same
+// * Q (fp32 or fp16 in memory) is scaled by log2(e)/sqrt(hd) (the softmax
+//   runs in base 2) and split into an fp16 pair (hi, lo); S accumulates
+//   Q_hi K^T + Q_lo K^T.  P is split the same
 //   way and O_j accumulates P_hi V + P_lo V.  K and V are fp16 already, so
 //   the products keep ~fp32 accuracy (as the other attention kernels).
 // * Operands in shared memory, 128-byte swizzled: Q and P K-major, K K-major
@@ -119,33 +120,71 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
   }
   pdl_trigger();
   pdl_wait();
+  __syncthreads();   // barriers initialised before the loader arrives on them
 
-  // ---- Q tile (all threads): scale, split into (hi, lo), K-major swizzled --
+  // ---- K / V block j into buffer j % 2 (cp.async, zeros past last_key) ----
+  auto load_kv = [&](int j) {
+    const int bb = j & 1;
+    unsigned char* ks = sm + Lay::k0 + bb * Lay::K_BYTES;
+    unsigned char* vs = sm + Lay::v0 + bb * Lay::V_BYTES;
+    const int j0 = j * kAtKeys;
+    for (int c = lane; c < kAtKeys * HD / 8; c += 32) {
+      const int key = c / (HD / 8), c16 = c % (HD / 8);
+      const bool ok = j0 + key <= last_key;
+      const size_t src = ok ? (size_t)(j0 + key) * HD + c16 * 8 : 0;
+      const int atom = c16 >> 3, j16 = c16 & 7;
+      cp_async16(ks + atom * kAtKeys * 128 + key * 128 + ((j16 ^ (key & 7)) << 4), kp + src, ok ? 16 : 0);
+      cp_async16(vs + atom * (kAtKeys * 128) + (key >> 3) * 1024 + (key & 7) * 128 + ((j16 ^ (key & 7)) << 4),
+                 vp + src, ok ? 16 : 0);
+    }
+    cp_async_mbar_arrive_noinc(&kv_full[bb]);
+  };
+  // the first two blocks go out before the Q tile is staged
+  if (warp == 1)
+    for (int j = 0; j < 2 && j < nblk; ++j) load_kv(j);
+
+  // ---- Q tile (all threads): scale by log2(e) / sqrt(hd) (the softmax works
+  // in base 2), split into (hi, lo), K-major swizzled; every load of a thread
+  // is issued before any is used ------------------------------------------
   {
-    const float scale = 1.0f / sqrtf((float)HD);
-    for (int c = threadIdx.x; c < kAtQ * HD / 8; c += kAtThreads) {
+    constexpr int NQ = (kAtQ * HD / 8 + kAtThreads - 1) / kAtThreads;
+    const float scale = 1.4426950408889634f / sqrtf((float)HD);
+    float4 xv[NQ][2];
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+      const int c = threadIdx.x + u * kAtThreads;
       const int row = c / (HD / 8), c16 = c % (HD / 8);
       const int t = q0 + row;
-      float v[8];
-      if (t < a.T) {
+      xv[u][0] = xv[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c < kAtQ * HD / 8 && t < a.T) {
         const size_t off = b * a.q_bstride + (size_t)t * a.ldq + (size_t)h * HD + c16 * 8;
         if (F32) {
-          const float4 x0 = *reinterpret_cast<const float4*>(a.qf + off);
-          const float4 x1 = *reinterpret_cast<const float4*>(a.qf + off + 4);
-          v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w; v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+          xv[u][0] = *reinterpret_cast<const float4*>(a.qf + off);
+          xv[u][1] = *reinterpret_cast<const float4*>(a.qf + off + 4);
         } else {
           const uint4 raw = *reinterpret_cast<const uint4*>(a.qh + off);
-          const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f = h2_to_f2(w4[i]);
-            v[2 * i] = f.x;
-            v[2 * i + 1] = f.y;
-          }
+          xv[u][0] = *reinterpret_cast<const float4*>(&raw);   // raw fp16 bits, widened below
         }
-      } else {
+      }
+    }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    for (int u = 0; u < NQ; ++u) {
+      const int c = threadIdx.x + u * kAtThreads;
+      if (c >= kAtQ * HD / 8) continue;
+      const int row = c / (HD / 8), c16 = c % (HD / 8);
+      float v[8];
+      if (F32) {
+        v[0] = xv[u][0].x; v[1] = xv[u][0].y; v[2] = xv[u][0].z; v[3] = xv[u][0].w;
+        v[4] = xv[u][1].x; v[5] = xv[u][1].y; v[6] = xv[u][1].z; v[7] = xv[u][1].w;
+      } else {
+        const uint32_t w4[4] = {__float_as_uint(xv[u][0].x), __float_as_uint(xv[u][0].y),
+                                __float_as_uint(xv[u][0].z), __float_as_uint(xv[u][0].w)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = h2_to_f2(w4[i]);
+          v[2 * i] = f.x;
+          v[2 * i + 1] = f.y;
+        }
       }
       uint32_t hw[4], lw[4];
 #pragma unroll
@@ -214,23 +253,10 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- K / V loader: block j into buffer j % 2 (zeros past last_key) ----
-    for (int j = 0; j < nblk; ++j) {
-      const int bb = j & 1;
-      if (j >= 2) mbar_wait_or_fail(&blk_done[bb], (unsigned)((j - 2) >> 1) & 1u, &s_fail);
-      unsigned char* ks = sm + Lay::k0 + bb * Lay::K_BYTES;
-      unsigned char* vs = sm + Lay::v0 + bb * Lay::V_BYTES;
-      const int j0 = j * kAtKeys;
-      for (int c = lane; c < kAtKeys * HD / 8; c += 32) {
-        const int key = c / (HD / 8), c16 = c % (HD / 8);
-        const bool ok = j0 + key <= last_key;
-        const size_t src = ok ? (size_t)(j0 + key) * HD + c16 * 8 : 0;
-        const int atom = c16 >> 3, j16 = c16 & 7;
-        cp_async16(ks + atom * kAtKeys * 128 + key * 128 + ((j16 ^ (key & 7)) << 4), kp + src, ok ? 16 : 0);
-        cp_async16(vs + atom * (kAtKeys * 128) + (key >> 3) * 1024 + (key & 7) * 128 + ((j16 ^ (key & 7)) << 4),
-                   vp + src, ok ? 16 : 0);
-      }
-      cp_async_mbar_arrive_noinc(&kv_full[bb]);
+    // ---- K / V loader: blocks 2 .. into the buffer block j - 2 released ----
+    for (int j = 2; j < nblk; ++j) {
+      mbar_wait_or_fail(&blk_done[j & 1], (unsigned)((j - 2) >> 1) & 1u, &s_fail);
+      load_kv(j);
     }
     cp_async_wait<0>();   // nothing of this warp in flight at exit
   } else if (warp < kAtOutWarp0) {
@@ -257,12 +283,13 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
       float mx = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
+      // scores are in base 2 (Q carries log2(e)): weights 2^(s - m)
       const float m_new = fmaxf(m_run, mx);
-      const float c = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
+      const float c = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_new);
       float sum = 0.f;
 #pragma unroll
       for (int i = 0; i < 64; ++i) {
-        s[i] = (m_new == -INFINITY || s[i] == -INFINITY) ? 0.f : expf(s[i] - m_new);
+        s[i] = (m_new == -INFINITY) ? 0.f : exp2f(s[i] - m_new);   // 2^-inf = 0 for masked keys
         sum += s[i];
       }
       m_run = m_new;

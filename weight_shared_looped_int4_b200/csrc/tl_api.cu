@@ -1833,6 +1833,18 @@ std::map<int, OpWorkspace> g_ws;
 
 // A zeroed per-device fault flag for the op entry points.
 std::map<int, int*> g_op_err;
+// Row descriptors of an op call, passed by value.
+constexpr int kOpRowsPerSetup = 128;
+struct OpRows {
+  int n;
+  RowCtx rows[kOpRowsPerSetup];
+};
+__global__ void op_rows_kernel(OpRows r, RowCtx* out) {
+  pdl_trigger();
+  pdl_wait();
+  if ((int)threadIdx.x < r.n) out[threadIdx.x] = r.rows[threadIdx.x];
+}
+
 int* op_err_flag(int dev) {
   std::lock_guard<std::mutex> lk(g_ws_mu);
   int*& f = g_op_err[dev];
@@ -2000,7 +2012,15 @@ tl_status tl_op_gqa_decode(const uint16_t* d_q, const uint16_t* d_k, const uint1
   RowCtx* d_rows = (RowCtx*)base;
   float* part = (float*)(base + ((rows_b + 255) / 256) * 256);
   cudaStream_t st = (cudaStream_t)stream;
-  TL_CUDA(cudaMemcpyAsync(d_rows, rows.data(), rows_b, cudaMemcpyHostToDevice, st));
+  // the row descriptors travel as kernel arguments (no copy from host memory
+  // that a captured graph would read again, after this call, at replay)
+  for (int b0 = 0; b0 < B; b0 += kOpRowsPerSetup) {
+    OpRows r{};
+    r.n = std::min(kOpRowsPerSetup, B - b0);
+    for (int i = 0; i < r.n; ++i) r.rows[i] = rows[b0 + i];
+    kclass(TL_KERNEL_SETUP);
+    TL_CUDA(launch(op_rows_kernel, dim3(1), dim3(kOpRowsPerSetup), 0, st, r, d_rows + b0));
+  }
   DecodeAttnArgs a{};
   a.qh = reinterpret_cast<const __half*>(d_q);
   a.ldq = n_q_heads * head_dim;
