@@ -876,15 +876,20 @@ def run_workload_attention(args):
                 qd = torch.from_numpy(np.ascontiguousarray(q)).to(dev)
                 out = torch.empty((B, T, HQ, HD), dtype=torch.float16, device=dev)
                 fn = lambda: tl.tl_op_gqa_prefill(qd, kc, vc, HKV * T * HD, T, T, 0, B, HQ, HKV, HD, out, st)
-                for _ in range(3):
-                    fn()
-                cold = _time_reps(torch, st, fn, 20, flush)
-                warm = _time_graph(torch, st, fn, 5, launches=5)
                 flops = B * 4 * HQ * HD * T * (T + 1) / 2
                 t_roof = flops / (peaks["bf16_tflops"] * 1e6)
-                pre.append({"B": B, "T": T, "us_l2_cold": round(1e3 * cold, 2), "us_graph": round(1e3 * warm, 2),
-                            "flops": int(flops), "tflops": round(flops / (min(cold, warm) * 1e9), 2),
-                            "frac": round(t_roof / (1e3 * min(cold, warm)), 4)})
+                rec = {"B": B, "T": T, "flops": int(flops)}
+                for min_tc, kname in ((1, "tcgen05"), (1 << 30, "mma_sync")):
+                    tl.tl_set_prefill_attention_tc_min(min_tc)
+                    for _ in range(3):
+                        fn()
+                    cold = _time_reps(torch, st, fn, 10, flush)
+                    warm = _time_graph(torch, st, fn, 5, launches=5)
+                    best = min(cold, warm)
+                    rec[kname] = {"us_l2_cold": round(1e3 * cold, 2), "us_graph": round(1e3 * warm, 2),
+                                  "tflops": round(flops / (best * 1e9), 2), "frac": round(t_roof / (1e3 * best), 4)}
+                tl.tl_set_prefill_attention_tc_min(512)
+                pre.append(rec)
                 del kc, vc, qd, out
     print(json.dumps({"workload": "GQA attention D2048 16q/4kv hd128 (fp16 KV)",
                       "metric": "per-case us and fraction of roofline", "peaks": peaks,

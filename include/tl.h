@@ -357,6 +357,13 @@ int tl_model_trace_grid(const tl_model *m);
  * the lanes whose caches the invalid step wrote).  Other paths ignore it. */
 tl_status tl_model_set_wait_test(tl_model *m, int extra_arrivals);
 
+/* Measurement and tuning control with no counterpart in the pages: causal
+ * prefill attention (prefill, tl_extend, tl_op_gqa_prefill) runs on the
+ * tcgen05 kernel (128-query tiles, TMEM accumulators) for passes of at least
+ * min_queries queries and on 16-query mma.sync tiles below that.  Process
+ * wide; default 512.  Both kernels compute the same attention. */
+tl_status tl_set_prefill_attention_tc_min(int min_queries);
+
 /* Number of kernels this library has launched in the process so far. */
 unsigned long long tl_kernel_launch_count(void);
 

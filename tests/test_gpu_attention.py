@@ -82,17 +82,25 @@ def _prefill_case(T, B, pos0, hq, hkv, hd, seed, sample=None):
     qpos = torch.arange(pos0, pos0 + T, dtype=torch.int32, device=DEV)
     for b in range(B):
         tl.tl_op_rope(qd[b], T, hq, hd, hq * hd, hd, qpos, THETA)
-    out = torch.empty((B, T, hq, hd), dtype=torch.float16, device=DEV)
-    tl.tl_op_gqa_prefill(qd, kc, vc, hkv * ctx * hd, ctx, T, pos0, B, hq, hkv, hd, out)
-    torch.cuda.synchronize()
-    got = out.cpu().numpy().astype(np.float64)
     rows = np.arange(T) if sample is None else np.asarray(sample)
+    expects = []
     for b in range(B):
         qr = ref.rope(q[b, rows].astype(np.float64), pos0 + rows, THETA)
         kr = ref.rope(k[b].astype(np.float64), np.arange(ctx), THETA)
-        expect = ref.gqa_attention(qr, kr, v[b], pos0 + rows)
-        err = rel_l2(got[b, rows], expect)
-        assert err <= KERNEL_REL_L2, (T, b, err)
+        expects.append(ref.gqa_attention(qr, kr, v[b], pos0 + rows))
+    # both kernels: tcgen05 (128-query tiles) and mma.sync (16-query tiles)
+    try:
+        for min_tc, kernel in ((1, "tcgen05"), (1 << 30, "mma.sync")):
+            tl.tl_set_prefill_attention_tc_min(min_tc)
+            out = torch.empty((B, T, hq, hd), dtype=torch.float16, device=DEV)
+            tl.tl_op_gqa_prefill(qd, kc, vc, hkv * ctx * hd, ctx, T, pos0, B, hq, hkv, hd, out)
+            torch.cuda.synchronize()
+            got = out.cpu().numpy().astype(np.float64)
+            for b in range(B):
+                err = rel_l2(got[b, rows], expects[b])
+                assert err <= KERNEL_REL_L2, (kernel, T, b, err)
+    finally:
+        tl.tl_set_prefill_attention_tc_min(512)
 
 
 @pytest.mark.parametrize("B", [1, 8])
@@ -110,8 +118,7 @@ def test_prefill_attention(T, B):
                                               (50, 77, 16, 4, 128), (130, 5, 8, 8, 64), (65, 0, 8, 1, 128),
                                               (300, 1000, 16, 4, 128)])
 def test_prefill_attention_ragged(T, pos0, hq, hkv, hd):
-    # below 32 queries the 16-query mma.sync kernel runs, from 32 on the
-    # tcgen05 kernel (128-query tiles): ragged tiles, offsets, GQA ratios
+    # both attention kernels: ragged tiles, offsets, GQA ratios
     _prefill_case(T, 2, pos0, hq, hkv, hd, seed=T + pos0)
 
 

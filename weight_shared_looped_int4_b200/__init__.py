@@ -32,7 +32,7 @@ __all__ = [
     "tl_model_set_graphs", "tl_model_set_decode_path", "DECODE_AUTO", "DECODE_LAYERED", "DECODE_FUSED",
     "tl_probe_read_bandwidth", "tl_model_set_trace", "tl_model_trace_grid",
     "tl_model_set_wait_test", "tl_extend", "tl_generate_speculative", "tl_score_logit_lens",
-    "tl_score_early_exit", "tl_lane_fork", "tl_spec_stats",
+    "tl_score_early_exit", "tl_lane_fork", "tl_spec_stats", "tl_set_prefill_attention_tc_min",
     "tl_linear_create", "tl_linear_destroy", "tl_linear_forward",
     "tl_op_rmsnorm", "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill",
     "tl_op_gqa_decode_noalloc",
@@ -107,6 +107,7 @@ def _load():
         "tl_score_logit_lens": (st, [P, P, c_int, c_int, P, P, P]),
         "tl_score_early_exit": (st, [P, P, c_int, c_int, c_int, P, P, POINTER(c_int), P]),
         "tl_lane_fork": (st, [P, c_int, c_int, c_int, P]),
+        "tl_set_prefill_attention_tc_min": (st, [c_int]),
         "tl_probe_read_bandwidth": (st, [P, c_size_t, c_int, P, POINTER(c_double)]),
         "tl_linear_create": (st, [POINTER(tl_int4_linear), c_int, c_int, c_int, POINTER(c_void_p)]),
         "tl_linear_destroy": (None, [P]),
@@ -149,7 +150,7 @@ EXPORTED = sorted(["tl_model_profile_start", "tl_model_profile_stop", "tl_kernel
                    "tl_model_set_graphs", "tl_model_set_decode_path", "tl_probe_read_bandwidth",
                    "tl_model_set_trace", "tl_model_trace_grid", "tl_model_set_wait_test",
                    "tl_extend", "tl_generate_speculative", "tl_score_logit_lens", "tl_score_early_exit",
-                   "tl_lane_fork",
+                   "tl_lane_fork", "tl_set_prefill_attention_tc_min",
                    "tl_model_create", "tl_model_destroy", "tl_prefill", "tl_decode_step",
                    "tl_score_last", "tl_lane_length", "tl_model_info", "tl_check_device_error",
                    "tl_linear_create", "tl_linear_destroy", "tl_linear_forward", "tl_op_rmsnorm",
@@ -299,6 +300,11 @@ def tl_score_early_exit(model, d_tokens, n_tokens, max_loops, stable_n, d_logits
 
 def tl_lane_fork(model, src_lane, dst_lane, n_tokens, stream=None) -> None:
     _check(_L().tl_lane_fork(model, int(src_lane), int(dst_lane), int(n_tokens), _stream(stream)))
+
+
+def tl_set_prefill_attention_tc_min(min_queries: int) -> None:
+    """Prefill attention on tcgen05 from this many queries on (default 512)."""
+    _check(_L().tl_set_prefill_attention_tc_min(int(min_queries)))
 
 
 def tl_lane_length(model, lane) -> int:

@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   }
   if (threadIdx.x == 32) {
     for (int i = 0; i < kTcStages; ++i) {
-      mbar_init(&bar_full[i], kTcUnpack + 32);  // + the copy warp's lanes (cp.async completion)
+      mbar_init(&bar_full[i], kTcUnpack + 1);   // + the copy lane's arrive with the B bytes
       mbar_init(&bar_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -433,7 +433,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
         if (!mbar_wait_or_fail(&bar_full[s], (unsigned)(h / kTcStages) & 1u, &s_fail)) break;
         if (half == 0 && it >= 2 && !mbar_wait_or_fail(&bar_tempty[b], (unsigned)((it - 2) >> 1) & 1u, &s_fail))
           break;
-        fence_proxy_async_smem();   // the B atom came through cp.async (generic proxy)
         tc_fence_after();
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -447,50 +446,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- copies ---------------------------------------------------------------
-    // Lane 0 keeps kTcRaw groups of raw INT4 words and scales/zeros in flight
-    // (bulk copies; the weights do not depend on earlier kernels, so the
-    // first ones go out before the dependency wait).  Each stage's B atom
-    // (32 KB) is copied by all 32 lanes with 16-byte cp.async as soon as the
-    // MMA has released the stage: per SM these stream several times faster
-    // than one lane's 1-D bulk copy.  Each lane's cp.async completion arrives
-    // on the stage's full barrier.
-    int g_issued = 0;
-    auto issue_raw = [&](int it) {
-      const int r = it % kTcRaw, g = gmap(it);
-      mbar_arrive_expect_tx(&raw_full[r], kTcRawBytes);
-      bulk_g2s(sR(r), a.wtc + ((size_t)tile * G + g) * kTcRawBytes, kTcRawBytes, &raw_full[r]);
-    };
-    if (lane == 0)
+    // ---- copy issuer (one lane) ----------------------------------------------
+    // Keeps kTcRaw groups of raw INT4 words and scales/zeros in flight (bulk
+    // copies; the weights do not depend on earlier kernels, so the first ones
+    // go out before the dependency wait) and issues each stage's B atom as
+    // soon as the MMA has released the stage.
+    if (lane == 0) {
+      int g_issued = 0;
+      auto issue_raw = [&](int it) {
+        const int r = it % kTcRaw, g = gmap(it);
+        mbar_arrive_expect_tx(&raw_full[r], kTcRawBytes);
+        bulk_g2s(sR(r), a.wtc + ((size_t)tile * G + g) * kTcRawBytes, kTcRawBytes, &raw_full[r]);
+      };
       for (; g_issued < ng && g_issued < kTcRaw; ++g_issued) issue_raw(g_issued);
-    pdl_wait();
-    bool live = true;
-    for (int h = 0; h < nh; ++h) {
-      const int s = h % kTcStages, it = h >> 1, half = h & 1, g = gmap(it);
-      if (h >= kTcStages && live && !mbar_wait_or_fail(&bar_empty[s], (unsigned)((h / kTcStages) - 1) & 1u, &s_fail))
-        live = false;
-      if (live) {
-        const uint4* src = reinterpret_cast<const uint4*>(a.bt + (((size_t)tt * G + g) * 2 + half) * B_BYTES);
-        unsigned char* dst = sB(s);
-#pragma unroll 4
-        for (int i = lane; i < (int)(B_BYTES / 16); i += 32) cp_async16(dst + i * 16, src + i, 16);
+      pdl_wait();
+      for (int h = 0; h < nh; ++h) {
+        const int s = h % kTcStages, it = h >> 1, half = h & 1, g = gmap(it);
+        if (h >= kTcStages && !mbar_wait_or_fail(&bar_empty[s], (unsigned)((h / kTcStages) - 1) & 1u, &s_fail))
+          break;
+        // arrive with the expected bytes: the stage cannot complete before
+        // this arrival, so the unpackers' arrivals cannot race past the copy
+        mbar_arrive_expect_tx(&bar_full[s], B_BYTES);
+        bulk_g2s(sB(s), a.bt + (((size_t)tt * G + g) * 2 + half) * B_BYTES, B_BYTES, &bar_full[s]);
+        if (half) {
+          // top up the raw ring: group g_issued reuses the slot of g_issued - kTcRaw
+          for (; g_issued < ng && g_issued < it + kTcRaw; ++g_issued)
+            if (mbar_wait_or_fail(&raw_empty[g_issued % kTcRaw], (unsigned)((g_issued / kTcRaw) - 1) & 1u,
+                                  &s_fail))
+              issue_raw(g_issued);
+        }
       }
-      // every lane arrives once per stage, even after a time-out, so the
-      // barrier counts stay consistent
-      cp_async_mbar_arrive_noinc(&bar_full[s]);
-      if (half && lane == 0 && live) {
-        // top up the raw ring: group g_issued reuses the slot of g_issued - kTcRaw
-        for (; g_issued < ng && g_issued < it + kTcRaw; ++g_issued)
-          if (mbar_wait_or_fail(&raw_empty[g_issued % kTcRaw], (unsigned)((g_issued / kTcRaw) - 1) & 1u,
-                                &s_fail))
-            issue_raw(g_issued);
-      }
+      // a CTA that gave up waits (bounded) for its raw copies still in flight
+      if (*reinterpret_cast<volatile int*>(&s_fail))
+        for (int it = g_issued - kTcRaw < 0 ? 0 : g_issued - kTcRaw; it < g_issued; ++it)
+          mbar_wait(&raw_full[it % kTcRaw], (unsigned)(it / kTcRaw) & 1u);
     }
-    cp_async_wait<0>();
-    // a CTA that gave up waits (bounded) for its raw copies still in flight
-    if (lane == 0 && *reinterpret_cast<volatile int*>(&s_fail))
-      for (int it = g_issued - kTcRaw < 0 ? 0 : g_issued - kTcRaw; it < g_issued; ++it)
-        mbar_wait(&raw_full[it % kTcRaw], (unsigned)(it / kTcRaw) & 1u);
     __syncwarp();
   } else if (warp < kTcEpiWarp0) {
     // ---- unpackers: A from the raw ring into the 128-byte swizzled K-major

@@ -20,12 +20,9 @@
 //   count of the small projections.  Partial sums are reduced through shared
 //   memory in a fixed order, so results are deterministic and each activation
 //   row's result does not depend on how many rows share the launch.
-// * Each lane loads its own weight words and scales straight into registers
-//   (16-byte loads, up to kGemvPre chunks ahead) before griddepcontrol.wait,
-//   so the fetch overlaps the tail of the previous kernel under programmatic
-//   dependent launch (the caller picks where the kernel releases its own
-//   dependent: PdlTrigger).  Plain loads stream faster per SM than bulk
-//   copies into shared memory, and the weights never touch shared memory.
+// * Weight prefetch is issued before griddepcontrol.wait, so it overlaps the
+//   tail of the previous kernel under programmatic dependent launch (the
+//   caller picks where the kernel releases its own dependent: PdlTrigger).
 // * fp32 activations are split into an fp16 pair x = hi + lo (lo is the fp16
 //   rounding of x - hi) and both halves go through the MMA, so the product
 //   keeps about 22 bits of the activation instead of fp16's 11.  The looped
@@ -93,17 +90,18 @@ struct GemvArgs {
 
 constexpr int kGemvThreads = 256;
 
-constexpr int kGemvPre = 12;   // 64-k chunks a lane holds in registers
-
-// Shared memory of a CTA: the activation planes (hi, and lo unless IN_F16)
-// of M rows, the K-slice reduction buffer and the RMSNorm partial sums.
+// Shared memory of a CTA: its weight tiles and scales (bulk-copied), the
+// activation planes (hi, and lo unless IN_F16) of M rows, the K-slice
+// reduction buffer and the RMSNorm partial sums.
 __host__ __device__ inline size_t gemv_act_bytes(int K, int M, bool lo) {
   return (((size_t)M * (K + 8) * 2 * (lo ? 2 : 1)) + 15) / 16 * 16;
 }
+__host__ __device__ inline size_t gemv_w_bytes(int K) { return (size_t)(K >> 6) * 512; }
+__host__ __device__ inline size_t gemv_sz_bytes(int K) { return (size_t)(K >> 7) * 64; }
 __host__ __device__ inline size_t gemv_smem_bytes(int K, int M, bool lo, int tpc) {
-  (void)tpc;
   const int nc = M <= 8 ? 8 : 16;
-  return gemv_act_bytes(K, M, lo) + (size_t)8 * 16 * nc * 4 + 16 * 8 * 4;
+  return (size_t)tpc * (gemv_w_bytes(K) + gemv_sz_bytes(K)) + gemv_act_bytes(K, M, lo) +
+         (size_t)8 * 16 * nc * 4 + 16 * 8 * 4;
 }
 
 // Tiles per CTA of each epilogue.
@@ -127,11 +125,16 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   constexpr int NC = NT == 2 ? 16 : 8;        // reduction columns
   constexpr int NTILES = NT == 2 ? 2 : 1;     // n8 tiles of the MMA
   extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t wbar;
+  __shared__ int s_ok;
   const int K = a.K;
   const int M = a.M;
   const int ldxs = K + 8;
   const int n_chunks = K >> 6;
-  __half* xs = reinterpret_cast<__half*>(smem);                   // hi plane [M][ldxs]
+  const size_t wt_bytes = gemv_w_bytes(K), sz_bytes = gemv_sz_bytes(K);
+  unsigned char* sw = smem;                                       // [TPC][chunks][32][16 B]
+  unsigned char* ssz = smem + TPC * wt_bytes;                     // [TPC][groups][8][8 B]
+  __half* xs = reinterpret_cast<__half*>(ssz + TPC * sz_bytes);   // hi plane [M][ldxs]
   __half* xl = xs + (size_t)M * ldxs;                             // lo plane [M][ldxs]
   float* red = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(xs) + gemv_act_bytes(K, M, LO));
   float* ssq = red + 8 * 16 * NC;                                 // [16 rows][8 warps]
@@ -156,21 +159,21 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
 
   trace_start(a.trace);
   if (a.trigger == TRIGGER_AT_START) pdl_trigger();
-  // This warp's chunks of its tile: c_begin .. c_begin + nc - 1.  The weights
-  // do not depend on earlier kernels: the first kGemvPre chunks (words and
-  // scales) are requested before waiting for the previous kernel.
-  const int c_begin = (n_chunks * kq) / KS;
-  const int nc = (n_chunks * (kq + 1)) / KS - c_begin;
-  const int my_tile = tsel ? t1 : t0;
-  const uint4* wsrc = a.w + (size_t)my_tile * n_chunks * 32 + lane;
-  const uint2* ssrc = a.sz + (size_t)my_tile * (K >> 7) * 8 + g;
-  uint4 wr[kGemvPre];
-  uint2 sr[kGemvPre];
-#pragma unroll
-  for (int i = 0; i < kGemvPre; ++i) {
-    if (i < nc) {
-      wr[i] = ldg_stream(wsrc + (size_t)(c_begin + i) * 32);
-      sr[i] = ldg_stream2(ssrc + (size_t)((c_begin + i) >> 1) * 8);
+  // The weights do not depend on earlier kernels: start their bulk copies
+  // before waiting for the previous kernel.
+  if (threadIdx.x == 0) {
+    mbar_init(&wbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&wbar, (unsigned)(TPC * (wt_bytes + sz_bytes)));
+    for (int ts = 0; ts < TPC; ++ts) {
+      const int tile = ts ? t1 : t0;
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
+      for (size_t off = 0; off < wt_bytes; off += 32768) {
+        const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
+        bulk_g2s(sw + ts * wt_bytes + off, src + off, n, &wbar);
+      }
+      bulk_g2s(ssz + ts * sz_bytes, reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes,
+               (unsigned)sz_bytes, &wbar);
     }
   }
 
@@ -282,11 +285,20 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
       }
     }
   }
-  if (threadIdx.x == 0) trace_mark(a.trace, 6);
+  if (threadIdx.x == 0) {
+    trace_mark(a.trace, 6);
+    s_ok = mbar_wait(&wbar, 0) ? 1 : 0;
+    if (!s_ok) atomicOr(a.err_flag, kErrTimeout);
+    trace_mark(a.trace, 3);
+  }
   __syncthreads();
-  if (threadIdx.x == 0) trace_mark(a.trace, 3);
+  if (!s_ok) return;  // uniform: every thread read the same flag after the barrier
 
-  // ---- main loop: 64-wide K chunks from registers, 4 k16 tiles each --------
+  // ---- main loop: 64-wide K chunks from shared memory, 4 k16 tiles each ----
+  const int c_begin = (n_chunks * kq) / KS;
+  const int nc = (n_chunks * (kq + 1)) / KS - c_begin;
+  const unsigned char* wbase = sw + tsel * wt_bytes + (size_t)lane * 16;
+  const unsigned char* sbase = ssz + tsel * sz_bytes + (size_t)g * 8;
   // B-fragment source of this lane: activation row and plane
   int brow, bplane;
   if (NT == 0 && LO) { brow = g >> 1; bplane = g & 1; }
@@ -299,22 +311,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
 
-  for (int base = 0; base < nc; base += kGemvPre) {
-    if (base > 0) {   // K beyond kGemvPre chunks per warp: the next batch
-#pragma unroll
-      for (int i = 0; i < kGemvPre; ++i) {
-        if (base + i < nc) {
-          wr[i] = ldg_stream(wsrc + (size_t)(c_begin + base + i) * 32);
-          sr[i] = ldg_stream2(ssrc + (size_t)((c_begin + base + i) >> 1) * 8);
-        }
-      }
-    }
-#pragma unroll
-  for (int i = 0; i < kGemvPre; ++i) {
-    if (base + i >= nc) break;
-    const int c = c_begin + base + i;
-    const uint4 wv = wr[i];
-    const uint2 sv = sr[i];
+#pragma unroll 2
+  for (int ci = 0; ci < nc; ++ci) {
+    const int c = c_begin + ci;
+    const uint4 wv = *reinterpret_cast<const uint4*>(wbase + (size_t)c * 512);
+    const uint2 sv = *reinterpret_cast<const uint2*>(sbase + (size_t)(c >> 1) * 64);
     const int kc = c * 64;
     float tmp[NTILES][4];
 #pragma unroll
@@ -361,7 +362,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
       acc[nt][2] = fmaf(s.y, tmp[nt][2], acc[nt][2]);
       acc[nt][3] = fmaf(s.y, tmp[nt][3], acc[nt][3]);
     }
-  }
   }
 
   trace_mark(a.trace, 4);

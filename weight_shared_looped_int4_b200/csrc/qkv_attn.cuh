@@ -162,26 +162,20 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   // gate_up's crowd onto the SMs this kernel leaves free; the decode step
   // measured faster without.
   if (tid == 0) {
-    mbar_init(&wbar, kQaThreads);   // every thread's cp.async completion
+    mbar_init(&wbar, 1);
     mbar_init(&kvbar, 1);
     fence_mbar_init();
-  }
-  __syncthreads();
-  // the weight tiles and scales, 16 bytes per cp.async from every thread
-  // (several times the per-SM rate of one thread's 1-D bulk copies)
-  {
-    const int w16 = (int)(wt_bytes / 16), s16 = (int)(sz_bytes / 16);
+    mbar_arrive_expect_tx(&wbar, (unsigned)(2 * nu * (wt_bytes + sz_bytes)));
     for (int i = 0; i < 2 * nu; ++i) {
       const int tile = unit_tile(c + (i >> 1) * kQaCluster, i & 1);
-      const uint4* wsrc = reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(a.w) +
-                                                         (size_t)tile * wt_bytes);
-      const uint4* ssrc = reinterpret_cast<const uint4*>(reinterpret_cast<const unsigned char*>(a.sz) +
-                                                         (size_t)tile * sz_bytes);
-      for (int e = tid; e < w16; e += kQaThreads) cp_async16(wsm + i * wt_bytes + (size_t)e * 16, wsrc + e, 16);
-      for (int e = tid; e < s16; e += kQaThreads)
-        cp_async16(wsm + 2 * nu * wt_bytes + i * sz_bytes + (size_t)e * 16, ssrc + e, 16);
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
+      for (size_t off = 0; off < wt_bytes; off += 32768) {
+        const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
+        bulk_g2s(wsm + i * wt_bytes + off, src + off, n, &wbar);
+      }
+      bulk_g2s(wsm + 2 * nu * wt_bytes + i * sz_bytes,
+               reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes, (unsigned)sz_bytes, &wbar);
     }
-    cp_async_mbar_arrive_noinc(&wbar);
   }
   // every rank of the cluster must be running before any distributed
   // shared-memory write reaches it (the first ones come after the GEMV)

@@ -557,18 +557,14 @@ cudaError_t launch_tc_linear(const uint8_t* wtc, const uint2* sz, int K, int N, 
   // tile run as one thread-block cluster and reduce in distributed shared
   // memory (as many splits as keep every cluster resident in one wave);
   // otherwise partial sums go to global scratch and a merge kernel adds them.
+  // (measured on the 400M model: a cluster reduction with fewer splits is
+  // slower than the partial buffer + merge kernel with more, so the cluster
+  // form is taken only where it keeps every split)
   int splits = std::max(1, std::min(G, sc.n_sm / (row_tiles * tok_tiles)));
+  while (splits > 1 && (size_t)splits * row_tiles * tok_tiles * kTcRows * kTcTokens * 4 > sc.partial_bytes) --splits;
   bool cluster = false;
-  if (splits > 1) {
-    int S = std::min(splits, kTcMaxCluster);
-    while (S > 1 && !tc_clusters_fit(kern, S, row_tiles * tok_tiles, smem)) --S;
-    if (S > 1) {
-      splits = S;
-      cluster = true;
-    }
-  }
-  if (!cluster)
-    while (splits > 1 && (size_t)splits * row_tiles * tok_tiles * kTcRows * kTcTokens * 4 > sc.partial_bytes) --splits;
+  if (splits > 1 && splits <= kTcMaxCluster && tc_clusters_fit(kern, splits, row_tiles * tok_tiles, smem))
+    cluster = true;
   ta.wtc = wtc; ta.sz = sz; ta.K = K; ta.N = N; ta.n16_tiles = n16_tiles;
   ta.bt = b_tiles ? b_tiles : sc.bt; ta.T = T; ta.splits = splits; ta.cluster = cluster ? 1 : 0;
   ta.partial = sc.partial; ta.tickets = sc.tickets; ta.err_flag = sc.err_flag;
@@ -598,11 +594,13 @@ cudaError_t launch_decode_attn(const DecodeAttnArgs& a, int rows, int hd, int re
   return cudaErrorInvalidValue;
 }
 
-constexpr int kAtMinTokens = 32;   // prefill attention on tcgen05 from this many queries
+// Prefill attention runs on tcgen05 from this many queries on, below it on
+// 16-query mma.sync tiles (tl_set_prefill_attention_tc_min).
+std::atomic<int> g_at_min_tokens{512};
 
 cudaError_t launch_prefill_attn(PrefillAttnArgs a, int B, int hd, int rep, bool f32, cudaStream_t st) {
   a.rep = rep;
-  if (a.T >= kAtMinTokens) {
+  if (a.T >= g_at_min_tokens.load(std::memory_order_relaxed)) {
     // tensor cores (tcgen05): one CTA per (128-query tile, query head, batch entry)
     const dim3 grid((a.T + kAtQ - 1) / kAtQ, a.Hkv * rep, B);
     if (hd == 128)
@@ -1771,6 +1769,12 @@ tl_status tl_model_set_trace(tl_model* m, unsigned long long* d_buf, long long n
 }
 
 int tl_model_trace_grid(const tl_model* m) { return m ? m->fused_grid : 0; }
+
+tl_status tl_set_prefill_attention_tc_min(int min_queries) {
+  if (min_queries < 1) return fail(TL_ERR_INVALID_ARG, "min_queries must be >= 1");
+  g_at_min_tokens.store(min_queries, std::memory_order_relaxed);
+  return TL_OK;
+}
 
 tl_status tl_model_set_wait_test(tl_model* m, int extra_arrivals) {
   if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
