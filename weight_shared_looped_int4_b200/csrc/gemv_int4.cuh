@@ -86,6 +86,7 @@ struct GemvArgs {
                               // released, weights arrived, main loop done,
                               // (6) activations staged
   int trigger;                // PdlTrigger
+  int l2_keep;                // 1: the weights are the loop block's (L2 evict-last), else evict-first
 };
 
 constexpr int kGemvThreads = 256;
@@ -165,15 +166,16 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
     mbar_init(&wbar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(&wbar, (unsigned)(TPC * (wt_bytes + sz_bytes)));
+    const uint64_t pol = a.l2_keep ? l2_evict_last() : l2_evict_first();
     for (int ts = 0; ts < TPC; ++ts) {
       const int tile = ts ? t1 : t0;
       const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
       for (size_t off = 0; off < wt_bytes; off += 32768) {
         const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
-        bulk_g2s(sw + ts * wt_bytes + off, src + off, n, &wbar);
+        bulk_g2s_hint(sw + ts * wt_bytes + off, src + off, n, &wbar, pol);
       }
-      bulk_g2s(ssz + ts * sz_bytes, reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes,
-               (unsigned)sz_bytes, &wbar);
+      bulk_g2s_hint(ssz + ts * sz_bytes, reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes,
+                    (unsigned)sz_bytes, &wbar, pol);
     }
   }
 

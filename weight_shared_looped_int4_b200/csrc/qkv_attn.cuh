@@ -60,6 +60,7 @@ struct QkvAttnArgs {
   long long lane_stride;
   int ctx;
   float* o;              // attention output [M][Hq*hd] fp32
+  int l2_keep;           // 1: loop-block weights (L2 evict-last), else evict-first
   int* err_flag;
   unsigned long long* trace;  // launch timeline (kTraceEvents entries) or NULL:
                               // released, q/k/v exchanged, partials exchanged,
@@ -166,15 +167,17 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     mbar_init(&kvbar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(&wbar, (unsigned)(2 * nu * (wt_bytes + sz_bytes)));
+    const uint64_t pol = a.l2_keep ? l2_evict_last() : l2_evict_first();
     for (int i = 0; i < 2 * nu; ++i) {
       const int tile = unit_tile(c + (i >> 1) * kQaCluster, i & 1);
       const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
       for (size_t off = 0; off < wt_bytes; off += 32768) {
         const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
-        bulk_g2s(wsm + i * wt_bytes + off, src + off, n, &wbar);
+        bulk_g2s_hint(wsm + i * wt_bytes + off, src + off, n, &wbar, pol);
       }
-      bulk_g2s(wsm + 2 * nu * wt_bytes + i * sz_bytes,
-               reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes, (unsigned)sz_bytes, &wbar);
+      bulk_g2s_hint(wsm + 2 * nu * wt_bytes + i * sz_bytes,
+                    reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes, (unsigned)sz_bytes, &wbar,
+                    pol);
     }
   }
   // every rank of the cluster must be running before any distributed

@@ -823,6 +823,7 @@ tl_status run_qkv(tl_model* m, int layer, int M, float* x, const RowCtx* rows, f
   a.rope_tab = m->rope_tab;
   a.err_flag = m->err_flag;
   a.trace = next_trace(m);
+  a.l2_keep = layer >= c.n_pre;
   kclass(TL_KERNEL_QKV);
   TL_CUDA(launch_gemv_rows(a, M, IN_NORM, EPI_ROPE_KV, (c.n_q_heads + 2 * c.n_kv_heads) * hd / 32, st));
   return TL_OK;
@@ -876,6 +877,7 @@ tl_status run_qkv_attn(tl_model* m, int layer, int M, const RowCtx* rows, cudaSt
     a.lane_stride = m->lane_stride; a.ctx = c.max_ctx;
     a.o = m->o + (size_t)r0 * qdim; a.err_flag = m->err_flag;
     a.trace = next_trace(m);
+    a.l2_keep = layer >= c.n_pre;
     const size_t smem = qa_layout(c.d_model, a.M, a.rep, c.head_dim).total;
     const dim3 grid(kQaCluster, c.n_kv_heads);
     if (c.head_dim == 64)
@@ -901,6 +903,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   a.err_flag = m->err_flag;
   a.trace = next_trace(m);
   a.trigger = TRIGGER_AT_START;
+  a.l2_keep = layer >= c.n_pre;
   kclass(TL_KERNEL_O_PROJ);
   TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, (b.o.N + 15) / 16, st));
   GemvArgs g{};
@@ -912,6 +915,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   g.err_flag = m->err_flag;
   g.trace = next_trace(m);
   g.trigger = TRIGGER_AFTER_LOOP;
+  g.l2_keep = layer >= c.n_pre;
   kclass(TL_KERNEL_GATE_UP);
   TL_CUDA(launch_gemv_rows(g, M, IN_NORM, EPI_SWIGLU, F / 16, st));
   GemvArgs dn{};
@@ -922,6 +926,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   dn.err_flag = m->err_flag;
   dn.trace = next_trace(m);
   dn.trigger = TRIGGER_AT_START;
+  dn.l2_keep = layer >= c.n_pre;
   kclass(TL_KERNEL_DOWN);
   TL_CUDA(launch_gemv_rows(dn, M, IN_F32, EPI_RESID, (b.down.N + 15) / 16, st));
   return TL_OK;
