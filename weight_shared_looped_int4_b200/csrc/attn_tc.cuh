@@ -23,11 +23,13 @@
 //                  block j runs while O_{j-1} is computed);
 //     warp 1       loads K/V blocks (cp.async, completion tracked by an
 //                  mbarrier), two blocks ahead;
-//     warps 2-5    softmax: one thread per query row reads its 64 scores from
-//                  TMEM, masks, keeps the running max / sum, writes P (hi, lo)
-//                  and the rescale factor of the block;
-//     warps 6-9    output: one thread per query row keeps O in registers and
-//                  applies O = O c_j + O_j as each O_j lands in TMEM.
+//     warps 2-9    softmax: two threads per query row (32 of its 64 scores
+//                  each, max and sum exchanged through shared memory) read
+//                  the scores from TMEM, mask, keep the running max / sum,
+//                  write P (hi, lo) and the rescale factor of the block;
+//     warps 10-17  output: two threads per query row (half of the head dims
+//                  each) keep O in registers and apply O = O c_j + O_j as
+//                  each O_j lands in TMEM.
 // * Every mbarrier wait is bounded; a CTA that gives up records kErrTimeout
 //   and still frees its TMEM.
 #pragma once
@@ -40,9 +42,9 @@ namespace tl {
 
 constexpr int kAtQ = 128;        // queries per CTA (MMA M)
 constexpr int kAtKeys = 64;      // keys per block (MMA N of S, K of P V)
-constexpr int kAtWarps = 10;
+constexpr int kAtWarps = 18;
 constexpr int kAtThreads = kAtWarps * 32;
-constexpr int kAtSoftWarp0 = 2, kAtOutWarp0 = 6;
+constexpr int kAtSoftWarp0 = 2, kAtOutWarp0 = 10;   // 8 softmax warps, 8 output warps
 
 // Shared-memory plan (bytes) for head_dim HD.
 template <int HD>
@@ -92,6 +94,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
   __shared__ int s_fail;
   __shared__ float cfac[2][kAtQ];   // rescale factor of block j for each row
   __shared__ float lfin[kAtQ];      // final row sums
+  __shared__ float xmax[2][kAtQ], xsum[2][kAtQ];   // the two softmax halves of a row
 
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -110,9 +113,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 32);          // the loader warp's lanes (cp.async completion)
       mbar_init(&s_full[i], 1);            // tcgen05.commit
-      mbar_init(&p_full[i], 128);          // softmax threads
+      mbar_init(&p_full[i], 256);          // softmax threads
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], 128);         // output threads
+      mbar_init(&o_empty[i], 256);         // output threads
       mbar_init(&blk_done[i], 1);
     }
     fence_mbar_init();
@@ -260,40 +263,39 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
     }
     cp_async_wait<0>();   // nothing of this warp in flight at exit
   } else if (warp < kAtOutWarp0) {
-    // ---- softmax: thread = query row r ---------------------------------------
-    const int quad = warp & 3, r = quad * 32 + lane;
+    // ---- softmax: two threads per query row r, 32 scores each ---------------
+    const int quad = warp & 3, half = (warp - kAtSoftWarp0) >> 2, r = quad * 32 + lane;
     const int pos = a.pos0 + q0 + r;
     float m_run = -INFINITY, l_run = 0.f;
     for (int j = 0; j < nblk; ++j) {
       const int bb = j & 1;
       mbar_wait_or_fail(&s_full[bb], (unsigned)(j >> 1) & 1u, &s_fail);
       tc_fence_after();
-      float s[64];
+      float s[32];
       {
         uint32_t raw[32];
-        const int k0 = j * kAtKeys;
+        const int k0 = j * kAtKeys + half * 32;
+        tmem_ld32(t_s(bb) + ((uint32_t)(quad * 32) << 16) + half * 32, raw);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          tmem_ld32(t_s(bb) + ((uint32_t)(quad * 32) << 16) + c0, raw);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c0 + i] = (k0 + c0 + i <= pos) ? __uint_as_float(raw[i]) : -INFINITY;
-        }
+        for (int i = 0; i < 32; ++i) s[i] = (k0 + i <= pos) ? __uint_as_float(raw[i]) : -INFINITY;
       }
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) mx = fmaxf(mx, s[i]);
+      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, s[i]);
+      xmax[half][r] = mx;
+      asm volatile("bar.sync 2, 256;" ::: "memory");   // the 8 softmax warps
       // scores are in base 2 (Q carries log2(e)): weights 2^(s - m)
-      const float m_new = fmaxf(m_run, mx);
+      const float m_new = fmaxf(m_run, fmaxf(mx, xmax[half ^ 1][r]));
       const float c = (m_run == -INFINITY) ? 0.f : exp2f(m_run - m_new);
       float sum = 0.f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
+      for (int i = 0; i < 32; ++i) {
         s[i] = (m_new == -INFINITY) ? 0.f : exp2f(s[i] - m_new);   // 2^-inf = 0 for masked keys
         sum += s[i];
       }
       m_run = m_new;
-      l_run = l_run * c + sum;
+      xsum[half][r] = sum;
       // P buffer bb was last read by O_{j-2}, cfac[bb] by the output warps'
       // update of block j - 2
       if (j >= 2) {
@@ -303,54 +305,59 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
       unsigned char* ph = sm + Lay::p0 + (bb * 2) * Lay::P_BYTES;
       unsigned char* pl = ph + Lay::P_BYTES;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 4; ++q) {
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) split_h2(s[q * 8 + 2 * i], s[q * 8 + 2 * i + 1], hw[i], lw[i]);
-        const int o = r * 128 + ((q ^ (r & 7)) << 4);
+        const int j16 = half * 4 + q;
+        const int o = r * 128 + ((j16 ^ (r & 7)) << 4);
         *reinterpret_cast<uint4*>(ph + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         *reinterpret_cast<uint4*>(pl + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
-      cfac[bb][r] = c;
+      if (half == 0) cfac[bb][r] = c;
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&p_full[bb]);
+      asm volatile("bar.sync 2, 256;" ::: "memory");
+      l_run = l_run * c + xsum[0][r] + xsum[1][r];
     }
-    lfin[r] = l_run;
+    if (half == 0) lfin[r] = l_run;
   } else {
-    // ---- output: thread = query row r, O kept in registers ------------------
-    const int quad = warp & 3, r = quad * 32 + lane;
-    float o_acc[HD];
+    // ---- output: two threads per query row r, O (HD / 2 columns each) kept
+    // in registers ---------------------------------------------------------------
+    constexpr int HO = HD / 2;
+    const int quad = warp & 3, half = (warp - kAtOutWarp0) >> 2, r = quad * 32 + lane;
+    float o_acc[HO];
 #pragma unroll
-    for (int i = 0; i < HD; ++i) o_acc[i] = 0.f;
+    for (int i = 0; i < HO; ++i) o_acc[i] = 0.f;
     for (int j = 0; j < nblk; ++j) {
       const int bb = j & 1;
       // cfac of block j first: p_full cannot move on to block j + 2 before
-      // this warp releases o_empty for block j, so the phase is unambiguous
+      // these warps release o_empty for block j, so the phase is unambiguous
       mbar_wait_or_fail(&p_full[bb], (unsigned)(j >> 1) & 1u, &s_fail);
       mbar_wait_or_fail(&o_full[bb], (unsigned)(j >> 1) & 1u, &s_fail);
       tc_fence_after();
       const float c = cfac[bb][r];
 #pragma unroll
-      for (int c0 = 0; c0 < HD; c0 += 32) {
-        uint32_t raw[32];
-        tmem_ld32(t_o(bb) + ((uint32_t)(quad * 32) << 16) + c0, raw);
+      for (int c0 = 0; c0 < HO; c0 += 16) {
+        uint32_t raw[16];
+        tmem_ld16(t_o(bb) + ((uint32_t)(quad * 32) << 16) + half * HO + c0, raw);
         tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o_acc[c0 + i] = fmaf(o_acc[c0 + i], c, __uint_as_float(raw[i]));
+        for (int i = 0; i < 16; ++i) o_acc[c0 + i] = fmaf(o_acc[c0 + i], c, __uint_as_float(raw[i]));
       }
       tc_fence_before();
       mbar_arrive(&o_empty[bb]);
     }
-    asm volatile("bar.sync 1, 256;" ::: "memory");   // softmax (lfin) and output warps
+    asm volatile("bar.sync 1, 512;" ::: "memory");   // softmax (lfin) and output warps
     const int t_row = q0 + r;
     if (t_row < a.T) {
       const float inv = 1.f / lfin[r];
       if (F32 && a.bt) {
         const int tt = t_row / kTcTokensB, tl_ = t_row % kTcTokensB;
 #pragma unroll
-        for (int i = 0; i < HD; i += 2) {
-          const int k = h * HD + i;   // column of the O projection's input
+        for (int i = 0; i < HO; i += 2) {
+          const int k = h * HD + half * HO + i;   // column of the O projection's input
           const int grp = k >> 7, kg = k & 127;
           uint32_t hw, lw;
           split_h2(o_acc[i] * inv, o_acc[i + 1] * inv, hw, lw);
@@ -359,16 +366,16 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
           *reinterpret_cast<uint32_t*>(blk + sw128_offset(kTcTokensB + tl_, kg, 2 * kTcTokensB)) = lw;
         }
       } else {
-        const size_t off = b * a.o_bstride + (size_t)t_row * a.ldo + (size_t)h * HD;
+        const size_t off = b * a.o_bstride + (size_t)t_row * a.ldo + (size_t)h * HD + half * HO;
 #pragma unroll
-        for (int i = 0; i < HD; i += 2) {
+        for (int i = 0; i < HO; i += 2) {
           if (F32) *reinterpret_cast<float2*>(a.of + off + i) = make_float2(o_acc[i] * inv, o_acc[i + 1] * inv);
           else *reinterpret_cast<uint32_t*>(a.oh + off + i) = pack_h2(o_acc[i] * inv, o_acc[i + 1] * inv);
         }
       }
     }
   }
-  if (warp >= kAtSoftWarp0 && warp < kAtOutWarp0) asm volatile("bar.arrive 1, 256;" ::: "memory");
+  if (warp >= kAtSoftWarp0 && warp < kAtOutWarp0) asm volatile("bar.arrive 1, 512;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0 && s_fail && a.err_flag) atomicOr(a.err_flag, kErrTimeout);
