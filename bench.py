@@ -888,7 +888,7 @@ def run_workload_attention(args):
                     best = min(cold, warm)
                     rec[kname] = {"us_l2_cold": round(1e3 * cold, 2), "us_graph": round(1e3 * warm, 2),
                                   "tflops": round(flops / (best * 1e9), 2), "frac": round(t_roof / (1e3 * best), 4)}
-                tl.tl_set_prefill_attention_tc_min(512)
+                tl.tl_set_prefill_attention_tc_min(1024)
                 pre.append(rec)
                 del kc, vc, qd, out
     print(json.dumps({"workload": "GQA attention D2048 16q/4kv hd128 (fp16 KV)",

@@ -361,7 +361,9 @@ tl_status tl_model_set_wait_test(tl_model *m, int extra_arrivals);
  * prefill attention (prefill, tl_extend, tl_op_gqa_prefill) runs on the
  * tcgen05 kernel (128-query tiles, TMEM accumulators) for passes of at least
  * min_queries queries and on 16-query mma.sync tiles below that.  Process
- * wide; default 512.  Both kernels compute the same attention. */
+ * wide; default 1024 (measured: below it the 16-query tiles are faster on
+ * B200, from it the tcgen05 kernel).  Both kernels compute the same
+ * attention. */
 tl_status tl_set_prefill_attention_tc_min(int min_queries);
 
 /* Number of kernels this library has launched in the process so far. */

@@ -100,7 +100,7 @@ def _prefill_case(T, B, pos0, hq, hkv, hd, seed, sample=None):
                 err = rel_l2(got[b, rows], expects[b])
                 assert err <= KERNEL_REL_L2, (kernel, T, b, err)
     finally:
-        tl.tl_set_prefill_attention_tc_min(512)
+        tl.tl_set_prefill_attention_tc_min(1024)
 
 
 @pytest.mark.parametrize("B", [1, 8])

@@ -303,7 +303,7 @@ def tl_lane_fork(model, src_lane, dst_lane, n_tokens, stream=None) -> None:
 
 
 def tl_set_prefill_attention_tc_min(min_queries: int) -> None:
-    """Prefill attention on tcgen05 from this many queries on (default 512)."""
+    """Prefill attention on tcgen05 from this many queries on (default 1024)."""
     _check(_L().tl_set_prefill_attention_tc_min(int(min_queries)))
 
 

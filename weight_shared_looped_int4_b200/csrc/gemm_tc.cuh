@@ -14,11 +14,12 @@
 //   registers.  So no weight is rounded and the activation keeps ~22 bits;
 //   fp16 weights or activations move the looped model's logits by ~0.05.
 // * Warp roles (16 warps): warp 0 allocates TMEM and one lane issues
-//   tcgen05.mma; one lane of warp 1 keeps the raw INT4 words + scales/zeros
-//   a few groups ahead with bulk copies; warps 2-7 copy each stage's prepared
-//   B atom (16-byte cp.async, 1/192 each) and dequantize A from the raw ring
-//   straight into the 128-byte swizzled K-major layout the MMA descriptor
-//   reads; warps 8-15 are the epilogue.  Stages of 64 k (4 deep), the raw ring (3 groups) and the TMEM
+//   tcgen05.mma; one lane of warp 1 issues the bulk asynchronous copies (raw
+//   INT4 words + scales/zeros a few groups ahead, the prepared B atoms per
+//   stage); warps 2-7 dequantize A from the raw ring straight into the
+//   128-byte swizzled K-major layout the MMA descriptor reads (the
+//   dequantisation, not the tensor core, paces this GEMM); warps 8-15 are the
+//   epilogue.  Stages of 64 k (4 deep), the raw ring (3 groups) and the TMEM
 //   buffers (2 groups) are handed over with mbarriers (tcgen05.commit signals
 //   MMA completion).
 // * Split-K partials go to a scratch buffer; a merge kernel (one CTA per 8
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   }
   if (threadIdx.x == 32) {
     for (int i = 0; i < kTcStages; ++i) {
-      mbar_init(&bar_full[i], 2 * kTcUnpack);   // each unpacker: A written + its B copies landed
+      mbar_init(&bar_full[i], kTcUnpack + 1);   // + the copy lane's arrive with the B bytes
       mbar_init(&bar_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -432,7 +433,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
         if (!mbar_wait_or_fail(&bar_full[s], (unsigned)(h / kTcStages) & 1u, &s_fail)) break;
         if (half == 0 && it >= 2 && !mbar_wait_or_fail(&bar_tempty[b], (unsigned)((it - 2) >> 1) & 1u, &s_fail))
           break;
-        fence_proxy_async_smem();   // the B atom came through cp.async (generic proxy)
         tc_fence_after();
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -446,24 +446,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---- raw weight copies (one lane) ------------------------------------------
+    // ---- copy issuer (one lane) ----------------------------------------------
     // Keeps kTcRaw groups of raw INT4 words and scales/zeros in flight (bulk
     // copies; the weights do not depend on earlier kernels, so the first ones
-    // go out before the dependency wait).  Group g_issued reuses the slot of
-    // g_issued - kTcRaw once the unpackers release it.
+    // go out before the dependency wait) and issues each stage's B atom as
+    // soon as the MMA has released the stage.
     if (lane == 0) {
+      int g_issued = 0;
       auto issue_raw = [&](int it) {
         const int r = it % kTcRaw, g = gmap(it);
         mbar_arrive_expect_tx(&raw_full[r], kTcRawBytes);
         bulk_g2s(sR(r), a.wtc + ((size_t)tile * G + g) * kTcRawBytes, kTcRawBytes, &raw_full[r]);
       };
-      int g_issued = 0;
       for (; g_issued < ng && g_issued < kTcRaw; ++g_issued) issue_raw(g_issued);
       pdl_wait();
-      for (; g_issued < ng; ++g_issued) {
-        if (!mbar_wait_or_fail(&raw_empty[g_issued % kTcRaw], (unsigned)((g_issued / kTcRaw) - 1) & 1u, &s_fail))
+      for (int h = 0; h < nh; ++h) {
+        const int s = h % kTcStages, it = h >> 1, half = h & 1, g = gmap(it);
+        if (h >= kTcStages && !mbar_wait_or_fail(&bar_empty[s], (unsigned)((h / kTcStages) - 1) & 1u, &s_fail))
           break;
-        issue_raw(g_issued);
+        // arrive with the expected bytes: the stage cannot complete before
+        // this arrival, so the unpackers' arrivals cannot race past the copy
+        mbar_arrive_expect_tx(&bar_full[s], B_BYTES);
+        bulk_g2s(sB(s), a.bt + (((size_t)tt * G + g) * 2 + half) * B_BYTES, B_BYTES, &bar_full[s]);
+        if (half) {
+          // top up the raw ring: group g_issued reuses the slot of g_issued - kTcRaw
+          for (; g_issued < ng && g_issued < it + kTcRaw; ++g_issued)
+            if (mbar_wait_or_fail(&raw_empty[g_issued % kTcRaw], (unsigned)((g_issued / kTcRaw) - 1) & 1u,
+                                  &s_fail))
+              issue_raw(g_issued);
+        }
       }
       // a CTA that gave up waits (bounded) for its raw copies still in flight
       if (*reinterpret_cast<volatile int*>(&s_fail))
@@ -474,20 +485,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
   } else if (warp < kTcEpiWarp0) {
     // ---- unpackers: A from the raw ring into the 128-byte swizzled K-major
     // layout the MMA descriptor reads --------------------------------------------
-    // Each unpacker also copies 1/192 of the stage's B atom (activations,
-    // 32 KB) with 16-byte cp.async as soon as the stage is free: many
-    // threads keep far more bytes in flight than one bulk copy per stage.
     const int p = threadIdx.x - 64;
-    pdl_wait();   // the B tiles were written by the previous kernel
     for (int h = 0; h < nh; ++h) {
       const int s = h % kTcStages, it = h >> 1, half = h & 1, r = it % kTcRaw;
       if (h >= kTcStages && !mbar_wait_or_fail(&bar_empty[s], (unsigned)((h / kTcStages) - 1) & 1u, &s_fail))
         break;
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(a.bt + (((size_t)tt * G + gmap(it)) * 2 + half) * B_BYTES);
-        unsigned char* dst = sB(s);
-        for (int i = p; i < (int)(B_BYTES / 16); i += kTcUnpack) cp_async16(dst + i * 16, src + i, 16);
-      }
       if (!mbar_wait_or_fail(&raw_full[r], (unsigned)(it / kTcRaw) & 1u, &s_fail)) break;
       const unsigned char* raw = sR(r);
       unsigned char* A = sA(s);
@@ -514,9 +516,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
       if (half) mbar_arrive(&raw_empty[r]);
       fence_proxy_async_smem();
       mbar_arrive(&bar_full[s]);
-      cp_async_mbar_arrive_noinc(&bar_full[s]);   // once this thread's B copies land
     }
-    cp_async_wait<0>();
   } else {
     // ---- epilogue: accumulate s * (P_hi + P_lo) per group --------------
     pdl_wait();   // it reads / writes what earlier kernels wrote

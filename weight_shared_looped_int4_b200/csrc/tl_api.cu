@@ -596,7 +596,7 @@ cudaError_t launch_decode_attn(const DecodeAttnArgs& a, int rows, int hd, int re
 
 // Prefill attention runs on tcgen05 from this many queries on, below it on
 // 16-query mma.sync tiles (tl_set_prefill_attention_tc_min).
-std::atomic<int> g_at_min_tokens{512};
+std::atomic<int> g_at_min_tokens{1024};
 
 cudaError_t launch_prefill_attn(PrefillAttnArgs a, int B, int hd, int rep, bool f32, cudaStream_t st) {
   a.rep = rep;
