@@ -57,13 +57,16 @@ BYTES_PER_LAUNCH = {
 }
 
 
-# DRAM bytes (read + write) of one launch of each decode kernel class, from an
-# `ncu --set full` capture of `bench.py --ncu-case decode` (cold cache, first
-# decode step: NCU_KEYS cached keys for the QKV + attention kernel).  Valid for the kernels as captured; the QKV class's cache part is
-# rescaled to the bench's mean context.
-NCU_TRAFFIC = {"qkv": 3683328, "o_proj": 2262528, "gate_up": 12306944, "down": 6176000,
-               "head": 131194368 + 6204160}
-NCU_KEYS = 133
+# DRAM bytes (read + write) of one launch of each decode kernel class, from
+#   ncu --clock-control none -k regex:"qkv_attn|gemv_int4|head_direct" -c 45 \
+#       --metrics dram__bytes_read.sum,dram__bytes_write.sum python bench.py --ncu-case decode --decode-steps 2
+# (ncu flushes the caches before every launch, so every launch reads its
+# weights from DRAM; first decode step, NCU_KEYS cached keys per layer for the
+# QKV + attention kernel).  Valid for the kernels as captured; the QKV
+# class's cache part is rescaled to the bench's mean context.
+NCU_TRAFFIC = {"qkv": 3684096, "o_proj": 2262528, "gate_up": 12307200, "down": 6176256,
+               "head": 131140864 + 135680}
+NCU_KEYS = PROMPT + 1
 
 
 
