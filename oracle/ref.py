@@ -51,11 +51,16 @@ Everything is float64; the fp16 inputs (scales, gains, embedding, head,
 activations) are widened exactly.  One precision is fixed by the pages and so
 kept: keys and values are stored in an FP16 KV cache (TinyLoop README, "Python
 API reference": KV cache modes, "FP16 KV"; the workload's "KV cache fp16").  By
-default (``kv_fp16=True``) the rotated keys and the values are rounded to fp16
-(round-to-nearest-even) when they are produced, on the cached and the uncached
-path alike, so attention always reads the stored fp16 values.  With
-``kv_fp16=False`` nothing at all is rounded (used to compare against a float64
-library model).  No other fp16 rounding is emulated.
+default (``kv_mode="fp16"``) the rotated keys and the values are rounded to
+fp16 (round-to-nearest-even) when they are produced, on the cached and the
+uncached path alike, so attention always reads the stored fp16 values.  The
+pages also name an INT8 KV mode (TinyLoop README, "Python API reference", KV
+cache modes) without its format; ``kv_mode="int8"`` takes the plainest reading:
+each produced key and value vector (one position, one kv head, hd elements) is
+stored as symmetric int8 codes with one fp32 scale, see ``quantize_kv_int8``,
+and attention reads the dequantized codes.  With ``kv_mode="none"`` (or
+``kv_fp16=False``) nothing at all is rounded (used to compare against a
+float64 library model).  No other rounding is emulated.
 """
 
 from __future__ import annotations
@@ -175,6 +180,37 @@ def to_fp16_storage(x: np.ndarray) -> np.ndarray:
     return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
 
 
+def quantize_kv_int8(x: np.ndarray):
+    """INT8 KV storage of vectors along the last axis (hd elements each).
+
+    Per vector: scale = max|x| / 127 and code = round-half-even(x / scale),
+    so the codes lie in [-127, 127] and the largest magnitude maps to +-127; an
+    all-zero vector has scale 0 and codes 0.  The stored value is code * scale.
+    The quantisation takes its integer decisions in float32, the precision the
+    kernels take them in (x rounded to float32, the scale and the quotient
+    float32 operations), so both sides choose the same codes for the same
+    float32 input.  Returns (codes int8 [..., hd], scales float32 [...]).
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.max(np.abs(x32), axis=-1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = np.rint((x32 / safe[..., None]).astype(np.float32))
+    q = np.where(scale[..., None] > 0, q, np.float32(0.0))
+    codes = np.clip(q, -127, 127).astype(np.int8)
+    return codes, scale
+
+
+def dequantize_kv_int8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """code * scale in float64 (the value an INT8 KV cache holds)."""
+    return np.asarray(codes, np.float64) * np.asarray(scales, np.float64)[..., None]
+
+
+def to_int8_storage(x: np.ndarray) -> np.ndarray:
+    """Quantise to the INT8 KV format and widen back: the value the cache holds."""
+    return dequantize_kv_int8(*quantize_kv_int8(x))
+
+
 def silu(u: np.ndarray) -> np.ndarray:
     return u / (1.0 + np.exp(-u))
 
@@ -261,10 +297,14 @@ class KVCache:
 class LoopedModel:
     """The looped transformer with the weights of a ``tl_synth.ModelWeights``."""
 
-    def __init__(self, weights, kv_fp16: bool = True):
+    def __init__(self, weights, kv_fp16: bool = True, kv_mode: Optional[str] = None):
         sh = weights.shape
         self.shape = sh
-        self.kv_fp16 = kv_fp16
+        if kv_mode is None:
+            kv_mode = "fp16" if kv_fp16 else "none"
+        if kv_mode not in ("fp16", "int8", "none"):
+            raise ValueError("kv_mode must be fp16, int8 or none")
+        self.kv_mode = kv_mode
         self.embed = np.asarray(weights.embed, np.float64)
         self.out_norm = np.asarray(weights.out_norm, np.float64)
         self.head = np.asarray(weights.head, np.float64)
@@ -291,8 +331,10 @@ class LoopedModel:
         v = qkv[:, (Hq + Hkv) * hd:].reshape(T, Hkv, hd)
         q = rope(q, positions, sh.rope_theta)
         k = rope(k, positions, sh.rope_theta)
-        if self.kv_fp16:
+        if self.kv_mode == "fp16":
             k, v = to_fp16_storage(k), to_fp16_storage(v)
+        elif self.kv_mode == "int8":
+            k, v = to_int8_storage(k), to_int8_storage(v)
         if cache is not None:
             k_all, v_all = cache.append(layer, k, v)
         else:
