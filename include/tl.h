@@ -69,7 +69,21 @@ typedef struct {
   int max_lanes;    /* decode lanes, 1..16 */
   float rms_eps;    /* RMSNorm epsilon */
   float rope_theta; /* RoPE base */
+  int kv_mode;      /* TL_KV_FP16 (0) or TL_KV_INT8, see below */
 } tl_config;
+
+/* KV cache storage (TinyLoop README, "Python API reference", KV cache modes:
+ * "FP16 KV" and "INT8 KV"; the pages give no INT8 format, so this is the
+ * plainest reading).  TL_KV_FP16 stores the rotated keys and the values as
+ * fp16.  TL_KV_INT8 stores each key or value vector (one position, one kv
+ * head: head_dim elements) as int8 codes with one fp32 scale, scale =
+ * max|x| / 127 and code = round-half-even(x / scale) in fp32 (an all-zero
+ * vector has scale 0); attention reads code * scale.  INT8 halves the cache's
+ * bytes.  It needs the clustered decode kernel (tl_model_create returns
+ * TL_ERR_UNSUPPORTED for shapes that do not fit it) and runs every prefill
+ * attention pass on the 16-query tile kernel; the single-kernel decode path
+ * (TL_DECODE_FUSED) is FP16 only. */
+enum { TL_KV_FP16 = 0, TL_KV_INT8 = 1 };
 
 /* One INT4 linear with K inputs and N outputs, HOST memory, storage format:
  *   qweight uint32 [N][K/8]        element k of row n is bits 4*(k%8)..+3 of
@@ -245,6 +259,19 @@ tl_status tl_score_early_exit(tl_model *m, const int32_t *d_tokens, int n_tokens
  * the prefix cache; forks continue from it without recomputing it.
  * 1 <= n_tokens <= length(src_lane); the lanes differ. */
 tl_status tl_lane_fork(tl_model *m, int src_lane, int dst_lane, int n_tokens, void *stream);
+
+/* Snapshot of one lane's KV slice `layer` (0 <= layer < n_pre + the lane's
+ * loops), positions [0, n_tokens), copied out of the cache as stored (the
+ * prefix cache's snapshot of a lane's slices; same pages as tl_lane_fork):
+ *   FP16 cache: d_k, d_v fp16 [n_kv_heads][n_tokens][head_dim] (rotated keys,
+ *               values); d_k_scales / d_v_scales are not touched (may be NULL)
+ *   INT8 cache: d_k, d_v int8 codes [n_kv_heads][n_tokens][head_dim] and
+ *               d_k_scales, d_v_scales fp32 [n_kv_heads][n_tokens]
+ * Device pointers, stream-ordered after the calls that wrote the lane.
+ * TL_ERR_NOT_PREFILLED for an empty lane, TL_ERR_INVALID_ARG for a layer or
+ * n_tokens out of range (n_tokens <= the lane's length) or a NULL pointer. */
+tl_status tl_lane_kv_export(const tl_model *m, int lane, int layer, int n_tokens, void *d_k, void *d_v,
+                            float *d_k_scales, float *d_v_scales, void *stream);
 
 /* Tokens currently held by a lane (0 if never prefilled). */
 tl_status tl_lane_length(const tl_model *m, int lane, int *h_length);
@@ -462,6 +489,16 @@ tl_status tl_op_gqa_prefill(const uint16_t *d_q, const uint16_t *d_k, const uint
                             long long batch_stride, int ctx_stride, int T, int pos0, int B,
                             int n_q_heads, int n_kv_heads, int head_dim, uint16_t *d_out,
                             void *stream);
+
+/* The INT8 KV quantisation of tl_config.kv_mode = TL_KV_INT8, as the model's
+ * prefill writes it: n vectors of head_dim fp32 elements
+ *   d_x fp32 [n][head_dim] -> d_codes int8 [n][head_dim], d_scales fp32 [n]
+ * with scale = max|x| / 127 and code = round-half-even(x / scale) (0 for an
+ * all-zero vector), both in fp32.  head_dim 64 or 128; n >= 0 (0 enqueues
+ * nothing).  Device pointers; TL_ERR_INVALID_ARG for a NULL pointer or n < 0,
+ * TL_ERR_UNSUPPORTED for another head_dim. */
+tl_status tl_op_kv_quant_int8(const float *d_x, int n, int head_dim, int8_t *d_codes, float *d_scales,
+                              void *stream);
 
 /* ------------------------------------------------------------------------
  * Misc

@@ -305,6 +305,10 @@ class LoopedModel:
         if kv_mode not in ("fp16", "int8", "none"):
             raise ValueError("kv_mode must be fp16, int8 or none")
         self.kv_mode = kv_mode
+        # when a list: (layer, k, v) of every block call, the rotated keys and
+        # the values before the cache's storage rounding (for checking what a
+        # cache stores against what it was given)
+        self.kv_trace: Optional[list] = None
         self.embed = np.asarray(weights.embed, np.float64)
         self.out_norm = np.asarray(weights.out_norm, np.float64)
         self.head = np.asarray(weights.head, np.float64)
@@ -331,6 +335,8 @@ class LoopedModel:
         v = qkv[:, (Hq + Hkv) * hd:].reshape(T, Hkv, hd)
         q = rope(q, positions, sh.rope_theta)
         k = rope(k, positions, sh.rope_theta)
+        if self.kv_trace is not None:
+            self.kv_trace.append((layer, k.copy(), v.copy()))
         if self.kv_mode == "fp16":
             k, v = to_fp16_storage(k), to_fp16_storage(v)
         elif self.kv_mode == "int8":

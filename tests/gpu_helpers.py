@@ -42,22 +42,23 @@ def f16_host(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy().astype(np.float64)
 
 
-def check_argmax(gpu_idx: int, oracle_logits: np.ndarray, where: str = ""):
-    """Greedy index must equal the oracle's unless its top-2 margin is < 1e-3."""
+def check_argmax(gpu_idx: int, oracle_logits: np.ndarray, where: str = "", margin: float = ARGMAX_MARGIN):
+    """Greedy index must equal the oracle's unless its top-2 margin is below
+    `margin` (1e-3; the INT8 KV tests pass their own logit bound)."""
     from oracle import ref
     o = ref.greedy(oracle_logits)
     if gpu_idx != o:
-        margin = ref.top2_margin(oracle_logits)
-        assert margin < ARGMAX_MARGIN, f"{where}: argmax {gpu_idx} != oracle {o} (margin {margin})"
+        m2 = ref.top2_margin(oracle_logits)
+        assert m2 < margin, f"{where}: argmax {gpu_idx} != oracle {o} (margin {m2})"
         # the GPU's pick must be one of the near-tied leaders
-        assert oracle_logits[o] - oracle_logits[gpu_idx] < ARGMAX_MARGIN, where
+        assert oracle_logits[o] - oracle_logits[gpu_idx] < margin, where
 
 
 class GpuModel:
     """A tl_model built from tl_synth weights, destroyed on close()."""
 
-    def __init__(self, weights, max_loops, max_ctx, max_lanes, device=0):
-        cfg = tl.make_config(weights.shape, max_loops, max_ctx, max_lanes)
+    def __init__(self, weights, max_loops, max_ctx, max_lanes, device=0, kv_mode=0):
+        cfg = tl.make_config(weights.shape, max_loops, max_ctx, max_lanes, kv_mode)
         tw, keep = tl.make_weights(weights)
         self.handle = tl.tl_model_create(cfg, tw, device)
         del keep

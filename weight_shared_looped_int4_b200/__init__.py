@@ -35,7 +35,7 @@ __all__ = [
     "tl_score_early_exit", "tl_lane_fork", "tl_spec_stats", "tl_set_prefill_attention_tc_min",
     "tl_linear_create", "tl_linear_destroy", "tl_linear_forward",
     "tl_op_rmsnorm", "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill",
-    "tl_op_gqa_decode_noalloc",
+    "tl_op_gqa_decode_noalloc", "tl_op_kv_quant_int8", "TL_KV_FP16", "TL_KV_INT8", "tl_lane_kv_export",
     "tl_status_string", "tl_last_error", "tl_version",
     "make_config", "make_weights", "make_int4_linear",
 ]
@@ -43,6 +43,7 @@ __all__ = [
 TL_OK, TL_ERR_INVALID_ARG, TL_ERR_OOM, TL_ERR_CUDA, TL_ERR_CONTEXT_FULL = 0, 1, 2, 3, 4
 TL_ERR_LOOPS_MISMATCH, TL_ERR_NOT_PREFILLED, TL_ERR_DEVICE_FLAG, TL_ERR_UNSUPPORTED = 5, 6, 7, 8
 TL_PATH_AUTO, TL_PATH_GEMV, TL_PATH_TC = 0, 1, 2
+TL_KV_FP16, TL_KV_INT8 = 0, 1
 
 
 class TLError(RuntimeError):
@@ -57,7 +58,7 @@ class tl_config(ctypes.Structure):
     _fields_ = [("d_model", c_int), ("n_q_heads", c_int), ("n_kv_heads", c_int),
                 ("head_dim", c_int), ("ffn_dim", c_int), ("vocab", c_int), ("n_pre", c_int),
                 ("max_loops", c_int), ("max_ctx", c_int), ("max_lanes", c_int),
-                ("rms_eps", c_float), ("rope_theta", c_float)]
+                ("rms_eps", c_float), ("rope_theta", c_float), ("kv_mode", c_int)]
 
 
 class tl_int4_linear(ctypes.Structure):
@@ -114,6 +115,8 @@ def _load():
         "tl_linear_forward": (st, [P, P, c_int, P, c_int, P]),
         "tl_op_rmsnorm": (st, [P, P, c_int, c_int, c_float, P, P]),
         "tl_op_rope": (st, [P, c_int, c_int, c_int, c_longlong, c_longlong, P, c_float, P]),
+        "tl_op_kv_quant_int8": (st, [P, c_int, c_int, P, P, P]),
+        "tl_lane_kv_export": (st, [P, c_int, c_int, c_int, P, P, P, P, P]),
         "tl_op_gqa_decode": (st, [P, P, P, c_longlong, c_int, P, c_int, c_int, c_int, c_int, P, P]),
         "tl_op_gqa_prefill": (st, [P, P, P, c_longlong, c_int, c_int, c_int, c_int, c_int, c_int,
                                    c_int, P, P]),
@@ -155,7 +158,7 @@ EXPORTED = sorted(["tl_model_profile_start", "tl_model_profile_stop", "tl_kernel
                    "tl_score_last", "tl_lane_length", "tl_model_info", "tl_check_device_error",
                    "tl_linear_create", "tl_linear_destroy", "tl_linear_forward", "tl_op_rmsnorm",
                    "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill", "tl_status_string",
-                   "tl_op_gqa_decode_noalloc",
+                   "tl_op_gqa_decode_noalloc", "tl_op_kv_quant_int8", "tl_lane_kv_export",
                    "tl_last_error", "tl_version"])
 
 
@@ -205,11 +208,12 @@ def _i32_host(values):
 
 # ------------------------------------------------------------ marshalling ---
 
-def make_config(shape, max_loops: int, max_ctx: int, max_lanes: int) -> tl_config:
-    """tl_config from an object with the ModelShape attribute names."""
+def make_config(shape, max_loops: int, max_ctx: int, max_lanes: int, kv_mode: int = 0) -> tl_config:
+    """tl_config from an object with the ModelShape attribute names
+    (kv_mode TL_KV_FP16 or TL_KV_INT8)."""
     return tl_config(shape.d_model, shape.n_q_heads, shape.n_kv_heads, shape.head_dim,
                      shape.ffn_dim, shape.vocab, shape.n_pre, max_loops, max_ctx, max_lanes,
-                     float(shape.rms_eps), float(shape.rope_theta))
+                     float(shape.rms_eps), float(shape.rope_theta), int(kv_mode))
 
 
 def make_int4_linear(lin) -> tl_int4_linear:
@@ -407,6 +411,17 @@ def tl_op_rope(d_x, n_tokens, n_heads, head_dim, token_stride, head_stride, d_po
                stream=None) -> None:
     _check(_L().tl_op_rope(_ptr(d_x), int(n_tokens), int(n_heads), int(head_dim), int(token_stride),
                           int(head_stride), _ptr(d_positions), float(theta), _stream(stream)))
+
+
+def tl_lane_kv_export(model, lane, layer, n_tokens, d_k, d_v, d_k_scales=None, d_v_scales=None,
+                      stream=None) -> None:
+    _check(_L().tl_lane_kv_export(model, int(lane), int(layer), int(n_tokens), _ptr(d_k), _ptr(d_v),
+                                 _ptr(d_k_scales), _ptr(d_v_scales), _stream(stream)))
+
+
+def tl_op_kv_quant_int8(d_x, n, head_dim, d_codes, d_scales, stream=None) -> None:
+    _check(_L().tl_op_kv_quant_int8(_ptr(d_x), int(n), int(head_dim), _ptr(d_codes), _ptr(d_scales),
+                                   _stream(stream)))
 
 
 def tl_op_gqa_decode(d_q, d_k, d_v, batch_stride, ctx_stride, n_keys, B, n_q_heads, n_kv_heads,

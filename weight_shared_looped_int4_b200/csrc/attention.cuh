@@ -317,7 +317,9 @@ struct PrefillAttnArgs {
   long long q_bstride;    // elements between batch entries
   int ldq;                // elements between tokens
   const __half* k;        // K plane of batch 0: [Hkv][ctx][hd]
-  const __half* v;
+  const __half* v;        // (INT8 cache: int8 codes at the same element offsets)
+  const float* ks;        // INT8 cache: K / V scales of batch 0 [Hkv][ctx]
+  const float* vs;        // (element offset / hd); NULL for fp16
   long long kv_bstride;
   int ctx;
   int T, pos0;
@@ -346,10 +348,14 @@ constexpr int kPfKeys = 64;   // keys per staged block
 constexpr int kPfPad = 8;     // fp16 padding per staged row
 
 __host__ __device__ inline size_t prefill_attn_smem_bytes(int hd) {
-  return (size_t)2 * kPfKeys * (hd + kPfPad) * 2;
+  return (size_t)2 * kPfKeys * (hd + kPfPad) * 2 + 2 * kPfKeys * 4;   // + INT8 cache scales
 }
 
-template <int HD, int REP, bool F32>
+// KV8: INT8 KV cache.  The codes are staged as fp16 (exact integers) and the
+// scales applied outside the MMAs: S column j times the key's scale, and the
+// softmax weights times the value's scale before P V (the weight sums use
+// the unscaled weights), so the result equals attention over code * scale.
+template <int HD, int REP, bool F32, bool KV8>
 __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const PrefillAttnArgs a) {
   constexpr int KC = HD / 16;        // k16 chunks of a head
   constexpr int NT = HD / 8;         // n8 tiles of the output
@@ -358,6 +364,8 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const Prefil
   extern __shared__ __align__(128) unsigned char psm[];
   __half* ks = reinterpret_cast<__half*>(psm);             // [64][LD]
   __half* vs = ks + kPfKeys * LD;                          // [64][LD]
+  float* sks = reinterpret_cast<float*>(vs + kPfKeys * LD);   // INT8: key / value scales [64] each
+  float* svs = sks + kPfKeys;
 
   const int qt = blockIdx.x, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -401,19 +409,46 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const Prefil
   const int nblk = last_key / kPfKeys + 1;
   const __half* kp = a.k + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
   const __half* vp = a.v + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
+  const int8_t* kp8 = reinterpret_cast<const int8_t*>(a.k) + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
+  const int8_t* vp8 = reinterpret_cast<const int8_t*>(a.v) + b * a.kv_bstride + (size_t)kvh * a.ctx * HD;
+  const float* ksp = KV8 ? a.ks + (b * a.kv_bstride) / HD + (size_t)kvh * a.ctx : nullptr;
+  const float* vsp = KV8 ? a.vs + (b * a.kv_bstride) / HD + (size_t)kvh * a.ctx : nullptr;
 
   for (int kb = 0; kb < nblk; ++kb) {
     const int j0 = kb * kPfKeys;
     __syncthreads();  // the previous block is no longer read
-    for (int c = threadIdx.x; c < kPfKeys * HD / 8; c += NTHR) {
-      const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
-      const bool ok = j0 + key <= last_key;
-      const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
-      cp_async16(ks + key * LD + off, kp + src, ok ? 16 : 0);
-      cp_async16(vs + key * LD + off, vp + src, ok ? 16 : 0);
+    if (KV8) {
+      // 16 codes per load, widened to fp16 (exact), zeros past the last key
+      for (int c = threadIdx.x; c < 2 * kPfKeys * HD / 16; c += NTHR) {
+        const int kv = c / (kPfKeys * HD / 16), rem = c % (kPfKeys * HD / 16);
+        const int key = rem / (HD / 16), off = (rem % (HD / 16)) * 16;
+        uint4 w = make_uint4(0, 0, 0, 0);
+        if (j0 + key <= last_key) w = __ldcg(reinterpret_cast<const uint4*>((kv ? vp8 : kp8) + (size_t)(j0 + key) * HD + off));
+        __half* dst = (kv ? vs : ks) + key * LD + off;
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint2 h;
+          h.x = pack_h2((float)(int8_t)(ws[i] & 0xffu), (float)(int8_t)((ws[i] >> 8) & 0xffu));
+          h.y = pack_h2((float)(int8_t)((ws[i] >> 16) & 0xffu), (float)(int8_t)(ws[i] >> 24));
+          *reinterpret_cast<uint2*>(dst + 4 * i) = h;
+        }
+      }
+      for (int c = threadIdx.x; c < 2 * kPfKeys; c += NTHR) {
+        const int kv = c / kPfKeys, key = c % kPfKeys;
+        sks[c] = (j0 + key <= last_key) ? __ldcg((kv ? vsp : ksp) + j0 + key) : 0.f;
+      }
+    } else {
+      for (int c = threadIdx.x; c < kPfKeys * HD / 8; c += NTHR) {
+        const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
+        const bool ok = j0 + key <= last_key;
+        const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
+        cp_async16(ks + key * LD + off, kp + src, ok ? 16 : 0);
+        cp_async16(vs + key * LD + off, vp + src, ok ? 16 : 0);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
     }
-    cp_async_commit();
-    cp_async_wait<0>();
     __syncthreads();
 
     // S = Q K^T for 64 keys: 8 n8 tiles
@@ -429,6 +464,11 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const Prefil
         const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kr + 8);
         mma_f16_16816(sc[n], qa[c], b0, b1);
         mma_f16_16816(sc[n], ql[c], b0, b1);
+      }
+      if (KV8) {   // column j of S times key j's scale
+        const float s0 = sks[n * 8 + 2 * t], s1 = sks[n * 8 + 2 * t + 1];
+        sc[n][0] *= s0; sc[n][1] *= s1;
+        sc[n][2] *= s0; sc[n][3] *= s1;
       }
     }
     // causal mask and online softmax (rows g and g+8 of the tile)
@@ -475,6 +515,14 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const Prefil
       o[n][2] *= c1; o[n][3] *= c1;
     }
     // O += P V: P as A fragments (hi, lo) straight from the S accumulators
+    if (KV8) {   // the weights times their value's scale (the sums above are unscaled)
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const float s0 = svs[n * 8 + 2 * t], s1 = svs[n * 8 + 2 * t + 1];
+        sc[n][0] *= s0; sc[n][1] *= s1;
+        sc[n][2] *= s0; sc[n][3] *= s1;
+      }
+    }
 #pragma unroll
     for (int kc = 0; kc < 4; ++kc) {
       uint32_t pa[4], pl[4];

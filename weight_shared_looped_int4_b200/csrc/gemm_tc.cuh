@@ -193,6 +193,9 @@ struct TcGemmArgs {
   int n_q_rows, n_kv_rows, hd;
   __half* k_plane;       // K plane [Hkv][ctx][hd] of this lane and layer
   __half* v_plane;
+  float* kv_stage;       // INT8 KV cache: rotated keys / values in fp32 at
+                         // [token][K|V][Hkv][hd] for the quantising pass
+                         // instead of the planes; NULL: fp16 cache
   int ctx, pos0;
   float theta;
   const float2* rope_tab;  // (cos, sin) [positions][hd/2], or NULL
@@ -218,6 +221,23 @@ struct TcGemmArgs {
   unsigned* tickets;     // [row tiles][token tiles], zero between launches
   int* err_flag;
 };
+
+// Key (kv = 0) or value elements j and j + hd/2 of kv head kvh for token t
+// (position pos): fp16 into the cache plane, or fp32 into the INT8 mode's
+// staging buffer.
+__device__ __forceinline__ void tc_kv_store(const TcGemmArgs& a, int t, int kv, int kvh, int pos, int j, float e0,
+                                            float e1) {
+  const int hd = a.hd;
+  if (a.kv_stage) {
+    float* dst = a.kv_stage + ((size_t)(t * 2 + kv) * (a.n_kv_rows / hd) + kvh) * hd;
+    dst[j] = e0;
+    dst[j + hd / 2] = e1;
+  } else {
+    __half* dst = (kv ? a.v_plane : a.k_plane) + ((size_t)kvh * a.ctx + pos) * hd;
+    dst[j] = __float2half_rn(e0);
+    dst[j + hd / 2] = __float2half_rn(e1);
+  }
+}
 
 // Final epilogue of `ntok` tokens of token tile tt (tile-local tokens tok0 ..
 // tok0 + ntok - 1) of row tile `tile`, whose sums are xch[ntok][kTcRows] in
@@ -301,14 +321,10 @@ __device__ void tc_epilogue_tokens(const TcGemmArgs& a, const float* xch, int ti
       } else if (na < a.n_q_rows + a.n_kv_rows) {
         const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
         const int kvh = (na - a.n_q_rows) / hd;
-        __half* dst = a.k_plane + ((size_t)kvh * a.ctx + pos) * hd;
-        dst[j] = __float2half_rn(va * cs.x - vb * cs.y);
-        dst[j + hh] = __float2half_rn(vb * cs.x + va * cs.y);
+        tc_kv_store(a, t, 0, kvh, pos, j, va * cs.x - vb * cs.y, vb * cs.x + va * cs.y);
       } else {
         const int kvh = (na - a.n_q_rows - a.n_kv_rows) / hd;
-        __half* dst = a.v_plane + ((size_t)kvh * a.ctx + pos) * hd;
-        dst[j] = __float2half_rn(va);
-        dst[j + hh] = __float2half_rn(vb);
+        tc_kv_store(a, t, 1, kvh, pos, j, va, vb);
       }
     }
   }
@@ -654,14 +670,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
           } else if (na < a.n_q_rows + a.n_kv_rows) {
             const float2 cs = rope_cs(a.rope_tab, pos, j, hd, a.theta);
             const int kvh = (na - a.n_q_rows) / hd;
-            __half* dst = a.k_plane + ((size_t)kvh * a.ctx + pos) * hd;
-            dst[j] = __float2half_rn(va * cs.x - vb * cs.y);
-            dst[j + hh] = __float2half_rn(vb * cs.x + va * cs.y);
+            tc_kv_store(a, t, 0, kvh, pos, j, va * cs.x - vb * cs.y, vb * cs.x + va * cs.y);
           } else {
             const int kvh = (na - a.n_q_rows - a.n_kv_rows) / hd;
-            __half* dst = a.v_plane + ((size_t)kvh * a.ctx + pos) * hd;
-            dst[j] = __float2half_rn(va);
-            dst[j + hh] = __float2half_rn(vb);
+            tc_kv_store(a, t, 1, kvh, pos, j, va, vb);
           }
         }
       }

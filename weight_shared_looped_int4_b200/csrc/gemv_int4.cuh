@@ -76,6 +76,9 @@ struct GemvArgs {
   int hd;
   __half* k_plane;     // K plane of this layer for lane 0: [Hkv][ctx][hd]
   __half* v_plane;     // V plane of this layer for lane 0
+  float* kv_stage;     // INT8 KV cache: the rotated keys and the values go here
+                       // in fp32, [row][K|V][Hkv][hd], for the quantising pass
+                       // (k_plane / v_plane unused); NULL: fp16 cache
   long long lane_stride;
   int ctx;
   const RowCtx* rows;  // per activation row
@@ -413,14 +416,27 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
     } else if (row0 < a.n_q_rows + a.n_kv_rows) {
       const float2 cs = rope_cs(a.rope_tab, rc.pos, j, hd, a.theta);
       const int kvh = (row0 - a.n_q_rows) / hd;
-      __half* dst = a.k_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
-      dst[j] = __float2half_rn(va * cs.x - vb * cs.y);
-      dst[j + hd / 2] = __float2half_rn(vb * cs.x + va * cs.y);
+      const float k0 = va * cs.x - vb * cs.y, k1 = vb * cs.x + va * cs.y;
+      if (a.kv_stage) {
+        float* dst = a.kv_stage + ((size_t)(m * 2) * (a.n_kv_rows / hd) + kvh) * hd;
+        dst[j] = k0;
+        dst[j + hd / 2] = k1;
+      } else {
+        __half* dst = a.k_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
+        dst[j] = __float2half_rn(k0);
+        dst[j + hd / 2] = __float2half_rn(k1);
+      }
     } else {
       const int kvh = (row0 - a.n_q_rows - a.n_kv_rows) / hd;
-      __half* dst = a.v_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
-      dst[j] = __float2half_rn(va);
-      dst[j + hd / 2] = __float2half_rn(vb);
+      if (a.kv_stage) {
+        float* dst = a.kv_stage + ((size_t)(m * 2 + 1) * (a.n_kv_rows / hd) + kvh) * hd;
+        dst[j] = va;
+        dst[j + hd / 2] = vb;
+      } else {
+        __half* dst = a.v_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
+        dst[j] = __float2half_rn(va);
+        dst[j + hd / 2] = __float2half_rn(vb);
+      }
     }
   }
   trace_mark(a.trace, 5);

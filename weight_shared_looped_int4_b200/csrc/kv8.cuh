@@ -1,0 +1,100 @@
+// INT8 KV cache storage: one fp32 scale per stored key or value vector (one
+// position, one kv head, HD elements), scale = max|x| / 127 and code =
+// round-half-even(x / scale), both decisions in fp32; an all-zero vector has
+// scale 0 and codes 0; the cache holds code * scale.  (TinyLoop README,
+// "Python API reference", KV cache modes: INT8 KV; the format is this
+// library's reading, the pages give none.)
+//
+// Layout: the int8 planes mirror the fp16 ones element for element
+// ([lanes][layers][K|V][Hkv][ctx][hd] at one byte per element); the scales
+// mirror them with the head dimension collapsed, so the scale of the vector
+// whose codes start at element offset e is at offset e / hd.
+#pragma once
+
+#include "common.cuh"
+
+namespace tl {
+
+// Quantise one vector held by a warp, E consecutive elements per lane: the
+// warp's max |x| gives the scale; q receives the codes.  Every lane returns
+// the scale.
+template <int E>
+__device__ __forceinline__ float kv8_quant_warp(const float (&x)[E], int (&q)[E]) {
+  float m = 0.f;
+#pragma unroll
+  for (int i = 0; i < E; ++i) m = fmaxf(m, fabsf(x[i]));
+  m = warp_max(m);
+  const float scale = m / 127.0f;   // IEEE division: the same fp32 value as the oracle's
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    int c = 0;
+    if (scale > 0.f) c = __float2int_rn(x[i] / scale);   // ties to even
+    q[i] = max(-127, min(127, c));
+  }
+  return scale;
+}
+
+// Four codes (one 32-bit word, lowest byte first) times their vector's scale.
+__device__ __forceinline__ float4 kv8_dequant4(uint32_t w, float scale) {
+  return make_float4((float)(int8_t)(w & 0xffu) * scale, (float)(int8_t)((w >> 8) & 0xffu) * scale,
+                     (float)(int8_t)((w >> 16) & 0xffu) * scale, (float)(int8_t)(w >> 24) * scale);
+}
+// Two codes (the low 16 bits, lowest byte first) times the scale.
+__device__ __forceinline__ float2 kv8_dequant2(uint32_t w, float scale) {
+  return make_float2((float)(int8_t)(w & 0xffu) * scale, (float)(int8_t)((w >> 8) & 0xffu) * scale);
+}
+
+struct Kv8QuantArgs {
+  const float* x;     // [n][HD] fp32
+  int n;
+  // flat output (op API): codes [n][HD], scales [n]
+  int8_t* codes;
+  float* scales;
+  // model staging (codes == NULL): vector v = (t * 2 + kv) * Hkv + head of a
+  // pass of tokens at positions pos0 + t goes to this layer's K (kv = 0) or V
+  // plane of the lane: codes at ((head * ctx + pos0 + t) * HD), scale at
+  // (head * ctx + pos0 + t)
+  int8_t* k8;
+  int8_t* v8;
+  float* ks;
+  float* vs;
+  int Hkv, ctx, pos0;
+};
+
+constexpr int kKv8Warps = 8;
+
+// One warp per vector.
+template <int HD>
+__global__ void __launch_bounds__(kKv8Warps * 32) kv8_quant_kernel(const Kv8QuantArgs a) {
+  constexpr int E = HD / 32;
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int v = blockIdx.x * kKv8Warps + (threadIdx.x >> 5);
+  if (v >= a.n) return;   // warp-uniform
+  float x[E];
+  const float* src = a.x + (size_t)v * HD + lane * E;
+#pragma unroll
+  for (int i = 0; i < E; ++i) x[i] = src[i];
+  int q[E];
+  const float scale = kv8_quant_warp<E>(x, q);
+  int8_t* dst;
+  float* sdst;
+  if (a.codes) {
+    dst = a.codes + (size_t)v * HD;
+    sdst = a.scales + v;
+  } else {
+    const int head = v % a.Hkv, kv = (v / a.Hkv) & 1, t = v / (2 * a.Hkv);
+    const size_t row = (size_t)head * a.ctx + a.pos0 + t;
+    dst = (kv ? a.v8 : a.k8) + row * HD;
+    sdst = (kv ? a.vs : a.ks) + row;
+  }
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < E; ++i) w |= ((uint32_t)q[i] & 0xffu) << (8 * i);
+  if (E == 4) *reinterpret_cast<uint32_t*>(dst + lane * E) = w;
+  else *reinterpret_cast<uint16_t*>(dst + lane * E) = (uint16_t)w;
+  if (lane == 0) *sdst = scale;
+}
+
+}  // namespace tl

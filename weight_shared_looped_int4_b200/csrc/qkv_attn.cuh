@@ -31,6 +31,7 @@
 
 #include "attention.cuh"
 #include "common.cuh"
+#include "kv8.cuh"
 
 namespace tl {
 
@@ -56,7 +57,9 @@ struct QkvAttnArgs {
   const float2* rope_tab;
   float theta;
   __half* k_plane;       // this layer's K plane of lane 0 [Hkv][ctx][hd]
-  __half* v_plane;
+  __half* v_plane;       // (INT8 cache: int8 codes at the same element offsets)
+  float* k_scale;        // INT8 cache: this layer's K / V scales of lane 0
+  float* v_scale;        // [Hkv][ctx] (element offset / hd)
   long long lane_stride;
   int ctx;
   float* o;              // attention output [M][Hq*hd] fp32
@@ -118,7 +121,10 @@ __device__ __forceinline__ void qa_st_peer2(unsigned addr, float x, float y) {
   asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
 }
 
-template <int HD>
+// KV8: INT8 KV cache (kv8.cuh): the new key / value are quantised by every
+// rank alike after the first exchange (rank 0 stores them) and the cached
+// keys / values are read as codes times their vector's scale.
+template <int HD, bool KV8>
 __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnArgs a) {
   constexpr int DPL = HD / 32;
   constexpr int ROW16 = HD / 8;
@@ -215,7 +221,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
         const int n = rcs[m].pos + 1, C = (n + kQaCluster - 1) / kQaCluster;
         lo[m] = min(n, c * C);
         const int hi = min(min(n, lo[m] + C), lo[m] + kQaChunk);
-        cnt[m] = max(0, min(hi, rcs[m].pos) - lo[m]);
+        cnt[m] = KV8 ? 0 : max(0, min(hi, rcs[m].pos) - lo[m]);   // INT8: plain loads below
         bytes += 2u * (unsigned)cnt[m] * HD * 2u;
       }
     }
@@ -362,12 +368,14 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     if (hh < rep) {
       dst_s = qb + (size_t)m * rep * HD + hh * HD;
     } else {
-      __half* cache = (hh == rep ? a.k_plane : a.v_plane) + rc.lane * a.lane_stride +
-                      ((size_t)grp * a.ctx + rc.pos) * HD;
-      const __half h0 = __float2half_rn(e0), h1 = __float2half_rn(e1);
-      if (ok) { cache[j] = h0; cache[j + HD / 2] = h1; }
-      e0 = __half2float(h0);    // attention reads the stored (fp16) key / value
-      e1 = __half2float(h1);
+      if (!KV8) {
+        __half* cache = (hh == rep ? a.k_plane : a.v_plane) + rc.lane * a.lane_stride +
+                        ((size_t)grp * a.ctx + rc.pos) * HD;
+        const __half h0 = __float2half_rn(e0), h1 = __float2half_rn(e1);
+        if (ok) { cache[j] = h0; cache[j + HD / 2] = h1; }
+        e0 = __half2float(h0);    // attention reads the stored (fp16) key / value
+        e1 = __half2float(h1);
+      }   // INT8: quantised after the exchange, below
       dst_s = (hh == rep ? knew : vnew) + (size_t)m * HD;
     }
     for (unsigned rk = 0; rk < kQaCluster; ++rk) {
@@ -378,6 +386,37 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   trace_mark(a.trace, 6);
   qa_cluster_sync();   // #1: q and the new key / value are in every rank
   trace_mark(a.trace, 3);
+  if (KV8) {
+    // INT8 cache: warp 2m + kv quantises row m's new key (kv = 0) or value;
+    // every rank computes the same codes, rank 0 stores them, and attention
+    // reads code * scale like any cached position
+    if (warp < 2 * M) {
+      const int m = warp >> 1, kv = warp & 1;
+      float* vec = (kv ? vnew : knew) + (size_t)m * HD;
+      float xv[DPL];
+      int qc[DPL];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) xv[i] = vec[lane * DPL + i];
+      const float sc8 = kv8_quant_warp<DPL>(xv, qc);
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) vec[lane * DPL + i] = (float)qc[i] * sc8;
+      if (c == 0 && ok) {
+        RowCtx rc = rcs[0];
+#pragma unroll
+        for (int q = 1; q < kQaMaxRows; ++q)
+          if (m == q) rc = rcs[q];
+        const size_t e = (size_t)rc.lane * a.lane_stride + ((size_t)grp * a.ctx + rc.pos) * HD;
+        int8_t* dst = reinterpret_cast<int8_t*>(kv ? a.v_plane : a.k_plane) + e;
+        uint32_t w = 0;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) w |= ((uint32_t)qc[i] & 0xffu) << (8 * i);
+        if (DPL == 4) *reinterpret_cast<uint32_t*>(dst + lane * 4) = w;
+        else *reinterpret_cast<uint16_t*>(dst + lane * 2) = (uint16_t)w;
+        if (lane == 0) (kv ? a.v_scale : a.k_scale)[e / HD] = sc8;
+      }
+    }
+    __syncthreads();
+  }
 
   // ---- attention over this rank's key split, per row: warp h < rep takes
   // query head h (scores, online softmax and P V stay inside the warp) ------
@@ -396,6 +435,16 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     const __half* vb = a.v_plane + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
     __half* ks = kvc + (size_t)m * 2 * kQaChunk * HD;      // [kQaChunk][HD]
     __half* vs = ks + kQaChunk * HD;
+    // INT8 cache: codes [K|V][kQaChunk][HD] then scales [K|V][kQaChunk] in the
+    // same area (half the fp16 chunk's bytes and then some)
+    const int8_t* kb8 = reinterpret_cast<const int8_t*>(a.k_plane) + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
+    const int8_t* vb8 = reinterpret_cast<const int8_t*>(a.v_plane) + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
+    const float* ksb = KV8 ? a.k_scale + (rc.lane * a.lane_stride) / HD + (size_t)grp * a.ctx : nullptr;
+    const float* vsb = KV8 ? a.v_scale + (rc.lane * a.lane_stride) / HD + (size_t)grp * a.ctx : nullptr;
+    int8_t* ks8 = reinterpret_cast<int8_t*>(ks);
+    int8_t* vs8 = ks8 + kQaChunk * HD;
+    float* ssk = reinterpret_cast<float*>(vs8 + kQaChunk * HD);   // [kQaChunk]
+    float* ssv = ssk + kQaChunk;
     // this lane's DPL dimensions of q (head `warp`) and of the new key / value
     float qv[DPL], kn[DPL], vn[DPL], o[DPL];
 #pragma unroll
@@ -410,7 +459,24 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     trace_mark(a.trace, 11);
     for (int jc = j0; jc < j1; jc += kQaChunk) {
       const int nk = min(kQaChunk, j1 - jc);
-      if (jc != j0) {
+      if (KV8) {
+        // every chunk by plain loads: 16 codes per load, then the scales; the
+        // new key is read from registers, not from here
+        __syncthreads();   // the previous chunk is consumed
+        constexpr int ROW16B = HD / 16;
+        for (int e = tid; e < 2 * kQaChunk * ROW16B; e += kQaThreads) {
+          const int kv = e / (kQaChunk * ROW16B), rem = e % (kQaChunk * ROW16B);
+          const int key = rem / ROW16B, pc = rem % ROW16B, jj = jc + key;
+          uint4 val = make_uint4(0, 0, 0, 0);
+          if (key < nk && jj != rc.pos) val = __ldcg(reinterpret_cast<const uint4*>((kv ? vb8 : kb8) + (size_t)jj * HD) + pc);
+          reinterpret_cast<uint4*>(ks8)[e] = val;
+        }
+        for (int e = tid; e < 2 * kQaChunk; e += kQaThreads) {
+          const int kv = e / kQaChunk, key = e % kQaChunk, jj = jc + key;
+          ssk[e] = (key < nk && jj != rc.pos) ? __ldcg((kv ? vsb : ksb) + jj) : 0.f;
+        }
+        __syncthreads();
+      } else if (jc != j0) {
         // later chunks (splits longer than kQaChunk keys): plain loads by
         // every thread; the new key is read from registers, not from here
         __syncthreads();   // the previous chunk is consumed
@@ -436,6 +502,12 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
               if (jc + jj == rc.pos) {
 #pragma unroll
                 for (int i = 0; i < DPL; ++i) kf[i] = kn[i];
+              } else if constexpr (KV8 && DPL == 4) {
+                const float4 f = kv8_dequant4(*reinterpret_cast<const uint32_t*>(ks8 + jj * HD + lane * 4), ssk[jj]);
+                kf[0] = f.x; kf[1] = f.y; kf[2] = f.z; kf[3] = f.w;
+              } else if constexpr (KV8) {
+                const float2 f = kv8_dequant2(*reinterpret_cast<const uint16_t*>(ks8 + jj * HD + lane * 2), ssk[jj]);
+                kf[0] = f.x; kf[1] = f.y;
               } else if constexpr (DPL == 4) {
                 const uint2 u2 = *reinterpret_cast<const uint2*>(ks + jj * HD + lane * 4);
                 const float2 f01 = h2_to_f2(u2.x), f23 = h2_to_f2(u2.y);
@@ -484,6 +556,12 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
           if (jc + jj == rc.pos) {
 #pragma unroll
             for (int i = 0; i < DPL; ++i) vf[i] = vn[i];
+          } else if constexpr (KV8 && DPL == 4) {
+            const float4 f = kv8_dequant4(*reinterpret_cast<const uint32_t*>(vs8 + jj * HD + lane * 4), ssv[jj]);
+            vf[0] = f.x; vf[1] = f.y; vf[2] = f.z; vf[3] = f.w;
+          } else if constexpr (KV8) {
+            const float2 f = kv8_dequant2(*reinterpret_cast<const uint16_t*>(vs8 + jj * HD + lane * 2), ssv[jj]);
+            vf[0] = f.x; vf[1] = f.y;
           } else if constexpr (DPL == 4) {
             const uint2 u2 = *reinterpret_cast<const uint2*>(vs + jj * HD + lane * 4);
             const float2 f01 = h2_to_f2(u2.x), f23 = h2_to_f2(u2.y);

@@ -204,12 +204,18 @@ cudaError_t init_device_kernels(int dev) {
   SET3(IN_F16, EPI_STORE) SET3(IN_F32, EPI_RESID) SET3(IN_NORM, EPI_SWIGLU) SET3(IN_NORM, EPI_ROPE_KV)
 #undef SET3
 #undef SET
-  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<64>, dev);
-  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<128>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<64, false>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<128, false>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<64, true>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<128, true>, dev);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(qkv_attn_kernel<64>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(qkv_attn_kernel<64, false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(qkv_attn_kernel<128>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(qkv_attn_kernel<64, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qkv_attn_kernel<128, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qkv_attn_kernel<128, false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess) e = allow_max_smem(decode_fused_kernel<64>, dev);
   if (e == cudaSuccess) e = allow_max_smem(decode_fused_kernel<128>, dev);
   if (e == cudaSuccess) e = allow_max_smem(head_argmax_kernel<1>, dev);
@@ -241,8 +247,9 @@ cudaError_t init_device_kernels(int dev) {
 #define ATT(HD, REP)                                                                  \
   if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, true>, dev);   \
   if (e == cudaSuccess) e = allow_max_smem(decode_attn_kernel<HD, REP, false>, dev);  \
-  if (e == cudaSuccess) e = allow_max_smem(prefill_attn_mma_kernel<HD, REP, true>, dev); \
-  if (e == cudaSuccess) e = allow_max_smem(prefill_attn_mma_kernel<HD, REP, false>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(prefill_attn_mma_kernel<HD, REP, true, false>, dev); \
+  if (e == cudaSuccess) e = allow_max_smem(prefill_attn_mma_kernel<HD, REP, false, false>, dev); \
+  if (e == cudaSuccess) e = allow_max_smem(prefill_attn_mma_kernel<HD, REP, true, true>, dev);
   ATT(64, 1) ATT(64, 2) ATT(64, 4) ATT(64, 8) ATT(128, 1) ATT(128, 2) ATT(128, 4) ATT(128, 8)
 #undef ATT
   if (e == cudaSuccess) g_dev_init[dev] = true;
@@ -285,6 +292,7 @@ cudaError_t launch_gemv_rows(GemvArgs a, int total, int in_mode, int epi, int gr
     if (c.y) c.y += (size_t)r0 * a.ldy;
     if (c.yf) c.yf += (size_t)r0 * a.ldy;
     if (c.resid) c.resid += (size_t)r0 * a.ldr;
+    if (c.kv_stage) c.kv_stage += (size_t)r0 * 2 * a.n_kv_rows;   // [row][K|V][Hkv * hd]
     const cudaError_t e = launch_gemv(c, grid, in_mode, epi, st);
     if (e != cudaSuccess) return e;
   }
@@ -600,7 +608,9 @@ std::atomic<int> g_at_min_tokens{1024};
 
 cudaError_t launch_prefill_attn(PrefillAttnArgs a, int B, int hd, int rep, bool f32, cudaStream_t st) {
   a.rep = rep;
-  if (a.T >= g_at_min_tokens.load(std::memory_order_relaxed)) {
+  const bool kv8 = a.ks != nullptr;   // INT8 KV cache: the 16-query tile kernel, fp32 queries
+  if (kv8 && !f32) return cudaErrorInvalidValue;
+  if (!kv8 && a.T >= g_at_min_tokens.load(std::memory_order_relaxed)) {
     // tensor cores (tcgen05): one CTA per (128-query tile, query head, batch entry)
     const dim3 grid((a.T + kAtQ - 1) / kAtQ, a.Hkv * rep, B);
     if (hd == 128)
@@ -621,8 +631,9 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, int B, int hd, int rep, bool 
   const size_t smem = prefill_attn_smem_bytes(hd);
 #define C(HD, REP)                                                                                       \
   if (hd == HD && hpc == REP)                                                                            \
-    return f32 ? launch(prefill_attn_mma_kernel<HD, REP, true>, grid, dim3(REP * 32), smem, st, a)       \
-               : launch(prefill_attn_mma_kernel<HD, REP, false>, grid, dim3(REP * 32), smem, st, a);
+    return kv8 ? launch(prefill_attn_mma_kernel<HD, REP, true, true>, grid, dim3(REP * 32), smem, st, a)  \
+               : f32 ? launch(prefill_attn_mma_kernel<HD, REP, true, false>, grid, dim3(REP * 32), smem, st, a) \
+                     : launch(prefill_attn_mma_kernel<HD, REP, false, false>, grid, dim3(REP * 32), smem, st, a);
   C(64, 1) C(64, 2) C(64, 4) C(64, 8) C(128, 1) C(128, 2) C(128, 4) C(128, 8)
 #undef C
   return cudaErrorInvalidValue;
@@ -644,8 +655,13 @@ struct tl_model {
   __half* embed = nullptr;
   __half* out_norm = nullptr;
   uint4* head_w = nullptr;
-  // KV cache: [max_lanes + 1][n_layers_max][2][Hkv][max_ctx][hd] fp16
+  // KV cache: [max_lanes + 1][n_layers_max][2][Hkv][max_ctx][hd] fp16, or
+  // with kv_int8 the same element layout in int8 codes (kv points at them)
+  // plus the scales kvs with the head dimension collapsed (kv8.cuh)
   __half* kv = nullptr;
+  float* kvs = nullptr;
+  float* kv_stage = nullptr;   // INT8: a pass's fp32 keys / values [rows][2][Hkv][hd]
+  bool kv_int8 = false;
   long long plane = 0, layer_stride = 0, lane_stride = 0;
   // workspaces
   float* x = nullptr;   // residual stream [rows][d]
@@ -696,8 +712,34 @@ struct tl_model {
 
   unsigned* attn_tickets() const { return tickets; }
   unsigned* head_ticket() const { return tickets + kMaxLanes * cfg.n_kv_heads; }
-  __half* k_plane(int layer) const { return kv + layer * layer_stride; }
-  __half* v_plane(int layer) const { return kv + layer * layer_stride + plane; }
+  // element pointers of lane 0's planes (int8 codes when kv_int8: same
+  // element offsets, reinterpreted by the kernels)
+  __half* k_plane(int layer) const {
+    return kv_int8 ? reinterpret_cast<__half*>(reinterpret_cast<int8_t*>(kv) + layer * layer_stride)
+                   : kv + layer * layer_stride;
+  }
+  __half* v_plane(int layer) const {
+    return kv_int8 ? reinterpret_cast<__half*>(reinterpret_cast<int8_t*>(kv) + layer * layer_stride + plane)
+                   : kv + layer * layer_stride + plane;
+  }
+  // INT8 scales of lane 0's planes (NULL for fp16); lane l adds l * lane_stride / hd
+  float* ks_plane(int layer) const { return kv_int8 ? kvs + layer * layer_stride / cfg.head_dim : nullptr; }
+  float* vs_plane(int layer) const {
+    return kv_int8 ? kvs + (layer * layer_stride + plane) / cfg.head_dim : nullptr;
+  }
+  // an element offset within the cache as a pointer into it (int8 or fp16)
+  __half* kv_at(long long e) const {
+    return kv_int8 ? reinterpret_cast<__half*>(reinterpret_cast<int8_t*>(kv) + e) : kv + e;
+  }
+  // planes and scales of one lane
+  __half* k_lane(int layer, int lane) const { return kv_at(layer * layer_stride + lane * lane_stride); }
+  __half* v_lane(int layer, int lane) const { return kv_at(layer * layer_stride + plane + lane * lane_stride); }
+  float* ks_lane(int layer, int lane) const {
+    return kv_int8 ? kvs + (layer * layer_stride + lane * lane_stride) / cfg.head_dim : nullptr;
+  }
+  float* vs_lane(int layer, int lane) const {
+    return kv_int8 ? kvs + (layer * layer_stride + plane + lane * lane_stride) / cfg.head_dim : nullptr;
+  }
   const BlockDev& block(int layer) const { return layer < cfg.n_pre ? pre[layer] : loop; }
 
   void free_all() {
@@ -707,7 +749,7 @@ struct tl_model {
       if (kv_.second.exec) cudaGraphExecDestroy(kv_.second.exec);
     graphs.clear();
     if (cap_stream) cudaStreamDestroy(cap_stream);
-    void* ptrs[] = {embed, out_norm, head_w, kv, x, q, o, h, rows, tok_index, out_row, spec_tok,
+    void* ptrs[] = {embed, out_norm, head_w, kv, kvs, kv_stage, x, q, o, h, rows, tok_index, out_row, spec_tok,
                     attn_part, tickets, head_val, head_idx, err_flag, io, tc.bt, tc.bt2, tc.bt3, tc.ss_attn,
                     tc.ss_ffn, tc.partial, tc.tickets,
                     rope_tab, fused_bar, fused_val, fused_idx};
@@ -762,6 +804,7 @@ tl_status validate_config(const tl_config* c) {
   if (c->max_ctx < 1 || c->max_ctx > 8192) return fail(TL_ERR_INVALID_ARG, "max_ctx must be in [1, 8192]");
   if (c->max_lanes < 1 || c->max_lanes > kMaxLanes) return fail(TL_ERR_INVALID_ARG, "max_lanes must be in [1, 16]");
   if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return fail(TL_ERR_INVALID_ARG, "bad eps or theta");
+  if (c->kv_mode != TL_KV_FP16 && c->kv_mode != TL_KV_INT8) return fail(TL_ERR_INVALID_ARG, "kv_mode must be TL_KV_FP16 or TL_KV_INT8");
   return TL_OK;
 }
 
@@ -819,6 +862,7 @@ tl_status run_qkv(tl_model* m, int layer, int M, float* x, const RowCtx* rows, f
   a.pair_mode = PAIR_ROPE; a.pair_off = hd / 32;
   a.q_out = q; a.ldq = qdim; a.n_q_rows = qdim; a.n_kv_rows = c.n_kv_heads * hd;
   a.k_plane = m->k_plane(layer); a.v_plane = m->v_plane(layer);
+  a.kv_stage = m->kv_stage;   // INT8: quantised by run_kv8 after this launch
   a.lane_stride = m->lane_stride; a.ctx = c.max_ctx;
   a.rope_tab = m->rope_tab;
   a.err_flag = m->err_flag;
@@ -880,10 +924,13 @@ tl_status run_qkv_attn(tl_model* m, int layer, int M, const RowCtx* rows, cudaSt
     a.l2_keep = layer >= c.n_pre;
     const size_t smem = qa_layout(c.d_model, a.M, a.rep, c.head_dim).total;
     const dim3 grid(kQaCluster, c.n_kv_heads);
-    if (c.head_dim == 64)
-      TL_CUDA(launch_impl(false, dim3(kQaCluster, 1, 1), qkv_attn_kernel<64>, grid, dim3(kQaThreads), smem, st, a));
-    else
-      TL_CUDA(launch_impl(false, dim3(kQaCluster, 1, 1), qkv_attn_kernel<128>, grid, dim3(kQaThreads), smem, st, a));
+    if (m->kv_int8) {
+      a.k_scale = m->ks_plane(layer);
+      a.v_scale = m->vs_plane(layer);
+    }
+    auto kern = c.head_dim == 64 ? (m->kv_int8 ? qkv_attn_kernel<64, true> : qkv_attn_kernel<64, false>)
+                                 : (m->kv_int8 ? qkv_attn_kernel<128, true> : qkv_attn_kernel<128, false>);
+    TL_CUDA(launch_impl(false, dim3(kQaCluster, 1, 1), kern, grid, dim3(kQaThreads), smem, st, a));
   }
   return TL_OK;
 }
@@ -953,12 +1000,32 @@ tl_status run_qkv_tc(tl_model* m, int layer, int lane, int T, int pos0, cudaStre
     ta.ss_k = (float)c.d_model; ta.ss_eps = c.rms_eps;
   }
   ta.q_out = m->q; ta.ldq = qdim; ta.n_q_rows = qdim; ta.n_kv_rows = c.n_kv_heads * hd; ta.hd = hd;
-  ta.k_plane = m->k_plane(layer) + lane * m->lane_stride;
-  ta.v_plane = m->v_plane(layer) + lane * m->lane_stride;
+  ta.k_plane = m->k_lane(layer, lane);
+  ta.v_plane = m->v_lane(layer, lane);
+  ta.kv_stage = m->kv_stage;   // INT8: quantised by run_kv8 after the GEMM
   ta.ctx = c.max_ctx; ta.pos0 = pos0; ta.theta = c.rope_theta; ta.rope_tab = m->rope_tab;
   kclass(TL_KERNEL_GEMM_TC);
   TL_CUDA(launch_tc_linear(b.qkv.tc, b.qkv.sz, c.d_model, b.qkv.N, b.qkv.n_tiles, handed ? PREP_NONE : PREP_NORM,
                            pa, ta, TC_ROPE_KV, T, m->tc, st));
+  return TL_OK;
+}
+
+// INT8 KV cache: quantise the pass's staged keys and values (T tokens at
+// positions pos0.. of `lane`) into the lane's slice `layer`.
+tl_status run_kv8(tl_model* m, int layer, int lane, int T, int pos0, cudaStream_t st) {
+  const tl_config& c = m->cfg;
+  Kv8QuantArgs ka{};
+  ka.x = m->kv_stage;
+  ka.n = T * 2 * c.n_kv_heads;
+  ka.k8 = reinterpret_cast<int8_t*>(m->k_lane(layer, lane));
+  ka.v8 = reinterpret_cast<int8_t*>(m->v_lane(layer, lane));
+  ka.ks = m->ks_lane(layer, lane);
+  ka.vs = m->vs_lane(layer, lane);
+  ka.Hkv = c.n_kv_heads; ka.ctx = c.max_ctx; ka.pos0 = pos0;
+  const dim3 grid((ka.n + kKv8Warps - 1) / kKv8Warps);
+  kclass(TL_KERNEL_SETUP);
+  if (c.head_dim == 64) TL_CUDA(launch(kv8_quant_kernel<64>, grid, dim3(kKv8Warps * 32), 0, st, ka));
+  else TL_CUDA(launch(kv8_quant_kernel<128>, grid, dim3(kKv8Warps * 32), 0, st, ka));
   return TL_OK;
 }
 
@@ -1061,11 +1128,14 @@ tl_status forward_tokens(tl_model* m, int lane, const int32_t* d_tokens, int T, 
   const bool tc = T >= kTcMinTokens;
   for (int layer = 0; layer < n_layers; ++layer) {
     tl_status rc = tc ? run_qkv_tc(m, layer, lane, T, pos0, st) : run_qkv(m, layer, T, m->x, m->rows, m->q, st);
+    if (rc == TL_OK && m->kv_int8) rc = run_kv8(m, layer, lane, T, pos0, st);
     if (rc != TL_OK) return rc;
     PrefillAttnArgs pa{};
     pa.qf = m->q; pa.q_bstride = 0; pa.ldq = qdim;
-    pa.k = m->k_plane(layer) + lane * m->lane_stride;
-    pa.v = m->v_plane(layer) + lane * m->lane_stride;
+    pa.k = m->k_lane(layer, lane);
+    pa.v = m->v_lane(layer, lane);
+    pa.ks = m->ks_lane(layer, lane);
+    pa.vs = m->vs_lane(layer, lane);
     pa.kv_bstride = 0; pa.ctx = c.max_ctx;
     pa.T = T; pa.pos0 = pos0; pa.Hkv = c.n_kv_heads;
     pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
@@ -1098,20 +1168,28 @@ tl_status decode_impl(tl_model* m, int n_lanes, const int32_t* h_lane_ids, const
                       const int32_t* h_loops, float* d_logits, int32_t* d_argmax, cudaStream_t st);
 
 // Copy positions [0, n) of every KV slice of `layers` layers from one lane to
-// another: runs of n * head_dim fp16 per (layer, K|V, kv head), 16 bytes per
-// thread, one CTA row per run (grid.y), the positions of a run over grid.x.
-__global__ void kv_copy_kernel(__half* __restrict__ kv, long long lane_stride, long long layer_stride,
-                               long long plane, int Hkv, int ctx, int hd, int src, int dst, int n) {
+// another: runs of n * head_dim elements of `esz` bytes (fp16 or int8 codes)
+// per (layer, K|V, kv head), 16 bytes per thread, one CTA row per run
+// (grid.y), the positions of a run over grid.x; with an INT8 cache also the
+// run's n scales (scales != NULL, their offsets are the codes' / hd).
+__global__ void kv_copy_kernel(unsigned char* __restrict__ kv, int esz, float* __restrict__ scales,
+                               long long lane_stride, long long layer_stride, long long plane, int Hkv, int ctx,
+                               int hd, int src, int dst, int n) {
   pdl_trigger();
   pdl_wait();
   const int run = blockIdx.y;                  // (layer * 2 + kv) * Hkv + head
   const int head = run % Hkv, kvsel = (run / Hkv) & 1, layer = run / (2 * Hkv);
   const size_t off = (size_t)layer * layer_stride + (size_t)kvsel * plane + (size_t)head * ctx * hd;
-  const uint4* s4 = reinterpret_cast<const uint4*>(kv + (size_t)src * lane_stride + off);
-  uint4* d4 = reinterpret_cast<uint4*>(kv + (size_t)dst * lane_stride + off);
-  const size_t n16 = (size_t)n * hd / 8;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
-    d4[i] = __ldcs(s4 + i);
+  const uint4* s4 = reinterpret_cast<const uint4*>(kv + ((size_t)src * lane_stride + off) * esz);
+  uint4* d4 = reinterpret_cast<uint4*>(kv + ((size_t)dst * lane_stride + off) * esz);
+  const size_t n16 = (size_t)n * hd * esz / 16;
+  const size_t i0 = (size_t)blockIdx.x * blockDim.x + threadIdx.x, step = (size_t)gridDim.x * blockDim.x;
+  for (size_t i = i0; i < n16; i += step) d4[i] = __ldcs(s4 + i);
+  if (scales) {
+    const float* ss = scales + ((size_t)src * lane_stride + off) / hd;
+    float* ds = scales + ((size_t)dst * lane_stride + off) / hd;
+    for (size_t i = i0; i < (size_t)n; i += step) ds[i] = __ldcs(ss + i);
+  }
 }
 
 }  // namespace
@@ -1195,8 +1273,17 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
   m->plane = (long long)c.n_kv_heads * c.max_ctx * hd;
   m->layer_stride = 2 * m->plane;
   m->lane_stride = (long long)m->n_layers_max * m->layer_stride;
-  m->kv_bytes = (size_t)(c.max_lanes + 1) * m->lane_stride * 2;
-  if (cudaMalloc(&m->kv, m->kv_bytes) != cudaSuccess) return bail(fail(TL_ERR_OOM, "KV cache (%zu bytes)", m->kv_bytes));
+  m->kv_int8 = c.kv_mode == TL_KV_INT8;
+  if (m->kv_int8) {   // one byte per element, then one fp32 scale per vector
+    const size_t codes = (size_t)(c.max_lanes + 1) * m->lane_stride;
+    const size_t scales = codes / hd * 4;
+    m->kv_bytes = codes + scales;
+    if (cudaMalloc(&m->kv, codes) != cudaSuccess || cudaMalloc(&m->kvs, scales) != cudaSuccess)
+      return bail(fail(TL_ERR_OOM, "KV cache (%zu bytes)", m->kv_bytes));
+  } else {
+    m->kv_bytes = (size_t)(c.max_lanes + 1) * m->lane_stride * 2;
+    if (cudaMalloc(&m->kv, m->kv_bytes) != cudaSuccess) return bail(fail(TL_ERR_OOM, "KV cache (%zu bytes)", m->kv_bytes));
+  }
 
   // workspaces
   const int rows = std::max(c.max_ctx, kMaxLanes);
@@ -1226,7 +1313,8 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
             alloc((void**)&m->head_idx, (size_t)std::max(m->head_grid, m->hd_grid) * 16 * 4) &&
             alloc((void**)&m->err_flag, 4) &&
             alloc((void**)&m->spec_tok, (2 * kMaxLanes + 2) * 4) &&
-            alloc((void**)&m->io, sizeof(HeadIO));
+            alloc((void**)&m->io, sizeof(HeadIO)) &&
+            (!m->kv_int8 || alloc((void**)&m->kv_stage, (size_t)rows * 2 * c.n_kv_heads * hd * 4));
   if (ok) {
     const int kmax = std::max(std::max(d, qdim), c.ffn_dim);
     m->tc.bt_bytes = tc_bt_bytes(rows, kmax, true);
@@ -1254,7 +1342,8 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
                   "fused partials ([4 rows][..][hd + 4]) must fit the layered path's buffer");
     int coop = 0;
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, device);
-    if (coop && (hd == 64 || hd == 128) && c.n_pre < kFusedMaxBlocks && rep_ok(rep)) {
+    // (the single-kernel step keeps an fp16 cache only)
+    if (coop && !m->kv_int8 && (hd == 64 || hd == 128) && c.n_pre < kFusedMaxBlocks && rep_ok(rep)) {
       FusedArgs& f = m->fused;
       for (int i = 0; i <= c.n_pre; ++i) {
         const BlockDev& b = i < c.n_pre ? m->pre[i] : m->loop;
@@ -1298,7 +1387,9 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
   {
     cudaFuncAttributes fa{};
     int optin = 0;
-    if (cudaFuncGetAttributes(&fa, hd == 64 ? qkv_attn_kernel<64> : qkv_attn_kernel<128>) == cudaSuccess &&
+    auto qa_kern = hd == 64 ? (m->kv_int8 ? qkv_attn_kernel<64, true> : qkv_attn_kernel<64, false>)
+                            : (m->kv_int8 ? qkv_attn_kernel<128, true> : qkv_attn_kernel<128, false>);
+    if (cudaFuncGetAttributes(&fa, qa_kern) == cudaSuccess &&
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) == cudaSuccess)
       m->qa_smem_max = optin - (int)fa.sharedSizeBytes;
     // the clustered kernel is used only if a cluster of its size fits the GPU
@@ -1315,12 +1406,14 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
     lc.numAttrs = 1;
     int n_clusters = 0;
     if (lc.dynamicSmemBytes > (size_t)m->qa_smem_max ||
-        cudaOccupancyMaxActiveClusters(&n_clusters, hd == 64 ? qkv_attn_kernel<64> : qkv_attn_kernel<128>, &lc) !=
+        cudaOccupancyMaxActiveClusters(&n_clusters, qa_kern, &lc) !=
             cudaSuccess ||
         n_clusters < 1)
       m->use_qkv_attn = false;
     cudaGetLastError();
   }
+  if (m->kv_int8 && !qkv_attn_ok(m))
+    return bail(fail(TL_ERR_UNSUPPORTED, "the INT8 KV cache needs the clustered decode kernel, which these shapes do not fit"));
   m->ws_bytes = ws;
   if (cudaStreamSynchronize(st) != cudaSuccess) return bail(fail(TL_ERR_CUDA, "setup sync"));
   m->lane_len.assign(c.max_lanes + 1, 0);
@@ -1658,11 +1751,14 @@ tl_status tl_score_early_exit(tl_model* m, const int32_t* d_tokens, int n_tokens
   int prev = -1, run = 0;
   for (int layer = 0; layer < c.n_pre + max_loops; ++layer) {
     tl_status rc = tc ? run_qkv_tc(m, layer, lane, T, 0, st) : run_qkv(m, layer, T, m->x, m->rows, m->q, st);
+    if (rc == TL_OK && m->kv_int8) rc = run_kv8(m, layer, lane, T, 0, st);
     if (rc != TL_OK) return rc;
     PrefillAttnArgs pa{};
     pa.qf = m->q; pa.q_bstride = 0; pa.ldq = qdim;
-    pa.k = m->k_plane(layer) + lane * m->lane_stride;
-    pa.v = m->v_plane(layer) + lane * m->lane_stride;
+    pa.k = m->k_lane(layer, lane);
+    pa.v = m->v_lane(layer, lane);
+    pa.ks = m->ks_lane(layer, lane);
+    pa.vs = m->vs_lane(layer, lane);
     pa.kv_bstride = 0; pa.ctx = c.max_ctx;
     pa.T = T; pa.pos0 = 0; pa.Hkv = c.n_kv_heads;
     pa.of = m->o; pa.o_bstride = 0; pa.ldo = qdim;
@@ -1711,11 +1807,39 @@ tl_status tl_lane_fork(tl_model* m, int src_lane, int dst_lane, int n_tokens, vo
   const int per_run16 = n_tokens * c.head_dim / 8;
   const int gx = std::max(1, std::min((per_run16 + 255) / 256, std::max(1, 4 * m->tc.n_sm / runs)));
   kclass(TL_KERNEL_SETUP);
-  TL_CUDA(launch(kv_copy_kernel, dim3(gx, runs), dim3(256), 0, (cudaStream_t)stream, m->kv,
-                 m->lane_stride, m->layer_stride, m->plane, c.n_kv_heads, c.max_ctx, c.head_dim, src_lane, dst_lane,
-                 n_tokens));
+  TL_CUDA(launch(kv_copy_kernel, dim3(gx, runs), dim3(256), 0, (cudaStream_t)stream,
+                 reinterpret_cast<unsigned char*>(m->kv), m->kv_int8 ? 1 : 2, m->kvs, m->lane_stride,
+                 m->layer_stride, m->plane, c.n_kv_heads, c.max_ctx, c.head_dim, src_lane, dst_lane, n_tokens));
   m->lane_len[dst_lane] = n_tokens;
   m->lane_loops[dst_lane] = m->lane_loops[src_lane];
+  return TL_OK;
+}
+
+tl_status tl_lane_kv_export(const tl_model* m, int lane, int layer, int n_tokens, void* d_k, void* d_v,
+                            float* d_k_scales, float* d_v_scales, void* stream) {
+  if (!m) return fail(TL_ERR_INVALID_ARG, "null model");
+  const tl_config& c = m->cfg;
+  if (lane < 0 || lane >= c.max_lanes) return fail(TL_ERR_INVALID_ARG, "lane %d out of range", lane);
+  if (m->lane_len[lane] == 0) return fail(TL_ERR_NOT_PREFILLED, "lane %d holds no prompt", lane);
+  if (layer < 0 || layer >= c.n_pre + m->lane_loops[lane])
+    return fail(TL_ERR_INVALID_ARG, "layer %d not in [0, %d)", layer, c.n_pre + m->lane_loops[lane]);
+  if (n_tokens < 1 || n_tokens > m->lane_len[lane])
+    return fail(TL_ERR_INVALID_ARG, "n_tokens %d not in [1, length of lane %d]", n_tokens, lane);
+  if (!d_k || !d_v || (m->kv_int8 && (!d_k_scales || !d_v_scales))) return fail(TL_ERR_INVALID_ARG, "null argument");
+  DeviceGuard guard(m->device);
+  if (!guard.ok) return fail(TL_ERR_CUDA, "cannot select device");
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t esz = m->kv_int8 ? 1 : 2, hd = c.head_dim;
+  for (int kv = 0; kv < 2; ++kv) {
+    const void* src = kv ? m->v_lane(layer, lane) : m->k_lane(layer, lane);
+    TL_CUDA(cudaMemcpy2DAsync(kv ? d_v : d_k, (size_t)n_tokens * hd * esz, src, (size_t)c.max_ctx * hd * esz,
+                              (size_t)n_tokens * hd * esz, c.n_kv_heads, cudaMemcpyDeviceToDevice, st));
+    if (m->kv_int8) {
+      const float* ssrc = kv ? m->vs_lane(layer, lane) : m->ks_lane(layer, lane);
+      TL_CUDA(cudaMemcpy2DAsync(kv ? d_v_scales : d_k_scales, (size_t)n_tokens * 4, ssrc, (size_t)c.max_ctx * 4,
+                                (size_t)n_tokens * 4, c.n_kv_heads, cudaMemcpyDeviceToDevice, st));
+    }
+  }
   return TL_OK;
 }
 
@@ -1989,6 +2113,19 @@ tl_status tl_op_rope(uint16_t* d_x, int n_tokens, int n_heads, int head_dim, lon
   TL_CUDA(launch(rope_inplace_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, (cudaStream_t)stream,
                  reinterpret_cast<__half*>(d_x), n_tokens, n_heads, head_dim, token_stride, head_stride,
                  d_positions, theta));
+  return TL_OK;
+}
+
+tl_status tl_op_kv_quant_int8(const float* d_x, int n, int head_dim, int8_t* d_codes, float* d_scales,
+                              void* stream) {
+  if (!d_x || !d_codes || !d_scales || n < 0) return fail(TL_ERR_INVALID_ARG, "null argument or n < 0");
+  if (head_dim != 64 && head_dim != 128) return fail(TL_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (n == 0) return TL_OK;
+  Kv8QuantArgs ka{};
+  ka.x = d_x; ka.n = n; ka.codes = d_codes; ka.scales = d_scales;
+  const dim3 grid((unsigned)((n + kKv8Warps - 1) / kKv8Warps));
+  if (head_dim == 64) TL_CUDA(launch(kv8_quant_kernel<64>, grid, dim3(kKv8Warps * 32), 0, (cudaStream_t)stream, ka));
+  else TL_CUDA(launch(kv8_quant_kernel<128>, grid, dim3(kKv8Warps * 32), 0, (cudaStream_t)stream, ka));
   return TL_OK;
 }
 
