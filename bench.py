@@ -905,10 +905,10 @@ def run_workload_attention(args):
     return 0
 
 
-def _lm_model(tl, tl_synth, max_loops, max_ctx, max_lanes):
+def _lm_model(tl, tl_synth, max_loops, max_ctx, max_lanes, kv_mode=0):
     shape = tl_synth.LOOPED_LM
     w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM)
-    cfg = tl.make_config(shape, max_loops=max_loops, max_ctx=max_ctx, max_lanes=max_lanes)
+    cfg = tl.make_config(shape, max_loops=max_loops, max_ctx=max_ctx, max_lanes=max_lanes, kv_mode=kv_mode)
     tw, keep = tl.make_weights(w)
     m = tl.tl_model_create(cfg, tw, 0)
     del keep
@@ -1124,7 +1124,72 @@ def run_workload_next(args):
     return 0
 
 
-WORKLOADS = {"tiny": run_workload_tiny, "linear": run_workload_linear,
+def run_workload_kv8(args):
+    """FP16 against INT8 KV cache on the 400M LM where the cache's bytes
+    count: 16 lanes with per-lane loops drawn from {4,8,16}, 1536-token
+    prompts, 256 greedy decode steps (context up to 1792 of 2048), and the
+    prefill of a 512-token prompt at L = 8.  Per mode: decode tokens/s, the
+    step's byte roofline (the cache's bytes per element: 2, or 1 + 4 / hd),
+    prefill ms and the cache's size."""
+    torch, dev, st = _dev_setup()
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    peaks = load_peaks()
+    P, n_dec, n = 1536, args.decode_steps if args.decode_steps != STEPS_DECODE else 256, 16
+    l2_gbs = None
+    res = []
+    launches0 = tl.tl_kernel_launch_count()
+    with ClockSampler(0) as clocks:
+        for mode, name in ((0, "fp16"), (1, "int8")):
+            w, m = _lm_model(tl, tl_synth, 16, 2048, n, kv_mode=mode)
+            if l2_gbs is None:
+                l2_gbs, _, _ = probe_read_bandwidths(tl, torch, dev, st)
+            prompts = tl_synth.make_lane_prompts(tl_synth.SEED_LSWEEP, w.shape.vocab, n, P + 1)
+            d_prompts = torch.as_tensor(prompts, device=dev)
+            hist = torch.zeros((n_dec + 1, n), dtype=torch.int32, device=dev)
+            hp = hist.data_ptr()
+            loops = [int(v) for v in tl_synth.make_lane_loops(tl_synth.SEED_LSWEEP, n)]
+            lanes = list(range(n))
+
+            def decode_run():
+                for i, lane in enumerate(lanes):
+                    tl.tl_prefill(m, lane, d_prompts[lane], P, loops[i], None, None, st)
+                with torch.cuda.stream(st):
+                    hist[0, :n].copy_(d_prompts[:n, P])
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(st)
+                for i in range(n_dec):
+                    tl.tl_decode_step(m, lanes, hp + 4 * n * i, loops, None, hp + 4 * n * (i + 1), st)
+                b.record(st)
+                b.synchronize()
+                return a.elapsed_time(b)
+
+            decode_run()     # warm (graph capture)
+            ms = decode_run()
+            per_elem = 2.0 if mode == 0 else 1.0 + 4.0 / HD
+            kv = sum((2 + L) * 2 * HKV * HD * per_elem * (P + n_dec / 2) for L in loops)
+            t_roof, _, _ = _decode_roofline_us(kv, loops, l2_gbs, peaks)
+            us_step = 1e3 * ms / n_dec
+            fn = lambda: tl.tl_prefill(m, 0, d_prompts[0, :512], 512, 8, None, None, st)
+            for _ in range(3):
+                fn()
+            pf = _time_reps(torch, st, fn, 10)
+            res.append({"kv": name, "kv_cache_bytes": tl.tl_model_info(m)["kv_bytes"],
+                        "decode_tok_s": round(n * n_dec / (ms / 1e3), 1), "us_per_step": round(us_step, 2),
+                        "kv_bytes_per_step": int(kv), "roofline_us_per_step": round(t_roof, 2),
+                        "frac": round(t_roof / us_step, 4), "prefill_T512_L8_ms": round(pf, 4)})
+            tl.tl_check_device_error(m)
+            tl.tl_model_destroy(m)
+    print(json.dumps({"workload": "400M looped LM, FP16 vs INT8 KV cache: 16 lanes, loops from {4,8,16}, "
+                                  "1536-token prompts, 256 decode steps (ctx 2048)",
+                      "metric": "decode tok/s, byte roofline fraction, prefill ms (T=512, L=8), cache bytes",
+                      "loops": loops, "decode_steps": n_dec, "peaks": peaks, "l2_read_gbs": round(l2_gbs, 1),
+                      "results": res, "gpu_launches": tl.tl_kernel_launch_count() - launches0,
+                      "clocks": clocks.summary()}))
+    return 0
+
+
+WORKLOADS = {"tiny": run_workload_tiny, "linear": run_workload_linear, "kv8": run_workload_kv8,
              "attention": run_workload_attention, "lsweep": run_workload_lsweep,
              "peaks": run_workload_peaks, "next": run_workload_next}
 
