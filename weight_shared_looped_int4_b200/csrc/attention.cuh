@@ -17,6 +17,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "kv8.cuh"
 
 namespace tl {
 
@@ -428,9 +429,11 @@ __global__ void __launch_bounds__(REP * 32) prefill_attn_mma_kernel(const Prefil
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
+          __half2 c01, c23;
+          kv8_codes_h2(ws[i], c01, c23);
           uint2 h;
-          h.x = pack_h2((float)(int8_t)(ws[i] & 0xffu), (float)(int8_t)((ws[i] >> 8) & 0xffu));
-          h.y = pack_h2((float)(int8_t)((ws[i] >> 16) & 0xffu), (float)(int8_t)(ws[i] >> 24));
+          h.x = *reinterpret_cast<const uint32_t*>(&c01);
+          h.y = *reinterpret_cast<const uint32_t*>(&c23);
           *reinterpret_cast<uint2*>(dst + 4 * i) = h;
         }
       }

@@ -34,14 +34,29 @@ __device__ __forceinline__ float kv8_quant_warp(const float (&x)[E], int (&q)[E]
   return scale;
 }
 
-// Four codes (one 32-bit word, lowest byte first) times their vector's scale.
-__device__ __forceinline__ float4 kv8_dequant4(uint32_t w, float scale) {
-  return make_float4((float)(int8_t)(w & 0xffu) * scale, (float)(int8_t)((w >> 8) & 0xffu) * scale,
-                     (float)(int8_t)((w >> 16) & 0xffu) * scale, (float)(int8_t)(w >> 24) * scale);
+// Four codes (one 32-bit word, lowest byte first) as two fp16 pairs, exact:
+// the biased byte code + 128 goes into the mantissa of 1024 (fp16 0x6400)
+// and 1152 = 1024 + 128 is subtracted.
+__device__ __forceinline__ void kv8_codes_h2(uint32_t w, __half2& c01, __half2& c23) {
+  const uint32_t u = w ^ 0x80808080u;                       // code + 128, per byte
+  const uint32_t lo = __byte_perm(u, 0x64646464u, 0x4140);  // (1024 + u0, 1024 + u1)
+  const uint32_t hi = __byte_perm(u, 0x64646464u, 0x4342);  // (1024 + u2, 1024 + u3)
+  const __half2 bias = __halves2half2(__ushort_as_half((unsigned short)0x6480), __ushort_as_half((unsigned short)0x6480));
+  c01 = __hsub2(*reinterpret_cast<const __half2*>(&lo), bias);
+  c23 = __hsub2(*reinterpret_cast<const __half2*>(&hi), bias);
 }
-// Two codes (the low 16 bits, lowest byte first) times the scale.
-__device__ __forceinline__ float2 kv8_dequant2(uint32_t w, float scale) {
-  return make_float2((float)(int8_t)(w & 0xffu) * scale, (float)(int8_t)((w >> 8) & 0xffu) * scale);
+// Four codes as floats (no scale).
+__device__ __forceinline__ float4 kv8_codes4(uint32_t w) {
+  __half2 a, b;
+  kv8_codes_h2(w, a, b);
+  const float2 fa = __half22float2(a), fb = __half22float2(b);
+  return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+// Two codes (the low 16 bits) as floats (no scale).
+__device__ __forceinline__ float2 kv8_codes2(uint32_t w) {
+  __half2 a, b;
+  kv8_codes_h2(w, a, b);
+  return __half22float2(a);
 }
 
 struct Kv8QuantArgs {

@@ -221,8 +221,8 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
         const int n = rcs[m].pos + 1, C = (n + kQaCluster - 1) / kQaCluster;
         lo[m] = min(n, c * C);
         const int hi = min(min(n, lo[m] + C), lo[m] + kQaChunk);
-        cnt[m] = KV8 ? 0 : max(0, min(hi, rcs[m].pos) - lo[m]);   // INT8: plain loads below
-        bytes += 2u * (unsigned)cnt[m] * HD * 2u;
+        cnt[m] = max(0, min(hi, rcs[m].pos) - lo[m]);
+        bytes += 2u * (unsigned)cnt[m] * HD * (KV8 ? 1u : 2u);
       }
     }
     mbar_arrive_expect_tx(&kvbar, bytes);
@@ -231,8 +231,35 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       if (cnt[m] > 0) {
         const size_t src = (size_t)rcs[m].lane * a.lane_stride + ((size_t)grp * a.ctx + lo[m]) * HD;
         __half* dst = kvc + (size_t)m * 2 * kQaChunk * HD;
-        bulk_g2s(dst, a.k_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
-        bulk_g2s(dst + kQaChunk * HD, a.v_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
+        if (KV8) {   // codes only (their scales follow with plain loads below)
+          int8_t* d8 = reinterpret_cast<int8_t*>(dst);
+          bulk_g2s(d8, reinterpret_cast<const int8_t*>(a.k_plane) + src, (unsigned)cnt[m] * HD, &kvbar);
+          bulk_g2s(d8 + kQaChunk * HD, reinterpret_cast<const int8_t*>(a.v_plane) + src, (unsigned)cnt[m] * HD,
+                   &kvbar);
+        } else {
+          bulk_g2s(dst, a.k_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
+          bulk_g2s(dst + kQaChunk * HD, a.v_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
+        }
+      }
+    }
+  }
+  // INT8: the first chunk's scales (their offsets are not 16-byte aligned,
+  // so plain loads) by warp 1, under the GEMV like the codes' bulk copies
+  if (KV8 && warp == 1) {
+    for (int m = 0; m < M; ++m) {
+      RowCtx rc = rcs[0];
+#pragma unroll
+      for (int q = 1; q < kQaMaxRows; ++q)
+        if (m == q) rc = rcs[q];
+      const int n = rc.pos + 1, C = (n + kQaCluster - 1) / kQaCluster;
+      const int j0 = min(n, c * C), j1 = min(n, j0 + C), nk = min(kQaChunk, j1 - j0);
+      float* ssk0 = reinterpret_cast<float*>(reinterpret_cast<int8_t*>(kvc + (size_t)m * 2 * kQaChunk * HD) +
+                                             2 * kQaChunk * HD);
+      const float* ksb = a.k_scale + (rc.lane * a.lane_stride) / HD + (size_t)grp * a.ctx;
+      const float* vsb = a.v_scale + (rc.lane * a.lane_stride) / HD + (size_t)grp * a.ctx;
+      for (int e = lane; e < 2 * kQaChunk; e += 32) {
+        const int kv = e / kQaChunk, key = e % kQaChunk, jj = j0 + key;
+        ssk0[e] = (key < nk && jj != rc.pos) ? __ldcg((kv ? vsb : ksb) + jj) : 0.f;
       }
     }
   }
@@ -459,9 +486,9 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     trace_mark(a.trace, 11);
     for (int jc = j0; jc < j1; jc += kQaChunk) {
       const int nk = min(kQaChunk, j1 - jc);
-      if (KV8) {
-        // every chunk by plain loads: 16 codes per load, then the scales; the
-        // new key is read from registers, not from here
+      if (KV8 && jc != j0) {
+        // later chunks by plain loads: 16 codes per load, then the scales;
+        // the new key is read from registers, not from here
         __syncthreads();   // the previous chunk is consumed
         constexpr int ROW16B = HD / 16;
         for (int e = tid; e < 2 * kQaChunk * ROW16B; e += kQaThreads) {
@@ -502,11 +529,11 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
               if (jc + jj == rc.pos) {
 #pragma unroll
                 for (int i = 0; i < DPL; ++i) kf[i] = kn[i];
-              } else if constexpr (KV8 && DPL == 4) {
-                const float4 f = kv8_dequant4(*reinterpret_cast<const uint32_t*>(ks8 + jj * HD + lane * 4), ssk[jj]);
+              } else if constexpr (KV8 && DPL == 4) {   // codes; the key's scale after the sum
+                const float4 f = kv8_codes4(*reinterpret_cast<const uint32_t*>(ks8 + jj * HD + lane * 4));
                 kf[0] = f.x; kf[1] = f.y; kf[2] = f.z; kf[3] = f.w;
               } else if constexpr (KV8) {
-                const float2 f = kv8_dequant2(*reinterpret_cast<const uint16_t*>(ks8 + jj * HD + lane * 2), ssk[jj]);
+                const float2 f = kv8_codes2(*reinterpret_cast<const uint16_t*>(ks8 + jj * HD + lane * 2));
                 kf[0] = f.x; kf[1] = f.y;
               } else if constexpr (DPL == 4) {
                 const uint2 u2 = *reinterpret_cast<const uint2*>(ks + jj * HD + lane * 4);
@@ -527,7 +554,8 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
             for (int u = 0; u < 8; ++u) p[u] += __shfl_xor_sync(0xffffffffu, p[u], off);
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            if (lane == u && j8 + u < nk) sh[j8 + u] = p[u] * scale;
+            if (lane == u && j8 + u < nk)
+              sh[j8 + u] = p[u] * scale * ((KV8 && jc + j8 + u != rc.pos) ? ssk[j8 + u] : 1.f);
         }
         __syncwarp();
         // online softmax over the chunk
@@ -551,16 +579,18 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
         for (int i = 0; i < DPL; ++i) o[i] *= alpha;
 #pragma unroll 4
         for (int jj = 0; jj < nk; ++jj) {
-          const float pj = sh[jj];
+          float pj = sh[jj];
           float vf[DPL];
           if (jc + jj == rc.pos) {
 #pragma unroll
             for (int i = 0; i < DPL; ++i) vf[i] = vn[i];
-          } else if constexpr (KV8 && DPL == 4) {
-            const float4 f = kv8_dequant4(*reinterpret_cast<const uint32_t*>(vs8 + jj * HD + lane * 4), ssv[jj]);
+          } else if constexpr (KV8 && DPL == 4) {   // codes; the weight carries the value's scale
+            pj *= ssv[jj];
+            const float4 f = kv8_codes4(*reinterpret_cast<const uint32_t*>(vs8 + jj * HD + lane * 4));
             vf[0] = f.x; vf[1] = f.y; vf[2] = f.z; vf[3] = f.w;
           } else if constexpr (KV8) {
-            const float2 f = kv8_dequant2(*reinterpret_cast<const uint16_t*>(vs8 + jj * HD + lane * 2), ssv[jj]);
+            pj *= ssv[jj];
+            const float2 f = kv8_codes2(*reinterpret_cast<const uint16_t*>(vs8 + jj * HD + lane * 2));
             vf[0] = f.x; vf[1] = f.y;
           } else if constexpr (DPL == 4) {
             const uint2 u2 = *reinterpret_cast<const uint2*>(vs + jj * HD + lane * 4);
