@@ -45,20 +45,6 @@ __device__ __forceinline__ void kv8_codes_h2(uint32_t w, __half2& c01, __half2& 
   c01 = __hsub2(*reinterpret_cast<const __half2*>(&lo), bias);
   c23 = __hsub2(*reinterpret_cast<const __half2*>(&hi), bias);
 }
-// Four codes as floats (no scale).
-__device__ __forceinline__ float4 kv8_codes4(uint32_t w) {
-  __half2 a, b;
-  kv8_codes_h2(w, a, b);
-  const float2 fa = __half22float2(a), fb = __half22float2(b);
-  return make_float4(fa.x, fa.y, fb.x, fb.y);
-}
-// Two codes (the low 16 bits) as floats (no scale).
-__device__ __forceinline__ float2 kv8_codes2(uint32_t w) {
-  __half2 a, b;
-  kv8_codes_h2(w, a, b);
-  return __half22float2(a);
-}
-
 struct Kv8QuantArgs {
   const float* x;     // [n][HD] fp32
   int n;

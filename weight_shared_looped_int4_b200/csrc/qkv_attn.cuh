@@ -80,7 +80,7 @@ __host__ __device__ inline int qa_units_per_cta(int rep, int hd) {
 // first chunk, then later chunks), the partials this rank merges, activation
 // planes, reduction buffer, q and the new key/value of every row, scores.
 struct QaLayout {
-  size_t w, kvc, pml, pv, act, red, q, kv, total;
+  size_t w, kvc, pml, pv, act, red, q, kv, kvs, total;
 };
 __host__ __device__ inline QaLayout qa_layout(int K, int M, int rep, int hd) {
   QaLayout L;
@@ -95,7 +95,8 @@ __host__ __device__ inline QaLayout qa_layout(int K, int M, int rep, int hd) {
   L.red = L.act + ((size_t)M * (K + 8) * 2 * 2 + 127) / 128 * 128;
   L.q = L.red + (size_t)kQaWarps * 2 * kQaMaxUnits * 64 * 4;
   L.kv = L.q + (size_t)M * rep * hd * 4;
-  L.total = L.kv + (size_t)2 * M * hd * 4 + 128;   // + scores and softmax state
+  L.kvs = L.kv + (size_t)2 * M * hd * 4;             // INT8 cache: the chunk's scales [m][K|V][kQaChunk]
+  L.total = L.kvs + (size_t)M * 2 * kQaChunk * 4 + 128;   // + scores and softmax state
   L.total += (size_t)(rep * kQaChunk + 4 * rep) * 4;
   return L;
 }
@@ -145,7 +146,8 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   float* qb = reinterpret_cast<float*>(qsm + L.q);          // [m][rep * hd]
   float* knew = reinterpret_cast<float*>(qsm + L.kv);       // [m][hd]
   float* vnew = knew + (size_t)M * HD;                       // [m][hd]
-  float* sc = vnew + (size_t)M * HD;                         // [rep][kQaChunk]
+  float* kvs = reinterpret_cast<float*>(qsm + L.kvs);      // INT8: [m][K|V][kQaChunk] scales
+  float* sc = kvs + (size_t)M * 2 * kQaChunk;                // [rep][kQaChunk]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, t4 = lane & 3;
   const unsigned crank = qa_cluster_rank();
@@ -231,8 +233,8 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       if (cnt[m] > 0) {
         const size_t src = (size_t)rcs[m].lane * a.lane_stride + ((size_t)grp * a.ctx + lo[m]) * HD;
         __half* dst = kvc + (size_t)m * 2 * kQaChunk * HD;
-        if (KV8) {   // codes only (their scales follow with plain loads below)
-          int8_t* d8 = reinterpret_cast<int8_t*>(dst);
+        if (KV8) {   // codes only, staged in the V half (their scales follow with plain loads below)
+          int8_t* d8 = reinterpret_cast<int8_t*>(dst + kQaChunk * HD);
           bulk_g2s(d8, reinterpret_cast<const int8_t*>(a.k_plane) + src, (unsigned)cnt[m] * HD, &kvbar);
           bulk_g2s(d8 + kQaChunk * HD, reinterpret_cast<const int8_t*>(a.v_plane) + src, (unsigned)cnt[m] * HD,
                    &kvbar);
@@ -253,8 +255,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
         if (m == q) rc = rcs[q];
       const int n = rc.pos + 1, C = (n + kQaCluster - 1) / kQaCluster;
       const int j0 = min(n, c * C), j1 = min(n, j0 + C), nk = min(kQaChunk, j1 - j0);
-      float* ssk0 = reinterpret_cast<float*>(reinterpret_cast<int8_t*>(kvc + (size_t)m * 2 * kQaChunk * HD) +
-                                             2 * kQaChunk * HD);
+      float* ssk0 = kvs + (size_t)m * 2 * kQaChunk;
       const float* ksb = a.k_scale + (rc.lane * a.lane_stride) / HD + (size_t)grp * a.ctx;
       const float* vsb = a.v_scale + (rc.lane * a.lane_stride) / HD + (size_t)grp * a.ctx;
       for (int e = lane; e < 2 * kQaChunk; e += 32) {
@@ -462,15 +463,15 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     const __half* vb = a.v_plane + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
     __half* ks = kvc + (size_t)m * 2 * kQaChunk * HD;      // [kQaChunk][HD]
     __half* vs = ks + kQaChunk * HD;
-    // INT8 cache: codes [K|V][kQaChunk][HD] then scales [K|V][kQaChunk] in the
-    // same area (half the fp16 chunk's bytes and then some)
+    // INT8 cache: each chunk's codes are widened once into the fp16 layout
+    // above (exact integers; the first chunk's bulk copy lands as int8 in the
+    // V half first), its scales go to ssk / ssv and are applied per key
     const int8_t* kb8 = reinterpret_cast<const int8_t*>(a.k_plane) + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
     const int8_t* vb8 = reinterpret_cast<const int8_t*>(a.v_plane) + rc.lane * a.lane_stride + (size_t)grp * a.ctx * HD;
     const float* ksb = KV8 ? a.k_scale + (rc.lane * a.lane_stride) / HD + (size_t)grp * a.ctx : nullptr;
     const float* vsb = KV8 ? a.v_scale + (rc.lane * a.lane_stride) / HD + (size_t)grp * a.ctx : nullptr;
-    int8_t* ks8 = reinterpret_cast<int8_t*>(ks);
-    int8_t* vs8 = ks8 + kQaChunk * HD;
-    float* ssk = reinterpret_cast<float*>(vs8 + kQaChunk * HD);   // [kQaChunk]
+    const int8_t* stage8 = reinterpret_cast<const int8_t*>(vs);   // [K|V][kQaChunk][HD] codes of the first chunk
+    float* ssk = kvs + (size_t)m * 2 * kQaChunk;                  // [kQaChunk]
     float* ssv = ssk + kQaChunk;
     // this lane's DPL dimensions of q (head `warp`) and of the new key / value
     float qv[DPL], kn[DPL], vn[DPL], o[DPL];
@@ -486,21 +487,45 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     trace_mark(a.trace, 11);
     for (int jc = j0; jc < j1; jc += kQaChunk) {
       const int nk = min(kQaChunk, j1 - jc);
-      if (KV8 && jc != j0) {
-        // later chunks by plain loads: 16 codes per load, then the scales;
-        // the new key is read from registers, not from here
-        __syncthreads();   // the previous chunk is consumed
+      if (KV8) {
+        // codes into registers (16 per load): the first chunk from its staged
+        // bulk copy, later ones from the cache; then widened to fp16 in the
+        // chunk layout; the new key is read from registers, not from here
         constexpr int ROW16B = HD / 16;
-        for (int e = tid; e < 2 * kQaChunk * ROW16B; e += kQaThreads) {
+        constexpr int PER = 2 * kQaChunk * ROW16B / kQaThreads;
+        static_assert(PER * kQaThreads == 2 * kQaChunk * ROW16B, "whole chunk per pass");
+        const bool first = jc == j0;
+        if (first && !mbar_wait(&kvbar, 0) && tid == 0) atomicOr(a.err_flag, kErrTimeout);
+        __syncthreads();   // the previous chunk is consumed
+        uint4 cv[PER];
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+          const int e = tid + u * kQaThreads;
           const int kv = e / (kQaChunk * ROW16B), rem = e % (kQaChunk * ROW16B);
           const int key = rem / ROW16B, pc = rem % ROW16B, jj = jc + key;
-          uint4 val = make_uint4(0, 0, 0, 0);
-          if (key < nk && jj != rc.pos) val = __ldcg(reinterpret_cast<const uint4*>((kv ? vb8 : kb8) + (size_t)jj * HD) + pc);
-          reinterpret_cast<uint4*>(ks8)[e] = val;
+          cv[u] = make_uint4(0, 0, 0, 0);
+          if (key < nk && jj != rc.pos)
+            cv[u] = first ? reinterpret_cast<const uint4*>(stage8)[e]
+                          : __ldcg(reinterpret_cast<const uint4*>((kv ? vb8 : kb8) + (size_t)jj * HD) + pc);
         }
-        for (int e = tid; e < 2 * kQaChunk; e += kQaThreads) {
-          const int kv = e / kQaChunk, key = e % kQaChunk, jj = jc + key;
-          ssk[e] = (key < nk && jj != rc.pos) ? __ldcg((kv ? vsb : ksb) + jj) : 0.f;
+        if (!first)
+          for (int e = tid; e < 2 * kQaChunk; e += kQaThreads) {
+            const int kv = e / kQaChunk, key = e % kQaChunk, jj = jc + key;
+            ssk[e] = (key < nk && jj != rc.pos) ? __ldcg((kv ? vsb : ksb) + jj) : 0.f;
+          }
+        __syncthreads();   // the staged codes are read
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+          const int e = tid + u * kQaThreads;   // 16 codes -> 16 fp16 at element 16 e of [K|V][kQaChunk][HD]
+          const uint32_t ws[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
+          uint4 h0, h1;
+          __half2 c01, c23;
+          kv8_codes_h2(ws[0], c01, c23); h0.x = *reinterpret_cast<uint32_t*>(&c01); h0.y = *reinterpret_cast<uint32_t*>(&c23);
+          kv8_codes_h2(ws[1], c01, c23); h0.z = *reinterpret_cast<uint32_t*>(&c01); h0.w = *reinterpret_cast<uint32_t*>(&c23);
+          kv8_codes_h2(ws[2], c01, c23); h1.x = *reinterpret_cast<uint32_t*>(&c01); h1.y = *reinterpret_cast<uint32_t*>(&c23);
+          kv8_codes_h2(ws[3], c01, c23); h1.z = *reinterpret_cast<uint32_t*>(&c01); h1.w = *reinterpret_cast<uint32_t*>(&c23);
+          reinterpret_cast<uint4*>(ks)[2 * e] = h0;
+          reinterpret_cast<uint4*>(ks)[2 * e + 1] = h1;
         }
         __syncthreads();
       } else if (jc != j0) {
@@ -529,13 +554,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
               if (jc + jj == rc.pos) {
 #pragma unroll
                 for (int i = 0; i < DPL; ++i) kf[i] = kn[i];
-              } else if constexpr (KV8 && DPL == 4) {   // codes; the key's scale after the sum
-                const float4 f = kv8_codes4(*reinterpret_cast<const uint32_t*>(ks8 + jj * HD + lane * 4));
-                kf[0] = f.x; kf[1] = f.y; kf[2] = f.z; kf[3] = f.w;
-              } else if constexpr (KV8) {
-                const float2 f = kv8_codes2(*reinterpret_cast<const uint16_t*>(ks8 + jj * HD + lane * 2));
-                kf[0] = f.x; kf[1] = f.y;
-              } else if constexpr (DPL == 4) {
+              } else if constexpr (DPL == 4) {   // (INT8: the codes; the key's scale after the sum)
                 const uint2 u2 = *reinterpret_cast<const uint2*>(ks + jj * HD + lane * 4);
                 const float2 f01 = h2_to_f2(u2.x), f23 = h2_to_f2(u2.y);
                 kf[0] = f01.x; kf[1] = f01.y; kf[2] = f23.x; kf[3] = f23.y;
@@ -584,19 +603,13 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
           if (jc + jj == rc.pos) {
 #pragma unroll
             for (int i = 0; i < DPL; ++i) vf[i] = vn[i];
-          } else if constexpr (KV8 && DPL == 4) {   // codes; the weight carries the value's scale
-            pj *= ssv[jj];
-            const float4 f = kv8_codes4(*reinterpret_cast<const uint32_t*>(vs8 + jj * HD + lane * 4));
-            vf[0] = f.x; vf[1] = f.y; vf[2] = f.z; vf[3] = f.w;
-          } else if constexpr (KV8) {
-            pj *= ssv[jj];
-            const float2 f = kv8_codes2(*reinterpret_cast<const uint16_t*>(vs8 + jj * HD + lane * 2));
-            vf[0] = f.x; vf[1] = f.y;
           } else if constexpr (DPL == 4) {
+            if (KV8) pj *= ssv[jj];   // INT8: the codes; the weight carries the value's scale
             const uint2 u2 = *reinterpret_cast<const uint2*>(vs + jj * HD + lane * 4);
             const float2 f01 = h2_to_f2(u2.x), f23 = h2_to_f2(u2.y);
             vf[0] = f01.x; vf[1] = f01.y; vf[2] = f23.x; vf[3] = f23.y;
           } else {
+            if (KV8) pj *= ssv[jj];
             const float2 f01 = h2_to_f2(*reinterpret_cast<const unsigned*>(vs + jj * HD + lane * 2));
             vf[0] = f01.x; vf[1] = f01.y;
           }
