@@ -15,7 +15,9 @@ What it computes, step by step, in the order the pages give it:
   1 and 2; TinyLoop docs, "Async API", "Scoring"/"Generation": ``loops=`` on every
   call);
 * group-wise INT4 weights with zero points, w = (q - z) * s, group 128 along K
-  (TinyLoop README, "Status", INT4 loop / pre linears with zero points);
+  (TinyLoop README, "Status", INT4 loop / pre linears with zero points), or the
+  INT2 body with the same form and 2-bit fields (TinyLoop README, "Current
+  Runtime Snapshot": INT2 is the default body; format read as INT4's);
 * RMSNorm (tiny-llm feature list, "Root Mean Square Normalizations");
 * RoPE applied to Q and K with a configurable theta (TinyLoop README, "Status",
   Rotary Position Embeddings; tiny-llm feature list, "Rotary Positional
@@ -103,6 +105,34 @@ def dequantize(qweight: np.ndarray, scales: np.ndarray, qzeros: np.ndarray,
     q = unpack_nibbles(qweight, K).astype(np.float64)            # [N][K]
     z = unpack_nibbles(qzeros, G).astype(np.float64)             # [N][G]
     s = np.asarray(scales, dtype=np.float16).astype(np.float64)  # [N][G]
+    group = np.arange(K) // GROUP_SIZE
+    return (q - z[:, group]) * s[:, group]
+
+
+def unpack_crumbs(words: np.ndarray, n: int) -> np.ndarray:
+    """Decode ``n`` 2-bit values per row from uint32 words, lowest field first.
+
+    Element k of a row is bits 2*(k % 16) .. 2*(k % 16)+1 of word k // 16 (the
+    INT2 body's storage, this library's reading; the pages name the INT2 body,
+    TinyLoop README "Current Runtime Snapshot", but give no format).
+    """
+    w = np.asarray(words, dtype=np.uint32)
+    out = np.empty(w.shape[:-1] + (w.shape[-1] * 16,), dtype=np.uint8)
+    for j in range(16):
+        out[..., j::16] = (w >> np.uint32(2 * j)) & np.uint32(0x3)
+    return out[..., :n]
+
+
+def dequantize_int2(qweight: np.ndarray, scales: np.ndarray, qzeros: np.ndarray,
+                    K: int) -> np.ndarray:
+    """W[n, k] = (q[n, k] - z[n, k // 128]) * s[n, k // 128] for the INT2
+    storage (q, z in [0, 3]), in float64; every value is exact."""
+    if K % GROUP_SIZE:
+        raise ValueError("K must be a multiple of 128")
+    G = K // GROUP_SIZE
+    q = unpack_crumbs(qweight, K).astype(np.float64)
+    z = unpack_crumbs(qzeros, G).astype(np.float64)
+    s = np.asarray(scales, dtype=np.float16).astype(np.float64)
     group = np.arange(K) // GROUP_SIZE
     return (q - z[:, group]) * s[:, group]
 
@@ -254,6 +284,8 @@ class DenseBlock:
 def dense_block(blk) -> DenseBlock:
     """Dequantize every linear of a ``tl_synth.BlockWeights``."""
     def deq(lin):
+        if getattr(lin, "bits", 4) == 2:
+            return dequantize_int2(lin.qweight, lin.scales, lin.qzeros, lin.K)
         return dequantize(lin.qweight, lin.scales, lin.qzeros, lin.K)
     return DenseBlock(
         attn_norm=np.asarray(blk.attn_norm, np.float64),

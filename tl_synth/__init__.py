@@ -18,6 +18,15 @@ definition w = (q - z) * s):
                                       unused nibbles are 0
 * no "+1" offset is applied to the stored zero point.
 
+The INT2 body (TinyLoop README, "Current Runtime Snapshot": INT2 is the
+default body; the pages give no format) uses the same layout with 2-bit
+fields, this library's reading: ``qweight`` uint32 [N][K/16] with element k in
+bits 2*(k%16)..2*(k%16)+1 of word k//16 (lowest field first), ``scales``
+float16 [N][K/128], ``qzeros`` uint32 [N][ceil(G/16)] (16 zero points per
+word), w = (q - z) * s with q, z in {0..3}.  Its draws: q ~ U{0..3},
+z ~ U{0..3}, s ~ U(0.02, 0.08) (a stated choice: it gives the weights about the
+INT4 draws' spread, std(q - z) * mean(s) ~ 0.08).
+
 Draw order for :func:`make_model_weights` (one ``numpy.random.default_rng(seed)``
 stream, PCG64): embedding, then for each block in the order pre[0] .. pre[n_pre-1],
 loop: attn_norm gain, ffn_norm gain, then the linears qkv, o, gate_up, down, each
@@ -99,17 +108,37 @@ def pack_nibbles(values: np.ndarray) -> np.ndarray:
     return out
 
 
+def pack_crumbs(values: np.ndarray) -> np.ndarray:
+    """Pack 2-bit values along the last axis, sixteen per uint32, lowest field
+    first: ``values[..., k]`` lands in bits 2*(k%16) of word ``k//16``.  The
+    last axis is zero-padded to a multiple of sixteen."""
+    v = np.asarray(values, dtype=np.uint32)
+    if v.size and (v.max() > 3):
+        raise ValueError("2-bit value out of range")
+    n = v.shape[-1]
+    pad = (-n) % 16
+    if pad:
+        v = np.concatenate([v, np.zeros(v.shape[:-1] + (pad,), np.uint32)], axis=-1)
+    v = v.reshape(v.shape[:-1] + (v.shape[-1] // 16, 16))
+    out = np.zeros(v.shape[:-1], dtype=np.uint32)
+    for j in range(16):
+        out |= v[..., j] << np.uint32(2 * j)
+    return out
+
+
 @dataclass
 class Int4Linear:
-    """One INT4 linear layer in the storage format, plus the raw draws."""
+    """One INT4 (or INT2: bits = 2) linear layer in the storage format, plus
+    the raw draws."""
 
     K: int
     N: int
-    qweight: np.ndarray  # uint32 [N][K/8]
+    qweight: np.ndarray  # uint32 [N][K/8] (INT2: [N][K/16])
     scales: np.ndarray   # float16 [N][K/128]
-    qzeros: np.ndarray   # uint32 [N][ceil(K/128/8)]
+    qzeros: np.ndarray   # uint32 [N][ceil(K/128/8)] (INT2: [N][ceil(K/128/16)])
     q: np.ndarray        # uint8 [N][K]   raw codes (kept for format tests)
     z: np.ndarray        # uint8 [N][K/128] raw zero points
+    bits: int = 4
 
     @property
     def n_groups(self) -> int:
@@ -126,6 +155,17 @@ def make_int4_linear(rng: np.random.Generator, N: int, K: int,
     s = rng.uniform(scale_lo, scale_hi, size=(N, G)).astype(np.float16)
     return Int4Linear(K=K, N=N, qweight=pack_nibbles(q), scales=s,
                       qzeros=pack_nibbles(z), q=q, z=z)
+
+
+def make_int2_linear(rng: np.random.Generator, N: int, K: int,
+                     scale_lo: float = 0.02, scale_hi: float = 0.08) -> Int4Linear:
+    if K % GROUP_SIZE:
+        raise ValueError("K must be a multiple of the group size")
+    G = K // GROUP_SIZE
+    q = rng.integers(0, 4, size=(N, K), dtype=np.uint8)
+    z = rng.integers(0, 4, size=(N, G), dtype=np.uint8)
+    s = rng.uniform(scale_lo, scale_hi, size=(N, G)).astype(np.float16)
+    return Int4Linear(K=K, N=N, qweight=pack_crumbs(q), scales=s, qzeros=pack_crumbs(z), q=q, z=z, bits=2)
 
 
 @dataclass
@@ -152,22 +192,26 @@ def _gain(rng, d):
     return rng.uniform(0.8, 1.2, size=d).astype(np.float16)
 
 
-def make_block(rng: np.random.Generator, shape: ModelShape) -> BlockWeights:
+def make_block(rng: np.random.Generator, shape: ModelShape, bits: int = 4) -> BlockWeights:
     d, F = shape.d_model, shape.ffn_dim
+    lin = make_int4_linear if bits == 4 else make_int2_linear
     attn_norm = _gain(rng, d)
     ffn_norm = _gain(rng, d)
-    qkv = make_int4_linear(rng, shape.qkv_rows, d)
-    o = make_int4_linear(rng, d, shape.n_q_heads * shape.head_dim)
-    gate_up = make_int4_linear(rng, 2 * F, d)
-    down = make_int4_linear(rng, d, F)
+    qkv = lin(rng, shape.qkv_rows, d)
+    o = lin(rng, d, shape.n_q_heads * shape.head_dim)
+    gate_up = lin(rng, 2 * F, d)
+    down = lin(rng, d, F)
     return BlockWeights(attn_norm, ffn_norm, qkv, o, gate_up, down)
 
 
-def make_model_weights(shape: ModelShape, seed: int) -> ModelWeights:
+def make_model_weights(shape: ModelShape, seed: int, bits: int = 4) -> ModelWeights:
+    """Every block's linears INT4 (bits = 4) or INT2 (bits = 2)."""
+    if bits not in (2, 4):
+        raise ValueError("bits must be 2 or 4")
     rng = np.random.default_rng(seed)
     embed = rng.normal(0.0, 0.02, size=(shape.vocab, shape.d_model)).astype(np.float16)
-    pre = [make_block(rng, shape) for _ in range(shape.n_pre)]
-    loop = make_block(rng, shape)
+    pre = [make_block(rng, shape, bits) for _ in range(shape.n_pre)]
+    loop = make_block(rng, shape, bits)
     out_norm = _gain(rng, shape.d_model)
     head = rng.normal(0.0, 0.02, size=(shape.vocab, shape.d_model)).astype(np.float16)
     return ModelWeights(shape=shape, embed=embed, out_norm=out_norm, head=head,
