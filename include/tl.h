@@ -70,6 +70,7 @@ typedef struct {
   float rms_eps;    /* RMSNorm epsilon */
   float rope_theta; /* RoPE base */
   int kv_mode;      /* TL_KV_FP16 (0) or TL_KV_INT8, see below */
+  int weight_bits;  /* block linears: 4 (or 0) INT4, 2 the INT2 body, see tl_int4_linear */
 } tl_config;
 
 /* KV cache storage (TinyLoop README, "Python API reference", KV cache modes:
@@ -85,7 +86,14 @@ typedef struct {
  * (TL_DECODE_FUSED) is FP16 only. */
 enum { TL_KV_FP16 = 0, TL_KV_INT8 = 1 };
 
-/* One INT4 linear with K inputs and N outputs, HOST memory, storage format:
+/* One INT4 linear with K inputs and N outputs, HOST memory, storage format
+ * (with tl_config.weight_bits = 2 / tl_linear_create_int2, the INT2 body of
+ * TinyLoop README, "Current Runtime Snapshot", whose format the pages do not
+ * give, read as the same layout with 2-bit fields: qweight uint32
+ * [N][K/16] with element k in bits 2*(k%16)..+1 of word k/16, qzeros uint32
+ * [N][ceil(K/2048)] with sixteen 2-bit zero points per word, q and z in
+ * 0..3; the decode kernels then read half the weight bytes, the prefill GEMM
+ * widens the codes to its 4-bit tile layout at load):
  *   qweight uint32 [N][K/8]        element k of row n is bits 4*(k%8)..+3 of
  *                                  word k/8 (low nibble first)
  *   scales  fp16   [N][K/128]      scale of (row, group)
@@ -405,6 +413,9 @@ unsigned long long tl_kernel_launch_count(void);
  * 1 <= N <= 65536.  The host arrays may be freed when this returns. */
 tl_status tl_linear_create(const tl_int4_linear *w, int K, int N, int device,
                            tl_linear **out);
+/* tl_linear_create for an INT2 linear (the 2-bit storage described above). */
+tl_status tl_linear_create_int2(const tl_int4_linear *w, int K, int N, int device,
+                                tl_linear **out);
 void tl_linear_destroy(tl_linear *l);
 
 /* Kernel family used by tl_linear_forward. */

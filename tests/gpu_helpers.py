@@ -57,8 +57,8 @@ def check_argmax(gpu_idx: int, oracle_logits: np.ndarray, where: str = "", margi
 class GpuModel:
     """A tl_model built from tl_synth weights, destroyed on close()."""
 
-    def __init__(self, weights, max_loops, max_ctx, max_lanes, device=0, kv_mode=0):
-        cfg = tl.make_config(weights.shape, max_loops, max_ctx, max_lanes, kv_mode)
+    def __init__(self, weights, max_loops, max_ctx, max_lanes, device=0, kv_mode=0, weight_bits=4):
+        cfg = tl.make_config(weights.shape, max_loops, max_ctx, max_lanes, kv_mode, weight_bits)
         tw, keep = tl.make_weights(weights)
         self.handle = tl.tl_model_create(cfg, tw, device)
         del keep

@@ -58,7 +58,7 @@ class tl_config(ctypes.Structure):
     _fields_ = [("d_model", c_int), ("n_q_heads", c_int), ("n_kv_heads", c_int),
                 ("head_dim", c_int), ("ffn_dim", c_int), ("vocab", c_int), ("n_pre", c_int),
                 ("max_loops", c_int), ("max_ctx", c_int), ("max_lanes", c_int),
-                ("rms_eps", c_float), ("rope_theta", c_float), ("kv_mode", c_int)]
+                ("rms_eps", c_float), ("rope_theta", c_float), ("kv_mode", c_int), ("weight_bits", c_int)]
 
 
 class tl_int4_linear(ctypes.Structure):
@@ -116,6 +116,7 @@ def _load():
         "tl_op_rmsnorm": (st, [P, P, c_int, c_int, c_float, P, P]),
         "tl_op_rope": (st, [P, c_int, c_int, c_int, c_longlong, c_longlong, P, c_float, P]),
         "tl_op_kv_quant_int8": (st, [P, c_int, c_int, P, P, P]),
+        "tl_linear_create_int2": (st, [POINTER(tl_int4_linear), c_int, c_int, c_int, POINTER(c_void_p)]),
         "tl_lane_kv_export": (st, [P, c_int, c_int, c_int, P, P, P, P, P]),
         "tl_op_gqa_decode": (st, [P, P, P, c_longlong, c_int, P, c_int, c_int, c_int, c_int, P, P]),
         "tl_op_gqa_prefill": (st, [P, P, P, c_longlong, c_int, c_int, c_int, c_int, c_int, c_int,
@@ -159,6 +160,7 @@ EXPORTED = sorted(["tl_model_profile_start", "tl_model_profile_stop", "tl_kernel
                    "tl_linear_create", "tl_linear_destroy", "tl_linear_forward", "tl_op_rmsnorm",
                    "tl_op_rope", "tl_op_gqa_decode", "tl_op_gqa_prefill", "tl_status_string",
                    "tl_op_gqa_decode_noalloc", "tl_op_kv_quant_int8", "tl_lane_kv_export",
+                   "tl_linear_create_int2",
                    "tl_last_error", "tl_version"])
 
 
@@ -208,12 +210,13 @@ def _i32_host(values):
 
 # ------------------------------------------------------------ marshalling ---
 
-def make_config(shape, max_loops: int, max_ctx: int, max_lanes: int, kv_mode: int = 0) -> tl_config:
+def make_config(shape, max_loops: int, max_ctx: int, max_lanes: int, kv_mode: int = 0,
+                weight_bits: int = 4) -> tl_config:
     """tl_config from an object with the ModelShape attribute names
-    (kv_mode TL_KV_FP16 or TL_KV_INT8)."""
+    (kv_mode TL_KV_FP16 or TL_KV_INT8; weight_bits 4 or 2 for the INT2 body)."""
     return tl_config(shape.d_model, shape.n_q_heads, shape.n_kv_heads, shape.head_dim,
                      shape.ffn_dim, shape.vocab, shape.n_pre, max_loops, max_ctx, max_lanes,
-                     float(shape.rms_eps), float(shape.rope_theta), int(kv_mode))
+                     float(shape.rms_eps), float(shape.rope_theta), int(kv_mode), int(weight_bits))
 
 
 def make_int4_linear(lin) -> tl_int4_linear:
@@ -388,9 +391,12 @@ def tl_kernel_launch_count() -> int:
 
 
 def tl_linear_create(lin, K: int, N: int, device: int = 0) -> int:
+    """A device linear from host storage arrays; INT2 (lin.bits == 2) goes
+    through tl_linear_create_int2."""
     out = c_void_p()
     w = make_int4_linear(lin)
-    _check(_L().tl_linear_create(ctypes.byref(w), int(K), int(N), int(device), ctypes.byref(out)))
+    fn = _L().tl_linear_create_int2 if getattr(lin, "bits", 4) == 2 else _L().tl_linear_create
+    _check(fn(ctypes.byref(w), int(K), int(N), int(device), ctypes.byref(out)))
     return out.value
 
 

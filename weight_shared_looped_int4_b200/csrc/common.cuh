@@ -202,6 +202,25 @@ __device__ __forceinline__ void unpack_a_frag(uint32_t w, uint32_t zz, uint32_t 
   a[3] = h2_sub(nib_pair_to_h2_biased(w >> 12), zhi);  // row g+8, k 2t+8..2t+9
 }
 
+// INT2 weights: two 2-bit fields (bits 0..1 and 16..17 of w) as an fp16 pair
+// biased by 1024, exact.
+__device__ __forceinline__ uint32_t crumb_pair_to_h2_biased(uint32_t w) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "r"(0x00030003u), "r"(0x64006400u));
+  return r;
+}
+// The m16n8k16 A fragment of k16 step s (0 or 1) held by one INT2 word: the
+// fields of step s sit at bits 8s + 2r (pair r, first element) and
+// 16 + 8s + 2r (second element), r = 0..3 in the order of unpack_a_frag.
+__device__ __forceinline__ void unpack_a_frag2(uint32_t w, int s, uint32_t zz, uint32_t (&a)[4]) {
+  const uint32_t zlo = h2_lo_lo(zz), zhi = h2_hi_hi(zz);
+  const uint32_t ws = w >> (8 * s);
+  a[0] = h2_sub(crumb_pair_to_h2_biased(ws), zlo);        // row g,   k 2t..2t+1
+  a[1] = h2_sub(crumb_pair_to_h2_biased(ws >> 2), zhi);   // row g+8, k 2t..2t+1
+  a[2] = h2_sub(crumb_pair_to_h2_biased(ws >> 4), zlo);   // row g,   k 2t+8..2t+9
+  a[3] = h2_sub(crumb_pair_to_h2_biased(ws >> 6), zhi);   // row g+8, k 2t+8..2t+9
+}
+
 // Byte offset of element pair (row, k..k+1), k even, in a 128-byte-swizzled
 // K-major tile of `rows` rows and 128 k (two 64-wide atoms): the operand
 // layout of the tcgen05 GEMM's B tiles and A stages.

@@ -696,9 +696,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_int4_tc_kernel(const TcGem
 // the tensor-core layout, from the storage format (qweight [N][K/8] words,
 // element k in bits 4 (k % 8); qzeros [N][ceil(G/8)] words).  perm_F != 0
 // interleaves gate and up rows per 128-row tile (see tc_row_orig).
+// bits = 2: the INT2 body's storage (element k in bits 2 (k % 16) of word
+// k / 16, 16 zero points per word), widened to the same nibble layout.
 __global__ void repack_int4_tc_kernel(const uint32_t* __restrict__ qweight, const uint32_t* __restrict__ qzeros,
-                                      int K, int N, int perm_F, uint8_t* __restrict__ out) {
-  const int G = K >> 7, zw = (G + 7) >> 3;
+                                      int K, int N, int perm_F, uint8_t* __restrict__ out, int bits) {
+  const int G = K >> 7, zw = bits == 2 ? (G + 15) >> 4 : (G + 7) >> 3;
   const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int row_tiles = (N + kTcRows - 1) / kTcRows;
   const size_t total = (size_t)row_tiles * G * kTcRows * 16;
@@ -711,11 +713,20 @@ __global__ void repack_int4_tc_kernel(const uint32_t* __restrict__ qweight, cons
   uint8_t* base = out + blk * kTcRawBytes;
   uint32_t word = 0, z = 0;
   if (n < N) {
-    const uint32_t src = qweight[(size_t)n * (K >> 3) + g * 16 + j];   // k = 128 g + 8 j + i at bits 4 i
-    // destination nibble slot of k_i: i even -> 4 (i / 2), i odd -> 16 + 4 (i / 2)
+    // k = 128 g + 8 j + i; destination nibble slot of k_i: i even -> 4 (i / 2),
+    // i odd -> 16 + 4 (i / 2)
+    if (bits == 2) {
+      const uint32_t src = qweight[(size_t)n * (K >> 4) + g * 8 + (j >> 1)];   // k_i at bits 2 (8 (j & 1) + i)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) word |= ((src >> (4 * i)) & 0xFu) << ((i & 1) * 16 + 4 * (i >> 1));
-    z = (qzeros[(size_t)n * zw + (g >> 3)] >> (4 * (g & 7))) & 0xFu;
+      for (int i = 0; i < 8; ++i)
+        word |= ((src >> (2 * (8 * (j & 1) + i))) & 0x3u) << ((i & 1) * 16 + 4 * (i >> 1));
+      z = (qzeros[(size_t)n * zw + (g >> 4)] >> (2 * (g & 15))) & 0x3u;
+    } else {
+      const uint32_t src = qweight[(size_t)n * (K >> 3) + g * 16 + j];   // k_i at bits 4 i
+#pragma unroll
+      for (int i = 0; i < 8; ++i) word |= ((src >> (4 * i)) & 0xFu) << ((i & 1) * 16 + 4 * (i >> 1));
+      z = (qzeros[(size_t)n * zw + (g >> 3)] >> (4 * (g & 7))) & 0xFu;
+    }
   }
   reinterpret_cast<uint32_t*>(base)[r * 16 + j] = word;
   if (j == 0) reinterpret_cast<uint16_t*>(base + kTcRows * 64)[r] = (uint16_t)(0x6400u + z);

@@ -90,6 +90,7 @@ struct GemvArgs {
                               // (6) activations staged
   int trigger;                // PdlTrigger
   int l2_keep;                // 1: the weights are the loop block's (L2 evict-last), else evict-first
+  int bits;                   // 4, or 2: INT2 weights (selects gemv_int4_kernel<.., 2>)
 };
 
 constexpr int kGemvThreads = 256;
@@ -100,7 +101,8 @@ constexpr int kGemvThreads = 256;
 __host__ __device__ inline size_t gemv_act_bytes(int K, int M, bool lo) {
   return (((size_t)M * (K + 8) * 2 * (lo ? 2 : 1)) + 15) / 16 * 16;
 }
-__host__ __device__ inline size_t gemv_w_bytes(int K) { return (size_t)(K >> 6) * 512; }
+// INT4: 16 bytes per lane per 64-k chunk; INT2: 8
+__host__ __device__ inline size_t gemv_w_bytes(int K, int bits = 4) { return (size_t)(K >> 6) * (bits == 2 ? 256 : 512); }
 __host__ __device__ inline size_t gemv_sz_bytes(int K) { return (size_t)(K >> 7) * 64; }
 __host__ __device__ inline size_t gemv_smem_bytes(int K, int M, bool lo, int tpc) {
   const int nc = M <= 8 ? 8 : 16;
@@ -121,7 +123,9 @@ __host__ __device__ inline int gemv_nt(int M, bool lo) {
   return M <= 8 ? 1 : 2;
 }
 
-template <int NT, int IN, int EPI>
+// BITS: 4 (INT4 weights) or 2 (INT2 body: half the weight bytes, the A
+// fragments of two k16 steps per 32-bit word, unpack_a_frag2).
+template <int NT, int IN, int EPI, int BITS = 4>
 __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs a) {
   constexpr bool LO = (IN != IN_F16);
   constexpr int TPC = gemv_tpc(EPI);
@@ -135,7 +139,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   const int M = a.M;
   const int ldxs = K + 8;
   const int n_chunks = K >> 6;
-  const size_t wt_bytes = gemv_w_bytes(K), sz_bytes = gemv_sz_bytes(K);
+  const size_t wt_bytes = gemv_w_bytes(K, BITS), sz_bytes = gemv_sz_bytes(K);
   unsigned char* sw = smem;                                       // [TPC][chunks][32][16 B]
   unsigned char* ssz = smem + TPC * wt_bytes;                     // [TPC][groups][8][8 B]
   __half* xs = reinterpret_cast<__half*>(ssz + TPC * sz_bytes);   // hi plane [M][ldxs]
@@ -302,7 +306,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
   // ---- main loop: 64-wide K chunks from shared memory, 4 k16 tiles each ----
   const int c_begin = (n_chunks * kq) / KS;
   const int nc = (n_chunks * (kq + 1)) / KS - c_begin;
-  const unsigned char* wbase = sw + tsel * wt_bytes + (size_t)lane * 16;
+  constexpr int LANE_B = BITS == 2 ? 8 : 16;    // weight bytes per lane per chunk
+  const unsigned char* wbase = sw + tsel * wt_bytes + (size_t)lane * LANE_B;
   const unsigned char* sbase = ssz + tsel * sz_bytes + (size_t)g * 8;
   // B-fragment source of this lane: activation row and plane
   int brow, bplane;
@@ -319,7 +324,14 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
 #pragma unroll 2
   for (int ci = 0; ci < nc; ++ci) {
     const int c = c_begin + ci;
-    const uint4 wv = *reinterpret_cast<const uint4*>(wbase + (size_t)c * 512);
+    uint32_t words[4];
+    if (BITS == 2) {
+      const uint2 w2 = *reinterpret_cast<const uint2*>(wbase + (size_t)c * 32 * LANE_B);
+      words[0] = w2.x; words[1] = w2.y; words[2] = 0u; words[3] = 0u;
+    } else {
+      const uint4 wv = *reinterpret_cast<const uint4*>(wbase + (size_t)c * 32 * LANE_B);
+      words[0] = wv.x; words[1] = wv.y; words[2] = wv.z; words[3] = wv.w;
+    }
     const uint2 sv = *reinterpret_cast<const uint2*>(sbase + (size_t)(c >> 1) * 64);
     const int kc = c * 64;
     float tmp[NTILES][4];
@@ -327,11 +339,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
     for (int nt = 0; nt < NTILES; ++nt)
 #pragma unroll
       for (int q = 0; q < 4; ++q) tmp[nt][q] = 0.f;
-    const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       uint32_t af[4];
-      unpack_a_frag(words[j], sv.y, af);
+      if (BITS == 2) unpack_a_frag2(words[j >> 1], j & 1, sv.y, af);
+      else unpack_a_frag(words[j], sv.y, af);
       const int ko = kc + j * 16;
       if (NT == 0) {
         uint32_t b0 = 0, b1 = 0;
@@ -476,13 +488,57 @@ __global__ void repack_int4_weights_kernel(const uint32_t* __restrict__ qweight,
   out[idx] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
 }
 
-// sz[T][group][g] = {(s[r0], s[r1]) fp16 pair, (1024 + z[r0], 1024 + z[r1]) fp16 pair}
+// INT2 body: for (tile T, chunk c, lane l) two words; word j2 holds k16
+// steps 2 j2 and 2 j2 + 1, step s's slots in the order above at fields
+// 4s + r (first element of the pair) and 8 + 4s + r (second), field f at bits
+// 2f, so that unpack_a_frag2 yields the A fragment.  Storage: element k of
+// row n in bits 2 (k % 16) of word k / 16.
+__global__ void repack_int2_weights_kernel(const uint32_t* __restrict__ qweight, int K, int N,
+                                           int n_tiles, uint2* __restrict__ out) {
+  const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int n_chunks = K >> 6;
+  const size_t total = (size_t)n_tiles * n_chunks * 32;
+  if (idx >= total) return;
+  const int l = (int)(idx & 31);
+  const size_t rest = idx >> 5;
+  const int c = (int)(rest % n_chunks);
+  const int T = (int)(rest / n_chunks);
+  const int g = l >> 2, t = l & 3;
+  const int r0 = T * 16 + g, r1 = r0 + 8;
+  const int kw = K >> 4;
+  auto q = [&](int r, int k) -> uint32_t {
+    if (r >= N) return 0u;
+    return (qweight[(size_t)r * kw + (k >> 4)] >> (2 * (k & 15))) & 0x3u;
+  };
+  uint32_t wd[2];
+#pragma unroll
+  for (int j2 = 0; j2 < 2; ++j2) {
+    uint32_t w = 0;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int kb = c * 64 + (2 * j2 + s) * 16 + 2 * t;
+      const uint32_t v[8] = {q(r0, kb), q(r1, kb), q(r0, kb + 8), q(r1, kb + 8),
+                             q(r0, kb + 1), q(r1, kb + 1), q(r0, kb + 9), q(r1, kb + 9)};
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        w |= v[r] << (2 * (4 * s + r));
+        w |= v[4 + r] << (2 * (8 + 4 * s + r));
+      }
+    }
+    wd[j2] = w;
+  }
+  out[idx] = make_uint2(wd[0], wd[1]);
+}
+
+// sz[T][group][g] = {(s[r0], s[r1]) fp16 pair, (1024 + z[r0], 1024 + z[r1]) fp16 pair};
+// the zero points are 4-bit (bits = 4) or 2-bit (bits = 2) fields
 __global__ void repack_int4_scales_kernel(const uint16_t* __restrict__ scales,
                                           const uint32_t* __restrict__ qzeros, int K, int N,
-                                          int n_tiles, uint2* __restrict__ out) {
+                                          int n_tiles, uint2* __restrict__ out, int bits) {
   const size_t idx = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int G = K >> 7;
-  const int zw = (G + 7) >> 3;
+  const int epw = 32 / bits;   // zero points per word
+  const int zw = (G + epw - 1) / epw;
   const size_t total = (size_t)n_tiles * G * 8;
   if (idx >= total) return;
   const int g = (int)(idx & 7);
@@ -492,7 +548,7 @@ __global__ void repack_int4_scales_kernel(const uint16_t* __restrict__ scales,
   const int r0 = T * 16 + g, r1 = r0 + 8;
   auto sc = [&](int r) -> uint32_t { return r < N ? (uint32_t)scales[(size_t)r * G + gr] : 0u; };
   auto zb = [&](int r) -> uint32_t {
-    const uint32_t z = r < N ? (qzeros[(size_t)r * zw + (gr >> 3)] >> (4 * (gr & 7))) & 0xFu : 0u;
+    const uint32_t z = r < N ? (qzeros[(size_t)r * zw + gr / epw] >> (bits * (gr % epw))) & ((1u << bits) - 1u) : 0u;
     return 0x6400u + z;  // fp16 bits of 1024 + z
   };
   out[idx] = make_uint2(sc(r0) | (sc(r1) << 16), zb(r0) | (zb(r1) << 16));

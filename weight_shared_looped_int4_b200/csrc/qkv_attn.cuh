@@ -82,9 +82,10 @@ __host__ __device__ inline int qa_units_per_cta(int rep, int hd) {
 struct QaLayout {
   size_t w, kvc, pml, pv, act, red, q, kv, kvs, total;
 };
-__host__ __device__ inline QaLayout qa_layout(int K, int M, int rep, int hd) {
+// bits: 4 (INT4 weights) or 2 (the INT2 body's half-size tiles)
+__host__ __device__ inline QaLayout qa_layout(int K, int M, int rep, int hd, int bits = 4) {
   QaLayout L;
-  const size_t tile = (size_t)(K / 64) * 512 + (size_t)(K / 128) * 64;
+  const size_t tile = (size_t)(K / 64) * (bits == 2 ? 256 : 512) + (size_t)(K / 128) * 64;
   const size_t wbytes = (size_t)2 * qa_units_per_cta(rep, hd) * tile;
   const size_t chunk = (size_t)2 * kQaChunk * hd * 2;   // keys then values, fp16
   L.w = 0;
@@ -125,7 +126,8 @@ __device__ __forceinline__ void qa_st_peer2(unsigned addr, float x, float y) {
 // KV8: INT8 KV cache (kv8.cuh): the new key / value are quantised by every
 // rank alike after the first exchange (rank 0 stores them) and the cached
 // keys / values are read as codes times their vector's scale.
-template <int HD, bool KV8>
+// BITS: 4 (INT4 weights) or 2 (INT2 body, unpack_a_frag2).
+template <int HD, bool KV8, int BITS = 4>
 __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnArgs a) {
   constexpr int DPL = HD / 32;
   constexpr int ROW16 = HD / 8;
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   __shared__ int s_ok;
   __shared__ float s_ss[kQaMaxRows][kQaWarps];
   const int K = a.K, M = a.M, rep = a.rep;
-  const QaLayout L = qa_layout(K, M, rep, HD);
+  const QaLayout L = qa_layout(K, M, rep, HD, BITS);
   unsigned char* wsm = qsm + L.w;
   __half* kvc = reinterpret_cast<__half*>(qsm + L.kvc);     // [m][keys, values][kQaChunk][hd]
   float2* pml = reinterpret_cast<float2*>(qsm + L.pml);     // [rank][m][h]: (max, sum of weights)
@@ -154,7 +156,8 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   const int c = (int)crank, grp = blockIdx.y;
   const int U = qa_units(rep, HD), hp = HD / 32;
   const int qdim = a.Hkv * rep * HD, kvdim = a.Hkv * HD;
-  const size_t wt_bytes = (size_t)(K / 64) * 512, sz_bytes = (size_t)(K / 128) * 64;
+  constexpr int LANE_B = BITS == 2 ? 8 : 16;   // weight bytes per lane per 64-k chunk
+  const size_t wt_bytes = (size_t)(K / 64) * 32 * LANE_B, sz_bytes = (size_t)(K / 128) * 64;
   // this CTA's units: c, c + kQaCluster, ... (nu of them)
   const int nu = c < U ? min(kQaMaxUnits, (U - 1 - c) / kQaCluster + 1) : 0;
   // group-local unit -> global 16-row tile of the QKV output: group heads are
@@ -339,15 +342,22 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
 #pragma unroll
       for (int i = 0; i < 2 * kQaMaxUnits; ++i) {
         if (i < 2 * nu) {
-          const uint4 wv = *reinterpret_cast<const uint4*>(wsm + i * wt_bytes + (size_t)ci * 512 + lane * 16);
+          uint32_t words[4];
+          if (BITS == 2) {
+            const uint2 w2 = *reinterpret_cast<const uint2*>(wsm + i * wt_bytes + (size_t)ci * 32 * LANE_B + lane * LANE_B);
+            words[0] = w2.x; words[1] = w2.y; words[2] = 0u; words[3] = 0u;
+          } else {
+            const uint4 wv = *reinterpret_cast<const uint4*>(wsm + i * wt_bytes + (size_t)ci * 32 * LANE_B + lane * LANE_B);
+            words[0] = wv.x; words[1] = wv.y; words[2] = wv.z; words[3] = wv.w;
+          }
           const uint2 sv =
               *reinterpret_cast<const uint2*>(wsm + 2 * nu * wt_bytes + i * sz_bytes + (size_t)(ci >> 1) * 64 + g8 * 8);
-          const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
           float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint32_t af[4];
-            unpack_a_frag(words[j], sv.y, af);
+            if (BITS == 2) unpack_a_frag2(words[j >> 1], j & 1, sv.y, af);
+            else unpack_a_frag(words[j], sv.y, af);
             if (j & 1) mma_f16_16816(t1, af, bf[j][0], bf[j][1]);
             else mma_f16_16816(t0, af, bf[j][0], bf[j][1]);
           }

@@ -191,7 +191,8 @@ cudaError_t allow_max_smem(K* kern, int dev) {
 
 template <int NT, int IN, int EPI>
 cudaError_t set_gemv_attr(int dev) {
-  return allow_max_smem(gemv_int4_kernel<NT, IN, EPI>, dev);
+  const cudaError_t e = allow_max_smem(gemv_int4_kernel<NT, IN, EPI, 4>, dev);
+  return e == cudaSuccess ? allow_max_smem(gemv_int4_kernel<NT, IN, EPI, 2>, dev) : e;
 }
 
 cudaError_t init_device_kernels(int dev) {
@@ -208,12 +209,24 @@ cudaError_t init_device_kernels(int dev) {
   if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<128, false>, dev);
   if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<64, true>, dev);
   if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<128, true>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<64, false, 2>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<128, false, 2>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<64, true, 2>, dev);
+  if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<128, true, 2>, dev);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qkv_attn_kernel<64, false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qkv_attn_kernel<64, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qkv_attn_kernel<128, true>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qkv_attn_kernel<64, false, 2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qkv_attn_kernel<128, false, 2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qkv_attn_kernel<64, true, 2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(qkv_attn_kernel<128, true, 2>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(qkv_attn_kernel<128, false>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess) e = allow_max_smem(decode_fused_kernel<64>, dev);
@@ -268,8 +281,10 @@ cudaError_t launch_gemv(const GemvArgs& a, int grid, int in_mode, int epi, cudaS
   const int nt = gemv_nt(a.M, lo);
   const size_t smem = gemv_smem_bytes(a.K, a.M, lo, gemv_tpc(epi));
   const dim3 g(grid), b(kGemvThreads);
-#define CASE(NT, IN, EPI) \
-  if (nt == NT && in_mode == IN && epi == EPI) return launch(gemv_int4_kernel<NT, IN, EPI>, g, b, smem, st, a);
+#define CASE(NT, IN, EPI)                                                                             \
+  if (nt == NT && in_mode == IN && epi == EPI)                                                        \
+    return a.bits == 2 ? launch(gemv_int4_kernel<NT, IN, EPI, 2>, g, b, smem, st, a)                  \
+                       : launch(gemv_int4_kernel<NT, IN, EPI, 4>, g, b, smem, st, a);
 #define CASE3(IN, EPI) CASE(0, IN, EPI) CASE(1, IN, EPI) CASE(2, IN, EPI)
   CASE3(IN_F16, EPI_STORE) CASE3(IN_F32, EPI_RESID) CASE3(IN_NORM, EPI_SWIGLU) CASE3(IN_NORM, EPI_ROPE_KV)
 #undef CASE3
@@ -304,14 +319,17 @@ cudaError_t launch_gemv_rows(GemvArgs a, int total, int in_mode, int epi, int gr
 // ============================================================================
 struct Int4Dev {
   int K = 0, N = 0, n_tiles = 0;
+  int bits = 4;            // 4, or 2 for the INT2 body (w then holds uint2 per lane and chunk)
   uint4* w = nullptr;
   uint2* sz = nullptr;
   uint8_t* tc = nullptr;   // tensor-core layout (prefill), always owned
   bool owned = true;   // false when w / sz live in a block's arena
   static size_t tc_bytes(int K, int N) { return (size_t)((N + kTcRows - 1) / kTcRows) * (K / 128) * kTcRawBytes; }
-  static size_t w_bytes(int K, int N) { return (size_t)(((N + 31) / 32) * 2) * (K / 64) * 32 * sizeof(uint4); }
+  static size_t w_bytes(int K, int N, int bits = 4) {
+    return (size_t)(((N + 31) / 32) * 2) * (K / 64) * 32 * (bits == 2 ? sizeof(uint2) : sizeof(uint4));
+  }
   static size_t sz_bytes(int K, int N) { return (size_t)(((N + 31) / 32) * 2) * (K / 128) * 8 * sizeof(uint2); }
-  size_t bytes() const { return w_bytes(K, N) + sz_bytes(K, N) + (tc ? tc_bytes(K, N) : 0); }
+  size_t bytes() const { return w_bytes(K, N, bits) + sz_bytes(K, N) + (tc ? tc_bytes(K, N) : 0); }
   void free_all() {
     if (owned) {
       if (w) cudaFree(w);
@@ -341,13 +359,15 @@ struct Arena {
 // perm_F != 0: the tensor-core copy interleaves gate rows [0, F) and up rows
 // [F, 2F) per 128-row tile (for the fused SwiGLU epilogue).
 tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaStream_t st, Arena* arena = nullptr,
-                      int perm_F = 0) {
+                      int perm_F = 0, int bits = 4) {
   if (!h.qweight || !h.scales || !h.qzeros) return fail(TL_ERR_INVALID_ARG, "null INT4 array");
-  const int G = K / 128, zw = (G + 7) / 8;
+  const int epw = 32 / bits;   // fields per storage word
+  const int G = K / 128, zw = (G + epw - 1) / epw;
   out->K = K;
   out->N = N;
+  out->bits = bits;
   out->n_tiles = ((N + 31) / 32) * 2;
-  const size_t qb = (size_t)N * (K / 8) * 4, sb = (size_t)N * G * 2, zb = (size_t)N * zw * 4;
+  const size_t qb = (size_t)N * (K / epw) * 4, sb = (size_t)N * G * 2, zb = (size_t)N * zw * 4;
   void *dq = nullptr, *ds = nullptr, *dz = nullptr;
   tl_status rc = TL_OK;
   cudaError_t e = cudaMalloc(&dq, qb);
@@ -355,11 +375,11 @@ tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaS
   if (e == cudaSuccess) e = cudaMalloc(&dz, zb);
   if (arena) {
     out->owned = false;
-    out->w = (uint4*)arena->take(Int4Dev::w_bytes(K, N));
+    out->w = (uint4*)arena->take(Int4Dev::w_bytes(K, N, bits));
     out->sz = (uint2*)arena->take(Int4Dev::sz_bytes(K, N));
     if (e == cudaSuccess && (!out->w || !out->sz)) e = cudaErrorMemoryAllocation;
   } else {
-    if (e == cudaSuccess) e = cudaMalloc(&out->w, Int4Dev::w_bytes(K, N));
+    if (e == cudaSuccess) e = cudaMalloc(&out->w, Int4Dev::w_bytes(K, N, bits));
     if (e == cudaSuccess) e = cudaMalloc(&out->sz, Int4Dev::sz_bytes(K, N));
   }
   if (e == cudaSuccess) e = cudaMalloc(&out->tc, Int4Dev::tc_bytes(K, N));
@@ -368,14 +388,18 @@ tl_status upload_int4(const tl_int4_linear& h, int K, int N, Int4Dev* out, cudaS
   if (e == cudaSuccess) e = cudaMemcpyAsync(dz, h.qzeros, zb, cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) {
     const size_t tw = (size_t)out->n_tiles * (K / 64) * 32;
-    repack_int4_weights_kernel<<<(unsigned)((tw + 255) / 256), 256, 0, st>>>(
-        (const uint32_t*)dq, K, N, out->n_tiles, out->w);
+    if (bits == 2)
+      repack_int2_weights_kernel<<<(unsigned)((tw + 255) / 256), 256, 0, st>>>(
+          (const uint32_t*)dq, K, N, out->n_tiles, reinterpret_cast<uint2*>(out->w));
+    else
+      repack_int4_weights_kernel<<<(unsigned)((tw + 255) / 256), 256, 0, st>>>(
+          (const uint32_t*)dq, K, N, out->n_tiles, out->w);
     const size_t ts = (size_t)out->n_tiles * G * 8;
     repack_int4_scales_kernel<<<(unsigned)((ts + 255) / 256), 256, 0, st>>>(
-        (const uint16_t*)ds, (const uint32_t*)dz, K, N, out->n_tiles, out->sz);
+        (const uint16_t*)ds, (const uint32_t*)dz, K, N, out->n_tiles, out->sz, bits);
     const size_t tt = (size_t)((N + kTcRows - 1) / kTcRows) * G * kTcRows * 16;
     repack_int4_tc_kernel<<<(unsigned)((tt + 255) / 256), 256, 0, st>>>((const uint32_t*)dq, (const uint32_t*)dz, K,
-                                                                       N, perm_F, out->tc);
+                                                                       N, perm_F, out->tc, bits);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
@@ -641,6 +665,17 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, int B, int hd, int rep, bool 
 
 bool rep_ok(int rep) { return rep == 1 || rep == 2 || rep == 4 || rep == 8; }
 
+// The clustered QKV + attention kernel for a head size, KV cache mode and
+// weight width.
+using QaKernel = void (*)(QkvAttnArgs);
+QaKernel qa_kernel(int hd, bool kv8, int bits) {
+  if (bits == 2)
+    return hd == 64 ? (kv8 ? qkv_attn_kernel<64, true, 2> : qkv_attn_kernel<64, false, 2>)
+                    : (kv8 ? qkv_attn_kernel<128, true, 2> : qkv_attn_kernel<128, false, 2>);
+  return hd == 64 ? (kv8 ? qkv_attn_kernel<64, true, 4> : qkv_attn_kernel<64, false, 4>)
+                  : (kv8 ? qkv_attn_kernel<128, true, 4> : qkv_attn_kernel<128, false, 4>);
+}
+
 }  // namespace
 
 // ============================================================================
@@ -805,6 +840,8 @@ tl_status validate_config(const tl_config* c) {
   if (c->max_lanes < 1 || c->max_lanes > kMaxLanes) return fail(TL_ERR_INVALID_ARG, "max_lanes must be in [1, 16]");
   if (!(c->rms_eps >= 0.f) || !(c->rope_theta > 0.f)) return fail(TL_ERR_INVALID_ARG, "bad eps or theta");
   if (c->kv_mode != TL_KV_FP16 && c->kv_mode != TL_KV_INT8) return fail(TL_ERR_INVALID_ARG, "kv_mode must be TL_KV_FP16 or TL_KV_INT8");
+  if (c->weight_bits != 0 && c->weight_bits != 4 && c->weight_bits != 2)
+    return fail(TL_ERR_INVALID_ARG, "weight_bits must be 4 (or 0) or 2");
   return TL_OK;
 }
 
@@ -817,13 +854,14 @@ tl_status upload_block(const tl_config& c, const tl_block& hb, BlockDev* b, cuda
   const int qdim = c.n_q_heads * hd;
   size_t total = 0;
   const int shapes[4][2] = {{d, qkv_rows}, {qdim, d}, {d, 2 * c.ffn_dim}, {c.ffn_dim, d}};
-  for (auto& sh : shapes) total += Int4Dev::w_bytes(sh[0], sh[1]) + Int4Dev::sz_bytes(sh[0], sh[1]) + 512;
+  const int bits = c.weight_bits == 2 ? 2 : 4;
+  for (auto& sh : shapes) total += Int4Dev::w_bytes(sh[0], sh[1], bits) + Int4Dev::sz_bytes(sh[0], sh[1]) + 512;
   if (cudaMalloc(&b->arena.base, total) != cudaSuccess) return fail(TL_ERR_OOM, "block weights (%zu bytes)", total);
   b->arena.size = total;
-  if ((rc = upload_int4(hb.qkv, d, qkv_rows, &b->qkv, st, &b->arena)) != TL_OK) return rc;
-  if ((rc = upload_int4(hb.o, qdim, d, &b->o, st, &b->arena)) != TL_OK) return rc;
-  if ((rc = upload_int4(hb.gate_up, d, 2 * c.ffn_dim, &b->gate_up, st, &b->arena, c.ffn_dim)) != TL_OK) return rc;
-  if ((rc = upload_int4(hb.down, c.ffn_dim, d, &b->down, st, &b->arena)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.qkv, d, qkv_rows, &b->qkv, st, &b->arena, 0, bits)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.o, qdim, d, &b->o, st, &b->arena, 0, bits)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.gate_up, d, 2 * c.ffn_dim, &b->gate_up, st, &b->arena, c.ffn_dim, bits)) != TL_OK) return rc;
+  if ((rc = upload_int4(hb.down, c.ffn_dim, d, &b->down, st, &b->arena, 0, bits)) != TL_OK) return rc;
   return TL_OK;
 }
 
@@ -857,7 +895,7 @@ tl_status run_qkv(tl_model* m, int layer, int M, float* x, const RowCtx* rows, f
   a.theta = c.rope_theta;
   a.rows = rows;
   a.hd = hd;
-  a.w = b.qkv.w; a.sz = b.qkv.sz; a.K = c.d_model; a.n_rows = b.qkv.N;
+  a.w = b.qkv.w; a.sz = b.qkv.sz; a.K = c.d_model; a.n_rows = b.qkv.N; a.bits = b.qkv.bits;
   a.x = x; a.ldx = c.d_model; a.gain = b.attn_norm;
   a.pair_mode = PAIR_ROPE; a.pair_off = hd / 32;
   a.q_out = q; a.ldq = qdim; a.n_q_rows = qdim; a.n_kv_rows = c.n_kv_heads * hd;
@@ -928,8 +966,7 @@ tl_status run_qkv_attn(tl_model* m, int layer, int M, const RowCtx* rows, cudaSt
       a.k_scale = m->ks_plane(layer);
       a.v_scale = m->vs_plane(layer);
     }
-    auto kern = c.head_dim == 64 ? (m->kv_int8 ? qkv_attn_kernel<64, true> : qkv_attn_kernel<64, false>)
-                                 : (m->kv_int8 ? qkv_attn_kernel<128, true> : qkv_attn_kernel<128, false>);
+    auto kern = qa_kernel(c.head_dim, m->kv_int8, b.qkv.bits);
     TL_CUDA(launch_impl(false, dim3(kQaCluster, 1, 1), kern, grid, dim3(kQaThreads), smem, st, a));
   }
   return TL_OK;
@@ -943,7 +980,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   const int d = c.d_model, F = c.ffn_dim, qdim = c.n_q_heads * c.head_dim;
   GemvArgs a{};
   a.eps = c.rms_eps;
-  a.w = b.o.w; a.sz = b.o.sz; a.K = qdim; a.n_rows = d;
+  a.w = b.o.w; a.sz = b.o.sz; a.K = qdim; a.n_rows = d; a.bits = b.o.bits;
   a.x = o; a.ldx = qdim;
   a.pair_mode = PAIR_NEIGHBOUR;
   a.resid = x; a.ldr = d;
@@ -955,7 +992,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, (b.o.N + 15) / 16, st));
   GemvArgs g{};
   g.eps = c.rms_eps;
-  g.w = b.gate_up.w; g.sz = b.gate_up.sz; g.K = d; g.n_rows = 2 * F;
+  g.w = b.gate_up.w; g.sz = b.gate_up.sz; g.K = d; g.n_rows = 2 * F; g.bits = b.gate_up.bits;
   g.x = x; g.ldx = d; g.gain = b.ffn_norm;
   g.pair_mode = PAIR_OFFSET; g.pair_off = F / 16;
   g.yf = h; g.ldy = F;
@@ -966,7 +1003,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   kclass(TL_KERNEL_GATE_UP);
   TL_CUDA(launch_gemv_rows(g, M, IN_NORM, EPI_SWIGLU, F / 16, st));
   GemvArgs dn{};
-  dn.w = b.down.w; dn.sz = b.down.sz; dn.K = F; dn.n_rows = d;
+  dn.w = b.down.w; dn.sz = b.down.sz; dn.K = F; dn.n_rows = d; dn.bits = b.down.bits;
   dn.x = h; dn.ldx = F;
   dn.pair_mode = PAIR_NEIGHBOUR;
   dn.resid = x; dn.ldr = d;
@@ -1342,8 +1379,9 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
                   "fused partials ([4 rows][..][hd + 4]) must fit the layered path's buffer");
     int coop = 0;
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, device);
-    // (the single-kernel step keeps an fp16 cache only)
-    if (coop && !m->kv_int8 && (hd == 64 || hd == 128) && c.n_pre < kFusedMaxBlocks && rep_ok(rep)) {
+    // (the single-kernel step keeps an fp16 cache and INT4 weights only)
+    if (coop && !m->kv_int8 && c.weight_bits != 2 && (hd == 64 || hd == 128) && c.n_pre < kFusedMaxBlocks &&
+        rep_ok(rep)) {
       FusedArgs& f = m->fused;
       for (int i = 0; i <= c.n_pre; ++i) {
         const BlockDev& b = i < c.n_pre ? m->pre[i] : m->loop;
@@ -1387,8 +1425,7 @@ tl_status tl_model_create(const tl_config* cfg, const tl_weights* w, int device,
   {
     cudaFuncAttributes fa{};
     int optin = 0;
-    auto qa_kern = hd == 64 ? (m->kv_int8 ? qkv_attn_kernel<64, true> : qkv_attn_kernel<64, false>)
-                            : (m->kv_int8 ? qkv_attn_kernel<128, true> : qkv_attn_kernel<128, false>);
+    auto qa_kern = qa_kernel(hd, m->kv_int8, m->loop.qkv.bits);
     if (cudaFuncGetAttributes(&fa, qa_kern) == cudaSuccess &&
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) == cudaSuccess)
       m->qa_smem_max = optin - (int)fa.sharedSizeBytes;
@@ -2016,7 +2053,7 @@ tl_status op_workspace(int dev, size_t bytes, void** out, unsigned** tickets) {
 
 extern "C" {
 
-tl_status tl_linear_create(const tl_int4_linear* w, int K, int N, int device, tl_linear** out) {
+static tl_status linear_create(const tl_int4_linear* w, int K, int N, int bits, int device, tl_linear** out) {
   if (!out || !w) return fail(TL_ERR_INVALID_ARG, "null argument");
   *out = nullptr;
   if (K < 128 || K % 128 || K > 12288) return fail(TL_ERR_UNSUPPORTED, "K must be a multiple of 128 in [128, 12288]");
@@ -2030,7 +2067,7 @@ tl_status tl_linear_create(const tl_int4_linear* w, int K, int N, int device, tl
   l->device = device;
   cudaStream_t st;
   TL_CUDA(cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking));
-  tl_status rc = upload_int4(*w, K, N, &l->w, st);
+  tl_status rc = upload_int4(*w, K, N, &l->w, st, nullptr, 0, bits);
   cudaStreamDestroy(st);
   if (rc != TL_OK) {
     delete l;
@@ -2038,6 +2075,14 @@ tl_status tl_linear_create(const tl_int4_linear* w, int K, int N, int device, tl
   }
   *out = l;
   return TL_OK;
+}
+
+tl_status tl_linear_create(const tl_int4_linear* w, int K, int N, int device, tl_linear** out) {
+  return linear_create(w, K, N, 4, device, out);
+}
+
+tl_status tl_linear_create_int2(const tl_int4_linear* w, int K, int N, int device, tl_linear** out) {
+  return linear_create(w, K, N, 2, device, out);
 }
 
 void tl_linear_destroy(tl_linear* l) {
@@ -2087,7 +2132,7 @@ tl_status tl_linear_forward(tl_linear* l, const uint16_t* d_x, int M, uint16_t* 
   GemvArgs a{};
   a.err_flag = op_err_flag(l->device);
   if (!a.err_flag) return fail(TL_ERR_OOM, "op error flag");
-  a.w = l->w.w; a.sz = l->w.sz; a.K = K; a.n_rows = N;
+  a.w = l->w.w; a.sz = l->w.sz; a.K = K; a.n_rows = N; a.bits = l->w.bits;
   a.xh = reinterpret_cast<const __half*>(d_x); a.ldx = K;
   a.pair_mode = PAIR_NEIGHBOUR;
   a.y = reinterpret_cast<__half*>(d_y); a.ldy = N;
