@@ -905,10 +905,11 @@ def run_workload_attention(args):
     return 0
 
 
-def _lm_model(tl, tl_synth, max_loops, max_ctx, max_lanes, kv_mode=0):
+def _lm_model(tl, tl_synth, max_loops, max_ctx, max_lanes, kv_mode=0, bits=4):
     shape = tl_synth.LOOPED_LM
-    w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM)
-    cfg = tl.make_config(shape, max_loops=max_loops, max_ctx=max_ctx, max_lanes=max_lanes, kv_mode=kv_mode)
+    w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM, bits=bits)
+    cfg = tl.make_config(shape, max_loops=max_loops, max_ctx=max_ctx, max_lanes=max_lanes, kv_mode=kv_mode,
+                         weight_bits=bits)
     tw, keep = tl.make_weights(w)
     m = tl.tl_model_create(cfg, tw, 0)
     del keep
@@ -1189,7 +1190,75 @@ def run_workload_kv8(args):
     return 0
 
 
+def run_workload_int2(args):
+    """INT4 against the INT2 body on the 400M LM at the headline shape: a
+    128-token no-logits prefill and 128 greedy decode steps at L = 8, batch 1
+    (graph replay).  Per width: decode tokens/s, its per-token byte roofline
+    (the INT2 linears read K N / 4 code bytes + a scale and a 2-bit zero per
+    group and row), prefill ms and the device bytes of the weights."""
+    torch, dev, st = _dev_setup()
+    import tl_synth
+    import weight_shared_looped_int4_b200 as tl
+    peaks = load_peaks()
+    n_dec = args.decode_steps
+    l2_gbs = None
+    res = []
+    launches0 = tl.tl_kernel_launch_count()
+
+    def lin_bytes(K, N, bits):
+        return K * N * bits // 8 + (K // 128) * N * (16 + bits) // 8
+
+    with ClockSampler(0) as clocks:
+        for bits in (4, 2):
+            w, m = _lm_model(tl, tl_synth, LOOPS, PROMPT + n_dec + 1, 1, bits=bits)
+            if l2_gbs is None:
+                l2_gbs, _, _ = probe_read_bandwidths(tl, torch, dev, st)
+            prompt = tl_synth.make_tokens(tl_synth.SEED_LM, w.shape.vocab, PROMPT + 1)
+            d_prompt = torch.as_tensor(prompt, device=dev)
+            hist = torch.zeros(n_dec + 1, dtype=torch.int32, device=dev)
+            hp = hist.data_ptr()
+            fn = lambda: tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS, None, None, st)
+            for _ in range(3):
+                fn()
+            pf = _time_reps(torch, st, fn, 10)
+
+            def decode_run():
+                tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS, None, None, st)
+                with torch.cuda.stream(st):
+                    hist[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(st)
+                for i in range(n_dec):
+                    tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1), st)
+                b.record(st)
+                b.synchronize()
+                return a.elapsed_time(b)
+
+            decode_run()     # warm (graph capture)
+            ms = decode_run()
+            layer = (lin_bytes(D, (HQ + 2 * HKV) * HD, bits) + lin_bytes(HQ * HD, D, bits) +
+                     lin_bytes(D, 2 * F, bits) + lin_bytes(F, D, bits))
+            kv = (2 + LOOPS) * 2 * HKV * HD * 2 * (PROMPT + n_dec / 2)
+            hbm = 2 * layer + BYTES_PER_LAUNCH["head"] + kv
+            l2 = LOOPS * layer
+            t_roof = hbm / (peaks["hbm_gbs"] * 1e3) + l2 / (l2_gbs * 1e3)
+            us_tok = 1e3 * ms / n_dec
+            res.append({"weight_bits": bits, "weight_bytes": tl.tl_model_info(m)["weight_bytes"],
+                        "block_linear_bytes": int(layer), "decode_tok_s": round(n_dec / (ms / 1e3), 1),
+                        "decode_us_per_token": round(us_tok, 2), "roofline_us_per_token": round(t_roof, 2),
+                        "frac": round(t_roof / us_tok, 4), "prefill_T128_ms": round(pf, 4)})
+            tl.tl_check_device_error(m)
+            tl.tl_model_destroy(m)
+    print(json.dumps({"workload": "400M looped LM, INT4 vs INT2 body: 128-token prefill (no logits), "
+                                  "%d greedy decode steps at L = 8, batch 1" % n_dec,
+                      "metric": "decode tok/s and byte roofline fraction, prefill ms, weight bytes",
+                      "peaks": peaks, "l2_read_gbs": round(l2_gbs, 1), "results": res,
+                      "gpu_launches": tl.tl_kernel_launch_count() - launches0, "clocks": clocks.summary()}))
+    return 0
+
+
 WORKLOADS = {"tiny": run_workload_tiny, "linear": run_workload_linear, "kv8": run_workload_kv8,
+             "int2": run_workload_int2,
              "attention": run_workload_attention, "lsweep": run_workload_lsweep,
              "peaks": run_workload_peaks, "next": run_workload_next}
 
