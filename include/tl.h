@@ -479,8 +479,8 @@ tl_status tl_op_gqa_decode(const uint16_t *d_q, const uint16_t *d_k, const uint1
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress, with that device current) and caches it for the
  * life of the process (a cudaDeviceReset makes the cached address stale; do
- * not call this entry point on a device after resetting it); make that first
- * call before any stream capture.  All calls share the one array and it
+ * not call this entry point on a device after resetting it).  All calls
+ * share the one array and it
  * keeps the last call's contents (each call re-zeroes what must start at
  * zero), so calls whose work overlaps on the GPU (different streams without
  * ordering between them) race and corrupt each other's results: order them on
