@@ -257,15 +257,17 @@ def run_reference(args):
 def run_ncu_case(args):
     """A small eager run of the same model for kernel profilers (no timing
     output): `decode` = prefill of the prompt + --decode-steps greedy steps,
-    `prefill` = two prefills of the prompt."""
+    `prefill` = two prefills of the prompt (--ncu-prompt tokens, default the
+    bench's 128)."""
     import torch
     import tl_synth
     import weight_shared_looped_int4_b200 as tl
     shape = tl_synth.LOOPED_LM
     w = tl_synth.make_model_weights(shape, tl_synth.SEED_LM)
-    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, shape.vocab, PROMPT + 1)
+    P = args.ncu_prompt
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, shape.vocab, P + 1)
     steps = args.decode_steps
-    cfg = tl.make_config(shape, max_loops=LOOPS, max_ctx=PROMPT + max(steps, 1), max_lanes=1)
+    cfg = tl.make_config(shape, max_loops=LOOPS, max_ctx=P + max(steps, 1), max_lanes=1)
     tw, keep = tl.make_weights(w)
     m = tl.tl_model_create(cfg, tw, 0)
     del keep
@@ -275,9 +277,9 @@ def run_ncu_case(args):
     hist = torch.zeros(steps + 1, dtype=torch.int32, device="cuda:0")
     hp = hist.data_ptr()
     for _ in range(2 if args.ncu_case == "prefill" else 1):
-        tl.tl_prefill(m, 0, d_prompt, PROMPT, LOOPS)
+        tl.tl_prefill(m, 0, d_prompt, P, LOOPS)
     if args.ncu_case == "decode":
-        hist[0:1].copy_(d_prompt[PROMPT:PROMPT + 1])
+        hist[0:1].copy_(d_prompt[P:P + 1])
         for i in range(steps):
             tl.tl_decode_step(m, [0], hp + 4 * i, [LOOPS], None, hp + 4 * (i + 1))
     torch.cuda.synchronize()
@@ -1284,6 +1286,8 @@ def main():
     ap.add_argument("--workload", choices=["lm"] + sorted(WORKLOADS), default="lm",
                     help="lm (default): the 400M-LM L=8 step; others time the kernels on the "
                          "shapes of the other workloads and print their own JSON line")
+    ap.add_argument("--ncu-prompt", type=int, default=PROMPT,
+                    help="prompt length of --ncu-case (e.g. 2048 for the tcgen05 prefill attention)")
     ap.add_argument("--ncu-case", choices=["none", "decode", "prefill"], default="none",
                     help="run a small eager case for kernel profilers and exit")
     args = ap.parse_args()
