@@ -96,7 +96,9 @@ __global__ void __launch_bounds__(kAtThreads, 1) prefill_attn_tc_kernel(const Pr
   __shared__ float lfin[kAtQ];      // final row sums
   __shared__ float xmax[2][kAtQ], xsum[2][kAtQ];   // the two softmax halves of a row
 
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // grid (heads, query tiles, batch): the last (longest, causal) query tiles
+  // are scheduled first so that the short ones fill the tail of the grid
+  const int qt = gridDim.y - 1 - blockIdx.y, h = blockIdx.x, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kvh = h / a.rep;
   const int q0 = qt * kAtQ;

@@ -635,8 +635,8 @@ cudaError_t launch_prefill_attn(PrefillAttnArgs a, int B, int hd, int rep, bool 
   const bool kv8 = a.ks != nullptr;   // INT8 KV cache: the 16-query tile kernel, fp32 queries
   if (kv8 && !f32) return cudaErrorInvalidValue;
   if (!kv8 && a.T >= g_at_min_tokens.load(std::memory_order_relaxed)) {
-    // tensor cores (tcgen05): one CTA per (128-query tile, query head, batch entry)
-    const dim3 grid((a.T + kAtQ - 1) / kAtQ, a.Hkv * rep, B);
+    // tensor cores (tcgen05): one CTA per (query head, 128-query tile, batch entry)
+    const dim3 grid(a.Hkv * rep, (a.T + kAtQ - 1) / kAtQ, B);   // heads fastest, longest tiles first
     if (hd == 128)
       return f32 ? launch(prefill_attn_tc_kernel<128, true>, grid, dim3(kAtThreads), attn_tc_smem_bytes<128>(), st, a)
                  : launch(prefill_attn_tc_kernel<128, false>, grid, dim3(kAtThreads), attn_tc_smem_bytes<128>(), st, a);
