@@ -377,10 +377,10 @@ __global__ void __launch_bounds__(kHeadThreads, 1) head_argmax_kernel(const Head
 
 // ---- output norm + head + argmax for up to 4 rows, direct loads -----------
 // One CTA per SM, 16 warps.  Warp w of CTA c owns the 16-row head tiles
-// c * 16 + w, then every P * 16 after that, and streams each whole tile
+// w * P + c, then every P * 16 after that, and streams each whole tile
 // (64 KB at d = 2048, in A-fragment order: lane l's 16-byte word of k16
-// chunk j is exactly its m16n8k16 A operand) with plain 16-byte loads, eight
-// in flight per lane, marked L2 evict-first (the head is read once per token
+// chunk j is exactly its m16n8k16 A operand) with plain 16-byte loads in
+// batches of eight per lane, two batches in flight, marked L2 evict-first (the head is read once per token
 // and must not push the loop block out of L2).  The first loads go out
 // before the wait on the previous kernel.  The B operand is the normalised
 // activation as fp16 (hi, lo) pairs from shared memory (columns 2t / 2t + 1
@@ -427,8 +427,11 @@ __global__ void __launch_bounds__(kHdThreads, 1) head_direct_kernel(const HeadAr
   stamp(0);
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  // warp-major order: every CTA gets a tile for its warp w before any CTA's
+  // warp w + 1 does, so all SMs stream (+-1 tile) even when the tiles do not
+  // fill every warp
   const int stride = P * kHdWarps;
-  int tile = c * kHdWarps + warp;
+  int tile = warp * P + c;
   uint4 wv[kHdUnroll];
   if (tile < nt) {   // the weights do not depend on earlier kernels
     const uint4* wt = a.w + (size_t)tile * nk16 * 32 + lane;
@@ -476,37 +479,38 @@ __global__ void __launch_bounds__(kHdThreads, 1) head_direct_kernel(const HeadAr
   const __half* bsrc = ((g & 1) ? xl : xs) + (size_t)(g >> 1) * ldx + 2 * t;
   float best_v = -INFINITY;
   int best_i = 0x7fffffff;
-  bool have = tile < nt;   // wv holds the first words of `tile`
+  bool have = tile < nt;   // wv holds the first batch of `tile`
+  // batches of kHdUnroll k16 chunks in two register sets used in turn (no
+  // copies between them, which would wait for the loads): while one set
+  // multiplies, the other set's loads are in flight
+  const int nb = nk16 / kHdUnroll;   // d is a multiple of 128
   for (; tile < nt; tile += stride) {
     const uint4* wt = a.w + (size_t)tile * nk16 * 32 + lane;
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, acc2[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int j0 = 0; j0 < nk16; j0 += kHdUnroll) {
-      if (!have) {
+    auto load = [&](uint4 (&v)[kHdUnroll], int b) {
 #pragma unroll
-        for (int u = 0; u < kHdUnroll; ++u) wv[u] = ldg_evict_first(wt + (size_t)(j0 + u) * 32, pol);
-      }
-      have = false;
-      uint4 nv[kHdUnroll];
-      const bool more = j0 + kHdUnroll < nk16;
-      if (more) {   // next batch in flight while this one multiplies
-#pragma unroll
-        for (int u = 0; u < kHdUnroll; ++u) nv[u] = ldg_evict_first(wt + (size_t)(j0 + kHdUnroll + u) * 32, pol);
-      }
+      for (int u = 0; u < kHdUnroll; ++u) v[u] = ldg_evict_first(wt + (size_t)(b * kHdUnroll + u) * 32, pol);
+    };
+    auto mul = [&](const uint4 (&v)[kHdUnroll], int b) {
 #pragma unroll
       for (int u = 0; u < kHdUnroll; ++u) {
-        const uint32_t af[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(bsrc + (j0 + u) * 16);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(bsrc + (j0 + u) * 16 + 8);
+        const int j = b * kHdUnroll + u;
+        const uint32_t af[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(bsrc + j * 16);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(bsrc + j * 16 + 8);
         if (u & 1) mma_f16_16816(acc2, af, b0, b1);
         else mma_f16_16816(acc, af, b0, b1);
       }
-      if (more) {
-#pragma unroll
-        for (int u = 0; u < kHdUnroll; ++u) wv[u] = nv[u];
-        have = true;
-      }
-    }
+    };
+    if (!have) load(wv, 0);
     have = false;
+    uint4 nv[kHdUnroll];
+    for (int b = 0; b < nb; b += 2) {
+      if (b + 1 < nb) load(nv, b + 1);
+      mul(wv, b);
+      if (b + 2 < nb) load(wv, b + 2);
+      if (b + 1 < nb) mul(nv, b + 1);
+    }
     // lane (g, t): columns 2t (hi) and 2t + 1 (lo) of row t
     const float v0 = (acc[0] + acc2[0]) + (acc[1] + acc2[1]);
     const float v1 = (acc[2] + acc2[2]) + (acc[3] + acc2[3]);
