@@ -37,7 +37,10 @@
 
 namespace tl {
 
-enum GemvIn { IN_NORM = 0, IN_F16 = 1, IN_F32 = 2 };
+// IN_F32W: IN_F32 for long rows (the down projection's input), staged with
+// every load of a row in flight at once; its extra registers would keep the
+// dependent kernel's CTAs off the SMs if the O projection used it too.
+enum GemvIn { IN_NORM = 0, IN_F16 = 1, IN_F32 = 2, IN_F32W = 3 };
 enum GemvEpi { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_ROPE_KV = 3 };
 enum PairMode { PAIR_NEIGHBOUR = 0, PAIR_OFFSET = 1, PAIR_ROPE = 2 };
 // When the kernel lets the next kernel of the stream launch (programmatic
@@ -241,6 +244,34 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
         const float2 r01 = __half22float2(h01), r23 = __half22float2(h23);
         const __half2 l01 = __floats2half2_rn(v.x - r01.x, v.y - r01.y);
         const __half2 l23 = __floats2half2_rn(v.z - r23.x, v.w - r23.y);
+        uint2 ph, pl;
+        ph.x = *reinterpret_cast<const uint32_t*>(&h01); ph.y = *reinterpret_cast<const uint32_t*>(&h23);
+        pl.x = *reinterpret_cast<const uint32_t*>(&l01); pl.y = *reinterpret_cast<const uint32_t*>(&l23);
+        *reinterpret_cast<uint2*>(xs + m * ldxs + k) = ph;
+        *reinterpret_cast<uint2*>(xl + m * ldxs + k) = pl;
+      }
+    }
+  } else if (IN == IN_F32W && M <= 2 && K <= 8 * 4 * kGemvThreads) {
+    // fp32 rows of up to 8 float4 per thread (the down input of a decode
+    // step): every load of a row is issued before the first conversion, one
+    // round trip to L2 instead of two
+    constexpr int R = 8;
+    for (int m = 0; m < M; ++m) {
+      const float* src = a.x + (size_t)m * a.ldx;
+      float4 v[R];
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const int k = threadIdx.x * 4 + j * 4 * kGemvThreads;
+        v[j] = k < K ? *reinterpret_cast<const float4*>(src + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const int k = threadIdx.x * 4 + j * 4 * kGemvThreads;
+        if (k >= K) continue;
+        const __half2 h01 = __floats2half2_rn(v[j].x, v[j].y), h23 = __floats2half2_rn(v[j].z, v[j].w);
+        const float2 r01 = __half22float2(h01), r23 = __half22float2(h23);
+        const __half2 l01 = __floats2half2_rn(v[j].x - r01.x, v[j].y - r01.y);
+        const __half2 l23 = __floats2half2_rn(v[j].z - r23.x, v[j].w - r23.y);
         uint2 ph, pl;
         ph.x = *reinterpret_cast<const uint32_t*>(&h01); ph.y = *reinterpret_cast<const uint32_t*>(&h23);
         pl.x = *reinterpret_cast<const uint32_t*>(&l01); pl.y = *reinterpret_cast<const uint32_t*>(&l23);

@@ -213,41 +213,6 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       xv[m][i] = (m < M && k < K) ? *reinterpret_cast<const float4*>(a.x + (size_t)m * K + k)
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // (issued after the row loads above, so that they overlap)
-  // the first chunk of this rank's key split of every row, minus the new key
-  if (tid == 0) {
-    unsigned bytes = 0;
-    int lo[kQaMaxRows], cnt[kQaMaxRows];
-#pragma unroll
-    for (int m = 0; m < kQaMaxRows; ++m) {
-      cnt[m] = 0;
-      lo[m] = 0;
-      if (m < M) {
-        const int n = rcs[m].pos + 1, C = (n + kQaCluster - 1) / kQaCluster;
-        lo[m] = min(n, c * C);
-        const int hi = min(min(n, lo[m] + C), lo[m] + kQaChunk);
-        cnt[m] = max(0, min(hi, rcs[m].pos) - lo[m]);
-        bytes += 2u * (unsigned)cnt[m] * HD * (KV8 ? 1u : 2u);
-      }
-    }
-    mbar_arrive_expect_tx(&kvbar, bytes);
-#pragma unroll
-    for (int m = 0; m < kQaMaxRows; ++m) {
-      if (cnt[m] > 0) {
-        const size_t src = (size_t)rcs[m].lane * a.lane_stride + ((size_t)grp * a.ctx + lo[m]) * HD;
-        __half* dst = kvc + (size_t)m * 2 * kQaChunk * HD;
-        if (KV8) {   // codes only, staged in the V half (their scales follow with plain loads below)
-          int8_t* d8 = reinterpret_cast<int8_t*>(dst + kQaChunk * HD);
-          bulk_g2s(d8, reinterpret_cast<const int8_t*>(a.k_plane) + src, (unsigned)cnt[m] * HD, &kvbar);
-          bulk_g2s(d8 + kQaChunk * HD, reinterpret_cast<const int8_t*>(a.v_plane) + src, (unsigned)cnt[m] * HD,
-                   &kvbar);
-        } else {
-          bulk_g2s(dst, a.k_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
-          bulk_g2s(dst + kQaChunk * HD, a.v_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
-        }
-      }
-    }
-  }
   // INT8: the first chunk's scales (their offsets are not 16-byte aligned,
   // so plain loads) by warp 1, under the GEMV like the codes' bulk copies
   if (KV8 && warp == 1) {
@@ -316,6 +281,42 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     s_ok = mbar_wait(&wbar, 0) ? 1 : 0;
     if (!s_ok) atomicOr(a.err_flag, kErrTimeout);
     trace_mark(a.trace, 9);
+  }
+  // The first chunk of this rank's key split of every row, minus the new key,
+  // goes out once the weights have landed, under the GEMV (issued during the
+  // RMSNorm it delayed the norm's block barrier by more than it saved).
+  if (tid == 0) {
+    unsigned bytes = 0;
+    int lo[kQaMaxRows], cnt[kQaMaxRows];
+#pragma unroll
+    for (int m = 0; m < kQaMaxRows; ++m) {
+      cnt[m] = 0;
+      lo[m] = 0;
+      if (m < M) {
+        const int n = rcs[m].pos + 1, C = (n + kQaCluster - 1) / kQaCluster;
+        lo[m] = min(n, c * C);
+        const int hi = min(min(n, lo[m] + C), lo[m] + kQaChunk);
+        cnt[m] = max(0, min(hi, rcs[m].pos) - lo[m]);
+        bytes += 2u * (unsigned)cnt[m] * HD * (KV8 ? 1u : 2u);
+      }
+    }
+    mbar_arrive_expect_tx(&kvbar, bytes);
+#pragma unroll
+    for (int m = 0; m < kQaMaxRows; ++m) {
+      if (cnt[m] > 0) {
+        const size_t src = (size_t)rcs[m].lane * a.lane_stride + ((size_t)grp * a.ctx + lo[m]) * HD;
+        __half* dst = kvc + (size_t)m * 2 * kQaChunk * HD;
+        if (KV8) {   // codes only, staged in the V half (their scales follow with plain loads below)
+          int8_t* d8 = reinterpret_cast<int8_t*>(dst + kQaChunk * HD);
+          bulk_g2s(d8, reinterpret_cast<const int8_t*>(a.k_plane) + src, (unsigned)cnt[m] * HD, &kvbar);
+          bulk_g2s(d8 + kQaChunk * HD, reinterpret_cast<const int8_t*>(a.v_plane) + src, (unsigned)cnt[m] * HD,
+                   &kvbar);
+        } else {
+          bulk_g2s(dst, a.k_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
+          bulk_g2s(dst + kQaChunk * HD, a.v_plane + src, (unsigned)cnt[m] * HD * 2u, &kvbar);
+        }
+      }
+    }
   }
   __syncthreads();
   const bool ok = s_ok != 0;   // on a time-out the control flow stays the same (cluster barriers)

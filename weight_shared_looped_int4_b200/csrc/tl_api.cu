@@ -202,7 +202,7 @@ cudaError_t init_device_kernels(int dev) {
 #define SET(NT, IN, EPI) \
   if (e == cudaSuccess) e = set_gemv_attr<NT, IN, EPI>(dev);
 #define SET3(IN, EPI) SET(0, IN, EPI) SET(1, IN, EPI) SET(2, IN, EPI)
-  SET3(IN_F16, EPI_STORE) SET3(IN_F32, EPI_RESID) SET3(IN_NORM, EPI_SWIGLU) SET3(IN_NORM, EPI_ROPE_KV)
+  SET3(IN_F16, EPI_STORE) SET3(IN_F32, EPI_RESID) SET3(IN_F32W, EPI_RESID) SET3(IN_NORM, EPI_SWIGLU) SET3(IN_NORM, EPI_ROPE_KV)
 #undef SET3
 #undef SET
   if (e == cudaSuccess) e = allow_max_smem(qkv_attn_kernel<64, false>, dev);
@@ -286,7 +286,7 @@ cudaError_t launch_gemv(const GemvArgs& a, int grid, int in_mode, int epi, cudaS
     return a.bits == 2 ? launch(gemv_int4_kernel<NT, IN, EPI, 2>, g, b, smem, st, a)                  \
                        : launch(gemv_int4_kernel<NT, IN, EPI, 4>, g, b, smem, st, a);
 #define CASE3(IN, EPI) CASE(0, IN, EPI) CASE(1, IN, EPI) CASE(2, IN, EPI)
-  CASE3(IN_F16, EPI_STORE) CASE3(IN_F32, EPI_RESID) CASE3(IN_NORM, EPI_SWIGLU) CASE3(IN_NORM, EPI_ROPE_KV)
+  CASE3(IN_F16, EPI_STORE) CASE3(IN_F32, EPI_RESID) CASE3(IN_F32W, EPI_RESID) CASE3(IN_NORM, EPI_SWIGLU) CASE3(IN_NORM, EPI_ROPE_KV)
 #undef CASE3
 #undef CASE
   return cudaErrorInvalidValue;
@@ -1012,7 +1012,7 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   dn.trigger = TRIGGER_AT_START;
   dn.l2_keep = layer >= c.n_pre;
   kclass(TL_KERNEL_DOWN);
-  TL_CUDA(launch_gemv_rows(dn, M, IN_F32, EPI_RESID, (b.down.N + 15) / 16, st));
+  TL_CUDA(launch_gemv_rows(dn, M, IN_F32W, EPI_RESID, (b.down.N + 15) / 16, st));
   return TL_OK;
 }
 
