@@ -19,14 +19,18 @@
 // That removes a kernel boundary (and its global round trips) per layer.
 //
 // The lane's cached keys and values (positions before the new one) do not
-// depend on this step: once the row table is read, one thread bulk-copies the
-// first chunk of the rank's key split into shared memory, and the copy runs
-// under the RMSNorm, the GEMV and the first exchange.
+// depend on this step: once the weights have landed, one thread bulk-copies
+// the first chunk of the rank's key split into shared memory, and the copy
+// runs under the GEMV and the first exchange.
 //
-// CTA c of cluster g: GEMV of RoPE pair units u = c, c + kQaCluster, ...
-// (tiles j and j + hd/32 of one head), weights bulk-copied into shared memory
-// before the programmatic-launch wait; 8 warps split K, each warp's B
-// fragments are loaded once per chunk and reused for every tile.
+// CTA c of cluster g: GEMV of the group's 16-row tiles c, c + kQaCluster, ...
+// ((rep + 2) hd / 16 tiles, 3 per rank for 4 query heads of 128), weights
+// bulk-copied into shared memory before the programmatic-launch wait; 8 warps
+// split K, each warp's B fragments are loaded once per chunk and reused for
+// every tile.  The raw projections go to every rank; RoPE (whose pairs j,
+// j + hd/2 sit in different tiles, often on different ranks) is applied by
+// every rank to its own copy after the exchange, and each rank writes its
+// hd / kQaCluster elements of the new key and value to the cache.
 #pragma once
 
 #include "attention.cuh"
@@ -39,9 +43,9 @@ constexpr int kQaCluster = 16;         // non-portable cluster size (B200 GPCs h
 constexpr int kQaThreads = 256;
 constexpr int kQaWarps = kQaThreads / 32;
 constexpr int kQaMaxRows = 2;
-constexpr int kQaMaxUnits = 2;        // RoPE pair units per CTA
+constexpr int kQaMaxTiles = 4;        // 16-row QKV tiles per CTA
 constexpr int kQaChunk = 64;          // keys per staged chunk
-static_assert(kQaMaxUnits * 16 * kQaMaxRows <= kQaThreads, "one epilogue element per thread");
+static_assert(kQaMaxTiles * 16 * kQaMaxRows <= kQaThreads, "one epilogue element per thread");
 static_assert(kQaMaxRows * 8 * 8 <= kQaThreads, "one merged (row, head, dimension) per thread");
 
 struct QkvAttnArgs {
@@ -72,21 +76,21 @@ struct QkvAttnArgs {
                               // (10) GEMV reduced, (11) key prefetch arrived
 };
 
-__host__ __device__ inline int qa_units(int rep, int hd) { return (rep + 2) * hd / 32; }
-__host__ __device__ inline int qa_units_per_cta(int rep, int hd) {
-  return (qa_units(rep, hd) + kQaCluster - 1) / kQaCluster;
+__host__ __device__ inline int qa_tiles(int rep, int hd) { return (rep + 2) * hd / 16; }
+__host__ __device__ inline int qa_tiles_per_cta(int rep, int hd) {
+  return (qa_tiles(rep, hd) + kQaCluster - 1) / kQaCluster;
 }
 // Shared memory: weight tiles, one key/value chunk per row (the prefetched
 // first chunk, then later chunks), the partials this rank merges, activation
 // planes, reduction buffer, q and the new key/value of every row, scores.
 struct QaLayout {
-  size_t w, kvc, pml, pv, act, red, q, kv, kvs, total;
+  size_t w, kvc, pml, pv, act, red, q, kv, kvs, cs, total;
 };
 // bits: 4 (INT4 weights) or 2 (the INT2 body's half-size tiles)
 __host__ __device__ inline QaLayout qa_layout(int K, int M, int rep, int hd, int bits = 4) {
   QaLayout L;
   const size_t tile = (size_t)(K / 64) * (bits == 2 ? 256 : 512) + (size_t)(K / 128) * 64;
-  const size_t wbytes = (size_t)2 * qa_units_per_cta(rep, hd) * tile;
+  const size_t wbytes = (size_t)qa_tiles_per_cta(rep, hd) * tile;
   const size_t chunk = (size_t)2 * kQaChunk * hd * 2;   // keys then values, fp16
   L.w = 0;
   L.kvc = (wbytes + 127) / 128 * 128;
@@ -94,11 +98,13 @@ __host__ __device__ inline QaLayout qa_layout(int K, int M, int rep, int hd, int
   L.pv = L.pml + ((size_t)kQaCluster * M * rep * 8 + 127) / 128 * 128;
   L.act = L.pv + ((size_t)kQaCluster * M * rep * (hd / kQaCluster) * 4 + 127) / 128 * 128;
   L.red = L.act + ((size_t)M * (K + 8) * 2 * 2 + 127) / 128 * 128;
-  L.q = L.red + (size_t)kQaWarps * 2 * kQaMaxUnits * 64 * 4;
+  L.q = L.red + (size_t)kQaWarps * kQaMaxTiles * 64 * 4;
   L.kv = L.q + (size_t)M * rep * hd * 4;
   L.kvs = L.kv + (size_t)2 * M * hd * 4;             // INT8 cache: the chunk's scales [m][K|V][kQaChunk]
   L.total = L.kvs + (size_t)M * 2 * kQaChunk * 4 + 128;   // + scores and softmax state
   L.total += (size_t)(rep * kQaChunk + 4 * rep) * 4;
+  L.cs = (L.total + 15) / 16 * 16;                    // RoPE (cos, sin) [m][hd / 2]
+  L.total = L.cs + (size_t)M * (hd / 2) * 8;
   return L;
 }
 
@@ -150,22 +156,23 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   float* vnew = knew + (size_t)M * HD;                       // [m][hd]
   float* kvs = reinterpret_cast<float*>(qsm + L.kvs);      // INT8: [m][K|V][kQaChunk] scales
   float* sc = kvs + (size_t)M * 2 * kQaChunk;                // [rep][kQaChunk]
+  float2* cst = reinterpret_cast<float2*>(qsm + L.cs);       // RoPE (cos, sin) [m][hd / 2]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g8 = lane >> 2, t4 = lane & 3;
   const unsigned crank = qa_cluster_rank();
   const int c = (int)crank, grp = blockIdx.y;
-  const int U = qa_units(rep, HD), hp = HD / 32;
+  const int TG = qa_tiles(rep, HD), hpt = HD / 16;
   const int qdim = a.Hkv * rep * HD, kvdim = a.Hkv * HD;
   constexpr int LANE_B = BITS == 2 ? 8 : 16;   // weight bytes per lane per 64-k chunk
   const size_t wt_bytes = (size_t)(K / 64) * 32 * LANE_B, sz_bytes = (size_t)(K / 128) * 64;
-  // this CTA's units: c, c + kQaCluster, ... (nu of them)
-  const int nu = c < U ? min(kQaMaxUnits, (U - 1 - c) / kQaCluster + 1) : 0;
-  // group-local unit -> global 16-row tile of the QKV output: group heads are
-  // rep query heads, then the key head, then the value head
-  auto unit_tile = [&](int u, int second) -> int {
-    const int hh = u / hp, j = u % hp;
+  // this CTA's group tiles: c, c + kQaCluster, ... (nt of them)
+  const int nt = c < TG ? min(kQaMaxTiles, (TG - 1 - c) / kQaCluster + 1) : 0;
+  // group tile -> global 16-row tile of the QKV output: group heads are rep
+  // query heads, then the key head, then the value head
+  auto group_tile = [&](int tau) -> int {
+    const int hh = tau / hpt, j = tau % hpt;
     const int row_base = hh < rep ? (grp * rep + hh) * HD : (hh == rep ? qdim + grp * HD : qdim + kvdim + grp * HD);
-    return row_base / 16 + j + (second ? hp : 0);
+    return row_base / 16 + j;
   };
 
   trace_start(a.trace);
@@ -177,16 +184,16 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     mbar_init(&wbar, 1);
     mbar_init(&kvbar, 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&wbar, (unsigned)(2 * nu * (wt_bytes + sz_bytes)));
+    mbar_arrive_expect_tx(&wbar, (unsigned)(nt * (wt_bytes + sz_bytes)));
     const uint64_t pol = a.l2_keep ? l2_evict_last() : l2_evict_first();
-    for (int i = 0; i < 2 * nu; ++i) {
-      const int tile = unit_tile(c + (i >> 1) * kQaCluster, i & 1);
+    for (int i = 0; i < nt; ++i) {
+      const int tile = group_tile(c + i * kQaCluster);
       const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
       for (size_t off = 0; off < wt_bytes; off += 32768) {
         const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
         bulk_g2s_hint(wsm + i * wt_bytes + off, src + off, n, &wbar, pol);
       }
-      bulk_g2s_hint(wsm + 2 * nu * wt_bytes + i * sz_bytes,
+      bulk_g2s_hint(wsm + nt * wt_bytes + i * sz_bytes,
                     reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes, (unsigned)sz_bytes, &wbar,
                     pol);
     }
@@ -232,12 +239,15 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       }
     }
   }
-  // RoPE (cos, sin) of this thread's epilogue element (loaded under the GEMV)
-  float2 cs_pre = make_float2(1.f, 0.f);
-  if (tid < nu * 16 * M) {
-    const int ul = tid / (16 * M), rem = tid % (16 * M), r = rem & 15, m = rem >> 4;
-    const int u = c + ul * kQaCluster, hh = u / hp, j = (u % hp) * 16 + r;
-    if (hh <= rep) cs_pre = rope_cs(a.rope_tab, rcs[m].pos, j, HD, a.theta);
+  // RoPE (cos, sin) of every row's position, applied after the exchange
+  // (published before the GEMV's block barrier)
+  for (int e = tid; e < M * (HD / 2); e += kQaThreads) {
+    const int m = e / (HD / 2), j = e % (HD / 2);
+    RowCtx rc = rcs[0];
+#pragma unroll
+    for (int q = 1; q < kQaMaxRows; ++q)
+      if (m == q) rc = rcs[q];
+    cst[e] = rope_cs(a.rope_tab, rc.pos, j, HD, a.theta);
   }
 
 #pragma unroll
@@ -328,9 +338,9 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
     const int brow = g8 >> 1;
     const __half* bsrc = ((g8 & 1) ? xl : xs) + (size_t)brow * (K + 8) + 2 * t4;
     const bool bok = brow < M;
-    float acc[2 * kQaMaxUnits][4];
+    float acc[kQaMaxTiles][4];
 #pragma unroll
-    for (int i = 0; i < 2 * kQaMaxUnits; ++i)
+    for (int i = 0; i < kQaMaxTiles; ++i)
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[i][q] = 0.f;
     for (int ci = c0; ok && ci < c1; ++ci) {
@@ -341,8 +351,8 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
         bf[j][1] = bok ? *reinterpret_cast<const uint32_t*>(bsrc + ci * 64 + j * 16 + 8) : 0u;
       }
 #pragma unroll
-      for (int i = 0; i < 2 * kQaMaxUnits; ++i) {
-        if (i < 2 * nu) {
+      for (int i = 0; i < kQaMaxTiles; ++i) {
+        if (i < nt) {
           uint32_t words[4];
           if (BITS == 2) {
             const uint2 w2 = *reinterpret_cast<const uint2*>(wsm + i * wt_bytes + (size_t)ci * 32 * LANE_B + lane * LANE_B);
@@ -352,7 +362,7 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
             words[0] = wv.x; words[1] = wv.y; words[2] = wv.z; words[3] = wv.w;
           }
           const uint2 sv =
-              *reinterpret_cast<const uint2*>(wsm + 2 * nu * wt_bytes + i * sz_bytes + (size_t)(ci >> 1) * 64 + g8 * 8);
+              *reinterpret_cast<const uint2*>(wsm + nt * wt_bytes + i * sz_bytes + (size_t)(ci >> 1) * 64 + g8 * 8);
           float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -371,9 +381,9 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
       }
     }
 #pragma unroll
-    for (int i = 0; i < 2 * kQaMaxUnits; ++i) {
-      if (i < 2 * nu) {
-        float* r = red + ((size_t)warp * 2 * kQaMaxUnits + i) * 64;
+    for (int i = 0; i < kQaMaxTiles; ++i) {
+      if (i < nt) {
+        float* r = red + ((size_t)warp * kQaMaxTiles + i) * 64;
         r[g8 * 4 + t4] = acc[i][0] + acc[i][1];        // tile row g8, activation row t4 (hi + lo)
         r[(g8 + 8) * 4 + t4] = acc[i][2] + acc[i][3];  // tile row g8 + 8
       }
@@ -382,49 +392,54 @@ __global__ void __launch_bounds__(kQaThreads, 1) qkv_attn_kernel(const QkvAttnAr
   __syncthreads();
   trace_mark(a.trace, 10);
 
-  // ---- epilogue: RoPE; q to every rank, k / v to the cache and every rank --
-  if (tid < nu * 16 * M) {   // nu * 16 * M <= 64: one element per thread
-    const int e = tid;
-    const int ul = e / (16 * M), rem = e % (16 * M), r = rem & 15, m = rem >> 4;
-    float va = 0.f, vb = 0.f;
+  // ---- epilogue: the raw projections of this rank's tiles to every rank ----
+  if (tid < nt * 16 * M) {   // nt * 16 * M <= 128: one element per thread
+    const int ti = tid / (16 * M), rem = tid % (16 * M), r = rem & 15, m = rem >> 4;
+    float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kQaWarps; ++w) {
-      va += red[((size_t)w * 2 * kQaMaxUnits + 2 * ul) * 64 + r * 4 + m];
-      vb += red[((size_t)w * 2 * kQaMaxUnits + 2 * ul + 1) * 64 + r * 4 + m];
-    }
-    const int u = c + ul * kQaCluster, hh = u / hp, j = (u % hp) * 16 + r;   // element j < hd/2 of group head hh
-    RowCtx rc = rcs[0];
-#pragma unroll
-    for (int q = 1; q < kQaMaxRows; ++q)
-      if (m == q) rc = rcs[q];
-    float e0 = va, e1 = vb;                                          // elements j and j + hd/2
-    if (hh <= rep) {                                                 // query or key: rotate
-      const float2 cs = cs_pre;
-      e0 = va * cs.x - vb * cs.y;
-      e1 = vb * cs.x + va * cs.y;
-    }
-    float* dst_s;
-    if (hh < rep) {
-      dst_s = qb + (size_t)m * rep * HD + hh * HD;
-    } else {
-      if (!KV8) {
-        __half* cache = (hh == rep ? a.k_plane : a.v_plane) + rc.lane * a.lane_stride +
-                        ((size_t)grp * a.ctx + rc.pos) * HD;
-        const __half h0 = __float2half_rn(e0), h1 = __float2half_rn(e1);
-        if (ok) { cache[j] = h0; cache[j + HD / 2] = h1; }
-        e0 = __half2float(h0);    // attention reads the stored (fp16) key / value
-        e1 = __half2float(h1);
-      }   // INT8: quantised after the exchange, below
-      dst_s = (hh == rep ? knew : vnew) + (size_t)m * HD;
-    }
-    for (unsigned rk = 0; rk < kQaCluster; ++rk) {
-      qa_st_peer(qa_peer(dst_s + j, rk), e0);
-      qa_st_peer(qa_peer(dst_s + j + HD / 2, rk), e1);
-    }
+    for (int w = 0; w < kQaWarps; ++w) v += red[((size_t)w * kQaMaxTiles + ti) * 64 + r * 4 + m];
+    const int gr = (c + ti * kQaCluster) * 16 + r;   // row of the group: q heads, key, value
+    float* dst_s = gr < rep * HD ? qb + (size_t)m * rep * HD + gr
+                                 : (gr < (rep + 1) * HD ? knew + (size_t)m * HD + (gr - rep * HD)
+                                                        : vnew + (size_t)m * HD + (gr - (rep + 1) * HD));
+    for (unsigned rk = 0; rk < kQaCluster; ++rk) qa_st_peer(qa_peer(dst_s, rk), v);
   }
   trace_mark(a.trace, 6);
   qa_cluster_sync();   // #1: q and the new key / value are in every rank
   trace_mark(a.trace, 3);
+  // RoPE on every query head and the key: pairs (j, j + hd/2); with an fp16
+  // cache the key and value become the fp16 values the cache stores (the
+  // attention reads the new position like any cached one)
+  for (int e = tid; e < M * (rep + 1) * (HD / 2); e += kQaThreads) {
+    const int m = e / ((rep + 1) * (HD / 2)), rem = e % ((rep + 1) * (HD / 2));
+    const int hh = rem / (HD / 2), j = rem % (HD / 2);
+    float* base = hh < rep ? qb + (size_t)m * rep * HD + hh * HD : knew + (size_t)m * HD;
+    const float va = base[j], vb = base[j + HD / 2];
+    const float2 cs = cst[m * (HD / 2) + j];
+    float e0 = va * cs.x - vb * cs.y, e1 = vb * cs.x + va * cs.y;
+    if (!KV8 && hh == rep) {
+      e0 = __half2float(__float2half_rn(e0));
+      e1 = __half2float(__float2half_rn(e1));
+    }
+    base[j] = e0;
+    base[j + HD / 2] = e1;
+  }
+  if (!KV8)
+    for (int e = tid; e < M * HD; e += kQaThreads) vnew[e] = __half2float(__float2half_rn(vnew[e]));
+  __syncthreads();
+  if (!KV8 && ok) {
+    // this rank's hd / kQaCluster elements of each row's new key and value
+    constexpr int PER = HD / kQaCluster;
+    if (tid < M * 2 * PER) {
+      const int m = tid / (2 * PER), kv = (tid / PER) & 1, j = c * PER + tid % PER;
+      RowCtx rc = rcs[0];
+#pragma unroll
+      for (int q = 1; q < kQaMaxRows; ++q)
+        if (m == q) rc = rcs[q];
+      __half* cache = (kv ? a.v_plane : a.k_plane) + rc.lane * a.lane_stride + ((size_t)grp * a.ctx + rc.pos) * HD;
+      cache[j] = __float2half_rn((kv ? vnew : knew)[(size_t)m * HD + j]);
+    }
+  }
   if (KV8) {
     // INT8 cache: warp 2m + kv quantises row m's new key (kv = 0) or value;
     // every rank computes the same codes, rank 0 stores them, and attention

@@ -936,7 +936,7 @@ bool qkv_attn_ok(const tl_model* m) {
   const tl_config& c = m->cfg;
   const int rep = c.n_q_heads / c.n_kv_heads;
   if (!m->use_qkv_attn || (c.head_dim != 64 && c.head_dim != 128) || c.d_model > 4 * 4 * kQaThreads) return false;
-  if (qa_units_per_cta(rep, c.head_dim) > kQaMaxUnits || rep * c.head_dim > 4 * kQaThreads) return false;
+  if (qa_tiles_per_cta(rep, c.head_dim) > kQaMaxTiles || rep * c.head_dim > 4 * kQaThreads) return false;
   return qa_layout(c.d_model, kQaMaxRows, rep, c.head_dim).total <= (size_t)m->qa_smem_max;
 }
 
