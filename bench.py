@@ -963,6 +963,9 @@ def run_workload_lsweep(args):
         return a.elapsed_time(b)
 
     with ClockSampler(0) as clocks:
+        # batch 1: the clustered per-op form (a model built for <= 2 lanes takes
+        # it by default; this one holds 16 lanes for the lane rows below)
+        tl.tl_model_set_clustered_decode(m, True)
         for L in (1, 2, 4, 8, 16):
             fn = lambda: tl.tl_prefill(m, 0, d_prompts[0], P, L, None, None, st)
             for _ in range(3):
@@ -974,12 +977,14 @@ def run_workload_lsweep(args):
             kv = (2 + L) * 2 * HKV * HD * 2 * (P + n_dec / 2)
             t_roof, _, _ = _decode_roofline_us(kv, [L], l2_gbs, peaks)
             us_tok = 1e3 * ms / n_dec
-            sweep.append({"L": L, "prefill_T512_ms": round(pf, 4), "prefill_flops": int(flops),
+            sweep.append({"L": L, "decode_form": "clustered", "prefill_T512_ms": round(pf, 4), "prefill_flops": int(flops),
                           "prefill_tflops": round(flops / (pf * 1e9), 2),
                           "prefill_frac": round(flops / (pf * 1e9) / peaks["bf16_tflops"], 4),
                           "decode_tok_s": round(n_dec / (ms / 1e3), 1), "decode_us_per_step": round(us_tok, 2),
                           "decode_roofline_us": round(t_roof, 2), "decode_frac": round(t_roof / us_tok, 4)})
         for n in (1, 4, 16):
+            # the form the library picks for a model built for n lanes
+            tl.tl_model_set_clustered_decode(m, n <= 2)
             loops = [int(v) for v in tl_synth.make_lane_loops(tl_synth.SEED_LSWEEP, n)]
             lanes = list(range(n))
             decode_run(lanes, loops)      # warm (graph capture)
@@ -987,7 +992,8 @@ def run_workload_lsweep(args):
             kv = sum((2 + L) * 2 * HKV * HD * 2 * (P + n_dec / 2) for L in loops)
             t_roof, _, _ = _decode_roofline_us(kv, loops, l2_gbs, peaks)
             us_step = 1e3 * ms / n_dec
-            lanes_res.append({"lanes": n, "loops": loops, "decode_tok_s": round(n * n_dec / (ms / 1e3), 1),
+            lanes_res.append({"lanes": n, "loops": loops, "decode_form": "clustered" if n <= 2 else "gemv+split-kv",
+                              "decode_tok_s": round(n * n_dec / (ms / 1e3), 1),
                               "us_per_step": round(us_step, 2), "roofline_us_per_step": round(t_roof, 2),
                               "frac": round(t_roof / us_step, 4)})
     tl.tl_check_device_error(m)
@@ -1055,6 +1061,9 @@ def run_workload_next(args):
     import weight_shared_looped_int4_b200 as tl
     peaks = load_peaks()
     w, m = _lm_model(tl, tl_synth, 16, 1024, 4)
+    # single-lane decoding throughout: the clustered per-op form (the default
+    # of a model built for <= 2 lanes; this one holds 4 for the prefix forks)
+    tl.tl_model_set_clustered_decode(m, True)
     P, n = 128, 128
     prompt = tl_synth.make_tokens(tl_synth.SEED_LM, w.shape.vocab, 1024)
     d_prompt = torch.as_tensor(prompt, device=dev)

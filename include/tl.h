@@ -80,10 +80,9 @@ typedef struct {
  * head: head_dim elements) as int8 codes with one fp32 scale, scale =
  * max|x| / 127 and code = round-half-even(x / scale) in fp32 (an all-zero
  * vector has scale 0); attention reads code * scale.  INT8 halves the cache's
- * bytes.  It needs the clustered decode kernel (tl_model_create returns
- * TL_ERR_UNSUPPORTED for shapes that do not fit it) and runs every prefill
- * attention pass on the 16-query tile kernel; the single-kernel decode path
- * (TL_DECODE_FUSED) is FP16 only. */
+ * bytes.  Both per-op decode forms (tl_model_set_clustered_decode) read and
+ * write it; every prefill attention pass runs on the 16-query tile kernel;
+ * the single-kernel decode path (TL_DECODE_FUSED) is FP16 only. */
 enum { TL_KV_FP16 = 0, TL_KV_INT8 = 1 };
 
 /* One INT4 linear with K inputs and N outputs, HOST memory, storage format
@@ -349,6 +348,19 @@ typedef enum {
   TL_DECODE_FUSED = 2
 } tl_decode_path;
 tl_status tl_model_set_decode_path(tl_model *m, int path);
+
+/* Which per-op (TL_DECODE_LAYERED) step a model takes: enable = 1 runs each
+ * layer's RMSNorm + QKV + RoPE + KV write + attention as ONE clustered kernel
+ * (a thread-block cluster per kv head, <= 2 rows per launch); enable = 0 runs
+ * the QKV GEMV and the split-KV attention kernel (every row in one launch
+ * each; with an INT8 cache a quantising pass between them).  The default,
+ * chosen at creation: clustered for max_lanes <= 2, otherwise the GEMV +
+ * split-KV form (faster from 3 lanes on).  It is per model, so a lane's
+ * results never depend on which lanes share a step.  Synchronises the device
+ * and drops captured decode graphs when it changes the form.
+ * TL_ERR_UNSUPPORTED: enable = 1 where the clustered kernel does not fit the
+ * shapes or device. */
+tl_status tl_model_set_clustered_decode(tl_model *m, int enable);
 
 /* Phase timeline of single-kernel decode steps (the counterpart of the pages'
  * per-phase timings, TinyLoop README, "Quick CLI Tour", Benchmark with

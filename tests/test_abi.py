@@ -73,6 +73,7 @@ def test_model_controls_reject_a_null_model_on_host():
     for call in (lambda: tl.tl_model_set_trace(None, None, 0),
                  lambda: tl.tl_model_set_decode_path(None, tl.DECODE_LAYERED),
                  lambda: tl.tl_model_set_graphs(None, True),
+                 lambda: tl.tl_model_set_clustered_decode(None, True),
                  lambda: tl.tl_model_set_wait_test(None, 0)):
         with pytest.raises(tl.TLError) as e:
             call()

@@ -7,12 +7,16 @@
 * What the cache stores after a prefill of the 400M LM, exported slice by
   slice: codes and scales against the oracle's quantisation of the keys and
   values it was given.
+* What a decode step stores for its new position, in both decode forms:
+  codes and scales against the oracle's quantisation of the same step's key
+  and value.
 * The model: every path that writes or reads the cache (the tensor-core
-  prefill and its quantising pass, the short GEMV pass, the clustered decode
-  kernel, the 16-query tile prefill attention, extend, fork, self-speculative
-  decode) against the INT8 oracle: logits max-abs <= 5e-2 (see
-  INT8_LOGIT_MAX_ABS), greedy tokens exact unless the oracle's top-2 margin
-  is below that bound.
+  prefill and its quantising pass, the short GEMV pass, both per-op decode
+  forms -- the clustered kernel, and the QKV GEMV + quantising pass + split-KV
+  attention -- the 16-query tile prefill attention, extend, fork,
+  self-speculative decode) against the INT8 oracle: logits max-abs <= 5e-2
+  (see INT8_LOGIT_MAX_ABS), greedy tokens exact unless the oracle's top-2
+  margin is below that bound.
 """
 
 import numpy as np
@@ -75,6 +79,14 @@ def tiny8():
     gm.close()
 
 
+FORMS = ["clustered", "split"]
+
+
+def _form(gm, form):
+    tl.tl_model_set_decode_path(gm.handle, tl.DECODE_LAYERED)
+    tl.tl_model_set_clustered_decode(gm.handle, form == "clustered")
+
+
 # End-to-end bound in INT8 mode.  A stored code is a rounding decision, and
 # the GPU takes it on its own fp32 key / value, which differs from the
 # oracle's by the linear's rounding: at a rounding boundary the two caches
@@ -98,25 +110,32 @@ def _teacher_forced(gm, om, lane, toks, P, L, steps, where):
         check_argmax(int(gam[0]), olg, f"{where} step {i}", margin=INT8_LOGIT_MAX_ABS)
 
 
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("P,L", [(32, 4), (9, 3), (31, 6), (200, 2)])
-def test_tiny_int8_prefill_decode(tiny8, P, L):
+def test_tiny_int8_prefill_decode(tiny8, P, L, form):
     # P >= 32: tensor-core prefill + quantising pass; P < 32: the GEMV pass
     # (31 rows: two row chunks of the GEMV launch)
     w, om, gm = tiny8
+    _form(gm, form)
     toks = tl_synth.make_tokens(500 + P, w.shape.vocab, P + 12)
     _teacher_forced(gm, om, 1, toks, P, L, 12, f"tiny int8 P={P} L={L}")
 
 
-def test_tiny_int8_long_prompt(tiny8):
+@pytest.mark.parametrize("form", FORMS)
+def test_tiny_int8_long_prompt(tiny8, form):
     # 1100 positions: the prefill attention stays on the 16-query tiles, and
-    # decode splits the keys over every cluster rank in several chunks
+    # decode splits the keys over every cluster rank in several chunks (or
+    # over five 256-key CTAs)
     w, om, gm = tiny8
+    _form(gm, form)
     toks = tl_synth.make_tokens(77, w.shape.vocab, 1104)
     _teacher_forced(gm, om, 2, toks, 1100, 3, 4, "tiny int8 long")
 
 
-def test_tiny_int8_two_lanes_extend_fork(tiny8):
+@pytest.mark.parametrize("form", FORMS)
+def test_tiny_int8_two_lanes_extend_fork(tiny8, form):
     w, om, gm = tiny8
+    _form(gm, form)
     L = 3
     toks = tl_synth.make_tokens(610, w.shape.vocab, 60)
     gm.prefill_lane(3, toks[:40], L, logits=False)
@@ -144,8 +163,10 @@ def test_tiny_int8_two_lanes_extend_fork(tiny8):
         check_argmax(int(gam[1]), olg2, f"fork {i}", margin=INT8_LOGIT_MAX_ABS)
 
 
-def test_tiny_int8_speculative(tiny8):
+@pytest.mark.parametrize("form", FORMS)
+def test_tiny_int8_speculative(tiny8, form):
     w, om, gm = tiny8
+    _form(gm, form)
     L, P, n = 6, 30, 24
     prompt = tl_synth.make_tokens(620, w.shape.vocab, P + 1)
     o_tokens, o_logits = om.generate_greedy(prompt, L, n)
@@ -161,6 +182,49 @@ def test_tiny_int8_speculative(tiny8):
             break
 
 
+@pytest.mark.parametrize("form", FORMS)
+def test_tiny_int8_decode_step_stores(tiny8, form):
+    # A decode step's own key and value, quantised by the step (the clustered
+    # kernel's rank 0, or the quantising pass after the QKV GEMV), against
+    # the oracle's quantisation of the same step's layer-0 key and value: the
+    # scales to float precision and every code a rounding of the oracle's
+    # x / scale to within 2e-3 of the rounding point (the GPU rounds its own
+    # fp32 value).
+    w, om, gm = tiny8
+    _form(gm, form)
+    sh = w.shape
+    L, P, lane = 3, 20, 6
+    toks = tl_synth.make_tokens(640, sh.vocab, P + 1)
+    gm.prefill_lane(lane, toks[:P], L, logits=False)
+    cache, _ = om.prefill(toks[:P], L)
+    om.kv_trace = []
+    try:
+        gm.decode([lane], [int(toks[P])], [L])
+        om.decode(cache, int(toks[P]), L)
+        trace = om.kv_trace
+    finally:
+        om.kv_trace = None
+    H, hd = sh.n_kv_heads, sh.head_dim
+    for layer, k, v in trace[:2]:   # the pre block and the first loop iteration
+        d_c = [torch.empty((H, P + 1, hd), dtype=torch.int8, device=DEV) for _ in range(2)]
+        d_s = [torch.empty((H, P + 1), dtype=torch.float32, device=DEV) for _ in range(2)]
+        tl.tl_lane_kv_export(gm.handle, lane, layer, P + 1, d_c[0], d_c[1], d_s[0], d_s[1])
+        torch.cuda.synchronize()
+        for kv, x in ((0, k), (1, v)):
+            xo = x[0]                                    # [H][hd], position P
+            oc, os_ = ref.quantize_kv_int8(xo)
+            gc = d_c[kv].cpu().numpy()[:, P].astype(np.int32)
+            gs = d_s[kv].cpu().numpy()[:, P]
+            where = f"{form} layer {layer} {'KV'[kv]}"
+            np.testing.assert_allclose(gs, os_, rtol=1e-4 if layer == 0 else 1e-2, err_msg=where)
+            if layer == 0:
+                safe = np.where(os_ > 0, os_, 1.0)[:, None]
+                dev = np.abs(gc - xo / safe)
+                assert dev.max() <= 0.5 + 2e-3, (where, float(dev.max()))
+            else:
+                assert np.abs(gc - oc.astype(np.int32)).max() <= 2, where
+
+
 def test_int8_fused_path_unsupported(tiny8):
     w, om, gm = tiny8
     with pytest.raises(tl.TLError) as e:
@@ -169,7 +233,8 @@ def test_int8_fused_path_unsupported(tiny8):
     gm.set_path(tl.DECODE_AUTO)
 
 
-def test_lm_int8_prefill_decode():
+@pytest.mark.parametrize("form", FORMS)
+def test_lm_int8_prefill_decode(form):
     # the 400M LM: 128-token prompt, 24 teacher-forced decode steps at L = 8,
     # and the KV cache takes about half the bytes of the fp16 one
     need_gpu()
@@ -182,7 +247,8 @@ def test_lm_int8_prefill_decode():
         kv16 = tl.tl_model_info(gm16.handle)["kv_bytes"]
         assert abs(kv8 / kv16 - (0.5 + 2.0 / w.shape.head_dim)) < 1e-9
         toks = tl_synth.make_tokens(tl_synth.SEED_LM, w.shape.vocab, 128 + 24)
-        _teacher_forced(gm, om, 0, toks, 128, 8, 24, "LM int8")
+        _form(gm, form)
+        _teacher_forced(gm, om, 0, toks, 128, 8, 24, f"LM int8 {form}")
     finally:
         gm.close()
         gm16.close()

@@ -42,13 +42,31 @@ def _max_abs(a, b):
     return float(np.max(np.abs(np.asarray(a) - np.asarray(b))))
 
 
-@pytest.fixture(params=[tl.DECODE_FUSED, tl.DECODE_LAYERED], ids=["fused", "layered"])
+# Decode forms: the single-kernel step, the per-op step through the clustered
+# QKV + attention kernel, and the per-op step through the QKV GEMV + split-KV
+# attention (a model's default between the last two follows its max_lanes).
+@pytest.fixture(params=["fused", "layered", "split"])
 def path(request):
     return request.param
 
 
+def _set_clustered(gm, enable):
+    """Select the per-op form; False where the clustered kernel does not fit."""
+    try:
+        tl.tl_model_set_clustered_decode(gm.handle, enable)
+        return enable
+    except tl.TLError as e:
+        assert enable and e.status == tl.TL_ERR_UNSUPPORTED
+        tl.tl_model_set_clustered_decode(gm.handle, False)
+        return False
+
+
 def _use(gm, path):
-    gm.set_path(path)
+    if path == "fused":
+        gm.set_path(tl.DECODE_FUSED)
+    else:
+        gm.set_path(tl.DECODE_LAYERED)
+        _set_clustered(gm, path == "layered")
     return gm
 
 
@@ -401,39 +419,51 @@ def test_lm_sixteen_lanes_every_lane(lm):
     # All 16 lanes in one decode step, per-lane loops drawn from {4, 8, 16},
     # ragged prompt lengths; every lane is compared with its own single-lane
     # oracle run, on two consecutive steps.
+    # Both per-op forms: the model's default (GEMV + split-KV: 16 lanes) and
+    # the clustered kernel (eight launches of two rows per layer).
     w, om, gm = lm
-    gm.set_path(tl.DECODE_AUTO)
     n = 16
     loops = [int(v) for v in tl_synth.make_lane_loops(tl_synth.SEED_LSWEEP + 16, n)]
     prompts = tl_synth.make_lane_prompts(tl_synth.SEED_LSWEEP + 16, w.shape.vocab, n, 100)
     lens = [40 + 4 * i for i in range(n)]       # 40 .. 100 tokens
-    caches = []
+    feeds = [[int(prompts[i, lens[i] - 1]) ^ 1 for i in range(n)]]   # any in-range ids
+    feeds.append([int((t * 7 + 3) % w.shape.vocab) for t in feeds[0]])
+    expects = [[], []]
     for i in range(n):
-        gm.prefill_lane(i, prompts[i, :lens[i]], loops[i], logits=False)
-        caches.append(om.prefill(prompts[i, :lens[i]], loops[i])[0])
-    fed = [int(prompts[i, lens[i] - 1]) ^ 1 for i in range(n)]   # any in-range ids
-    for step in range(2):
-        lg, am = gm.decode(list(range(n)), fed, loops)
+        cache = om.prefill(prompts[i, :lens[i]], loops[i])[0]
+        for step in range(2):
+            expects[step].append(om.decode(cache, feeds[step][i], loops[i]))
+    for clustered in (False, True):
+        gm.set_path(tl.DECODE_LAYERED)
+        assert _set_clustered(gm, clustered) == clustered
         for i in range(n):
-            expect = om.decode(caches[i], fed[i], loops[i])
-            err = _max_abs(lg[i], expect)
-            assert err <= LOGIT_MAX_ABS, (step, i, loops[i], err)
-            check_argmax(int(am[i]), expect, f"step {step} lane {i}")
-        fed = [int((t * 7 + 3) % w.shape.vocab) for t in fed]
+            gm.prefill_lane(i, prompts[i, :lens[i]], loops[i], logits=False)
+        for step in range(2):
+            lg, am = gm.decode(list(range(n)), feeds[step], loops)
+            for i in range(n):
+                err = _max_abs(lg[i], expects[step][i])
+                assert err <= LOGIT_MAX_ABS, (clustered, step, i, loops[i], err)
+                check_argmax(int(am[i]), expects[step][i], f"clustered {clustered} step {step} lane {i}")
+    _set_clustered(gm, False)
 
 
 def test_lm_long_context(lm):
     # One lane decoding at the end of the 2048-token context: a 2040-token
     # prompt at L = 2, then decode steps up to position 2047 (the last slot).
+    # Both per-op forms (the clustered kernel's key split spans several
+    # 64-key chunks per rank here).
     w, om, gm = lm
-    gm.set_path(tl.DECODE_AUTO)
     L, P = 2, 2040
     prompt = tl_synth.make_tokens(tl_synth.SEED_LSWEEP + 2048, w.shape.vocab, 2048)
     cache, _ = om.prefill(prompt[:P], L)
-    gm.prefill_lane(8, prompt[:P], L, logits=False)
-    for pos in range(P, 2048):
-        expect = om.decode(cache, int(prompt[pos]), L)
-        glg, gam = gm.decode([8], [int(prompt[pos])], [L])
-        err = _max_abs(glg[0], expect)
-        assert err <= LOGIT_MAX_ABS, (pos, err)
-        check_argmax(int(gam[0]), expect, f"position {pos}")
+    expects = [om.decode(cache, int(prompt[pos]), L) for pos in range(P, 2048)]
+    for clustered in (False, True):
+        gm.set_path(tl.DECODE_LAYERED)
+        assert _set_clustered(gm, clustered) == clustered
+        gm.prefill_lane(8, prompt[:P], L, logits=False)
+        for pos in range(P, 2048):
+            glg, gam = gm.decode([8], [int(prompt[pos])], [L])
+            err = _max_abs(glg[0], expects[pos - P])
+            assert err <= LOGIT_MAX_ABS, (clustered, pos, err)
+            check_argmax(int(gam[0]), expects[pos - P], f"clustered {clustered} position {pos}")
+    _set_clustered(gm, False)

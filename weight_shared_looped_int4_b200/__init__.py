@@ -30,6 +30,7 @@ __all__ = [
     "tl_lane_length", "tl_model_info", "tl_check_device_error",
     "tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count", "KERNEL_CLASSES",
     "tl_model_set_graphs", "tl_model_set_decode_path", "DECODE_AUTO", "DECODE_LAYERED", "DECODE_FUSED",
+    "tl_model_set_clustered_decode",
     "tl_probe_read_bandwidth", "tl_model_set_trace", "tl_model_trace_grid",
     "tl_model_set_wait_test", "tl_extend", "tl_generate_speculative", "tl_score_logit_lens",
     "tl_score_early_exit", "tl_lane_fork", "tl_spec_stats", "tl_set_prefill_attention_tc_min",
@@ -100,6 +101,7 @@ def _load():
         "tl_kernel_launch_count": (ctypes.c_ulonglong, []),
         "tl_model_set_graphs": (st, [P, c_int]),
         "tl_model_set_decode_path": (st, [P, c_int]),
+        "tl_model_set_clustered_decode": (st, [P, c_int]),
         "tl_model_set_trace": (st, [P, P, c_longlong]),
         "tl_model_trace_grid": (c_int, [P]),
         "tl_model_set_wait_test": (st, [P, c_int]),
@@ -151,7 +153,8 @@ def __getattr__(name):
 
 # names every header declaration must have in the library (checked by tests)
 EXPORTED = sorted(["tl_model_profile_start", "tl_model_profile_stop", "tl_kernel_launch_count",
-                   "tl_model_set_graphs", "tl_model_set_decode_path", "tl_probe_read_bandwidth",
+                   "tl_model_set_graphs", "tl_model_set_decode_path", "tl_model_set_clustered_decode",
+                   "tl_probe_read_bandwidth",
                    "tl_model_set_trace", "tl_model_trace_grid", "tl_model_set_wait_test",
                    "tl_extend", "tl_generate_speculative", "tl_score_logit_lens", "tl_score_early_exit",
                    "tl_lane_fork", "tl_set_prefill_attention_tc_min",
@@ -379,6 +382,12 @@ def tl_model_set_wait_test(model, extra_arrivals: int) -> None:
     """Test hook: 1 makes the next single-kernel steps' grid barriers run out
     of time (see tl.h); 0 restores normal steps."""
     _check(_L().tl_model_set_wait_test(model, int(extra_arrivals)))
+
+
+def tl_model_set_clustered_decode(model, enable: bool) -> None:
+    """Per-op decode through the clustered QKV + attention kernel (True) or
+    the QKV GEMV + split-KV attention (False); see include/tl.h."""
+    _check(_L().tl_model_set_clustered_decode(model, 1 if enable else 0))
 
 
 def tl_model_set_decode_path(model, path: int) -> None:

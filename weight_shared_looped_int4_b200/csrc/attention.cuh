@@ -44,9 +44,11 @@ constexpr int kTcTokensB = 128;
 // weights, 2 pad) floats, so every head's block starts 16-byte aligned.
 constexpr int kPartPad = 4;
 
-__host__ __device__ inline size_t decode_attn_smem_bytes(int hd, int rep) {
+// K and V of one split as fp16 rows; with the INT8 cache also their codes as
+// copied and the split's scales
+__host__ __device__ inline size_t decode_attn_smem_bytes(int hd, int rep, bool kv8 = false) {
   (void)rep;
-  return (size_t)2 * kDecodeSub * (hd + kKeyPad) * 2;  // K and V of one split
+  return (size_t)2 * kDecodeSub * (hd + kKeyPad) * 2 + (kv8 ? (size_t)2 * kDecodeSub * (hd + 4) : 0);
 }
 
 // Queries and outputs are fp32 inside the model (no rounding between the QKV
@@ -55,8 +57,10 @@ struct DecodeAttnArgs {
   const float* qf;       // [rows][Hq*hd] rotated queries (fp32), or
   const __half* qh;      // the same in fp16
   int ldq;
-  const __half* k;       // K plane of lane 0 (this layer)
-  const __half* v;       // V plane of lane 0
+  const __half* k;       // K plane of lane 0 (this layer); INT8 cache: int8
+  const __half* v;       // codes at the same element offsets
+  const float* ks;       // INT8 cache: K / V scales of lane 0 [Hkv][ctx]
+  const float* vs;       // (element offset / hd); NULL for fp16
   long long lane_stride; // elements between lanes
   int ctx;
   const RowCtx* rows;    // lane and position of each row; keys 0..pos
@@ -115,7 +119,11 @@ __device__ __forceinline__ void split_h2(float a, float b, uint32_t& hi, uint32_
 // split, then warp w computes output dims 8w..8w+7 over all keys (O = P V).
 // Q and P are split into fp16 pairs (hi, lo).  Splits are merged by the last
 // CTA of the (row, kv head) to finish (see above).
-template <int HD, int REP, bool F32>
+// KV8 (INT8 cache): the codes are copied as they are stored and widened to
+// fp16 rows (exact integers) once they land; S column j is multiplied by
+// key j's scale and the softmax weights by the value's scale before P V (the
+// weight sums use the unscaled weights): attention over code * scale.
+template <int HD, int REP, bool F32, bool KV8 = false>
 __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const DecodeAttnArgs a) {
   constexpr int SUB = kDecodeSub;
   constexpr int KC = HD / 16;
@@ -124,6 +132,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   extern __shared__ __align__(128) unsigned char dsm[];
   __half* ks = reinterpret_cast<__half*>(dsm);                 // [SUB][LDK]
   __half* vs = ks + (size_t)SUB * LDK;                         // [SUB][LDK]
+  int8_t* kc8 = reinterpret_cast<int8_t*>(vs + (size_t)SUB * LDK);   // KV8: codes [SUB][HD]
+  int8_t* vc8 = kc8 + (size_t)SUB * HD;
+  float* ksc = reinterpret_cast<float*>(vc8 + (size_t)SUB * HD);    // KV8: scales [SUB]
+  float* vsc = ksc + SUB;
   __shared__ __align__(16) float sc[REP][SUB + 4];
   __shared__ float s_m[REP], s_l[REP];
   __shared__ int s_last;
@@ -142,24 +154,58 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   const int j0 = split * C, j1 = min(n, j0 + C), nk = j1 - j0;
   const float scale = 1.0f / sqrtf((float)HD);
 
-  const __half* kp = a.k + rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;
-  const __half* vp = a.v + rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;
+  const size_t lane_kv = (size_t)rc.lane * a.lane_stride + (size_t)kvh * a.ctx * HD;   // elements
   // keys first, values in a second group: the scores and the softmax run
   // while the values are still arriving
-  for (int c = threadIdx.x; c < CHUNKS; c += kDecodeThreads) {
-    const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
-    const bool ok = key < nk;
-    const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
-    cp_async16(ks + key * LDK + off, kp + src, ok ? 16 : 0);
+  if (KV8) {
+    constexpr int CCH = SUB * HD / 16;   // 16-byte pieces of the codes
+    const int8_t* kp8 = reinterpret_cast<const int8_t*>(a.k) + lane_kv;
+    const int8_t* vp8 = reinterpret_cast<const int8_t*>(a.v) + lane_kv;
+    for (int c = threadIdx.x; c < CCH; c += kDecodeThreads) {
+      const int key = c / (HD / 16), off = (c % (HD / 16)) * 16;
+      const bool ok = key < nk;
+      cp_async16(kc8 + key * HD + off, kp8 + (ok ? (size_t)(j0 + key) * HD + off : 0), ok ? 16 : 0);
+    }
+    cp_async_commit();
+    for (int c = threadIdx.x; c < CCH; c += kDecodeThreads) {
+      const int key = c / (HD / 16), off = (c % (HD / 16)) * 16;
+      const bool ok = key < nk;
+      cp_async16(vc8 + key * HD + off, vp8 + (ok ? (size_t)(j0 + key) * HD + off : 0), ok ? 16 : 0);
+    }
+    cp_async_commit();
+    const size_t s0 = lane_kv / HD + j0;
+    for (int j = threadIdx.x; j < SUB; j += kDecodeThreads) {
+      ksc[j] = j < nk ? __ldcg(a.ks + s0 + j) : 0.f;
+      vsc[j] = j < nk ? __ldcg(a.vs + s0 + j) : 0.f;
+    }
+  } else {
+    const __half* kp = a.k + lane_kv;
+    const __half* vp = a.v + lane_kv;
+    for (int c = threadIdx.x; c < CHUNKS; c += kDecodeThreads) {
+      const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
+      const bool ok = key < nk;
+      const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
+      cp_async16(ks + key * LDK + off, kp + src, ok ? 16 : 0);
+    }
+    cp_async_commit();
+    for (int c = threadIdx.x; c < CHUNKS; c += kDecodeThreads) {
+      const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
+      const bool ok = key < nk;
+      const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
+      cp_async16(vs + key * LDK + off, vp + src, ok ? 16 : 0);
+    }
+    cp_async_commit();
   }
-  cp_async_commit();
-  for (int c = threadIdx.x; c < CHUNKS; c += kDecodeThreads) {
-    const int key = c / (HD / 8), off = (c % (HD / 8)) * 8;
-    const bool ok = key < nk;
-    const size_t src = ok ? (size_t)(j0 + key) * HD + off : 0;
-    cp_async16(vs + key * LDK + off, vp + src, ok ? 16 : 0);
-  }
-  cp_async_commit();
+  // KV8: widen the landed codes of one plane to fp16 rows
+  auto widen = [&](const int8_t* src8, __half* dst) {
+    for (int e = threadIdx.x; e < SUB * HD / 4; e += kDecodeThreads) {
+      const int key = e / (HD / 4), d4 = (e % (HD / 4)) * 4;
+      __half2 c01, c23;
+      kv8_codes_h2(*reinterpret_cast<const uint32_t*>(src8 + key * HD + d4), c01, c23);
+      *reinterpret_cast<__half2*>(dst + key * LDK + d4) = c01;
+      *reinterpret_cast<__half2*>(dst + key * LDK + d4 + 2) = c23;
+    }
+  };
 
   // Q fragments (hi, lo): MMA row g is q head g of the group (zero beyond REP)
   const size_t qoff = (size_t)row * a.ldq + (size_t)kvh * REP * HD;
@@ -182,6 +228,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   }
   cp_async_wait<1>();   // the keys
   __syncthreads();
+  if (KV8) {
+    widen(kc8, ks);
+    __syncthreads();
+  }
 
   // S for keys kb .. kb+15 of this warp (two n8 tiles) -> shared memory
   const int kb = warp * 16;
@@ -201,8 +251,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
       }
       if (g < REP) {
         const int key = kb + nt * 8 + 2 * t;
-        sc[g][key] = key < nk ? acc0[0] + acc1[0] : -INFINITY;
-        sc[g][key + 1] = key + 1 < nk ? acc0[1] + acc1[1] : -INFINITY;
+        const float f0 = KV8 ? ksc[key] : 1.f, f1 = KV8 ? ksc[key + 1] : 1.f;
+        sc[g][key] = key < nk ? (acc0[0] + acc1[0]) * f0 : -INFINITY;
+        sc[g][key + 1] = key + 1 < nk ? (acc0[1] + acc1[1]) * f1 : -INFINITY;
       }
     }
   }
@@ -227,6 +278,10 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
   }
   cp_async_wait<0>();   // the values
   __syncthreads();
+  if (KV8) {
+    widen(vc8, vs);
+    __syncthreads();
+  }
 
   // O = P V: warp w takes output dims 8w .. 8w+7 over all keys of the split
   const int dt = warp;
@@ -236,8 +291,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attn_kernel(const Decod
     for (int c = 0; c < nch; ++c) {
       uint32_t pa[4] = {0u, 0u, 0u, 0u}, pl[4] = {0u, 0u, 0u, 0u};
       if (g < REP) {
-        const float2 p0 = *reinterpret_cast<const float2*>(&sc[g][c * 16 + 2 * t]);
-        const float2 p1 = *reinterpret_cast<const float2*>(&sc[g][c * 16 + 8 + 2 * t]);
+        float2 p0 = *reinterpret_cast<const float2*>(&sc[g][c * 16 + 2 * t]);
+        float2 p1 = *reinterpret_cast<const float2*>(&sc[g][c * 16 + 8 + 2 * t]);
+        if (KV8) {   // the values' scales (the weight sums stay unscaled)
+          const float2 v0 = *reinterpret_cast<const float2*>(&vsc[c * 16 + 2 * t]);
+          const float2 v1 = *reinterpret_cast<const float2*>(&vsc[c * 16 + 8 + 2 * t]);
+          p0.x *= v0.x; p0.y *= v0.y; p1.x *= v1.x; p1.y *= v1.y;
+        }
         split_h2(p0.x, p0.y, pa[0], pl[0]);
         split_h2(p1.x, p1.y, pa[2], pl[2]);
       }

@@ -60,6 +60,11 @@ struct Kv8QuantArgs {
   float* ks;
   float* vs;
   int Hkv, ctx, pos0;
+  // decode rows (rows != NULL): t indexes the step's rows, each at its own
+  // lane and position; k8 .. vs are lane 0's planes and lane l's start
+  // lane_stride elements (codes) further
+  const RowCtx* rows;
+  long long lane_stride;
 };
 
 constexpr int kKv8Warps = 8;
@@ -86,9 +91,16 @@ __global__ void __launch_bounds__(kKv8Warps * 32) kv8_quant_kernel(const Kv8Quan
     sdst = a.scales + v;
   } else {
     const int head = v % a.Hkv, kv = (v / a.Hkv) & 1, t = v / (2 * a.Hkv);
-    const size_t row = (size_t)head * a.ctx + a.pos0 + t;
-    dst = (kv ? a.v8 : a.k8) + row * HD;
-    sdst = (kv ? a.vs : a.ks) + row;
+    size_t lane_off = 0;
+    int pos = a.pos0 + t;
+    if (a.rows) {
+      const RowCtx rc = a.rows[t];
+      lane_off = (size_t)rc.lane * a.lane_stride;
+      pos = rc.pos;
+    }
+    const size_t row = (size_t)head * a.ctx + pos;
+    dst = (kv ? a.v8 : a.k8) + lane_off + row * HD;
+    sdst = (kv ? a.vs : a.ks) + lane_off / HD + row;
   }
   uint32_t w = 0;
 #pragma unroll
