@@ -107,10 +107,16 @@ __host__ __device__ inline size_t gemv_act_bytes(int K, int M, bool lo) {
 // INT4: 16 bytes per lane per 64-k chunk; INT2: 8
 __host__ __device__ inline size_t gemv_w_bytes(int K, int bits = 4) { return (size_t)(K >> 6) * (bits == 2 ? 256 : 512); }
 __host__ __device__ inline size_t gemv_sz_bytes(int K) { return (size_t)(K >> 7) * 64; }
+// Activation planes of gemv_rows_kernel: kGemvPhaseK columns per phase.
+constexpr int kGemvPhaseK = 512;
+__host__ __device__ inline size_t gemv_rows_act_bytes(int M, bool lo) {
+  return (((size_t)M * (kGemvPhaseK + 8) * 2 * (lo ? 2 : 1)) + 15) / 16 * 16;
+}
+__host__ __device__ inline int gemv_nt(int M, bool lo);
 __host__ __device__ inline size_t gemv_smem_bytes(int K, int M, bool lo, int tpc) {
   const int nc = M <= 8 ? 8 : 16;
-  return (size_t)tpc * (gemv_w_bytes(K) + gemv_sz_bytes(K)) + gemv_act_bytes(K, M, lo) +
-         (size_t)8 * 16 * nc * 4 + 16 * 8 * 4;
+  const size_t act = gemv_nt(M, lo) == 0 ? gemv_act_bytes(K, M, lo) : gemv_rows_act_bytes(M, lo);
+  return (size_t)tpc * (gemv_w_bytes(K) + gemv_sz_bytes(K)) + act + (size_t)8 * 16 * nc * 4 + 16 * 8 * 4;
 }
 
 // Tiles per CTA of each epilogue.
@@ -410,6 +416,280 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
       acc[nt][2] = fmaf(s.y, tmp[nt][2], acc[nt][2]);
       acc[nt][3] = fmaf(s.y, tmp[nt][3], acc[nt][3]);
     }
+  }
+
+  trace_mark(a.trace, 4);
+  if (a.trigger == TRIGGER_AFTER_LOOP) pdl_trigger();
+  // ---- reduce the K slices (fixed order) ---------------------------------
+  float* myred = red + (kq * TPC + tsel) * 16 * NC;
+  if (NT == 0 && LO) {  // columns (2m, 2m+1) = (hi, lo) parts of row m = t
+    myred[g * NC + t] = acc[0][0] + acc[0][1];
+    myred[(g + 8) * NC + t] = acc[0][2] + acc[0][3];
+  } else {
+#pragma unroll
+    for (int nt = 0; nt < NTILES; ++nt) {
+      const int col = nt * 8 + 2 * t;
+      myred[g * NC + col] = acc[nt][0];
+      myred[g * NC + col + 1] = acc[nt][1];
+      myred[(g + 8) * NC + col] = acc[nt][2];
+      myred[(g + 8) * NC + col + 1] = acc[nt][3];
+    }
+  }
+  __syncthreads();
+
+  const int r = threadIdx.x & 15, m = threadIdx.x >> 4;
+  if (m >= M || m >= NC) return;
+  float va = 0.f, vb = 0.f;
+#pragma unroll
+  for (int q = 0; q < KS; ++q) {
+    va += red[(q * TPC + 0) * 16 * NC + r * NC + m];
+    if (TPC == 2) vb += red[(q * TPC + 1) * 16 * NC + r * NC + m];
+  }
+  const int row0 = t0 * 16 + r, row1 = t1 * 16 + r;
+
+  if (EPI == EPI_STORE) {
+    if (row0 < a.n_rows) a.y[(size_t)m * a.ldy + row0] = __float2half_rn(va);
+  } else if (EPI == EPI_RESID) {
+    if (row0 < a.n_rows) a.resid[(size_t)m * a.ldr + row0] += va;
+  } else if (EPI == EPI_SWIGLU) {
+    a.yf[(size_t)m * a.ldy + row0] = silu(va) * vb;
+  } else {  // EPI_ROPE_KV: row0 is element j < hd/2 of a head, row1 = row0 + hd/2
+    const int hd = a.hd;
+    const int j = row0 % hd;
+    const RowCtx rc = a.rows[m];
+    if (row0 < a.n_q_rows) {
+      const float2 cs = rope_cs(a.rope_tab, rc.pos, j, hd, a.theta);
+      float* qo = a.q_out + (size_t)m * a.ldq;
+      qo[row0] = va * cs.x - vb * cs.y;
+      qo[row1] = vb * cs.x + va * cs.y;
+    } else if (row0 < a.n_q_rows + a.n_kv_rows) {
+      const float2 cs = rope_cs(a.rope_tab, rc.pos, j, hd, a.theta);
+      const int kvh = (row0 - a.n_q_rows) / hd;
+      const float k0 = va * cs.x - vb * cs.y, k1 = vb * cs.x + va * cs.y;
+      if (a.kv_stage) {
+        float* dst = a.kv_stage + ((size_t)(m * 2) * (a.n_kv_rows / hd) + kvh) * hd;
+        dst[j] = k0;
+        dst[j + hd / 2] = k1;
+      } else {
+        __half* dst = a.k_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
+        dst[j] = __float2half_rn(k0);
+        dst[j + hd / 2] = __float2half_rn(k1);
+      }
+    } else {
+      const int kvh = (row0 - a.n_q_rows - a.n_kv_rows) / hd;
+      if (a.kv_stage) {
+        float* dst = a.kv_stage + ((size_t)(m * 2 + 1) * (a.n_kv_rows / hd) + kvh) * hd;
+        dst[j] = va;
+        dst[j + hd / 2] = vb;
+      } else {
+        __half* dst = a.v_plane + rc.lane * a.lane_stride + ((size_t)kvh * a.ctx + rc.pos) * hd;
+        dst[j] = __float2half_rn(va);
+        dst[j + hd / 2] = __float2half_rn(vb);
+      }
+    }
+  }
+  trace_mark(a.trace, 5);
+}
+
+// The same GEMV for 5..16 activation rows (NT = 1, 2): the activation planes
+// hold K in phases of kGemvPhaseK columns, a share of every warp's K slice
+// each, so a CTA's planes stay small and several CTAs share an SM (whole
+// 16-row planes held one CTA per SM and spread a 352-CTA grid over 2.4
+// waves).  Every warp keeps its contiguous K slice, chunk order and
+// accumulation, so a row's result equals what the one-pass layout gives.
+template <int NT, int IN, int EPI, int BITS = 4>
+__global__ void __launch_bounds__(kGemvThreads) gemv_rows_kernel(const GemvArgs a) {
+  static_assert(NT != 0, "the one-pass layout is gemv_int4_kernel");
+  constexpr bool LO = (IN != IN_F16);
+  constexpr int TPC = gemv_tpc(EPI);
+  constexpr int KS = 8 / TPC;                 // K slices
+  constexpr int NC = NT == 2 ? 16 : 8;        // reduction columns
+  constexpr int NTILES = NT == 2 ? 2 : 1;     // n8 tiles of the MMA
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t wbar;
+  __shared__ int s_ok;
+  const int K = a.K;
+  const int M = a.M;
+  const int ldxs = kGemvPhaseK + 8;
+  const int n_chunks = K >> 6;
+  const size_t wt_bytes = gemv_w_bytes(K, BITS), sz_bytes = gemv_sz_bytes(K);
+  unsigned char* sw = smem;                                       // [TPC][chunks][32][16 B]
+  unsigned char* ssz = smem + TPC * wt_bytes;                     // [TPC][groups][8][8 B]
+  __half* xs = reinterpret_cast<__half*>(ssz + TPC * sz_bytes);   // hi plane [M][ldxs]
+  __half* xl = xs + (size_t)M * ldxs;                             // lo plane [M][ldxs]
+  float* red = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(xs) + gemv_rows_act_bytes(M, LO));
+  float* ssq = red + 8 * 16 * NC;                                 // [16 rows][8 warps]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int tsel = TPC == 2 ? (warp & 1) : 0;
+  const int kq = TPC == 2 ? (warp >> 1) : warp;
+
+  int t0, t1;
+  if (TPC == 1) {
+    t0 = blockIdx.x;
+    t1 = t0;
+  } else if (a.pair_mode == PAIR_OFFSET) {
+    t0 = blockIdx.x;
+    t1 = t0 + a.pair_off;
+  } else {
+    const int head = blockIdx.x / a.pair_off, j16 = blockIdx.x % a.pair_off;
+    t0 = head * 2 * a.pair_off + j16;
+    t1 = t0 + a.pair_off;
+  }
+
+  trace_start(a.trace);
+  if (a.trigger == TRIGGER_AT_START) pdl_trigger();
+  // The weights do not depend on earlier kernels: start their bulk copies
+  // before waiting for the previous kernel.
+  if (threadIdx.x == 0) {
+    mbar_init(&wbar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&wbar, (unsigned)(TPC * (wt_bytes + sz_bytes)));
+    const uint64_t pol = a.l2_keep ? l2_evict_last() : l2_evict_first();
+    for (int ts = 0; ts < TPC; ++ts) {
+      const int tile = ts ? t1 : t0;
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(a.w) + (size_t)tile * wt_bytes;
+      for (size_t off = 0; off < wt_bytes; off += 32768) {
+        const unsigned n = (unsigned)((wt_bytes - off) < 32768 ? (wt_bytes - off) : 32768);
+        bulk_g2s_hint(sw + ts * wt_bytes + off, src + off, n, &wbar, pol);
+      }
+      bulk_g2s_hint(ssz + ts * sz_bytes, reinterpret_cast<const unsigned char*>(a.sz) + (size_t)tile * sz_bytes,
+                    (unsigned)sz_bytes, &wbar, pol);
+    }
+  }
+
+  pdl_wait();
+  trace_mark(a.trace, 2);
+
+  float acc[NTILES][4];
+  // ---- many rows: the planes hold K in phases of kGemvPhaseK columns -------
+  // a phase stages the next CPW chunks of every warp's K slice
+  constexpr int CPW = kGemvPhaseK / 64 / KS;   // chunks per slice and phase
+  constexpr int LANE_B = BITS == 2 ? 8 : 16;    // weight bytes per lane per chunk
+  const unsigned char* wbase = sw + tsel * wt_bytes + (size_t)lane * LANE_B;
+  const unsigned char* sbase = ssz + tsel * sz_bytes + (size_t)g * 8;
+  const int c_begin = (n_chunks * kq) / KS;
+  const int nc = (n_chunks * (kq + 1)) / KS - c_begin;
+  const int n_ph = ((n_chunks + KS - 1) / KS + CPW - 1) / CPW;   // phases of the longest slice
+#pragma unroll
+  for (int nt = 0; nt < NTILES; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+  __shared__ float s_rs[16];
+  if (IN == IN_NORM) {   // every row's RMS factor over the whole row first
+    for (int m = 0; m < M; ++m) {
+      const float* src = a.x + (size_t)m * a.ldx;
+      float ss = 0.f;
+      for (int k = threadIdx.x * 4; k < K; k += 4 * kGemvThreads) {
+        const float4 v = *reinterpret_cast<const float4*>(src + k);
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) ssq[m * 8 + warp] = ss;
+    }
+    __syncthreads();
+    if (threadIdx.x < M) {
+      float ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) ss += ssq[threadIdx.x * 8 + w];
+      s_rs[threadIdx.x] = 1.0f / sqrtf(ss / (float)K + a.eps);
+    }
+    __syncthreads();
+  }
+  for (int ph = 0; ph < n_ph; ++ph) {
+    // stage chunk l < CPW of phase ph of every slice q at plane column
+    // (q * CPW + l) * 64; chunks past a slice's end are not staged
+    constexpr int G4 = 16;   // 4-column groups per chunk
+    for (int e = threadIdx.x; e < M * KS * CPW * G4; e += kGemvThreads) {
+      const int m = e / (KS * CPW * G4), rem = e % (KS * CPW * G4);
+      const int q = rem / (CPW * G4), l = (rem / G4) % CPW, k4 = (rem % G4) * 4;
+      const int qb = (n_chunks * q) / KS, qe = (n_chunks * (q + 1)) / KS;
+      const int c = qb + ph * CPW + l;
+      if (c >= qe) continue;
+      const int kg = c * 64 + k4, col = (q * CPW + l) * 64 + k4;
+      if (IN == IN_F16) {
+        *reinterpret_cast<uint2*>(xs + m * ldxs + col) =
+            *reinterpret_cast<const uint2*>(a.xh + (size_t)m * a.ldx + kg);
+      } else {
+        float4 v = *reinterpret_cast<const float4*>(a.x + (size_t)m * a.ldx + kg);
+        if (IN == IN_NORM) {
+          const float rs = s_rs[m];
+          const float2 g01 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + kg));
+          const float2 g23 = __half22float2(*reinterpret_cast<const __half2*>(a.gain + kg + 2));
+          v.x = (v.x * rs) * g01.x; v.y = (v.y * rs) * g01.y;
+          v.z = (v.z * rs) * g23.x; v.w = (v.w * rs) * g23.y;
+        }
+        const __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+        const float2 r01 = __half22float2(h01), r23 = __half22float2(h23);
+        const __half2 l01 = __floats2half2_rn(v.x - r01.x, v.y - r01.y);
+        const __half2 l23 = __floats2half2_rn(v.z - r23.x, v.w - r23.y);
+        uint2 ph2, pl2;
+        ph2.x = *reinterpret_cast<const uint32_t*>(&h01); ph2.y = *reinterpret_cast<const uint32_t*>(&h23);
+        pl2.x = *reinterpret_cast<const uint32_t*>(&l01); pl2.y = *reinterpret_cast<const uint32_t*>(&l23);
+        *reinterpret_cast<uint2*>(xs + m * ldxs + col) = ph2;
+        *reinterpret_cast<uint2*>(xl + m * ldxs + col) = pl2;
+      }
+    }
+    if (ph == 0 && threadIdx.x == 0) {
+      trace_mark(a.trace, 6);
+      s_ok = mbar_wait(&wbar, 0) ? 1 : 0;
+      if (!s_ok) atomicOr(a.err_flag, kErrTimeout);
+      trace_mark(a.trace, 3);
+    }
+    __syncthreads();
+    if (!s_ok) return;  // uniform: every thread read the same flag after the barrier
+    for (int l = 0; l < CPW; ++l) {
+      const int ci = ph * CPW + l;
+      if (ci >= nc) break;
+      const int c = c_begin + ci;
+      uint32_t words[4];
+      if (BITS == 2) {
+        const uint2 w2 = *reinterpret_cast<const uint2*>(wbase + (size_t)c * 32 * LANE_B);
+        words[0] = w2.x; words[1] = w2.y; words[2] = 0u; words[3] = 0u;
+      } else {
+        const uint4 wv = *reinterpret_cast<const uint4*>(wbase + (size_t)c * 32 * LANE_B);
+        words[0] = wv.x; words[1] = wv.y; words[2] = wv.z; words[3] = wv.w;
+      }
+      const uint2 sv = *reinterpret_cast<const uint2*>(sbase + (size_t)(c >> 1) * 64);
+      float tmp[NTILES][4];
+#pragma unroll
+      for (int nt = 0; nt < NTILES; ++nt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmp[nt][q] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t af[4];
+        if (BITS == 2) unpack_a_frag2(words[j >> 1], j & 1, sv.y, af);
+        else unpack_a_frag(words[j], sv.y, af);
+        const int ko = (kq * CPW + l) * 64 + j * 16;   // column within the staged phase
+#pragma unroll
+        for (int nt = 0; nt < NTILES; ++nt) {
+          const int row = nt * 8 + g;
+          uint32_t b0 = 0, b1 = 0, c0 = 0, c1 = 0;
+          if (row < M) {
+            const size_t off = (size_t)row * ldxs + ko + 2 * t;
+            b0 = *reinterpret_cast<const uint32_t*>(xs + off);
+            b1 = *reinterpret_cast<const uint32_t*>(xs + off + 8);
+            if (LO) {
+              c0 = *reinterpret_cast<const uint32_t*>(xl + off);
+              c1 = *reinterpret_cast<const uint32_t*>(xl + off + 8);
+            }
+          }
+          mma_f16_16816(tmp[nt], af, b0, b1);
+          if (LO) mma_f16_16816(tmp[nt], af, c0, c1);
+        }
+      }
+      const float2 sc2 = h2_to_f2(sv.x);
+#pragma unroll
+      for (int nt = 0; nt < NTILES; ++nt) {
+        acc[nt][0] = fmaf(sc2.x, tmp[nt][0], acc[nt][0]);
+        acc[nt][1] = fmaf(sc2.x, tmp[nt][1], acc[nt][1]);
+        acc[nt][2] = fmaf(sc2.y, tmp[nt][2], acc[nt][2]);
+        acc[nt][3] = fmaf(sc2.y, tmp[nt][3], acc[nt][3]);
+      }
+    }
+    __syncthreads();   // the planes are restaged for the next phase
   }
 
   trace_mark(a.trace, 4);

@@ -191,8 +191,13 @@ cudaError_t allow_max_smem(K* kern, int dev) {
 
 template <int NT, int IN, int EPI>
 cudaError_t set_gemv_attr(int dev) {
-  const cudaError_t e = allow_max_smem(gemv_int4_kernel<NT, IN, EPI, 4>, dev);
-  return e == cudaSuccess ? allow_max_smem(gemv_int4_kernel<NT, IN, EPI, 2>, dev) : e;
+  if constexpr (NT == 0) {
+    const cudaError_t e = allow_max_smem(gemv_int4_kernel<NT, IN, EPI, 4>, dev);
+    return e == cudaSuccess ? allow_max_smem(gemv_int4_kernel<NT, IN, EPI, 2>, dev) : e;
+  } else {
+    const cudaError_t e = allow_max_smem(gemv_rows_kernel<NT, IN, EPI, 4>, dev);
+    return e == cudaSuccess ? allow_max_smem(gemv_rows_kernel<NT, IN, EPI, 2>, dev) : e;
+  }
 }
 
 cudaError_t init_device_kernels(int dev) {
@@ -282,11 +287,12 @@ cudaError_t launch_gemv(const GemvArgs& a, int grid, int in_mode, int epi, cudaS
   const int nt = gemv_nt(a.M, lo);
   const size_t smem = gemv_smem_bytes(a.K, a.M, lo, gemv_tpc(epi));
   const dim3 g(grid), b(kGemvThreads);
-#define CASE(NT, IN, EPI)                                                                             \
+#define CASE(NT, IN, EPI, KERN)                                                                       \
   if (nt == NT && in_mode == IN && epi == EPI)                                                        \
-    return a.bits == 2 ? launch(gemv_int4_kernel<NT, IN, EPI, 2>, g, b, smem, st, a)                  \
-                       : launch(gemv_int4_kernel<NT, IN, EPI, 4>, g, b, smem, st, a);
-#define CASE3(IN, EPI) CASE(0, IN, EPI) CASE(1, IN, EPI) CASE(2, IN, EPI)
+    return a.bits == 2 ? launch(KERN<NT, IN, EPI, 2>, g, b, smem, st, a)                              \
+                       : launch(KERN<NT, IN, EPI, 4>, g, b, smem, st, a);
+  // one row pass for <= 4 rows (8 without the lo plane), phases of K above
+#define CASE3(IN, EPI) CASE(0, IN, EPI, gemv_int4_kernel) CASE(1, IN, EPI, gemv_rows_kernel) CASE(2, IN, EPI, gemv_rows_kernel)
   CASE3(IN_F16, EPI_STORE) CASE3(IN_F32, EPI_RESID) CASE3(IN_F32W, EPI_RESID) CASE3(IN_NORM, EPI_SWIGLU) CASE3(IN_NORM, EPI_ROPE_KV)
 #undef CASE3
 #undef CASE
