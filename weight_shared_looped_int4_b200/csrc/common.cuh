@@ -118,6 +118,10 @@ __device__ __forceinline__ bool mbar_wait_or_fail(uint64_t* bar, unsigned parity
   atomicOr(fail, 1);
   return false;
 }
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // Global -> shared bulk copy of `bytes` (multiple of 16, both addresses 16-byte
 // aligned); completion is signalled on `bar` as transaction bytes.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {

@@ -94,6 +94,14 @@ struct GemvArgs {
   int trigger;                // PdlTrigger
   int l2_keep;                // 1: the weights are the loop block's (L2 evict-last), else evict-first
   int bits;                   // 4, or 2: INT2 weights (selects gemv_int4_kernel<.., 2>)
+  // L2 prefetch issued at the start (pf NULL: none): pf_count pieces of
+  // pf_piece bytes (a multiple of 16, at most 32 KB) at pf + i * pf_stride,
+  // dealt over the CTAs -- the start of every head tile, read from HBM while
+  // the loop block runs from L2 and HBM is otherwise idle
+  const unsigned char* pf;
+  int pf_count;
+  unsigned pf_piece;
+  size_t pf_stride;
 };
 
 constexpr int kGemvThreads = 256;
@@ -194,6 +202,9 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_int4_kernel(const GemvArgs 
                     (unsigned)sz_bytes, &wbar, pol);
     }
   }
+
+  if (a.pf && threadIdx.x == 32)
+    for (int i = blockIdx.x; i < a.pf_count; i += gridDim.x) bulk_prefetch_l2(a.pf + i * a.pf_stride, a.pf_piece);
 
   pdl_wait();
   trace_mark(a.trace, 2);

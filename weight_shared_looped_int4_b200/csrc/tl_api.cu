@@ -701,6 +701,7 @@ struct tl_model {
   __half* embed = nullptr;
   __half* out_norm = nullptr;
   uint4* head_w = nullptr;
+  int head_pf_layer = -1;         // decode step: the layer whose O projection prefetches the head
   // KV cache: [max_lanes + 1][n_layers_max][2][Hkv][max_ctx][hd] fp16, or
   // with kv_int8 the same element layout in int8 codes (kv points at them)
   // plus the scales kvs with the head dimension collapsed (kv8.cuh)
@@ -986,6 +987,10 @@ tl_status run_qkv_attn(tl_model* m, int layer, int M, const RowCtx* rows, cudaSt
   return TL_OK;
 }
 
+// Bytes of every head tile prefetched into L2 during a decode step's last
+// layer (the loop block runs from L2 then, and HBM is otherwise idle).
+static unsigned g_head_pf_piece = 24576;
+
 // O projection + residual, RMSNorm + gate_up + SwiGLU, down + residual.
 tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float* h, cudaStream_t st) {
   WindowScope window_scope(m, layer);
@@ -1002,6 +1007,15 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   a.trace = next_trace(m);
   a.trigger = TRIGGER_AT_START;
   a.l2_keep = layer >= c.n_pre;
+  if (layer == m->head_pf_layer && g_head_pf_piece > 0) {
+    // the start of every 16-row head tile into L2 while the last layer runs
+    // from it: each warp of the head then begins its tile from L2
+    const size_t tile_bytes = (size_t)16 * c.d_model * 2;
+    a.pf = reinterpret_cast<const unsigned char*>(m->head_w);
+    a.pf_count = c.vocab / 16;
+    a.pf_stride = tile_bytes;
+    a.pf_piece = (unsigned)std::min<size_t>(g_head_pf_piece, tile_bytes);
+  }
   kclass(TL_KERNEL_O_PROJ);
   TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, (b.o.N + 15) / 16, st));
   GemvArgs g{};
@@ -1642,7 +1656,8 @@ tl_status decode_impl(tl_model* m, int n_lanes, const int32_t* h_lane_ids, const
   }
   auto body = [&](cudaStream_t s) -> tl_status {
     m->trace_i = 0;   // layer launches of this step take timeline records 0, 1, ...
-    struct TraceOff { tl_model* m; ~TraceOff() { m->trace_i = -1; } } trace_off{m};
+    m->head_pf_layer = max_layers - 1;
+    struct TraceOff { tl_model* m; ~TraceOff() { m->trace_i = -1; m->head_pf_layer = -1; } } trace_off{m};
     for (int layer = 0; layer < max_layers; ++layer) {
       const int M = active[layer];
       tl_status rc = TL_OK;
