@@ -467,3 +467,56 @@ def test_lm_long_context(lm):
             assert err <= LOGIT_MAX_ABS, (clustered, pos, err)
             check_argmax(int(gam[0]), expects[pos - P], f"clustered {clustered} position {pos}")
     _set_clustered(gm, False)
+
+
+def test_lm_benchmark_model_one_lane(lm):
+    # The benchmark's own configuration: a model built for one lane (so every
+    # clustered launch carries one row), the 128-token prompt prefilled with
+    # no logits, then all 128 teacher-forced greedy steps (contexts 129 ..
+    # 256), every step checked.
+    w, om, _ = lm
+    L, P, steps = 8, 128, 128
+    prompt = tl_synth.make_tokens(tl_synth.SEED_LM, w.shape.vocab, P + 1)
+    o_tokens, o_logits = _memo(om, "greedy", lambda: om.generate_greedy(prompt, L, steps))
+    gm = GpuModel(w, max_loops=8, max_ctx=P + steps, max_lanes=1)
+    try:
+        gm.set_path(tl.DECODE_LAYERED)
+        gm.prefill_lane(0, prompt[:P], L, logits=False)
+        fed = int(prompt[P])
+        for i in range(steps):
+            glg, gam = gm.decode([0], [fed], [L])
+            err = _max_abs(glg[0], o_logits[i])
+            assert err <= LOGIT_MAX_ABS, (i, err)
+            check_argmax(int(gam[0]), o_logits[i], f"step {i}")
+            fed = o_tokens[i]
+    finally:
+        gm.close()
+
+
+@pytest.mark.parametrize("kv_mode", [tl.TL_KV_FP16, tl.TL_KV_INT8])
+def test_tiny_one_lane_decode_250_to_262(kv_mode):
+    # A one-lane model decoding from 250 to 262 cached positions (the
+    # clustered kernel's key split then changes length between steps) in
+    # both cache modes, against the oracle in the same mode.
+    need_gpu()
+    w = tl_synth.make_model_weights(tl_synth.TINY_LM, tl_synth.SEED_TINY)
+    om = ref.LoopedModel(w, kv_mode="int8" if kv_mode == tl.TL_KV_INT8 else None)
+    bound = 5e-2 if kv_mode == tl.TL_KV_INT8 else LOGIT_MAX_ABS   # see test_gpu_kv8.INT8_LOGIT_MAX_ABS
+    gm = GpuModel(w, max_loops=4, max_ctx=272, max_lanes=1, kv_mode=kv_mode)
+    try:
+        gm.set_path(tl.DECODE_LAYERED)
+        L, P = 3, 250
+        toks = tl_synth.make_tokens(909, w.shape.vocab, P + 12)
+        cache, _ = om.prefill(toks[:P], L)
+        gm.prefill_lane(0, toks[:P], L, logits=False)
+        for pos in range(P, P + 12):
+            expect = om.decode(cache, int(toks[pos]), L)
+            glg, gam = gm.decode([0], [int(toks[pos])], [L])
+            err = _max_abs(glg[0], expect)
+            assert err <= bound, (kv_mode, pos, err)
+            if kv_mode == tl.TL_KV_INT8:
+                check_argmax(int(gam[0]), expect, f"kv {kv_mode} position {pos}", margin=bound)
+            else:
+                check_argmax(int(gam[0]), expect, f"kv {kv_mode} position {pos}")
+    finally:
+        gm.close()
