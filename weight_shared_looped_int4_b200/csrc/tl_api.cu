@@ -989,7 +989,7 @@ tl_status run_qkv_attn(tl_model* m, int layer, int M, const RowCtx* rows, cudaSt
 
 // Bytes of every head tile prefetched into L2 during a decode step's last
 // layer (the loop block runs from L2 then, and HBM is otherwise idle).
-static unsigned g_head_pf_piece = 24576;
+constexpr unsigned kHeadPfPiece = 24576;
 
 // O projection + residual, RMSNorm + gate_up + SwiGLU, down + residual.
 tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float* h, cudaStream_t st) {
@@ -1007,14 +1007,14 @@ tl_status run_ffn(tl_model* m, int layer, int M, float* x, const float* o, float
   a.trace = next_trace(m);
   a.trigger = TRIGGER_AT_START;
   a.l2_keep = layer >= c.n_pre;
-  if (layer == m->head_pf_layer && g_head_pf_piece > 0) {
+  if (layer == m->head_pf_layer) {
     // the start of every 16-row head tile into L2 while the last layer runs
     // from it: each warp of the head then begins its tile from L2
     const size_t tile_bytes = (size_t)16 * c.d_model * 2;
     a.pf = reinterpret_cast<const unsigned char*>(m->head_w);
     a.pf_count = c.vocab / 16;
     a.pf_stride = tile_bytes;
-    a.pf_piece = (unsigned)std::min<size_t>(g_head_pf_piece, tile_bytes);
+    a.pf_piece = (unsigned)std::min<size_t>(kHeadPfPiece, tile_bytes);
   }
   kclass(TL_KERNEL_O_PROJ);
   TL_CUDA(launch_gemv_rows(a, M, IN_F32, EPI_RESID, (b.o.N + 15) / 16, st));
