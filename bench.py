@@ -64,8 +64,8 @@ BYTES_PER_LAUNCH = {
 # weights from DRAM; first decode step, NCU_KEYS cached keys per layer for the
 # QKV + attention kernel).  Valid for the kernels as captured; the QKV
 # class's cache part is rescaled to the bench's mean context.
-NCU_TRAFFIC = {"qkv": 3683840, "o_proj": 2262528, "gate_up": 12307200, "down": 6179584,
-               "head": 131147264 + 450816}
+NCU_TRAFFIC = {"qkv": 3683840, "o_proj": 2263040, "gate_up": 12307456, "down": 6179584,
+               "head": 131139584 + 55552}
 NCU_KEYS = PROMPT + 1
 
 
