@@ -393,6 +393,7 @@ constexpr int kHdWarps = 16;
 constexpr int kHdThreads = kHdWarps * 32;
 constexpr int kHdMaxRows = 4;
 constexpr int kHdUnroll = 8;
+constexpr int kHdXChunks = 4;   // float4 columns per thread and row: d <= 8192
 
 __host__ __device__ inline size_t head_direct_smem(int d) { return (size_t)2 * kHdMaxRows * (d + 8) * 2; }
 
@@ -438,40 +439,80 @@ __global__ void __launch_bounds__(kHdThreads, 1) head_direct_kernel(const HeadAr
 #pragma unroll
     for (int u = 0; u < kHdUnroll; ++u) wv[u] = ldg_evict_first(wt + u * 32, pol);
   }
+  // the gains of this thread's columns and the zero rows >= M do not depend
+  // on earlier kernels either; each thread owns columns 4 * (tid + i * T) ..
+  // + 3 of every row (d <= kHdXChunks * 4 * T)
+  uint2 gr[kHdXChunks];
+#pragma unroll
+  for (int i = 0; i < kHdXChunks; ++i) {
+    const int k = (threadIdx.x + i * kHdThreads) * 4;
+    gr[i] = k < d ? *reinterpret_cast<const uint2*>(a.gain + k) : make_uint2(0u, 0u);
+  }
+  for (int e = threadIdx.x; e < (kHdMaxRows - M) * (d / 2); e += kHdThreads) {
+    const int m = M + e / (d / 2), k = (e % (d / 2)) * 2;
+    *reinterpret_cast<uint32_t*>(xs + (size_t)m * ldx + k) = 0u;
+    *reinterpret_cast<uint32_t*>(xl + (size_t)m * ldx + k) = 0u;
+  }
   pdl_trigger();
   pdl_wait();
   float* const logits = a.io ? a.io->logits : a.logits;
   int32_t* const argmax = a.io ? a.io->argmax : a.argmax;
 
-  // RMSNorm of the M rows, staged as fp16 (hi, lo); rows >= M are zero
-  for (int m = 0; m < M; ++m) {
-    float ss = 0.f;
-    for (int k = threadIdx.x * 4; k < d; k += kHdThreads * 4) {
-      const float4 v = *reinterpret_cast<const float4*>(a.x + (size_t)m * d + k);
-      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  // RMSNorm of the M rows, staged as fp16 (hi, lo): every row's loads go out
+  // together, then one block reduction of the sums of squares
+  float4 xr[kHdMaxRows][kHdXChunks];
+#pragma unroll
+  for (int m = 0; m < kHdMaxRows; ++m) {
+#pragma unroll
+    for (int i = 0; i < kHdXChunks; ++i) {
+      const int k = (threadIdx.x + i * kHdThreads) * 4;
+      xr[m][i] = (m < M && k < d) ? *reinterpret_cast<const float4*>(a.x + (size_t)m * d + k)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    ss = warp_sum(ss);
-    if (lane == 0) s_ss[m][warp] = ss;
+  }
+#pragma unroll
+  for (int m = 0; m < kHdMaxRows; ++m) {
+    if (m < M) {
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < kHdXChunks; ++i) {
+        const float4 v = xr[m][i];
+        ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) s_ss[m][warp] = ss;
+    }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kHdMaxRows * (d / 2); e += kHdThreads) {
-    const int m = e / (d / 2), k = (e % (d / 2)) * 2;
-    uint32_t hw = 0, lw = 0;
+#pragma unroll
+  for (int m = 0; m < kHdMaxRows; ++m) {
     if (m < M) {
       float tot = 0.f;
 #pragma unroll
       for (int w = 0; w < kHdWarps; ++w) tot += s_ss[m][w];
       const float rs = 1.0f / sqrtf(tot / (float)d + a.eps);
-      const float2 xv = *reinterpret_cast<const float2*>(a.x + (size_t)m * d + k);
-      const float2 gv = __half22float2(*reinterpret_cast<const __half2*>(a.gain + k));
-      const __half2 h = __floats2half2_rn(xv.x * rs * gv.x, xv.y * rs * gv.y);
-      const float2 r = __half22float2(h);
-      const __half2 l = __floats2half2_rn(xv.x * rs * gv.x - r.x, xv.y * rs * gv.y - r.y);
-      hw = *reinterpret_cast<const uint32_t*>(&h);
-      lw = *reinterpret_cast<const uint32_t*>(&l);
+#pragma unroll
+      for (int i = 0; i < kHdXChunks; ++i) {
+        const int k = (threadIdx.x + i * kHdThreads) * 4;
+        if (k < d) {
+          const float xv[4] = {xr[m][i].x, xr[m][i].y, xr[m][i].z, xr[m][i].w};
+          const uint32_t gw[2] = {gr[i].x, gr[i].y};
+          uint32_t hw[2], lw[2];
+#pragma unroll
+          for (int p = 0; p < 2; ++p) {
+            const float2 gv = __half22float2(*reinterpret_cast<const __half2*>(&gw[p]));
+            const float y0 = xv[2 * p] * rs * gv.x, y1 = xv[2 * p + 1] * rs * gv.y;
+            const __half2 h = __floats2half2_rn(y0, y1);
+            const float2 r = __half22float2(h);
+            const __half2 l = __floats2half2_rn(y0 - r.x, y1 - r.y);
+            hw[p] = *reinterpret_cast<const uint32_t*>(&h);
+            lw[p] = *reinterpret_cast<const uint32_t*>(&l);
+          }
+          *reinterpret_cast<uint2*>(xs + (size_t)m * ldx + k) = make_uint2(hw[0], hw[1]);
+          *reinterpret_cast<uint2*>(xl + (size_t)m * ldx + k) = make_uint2(lw[0], lw[1]);
+        }
+      }
     }
-    *reinterpret_cast<uint32_t*>(xs + (size_t)m * ldx + k) = hw;
-    *reinterpret_cast<uint32_t*>(xl + (size_t)m * ldx + k) = lw;
   }
   __syncthreads();
   stamp(1);
