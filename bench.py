@@ -219,6 +219,23 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(pg, values, device):
+    """Element-wise maximum over all ranks of this rank's device-timed values
+    (ms); `pg` is torch.distributed (every rank calls this in the same order)
+    or None for one process, which returns the values unchanged."""
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_rate(world, units_per_rank, slowest_ms):
+    """Units per second of the whole job: every rank's units over the slowest
+    rank's time (replicas, weak scaling)."""
+    return world * units_per_rank / (slowest_ms / 1e3)
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -522,12 +539,8 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     prefill_ms = [e[0].elapsed_time(e[1]) for e in evs]
     decode_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    stats = torch.tensor([total_ms, sum(prefill_ms), sum(decode_ms)], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(stats, op=pg.ReduceOp.MAX)
-    total_ms, prefill_sum, decode_sum = (float(v) for v in stats.cpu())
-    tokens = world * n_dec * args.steps
-    value = tokens / (decode_sum / 1e3)
+    total_ms, prefill_sum, decode_sum = max_over_ranks(pg, [total_ms, sum(prefill_ms), sum(decode_ms)], dev)
+    value = whole_job_rate(world, n_dec * args.steps, decode_sum)
     generated = hist[1:].cpu().numpy().copy()
 
     # ---- end to end: pinned host prompt in, generated tokens out, per step --
@@ -545,10 +558,8 @@ def run_ours(args):
         b.synchronize()
         if i >= args.warmup:
             e2e_ms.append(a.elapsed_time(b))
-    e2e = torch.tensor([sum(e2e_ms) if e2e_ms else float("nan")], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(e2e, op=pg.ReduceOp.MAX)
-    e2e_value = world * n_dec * args.steps / (float(e2e.item()) / 1e3) if e2e_ms else None
+    (e2e_slowest,) = max_over_ranks(pg, [sum(e2e_ms) if e2e_ms else float("nan")], dev)
+    e2e_value = whole_job_rate(world, n_dec * args.steps, e2e_slowest) if e2e_ms else None
     if e2e_ms:
         assert np.array_equal(h_out.numpy(), generated), "end-to-end run diverged from the timed run"
 
