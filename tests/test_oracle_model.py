@@ -224,3 +224,23 @@ def test_fp16_storage_rounding():
     assert ref.to_fp16_storage(np.array([2051.0]))[0] == 2052.0
     assert ref.to_fp16_storage(np.array([1.0 + 2.0 ** -11]))[0] == 1.0
     assert ref.to_fp16_storage(np.array([65504.0]))[0] == 65504.0
+
+
+def test_dense_block_wiring(tiny):
+    # every dense weight is its own linear's dequantisation, in [out][in]
+    # orientation (a swapped or transposed operand changes a shape or a value)
+    w, _ = tiny
+    s = w.shape
+    for blk in list(w.pre) + [w.loop]:
+        db = ref.dense_block(blk)
+        qkv_rows = (s.n_q_heads + 2 * s.n_kv_heads) * s.head_dim
+        assert db.w_qkv.shape == (qkv_rows, s.d_model)
+        assert db.w_o.shape == (s.d_model, s.n_q_heads * s.head_dim)
+        assert db.w_gate_up.shape == (2 * s.ffn_dim, s.d_model)
+        assert db.w_down.shape == (s.d_model, s.ffn_dim)
+        for name, lin in (("w_qkv", blk.qkv), ("w_o", blk.o), ("w_gate_up", blk.gate_up), ("w_down", blk.down)):
+            np.testing.assert_array_equal(getattr(db, name),
+                                          ref.dequantize(lin.qweight, lin.scales, lin.qzeros, lin.K))
+        np.testing.assert_array_equal(db.attn_norm, np.asarray(blk.attn_norm, np.float64))
+        np.testing.assert_array_equal(db.ffn_norm, np.asarray(blk.ffn_norm, np.float64))
+        assert not np.array_equal(db.attn_norm, db.ffn_norm)
